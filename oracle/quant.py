@@ -7,7 +7,7 @@ plainest reading of a 4-bit asymmetric group quantiser:
 
   for each group of (up to) 32 consecutive latent coordinates of one token,
     mn, mx  = min, max over the group's real elements (fp32 values)
-    zero    = fp16(mn)                       (round to nearest even)
+    zero    = fp16(mn)                       (round to nearest even; -0 stored as +0)
     scale   = fp16((mx - mn) / 15)           (fp32 subtract, fp32 divide, then fp16)
     code    = 0                               if scale == 0
             = clamp(rint((x - zero) / scale), 0, 15)   otherwise,
@@ -49,6 +49,7 @@ def quantize_int4(z: np.ndarray, group: int = GROUP):
         mn = seg.min(axis=-1)
         mx = seg.max(axis=-1)
         zg = mn.astype(np.float16)
+        zg = np.where(zg == 0, np.float16(0.0), zg)      # a -0 zero point is stored as +0
         sg = ((mx - mn) / fifteen).astype(np.float16)   # fp32 ops, then fp16 rounding
         zero[..., g] = zg
         scale[..., g] = sg

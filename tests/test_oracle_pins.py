@@ -82,6 +82,9 @@ def test_signed_zero_and_negative_range():
     x[::2] = -0.0
     codes, scale, zero = quant.quantize_int4(x[None])
     assert np.all(codes == 0) and float(scale[0, 0]) == 0.0
+    assert zero.view(np.uint16)[0, 0] == 0          # zero point stored as +0, not -0
+    _, _, z2 = quant.quantize_int4(np.full((1, 32), -0.0, np.float32))
+    assert z2.view(np.uint16)[0, 0] == 0
     y = np.linspace(-7.5, 0.0, 32).astype(np.float32)   # min -7.5 -> code 0, max 0 -> 15
     codes, scale, zero = quant.quantize_int4(y[None])
     assert codes[0, 0] == 0 and codes[0, -1] == 15 and float(zero[0, 0]) == -7.5
