@@ -1,0 +1,200 @@
+/*
+ * lr_kv.h — C ABI of the low-rank KV-cache decode library (NVIDIA B200, sm_100a).
+ *
+ * What the library computes (the pages describe the method; no code is given):
+ *   TraceKV: Policy-Preserving Low-Rank KV Cache Compression for Reasoning
+ *   Vision-Language Models, abstract — the KV cache stores low-dimensional
+ *   latents of the key/value states (Z_k = K A_k, Z_v = V A_v), optionally
+ *   combined with quantization, and "optimized low-rank attention kernels" run
+ *   decode on them; keys and values are recovered through shared bases
+ *   (K ~ Z_k B_k, V ~ Z_v B_v).  The ai4snews digest, Perspective section, fixes
+ *   the latency workload: Qwen2.5-VL-7B decode at batch 16, 4K-32K context.
+ *   iS-KV: Online Low-Rank KV Cache Compression via Block-Incremental SVD,
+ *   abstract and method section — an exact recent window next to the low-rank
+ *   history, older tokens folded into latents as they leave the window, and
+ *   stored historical coordinates synchronised when the basis changes.
+ *
+ * Notation (per layer): B batch, Hq query heads, Hkv KV heads, d head_dim,
+ * D = Hkv*d, r_k / r_v latent ranks, T tokens.  One latent group spans all KV
+ * heads: the latent of a token is z_k = k_cat A_k with k_cat in R^D the
+ * concatenation of its KV heads.  Query head j reads KV head j / (Hq/Hkv).
+ *
+ * Conventions for every call:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *     row-major, borrowed only for the call (stream-ordered).  The cache owns
+ *     its own device buffers and copies A and B at creation.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream; argument and capacity errors are
+ *     returned before anything is launched.  LR_ERR_CUDA reports a launch or
+ *     runtime error (cudaGetLastError after the launch).
+ *   - Element type of q, out, k, v, A, B, stored latents and the window is the
+ *     cache dtype (LR_F32 or LR_BF16).  Latent fills are always fp32; basis-sync
+ *     rotations are always fp32.
+ *   - A cache is not thread-safe; calls on one cache must be serialised.
+ */
+#ifndef LR_KV_H
+#define LR_KV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lr_status {
+  LR_OK = 0,
+  LR_ERR_INVALID_ARG = 1,   /* bad pointer, shape or combination of options      */
+  LR_ERR_UNSUPPORTED = 2,   /* valid but not implemented for this configuration  */
+  LR_ERR_CAPACITY = 3,      /* the cache is full                                  */
+  LR_ERR_CUDA = 4,          /* a CUDA runtime / launch error                      */
+  LR_ERR_OOM = 5,           /* device allocation failed                           */
+  LR_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up (see lr_device_error) */
+} lr_status;
+
+typedef enum lr_dtype { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
+
+/* Kernel path selection for lr_attn_decode. */
+typedef enum lr_path {
+  LR_PATH_AUTO = 0,   /* tensor-core path where supported, else SIMT           */
+  LR_PATH_SIMT = 1,   /* fp32 CUDA-core path (every configuration)             */
+  LR_PATH_TC = 2      /* tcgen05 path (bf16 / int4 latents, keys after RoPE)   */
+} lr_path;
+
+/* Cache description.  All counts are per layer; one cache holds one layer. */
+typedef struct lr_cache_desc {
+  int32_t batch;          /* B >= 1                                               */
+  int32_t n_q_heads;      /* Hq, a multiple of n_kv_heads                          */
+  int32_t n_kv_heads;     /* Hkv >= 1                                              */
+  int32_t head_dim;       /* d, even, <= 256                                       */
+  int32_t rank_k;         /* r_k, multiple of 16, 16..512                          */
+  int32_t rank_v;         /* r_v, multiple of 16, 16..512                          */
+  int32_t capacity;       /* max tokens per sequence (history + window)            */
+  int32_t window;         /* exact recent window W (0 = none)                      */
+  int32_t quant_bits;     /* 0 = latents stored in dtype; 4 = int4 group quant     */
+  int32_t quant_group;    /* group size along the rank axis; must be 32 when quant_bits = 4 */
+  int32_t dtype;          /* lr_dtype                                              */
+  int32_t rope_in_kernel; /* 1 = keys were compressed before RoPE: rotate (rotate-half)
+                             each reconstructed key at its absolute position        */
+  double rope_theta;      /* RoPE base, e.g. 1e6                                   */
+  float softmax_scale;    /* 0 -> 1/sqrt(head_dim)                                 */
+  int32_t reserved[5];    /* must be zero                                          */
+} lr_cache_desc;
+
+typedef struct lr_cache lr_cache;   /* opaque */
+
+/* Device pointers and strides of the cache's storage, for inspection.
+ * Int4 latents: codes [B][capacity][groups*4] uint32 (element e of group g in
+ * word 4g + e/8, bits 4(e%8)..+3), params [B][capacity][groups] as a pair of
+ * fp16 {scale (low half), zero (high half)} in one 32-bit word.
+ * Unquantised latents: z [B][capacity][rank] in dtype.
+ * Window ring: [B][window+1][D] in dtype; token t lives in slot t % (window+1). */
+typedef struct lr_cache_view {
+  void* z_k; void* z_v;                 /* unquantised latents or NULL            */
+  uint32_t* codes_k; uint32_t* codes_v; /* int4 codes or NULL                     */
+  uint32_t* params_k; uint32_t* params_v; /* int4 {scale, zero} or NULL           */
+  void* win_k; void* win_v;             /* window ring or NULL                    */
+  void* A_k; void* B_k; void* A_v; void* B_v;   /* current bases (dtype)         */
+  int32_t groups_k, groups_v;           /* ceil(rank/32) for int4 caches, else 0 */
+  int32_t capacity, window_slots;
+} lr_cache_view;
+
+/* Decode plan (host arithmetic only; exposed for tests and tooling). */
+typedef struct lr_plan {
+  int32_t path;          /* lr_path actually used                                 */
+  int32_t n_splits;      /* sequence splits per batch row (history part)          */
+  int32_t tile_tokens;   /* tokens per tile                                       */
+  int32_t split_tokens;  /* tokens per split (multiple of tile_tokens)            */
+  int32_t ctas;          /* main-kernel CTAs                                      */
+} lr_plan;
+
+/* ---- lifetime -------------------------------------------------------------
+ * lr_cache_create — allocate a cache for `desc` and copy the bases.
+ *   A_k [D][r_k], B_k [r_k][D], A_v [D][r_v], B_v [r_v][D], device, dtype.
+ *   A_* may be NULL when the caller only fills latents (lr_kv_append then
+ *   returns LR_ERR_INVALID_ARG).  Returns LR_ERR_INVALID_ARG / LR_ERR_UNSUPPORTED
+ *   for bad descriptions before touching the device, LR_ERR_OOM if allocation
+ *   fails.  All cache memory is zero-initialised.  Blocks until the copies end. */
+lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void* B_k,
+                          const void* A_v, const void* B_v, void* stream, lr_cache** out);
+
+/* lr_cache_destroy — synchronise the device and free all cache memory. NULL is a no-op. */
+lr_status lr_cache_destroy(lr_cache* cache);
+
+/* ---- append (TraceKV abstract: latents of the KV states, with quantization;
+ *      iS-KV abstract: exact recent window, older states folded into latents) --
+ * lr_kv_append — append one token per sequence.
+ *   k, v: [B][D] in dtype (keys as compressed: before RoPE when rope_in_kernel).
+ *   Without a window: z = k A_k and z_v = v A_v are computed in fp32 and stored
+ *   (rounded to dtype, or int4-quantised) at slot len.  With a window: the token
+ *   goes to ring slot len % (W+1); if the window already held W tokens, its
+ *   oldest token is first folded into history slot hist_len (z = k_old A).
+ *   LR_ERR_CAPACITY when len == capacity. */
+lr_status lr_kv_append(lr_cache* cache, const void* k, const void* v, void* stream);
+
+/* lr_kv_append_latent — bulk fill of n history tokens from given latents.
+ *   z_k [B][n][r_k], z_v [B][n][r_v] fp32, device.  Stored rounded to dtype or
+ *   int4-quantised (group 32, fp16 scale/zero; reading stated in the oracle).
+ *   Requires an empty window (history tokens precede window tokens).
+ *   LR_ERR_CAPACITY if len + n > capacity. */
+lr_status lr_kv_append_latent(lr_cache* cache, const float* z_k, const float* z_v,
+                              int32_t n, void* stream);
+
+/* ---- decode (TraceKV abstract: low-rank attention kernels) ------------------
+ * lr_attn_decode — one decode step of attention over all len cached tokens.
+ *   q [B][Hq][d] (dtype; already rotated at position len-1 when keys carry
+ *   RoPE), out [B][Hq][d] (dtype), lse [B][Hq] fp32 natural-log log-sum-exp of
+ *   the scaled logits, or NULL.  Computes, for every query head j of KV head h:
+ *   softmax over t of s * q_j . k^_t,h, then the weighted sum of v^_t,h, where
+ *   k^, v^ are the latents reconstructed through B (RoPE-rotated if requested)
+ *   for history tokens and the exact tokens for the window.  len == 0 returns
+ *   LR_ERR_INVALID_ARG. */
+lr_status lr_attn_decode(lr_cache* cache, const void* q, void* out, float* lse, void* stream);
+
+/* ---- basis sync (iS-KV abstract: historical coordinates synchronised with the
+ *      updated basis) ---------------------------------------------------------
+ * lr_basis_sync — Z_hist <- Z_hist R for the history latents of every sequence,
+ *   then install new bases.  R_k [r_k][r_k], R_v [r_v][r_v] fp32 device, or NULL
+ *   to leave that side's latents unchanged; B_k_new, B_v_new, A_k_new, A_v_new
+ *   (dtype) or NULL to keep the current basis.  For orthogonal R, passing
+ *   B' = R^T B keeps every reconstructed key/value unchanged.  The window is
+ *   untouched.  Unquantised caches only (int4: LR_ERR_UNSUPPORTED). */
+lr_status lr_basis_sync(lr_cache* cache, const float* R_k, const float* R_v,
+                        const void* B_k_new, const void* B_v_new, const void* A_k_new,
+                        const void* A_v_new, void* stream);
+
+/* ---- bookkeeping ------------------------------------------------------------ */
+/* Current total length, history length and window length (host-side counters). */
+lr_status lr_cache_get_len(const lr_cache* cache, int32_t* len, int32_t* hist_len,
+                           int32_t* win_len);
+/* Drop tokens at positions >= len (no device work).  Caches without a window only. */
+lr_status lr_cache_truncate(lr_cache* cache, int32_t len);
+/* Device pointers of the storage (see lr_cache_view). */
+lr_status lr_cache_view_get(const lr_cache* cache, lr_cache_view* out);
+/* Force a decode path (LR_PATH_*) and/or a split count (0 = automatic). */
+lr_status lr_cache_set_path(lr_cache* cache, int32_t path, int32_t n_splits);
+/* The plan lr_attn_decode would use at the current length. */
+lr_status lr_cache_plan(const lr_cache* cache, lr_plan* out);
+/* Host-only planner: the plan for `desc` at length len on a GPU with num_sms SMs. */
+lr_status lr_plan_decode(const lr_cache_desc* desc, int32_t len, int32_t num_sms,
+                         int32_t path, int32_t n_splits, lr_plan* out);
+/* Synchronise the cache's last stream and read its device error word
+ * (0 = none; otherwise an LR_ERR_* code a kernel recorded, e.g. LR_ERR_TIMEOUT
+ * from a bounded wait).  Clears the word. */
+lr_status lr_device_error(lr_cache* cache, int32_t* code);
+/* Record caller-owned CUDA events (cudaEvent_t passed as void*) immediately before and
+ * after the main decode kernel (the split-sequence attention kernel) of every following
+ * lr_attn_decode on this cache, on the call's stream, so that the kernel alone can be
+ * timed; both NULL to stop.  The events must stay valid while set. */
+lr_status lr_cache_set_kernel_events(lr_cache* cache, void* ev_start, void* ev_stop);
+/* sizeof(lr_cache_desc), sizeof(lr_cache_view), sizeof(lr_plan) as compiled (binding checks). */
+void lr_abi_struct_sizes(int32_t* desc_size, int32_t* view_size, int32_t* plan_size);
+/* Human-readable name of a status. */
+const char* lr_status_string(lr_status status);
+/* Number of kernel launches this library issued since load (all caches). */
+int64_t lr_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LR_KV_H */

@@ -1,0 +1,595 @@
+// CUDA-core kernels of the low-rank KV-cache path: query projection, the
+// fp32 split-sequence decode (every configuration, the only path for fp32
+// caches), the exact window, the split merge with the output projection,
+// append/fold/quantise, the latent bulk fill and the basis sync.
+//
+// Method: TraceKV abstract (latent KV storage with quantization, low-rank
+// attention kernels) and iS-KV abstract/method section (exact recent window,
+// folding, historical-coordinate synchronisation).  Attention is computed in
+// rank space: q~_j = s log2(e) B_k,h(j) q_j, score_t = q~_j . z_t,
+// o~_j = sum_t p_t z_v,t, o_j = o~_j B_v,h(j) / l — the exact identity
+// q . (z B_h) = (B_h q) . z, so the result equals attention over the
+// reconstructed keys and values.
+#include "lr_internal.cuh"
+
+#include <math.h>
+
+namespace {
+
+constexpr int kTileSimt = 16;     // tokens per tile in the SIMT decode
+constexpr int kSyncRows = 16;     // rows per CTA in the SIMT basis sync
+
+__device__ __forceinline__ float elem_f(const void* p, long long idx, int dtype) {
+  if (dtype == LR_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[idx]);
+  return reinterpret_cast<const float*>(p)[idx];
+}
+
+__device__ __forceinline__ void store_elem(void* p, long long idx, float v, int dtype) {
+  if (dtype == LR_BF16) reinterpret_cast<__nv_bfloat16*>(p)[idx] = __float2bfloat16_rn(v);
+  else reinterpret_cast<float*>(p)[idx] = v;
+}
+
+// One stored latent coordinate as fp32.  int4: x^ = code * scale + zero (the
+// product is exact in fp32, so this is the fp32 rounding of the exact value).
+__device__ __forceinline__ float latent_f(const LatentRef& L, int kind, int dtype,
+                                          long long row, int i) {
+  if (kind == LK_INT4) {
+    const uint32_t w = L.codes[row * (L.G * 4) + (i >> 3)];
+    const float code = (float)((w >> (4 * (i & 7))) & 15u);
+    const uint32_t p = L.params[row * L.G + (i >> 5)];
+    const float scale = __half2float(__ushort_as_half((unsigned short)(p & 0xFFFFu)));
+    const float zero = __half2float(__ushort_as_half((unsigned short)(p >> 16)));
+    return fmaf(code, scale, zero);
+  }
+  return elem_f(L.z, row * L.r + i, dtype);
+}
+
+// Warp-cooperative int4 quantisation of one group of 32 coordinates (lane = element;
+// lanes with valid == false are padding).  Reading of the quantiser (the pages give
+// none): zero = fp16(min), scale = fp16((max - min) / 15) in fp32, code =
+// clamp(rint((x - zero) / scale), 0, 15) in IEEE fp32, 0 if scale == 0; a zero
+// point of -0 is stored as +0.  Writes 4 packed words and the {scale, zero} word.
+__device__ __forceinline__ void quant_group_warp(float x, bool valid, uint32_t* words,
+                                                 uint32_t* param) {
+  const int lane = threadIdx.x & 31;
+  float mn = valid ? x : INFINITY;
+  float mx = valid ? x : -INFINITY;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  __half zh = __float2half_rn(mn);
+  if (__half2float(zh) == 0.0f) zh = __ushort_as_half((unsigned short)0);
+  const __half sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+  const float zf = __half2float(zh), sf = __half2float(sh);
+  uint32_t code = 0;
+  if (valid && sf != 0.0f) {
+    float t = rintf(__fdiv_rn(__fsub_rn(x, zf), sf));
+    t = fminf(fmaxf(t, 0.0f), 15.0f);
+    code = (uint32_t)t;
+  }
+  uint32_t v = code << (4 * (lane & 7));
+  v |= __shfl_xor_sync(0xffffffffu, v, 1);
+  v |= __shfl_xor_sync(0xffffffffu, v, 2);
+  v |= __shfl_xor_sync(0xffffffffu, v, 4);
+  if ((lane & 7) == 0) words[lane >> 3] = v;
+  if (lane == 0) *param = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
+}
+
+// Store one warp's 32-coordinate chunk `ch` of a latent row (lane = coordinate).
+__device__ __forceinline__ void store_latent_chunk(float z, int ch, int r, int kind, int dtype,
+                                                   void* Z, uint32_t* codes, uint32_t* params,
+                                                   int G, long long row) {
+  const int lane = threadIdx.x & 31;
+  const int i = ch * 32 + lane;
+  const bool valid = i < r;
+  if (kind == LK_INT4) {
+    quant_group_warp(z, valid, codes + row * (G * 4) + ch * 4, params + row * G + ch);
+  } else if (valid) {
+    store_elem(Z, row * r + i, z, dtype);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// query projection: q~ = s log2(e) B_k,h q  (latent path) and/or s log2(e) q
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_qproj(const void* q, const void* Bk, float* qt, float* qd,
+                                               int Hq, int Hkv, int d, int D, int rk, int dtype,
+                                               float scale_log2, int want_latent) {
+  __shared__ float qs[256];
+  const int j = blockIdx.x, b = blockIdx.y;
+  const int h = j / (Hq / Hkv);
+  const long long qoff = ((long long)b * Hq + j) * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const float v = elem_f(q, qoff + c, dtype);
+    qs[c] = v;
+    if (qd) qd[qoff + c] = v * scale_log2;
+  }
+  __syncthreads();
+  if (!want_latent) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int i = warp; i < rk; i += nw) {
+    float s = 0.f;
+    for (int c = lane; c < d; c += 32) s = fmaf(elem_f(Bk, (long long)i * D + h * d + c, dtype), qs[c], s);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) qt[((long long)b * Hq + j) * rk + i] = s * scale_log2;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// split-sequence decode on CUDA cores (fp32 arithmetic throughout)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind) {
+  extern __shared__ float sm[];
+  const int split = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
+  const int Hq = a.Hq, rk = a.k.r, rv = a.v.r;
+  const int qdim = a.rope ? a.d : rk;
+  const int qstride = qdim + 1;
+  float* q_s = sm;                        // [Hq][qdim+1]
+  float* zk_s = q_s + Hq * qstride;       // [T][rk]
+  float* zv_s = zk_s + kTileSimt * rk;    // [T][rv]
+  float* sc = zv_s + kTileSimt * rv;      // [T][Hq]
+  float* acc = sc + kTileSimt * Hq;       // [Hq][rv]
+  float* m_s = acc + Hq * rv;
+  float* l_s = m_s + Hq;
+  float* al_s = l_s + Hq;
+  float* kh = al_s + Hq;                  // [T][D] (RoPE path)
+
+  const float* qsrc = a.qs + (size_t)b * Hq * qdim;
+  for (int idx = tid; idx < Hq * qdim; idx += nt) q_s[(idx / qdim) * qstride + idx % qdim] = qsrc[idx];
+  for (int idx = tid; idx < Hq * rv; idx += nt) acc[idx] = 0.f;
+  for (int j = tid; j < Hq; j += nt) { m_s[j] = -INFINITY; l_s[j] = 0.f; }
+  __syncthreads();
+
+  const int group = Hq / a.Hkv;
+  const int t_begin = split * a.split_tokens;
+  const int t_end = min(a.hist_len, t_begin + a.split_tokens);
+  for (int t0 = t_begin; t0 < t_end; t0 += kTileSimt) {
+    const int n = min(kTileSimt, t_end - t0);
+    const long long row0 = (long long)b * a.k.cap + t0;
+    for (int idx = tid; idx < n * rk; idx += nt) {
+      const int t = idx / rk, i = idx % rk;
+      zk_s[t * rk + i] = latent_f(a.k, kind, a.dtype, row0 + t, i);
+    }
+    for (int idx = tid; idx < n * rv; idx += nt) {
+      const int t = idx / rv, i = idx % rv;
+      zv_s[t * rv + i] = latent_f(a.v, kind, a.dtype, row0 + t, i);
+    }
+    __syncthreads();
+    if (a.rope) {
+      for (int c = tid; c < a.D; c += nt) {
+        float accum[kTileSimt];
+#pragma unroll
+        for (int t = 0; t < kTileSimt; ++t) accum[t] = 0.f;
+        for (int i = 0; i < rk; ++i) {
+          const float bv = elem_f(a.B_k, (long long)i * a.D + c, a.dtype);
+#pragma unroll
+          for (int t = 0; t < kTileSimt; ++t) accum[t] = fmaf(zk_s[t * rk + i], bv, accum[t]);
+        }
+        for (int t = 0; t < n; ++t) kh[t * a.D + c] = accum[t];
+      }
+      __syncthreads();
+      const int half = a.d / 2;
+      for (int idx = tid; idx < n * a.Hkv * half; idx += nt) {
+        const int t = idx / (a.Hkv * half);
+        const int rem = idx % (a.Hkv * half);
+        const int h = rem / half, i = rem % half;
+        const float2 cs = a.rope_cs[(long long)(t0 + t) * half + i];
+        float* row = kh + t * a.D + h * a.d;
+        const float x1 = row[i], x2 = row[i + half];
+        row[i] = x1 * cs.x - x2 * cs.y;
+        row[i + half] = x2 * cs.x + x1 * cs.y;
+      }
+      __syncthreads();
+    }
+    for (int p = tid; p < n * Hq; p += nt) {
+      const int t = p / Hq, j = p % Hq;
+      const float* qv = q_s + j * qstride;
+      float s = 0.f;
+      if (a.rope) {
+        const float* kv = kh + t * a.D + (j / group) * a.d;
+        for (int c = 0; c < a.d; ++c) s = fmaf(qv[c], kv[c], s);
+      } else {
+        const float* zr = zk_s + t * rk;
+        for (int i = 0; i < rk; ++i) s = fmaf(qv[i], zr[i], s);
+      }
+      sc[t * Hq + j] = s;
+    }
+    __syncthreads();
+    for (int j = tid; j < Hq; j += nt) {
+      float mt = -INFINITY;
+      for (int t = 0; t < n; ++t) mt = fmaxf(mt, sc[t * Hq + j]);
+      const float mo = m_s[j];
+      const float mnew = fmaxf(mo, mt);
+      const float alpha = (mo == -INFINITY) ? 0.f : exp2f(mo - mnew);
+      float sum = 0.f;
+      for (int t = 0; t < n; ++t) {
+        const float p = exp2f(sc[t * Hq + j] - mnew);
+        sc[t * Hq + j] = p;
+        sum += p;
+      }
+      l_s[j] = l_s[j] * alpha + sum;
+      m_s[j] = mnew;
+      al_s[j] = alpha;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < Hq * rv; idx += nt) {
+      const int j = idx / rv, i = idx % rv;
+      float o = acc[idx] * al_s[j];
+      for (int t = 0; t < n; ++t) o = fmaf(sc[t * Hq + j], zv_s[t * rv + i], o);
+      acc[idx] = o;
+    }
+    __syncthreads();
+  }
+  const size_t base = ((size_t)b * a.n_splits + split) * Hq;
+  for (int idx = tid; idx < Hq * rv; idx += nt) a.part_o[base * rv + idx] = acc[idx];
+  for (int j = tid; j < Hq; j += nt) {
+    a.part_ml[(base + j) * 2] = m_s[j];
+    a.part_ml[(base + j) * 2 + 1] = l_s[j];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// exact window (iS-KV): attention of each query head over the window tokens of
+// its KV head, as one more partial (in head space, relative to its own max)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) k_window(const void* win_k, const void* win_v, const float* qd,
+                                                float* win_o, float* win_ml, int Hq, int Hkv, int d,
+                                                int D, int slots, int hist_len, int win_len, int dtype) {
+  extern __shared__ float wsm[];
+  float* q_s = wsm;           // [d]
+  float* p_s = wsm + d;       // [win_len]
+  __shared__ float red[2];
+  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int h = j / (Hq / Hkv);
+  const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  for (int c = tid; c < d; c += blockDim.x) q_s[c] = qd[((long long)b * Hq + j) * d + c];
+  __syncthreads();
+  for (int t = warp; t < win_len; t += nw) {
+    const int slot = (hist_len + t) % slots;
+    const long long off = ((long long)b * slots + slot) * D + (long long)h * d;
+    float s = 0.f;
+    for (int c = lane; c < d; c += 32) s = fmaf(q_s[c], elem_f(win_k, off + c, dtype), s);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) p_s[t] = s;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float m = -INFINITY;
+    for (int t = 0; t < win_len; ++t) m = fmaxf(m, p_s[t]);
+    float l = 0.f;
+    for (int t = 0; t < win_len; ++t) {
+      const float p = exp2f(p_s[t] - m);
+      p_s[t] = p;
+      l += p;
+    }
+    red[0] = m;
+    red[1] = l;
+  }
+  __syncthreads();
+  for (int c = tid; c < d; c += blockDim.x) {
+    float o = 0.f;
+    for (int t = 0; t < win_len; ++t) {
+      const int slot = (hist_len + t) % slots;
+      o = fmaf(p_s[t], elem_f(win_v, ((long long)b * slots + slot) * D + (long long)h * d + c, dtype), o);
+    }
+    win_o[((long long)b * Hq + j) * d + c] = o;
+  }
+  if (tid == 0) {
+    win_ml[((long long)b * Hq + j) * 2] = red[0];
+    win_ml[((long long)b * Hq + j) * 2 + 1] = red[1];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// split merge (log-sum-exp) and output projection o = o~ B_v,h / l
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) k_merge(const float* part_o, const float* part_ml,
+                                               const float* win_o, const float* win_ml,
+                                               const void* Bv, void* out, float* lse, int S,
+                                               int Hq, int Hkv, int d, int D, int rv, int dtype) {
+  extern __shared__ float msm[];
+  float* ot = msm;            // [rv]
+  float* w_s = msm + rv;      // [S]
+  __shared__ float ml[3];     // m*, l, window weight
+  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int h = j / (Hq / Hkv);
+  if (tid < 32) {
+    float m = -INFINITY;
+    for (int s = tid; s < S; s += 32) m = fmaxf(m, part_ml[(((size_t)b * S + s) * Hq + j) * 2]);
+    const float mw = win_ml ? win_ml[((size_t)b * Hq + j) * 2] : -INFINITY;
+    m = fmaxf(m, mw);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    for (int s = tid; s < S; s += 32) {
+      const size_t e = (((size_t)b * S + s) * Hq + j) * 2;
+      const float ms = part_ml[e];
+      const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - m);
+      w_s[s] = w;
+      l = fmaf(w, part_ml[e + 1], l);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (tid == 0) {
+      float ww = 0.f;
+      if (win_ml && mw != -INFINITY) {
+        ww = exp2f(mw - m);
+        l = fmaf(ww, win_ml[((size_t)b * Hq + j) * 2 + 1], l);
+      }
+      ml[0] = m;
+      ml[1] = l;
+      ml[2] = ww;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < rv; i += blockDim.x) {
+    float o = 0.f;
+    for (int s = 0; s < S; ++s) o = fmaf(w_s[s], part_o[(((size_t)b * S + s) * Hq + j) * rv + i], o);
+    ot[i] = o;
+  }
+  __syncthreads();
+  const float inv_l = 1.0f / ml[1];
+  const long long ooff = ((long long)b * Hq + j) * d;
+  for (int c = tid; c < d; c += blockDim.x) {
+    float o = 0.f;
+    for (int i = 0; i < rv; ++i) o = fmaf(ot[i], elem_f(Bv, (long long)i * D + (long long)h * d + c, dtype), o);
+    if (win_o) o = fmaf(ml[2], win_o[ooff + c], o);
+    store_elem(out, ooff + c, o * inv_l, dtype);
+  }
+  if (lse && tid == 0) lse[(long long)b * Hq + j] = (ml[0] + log2f(ml[1])) * LR_LN2;
+}
+
+// ---------------------------------------------------------------------------
+// append: project one token per sequence (z = x A) and store / quantise it;
+// optionally write the new exact token into the window ring
+// ---------------------------------------------------------------------------
+struct AppendArgs {
+  const void* src_k; const void* src_v;   // rows to project (input or evicted ring rows)
+  long long src_bstride;                  // elements between batch rows of src
+  const void* A_k; const void* A_v;
+  void* Zk; void* Zv; uint32_t* codes_k; uint32_t* codes_v; uint32_t* params_k; uint32_t* params_v;
+  int rk, rv, Gk, Gv, chunks_k, chunks_v;
+  long long cap; int dst_slot; int project;
+  const void* new_k; const void* new_v;   // exact token for the ring, or null
+  void* win_k; void* win_v; int slots; int new_slot;
+  int B, D, kind, dtype;
+};
+
+__global__ void __launch_bounds__(256) k_append(AppendArgs a) {
+  const int x = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int nproj = a.project ? (a.chunks_k + a.chunks_v) : 0;
+  if (x < nproj) {
+    const bool is_k = x < a.chunks_k;
+    const int ch = is_k ? x : x - a.chunks_k;
+    const int r = is_k ? a.rk : a.rv;
+    const void* A = is_k ? a.A_k : a.A_v;
+    const void* src = is_k ? a.src_k : a.src_v;
+    const int i = ch * 32 + lane;
+    const bool valid = i < r;
+    for (int b = warp; b < a.B; b += nw) {
+      float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+      if (valid) {
+        const long long so = (long long)b * a.src_bstride;
+        int c = 0;
+        for (; c + 3 < a.D; c += 4) {
+          z0 = fmaf(elem_f(src, so + c, a.dtype), elem_f(A, (long long)c * r + i, a.dtype), z0);
+          z1 = fmaf(elem_f(src, so + c + 1, a.dtype), elem_f(A, (long long)(c + 1) * r + i, a.dtype), z1);
+          z2 = fmaf(elem_f(src, so + c + 2, a.dtype), elem_f(A, (long long)(c + 2) * r + i, a.dtype), z2);
+          z3 = fmaf(elem_f(src, so + c + 3, a.dtype), elem_f(A, (long long)(c + 3) * r + i, a.dtype), z3);
+        }
+        for (; c < a.D; ++c) z0 = fmaf(elem_f(src, so + c, a.dtype), elem_f(A, (long long)c * r + i, a.dtype), z0);
+      }
+      const float z = (z0 + z1) + (z2 + z3);
+      const long long row = (long long)b * a.cap + a.dst_slot;
+      store_latent_chunk(z, ch, r, a.kind, a.dtype, is_k ? a.Zk : a.Zv, is_k ? a.codes_k : a.codes_v,
+                         is_k ? a.params_k : a.params_v, is_k ? a.Gk : a.Gv, row);
+    }
+    return;
+  }
+  // ring write of the exact new token
+  const bool is_k = (x - nproj) == 0;
+  const void* src = is_k ? a.new_k : a.new_v;
+  void* dst = is_k ? a.win_k : a.win_v;
+  const size_t es = a.dtype == LR_BF16 ? 2 : 4;
+  for (int idx = threadIdx.x; idx < a.B * a.D; idx += blockDim.x) {
+    const int b = idx / a.D, c = idx % a.D;
+    const long long so = (long long)b * a.D + c;
+    const long long dof = ((long long)b * a.slots + a.new_slot) * a.D + c;
+    if (es == 2) reinterpret_cast<uint16_t*>(dst)[dof] = reinterpret_cast<const uint16_t*>(src)[so];
+    else reinterpret_cast<uint32_t*>(dst)[dof] = reinterpret_cast<const uint32_t*>(src)[so];
+  }
+}
+
+// bulk latent fill: one warp per (token, 32-coordinate chunk)
+__global__ void __launch_bounds__(256) k_append_latent(const float* zk, const float* zv, int n, int B,
+                                                       int rk, int rv, int chunks_k, int chunks_v,
+                                                       void* Zk, void* Zv, uint32_t* codes_k,
+                                                       uint32_t* codes_v, uint32_t* params_k,
+                                                       uint32_t* params_v, int Gk, int Gv,
+                                                       long long cap, int slot0, int kind, int dtype) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long pi = (long long)blockIdx.x * (blockDim.x >> 5) + warp;
+  const int per_tok = chunks_k + chunks_v;
+  const int b = blockIdx.y;
+  if (pi >= (long long)n * per_tok) return;
+  const int t = (int)(pi / per_tok), c = (int)(pi % per_tok);
+  const bool is_k = c < chunks_k;
+  const int ch = is_k ? c : c - chunks_k;
+  const int r = is_k ? rk : rv;
+  const float* src = is_k ? zk : zv;
+  const int i = ch * 32 + lane;
+  const float z = i < r ? src[((long long)b * n + t) * r + i] : 0.f;
+  const long long row = (long long)b * cap + slot0 + t;
+  store_latent_chunk(z, ch, r, kind, dtype, is_k ? Zk : Zv, is_k ? codes_k : codes_v,
+                     is_k ? params_k : params_v, is_k ? Gk : Gv, row);
+}
+
+// basis sync on CUDA cores: Z[b][t][:] <- Z[b][t][:] R for t < hist_len (in place)
+__global__ void __launch_bounds__(256) k_sync_simt(void* Z, const float* R, int r, long long cap,
+                                                   int hist_len, int dtype) {
+  extern __shared__ float zs[];   // [kSyncRows][r]
+  const int b = blockIdx.y;
+  const int t0 = blockIdx.x * kSyncRows;
+  const int n = min(kSyncRows, hist_len - t0);
+  for (int idx = threadIdx.x; idx < n * r; idx += blockDim.x) {
+    const int t = idx / r, k = idx % r;
+    zs[t * r + k] = elem_f(Z, ((long long)b * cap + t0 + t) * r + k, dtype);
+  }
+  __syncthreads();
+  for (int col = threadIdx.x; col < r; col += blockDim.x) {
+    float acc[kSyncRows];
+#pragma unroll
+    for (int t = 0; t < kSyncRows; ++t) acc[t] = 0.f;
+    for (int k = 0; k < r; ++k) {
+      const float rv = R[(long long)k * r + col];
+#pragma unroll
+      for (int t = 0; t < kSyncRows; ++t) acc[t] = fmaf(zs[t * r + k], rv, acc[t]);
+    }
+    for (int t = 0; t < n; ++t) store_elem(Z, ((long long)b * cap + t0 + t) * r + col, acc[t], dtype);
+  }
+}
+
+LatentRef latent_ref(const lr_cache* c, bool k) {
+  LatentRef L;
+  L.z = k ? c->z_k : c->z_v;
+  L.codes = k ? c->codes_k : c->codes_v;
+  L.params = k ? c->params_k : c->params_v;
+  L.r = k ? c->desc.rank_k : c->desc.rank_v;
+  L.G = k ? c->G_k : c->G_v;
+  L.cap = c->desc.capacity;
+  return L;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+
+cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  const bool rope = d.rope_in_kernel != 0;
+  float* qd = (rope || c->win_slots) ? (rope ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k) : nullptr;
+  dim3 grid(d.n_q_heads, d.batch);
+  k_qproj<<<grid, 256, 0, s>>>(q, c->B_k, c->qt, qd, d.n_q_heads, d.n_kv_heads, d.head_dim, c->D,
+                               d.rank_k, d.dtype, c->scale_log2, rope ? 0 : 1);
+  lr_count_launch();
+  return cudaGetLastError();
+}
+
+size_t decode_simt_smem(const lr_cache* c) {
+  const lr_cache_desc& d = c->desc;
+  const int qdim = d.rope_in_kernel ? d.head_dim : d.rank_k;
+  size_t f = (size_t)d.n_q_heads * (qdim + 1) + (size_t)kTileSimt * d.rank_k + (size_t)kTileSimt * d.rank_v +
+             (size_t)kTileSimt * d.n_q_heads + (size_t)d.n_q_heads * d.rank_v + 3 * (size_t)d.n_q_heads;
+  if (d.rope_in_kernel) f += (size_t)kTileSimt * c->D;
+  return f * sizeof(float);
+}
+
+cudaError_t launch_decode_simt(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  DecodeSimtArgs a;
+  a.k = latent_ref(c, true);
+  a.v = latent_ref(c, false);
+  a.qs = c->qt;
+  a.B_k = c->B_k;
+  a.rope_cs = c->rope_cs;
+  a.part_o = c->part_o;
+  a.part_ml = c->part_ml;
+  a.Hq = d.n_q_heads; a.Hkv = d.n_kv_heads; a.d = d.head_dim; a.D = c->D;
+  a.hist_len = c->hist_len; a.split_tokens = split_tokens; a.n_splits = n_splits;
+  a.rope = d.rope_in_kernel; a.dtype = d.dtype;
+  const size_t smem = decode_simt_smem(c);
+  cudaError_t e = cudaFuncSetAttribute(k_decode_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(n_splits, d.batch);
+  k_decode_simt<<<grid, 256, smem, s>>>(a, c->latent_kind);
+  lr_count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  const float* qd = d.rope_in_kernel ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k;
+  const size_t smem = (size_t)(d.head_dim + c->win_len + 1) * sizeof(float);
+  dim3 grid(d.n_q_heads, d.batch);
+  k_window<<<grid, 128, smem, s>>>(c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads, d.n_kv_heads,
+                                   d.head_dim, c->D, c->win_slots, c->hist_len, c->win_len, d.dtype);
+  lr_count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  const bool win = c->win_slots > 0;
+  const size_t smem = (size_t)(d.rank_v + n_splits) * sizeof(float);
+  dim3 grid(d.n_q_heads, d.batch);
+  k_merge<<<grid, 128, smem, s>>>(c->part_o, c->part_ml, win ? c->win_o : nullptr, win ? c->win_ml : nullptr,
+                                  c->B_v, out, lse, n_splits, d.n_q_heads, d.n_kv_heads, d.head_dim, c->D,
+                                  d.rank_v, d.dtype);
+  lr_count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  AppendArgs a;
+  const bool win = c->win_slots > 0;
+  const bool fold = win && c->win_len == d.window;
+  a.project = win ? (fold ? 1 : 0) : 1;
+  if (win) {
+    const int old_slot = c->hist_len % c->win_slots;
+    const size_t es = c->esize;
+    a.src_k = (const char*)c->win_k + (size_t)old_slot * c->D * es;
+    a.src_v = (const char*)c->win_v + (size_t)old_slot * c->D * es;
+    a.src_bstride = (long long)c->win_slots * c->D;
+  } else {
+    a.src_k = k; a.src_v = v; a.src_bstride = c->D;
+  }
+  a.A_k = c->A_k; a.A_v = c->A_v;
+  a.Zk = c->z_k; a.Zv = c->z_v; a.codes_k = c->codes_k; a.codes_v = c->codes_v;
+  a.params_k = c->params_k; a.params_v = c->params_v;
+  a.rk = d.rank_k; a.rv = d.rank_v; a.Gk = c->G_k; a.Gv = c->G_v;
+  a.chunks_k = (d.rank_k + 31) / 32; a.chunks_v = (d.rank_v + 31) / 32;
+  a.cap = d.capacity; a.dst_slot = c->hist_len;
+  a.new_k = win ? k : nullptr; a.new_v = win ? v : nullptr;
+  a.win_k = c->win_k; a.win_v = c->win_v; a.slots = c->win_slots;
+  a.new_slot = win ? (c->len % c->win_slots) : 0;
+  a.B = d.batch; a.D = c->D; a.kind = c->latent_kind; a.dtype = d.dtype;
+  const int nproj = a.project ? a.chunks_k + a.chunks_v : 0;
+  const int grid = nproj + (win ? 2 : 0);
+  k_append<<<grid, 256, 0, s>>>(a);
+  lr_count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, int n, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  const int chunks_k = (d.rank_k + 31) / 32, chunks_v = (d.rank_v + 31) / 32;
+  const long long pairs = (long long)n * (chunks_k + chunks_v);
+  dim3 grid((unsigned)((pairs + 7) / 8), d.batch);
+  k_append_latent<<<grid, 256, 0, s>>>(zk, zv, n, d.batch, d.rank_k, d.rank_v, chunks_k, chunks_v, c->z_k,
+                                       c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->G_k,
+                                       c->G_v, d.capacity, c->hist_len, c->latent_kind, d.dtype);
+  lr_count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sync_simt(lr_cache* c, const float* R, int which, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  const int r = which == 0 ? d.rank_k : d.rank_v;
+  void* Z = which == 0 ? c->z_k : c->z_v;
+  if (c->hist_len == 0) return cudaSuccess;
+  const size_t smem = (size_t)kSyncRows * r * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(k_sync_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((c->hist_len + kSyncRows - 1) / kSyncRows, d.batch);
+  k_sync_simt<<<grid, 256, smem, s>>>(Z, R, r, d.capacity, c->hist_len, d.dtype);
+  lr_count_launch();
+  return cudaGetLastError();
+}

@@ -1,0 +1,366 @@
+// Host layer of the C ABI declared in include/lr_kv.h: validation, cache
+// lifetime, length bookkeeping, decode planning and kernel launches.
+#include "lr_internal.cuh"
+
+#include <atomic>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+namespace {
+
+std::atomic<long long> g_launches{0};
+
+lr_status validate_desc(const lr_cache_desc* d) {
+  if (!d) return LR_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1) return LR_ERR_INVALID_ARG;
+  if (d->n_q_heads % d->n_kv_heads) return LR_ERR_INVALID_ARG;
+  if (d->head_dim < 2 || d->head_dim % 2 || d->head_dim > 256) return LR_ERR_INVALID_ARG;
+  if (d->rank_k < 16 || d->rank_k % 16 || d->rank_k > 512) return LR_ERR_INVALID_ARG;
+  if (d->rank_v < 16 || d->rank_v % 16 || d->rank_v > 512) return LR_ERR_INVALID_ARG;
+  if (d->capacity < 1 || d->window < 0 || d->window > d->capacity) return LR_ERR_INVALID_ARG;
+  if (d->quant_bits != 0 && d->quant_bits != 4) return LR_ERR_INVALID_ARG;
+  if (d->quant_bits == 4 && d->quant_group != 32) return LR_ERR_UNSUPPORTED;
+  if (d->dtype != LR_F32 && d->dtype != LR_BF16) return LR_ERR_INVALID_ARG;
+  if (d->rope_in_kernel != 0 && d->rope_in_kernel != 1) return LR_ERR_INVALID_ARG;
+  if (d->rope_in_kernel && !(d->rope_theta > 0.0)) return LR_ERR_INVALID_ARG;
+  if (d->rope_in_kernel && d->window > 0) return LR_ERR_UNSUPPORTED;
+  if (!(d->softmax_scale >= 0.0f) || std::isinf(d->softmax_scale)) return LR_ERR_INVALID_ARG;
+  for (int i = 0; i < 5; ++i)
+    if (d->reserved[i] != 0) return LR_ERR_INVALID_ARG;
+  if ((long long)d->n_kv_heads * d->head_dim > 4096) return LR_ERR_UNSUPPORTED;
+  if (d->n_q_heads > 128) return LR_ERR_UNSUPPORTED;
+  return LR_OK;
+}
+
+int pick_path(const lr_cache_desc* d, int forced) {
+  if (forced == LR_PATH_SIMT) return LR_PATH_SIMT;
+  if (forced == LR_PATH_TC) return tc_supported(d) ? LR_PATH_TC : -1;
+  return tc_supported(d) ? LR_PATH_TC : LR_PATH_SIMT;
+}
+
+// Split the history into tiles and spread them over about two CTAs per SM.
+lr_status plan(const lr_cache_desc* d, int hist_len, int num_sms, int path, int n_splits,
+               lr_plan* out) {
+  const int p = pick_path(d, path);
+  if (p < 0) return LR_ERR_UNSUPPORTED;
+  const int tile = (p == LR_PATH_TC) ? 128 : 16;
+  const int tiles = std::max(1, (hist_len + tile - 1) / tile);
+  int splits = n_splits;
+  if (splits <= 0) {
+    const int target = std::max(1, (2 * std::max(num_sms, 1) + d->batch - 1) / d->batch);
+    splits = std::min(tiles, target);
+  }
+  splits = std::max(1, std::min(splits, tiles));
+  const int tiles_per = (tiles + splits - 1) / splits;
+  splits = (tiles + tiles_per - 1) / tiles_per;
+  out->path = p;
+  out->n_splits = splits;
+  out->tile_tokens = tile;
+  out->split_tokens = tiles_per * tile;
+  out->ctas = splits * d->batch;
+  return LR_OK;
+}
+
+// Partial buffers hold up to max(64, the automatic split count) splits per sequence,
+// and never more than one split per 16-token tile.
+int max_splits_for(const lr_cache_desc* d, int num_sms) {
+  const int tiles = std::max(1, (d->capacity + 15) / 16);
+  const int target = std::max(1, (2 * std::max(num_sms, 1) + d->batch - 1) / d->batch);
+  return std::min(tiles, std::max(64, target));
+}
+
+template <typename T>
+cudaError_t dalloc(T** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) return cudaSuccess;
+  cudaError_t e = cudaMalloc((void**)p, bytes);
+  if (e != cudaSuccess) return e;
+  return cudaMemset(*p, 0, bytes);
+}
+
+void free_all(lr_cache* c) {
+  if (!c) return;
+  tc_release(c);
+  void* ptrs[] = {c->z_k, c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->win_k, c->win_v,
+                  c->A_k, c->B_k, c->A_v, c->B_v, c->rope_cs, c->qt, c->qt16, c->part_o, c->part_ml,
+                  c->win_o, c->win_ml, c->dev_err};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+}
+
+lr_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return LR_OK;
+  if (e == cudaErrorMemoryAllocation) return LR_ERR_OOM;
+  return LR_ERR_CUDA;
+}
+
+}  // namespace
+
+void lr_count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+extern "C" {
+
+const char* lr_status_string(lr_status s) {
+  switch (s) {
+    case LR_OK: return "LR_OK";
+    case LR_ERR_INVALID_ARG: return "LR_ERR_INVALID_ARG";
+    case LR_ERR_UNSUPPORTED: return "LR_ERR_UNSUPPORTED";
+    case LR_ERR_CAPACITY: return "LR_ERR_CAPACITY";
+    case LR_ERR_CUDA: return "LR_ERR_CUDA";
+    case LR_ERR_OOM: return "LR_ERR_OOM";
+    case LR_ERR_TIMEOUT: return "LR_ERR_TIMEOUT";
+  }
+  return "LR_ERR_UNKNOWN";
+}
+
+int64_t lr_launch_count(void) { return g_launches.load(); }
+
+lr_status lr_plan_decode(const lr_cache_desc* desc, int32_t len, int32_t num_sms, int32_t path,
+                         int32_t n_splits, lr_plan* out) {
+  lr_status st = validate_desc(desc);
+  if (st != LR_OK) return st;
+  if (!out || len < 0 || len > desc->capacity || num_sms < 1) return LR_ERR_INVALID_ARG;
+  if (path < 0 || path > 2 || n_splits < 0) return LR_ERR_INVALID_ARG;
+  const int hist = desc->window > 0 ? std::max(0, len - desc->window) : len;
+  return plan(desc, hist, num_sms, path, n_splits, out);
+}
+
+lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void* B_k, const void* A_v,
+                          const void* B_v, void* stream, lr_cache** out) {
+  if (!out) return LR_ERR_INVALID_ARG;
+  *out = nullptr;
+  lr_status st = validate_desc(desc);
+  if (st != LR_OK) return st;
+  if (!B_k || !B_v) return LR_ERR_INVALID_ARG;
+  if ((A_k == nullptr) != (A_v == nullptr)) return LR_ERR_INVALID_ARG;
+
+  lr_cache* c = new (std::nothrow) lr_cache();
+  if (!c) return LR_ERR_OOM;
+  c->desc = *desc;
+  const lr_cache_desc& d = c->desc;
+  c->D = d.n_kv_heads * d.head_dim;
+  c->esize = d.dtype == LR_BF16 ? 2 : 4;
+  c->latent_kind = d.quant_bits == 4 ? LK_INT4 : (d.dtype == LR_BF16 ? LK_BF16 : LK_F32);
+  c->G_k = d.quant_bits == 4 ? (d.rank_k + 31) / 32 : 0;
+  c->G_v = d.quant_bits == 4 ? (d.rank_v + 31) / 32 : 0;
+  c->win_slots = d.window > 0 ? d.window + 1 : 0;
+  c->len = c->hist_len = c->win_len = 0;
+  const float sm_scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / std::sqrt((float)d.head_dim);
+  c->scale_log2 = sm_scale * LR_LOG2E;
+  c->last_stream = (cudaStream_t)stream;
+
+  cudaError_t e = cudaGetDevice(&c->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+  c->S_max = max_splits_for(&d, c->num_sms);
+  const size_t B = d.batch, cap = d.capacity, es = c->esize, D = c->D;
+  if (e == cudaSuccess) {
+    if (c->latent_kind == LK_INT4) {
+      e = dalloc(&c->codes_k, B * cap * c->G_k * 4 * sizeof(uint32_t));
+      if (e == cudaSuccess) e = dalloc(&c->codes_v, B * cap * c->G_v * 4 * sizeof(uint32_t));
+      if (e == cudaSuccess) e = dalloc(&c->params_k, B * cap * c->G_k * sizeof(uint32_t));
+      if (e == cudaSuccess) e = dalloc(&c->params_v, B * cap * c->G_v * sizeof(uint32_t));
+    } else {
+      e = dalloc(&c->z_k, B * cap * d.rank_k * es);
+      if (e == cudaSuccess) e = dalloc(&c->z_v, B * cap * d.rank_v * es);
+    }
+  }
+  if (e == cudaSuccess && c->win_slots) {
+    e = dalloc(&c->win_k, B * c->win_slots * D * es);
+    if (e == cudaSuccess) e = dalloc(&c->win_v, B * c->win_slots * D * es);
+  }
+  if (e == cudaSuccess) e = dalloc(&c->B_k, (size_t)d.rank_k * D * es);
+  if (e == cudaSuccess) e = dalloc(&c->B_v, (size_t)d.rank_v * D * es);
+  if (e == cudaSuccess) e = dalloc(&c->A_k, D * d.rank_k * es);
+  if (e == cudaSuccess) e = dalloc(&c->A_v, D * d.rank_v * es);
+  if (e == cudaSuccess) e = dalloc(&c->qt, B * d.n_q_heads * ((size_t)d.rank_k + d.head_dim) * sizeof(float));
+  if (e == cudaSuccess) e = dalloc(&c->part_o, B * c->S_max * d.n_q_heads * (size_t)d.rank_v * sizeof(float));
+  if (e == cudaSuccess) e = dalloc(&c->part_ml, B * c->S_max * d.n_q_heads * 2 * sizeof(float));
+  if (e == cudaSuccess && c->win_slots) {
+    e = dalloc(&c->win_o, B * d.n_q_heads * (size_t)d.head_dim * sizeof(float));
+    if (e == cudaSuccess) e = dalloc(&c->win_ml, B * d.n_q_heads * 2 * sizeof(float));
+  }
+  if (e == cudaSuccess) e = dalloc(&c->dev_err, sizeof(int));
+  if (e == cudaSuccess && d.rope_in_kernel) {
+    const int half = d.head_dim / 2;
+    std::vector<float2> cs((size_t)cap * half);
+    std::vector<double> omega(half);
+    for (int i = 0; i < half; ++i) omega[i] = std::pow(d.rope_theta, -2.0 * i / d.head_dim);
+    for (size_t t = 0; t < cap; ++t)
+      for (int i = 0; i < half; ++i) {
+        const double ang = (double)t * omega[i];
+        cs[t * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+      }
+    e = dalloc(&c->rope_cs, cs.size() * sizeof(float2));
+    if (e == cudaSuccess) e = cudaMemcpy(c->rope_cs, cs.data(), cs.size() * sizeof(float2), cudaMemcpyHostToDevice);
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->B_k, B_k, (size_t)d.rank_k * D * es, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->B_v, B_v, (size_t)d.rank_v * D * es, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && A_k) e = cudaMemcpyAsync(c->A_k, A_k, D * d.rank_k * es, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && A_v) e = cudaMemcpyAsync(c->A_v, A_v, D * d.rank_v * es, cudaMemcpyDeviceToDevice, s);
+  c->has_A = A_k != nullptr;
+  if (e == cudaSuccess && tc_supported(&d)) e = tc_prepare(c);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    free_all(c);
+    delete c;
+    return cuda_status(e);
+  }
+  *out = c;
+  return LR_OK;
+}
+
+lr_status lr_cache_destroy(lr_cache* c) {
+  if (!c) return LR_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  free_all(c);
+  delete c;
+  return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
+}
+
+lr_status lr_kv_append(lr_cache* c, const void* k, const void* v, void* stream) {
+  if (!c || !k || !v || !c->has_A) return LR_ERR_INVALID_ARG;
+  if (c->len >= c->desc.capacity) return LR_ERR_CAPACITY;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  cudaError_t e = launch_append(c, k, v, s);
+  if (e != cudaSuccess) return LR_ERR_CUDA;
+  if (c->win_slots) {
+    if (c->win_len == c->desc.window) ++c->hist_len;
+    else ++c->win_len;
+  } else {
+    ++c->hist_len;
+  }
+  ++c->len;
+  return LR_OK;
+}
+
+lr_status lr_kv_append_latent(lr_cache* c, const float* zk, const float* zv, int32_t n, void* stream) {
+  if (!c || !zk || !zv || n < 0) return LR_ERR_INVALID_ARG;
+  if (c->win_len > 0) return LR_ERR_INVALID_ARG;
+  if ((long long)c->len + n > c->desc.capacity) return LR_ERR_CAPACITY;
+  if (n == 0) return LR_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  cudaError_t e = launch_append_latent(c, zk, zv, n, s);
+  if (e != cudaSuccess) return LR_ERR_CUDA;
+  c->hist_len += n;
+  c->len += n;
+  return LR_OK;
+}
+
+lr_status lr_cache_plan(const lr_cache* c, lr_plan* out) {
+  if (!c || !out) return LR_ERR_INVALID_ARG;
+  return plan(&c->desc, c->hist_len, c->num_sms, c->path_force, c->splits_force, out);
+}
+
+lr_status lr_attn_decode(lr_cache* c, const void* q, void* out, float* lse, void* stream) {
+  if (!c || !q || !out) return LR_ERR_INVALID_ARG;
+  if (c->len == 0) return LR_ERR_INVALID_ARG;
+  lr_plan p;
+  lr_status st = plan(&c->desc, c->hist_len, c->num_sms, c->path_force, c->splits_force, &p);
+  if (st != LR_OK) return st;
+  if (p.n_splits > c->S_max) return LR_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  cudaError_t e;
+  if (p.path != LR_PATH_TC && c->hist_len > 0 && decode_simt_smem(c) > 227 * 1024) return LR_ERR_UNSUPPORTED;
+  e = p.path == LR_PATH_TC ? launch_qproj_tc(c, q, s) : launch_qproj(c, q, s);
+  if (e == cudaSuccess && c->hist_len > 0) {
+    if (c->ev_start) e = cudaEventRecord(c->ev_start, s);
+    if (e == cudaSuccess)
+      e = p.path == LR_PATH_TC ? launch_decode_tc(c, p.n_splits, p.split_tokens, s)
+                               : launch_decode_simt(c, p.n_splits, p.split_tokens, s);
+    if (e == cudaSuccess && c->ev_stop) e = cudaEventRecord(c->ev_stop, s);
+  }
+  const int S = c->hist_len > 0 ? p.n_splits : 0;
+  if (e == cudaSuccess && c->win_slots) e = launch_window(c, s);
+  if (e == cudaSuccess) e = launch_merge(c, S, out, lse, s);
+  return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
+}
+
+lr_status lr_basis_sync(lr_cache* c, const float* R_k, const float* R_v, const void* B_k_new,
+                        const void* B_v_new, const void* A_k_new, const void* A_v_new, void* stream) {
+  if (!c) return LR_ERR_INVALID_ARG;
+  if (c->latent_kind == LK_INT4 && (R_k || R_v)) return LR_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  const lr_cache_desc& d = c->desc;
+  const size_t es = c->esize, D = c->D;
+  cudaError_t e = cudaSuccess;
+  if (R_k) e = launch_sync_simt(c, R_k, 0, s);
+  if (e == cudaSuccess && R_v) e = launch_sync_simt(c, R_v, 1, s);
+  if (e == cudaSuccess && B_k_new) e = cudaMemcpyAsync(c->B_k, B_k_new, (size_t)d.rank_k * D * es, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && B_v_new) e = cudaMemcpyAsync(c->B_v, B_v_new, (size_t)d.rank_v * D * es, cudaMemcpyDeviceToDevice, s);
+  if (A_k_new || A_v_new) c->has_A = true;
+  if (e == cudaSuccess && A_k_new) e = cudaMemcpyAsync(c->A_k, A_k_new, D * d.rank_k * es, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && A_v_new) e = cudaMemcpyAsync(c->A_v, A_v_new, D * d.rank_v * es, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && (B_k_new || B_v_new)) e = tc_prepare(c);
+  return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
+}
+
+lr_status lr_cache_get_len(const lr_cache* c, int32_t* len, int32_t* hist_len, int32_t* win_len) {
+  if (!c) return LR_ERR_INVALID_ARG;
+  if (len) *len = c->len;
+  if (hist_len) *hist_len = c->hist_len;
+  if (win_len) *win_len = c->win_len;
+  return LR_OK;
+}
+
+lr_status lr_cache_truncate(lr_cache* c, int32_t len) {
+  if (!c || len < 0 || len > c->len) return LR_ERR_INVALID_ARG;
+  if (c->win_slots) return LR_ERR_UNSUPPORTED;
+  c->len = c->hist_len = len;
+  return LR_OK;
+}
+
+lr_status lr_cache_view_get(const lr_cache* c, lr_cache_view* v) {
+  if (!c || !v) return LR_ERR_INVALID_ARG;
+  std::memset(v, 0, sizeof(*v));
+  v->z_k = c->z_k; v->z_v = c->z_v;
+  v->codes_k = c->codes_k; v->codes_v = c->codes_v;
+  v->params_k = c->params_k; v->params_v = c->params_v;
+  v->win_k = c->win_k; v->win_v = c->win_v;
+  v->A_k = c->A_k; v->B_k = c->B_k; v->A_v = c->A_v; v->B_v = c->B_v;
+  v->groups_k = c->G_k; v->groups_v = c->G_v;
+  v->capacity = c->desc.capacity; v->window_slots = c->win_slots;
+  return LR_OK;
+}
+
+lr_status lr_cache_set_path(lr_cache* c, int32_t path, int32_t n_splits) {
+  if (!c || path < 0 || path > 2 || n_splits < 0) return LR_ERR_INVALID_ARG;
+  if (path == LR_PATH_TC && !tc_supported(&c->desc)) return LR_ERR_UNSUPPORTED;
+  if (n_splits > c->S_max) return LR_ERR_INVALID_ARG;
+  c->path_force = path;
+  c->splits_force = n_splits;
+  return LR_OK;
+}
+
+lr_status lr_cache_set_kernel_events(lr_cache* c, void* ev_start, void* ev_stop) {
+  if (!c || ((ev_start == nullptr) != (ev_stop == nullptr))) return LR_ERR_INVALID_ARG;
+  c->ev_start = (cudaEvent_t)ev_start;
+  c->ev_stop = (cudaEvent_t)ev_stop;
+  return LR_OK;
+}
+
+void lr_abi_struct_sizes(int32_t* desc_size, int32_t* view_size, int32_t* plan_size) {
+  if (desc_size) *desc_size = (int32_t)sizeof(lr_cache_desc);
+  if (view_size) *view_size = (int32_t)sizeof(lr_cache_view);
+  if (plan_size) *plan_size = (int32_t)sizeof(lr_plan);
+}
+
+lr_status lr_device_error(lr_cache* c, int32_t* code) {
+  if (!c || !code) return LR_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(c->last_stream);
+  if (e != cudaSuccess) return LR_ERR_CUDA;
+  int h = 0;
+  e = cudaMemcpy(&h, c->dev_err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(c->dev_err, 0, sizeof(int));
+  *code = h;
+  return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+// Internal definitions shared by the host layer and the kernels of the
+// low-rank KV-cache decode library.  Not part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "lr_kv.h"
+
+#define LR_LOG2E 1.4426950408889634f
+#define LR_LN2 0.6931471805599453f
+
+// Latent storage kinds.
+enum LatentKind { LK_F32 = 0, LK_BF16 = 1, LK_INT4 = 2 };
+
+struct lr_cache {
+  lr_cache_desc desc;
+  int D;                 // n_kv_heads * head_dim
+  int G_k, G_v;          // int4 groups per token (0 when unquantised)
+  int win_slots;         // window + 1 (ring), or 0
+  int32_t len, hist_len, win_len;
+  float scale_log2;      // softmax_scale * log2(e)
+  int latent_kind;       // LatentKind
+  size_t esize;          // bytes per dtype element
+
+  // storage
+  void* z_k = nullptr; void* z_v = nullptr;
+  uint32_t* codes_k = nullptr; uint32_t* codes_v = nullptr;
+  uint32_t* params_k = nullptr; uint32_t* params_v = nullptr;
+  void* win_k = nullptr; void* win_v = nullptr;
+  void* A_k = nullptr; void* B_k = nullptr; void* A_v = nullptr; void* B_v = nullptr;
+  float2* rope_cs = nullptr;   // [capacity][head_dim/2] (cos, sin), fp32 from fp64 angles
+
+  // scratch
+  float* qt = nullptr;         // [B][Hq][r_k] fp32 scaled query latents (or [B][Hq][d] for RoPE)
+  void* qt16 = nullptr;        // [B][Hpad][r_k] 16-bit query latents for the tensor-core path
+  float* part_o = nullptr;     // [B][S_max][Hq][r_v]
+  float* part_ml = nullptr;    // [B][S_max][Hq][2]
+  float* win_o = nullptr;      // [B][Hq][d]
+  float* win_ml = nullptr;     // [B][Hq][2]
+  int* dev_err = nullptr;      // device error word
+  int S_max = 1;
+
+  bool has_A = false;         // projections given at creation (needed by lr_kv_append)
+  int path_force = 0, splits_force = 0;
+  int num_sms = 148;
+  int device = 0;
+  cudaStream_t last_stream = nullptr;
+  void* tc_state = nullptr;    // tensor-core path state (tensor maps), owned
+  cudaEvent_t ev_start = nullptr, ev_stop = nullptr;   // caller-owned kernel timing events
+};
+
+// ---- argument blocks --------------------------------------------------------
+
+struct LatentRef {
+  const void* z;          // unquantised [B][cap][r]
+  const uint32_t* codes;  // int4 [B][cap][G*4]
+  const uint32_t* params; // int4 [B][cap][G]
+  int r, G;
+  long long cap;
+};
+
+struct DecodeSimtArgs {
+  LatentRef k, v;
+  const float* qs;        // [B][Hq][r_k] (latent path) or [B][Hq][d] (RoPE path), pre-scaled
+  const void* B_k;        // RoPE path: [r_k][D]
+  const float2* rope_cs;  // RoPE path: [cap][d/2]
+  float* part_o;          // [B][S][Hq][r_v]
+  float* part_ml;         // [B][S][Hq][2]
+  int Hq, Hkv, d, D;
+  int hist_len, split_tokens, n_splits;
+  int rope;
+  int dtype;
+};
+
+// ---- launchers (return cudaGetLastError) ------------------------------------
+cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s);
+cudaError_t launch_decode_simt(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s);
+cudaError_t launch_window(const lr_cache* c, cudaStream_t s);
+cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s);
+cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s);
+cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, int n,
+                                 cudaStream_t s);
+cudaError_t launch_sync_simt(lr_cache* c, const float* R, int which, cudaStream_t s);
+size_t decode_simt_smem(const lr_cache* c);
+
+// tensor-core path (k_decode_tc.cu)
+bool tc_supported(const lr_cache_desc* d);
+cudaError_t tc_prepare(lr_cache* c);
+void tc_release(lr_cache* c);
+cudaError_t launch_qproj_tc(const lr_cache* c, const void* q, cudaStream_t s);
+cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s);
+
+void lr_count_launch(int n = 1);

@@ -1,0 +1,109 @@
+"""CPU-only checks of the C ABI: the library loads and exports every symbol the header
+declares, struct layouts agree with the binding, and the host-side logic (validation,
+planning, status names) behaves without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lr_kv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(lr_[a-z0-9_]+)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary_calls():
+    names = declared_functions()
+    for must in ("lr_cache_create", "lr_cache_destroy", "lr_kv_append", "lr_kv_append_latent",
+                 "lr_attn_decode", "lr_basis_sync"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    so = ctypes.CDLL(lib.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(so, n)]
+    assert not missing, missing
+
+
+def test_struct_sizes_match_binding(lib):
+    assert lib.lr_abi_struct_sizes() == (ctypes.sizeof(lib.lr_cache_desc),
+                                         ctypes.sizeof(lib.lr_cache_view),
+                                         ctypes.sizeof(lib.lr_plan))
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "LR_OK"), (1, "LR_ERR_INVALID_ARG"), (2, "LR_ERR_UNSUPPORTED"),
+                       (3, "LR_ERR_CAPACITY"), (4, "LR_ERR_CUDA"), (5, "LR_ERR_OOM"),
+                       (6, "LR_ERR_TIMEOUT"), (99, "LR_ERR_UNKNOWN")]:
+        assert lib.lr_status_string(code) == name
+
+
+def _qwen(lib, **kw):
+    base = dict(batch=16, n_q_heads=28, n_kv_heads=4, head_dim=128, rank_k=256, rank_v=256,
+                capacity=4096)
+    base.update(kw)
+    return lib.make_desc(**base)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("n_q_heads", 27, 1), ("head_dim", 127, 1), ("rank_k", 250, 1), ("rank_v", 1024, 1),
+    ("quant_bits", 3, 1), ("quant_group", 64, 2), ("dtype", 7, 1), ("window", 5000, 1),
+    ("batch", 0, 1), ("capacity", 0, 1)])
+def test_invalid_descriptions_rejected_before_device(lib, field, value, status):
+    kw = {field: value}
+    if field == "quant_group":
+        kw["quant_bits"] = 4
+    d = _qwen(lib, **kw)
+    out = ctypes.c_void_p()
+    st = lib.raw_status("lr_cache_create", ctypes.byref(d), None, ctypes.c_void_p(1), None,
+                        ctypes.c_void_p(1), None, ctypes.byref(out))
+    assert st == status and not out.value
+
+
+def test_rope_with_window_is_unsupported(lib):
+    d = _qwen(lib, rope_in_kernel=1, window=128)
+    with pytest.raises(lib.LRError) as e:
+        lib.lr_plan_decode(d, 1000, 148)
+    assert e.value.status == lib.LR_ERR_UNSUPPORTED
+
+
+def test_reserved_fields_must_be_zero(lib):
+    d = _qwen(lib)
+    d.reserved[2] = 1
+    with pytest.raises(lib.LRError):
+        lib.lr_plan_decode(d, 10, 148)
+
+
+def test_null_arguments(lib):
+    assert lib.raw_status("lr_kv_append", None, None, None, None) == lib.LR_ERR_INVALID_ARG
+    assert lib.raw_status("lr_attn_decode", None, None, None, None, None) == lib.LR_ERR_INVALID_ARG
+    assert lib.raw_status("lr_cache_destroy", None) == lib.LR_OK
+
+
+@pytest.mark.parametrize("length", [1, 17, 128, 1000, 4096, 4095])
+@pytest.mark.parametrize("batch", [1, 8, 16])
+@pytest.mark.parametrize("path", [1, 0])
+def test_plan_covers_history_exactly(lib, length, batch, path):
+    d = _qwen(lib, batch=batch)
+    p = lib.lr_plan_decode(d, length, 148, path)
+    assert p.split_tokens % p.tile_tokens == 0
+    assert (p.n_splits - 1) * p.split_tokens < length <= p.n_splits * p.split_tokens
+    assert p.ctas == p.n_splits * batch
+    assert p.n_splits * batch <= max(2 * 148 + batch, batch)
+
+
+def test_plan_forced_splits_and_window(lib):
+    d = _qwen(lib, capacity=8192)
+    p = lib.lr_plan_decode(d, 4096, 148, 1, 7)
+    assert p.n_splits == 7 and p.split_tokens * 7 >= 4096
+    dw = _qwen(lib, batch=8, n_q_heads=32, n_kv_heads=8, capacity=32768, window=128)
+    p = lib.lr_plan_decode(dw, 32768, 148, 1)
+    assert p.n_splits * p.split_tokens >= 32768 - 128
+    assert (p.n_splits - 1) * p.split_tokens < 32768 - 128
