@@ -204,39 +204,60 @@ def run_ours(args):
         step(k_d, v_d, q_d, out, lse)
     torch.cuda.synchronize()
 
+    # kernel-only events around the main decode kernel (recorded by the library)
+    kev0, kev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kev0.record(); kev1.record()
+    torch.cuda.synchronize()
+    lr.lr_cache_set_kernel_events(cache, kev0, kev1)
+    graph = None
+    n0 = lr.lr_launch_count()
+    if args.graph:
+        # the step is replayed as a CUDA graph: the context is fixed (append at slot T-1,
+        # decode over T tokens, truncate back), so the captured launches are the step
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(k_d, v_d, q_d, out, lse)
+        torch.cuda.synchronize()
+        run = graph.replay
+    else:
+        step(k_d, v_d, q_d, out, lse)
+        torch.cuda.synchronize()
+        run = lambda: step(k_d, v_d, q_d, out, lse)  # noqa: E731
+    launches_per_step = lr.lr_launch_count() - n0
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+
     uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "")
     sampler = ClockSampler(uuid)
     sampler.start()
     t_end = time.time() + args.load_seconds          # sustained load so the sampler sees the
     while time.time() < t_end:                        # clocks of this very step
         for _ in range(50):
-            step(k_d, v_d, q_d, out, lse)
+            run()
         torch.cuda.synchronize()
 
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for a, b in kev:
-        a.record(); b.record()
+    kern_ms = []
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    launches0 = lr.lr_launch_count()
     for i in range(K):
         flush.zero_()
-        lr.lr_cache_set_kernel_events(cache, kev[i][0], kev[i][1])
         ev[i][0].record()
-        step(k_d, v_d, q_d, out, lse)
+        run()
         ev[i][1].record()
+        kev1.synchronize()
+        kern_ms.append(kev0.elapsed_time(kev1))
     torch.cuda.synchronize()
     barrier()
-    launches = lr.lr_launch_count() - launches0
-    lr.lr_cache_set_kernel_events(cache)
+    launches = launches_per_step * K
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    kern_ms = [a.elapsed_time(b) for a, b in kev]
     total_ms = sum(step_ms)
 
-    # end to end through the public API with host buffers (pinned), copies timed
+    # end to end with host buffers (pinned): H2D of the step's inputs, the step through
+    # the public API (replayed graph of lr_kv_append + lr_attn_decode), D2H of the result
     q_host = torch.from_numpy(np.ascontiguousarray(p.q).view(np.int16)).view(torch.bfloat16).pin_memory()
     k_host = torch.from_numpy(k_h.view(np.int16)).view(torch.bfloat16).pin_memory()
     v_host = torch.from_numpy(v_h.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -251,13 +272,14 @@ def run_ours(args):
         q_d.copy_(q_host, non_blocking=True)
         k_d.copy_(k_host, non_blocking=True)
         v_d.copy_(v_host, non_blocking=True)
-        step(k_d, v_d, q_d, out, lse)
+        run()
         out_host.copy_(out, non_blocking=True)
         lse_host.copy_(lse, non_blocking=True)
         e2e_ev[i][1].record()
     torch.cuda.synchronize()
     barrier()
     sampler.stop()
+    lr.lr_cache_set_kernel_events(cache)
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
     h2d = (q_host.numel() + k_host.numel() + v_host.numel()) * 2
     d2h = out_host.numel() * 2 + lse_host.numel() * 4
@@ -286,7 +308,8 @@ def run_ours(args):
                    "step": "lr_kv_append + lr_attn_decode", "l2": "flushed (256 MiB write) before every timed step, outside the events",
                    "parallelism": f"dp{world} (independent sequences per GPU)",
                    "decode_path": "tcgen05" if plan.path == lr.LR_PATH_TC else "simt",
-                   "splits": plan.n_splits},
+                   "splits": plan.n_splits, "cuda_graph": bool(args.graph),
+                   "launches_per_step": launches_per_step},
         "roofline": {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
                      "peak": peaks.get("hbm_gbs", FALLBACK_HBM_GBS), "peak_source": peak_src,
                      "unit": "GB/s", "frac": round(achieved / peaks.get("hbm_gbs", FALLBACK_HBM_GBS), 4),
@@ -302,6 +325,7 @@ def run_ours(args):
         res["cpu_baseline"] = cpu_baseline(args.workload, p, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(res), flush=True)
+    del graph
     lr.lr_cache_destroy(cache)
     if world > 1:
         import torch.distributed as dist
@@ -400,6 +424,8 @@ def main():
     ap.add_argument("--load-seconds", type=float, default=1.5)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch the step's calls directly instead of replaying a CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -63,9 +63,9 @@ typedef enum lr_path {
 /* Cache description.  All counts are per layer; one cache holds one layer. */
 typedef struct lr_cache_desc {
   int32_t batch;          /* B >= 1                                               */
-  int32_t n_q_heads;      /* Hq, a multiple of n_kv_heads                          */
-  int32_t n_kv_heads;     /* Hkv >= 1                                              */
-  int32_t head_dim;       /* d, even, <= 256                                       */
+  int32_t n_q_heads;      /* Hq <= 128, a multiple of n_kv_heads, Hq/Hkv <= 64      */
+  int32_t n_kv_heads;     /* Hkv >= 1, Hkv * head_dim <= 4096                       */
+  int32_t head_dim;       /* d, a multiple of 8, <= 256                            */
   int32_t rank_k;         /* r_k, multiple of 16, 16..512                          */
   int32_t rank_v;         /* r_v, multiple of 16, 16..512                          */
   int32_t capacity;       /* max tokens per sequence (history + window)            */
@@ -123,7 +123,8 @@ lr_status lr_cache_destroy(lr_cache* cache);
 /* ---- append (TraceKV abstract: latents of the KV states, with quantization;
  *      iS-KV abstract: exact recent window, older states folded into latents) --
  * lr_kv_append — append one token per sequence.
- *   k, v: [B][D] in dtype (keys as compressed: before RoPE when rope_in_kernel).
+ *   k, v: [B][D] in dtype (keys as compressed: before RoPE when rope_in_kernel),
+ *   16-byte aligned (else LR_ERR_INVALID_ARG).
  *   Without a window: z = k A_k and z_v = v A_v are computed in fp32 and stored
  *   (rounded to dtype, or int4-quantised) at slot len.  With a window: the token
  *   goes to ring slot len % (W+1); if the window already held W tokens, its

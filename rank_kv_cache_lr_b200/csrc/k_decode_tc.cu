@@ -1,8 +1,533 @@
-// Tensor-core (tcgen05) decode path: placeholder until the kernel lands.
+// Tensor-core (tcgen05) split-sequence decode over bf16 latents.
+//
+// Method: TraceKV abstract ("optimized low-rank attention kernels" over latent KV
+// states).  Attention runs in rank space (exact identity q . (z B_h) = (B_h q) . z):
+//   S[t, j]  = z_k,t . q~_j          GEMM1: M = 128 tokens, N = 64, K = r_k
+//   p[t, j]  = exp2(S[t, j] - m_j)   online softmax, lazy max (rescale only when the
+//                                    running max grows by more than 2^8)
+//   O~[e, j] += sum_t z_v,t[e] p[t,j] GEMM2: M = 128 ranks per chunk, N = 64, K = 128 tokens
+// The query latent q~ (scaled by s log2 e) enters GEMM1 as two bf16 halves, hi and
+// lo = q~ - hi, stacked on N (columns 0..31 and 32..63), so the scores carry almost
+// fp32 precision while the stored latents stay bf16.  The probabilities enter GEMM2
+// the same way (p = p_hi + p_lo), so the value mix and the normaliser l are both
+// computed from ~fp32 weights; a single bf16 rounding of p would bias l when the
+// weights cluster (near-uniform softmax).  Accumulators live in TMEM: S double-
+// buffered (2 x 64 columns), O~ in ceil(r_v/128) chunks of 64 columns (hi | lo).
+//
+// Roles (192 threads): warp 0 issues TMA tile loads (128 tokens x 64 ranks boxes,
+// 128-byte swizzle, no multicast) into a ring of 32 KB slots (one 128-rank chunk of
+// K or V for one 128-token tile); warp 1 owns TMEM and issues tcgen05.mma from one
+// thread; warps 2..5 run the softmax (thread = token row = TMEM lane) and the
+// epilogue (thread = rank row).  Every wait is bounded: on timeout the kernel records
+// LR_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #include "lr_internal.cuh"
+#include "ptx.cuh"
 
-bool tc_supported(const lr_cache_desc*) { return false; }
-cudaError_t tc_prepare(lr_cache*) { return cudaSuccess; }
-void tc_release(lr_cache*) {}
-cudaError_t launch_qproj_tc(const lr_cache*, const void*, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_decode_tc(const lr_cache*, int, int, cudaStream_t) { return cudaErrorNotSupported; }
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kTile = 128;                 // tokens per tile
+constexpr int kSubBytes = 128 * 128;       // 128 tokens x 64 ranks x 2 B
+constexpr int kSlotBytes = 2 * kSubBytes;  // 128 tokens x 128 ranks
+constexpr int kQRows = 64;                 // 32 head rows (hi) + 32 head rows (lo)
+constexpr int kQSubBytes = kQRows * 128;   // 64 rows x 64 ranks x 2 B
+constexpr int kPBytes = 128 * 64 * 2;      // 128 tokens x (32 hi + 32 lo heads) x 2 B
+constexpr int kOColsPerChunk = 64;         // hi | lo
+constexpr int kOCol = 128;                 // first TMEM column of O~
+constexpr int kMaxSlots = 12;
+constexpr float kLazy = 8.0f;              // log2 of the allowed growth before a rescale
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kSmemLimit = 232448;         // 227 KB opt-in per block
+
+struct TcParams {
+  int r_k, r_v, ck, cv, kb_k, tmem_cols;
+  int Hq, hist_len, split_tokens, n_splits, nslot, lookahead;
+  uint32_t q_bytes;
+  float* part_o;
+  float* part_ml;
+  int* err;
+};
+
+struct Aux {
+  uint64_t slot_full[kMaxSlots];
+  uint64_t slot_empty[kMaxSlots];
+  uint64_t q_full, o_done, o_final;
+  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  float red[4][32];
+  float m_s[32];
+  float alpha_s[32];
+};
+
+struct TcState {
+  CUtensorMap q, zk, zv;
+  int nslot;
+  int lookahead;
+  size_t smem;
+};
+
+__device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((it & 31) == 0) {
+      if (*(volatile int*)&aux->abort_flag) return false;
+      if (ptx::globaltimer() - t0 > kTimeoutNs) {
+        *(volatile int*)&aux->abort_flag = 1;
+        atomicExch(err, (int)LR_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Wait that ignores the abort flag (used to drain in-flight work after an abort).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait(bar, parity))
+    if (ptx::globaltimer() - t0 > kTimeoutNs) return;
+}
+
+// Butterfly reduce-scatter over a warp: on return lane l holds op over all lanes of
+// v[l] (v is destroyed).
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool up = (lane & w) != 0;
+#pragma unroll
+    for (int k = 0; k < w; ++k) {
+      const float keep = up ? v[k + w] : v[k];
+      const float send = up ? v[k] : v[k + w];
+      const float got = __shfl_xor_sync(0xffffffffu, send, w);
+      v[k] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return v[0];
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_decode_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_zk,
+                const __grid_constant__ CUtensorMap tm_zv, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = base;
+  uint8_t* ring = base + p.q_bytes;
+  uint8_t* p_s = ring + p.nslot * kSlotBytes;
+  Aux* aux = reinterpret_cast<Aux*>(p_s + 2 * kPBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, b = blockIdx.y;
+  const int tok_begin = split * p.split_tokens;
+  const int tok_end = min(p.hist_len, tok_begin + p.split_tokens);
+  const int ntiles = tok_end > tok_begin ? (tok_end - tok_begin + kTile - 1) / kTile : 0;
+  const int per_tile = p.ck + p.cv;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.nslot; ++s) {
+      ptx::mbar_init(&aux->slot_full[s], 1);
+      ptx::mbar_init(&aux->slot_empty[s], 1);
+    }
+    ptx::mbar_init(&aux->q_full, 1);
+    ptx::mbar_init(&aux->o_done, 1);
+    ptx::mbar_init(&aux->o_final, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&aux->s_full[i], 1);
+      ptx::mbar_init(&aux->s_empty[i], 128);
+      ptx::mbar_init(&aux->p_full[i], 128);
+      ptx::mbar_init(&aux->p_empty[i], 1);
+    }
+    aux->abort_flag = 0;
+    for (int j = 0; j < 32; ++j) aux->m_s[j] = -INFINITY;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tm_q);
+    ptx::prefetch_tmap(&tm_zk);
+    ptx::prefetch_tmap(&tm_zv);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&aux->tmem_base, p.tmem_cols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = aux->tmem_base;
+  if (!(warp == 0 && lane == 0)) pdl_wait();   // the producer waits after its first loads
+  pdl_trigger();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0 && ntiles > 0) {
+      // The first tile's key chunks are issued before the grid-dependency wait: the
+      // cache was written by kernels that completed before the preceding (query
+      // projection) kernel allowed this one to start.  The query latents are not.
+      int issued = 0;
+      bool ok = true;
+      bool q_issued = false;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int t0 = tok_begin + i * kTile;
+        for (int u = 0; u < per_tile; ++u) {
+          const int pos = i * per_tile + u;
+          const int slot = pos % p.nslot, round = pos / p.nslot;
+          if (pos >= p.ck && !q_issued) {
+            pdl_wait();
+            ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
+            for (int sb = 0; sb < p.kb_k; ++sb)
+              ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
+            q_issued = true;
+          }
+          if (round > 0 && !wait_b(&aux->slot_empty[slot], (round - 1) & 1, aux, p.err)) {
+            ok = false;
+            break;
+          }
+          const bool isk = u < p.ck;
+          const int c = isk ? u : u - p.ck;
+          const int r = isk ? p.r_k : p.r_v;
+          const int nsub = (c * 128 + 64 < r) ? 2 : 1;
+          uint8_t* dst = ring + slot * kSlotBytes;
+          ptx::mbar_arrive_expect_tx(&aux->slot_full[slot], nsub * kSubBytes);
+          for (int sb = 0; sb < nsub; ++sb)
+            ptx::tma_load_3d(dst + sb * kSubBytes, isk ? &tm_zk : &tm_zv, &aux->slot_full[slot],
+                             c * 128 + sb * 64, t0, b);
+          issued = pos + 1;
+        }
+      }
+      if (!q_issued) {
+        pdl_wait();
+        ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
+        for (int sb = 0; sb < p.kb_k; ++sb)
+          ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
+        q_issued = true;
+      }
+      if (!ok) {
+        drain_wait(&aux->q_full, 0);
+        for (int pos = max(0, issued - p.nslot); pos < issued; ++pos)
+          drain_wait(&aux->slot_full[pos % p.nslot], (pos / p.nslot) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0 && ntiles > 0) {
+      const uint32_t id1 = ptx::idesc_f16(1, 0, 0, 128, 64);
+      const uint32_t id2 = ptx::idesc_f16(1, 1, 1, 128, 64);
+      const uint32_t q_addr = ptx::smem_u32(q_s), ring_addr = ptx::smem_u32(ring), p_addr = ptx::smem_u32(p_s);
+      bool ok = wait_b(&aux->q_full, 0, aux, p.err);
+      ptx::tc_fence_after();
+      auto gemm1 = [&](int i) -> bool {
+        const int buf = i & 1;
+        if (i >= 2 && !wait_b(&aux->s_empty[buf], ((i - 2) >> 1) & 1, aux, p.err)) return false;
+        ptx::tc_fence_after();
+        const uint32_t d = tmem + buf * 64;
+        for (int c = 0; c < p.ck; ++c) {
+          const int pos = i * per_tile + c;
+          const int slot = pos % p.nslot;
+          if (!wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err)) return false;
+          ptx::tc_fence_after();
+          const uint32_t sa = ring_addr + slot * kSlotBytes;
+#pragma unroll
+          for (int sb = 0; sb < 2; ++sb) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const int k0 = c * 128 + sb * 64 + kk * 16;
+              if (k0 < p.r_k) {
+                const uint64_t ad = ptx::smem_desc(sa + sb * kSubBytes + kk * 32, 16, 1024, 2);
+                const uint64_t bd = ptx::smem_desc(q_addr + (c * 2 + sb) * kQSubBytes + kk * 32, 16, 1024, 2);
+                ptx::mma_f16(d, ad, bd, id1, k0 > 0 ? 1u : 0u);
+              }
+            }
+          }
+          ptx::mma_commit(&aux->slot_empty[slot]);
+        }
+        ptx::mma_commit(&aux->s_full[buf]);
+        return true;
+      };
+      auto gemm2 = [&](int i) -> bool {
+        const int buf = i & 1;
+        if (!wait_b(&aux->p_full[buf], (i >> 1) & 1, aux, p.err)) return false;
+        ptx::tc_fence_after();
+        for (int c = 0; c < p.cv; ++c) {
+          const int pos = i * per_tile + p.ck + c;
+          const int slot = pos % p.nslot;
+          if (!wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err)) return false;
+          ptx::tc_fence_after();
+          const uint32_t sa = ring_addr + slot * kSlotBytes;
+#pragma unroll
+          for (int kt = 0; kt < 8; ++kt) {
+            const uint64_t ad = ptx::smem_desc(sa + kt * 2048, kSubBytes, 1024, 2);
+            const uint64_t bd = ptx::smem_desc(p_addr + buf * kPBytes + kt * 256, 128, 2048, 0);
+            ptx::mma_f16(tmem + kOCol + c * kOColsPerChunk, ad, bd, id2, (i > 0 || kt > 0) ? 1u : 0u);
+          }
+          ptx::mma_commit(&aux->slot_empty[slot]);
+        }
+        ptx::mma_commit(&aux->p_empty[buf]);
+        ptx::mma_commit(&aux->o_done);
+        return true;
+      };
+      if (ok) {
+        if (p.lookahead) {
+          ok = gemm1(0);
+          for (int i = 0; i < ntiles && ok; ++i) {
+            if (i + 1 < ntiles) ok = gemm1(i + 1);
+            if (ok) ok = gemm2(i);
+          }
+        } else {
+          for (int i = 0; i < ntiles && ok; ++i) {
+            ok = gemm1(i);
+            if (ok) ok = gemm2(i);
+          }
+        }
+      }
+      ptx::mma_commit(&aux->o_final);
+      if (!ok) drain_wait(&aux->o_final, 0);
+    }
+    __syncwarp();
+  } else if (ntiles > 0) {
+    // ------------------------------------------------------------- softmax / epilogue
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    float m[32], l[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      m[j] = -INFINITY;
+      l[j] = 0.f;
+    }
+    bool ok = true;
+    for (int i = 0; i < ntiles; ++i) {
+      const int buf = i & 1;
+      const bool valid = tok_begin + i * kTile + row < tok_end;
+      ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full[buf], (i >> 1) & 1, aux, p.err));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      uint32_t hi[32], lo[32];
+      ptx::tmem_ld32(tmem + lane_off + buf * 64, hi);
+      ptx::tmem_ld32(tmem + lane_off + buf * 64 + 32, lo);
+      ptx::tmem_wait_ld();
+      float s[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(hi[j]) + __uint_as_float(lo[j]) : -INFINITY;
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&aux->s_empty[buf]);
+
+      bool ex = false;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ex |= s[j] > m[j] + kLazy;
+      ex = ptx::named_bar_or(1, 128, ex);
+      if (i >= 2) {
+        ok = ptx::named_bar_and(1, 128, wait_b(&aux->p_empty[buf], ((i - 2) >> 1) & 1, aux, p.err));
+        if (!ok) break;
+      }
+      if (ex) {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = s[j];
+        aux->red[qd][lane] = warp_reduce_scatter32<true>(v, lane);
+        ptx::named_bar_sync(1, 128);
+        if (qd == 0) {
+          const float mt = fmaxf(fmaxf(aux->red[0][lane], aux->red[1][lane]), fmaxf(aux->red[2][lane], aux->red[3][lane]));
+          const float mo = aux->m_s[lane];
+          const float mn = fmaxf(mo, mt);
+          aux->alpha_s[lane] = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+          aux->m_s[lane] = mn;
+        }
+        ptx::named_bar_sync(1, 128);
+        float alpha[32];
+        bool need_o = false;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          m[j] = aux->m_s[j];
+          alpha[j] = aux->alpha_s[j];
+          l[j] *= alpha[j];
+          need_o |= alpha[j] < 1.f;
+        }
+        if (need_o && i > 0) {
+          ok = ptx::named_bar_and(1, 128, wait_b(&aux->o_done, (i - 1) & 1, aux, p.err));
+          if (!ok) break;
+          ptx::tc_fence_after();
+          for (int c = 0; c < 2 * p.cv; ++c) {
+            uint32_t v2[32];
+            ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v2[j] = __float_as_uint(__uint_as_float(v2[j]) * alpha[j]);
+            ptx::tmem_st32(tmem + lane_off + kOCol + c * 32, v2);
+          }
+          ptx::tmem_wait_st();
+        }
+      }
+      uint32_t pk[32];   // [0..15] hi pairs, [16..31] lo pairs
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const float p0 = exp2f(s[2 * jj] - m[2 * jj]);
+        const float p1 = exp2f(s[2 * jj + 1] - m[2 * jj + 1]);
+        const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(p0 - __low2float(h), p1 - __high2float(h));
+        l[2 * jj] += p0;
+        l[2 * jj + 1] += p1;
+        pk[jj] = *reinterpret_cast<const uint32_t*>(&h);
+        pk[16 + jj] = *reinterpret_cast<const uint32_t*>(&lo2);
+      }
+      const uint32_t prow = ptx::smem_u32(p_s + buf * kPBytes + row * 16);
+#pragma unroll
+      for (int hg = 0; hg < 8; ++hg)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + hg * 2048), "r"(pk[4 * hg]),
+                     "r"(pk[4 * hg + 1]), "r"(pk[4 * hg + 2]), "r"(pk[4 * hg + 3])
+                     : "memory");
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&aux->p_full[buf]);
+    }
+    if (ok) ok = ptx::named_bar_and(1, 128, wait_b(&aux->o_final, 0, aux, p.err));
+    if (ok) {
+      ptx::tc_fence_after();
+      const size_t base_out = ((size_t)b * p.n_splits + split) * p.Hq;
+      for (int c = 0; c < p.cv; ++c) {
+        uint32_t vh[32], vl[32];
+        ptx::tmem_ld32(tmem + lane_off + kOCol + c * kOColsPerChunk, vh);
+        ptx::tmem_ld32(tmem + lane_off + kOCol + c * kOColsPerChunk + 32, vl);
+        ptx::tmem_wait_ld();
+        const int e = c * 128 + qd * 32 + lane;
+        if (e < p.r_v) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < p.Hq) p.part_o[(base_out + j) * p.r_v + e] = __uint_as_float(vh[j]) + __uint_as_float(vl[j]);
+        }
+      }
+      aux->red[qd][lane] = warp_reduce_scatter32<false>(l, lane);
+      ptx::named_bar_sync(1, 128);
+      if (qd == 0 && lane < p.Hq) {
+        const float lt = (aux->red[0][lane] + aux->red[1][lane]) + (aux->red[2][lane] + aux->red[3][lane]);
+        p.part_ml[(base_out + lane) * 2] = aux->m_s[lane];
+        p.part_ml[(base_out + lane) * 2 + 1] = lt;
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+              const cuuint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int q_bytes_for(int r_k) { return ((r_k + 63) / 64) * kQSubBytes; }
+
+int slots_that_fit(const lr_cache_desc* d) {
+  const int fixed = 1024 + q_bytes_for(d->rank_k) + 2 * kPBytes + (int)sizeof(Aux);
+  return std::min(kMaxSlots, (kSmemLimit - fixed) / kSlotBytes);
+}
+
+}  // namespace
+
+bool tc_supported(const lr_cache_desc* d) {
+  if (d->dtype != LR_BF16 || d->quant_bits != 0 || d->rope_in_kernel) return false;
+  if (d->n_q_heads > 32) return false;
+  const int ck = (d->rank_k + 127) / 128, cv = (d->rank_v + 127) / 128;
+  return slots_that_fit(d) >= std::max(std::max(ck, cv), 2);
+}
+
+cudaError_t tc_prepare(lr_cache* c) {
+  const lr_cache_desc& d = c->desc;
+  if (!tc_supported(&d)) return cudaSuccess;
+  TcState* st = reinterpret_cast<TcState*>(c->tc_state);
+  if (!st) {
+    st = new (std::nothrow) TcState();
+    if (!st) return cudaErrorMemoryAllocation;
+    c->tc_state = st;
+  }
+  if (!c->qt16) {
+    cudaError_t e = cudaMalloc(&c->qt16, (size_t)d.batch * kQRows * d.rank_k * 2);
+    if (e != cudaSuccess) return e;
+    e = cudaMemset(c->qt16, 0, (size_t)d.batch * kQRows * d.rank_k * 2);
+    if (e != cudaSuccess) return e;
+  }
+  const cuuint64_t cap = d.capacity, B = d.batch;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)d.rank_k, B * kQRows};
+    cuuint64_t strides[1] = {(cuuint64_t)d.rank_k * 2};
+    cuuint32_t box[2] = {64, kQRows};
+    if (!make_map(&st->q, c->qt16, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  for (int side = 0; side < 2; ++side) {
+    const int r = side ? d.rank_v : d.rank_k;
+    cuuint64_t dims[3] = {(cuuint64_t)r, cap, B};
+    cuuint64_t strides[2] = {(cuuint64_t)r * 2, cap * r * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+    if (!make_map(side ? &st->zv : &st->zk, side ? c->z_v : c->z_k, 3, dims, strides, box))
+      return cudaErrorInvalidValue;
+  }
+  const int ck = (d.rank_k + 127) / 128, cv = (d.rank_v + 127) / 128;
+  st->nslot = slots_that_fit(&d);
+  st->lookahead = st->nslot >= ck + cv ? 1 : 0;
+  if (st->lookahead) st->nslot = std::min(st->nslot, std::max(ck + cv + 1, 4));
+  st->smem = 1024 + q_bytes_for(d.rank_k) + (size_t)st->nslot * kSlotBytes + 2 * kPBytes + sizeof(Aux);
+  return cudaSuccess;
+}
+
+void tc_release(lr_cache* c) {
+  delete reinterpret_cast<TcState*>(c->tc_state);
+  c->tc_state = nullptr;
+}
+
+cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  const TcState* st = reinterpret_cast<const TcState*>(c->tc_state);
+  if (!st) return cudaErrorNotSupported;
+  TcParams p;
+  p.r_k = d.rank_k;
+  p.r_v = d.rank_v;
+  p.ck = (d.rank_k + 127) / 128;
+  p.cv = (d.rank_v + 127) / 128;
+  p.kb_k = (d.rank_k + 63) / 64;
+  p.tmem_cols = (kOCol + p.cv * kOColsPerChunk) <= 256 ? 256 : 512;
+  p.Hq = d.n_q_heads;
+  p.hist_len = c->hist_len;
+  p.split_tokens = split_tokens;
+  p.n_splits = n_splits;
+  p.nslot = st->nslot;
+  p.lookahead = st->lookahead;
+  p.q_bytes = q_bytes_for(d.rank_k);
+  p.part_o = c->part_o;
+  p.part_ml = c->part_ml;
+  p.err = c->dev_err;
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_decode_tc, optin_done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_decode_tc, dim3(n_splits, d.batch), dim3(kThreads), st->smem, s, st->q, st->zk, st->zv, p);
+}

@@ -14,6 +14,8 @@
 
 #include <math.h>
 
+#include <algorithm>
+
 namespace {
 
 constexpr int kTileSimt = 16;     // tokens per tile in the SIMT decode
@@ -91,30 +93,108 @@ __device__ __forceinline__ void store_latent_chunk(float z, int ch, int r, int k
   }
 }
 
+// ---- cp.async staging (16-byte asynchronous global -> shared copies) --------------
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+               "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
+// Copy rows [r0, r0 + nr) x columns [col0, col0 + ncol) of a row-major matrix with row
+// stride ld (elements of `es` bytes) into shared memory with row pitch `pitch` bytes.
+// ncol * es must be a multiple of 16 and the source 16-byte aligned.
+__device__ __forceinline__ void stage_rows(uint8_t* dst, int pitch, const void* src, long long ld, int es,
+                                           int r0, int nr, long long col0, int ncol) {
+  const int vec_per_row = ncol * es / 16;
+  const int total = nr * vec_per_row;
+  const uint8_t* g = reinterpret_cast<const uint8_t*>(src);
+  for (int v = threadIdx.x; v < total; v += blockDim.x) {
+    const int rr = v / vec_per_row, cc = v % vec_per_row;
+    cp_async16(dst + rr * pitch + cc * 16, g + (((long long)(r0 + rr) * ld + col0) * es) + cc * 16);
+  }
+}
+
+__device__ __forceinline__ float smem_elem(const uint8_t* p, int dtype) {
+  if (dtype == LR_BF16) return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+  return *reinterpret_cast<const float*>(p);
+}
+
 // ---------------------------------------------------------------------------
 // query projection: q~ = s log2(e) B_k,h q  (latent path) and/or s log2(e) q
 // ---------------------------------------------------------------------------
+// One CTA per (32-row chunk of B_k,h, KV head h, sequence b).  The chunk's rows
+// (32 x d) and the group's queries are staged in shared memory; thread = (rank row,
+// query head): one d-long dot product each.
+// qt16 (tensor-core path): rows [b][j] and [b][32 + j] of a [B][64][r_k] bf16 array get
+// hi = bf16(q~) and lo = bf16(q~ - hi), so that hi + lo carries q~ to ~16 significant bits.
+constexpr int kRowsQ = 32;
+
 __global__ void __launch_bounds__(256) k_qproj(const void* q, const void* Bk, float* qt, float* qd,
-                                               int Hq, int Hkv, int d, int D, int rk, int dtype,
-                                               float scale_log2, int want_latent) {
-  __shared__ float qs[256];
-  const int j = blockIdx.x, b = blockIdx.y;
-  const int h = j / (Hq / Hkv);
-  const long long qoff = ((long long)b * Hq + j) * d;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    const float v = elem_f(q, qoff + c, dtype);
-    qs[c] = v;
-    if (qd) qd[qoff + c] = v * scale_log2;
+                                               __nv_bfloat16* qt16, int Hq, int Hkv, int d, int D, int rk,
+                                               int dtype, float scale_log2, int want_latent) {
+  extern __shared__ __align__(16) uint8_t qsm[];
+  pdl_wait();
+  pdl_trigger();
+  const int G = Hq / Hkv;
+  const int r0 = blockIdx.x * kRowsQ, h = blockIdx.y, b = blockIdx.z;
+  const int j0 = h * G;
+  const int es = dtype == LR_BF16 ? 2 : 4;
+  const int pitch = d * es + 16;
+  float* qs = reinterpret_cast<float*>(qsm);                                   // [G][d]
+  uint8_t* bs = qsm + (((size_t)G * d * sizeof(float) + 15) & ~size_t(15));   // [32][pitch]
+  const int nr = min(kRowsQ, rk - r0);
+  if (want_latent && nr > 0) stage_rows(bs, pitch, Bk, D, es, r0, nr, (long long)h * d, d);
+  for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) {
+    const long long off = ((long long)b * Hq + j0) * d + idx;
+    const float v = elem_f(q, off, dtype);
+    qs[idx] = v;
+    if (qd && blockIdx.x == 0) qd[off] = v * scale_log2;
   }
-  __syncthreads();
   if (!want_latent) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  for (int i = warp; i < rk; i += nw) {
-    float s = 0.f;
-    for (int c = lane; c < d; c += 32) s = fmaf(elem_f(Bk, (long long)i * D + h * d + c, dtype), qs[c], s);
+  cp_async_wait_all();
+  __syncthreads();
+  const int lane = threadIdx.x & 31, hs0 = threadIdx.x >> 5;
+  if (lane >= nr) return;
+  const uint8_t* row = bs + lane * pitch;
+  const int i = r0 + lane;
+  for (int hs = hs0; hs < G; hs += 8) {
+    const float* qr = qs + hs * d;
+    float a0 = 0.f, a1 = 0.f;
+    for (int c = 0; c < d; c += 8) {
+      float bv[8];
+      if (dtype == LR_BF16) {
+        const uint4 u4 = *reinterpret_cast<const uint4*>(row + c * 2);
+        const uint32_t w[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) qt[((long long)b * Hq + j) * rk + i] = s * scale_log2;
+        for (int k = 0; k < 4; ++k) {
+          bv[2 * k] = __uint_as_float(w[k] << 16);
+          bv[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+        }
+      } else {
+        const float4 f0 = *reinterpret_cast<const float4*>(row + c * 4);
+        const float4 f1 = *reinterpret_cast<const float4*>(row + c * 4 + 16);
+        bv[0] = f0.x; bv[1] = f0.y; bv[2] = f0.z; bv[3] = f0.w;
+        bv[4] = f1.x; bv[5] = f1.y; bv[6] = f1.z; bv[7] = f1.w;
+      }
+      const float4 q0 = *reinterpret_cast<const float4*>(qr + c);
+      const float4 q1 = *reinterpret_cast<const float4*>(qr + c + 4);
+      a0 = fmaf(bv[0], q0.x, a0); a1 = fmaf(bv[1], q0.y, a1);
+      a0 = fmaf(bv[2], q0.z, a0); a1 = fmaf(bv[3], q0.w, a1);
+      a0 = fmaf(bv[4], q1.x, a0); a1 = fmaf(bv[5], q1.y, a1);
+      a0 = fmaf(bv[6], q1.z, a0); a1 = fmaf(bv[7], q1.w, a1);
+    }
+    const int j = j0 + hs;
+    const float v = (a0 + a1) * scale_log2;
+    qt[((long long)b * Hq + j) * rk + i] = v;
+    if (qt16) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+      qt16[((long long)b * 64 + j) * rk + i] = hi;
+      qt16[((long long)b * 64 + 32 + j) * rk + i] = lo;
+    }
   }
 }
 
@@ -123,6 +203,8 @@ __global__ void __launch_bounds__(256) k_qproj(const void* q, const void* Bk, fl
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind) {
   extern __shared__ float sm[];
+  pdl_wait();
+  pdl_trigger();
   const int split = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
   const int Hq = a.Hq, rk = a.k.r, rv = a.v.r;
   const int qdim = a.rope ? a.d : rk;
@@ -242,6 +324,8 @@ __global__ void __launch_bounds__(128) k_window(const void* win_k, const void* w
   float* q_s = wsm;           // [d]
   float* p_s = wsm + d;       // [win_len]
   __shared__ float red[2];
+  pdl_wait();
+  pdl_trigger();
   const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int h = j / (Hq / Hkv);
   const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
@@ -285,62 +369,113 @@ __global__ void __launch_bounds__(128) k_window(const void* win_k, const void* w
 }
 
 // ---------------------------------------------------------------------------
-// split merge (log-sum-exp) and output projection o = o~ B_v,h / l
+// split merge (log-sum-exp) and output projection o = o~ B_v,h / l.
+// One CTA (512 threads) per (KV head h, sequence b).  The B_v,h slice is prefetched
+// into shared memory with asynchronous copies while the split weights and the
+// combined rank-space outputs o~ of the group's query heads are formed (every thread
+// issues all of its partial loads before using any); then thread = (output column,
+// query-head slot).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) k_merge(const float* part_o, const float* part_ml,
-                                               const float* win_o, const float* win_ml,
-                                               const void* Bv, void* out, float* lse, int S,
-                                               int Hq, int Hkv, int d, int D, int rv, int dtype) {
-  extern __shared__ float msm[];
-  float* ot = msm;            // [rv]
-  float* w_s = msm + rv;      // [S]
-  __shared__ float ml[3];     // m*, l, window weight
-  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int h = j / (Hq / Hkv);
-  if (tid < 32) {
+constexpr int kMergeThreads = 512;
+constexpr size_t kMergeStage = 96 * 1024;   // bytes of B_v,h rows staged in shared memory
+constexpr int kMergeSlots = 8;    // partial outputs per thread held in flight
+
+__global__ void __launch_bounds__(kMergeThreads) k_merge(const float* part_o, const float* part_ml,
+                                                         const float* win_o, const float* win_ml,
+                                                         const void* Bv, void* out, float* lse, int S,
+                                                         int Hq, int Hkv, int d, int D, int rv, int dtype) {
+  extern __shared__ __align__(16) float msm[];
+  const int G = Hq / Hkv;
+  float* ot = msm;               // [G][rv]
+  float* w_s = ot + G * rv;      // [G][S]
+  float* hdr = w_s + G * S;      // [G][3]: m*, 1/l, window weight
+  uint8_t* bs = reinterpret_cast<uint8_t*>(msm) + ((((size_t)G * (rv + S + 3)) * sizeof(float) + 15) & ~size_t(15));
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int j0 = h * G;
+  const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
+  const int es = dtype == LR_BF16 ? 2 : 4;
+  const int pitch = d * es;
+  const int rows_staged = min(rv, (int)(kMergeStage / pitch));
+  stage_rows(bs, pitch, Bv, D, es, 0, rows_staged, (long long)h * d, d);   // bases: stable data
+  pdl_wait();
+  pdl_trigger();
+  for (int jj = warp; jj < G; jj += nw) {
+    const int j = j0 + jj;
     float m = -INFINITY;
-    for (int s = tid; s < S; s += 32) m = fmaxf(m, part_ml[(((size_t)b * S + s) * Hq + j) * 2]);
+    for (int s = lane; s < S; s += 32) m = fmaxf(m, part_ml[(((size_t)b * S + s) * Hq + j) * 2]);
     const float mw = win_ml ? win_ml[((size_t)b * Hq + j) * 2] : -INFINITY;
     m = fmaxf(m, mw);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float l = 0.f;
-    for (int s = tid; s < S; s += 32) {
+    for (int s = lane; s < S; s += 32) {
       const size_t e = (((size_t)b * S + s) * Hq + j) * 2;
       const float ms = part_ml[e];
       const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - m);
-      w_s[s] = w;
+      w_s[jj * S + s] = w;
       l = fmaf(w, part_ml[e + 1], l);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (tid == 0) {
+    if (lane == 0) {
       float ww = 0.f;
       if (win_ml && mw != -INFINITY) {
         ww = exp2f(mw - m);
         l = fmaf(ww, win_ml[((size_t)b * Hq + j) * 2 + 1], l);
       }
-      ml[0] = m;
-      ml[1] = l;
-      ml[2] = ww;
+      hdr[jj * 3] = m;
+      hdr[jj * 3 + 1] = 1.0f / l;
+      hdr[jj * 3 + 2] = ww;
+      if (lse) lse[(long long)b * Hq + j] = (m + log2f(l)) * LR_LN2;
     }
   }
   __syncthreads();
-  for (int i = tid; i < rv; i += blockDim.x) {
-    float o = 0.f;
-    for (int s = 0; s < S; ++s) o = fmaf(w_s[s], part_o[(((size_t)b * S + s) * Hq + j) * rv + i], o);
-    ot[i] = o;
+  const size_t sstride = (size_t)Hq * rv;
+  const float* pbase = part_o + ((size_t)b * S * Hq + j0) * rv;
+  for (int base = 0; base < G * rv; base += nt * kMergeSlots) {
+    float acc[kMergeSlots];
+#pragma unroll
+    for (int k = 0; k < kMergeSlots; ++k) acc[k] = 0.f;
+    for (int s = 0; s < S; ++s) {
+#pragma unroll
+      for (int k = 0; k < kMergeSlots; ++k) {
+        const int idx = base + k * nt + tid;
+        if (idx < G * rv) {
+          const int jj = idx / rv;
+          acc[k] = fmaf(w_s[jj * S + s], pbase[(size_t)s * sstride + idx], acc[k]);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kMergeSlots; ++k) {
+      const int idx = base + k * nt + tid;
+      if (idx < G * rv) ot[idx] = acc[k];
+    }
   }
+  cp_async_wait_all();
   __syncthreads();
-  const float inv_l = 1.0f / ml[1];
-  const long long ooff = ((long long)b * Hq + j) * d;
-  for (int c = tid; c < d; c += blockDim.x) {
-    float o = 0.f;
-    for (int i = 0; i < rv; ++i) o = fmaf(ot[i], elem_f(Bv, (long long)i * D + (long long)h * d + c, dtype), o);
-    if (win_o) o = fmaf(ml[2], win_o[ooff + c], o);
-    store_elem(out, ooff + c, o * inv_l, dtype);
+  // projection: thread = (column c, head slot); ranks beyond the staged rows are read
+  // from global memory (only when the slice does not fit the staging buffer)
+  const int slots = nt / d > 0 ? nt / d : 1;
+  const int c = tid % d, slot = tid / d;
+  if (slot >= slots || c >= d) return;
+  for (int jj = slot; jj < G; jj += slots) {
+    const float* orow = ot + jj * rv;
+    float a0 = 0.f, a1 = 0.f;
+    int i = 0;
+    for (; i + 1 < rows_staged; i += 2) {
+      a0 = fmaf(orow[i], smem_elem(bs + i * pitch + c * es, dtype), a0);
+      a1 = fmaf(orow[i + 1], smem_elem(bs + (i + 1) * pitch + c * es, dtype), a1);
+    }
+    for (; i < rv; ++i)
+      a0 = fmaf(orow[i], i < rows_staged ? smem_elem(bs + i * pitch + c * es, dtype)
+                                         : elem_f(Bv, (long long)i * D + (long long)h * d + c, dtype), a0);
+    const long long ooff = ((long long)b * Hq + j0 + jj) * d + c;
+    float o = a0 + a1;
+    if (win_o) o = fmaf(hdr[jj * 3 + 2], win_o[ooff], o);
+    store_elem(out, ooff, o * hdr[jj * 3 + 1], dtype);
   }
-  if (lse && tid == 0) lse[(long long)b * Hq + j] = (ml[0] + log2f(ml[1])) * LR_LN2;
 }
 
 // ---------------------------------------------------------------------------
@@ -359,48 +494,64 @@ struct AppendArgs {
   int B, D, kind, dtype;
 };
 
+// One CTA per (32-coordinate chunk of K or V, sequence b).  The chunk's columns of A
+// ([D][32]) and the source row are staged in shared memory with asynchronous copies;
+// the 8 warps take fixed eighths of the D-long dot products and the partial sums are
+// added in a fixed order, so the result does not depend on the storage kind.
 __global__ void __launch_bounds__(256) k_append(AppendArgs a) {
-  const int x = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  extern __shared__ __align__(16) uint8_t asm_[];
+  __shared__ float red[8][32];
+  pdl_wait();
+  pdl_trigger();
+  const int x = blockIdx.x, b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nproj = a.project ? (a.chunks_k + a.chunks_v) : 0;
+  const int es = a.dtype == LR_BF16 ? 2 : 4;
   if (x < nproj) {
     const bool is_k = x < a.chunks_k;
     const int ch = is_k ? x : x - a.chunks_k;
     const int r = is_k ? a.rk : a.rv;
     const void* A = is_k ? a.A_k : a.A_v;
     const void* src = is_k ? a.src_k : a.src_v;
-    const int i = ch * 32 + lane;
-    const bool valid = i < r;
-    for (int b = warp; b < a.B; b += nw) {
-      float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
-      if (valid) {
-        const long long so = (long long)b * a.src_bstride;
-        int c = 0;
-        for (; c + 3 < a.D; c += 4) {
-          z0 = fmaf(elem_f(src, so + c, a.dtype), elem_f(A, (long long)c * r + i, a.dtype), z0);
-          z1 = fmaf(elem_f(src, so + c + 1, a.dtype), elem_f(A, (long long)(c + 1) * r + i, a.dtype), z1);
-          z2 = fmaf(elem_f(src, so + c + 2, a.dtype), elem_f(A, (long long)(c + 2) * r + i, a.dtype), z2);
-          z3 = fmaf(elem_f(src, so + c + 3, a.dtype), elem_f(A, (long long)(c + 3) * r + i, a.dtype), z3);
-        }
-        for (; c < a.D; ++c) z0 = fmaf(elem_f(src, so + c, a.dtype), elem_f(A, (long long)c * r + i, a.dtype), z0);
+    const int ncol = min(32, r - ch * 32);         // 16 or 32 (ranks are multiples of 16)
+    uint8_t* As = asm_;                            // [D][32], pitch 32 * es
+    uint8_t* xs = asm_ + (size_t)a.D * 32 * es;    // [D]
+    stage_rows(As, 32 * es, A, r, es, 0, a.D, (long long)ch * 32, ncol);
+    const uint8_t* g = reinterpret_cast<const uint8_t*>(src) + (size_t)b * a.src_bstride * es;
+    for (int v = threadIdx.x; v < a.D * es / 16; v += blockDim.x) cp_async16(xs + v * 16, g + v * 16);
+    cp_async_wait_all();
+    __syncthreads();
+    const int per = (a.D + 7) / 8;
+    const int cb = warp * per, ce = min(a.D, cb + per);
+    float z0 = 0.f, z1 = 0.f;
+    if (lane < ncol) {
+      int c = cb;
+      for (; c + 1 < ce; c += 2) {
+        z0 = fmaf(smem_elem(xs + c * es, a.dtype), smem_elem(As + (c * 32 + lane) * es, a.dtype), z0);
+        z1 = fmaf(smem_elem(xs + (c + 1) * es, a.dtype), smem_elem(As + ((c + 1) * 32 + lane) * es, a.dtype), z1);
       }
-      const float z = (z0 + z1) + (z2 + z3);
+      if (c < ce) z0 = fmaf(smem_elem(xs + c * es, a.dtype), smem_elem(As + (c * 32 + lane) * es, a.dtype), z0);
+    }
+    red[warp][lane] = z0 + z1;
+    __syncthreads();
+    if (warp == 0) {
+      float z = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) z += red[w][lane];
       const long long row = (long long)b * a.cap + a.dst_slot;
       store_latent_chunk(z, ch, r, a.kind, a.dtype, is_k ? a.Zk : a.Zv, is_k ? a.codes_k : a.codes_v,
                          is_k ? a.params_k : a.params_v, is_k ? a.Gk : a.Gv, row);
     }
     return;
   }
-  // ring write of the exact new token
+  // ring write of the exact new token of sequence b
   const bool is_k = (x - nproj) == 0;
   const void* src = is_k ? a.new_k : a.new_v;
   void* dst = is_k ? a.win_k : a.win_v;
-  const size_t es = a.dtype == LR_BF16 ? 2 : 4;
-  for (int idx = threadIdx.x; idx < a.B * a.D; idx += blockDim.x) {
-    const int b = idx / a.D, c = idx % a.D;
+  for (int c = threadIdx.x; c < a.D; c += blockDim.x) {
     const long long so = (long long)b * a.D + c;
     const long long dof = ((long long)b * a.slots + a.new_slot) * a.D + c;
-    if (es == 2) reinterpret_cast<uint16_t*>(dst)[dof] = reinterpret_cast<const uint16_t*>(src)[so];
+    if (a.dtype == LR_BF16) reinterpret_cast<uint16_t*>(dst)[dof] = reinterpret_cast<const uint16_t*>(src)[so];
     else reinterpret_cast<uint32_t*>(dst)[dof] = reinterpret_cast<const uint32_t*>(src)[so];
   }
 }
@@ -412,6 +563,8 @@ __global__ void __launch_bounds__(256) k_append_latent(const float* zk, const fl
                                                        uint32_t* codes_v, uint32_t* params_k,
                                                        uint32_t* params_v, int Gk, int Gv,
                                                        long long cap, int slot0, int kind, int dtype) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long pi = (long long)blockIdx.x * (blockDim.x >> 5) + warp;
   const int per_tok = chunks_k + chunks_v;
@@ -433,6 +586,8 @@ __global__ void __launch_bounds__(256) k_append_latent(const float* zk, const fl
 __global__ void __launch_bounds__(256) k_sync_simt(void* Z, const float* R, int r, long long cap,
                                                    int hist_len, int dtype) {
   extern __shared__ float zs[];   // [kSyncRows][r]
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.y;
   const int t0 = blockIdx.x * kSyncRows;
   const int n = min(kSyncRows, hist_len - t0);
@@ -471,15 +626,25 @@ LatentRef latent_ref(const lr_cache* c, bool k) {
 // launchers
 // ---------------------------------------------------------------------------
 
-cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s) {
+static cudaError_t qproj(const lr_cache* c, const void* q, cudaStream_t s, bool tc) {
   const lr_cache_desc& d = c->desc;
   const bool rope = d.rope_in_kernel != 0;
   float* qd = (rope || c->win_slots) ? (rope ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k) : nullptr;
-  dim3 grid(d.n_q_heads, d.batch);
-  k_qproj<<<grid, 256, 0, s>>>(q, c->B_k, c->qt, qd, d.n_q_heads, d.n_kv_heads, d.head_dim, c->D,
-                               d.rank_k, d.dtype, c->scale_log2, rope ? 0 : 1);
-  lr_count_launch();
-  return cudaGetLastError();
+  dim3 grid(rope ? 1 : (d.rank_k + kRowsQ - 1) / kRowsQ, d.n_kv_heads, d.batch);
+  const size_t smem = (((size_t)(d.n_q_heads / d.n_kv_heads) * d.head_dim * sizeof(float) + 15) & ~size_t(15)) +
+                      (size_t)kRowsQ * (d.head_dim * c->esize + 16);
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_qproj, optin_done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_qproj, grid, dim3(256), smem, s, q, c->B_k, c->qt, qd, tc ? (__nv_bfloat16*)c->qt16 : nullptr, d.n_q_heads,
+                               d.n_kv_heads, d.head_dim, c->D, d.rank_k, d.dtype, c->scale_log2, rope ? 0 : 1);
+}
+
+cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s) { return qproj(c, q, s, false); }
+
+cudaError_t launch_qproj_tc(const lr_cache* c, const void* q, cudaStream_t s) {
+  if (!c->qt16) return cudaErrorNotSupported;
+  return qproj(c, q, s, true);
 }
 
 size_t decode_simt_smem(const lr_cache* c) {
@@ -505,12 +670,11 @@ cudaError_t launch_decode_simt(const lr_cache* c, int n_splits, int split_tokens
   a.hist_len = c->hist_len; a.split_tokens = split_tokens; a.n_splits = n_splits;
   a.rope = d.rope_in_kernel; a.dtype = d.dtype;
   const size_t smem = decode_simt_smem(c);
-  cudaError_t e = cudaFuncSetAttribute(k_decode_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_decode_simt, optin_done);
   if (e != cudaSuccess) return e;
   dim3 grid(n_splits, d.batch);
-  k_decode_simt<<<grid, 256, smem, s>>>(a, c->latent_kind);
-  lr_count_launch();
-  return cudaGetLastError();
+  return launch_pdl(k_decode_simt, grid, dim3(256), smem, s, a, c->latent_kind);
 }
 
 cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
@@ -518,22 +682,23 @@ cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
   const float* qd = d.rope_in_kernel ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k;
   const size_t smem = (size_t)(d.head_dim + c->win_len + 1) * sizeof(float);
   dim3 grid(d.n_q_heads, d.batch);
-  k_window<<<grid, 128, smem, s>>>(c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads, d.n_kv_heads,
+  return launch_pdl(k_window, grid, dim3(128), smem, s, c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads, d.n_kv_heads,
                                    d.head_dim, c->D, c->win_slots, c->hist_len, c->win_len, d.dtype);
-  lr_count_launch();
-  return cudaGetLastError();
 }
 
 cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s) {
   const lr_cache_desc& d = c->desc;
   const bool win = c->win_slots > 0;
-  const size_t smem = (size_t)(d.rank_v + n_splits) * sizeof(float);
-  dim3 grid(d.n_q_heads, d.batch);
-  k_merge<<<grid, 128, smem, s>>>(c->part_o, c->part_ml, win ? c->win_o : nullptr, win ? c->win_ml : nullptr,
+  const int G = d.n_q_heads / d.n_kv_heads;
+  const size_t stage = std::min(kMergeStage, (size_t)d.rank_v * d.head_dim * c->esize);
+  const size_t smem = (((size_t)G * (d.rank_v + n_splits + 3) * sizeof(float) + 15) & ~size_t(15)) + stage;
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_merge, optin_done);
+  if (e != cudaSuccess) return e;
+  dim3 grid(d.n_kv_heads, d.batch);
+  return launch_pdl(k_merge, grid, dim3(kMergeThreads), smem, s, c->part_o, c->part_ml, win ? c->win_o : nullptr, win ? c->win_ml : nullptr,
                                   c->B_v, out, lse, n_splits, d.n_q_heads, d.n_kv_heads, d.head_dim, c->D,
                                   d.rank_v, d.dtype);
-  lr_count_launch();
-  return cudaGetLastError();
 }
 
 cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s) {
@@ -562,10 +727,12 @@ cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_
   a.new_slot = win ? (c->len % c->win_slots) : 0;
   a.B = d.batch; a.D = c->D; a.kind = c->latent_kind; a.dtype = d.dtype;
   const int nproj = a.project ? a.chunks_k + a.chunks_v : 0;
-  const int grid = nproj + (win ? 2 : 0);
-  k_append<<<grid, 256, 0, s>>>(a);
-  lr_count_launch();
-  return cudaGetLastError();
+  dim3 grid(nproj + (win ? 2 : 0), d.batch);
+  const size_t smem = (size_t)c->D * 32 * c->esize + (size_t)c->D * c->esize;
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_append, optin_done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_append, grid, dim3(256), smem, s, a);
 }
 
 cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, int n, cudaStream_t s) {
@@ -573,11 +740,9 @@ cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, 
   const int chunks_k = (d.rank_k + 31) / 32, chunks_v = (d.rank_v + 31) / 32;
   const long long pairs = (long long)n * (chunks_k + chunks_v);
   dim3 grid((unsigned)((pairs + 7) / 8), d.batch);
-  k_append_latent<<<grid, 256, 0, s>>>(zk, zv, n, d.batch, d.rank_k, d.rank_v, chunks_k, chunks_v, c->z_k,
+  return launch_pdl(k_append_latent, grid, dim3(256), 0, s, zk, zv, n, d.batch, d.rank_k, d.rank_v, chunks_k, chunks_v, c->z_k,
                                        c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->G_k,
                                        c->G_v, d.capacity, c->hist_len, c->latent_kind, d.dtype);
-  lr_count_launch();
-  return cudaGetLastError();
 }
 
 cudaError_t launch_sync_simt(lr_cache* c, const float* R, int which, cudaStream_t s) {
@@ -586,10 +751,9 @@ cudaError_t launch_sync_simt(lr_cache* c, const float* R, int which, cudaStream_
   void* Z = which == 0 ? c->z_k : c->z_v;
   if (c->hist_len == 0) return cudaSuccess;
   const size_t smem = (size_t)kSyncRows * r * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(k_sync_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_sync_simt, optin_done);
   if (e != cudaSuccess) return e;
   dim3 grid((c->hist_len + kSyncRows - 1) / kSyncRows, d.batch);
-  k_sync_simt<<<grid, 256, smem, s>>>(Z, R, r, d.capacity, c->hist_len, d.dtype);
-  lr_count_launch();
-  return cudaGetLastError();
+  return launch_pdl(k_sync_simt, grid, dim3(256), smem, s, Z, R, r, d.capacity, c->hist_len, d.dtype);
 }

@@ -17,7 +17,7 @@ lr_status validate_desc(const lr_cache_desc* d) {
   if (!d) return LR_ERR_INVALID_ARG;
   if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1) return LR_ERR_INVALID_ARG;
   if (d->n_q_heads % d->n_kv_heads) return LR_ERR_INVALID_ARG;
-  if (d->head_dim < 2 || d->head_dim % 2 || d->head_dim > 256) return LR_ERR_INVALID_ARG;
+  if (d->head_dim < 8 || d->head_dim % 8 || d->head_dim > 256) return LR_ERR_INVALID_ARG;
   if (d->rank_k < 16 || d->rank_k % 16 || d->rank_k > 512) return LR_ERR_INVALID_ARG;
   if (d->rank_v < 16 || d->rank_v % 16 || d->rank_v > 512) return LR_ERR_INVALID_ARG;
   if (d->capacity < 1 || d->window < 0 || d->window > d->capacity) return LR_ERR_INVALID_ARG;
@@ -31,7 +31,7 @@ lr_status validate_desc(const lr_cache_desc* d) {
   for (int i = 0; i < 5; ++i)
     if (d->reserved[i] != 0) return LR_ERR_INVALID_ARG;
   if ((long long)d->n_kv_heads * d->head_dim > 4096) return LR_ERR_UNSUPPORTED;
-  if (d->n_q_heads > 128) return LR_ERR_UNSUPPORTED;
+  if (d->n_q_heads > 128 || d->n_q_heads / d->n_kv_heads > 64) return LR_ERR_UNSUPPORTED;
   return LR_OK;
 }
 
@@ -50,7 +50,10 @@ lr_status plan(const lr_cache_desc* d, int hist_len, int num_sms, int path, int 
   const int tiles = std::max(1, (hist_len + tile - 1) / tile);
   int splits = n_splits;
   if (splits <= 0) {
-    const int target = std::max(1, (2 * std::max(num_sms, 1) + d->batch - 1) / d->batch);
+    // SIMT: about two CTAs per SM; tensor-core path: one CTA per SM (one wave)
+    const int sms = std::max(num_sms, 1);
+    const int target = (p == LR_PATH_TC) ? std::max(1, sms / d->batch)
+                                         : std::max(1, (2 * sms + d->batch - 1) / d->batch);
     splits = std::min(tiles, target);
   }
   splits = std::max(1, std::min(splits, tiles));
@@ -89,6 +92,16 @@ void free_all(lr_cache* c) {
                   c->win_o, c->win_ml, c->dev_err};
   for (void* p : ptrs)
     if (p) cudaFree(p);
+}
+
+// Record a caller's timing event; inside stream capture it becomes an external event
+// node, so that every replay of the graph records it.
+cudaError_t record_event(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
+  if (cs == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+  return cudaEventRecord(ev, s);
 }
 
 lr_status cuda_status(cudaError_t e) {
@@ -223,6 +236,7 @@ lr_status lr_cache_destroy(lr_cache* c) {
 
 lr_status lr_kv_append(lr_cache* c, const void* k, const void* v, void* stream) {
   if (!c || !k || !v || !c->has_A) return LR_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15) return LR_ERR_INVALID_ARG;
   if (c->len >= c->desc.capacity) return LR_ERR_CAPACITY;
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
@@ -270,11 +284,11 @@ lr_status lr_attn_decode(lr_cache* c, const void* q, void* out, float* lse, void
   if (p.path != LR_PATH_TC && c->hist_len > 0 && decode_simt_smem(c) > 227 * 1024) return LR_ERR_UNSUPPORTED;
   e = p.path == LR_PATH_TC ? launch_qproj_tc(c, q, s) : launch_qproj(c, q, s);
   if (e == cudaSuccess && c->hist_len > 0) {
-    if (c->ev_start) e = cudaEventRecord(c->ev_start, s);
+    if (c->ev_start) e = record_event(c->ev_start, s);
     if (e == cudaSuccess)
       e = p.path == LR_PATH_TC ? launch_decode_tc(c, p.n_splits, p.split_tokens, s)
                                : launch_decode_simt(c, p.n_splits, p.split_tokens, s);
-    if (e == cudaSuccess && c->ev_stop) e = cudaEventRecord(c->ev_stop, s);
+    if (e == cudaSuccess && c->ev_stop) e = record_event(c->ev_stop, s);
   }
   const int S = c->hist_len > 0 ? p.n_splits : 0;
   if (e == cudaSuccess && c->win_slots) e = launch_window(c, s);

@@ -7,6 +7,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "lr_kv.h"
 
 #define LR_LOG2E 1.4426950408889634f
@@ -94,3 +96,48 @@ cudaError_t launch_qproj_tc(const lr_cache* c, const void* q, cudaStream_t s);
 cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s);
 
 void lr_count_launch(int n = 1);
+
+// Programmatic dependent launch.  Every kernel of the library does its prologue on data
+// no in-flight kernel writes, then pdl_wait() (the preceding grid has completed and its
+// memory is visible), then pdl_trigger() (the next grid may start its own prologue).
+// Because each kernel triggers only after its wait, everything before the preceding
+// kernel has completed whenever a prologue runs.  Both are no-ops without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch with the programmatic-stream-serialization attribute; returns the launch error.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  lr_count_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Raise a kernel's dynamic shared-memory limit to the 227 KB opt-in maximum (less its
+// static shared memory) once per device; later launches skip the call, so launches stay
+// legal inside stream capture.
+template <typename Kernel>
+inline cudaError_t smem_optin(Kernel k, std::atomic<uint32_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint32_t bit = 1u << (dev & 31);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, k);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448 - (int)fa.sharedSizeBytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  else (void)cudaGetLastError();   // do not leave a stale error for a later launch check
+  return e;
+}

@@ -141,6 +141,8 @@ def compare(p: synth.Problem, got, ref, got_lse=None, ref_lse=None, pairs=None, 
 def sharp_factor(p: synth.Problem, target_std: float = 2.0) -> float:
     """Query multiplier that makes the logits' spread about `target_std` (natural-log
     units), so the softmax is far from uniform."""
+    if p.hist_len < 2:
+        return 1.0
     b = 0
     qv = stored_value(p, p.q)[b]
     Zk = oracle_latents(p, p.z_k[b][: min(256, p.hist_len)])

@@ -11,8 +11,16 @@ from tests import helpers as H
 pytestmark = pytest.mark.gpu
 
 
-def paths(lr):
+def paths(lr, p=None):
+    """Decode paths to check: the fp32 CUDA-core path always, the tcgen05 path where the
+    cache supports it."""
     out = [lr.LR_PATH_SIMT]
+    if p is not None:
+        try:
+            lr.lr_plan_decode(H.desc_for(lr, p), max(p.length, 1), 148, lr.LR_PATH_TC)
+            out.append(lr.LR_PATH_TC)
+        except lr.LRError:
+            pass
     return out
 
 
@@ -33,7 +41,7 @@ def test_decode_parity(lib, kind, sharp):
     c = H.fill_cache(lib, p)
     q = _sharp(p) if sharp else p.q
     ref, ref_lse = H.oracle_decode(p, q)
-    for path in paths(lib):
+    for path in paths(lib, p):
         lib.lr_cache_set_path(c, path)
         got, lse = H.gpu_decode(lib, p, c, q)
         H.compare(p, got, ref, lse, ref_lse, tag=f"{kind} sharp={sharp} path={path}")
@@ -289,8 +297,8 @@ def test_split_count_invariance(lib, kind):
     c = H.fill_cache(lib, p)
     q = _sharp(p)
     outs = []
-    for path in paths(lib):
-        for s in (1, 2, 7, 60):
+    for path in paths(lib, p):
+        for s in ((1, 2, 7, 60) if path == lib.LR_PATH_SIMT else (1, 2, 3, 8)):
             lib.lr_cache_set_path(c, path, s)
             got, lse = H.gpu_decode(lib, p, c, q)
             outs.append((got, lse))
@@ -300,12 +308,17 @@ def test_split_count_invariance(lib, kind):
         assert np.max(np.abs(lse - ref[1])) <= 1e-4
 
 
-def test_single_token_returns_value(lib):
-    p = synth.small_variant("qwen4k", length=1, batch=2)
+@pytest.mark.parametrize("length", [1, 127, 128, 129, 255, 257])
+def test_tile_edges(lib, length):
+    """Lengths around the 128-token tile: T=1 returns v^ (up to rounding), ragged tails."""
+    p = synth.small_variant("qwen4k", length=length, batch=2)
     c = H.fill_cache(lib, p)
-    got, lse = H.gpu_decode(lib, p, c)
-    ref, ref_lse = H.oracle_decode(p)
-    H.compare(p, got, ref, lse, ref_lse, tag="T=1")
+    q = _sharp(p)
+    ref, ref_lse = H.oracle_decode(p, q)
+    for path in paths(lib, p):
+        lib.lr_cache_set_path(c, path)
+        got, lse = H.gpu_decode(lib, p, c, q)
+        H.compare(p, got, ref, lse, ref_lse, tag=f"T={length} path={path}")
 
 
 def test_gqa_identical_queries_identical_outputs(lib):
@@ -313,9 +326,11 @@ def test_gqa_identical_queries_identical_outputs(lib):
     q = p.q.copy()
     q[:, 1:7] = q[:, 0:1]                  # heads 0..6 share KV head 0
     c = H.fill_cache(lib, p)
-    got, _ = H.gpu_decode(lib, p, c, q)
-    for j in range(1, 7):
-        assert np.array_equal(got[:, j], got[:, 0])
+    for path in paths(lib, p):
+        lib.lr_cache_set_path(c, path)
+        got, _ = H.gpu_decode(lib, p, c, q)
+        for j in range(1, 7):
+            assert np.array_equal(got[:, j], got[:, 0])
 
 
 def test_window_only_and_history_only(lib):
