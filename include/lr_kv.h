@@ -163,6 +163,34 @@ lr_status lr_basis_sync(lr_cache* cache, const float* R_k, const float* R_v,
                         const void* B_k_new, const void* B_v_new, const void* A_k_new,
                         const void* A_v_new, void* stream);
 
+/* ---- decode without device allocation ----------------------------------------
+ * (No counterpart on the pages; this entry point exists for callers that cannot
+ * allocate device memory at decode time: serving engines that reserve almost all HBM
+ * up front for their own pools, and latency-critical loops that cannot take the
+ * implicit device synchronisation of cudaMalloc.)
+ * lr_attn_decode_noalloc — the decode of lr_attn_decode, computed on the fp32
+ *   CUDA-core path over caller-owned unquantised latents, without allocating: its
+ *   working memory (query latents and per-split partial results) is one static device
+ *   array of LR_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
+ *   process exit.
+ *   desc: as for lr_cache_create, with window 0, quant_bits 0 and rope_in_kernel 0
+ *     (otherwise LR_ERR_UNSUPPORTED); len: tokens to attend, 1..capacity.
+ *   z_k [B][capacity][r_k], z_v [B][capacity][r_v]: latents in the cache layout;
+ *   B_k [r_k][D], B_v [r_v][D], q [B][Hq][d], out [B][Hq][d]: dtype, device;
+ *   lse [B][Hq] fp32 or NULL.
+ *   Uses fewer sequence splits when needed to fit the array, and returns
+ *   LR_ERR_CAPACITY when even one split's working set exceeds it
+ *   (4 * B * Hq * (r_k + r_v + 2) bytes > LR_NOALLOC_SCRATCH_BYTES).
+ *   The first call on a device looks up the array's device address with that device
+ *   current (cudaGetSymbolAddress); make that first call outside any stream capture.
+ *   Every call overwrites the parts of the array it reads, so nothing carries over
+ *   between calls; but all calls share the one array, so calls whose kernels can
+ *   overlap on the GPU (unordered streams) race and corrupt each other's results. */
+#define LR_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+lr_status lr_attn_decode_noalloc(const lr_cache_desc* desc, int32_t len, const void* z_k,
+                                 const void* z_v, const void* B_k, const void* B_v,
+                                 const void* q, void* out, float* lse, void* stream);
+
 /* ---- bookkeeping ------------------------------------------------------------ */
 /* Current total length, history length and window length (host-side counters). */
 lr_status lr_cache_get_len(const lr_cache* cache, int32_t* len, int32_t* hist_len,

@@ -10,7 +10,7 @@ Functions keep the C names: lr_cache_create, lr_cache_destroy, lr_kv_append,
 lr_kv_append_latent, lr_attn_decode, lr_basis_sync, lr_cache_get_len,
 lr_cache_truncate, lr_cache_view_get, lr_cache_set_path, lr_cache_plan,
 lr_plan_decode, lr_cache_set_kernel_events, lr_device_error, lr_abi_struct_sizes,
-lr_status_string, lr_launch_count.
+lr_status_string, lr_launch_count, lr_attn_decode_noalloc.
 """
 from __future__ import annotations
 
@@ -81,6 +81,7 @@ def _load() -> ctypes.CDLL:
         "lr_plan_decode": [ctypes.POINTER(lr_cache_desc), i32, i32, i32, i32, ctypes.POINTER(lr_plan)],
         "lr_device_error": [vp, ctypes.POINTER(i32)],
         "lr_cache_set_kernel_events": [vp, vp, vp],
+        "lr_attn_decode_noalloc": [ctypes.POINTER(lr_cache_desc), i32, vp, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -231,6 +232,24 @@ def lr_basis_sync(cache: Cache, R_k=None, R_v=None, B_k_new=None, B_v_new=None, 
                               _ptr(A_k_new, dt, (D, d.rank_k), "A_k_new", True),
                               _ptr(A_v_new, dt, (D, d.rank_v), "A_v_new", True),
                               _stream(stream)), "lr_basis_sync")
+
+
+LR_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
+
+
+def lr_attn_decode_noalloc(desc: lr_cache_desc, length: int, z_k: int, z_v: int, B_k: int, B_v: int,
+                           q, out, lse=None, stream=None) -> None:
+    """Decode without device allocation (working memory in the library's static device
+    array).  z_k, z_v, B_k, B_v: device addresses (ints) of caller-owned buffers in the
+    cache layout; q, out (and lse) are CUDA tensors."""
+    import torch
+    dt = _torch_dtype(desc.dtype)
+    shp = (desc.batch, desc.n_q_heads, desc.head_dim)
+    _check(_lib.lr_attn_decode_noalloc(ctypes.byref(desc), int(length), ctypes.c_void_p(z_k),
+                                       ctypes.c_void_p(z_v), ctypes.c_void_p(B_k), ctypes.c_void_p(B_v),
+                                       _ptr(q, dt, shp, "q"), _ptr(out, dt, shp, "out"),
+                                       _ptr(lse, torch.float32, (desc.batch, desc.n_q_heads), "lse", True),
+                                       _stream(stream)), "lr_attn_decode_noalloc")
 
 
 def lr_cache_get_len(cache: Cache):
