@@ -1,10 +1,10 @@
 #!/usr/bin/env python
 """Decode-step benchmark of the low-rank KV-cache library on B200.
 
-One step = the whole hot path for one batch: lr_kv_append of one new token per
-sequence (project, round/quantise, store) followed by lr_attn_decode over the
-full context (query projection, split-sequence latent attention, split merge
-and output projection).  The context is held fixed by truncating the appended
+One step = the whole hot path for one batch: lr_decode_step, i.e. lr_kv_append of
+one new token per sequence (project, round/quantise, store) followed by
+lr_attn_decode over the full context (query projection, split-sequence latent
+attention, split merge and output projection).  The context is held fixed by truncating the appended
 token after each step (host bookkeeping only).
 
 Default workload: one Qwen2.5-VL-7B-shaped layer, batch 16, 28 query heads over
@@ -190,8 +190,7 @@ def run_ours(args):
     plan = lr.lr_cache_plan(cache)
 
     def step(kk, vv, qq, oo, ll):
-        lr.lr_kv_append(cache, kk, vv)
-        lr.lr_attn_decode(cache, qq, oo, ll)
+        lr.lr_decode_step(cache, kk, vv, qq, oo, ll)   # lr_kv_append + lr_attn_decode, fused launches
         lr.lr_cache_truncate(cache, T - 1)
 
     def barrier():
@@ -305,7 +304,7 @@ def run_ours(args):
         "data": "synthetic (seeded; one seed per rank)",
         "config": {"workload": W["desc"], "batch": Bsz, "context": T, "rank": r,
                    "quant_bits": qb, "latent_bytes_per_step": bytes_per_step,
-                   "step": "lr_kv_append + lr_attn_decode", "l2": "flushed (256 MiB write) before every timed step, outside the events",
+                   "step": "lr_decode_step (= lr_kv_append + lr_attn_decode)", "l2": "flushed (256 MiB write) before every timed step, outside the events",
                    "parallelism": f"dp{world} (independent sequences per GPU)",
                    "decode_path": "tcgen05" if plan.path == lr.LR_PATH_TC else "simt",
                    "splits": plan.n_splits, "cuda_graph": bool(args.graph),

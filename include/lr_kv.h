@@ -151,6 +151,12 @@ lr_status lr_kv_append_latent(lr_cache* cache, const float* z_k, const float* z_
  *   LR_ERR_INVALID_ARG. */
 lr_status lr_attn_decode(lr_cache* cache, const void* q, void* out, float* lse, void* stream);
 
+/* lr_decode_step — one whole decode step: lr_kv_append(k, v) then lr_attn_decode(q,
+ *   out, lse), with identical arguments, results and errors, but with the projection
+ *   of the new token and the projection of the query run in one launch. */
+lr_status lr_decode_step(lr_cache* cache, const void* k, const void* v, const void* q, void* out,
+                         float* lse, void* stream);
+
 /* ---- basis sync (iS-KV abstract: historical coordinates synchronised with the
  *      updated basis) ---------------------------------------------------------
  * lr_basis_sync — Z_hist <- Z_hist R for the history latents of every sequence,
@@ -215,6 +221,15 @@ lr_status lr_device_error(lr_cache* cache, int32_t* code);
  * lr_attn_decode on this cache, on the call's stream, so that the kernel alone can be
  * timed; both NULL to stop.  The events must stay valid while set. */
 lr_status lr_cache_set_kernel_events(lr_cache* cache, void* ev_start, void* ev_stop);
+/* Timeline trace of the tensor-core decode kernel: when buf (device, capacity_words
+ * 64-bit words >= LR_TRACE_SLOTS * batch * max splits) is set, every CTA of each
+ * following decode writes %globaltimer stamps (ns) to
+ * buf[((b * n_splits) + split) * LR_TRACE_SLOTS + slot]: 0 start, 1 set-up done,
+ * 2 query latents in shared memory, 3+4i key tile i consumed, 4+4i its scores read,
+ * 5+4i its probabilities written, 6+4i its value mix issued (tiles i < 16), 71 end.
+ * NULL stops tracing.  LR_ERR_CAPACITY if buf is too small. */
+#define LR_TRACE_SLOTS 72
+lr_status lr_cache_set_trace(lr_cache* cache, uint64_t* buf, int64_t capacity_words);
 /* sizeof(lr_cache_desc), sizeof(lr_cache_view), sizeof(lr_plan) as compiled (binding checks). */
 void lr_abi_struct_sizes(int32_t* desc_size, int32_t* view_size, int32_t* plan_size);
 /* Human-readable name of a status. */

@@ -6,10 +6,10 @@ come from PyTorch); they are checked for device, dtype, shape and contiguity
 and passed by pointer.  There is no fallback: if the library is missing,
 importing this package raises.
 
-Functions keep the C names: lr_cache_create, lr_cache_destroy, lr_kv_append,
+Functions keep the C names: lr_cache_create, lr_cache_destroy, lr_kv_append, lr_decode_step,
 lr_kv_append_latent, lr_attn_decode, lr_basis_sync, lr_cache_get_len,
 lr_cache_truncate, lr_cache_view_get, lr_cache_set_path, lr_cache_plan,
-lr_plan_decode, lr_cache_set_kernel_events, lr_device_error, lr_abi_struct_sizes,
+lr_plan_decode, lr_cache_set_kernel_events, lr_cache_set_trace, lr_device_error, lr_abi_struct_sizes,
 lr_status_string, lr_launch_count, lr_attn_decode_noalloc.
 """
 from __future__ import annotations
@@ -72,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "lr_kv_append": [vp, vp, vp, vp],
         "lr_kv_append_latent": [vp, vp, vp, i32, vp],
         "lr_attn_decode": [vp, vp, vp, vp, vp],
+        "lr_decode_step": [vp, vp, vp, vp, vp, vp, vp],
         "lr_basis_sync": [vp, vp, vp, vp, vp, vp, vp, vp],
         "lr_cache_get_len": [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)],
         "lr_cache_truncate": [vp, i32],
@@ -81,6 +82,7 @@ def _load() -> ctypes.CDLL:
         "lr_plan_decode": [ctypes.POINTER(lr_cache_desc), i32, i32, i32, i32, ctypes.POINTER(lr_plan)],
         "lr_device_error": [vp, ctypes.POINTER(i32)],
         "lr_cache_set_kernel_events": [vp, vp, vp],
+        "lr_cache_set_trace": [vp, vp, ctypes.c_int64],
         "lr_attn_decode_noalloc": [ctypes.POINTER(lr_cache_desc), i32, vp, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
@@ -219,6 +221,17 @@ def lr_attn_decode(cache: Cache, q, out, lse=None, stream=None) -> None:
                                _stream(stream)), "lr_attn_decode")
 
 
+def lr_decode_step(cache: Cache, k, v, q, out, lse=None, stream=None) -> None:
+    import torch
+    d, dt = cache.desc, _torch_dtype(cache.desc.dtype)
+    shp = (d.batch, d.n_q_heads, d.head_dim)
+    _check(_lib.lr_decode_step(cache.handle, _ptr(k, dt, (d.batch, cache.D), "k"),
+                               _ptr(v, dt, (d.batch, cache.D), "v"), _ptr(q, dt, shp, "q"),
+                               _ptr(out, dt, shp, "out"),
+                               _ptr(lse, torch.float32, (d.batch, d.n_q_heads), "lse", True),
+                               _stream(stream)), "lr_decode_step")
+
+
 def lr_basis_sync(cache: Cache, R_k=None, R_v=None, B_k_new=None, B_v_new=None, A_k_new=None,
                   A_v_new=None, stream=None) -> None:
     import torch
@@ -292,6 +305,18 @@ def lr_cache_set_kernel_events(cache: Cache, ev_start=None, ev_stop=None) -> Non
     a = ctypes.c_void_p(ev_start.cuda_event) if ev_start is not None else None
     b = ctypes.c_void_p(ev_stop.cuda_event) if ev_stop is not None else None
     _check(_lib.lr_cache_set_kernel_events(cache.handle, a, b), "lr_cache_set_kernel_events")
+
+
+LR_TRACE_SLOTS = 72
+
+
+def lr_cache_set_trace(cache: Cache, buf=None) -> None:
+    """buf: int64 CUDA tensor with >= LR_TRACE_SLOTS * batch * max-splits elements, or None."""
+    if buf is None:
+        _check(_lib.lr_cache_set_trace(cache.handle, None, 0), "lr_cache_set_trace")
+        return
+    _check(_lib.lr_cache_set_trace(cache.handle, _ptr(buf, None, None, "trace"), buf.numel()),
+           "lr_cache_set_trace")
 
 
 def lr_abi_struct_sizes():

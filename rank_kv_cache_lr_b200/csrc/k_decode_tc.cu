@@ -42,6 +42,10 @@ constexpr int kMaxSlots = 12;
 constexpr float kLazy = 8.0f;              // log2 of the allowed growth before a rescale
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kSmemLimit = 232448;         // 227 KB opt-in per block
+constexpr int kTraceSlots = 72;            // 0 start, 1 setup done, 2 query latents in,
+                                           // 3+4i: key tile i in, 4+4i: scores of tile i in,
+                                           // 5+4i: probabilities of tile i written,
+                                           // 6+4i: value mix of tile i issued (i < 16), 71 end
 
 struct TcParams {
   int r_k, r_v, ck, cv, kb_k, tmem_cols;
@@ -50,6 +54,7 @@ struct TcParams {
   float* part_o;
   float* part_ml;
   int* err;
+  unsigned long long* trace;   // optional per-CTA timeline (kTraceSlots stamps per CTA), or null
 };
 
 struct Aux {
@@ -85,6 +90,10 @@ __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux,
       }
     }
   }
+}
+
+__device__ __forceinline__ void trace_stamp(const TcParams& p, int slot) {
+  if (p.trace) p.trace[((size_t)blockIdx.y * gridDim.x + blockIdx.x) * kTraceSlots + slot] = ptx::globaltimer();
 }
 
 // Wait that ignores the abort flag (used to drain in-flight work after an abort).
@@ -130,6 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int per_tile = p.ck + p.cv;
 
   if (threadIdx.x == 0) {
+    trace_stamp(p, 0);
     for (int s = 0; s < p.nslot; ++s) {
       ptx::mbar_init(&aux->slot_full[s], 1);
       ptx::mbar_init(&aux->slot_empty[s], 1);
@@ -162,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = aux->tmem_base;
   if (!(warp == 0 && lane == 0)) pdl_wait();   // the producer waits after its first loads
   pdl_trigger();
+  if (threadIdx.x == 32) trace_stamp(p, 1);
 
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
@@ -221,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_addr = ptx::smem_u32(q_s), ring_addr = ptx::smem_u32(ring), p_addr = ptx::smem_u32(p_s);
       bool ok = wait_b(&aux->q_full, 0, aux, p.err);
       ptx::tc_fence_after();
+      trace_stamp(p, 2);
       auto gemm1 = [&](int i) -> bool {
         const int buf = i & 1;
         if (i >= 2 && !wait_b(&aux->s_empty[buf], ((i - 2) >> 1) & 1, aux, p.err)) return false;
@@ -247,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::mma_commit(&aux->slot_empty[slot]);
         }
         ptx::mma_commit(&aux->s_full[buf]);
+        if (i < 16) trace_stamp(p, 3 + 4 * i);
         return true;
       };
       auto gemm2 = [&](int i) -> bool {
@@ -269,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::mma_commit(&aux->p_empty[buf]);
         ptx::mma_commit(&aux->o_done);
+        if (i < 16) trace_stamp(p, 6 + 4 * i);
         return true;
       };
       if (ok) {
@@ -307,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full[buf], (i >> 1) & 1, aux, p.err));
       if (!ok) break;
       ptx::tc_fence_after();
+      if (i < 16 && threadIdx.x == 64) trace_stamp(p, 4 + 4 * i);
       uint32_t hi[32], lo[32];
       ptx::tmem_ld32(tmem + lane_off + buf * 64, hi);
       ptx::tmem_ld32(tmem + lane_off + buf * 64 + 32, lo);
@@ -384,6 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&aux->p_full[buf]);
+      if (i < 16 && threadIdx.x == 64) trace_stamp(p, 5 + 4 * i);
     }
     if (ok) ok = ptx::named_bar_and(1, 128, wait_b(&aux->o_final, 0, aux, p.err));
     if (ok) {
@@ -408,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.part_ml[(base_out + lane) * 2] = aux->m_s[lane];
         p.part_ml[(base_out + lane) * 2 + 1] = lt;
       }
+      if (threadIdx.x == 64) trace_stamp(p, kTraceSlots - 1);
     }
   }
   ptx::tc_fence_before();
@@ -526,6 +543,7 @@ cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, 
   p.part_o = c->part_o;
   p.part_ml = c->part_ml;
   p.err = c->dev_err;
+  p.trace = c->trace;
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_decode_tc, optin_done);
   if (e != cudaSuccess) return e;

@@ -132,28 +132,33 @@ __device__ __forceinline__ float smem_elem(const uint8_t* p, int dtype) {
 // hi = bf16(q~) and lo = bf16(q~ - hi), so that hi + lo carries q~ to ~16 significant bits.
 constexpr int kRowsQ = 32;
 
-__global__ void __launch_bounds__(256) k_qproj(const void* q, const void* Bk, float* qt, float* qd,
-                                               __nv_bfloat16* qt16, int Hq, int Hkv, int d, int D, int rk,
-                                               int dtype, float scale_log2, int want_latent) {
-  extern __shared__ __align__(16) uint8_t qsm[];
-  pdl_wait();
-  pdl_trigger();
-  const int G = Hq / Hkv;
-  const int r0 = blockIdx.x * kRowsQ, h = blockIdx.y, b = blockIdx.z;
+struct QprojArgs {
+  const void* q; const void* Bk; float* qt; float* qd; __nv_bfloat16* qt16;
+  int Hq, Hkv, d, D, rk, dtype;
+  float scale_log2;
+  int want_latent;
+};
+
+__device__ __forceinline__ void qproj_body(const QprojArgs& a, int rchunk, int h, int b, uint8_t* qsm) {
+  const int Hq = a.Hq, d = a.d, D = a.D, rk = a.rk, dtype = a.dtype;
+  const float scale_log2 = a.scale_log2;
+  const int G = Hq / a.Hkv;
+  const int r0 = rchunk * kRowsQ;
   const int j0 = h * G;
   const int es = dtype == LR_BF16 ? 2 : 4;
   const int pitch = d * es + 16;
   float* qs = reinterpret_cast<float*>(qsm);                                   // [G][d]
   uint8_t* bs = qsm + (((size_t)G * d * sizeof(float) + 15) & ~size_t(15));   // [32][pitch]
   const int nr = min(kRowsQ, rk - r0);
-  if (want_latent && nr > 0) stage_rows(bs, pitch, Bk, D, es, r0, nr, (long long)h * d, d);
+  if (a.want_latent && nr > 0) stage_rows(bs, pitch, a.Bk, D, es, r0, nr, (long long)h * d, d);
+#pragma unroll 4
   for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) {
     const long long off = ((long long)b * Hq + j0) * d + idx;
-    const float v = elem_f(q, off, dtype);
+    const float v = elem_f(a.q, off, dtype);
     qs[idx] = v;
-    if (qd && blockIdx.x == 0) qd[off] = v * scale_log2;
+    if (a.qd && rchunk == 0) a.qd[off] = v * scale_log2;
   }
-  if (!want_latent) return;
+  if (!a.want_latent) return;
   cp_async_wait_all();
   __syncthreads();
   const int lane = threadIdx.x & 31, hs0 = threadIdx.x >> 5;
@@ -188,14 +193,26 @@ __global__ void __launch_bounds__(256) k_qproj(const void* q, const void* Bk, fl
     }
     const int j = j0 + hs;
     const float v = (a0 + a1) * scale_log2;
-    qt[((long long)b * Hq + j) * rk + i] = v;
-    if (qt16) {
+    a.qt[((long long)b * Hq + j) * rk + i] = v;
+    if (a.qt16) {
       const __nv_bfloat16 hi = __float2bfloat16_rn(v);
       const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-      qt16[((long long)b * 64 + j) * rk + i] = hi;
-      qt16[((long long)b * 64 + 32 + j) * rk + i] = lo;
+      a.qt16[((long long)b * 64 + j) * rk + i] = hi;
+      a.qt16[((long long)b * 64 + 32 + j) * rk + i] = lo;
     }
   }
+}
+
+__global__ void __launch_bounds__(256) k_qproj(QprojArgs a) {
+  extern __shared__ __align__(16) uint8_t qsm[];
+  pdl_wait();
+  pdl_trigger();
+  qproj_body(a, blockIdx.x, blockIdx.y, blockIdx.z, qsm);
+}
+
+size_t qproj_smem(const lr_cache_desc& d, size_t es) {
+  return (((size_t)(d.n_q_heads / d.n_kv_heads) * d.head_dim * sizeof(float) + 15) & ~size_t(15)) +
+         (size_t)kRowsQ * (d.head_dim * es + 16);
 }
 
 // ---------------------------------------------------------------------------
@@ -372,30 +389,50 @@ __global__ void __launch_bounds__(128) k_window(const void* win_k, const void* w
 // split merge (log-sum-exp) and output projection o = o~ B_v,h / l.
 // One CTA (512 threads) per (KV head h, sequence b).  The B_v,h slice is prefetched
 // into shared memory with asynchronous copies while the split weights and the
-// combined rank-space outputs o~ of the group's query heads are formed (every thread
-// issues all of its partial loads before using any); then thread = (output column,
-// query-head slot).
+// combined rank-space outputs o~ of the group's query heads are formed; o~ is kept
+// rank-major with the heads padded to a multiple of 4.  The projection is register
+// blocked: thread = (column pair, block of 4 heads, rank slice), and the rank slices
+// are summed through shared memory in a fixed order.
 // ---------------------------------------------------------------------------
 constexpr int kMergeThreads = 512;
 constexpr size_t kMergeStage = 96 * 1024;   // bytes of B_v,h rows staged in shared memory
-constexpr int kMergeSlots = 8;    // partial outputs per thread held in flight
 
+template <typename T>
+__device__ __forceinline__ float2 load_pair(const uint8_t* p);
+template <>
+__device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const uint8_t* p) {
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+template <>
+__device__ __forceinline__ float2 load_pair<float>(const uint8_t* p) {
+  return *reinterpret_cast<const float2*>(p);
+}
+
+template <typename T>
 __global__ void __launch_bounds__(kMergeThreads) k_merge(const float* part_o, const float* part_ml,
                                                          const float* win_o, const float* win_ml,
-                                                         const void* Bv, void* out, float* lse, int S,
-                                                         int Hq, int Hkv, int d, int D, int rv, int dtype) {
+                                                         const T* Bv, T* out, float* lse, int S, int Hq,
+                                                         int Hkv, int d, int D, int rv) {
   extern __shared__ __align__(16) float msm[];
   const int G = Hq / Hkv;
-  float* ot = msm;               // [G][rv]
-  float* w_s = ot + G * rv;      // [G][S]
-  float* hdr = w_s + G * S;      // [G][3]: m*, 1/l, window weight
-  uint8_t* bs = reinterpret_cast<uint8_t*>(msm) + ((((size_t)G * (rv + S + 3)) * sizeof(float) + 15) & ~size_t(15));
+  const int G4 = (G + 3) & ~3;
+  const int HB = G4 / 4;
+  float* ot = msm;                 // [rv][G4]  (rank-major)
+  float* w_s = ot + rv * G4;       // [G][S]
+  float* hdr = w_s + G * S;        // [G][3]: m*, 1/l, window weight
+  float* red = hdr + G * 3;        // [RS][G4][d] partial projections
   const int h = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, nt = blockDim.x;
   const int j0 = h * G;
   const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
-  const int es = dtype == LR_BF16 ? 2 : 4;
+  constexpr int es = sizeof(T);
   const int pitch = d * es;
+  const int npairs = d / 2;
+  const int combos = npairs * HB;
+  const int RS = max(1, nt / combos);
+  const size_t fl = (size_t)rv * G4 + (size_t)G * S + 3 * G + (size_t)RS * G4 * d;
+  uint8_t* bs = reinterpret_cast<uint8_t*>(msm) + ((fl * sizeof(float) + 15) & ~size_t(15));   // 16-B aligned
   const int rows_staged = min(rv, (int)(kMergeStage / pitch));
   stage_rows(bs, pitch, Bv, D, es, 0, rows_staged, (long long)h * d, d);   // bases: stable data
   pdl_wait();
@@ -430,52 +467,94 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(const float* part_o, co
       if (lse) lse[(long long)b * Hq + j] = (m + log2f(l)) * LR_LN2;
     }
   }
+  for (int idx = tid; idx < rv * (G4 - G); idx += nt) {       // zero the padding heads
+    const int i = idx / (G4 - G), jj = G + idx % (G4 - G);
+    ot[i * G4 + jj] = 0.f;
+  }
   __syncthreads();
+  // combine: thread = (rank i, head slot); the loads of 2 heads x 8 splits are issued
+  // together before any is used, so each thread waits for about one memory round trip
+  // per 16 partial values
   const size_t sstride = (size_t)Hq * rv;
-  const float* pbase = part_o + ((size_t)b * S * Hq + j0) * rv;
-  for (int base = 0; base < G * rv; base += nt * kMergeSlots) {
-    float acc[kMergeSlots];
+  const int jslots = max(1, nt / rv);
+  for (int t = tid; t < rv * jslots; t += nt) {
+    const int i = t % rv, js = t / rv;
+    for (int jj = js; jj < G; jj += 2 * jslots) {
+      const int jj2 = jj + jslots;
+      const bool two = jj2 < G;
+      const float* src = part_o + (((size_t)b * S) * Hq + j0 + jj) * rv + i;
+      const float* src2 = part_o + (((size_t)b * S) * Hq + j0 + (two ? jj2 : jj)) * rv + i;
+      float acc = 0.f, acc2 = 0.f;
+      for (int s0 = 0; s0 < S; s0 += 8) {
+        float v[8], v2[8];
 #pragma unroll
-    for (int k = 0; k < kMergeSlots; ++k) acc[k] = 0.f;
-    for (int s = 0; s < S; ++s) {
+        for (int k = 0; k < 8; ++k) {
+          const bool in = s0 + k < S;
+          v[k] = in ? __ldg(src + (size_t)(s0 + k) * sstride) : 0.f;
+          v2[k] = (in && two) ? __ldg(src2 + (size_t)(s0 + k) * sstride) : 0.f;
+        }
 #pragma unroll
-      for (int k = 0; k < kMergeSlots; ++k) {
-        const int idx = base + k * nt + tid;
-        if (idx < G * rv) {
-          const int jj = idx / rv;
-          acc[k] = fmaf(w_s[jj * S + s], pbase[(size_t)s * sstride + idx], acc[k]);
+        for (int k = 0; k < 8; ++k) {
+          if (s0 + k < S) {
+            acc = fmaf(w_s[jj * S + s0 + k], v[k], acc);
+            if (two) acc2 = fmaf(w_s[jj2 * S + s0 + k], v2[k], acc2);
+          }
         }
       }
-    }
-#pragma unroll
-    for (int k = 0; k < kMergeSlots; ++k) {
-      const int idx = base + k * nt + tid;
-      if (idx < G * rv) ot[idx] = acc[k];
+      ot[i * G4 + jj] = acc;
+      if (two) ot[i * G4 + jj2] = acc2;
     }
   }
   cp_async_wait_all();
   __syncthreads();
-  // projection: thread = (column c, head slot); ranks beyond the staged rows are read
-  // from global memory (only when the slice does not fit the staging buffer)
-  const int slots = nt / d > 0 ? nt / d : 1;
-  const int c = tid % d, slot = tid / d;
-  if (slot >= slots || c >= d) return;
-  for (int jj = slot; jj < G; jj += slots) {
-    const float* orow = ot + jj * rv;
-    float a0 = 0.f, a1 = 0.f;
-    int i = 0;
-    for (; i + 1 < rows_staged; i += 2) {
-      a0 = fmaf(orow[i], smem_elem(bs + i * pitch + c * es, dtype), a0);
-      a1 = fmaf(orow[i + 1], smem_elem(bs + (i + 1) * pitch + c * es, dtype), a1);
+  // projection
+  for (int t = tid; t < combos * RS; t += nt) {
+    const int cp = t % npairs;
+    const int hb = (t / npairs) % HB;
+    const int rs = t / combos;
+    const int per = (rv + RS - 1) / RS;
+    const int i0 = rs * per, i1 = min(rv, i0 + per);
+    float acc[4][2];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = 0.f;
+    for (int i = i0; i < i1; ++i) {
+      const float2 bv = i < rows_staged
+                            ? load_pair<T>(bs + i * pitch + cp * 2 * es)
+                            : load_pair<T>(reinterpret_cast<const uint8_t*>(Bv + (size_t)i * D + (size_t)h * d + 2 * cp));
+      const float4 o4 = *reinterpret_cast<const float4*>(ot + i * G4 + hb * 4);
+      acc[0][0] = fmaf(o4.x, bv.x, acc[0][0]); acc[0][1] = fmaf(o4.x, bv.y, acc[0][1]);
+      acc[1][0] = fmaf(o4.y, bv.x, acc[1][0]); acc[1][1] = fmaf(o4.y, bv.y, acc[1][1]);
+      acc[2][0] = fmaf(o4.z, bv.x, acc[2][0]); acc[2][1] = fmaf(o4.z, bv.y, acc[2][1]);
+      acc[3][0] = fmaf(o4.w, bv.x, acc[3][0]); acc[3][1] = fmaf(o4.w, bv.y, acc[3][1]);
     }
-    for (; i < rv; ++i)
-      a0 = fmaf(orow[i], i < rows_staged ? smem_elem(bs + i * pitch + c * es, dtype)
-                                         : elem_f(Bv, (long long)i * D + (long long)h * d + c, dtype), a0);
-    const long long ooff = ((long long)b * Hq + j0 + jj) * d + c;
-    float o = a0 + a1;
-    if (win_o) o = fmaf(hdr[jj * 3 + 2], win_o[ooff], o);
-    store_elem(out, ooff, o * hdr[jj * 3 + 1], dtype);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float* rr = red + ((size_t)rs * G4 + hb * 4 + u) * d + 2 * cp;
+      rr[0] = acc[u][0];
+      rr[1] = acc[u][1];
+    }
   }
+  __syncthreads();
+  for (int idx = tid; idx < G * d; idx += nt) {
+    const int jj = idx / d, c = idx % d;
+    float o = 0.f;
+    for (int r = 0; r < RS; ++r) o += red[((size_t)r * G4 + jj) * d + c];
+    const long long ooff = ((long long)b * Hq + j0 + jj) * d + c;
+    if (win_o) o = fmaf(hdr[jj * 3 + 2], win_o[ooff], o);
+    o *= hdr[jj * 3 + 1];
+    if constexpr (sizeof(T) == 2) out[ooff] = __float2bfloat16_rn(o);
+    else out[ooff] = o;
+  }
+}
+
+size_t merge_smem(const lr_cache_desc& d, int S, size_t es) {
+  const int G = d.n_q_heads / d.n_kv_heads;
+  const int G4 = (G + 3) & ~3;
+  const int combos = (d.head_dim / 2) * (G4 / 4);
+  const int RS = std::max(1, kMergeThreads / combos);
+  const size_t stage = std::min(kMergeStage, (size_t)d.rank_v * d.head_dim * es);
+  const size_t fl = (size_t)d.rank_v * G4 + (size_t)G * S + 3 * G + (size_t)RS * G4 * d.head_dim;
+  return ((fl * sizeof(float) + 15) & ~size_t(15)) + stage;
 }
 
 // ---------------------------------------------------------------------------
@@ -498,12 +577,7 @@ struct AppendArgs {
 // ([D][32]) and the source row are staged in shared memory with asynchronous copies;
 // the 8 warps take fixed eighths of the D-long dot products and the partial sums are
 // added in a fixed order, so the result does not depend on the storage kind.
-__global__ void __launch_bounds__(256) k_append(AppendArgs a) {
-  extern __shared__ __align__(16) uint8_t asm_[];
-  __shared__ float red[8][32];
-  pdl_wait();
-  pdl_trigger();
-  const int x = blockIdx.x, b = blockIdx.y;
+__device__ __forceinline__ void append_body(const AppendArgs& a, int x, int b, uint8_t* asm_, float (*red)[32]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nproj = a.project ? (a.chunks_k + a.chunks_v) : 0;
   const int es = a.dtype == LR_BF16 ? 2 : 4;
@@ -554,6 +628,27 @@ __global__ void __launch_bounds__(256) k_append(AppendArgs a) {
     if (a.dtype == LR_BF16) reinterpret_cast<uint16_t*>(dst)[dof] = reinterpret_cast<const uint16_t*>(src)[so];
     else reinterpret_cast<uint32_t*>(dst)[dof] = reinterpret_cast<const uint32_t*>(src)[so];
   }
+}
+
+__global__ void __launch_bounds__(256) k_append(AppendArgs a) {
+  extern __shared__ __align__(16) uint8_t asm_[];
+  __shared__ float red[8][32];
+  pdl_wait();
+  pdl_trigger();
+  append_body(a, blockIdx.x, blockIdx.y, asm_, red);
+}
+
+// One decode step's independent first half in one grid: CTAs [0, x_app) of each row
+// are the append of the new token (projection / ring write), the others the query
+// projection (rank chunk, KV head).
+__global__ void __launch_bounds__(256) k_step_pre(AppendArgs aa, QprojArgs qa, int x_app, int nchunks_q) {
+  extern __shared__ __align__(16) uint8_t psm[];
+  __shared__ float red[8][32];
+  pdl_wait();
+  pdl_trigger();
+  const int x = blockIdx.x, b = blockIdx.y;
+  if (x < x_app) append_body(aa, x, b, psm, red);
+  else qproj_body(qa, (x - x_app) % nchunks_q, (x - x_app) / nchunks_q, b, psm);
 }
 
 // bulk latent fill: one warp per (token, 32-coordinate chunk)
@@ -626,18 +721,32 @@ LatentRef latent_ref(const lr_cache* c, bool k) {
 // launchers
 // ---------------------------------------------------------------------------
 
-static cudaError_t qproj(const lr_cache* c, const void* q, cudaStream_t s, bool tc) {
+static QprojArgs make_qproj_args(const lr_cache* c, const void* q, bool tc) {
   const lr_cache_desc& d = c->desc;
   const bool rope = d.rope_in_kernel != 0;
-  float* qd = (rope || c->win_slots) ? (rope ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k) : nullptr;
-  dim3 grid(rope ? 1 : (d.rank_k + kRowsQ - 1) / kRowsQ, d.n_kv_heads, d.batch);
-  const size_t smem = (((size_t)(d.n_q_heads / d.n_kv_heads) * d.head_dim * sizeof(float) + 15) & ~size_t(15)) +
-                      (size_t)kRowsQ * (d.head_dim * c->esize + 16);
+  QprojArgs a;
+  a.q = q;
+  a.Bk = c->B_k;
+  a.qt = c->qt;
+  a.qd = (rope || c->win_slots) ? (rope ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k) : nullptr;
+  a.qt16 = tc ? (__nv_bfloat16*)c->qt16 : nullptr;
+  a.Hq = d.n_q_heads; a.Hkv = d.n_kv_heads; a.d = d.head_dim; a.D = c->D; a.rk = d.rank_k; a.dtype = d.dtype;
+  a.scale_log2 = c->scale_log2;
+  a.want_latent = rope ? 0 : 1;
+  return a;
+}
+
+static int qproj_chunks(const lr_cache* c) {
+  return c->desc.rope_in_kernel ? 1 : (c->desc.rank_k + kRowsQ - 1) / kRowsQ;
+}
+
+static cudaError_t qproj(const lr_cache* c, const void* q, cudaStream_t s, bool tc) {
+  const lr_cache_desc& d = c->desc;
+  dim3 grid(qproj_chunks(c), d.n_kv_heads, d.batch);
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_qproj, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_qproj, grid, dim3(256), smem, s, q, c->B_k, c->qt, qd, tc ? (__nv_bfloat16*)c->qt16 : nullptr, d.n_q_heads,
-                               d.n_kv_heads, d.head_dim, c->D, d.rank_k, d.dtype, c->scale_log2, rope ? 0 : 1);
+  return launch_pdl(k_qproj, grid, dim3(256), qproj_smem(d, c->esize), s, make_qproj_args(c, q, tc));
 }
 
 cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s) { return qproj(c, q, s, false); }
@@ -682,6 +791,9 @@ cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
   const float* qd = d.rope_in_kernel ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k;
   const size_t smem = (size_t)(d.head_dim + c->win_len + 1) * sizeof(float);
   dim3 grid(d.n_q_heads, d.batch);
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_window, optin_done);
+  if (e != cudaSuccess) return e;
   return launch_pdl(k_window, grid, dim3(128), smem, s, c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads, d.n_kv_heads,
                                    d.head_dim, c->D, c->win_slots, c->hist_len, c->win_len, d.dtype);
 }
@@ -689,19 +801,28 @@ cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
 cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s) {
   const lr_cache_desc& d = c->desc;
   const bool win = c->win_slots > 0;
-  const int G = d.n_q_heads / d.n_kv_heads;
-  const size_t stage = std::min(kMergeStage, (size_t)d.rank_v * d.head_dim * c->esize);
-  const size_t smem = (((size_t)G * (d.rank_v + n_splits + 3) * sizeof(float) + 15) & ~size_t(15)) + stage;
-  static std::atomic<uint32_t> optin_done{0};
-  cudaError_t e = smem_optin(k_merge, optin_done);
-  if (e != cudaSuccess) return e;
+  const size_t smem = merge_smem(d, n_splits, c->esize);
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   dim3 grid(d.n_kv_heads, d.batch);
-  return launch_pdl(k_merge, grid, dim3(kMergeThreads), smem, s, c->part_o, c->part_ml, win ? c->win_o : nullptr, win ? c->win_ml : nullptr,
-                                  c->B_v, out, lse, n_splits, d.n_q_heads, d.n_kv_heads, d.head_dim, c->D,
-                                  d.rank_v, d.dtype);
+  const float* wo = win ? c->win_o : nullptr;
+  const float* wm = win ? c->win_ml : nullptr;
+  if (d.dtype == LR_BF16) {
+    static std::atomic<uint32_t> optin_done{0};
+    cudaError_t e = smem_optin(k_merge<__nv_bfloat16>, optin_done);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_merge<__nv_bfloat16>, grid, dim3(kMergeThreads), smem, s, c->part_o, c->part_ml, wo, wm,
+                      (const __nv_bfloat16*)c->B_v, (__nv_bfloat16*)out, lse, n_splits, d.n_q_heads, d.n_kv_heads,
+                      d.head_dim, c->D, d.rank_v);
+  }
+  static std::atomic<uint32_t> optin_done32{0};
+  cudaError_t e = smem_optin(k_merge<float>, optin_done32);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_merge<float>, grid, dim3(kMergeThreads), smem, s, c->part_o, c->part_ml, wo, wm,
+                    (const float*)c->B_v, (float*)out, lse, n_splits, d.n_q_heads, d.n_kv_heads, d.head_dim, c->D,
+                    d.rank_v);
 }
 
-cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s) {
+static AppendArgs make_append_args(const lr_cache* c, const void* k, const void* v) {
   const lr_cache_desc& d = c->desc;
   AppendArgs a;
   const bool win = c->win_slots > 0;
@@ -726,13 +847,37 @@ cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_
   a.win_k = c->win_k; a.win_v = c->win_v; a.slots = c->win_slots;
   a.new_slot = win ? (c->len % c->win_slots) : 0;
   a.B = d.batch; a.D = c->D; a.kind = c->latent_kind; a.dtype = d.dtype;
-  const int nproj = a.project ? a.chunks_k + a.chunks_v : 0;
-  dim3 grid(nproj + (win ? 2 : 0), d.batch);
-  const size_t smem = (size_t)c->D * 32 * c->esize + (size_t)c->D * c->esize;
+  return a;
+}
+
+static int append_ctas(const AppendArgs& a) {
+  return (a.project ? a.chunks_k + a.chunks_v : 0) + (a.new_k ? 2 : 0);
+}
+
+static size_t append_smem(const lr_cache* c) {
+  return (size_t)c->D * 32 * c->esize + (size_t)c->D * c->esize;
+}
+
+cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s) {
+  const AppendArgs a = make_append_args(c, k, v);
+  dim3 grid(append_ctas(a), c->desc.batch);
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_append, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_append, grid, dim3(256), smem, s, a);
+  return launch_pdl(k_append, grid, dim3(256), append_smem(c), s, a);
+}
+
+cudaError_t launch_step_pre(lr_cache* c, const void* k, const void* v, const void* q, bool tc, cudaStream_t s) {
+  const AppendArgs aa = make_append_args(c, k, v);
+  const QprojArgs qa = make_qproj_args(c, q, tc);
+  const int x_app = append_ctas(aa);
+  const int nq = qproj_chunks(c);
+  dim3 grid(x_app + nq * c->desc.n_kv_heads, c->desc.batch);
+  const size_t smem = std::max(append_smem(c), qproj_smem(c->desc, c->esize));
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_step_pre, optin_done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_step_pre, grid, dim3(256), smem, s, aa, qa, x_app, nq);
 }
 
 cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, int n, cudaStream_t s) {
@@ -740,6 +885,9 @@ cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, 
   const int chunks_k = (d.rank_k + 31) / 32, chunks_v = (d.rank_v + 31) / 32;
   const long long pairs = (long long)n * (chunks_k + chunks_v);
   dim3 grid((unsigned)((pairs + 7) / 8), d.batch);
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_append_latent, optin_done);
+  if (e != cudaSuccess) return e;
   return launch_pdl(k_append_latent, grid, dim3(256), 0, s, zk, zv, n, d.batch, d.rank_k, d.rank_v, chunks_k, chunks_v, c->z_k,
                                        c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->G_k,
                                        c->G_v, d.capacity, c->hist_len, c->latent_kind, d.dtype);

@@ -271,19 +271,15 @@ lr_status lr_cache_plan(const lr_cache* c, lr_plan* out) {
   return plan(&c->desc, c->hist_len, c->num_sms, c->path_force, c->splits_force, out);
 }
 
-lr_status lr_attn_decode(lr_cache* c, const void* q, void* out, float* lse, void* stream) {
-  if (!c || !q || !out) return LR_ERR_INVALID_ARG;
-  if (c->len == 0) return LR_ERR_INVALID_ARG;
-  lr_plan p;
-  lr_status st = plan(&c->desc, c->hist_len, c->num_sms, c->path_force, c->splits_force, &p);
-  if (st != LR_OK) return st;
-  if (p.n_splits > c->S_max) return LR_ERR_UNSUPPORTED;
-  cudaStream_t s = (cudaStream_t)stream;
-  c->last_stream = s;
-  cudaError_t e;
-  if (p.path != LR_PATH_TC && c->hist_len > 0 && decode_simt_smem(c) > 227 * 1024) return LR_ERR_UNSUPPORTED;
-  e = p.path == LR_PATH_TC ? launch_qproj_tc(c, q, s) : launch_qproj(c, q, s);
-  if (e == cudaSuccess && c->hist_len > 0) {
+}  // extern "C"
+
+namespace {
+
+// The decode after its query projection: split-sequence attention (timed by the
+// caller's events when set), exact window, split merge and output projection.
+cudaError_t decode_rest(lr_cache* c, const lr_plan& p, void* out, float* lse, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  if (c->hist_len > 0) {
     if (c->ev_start) e = record_event(c->ev_start, s);
     if (e == cudaSuccess)
       e = p.path == LR_PATH_TC ? launch_decode_tc(c, p.n_splits, p.split_tokens, s)
@@ -293,6 +289,57 @@ lr_status lr_attn_decode(lr_cache* c, const void* q, void* out, float* lse, void
   const int S = c->hist_len > 0 ? p.n_splits : 0;
   if (e == cudaSuccess && c->win_slots) e = launch_window(c, s);
   if (e == cudaSuccess) e = launch_merge(c, S, out, lse, s);
+  return e;
+}
+
+lr_status decode_plan(const lr_cache* c, int hist_len, lr_plan* p) {
+  lr_status st = plan(&c->desc, hist_len, c->num_sms, c->path_force, c->splits_force, p);
+  if (st != LR_OK) return st;
+  if (p->n_splits > c->S_max) return LR_ERR_UNSUPPORTED;
+  if (p->path != LR_PATH_TC && hist_len > 0 && decode_simt_smem(c) > 227 * 1024) return LR_ERR_UNSUPPORTED;
+  return LR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lr_status lr_attn_decode(lr_cache* c, const void* q, void* out, float* lse, void* stream) {
+  if (!c || !q || !out) return LR_ERR_INVALID_ARG;
+  if (c->len == 0) return LR_ERR_INVALID_ARG;
+  lr_plan p;
+  lr_status st = decode_plan(c, c->hist_len, &p);
+  if (st != LR_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  cudaError_t e = p.path == LR_PATH_TC ? launch_qproj_tc(c, q, s) : launch_qproj(c, q, s);
+  if (e == cudaSuccess) e = decode_rest(c, p, out, lse, s);
+  return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
+}
+
+lr_status lr_decode_step(lr_cache* c, const void* k, const void* v, const void* q, void* out, float* lse,
+                         void* stream) {
+  if (!c || !k || !v || !q || !out || !c->has_A) return LR_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15) return LR_ERR_INVALID_ARG;
+  if (c->len >= c->desc.capacity) return LR_ERR_CAPACITY;
+  int32_t hist1 = c->hist_len, win1 = c->win_len;
+  if (c->win_slots) {
+    if (c->win_len == c->desc.window) ++hist1;
+    else ++win1;
+  } else {
+    ++hist1;
+  }
+  lr_plan p;
+  lr_status st = decode_plan(c, hist1, &p);
+  if (st != LR_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  cudaError_t e = launch_step_pre(c, k, v, q, p.path == LR_PATH_TC, s);   // uses the pre-append counters
+  if (e != cudaSuccess) return LR_ERR_CUDA;
+  c->hist_len = hist1;
+  c->win_len = win1;
+  ++c->len;
+  e = decode_rest(c, p, out, lse, s);
   return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
 }
 
@@ -357,6 +404,13 @@ lr_status lr_cache_set_kernel_events(lr_cache* c, void* ev_start, void* ev_stop)
   if (!c || ((ev_start == nullptr) != (ev_stop == nullptr))) return LR_ERR_INVALID_ARG;
   c->ev_start = (cudaEvent_t)ev_start;
   c->ev_stop = (cudaEvent_t)ev_stop;
+  return LR_OK;
+}
+
+lr_status lr_cache_set_trace(lr_cache* c, uint64_t* buf, int64_t capacity_words) {
+  if (!c) return LR_ERR_INVALID_ARG;
+  if (buf && capacity_words < (int64_t)LR_TRACE_SLOTS * c->desc.batch * c->S_max) return LR_ERR_CAPACITY;
+  c->trace = reinterpret_cast<unsigned long long*>(buf);
   return LR_OK;
 }
 

@@ -52,6 +52,7 @@ struct lr_cache {
   cudaStream_t last_stream = nullptr;
   void* tc_state = nullptr;    // tensor-core path state (tensor maps), owned
   cudaEvent_t ev_start = nullptr, ev_stop = nullptr;   // caller-owned kernel timing events
+  unsigned long long* trace = nullptr;                 // caller-owned decode timeline buffer
 };
 
 // ---- argument blocks --------------------------------------------------------
@@ -83,6 +84,8 @@ cudaError_t launch_decode_simt(const lr_cache* c, int n_splits, int split_tokens
 cudaError_t launch_window(const lr_cache* c, cudaStream_t s);
 cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s);
 cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s);
+// append (with the cache's current counters) and query projection in one grid
+cudaError_t launch_step_pre(lr_cache* c, const void* k, const void* v, const void* q, bool tc, cudaStream_t s);
 cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, int n,
                                  cudaStream_t s);
 cudaError_t launch_sync_simt(lr_cache* c, const float* R, int which, cudaStream_t s);
@@ -137,6 +140,10 @@ inline cudaError_t smem_optin(Kernel k, std::atomic<uint32_t>& done) {
   e = cudaFuncGetAttributes(&fa, k);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448 - (int)fa.sharedSizeBytes);
+  // one carveout for every kernel of the library, so consecutive kernels do not
+  // reconfigure the L1 / shared-memory split of the SMs between them
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
   else (void)cudaGetLastError();   // do not leave a stale error for a later launch check
   return e;

@@ -378,3 +378,25 @@ def test_truncate_replays_same_step(lib):
         lib.lr_cache_truncate(c, p.length)
     again, _ = H.gpu_decode(lib, p, c)
     assert np.array_equal(first, again)
+
+
+@pytest.mark.parametrize("kind", ["tiny", "qwen4k", "qwen16k", "hybrid"])
+def test_decode_step_equals_append_then_decode(lib, kind):
+    """lr_decode_step is lr_kv_append followed by lr_attn_decode, bit for bit."""
+    import torch
+    p = synth.small_variant(kind)
+    c1, c2 = H.fill_cache(lib, p), H.fill_cache(lib, p)
+    D = p.kv_dim
+    q = _sharp(p)
+    for step in range(3):
+        k, v = synth.hybrid_token("step", 0, step, p.batch, D, H.stored_value(p, p.B_k), H.stored_value(p, p.B_v))
+        kd, vd, qd = H.to_dev(p, p.store(k)), H.to_dev(p, p.store(v)), H.to_dev(p, q)
+        o1, o2 = torch.empty_like(qd), torch.empty_like(qd)
+        l1 = torch.empty((p.batch, p.n_q_heads), dtype=torch.float32, device="cuda")
+        l2 = torch.empty_like(l1)
+        lib.lr_kv_append(c1, kd, vd)
+        lib.lr_attn_decode(c1, qd, o1, l1)
+        lib.lr_decode_step(c2, kd, vd, qd, o2, l2)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+        assert lib.lr_cache_get_len(c1) == lib.lr_cache_get_len(c2)
