@@ -35,21 +35,25 @@ constexpr int kSubBytes = 128 * 128;       // 128 tokens x 64 ranks x 2 B
 constexpr int kSlotBytes = 2 * kSubBytes;  // 128 tokens x 128 ranks
 constexpr int kQRows = 64;                 // 32 head rows (hi) + 32 head rows (lo)
 constexpr int kQSubBytes = kQRows * 128;   // 64 rows x 64 ranks x 2 B
-constexpr int kPBytes = 128 * 64 * 2;      // 128 tokens x (32 hi + 32 lo heads) x 2 B
-constexpr int kOColsPerChunk = 64;         // hi | lo
-constexpr int kOCol = 128;                 // first TMEM column of O~
-constexpr int kMaxSlots = 12;
+constexpr int kQLoOffset = 32 * 128;       // lo rows start 32 rows into each sub-block
+constexpr int kPHalfBytes = 128 * 32 * 2;  // 128 tokens x 32 heads x 2 B (one of hi, lo)
+constexpr int kPBytes = 2 * kPHalfBytes;
+constexpr int kAuxBytes = 1024;            // barriers and reduction scratch, first in smem
+constexpr int kSCol = 0;                   // TMEM: S in columns [0, 32)
+constexpr int kOCol = 32;                  // TMEM: O~ chunk c in columns [32 + 32c, 64 + 32c)
+constexpr int kMaxSlots = 8;
 constexpr float kLazy = 8.0f;              // log2 of the allowed growth before a rescale
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kSmemLimit = 232448;         // 227 KB opt-in per block
+constexpr int kSmemPair = 115712;          // per block when two blocks share an SM (228 KB - 2 x 1 KB)
 constexpr int kTraceSlots = 72;            // 0 start, 1 setup done, 2 query latents in,
-                                           // 3+4i: key tile i in, 4+4i: scores of tile i in,
+                                           // 3+4i: key tile i consumed, 4+4i: scores of tile i read,
                                            // 5+4i: probabilities of tile i written,
                                            // 6+4i: value mix of tile i issued (i < 16), 71 end
 
 struct TcParams {
   int r_k, r_v, ck, cv, kb_k, tmem_cols;
-  int Hq, hist_len, split_tokens, n_splits, nslot, lookahead;
+  int Hq, hist_len, split_tokens, n_splits, nslot;
   uint32_t q_bytes;
   float* part_o;
   float* part_ml;
@@ -60,19 +64,19 @@ struct TcParams {
 struct Aux {
   uint64_t slot_full[kMaxSlots];
   uint64_t slot_empty[kMaxSlots];
-  uint64_t q_full, o_done, o_final;
-  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
+  uint64_t q_full, s_full, s_empty, p_full, p_empty, o_final;
   uint32_t tmem_base;
   int abort_flag;
   float red[4][32];
   float m_s[32];
   float alpha_s[32];
 };
+static_assert(sizeof(Aux) <= kAuxBytes, "aux block");
 
 struct TcState {
   CUtensorMap q, zk, zv;
   int nslot;
-  int lookahead;
+  int ctas_per_sm;
   size_t smem;
 };
 
@@ -121,15 +125,21 @@ __device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane)
   return v[0];
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Shared memory: [aux 1 KB][q~ hi|lo per 64-rank sub-block][ring of nslot x 32 KB][P hi | P lo].
+// The dynamic shared-memory window starts 1024-byte aligned (checked); the swizzled
+// operands sit at 1024-byte multiples.
+__global__ void __launch_bounds__(kThreads, 2)
     k_decode_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_zk,
                 const __grid_constant__ CUtensorMap tm_zv, const TcParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_s = base;
-  uint8_t* ring = base + p.q_bytes;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (ptx::smem_u32(smem_raw) & 1023) {      // layout precondition; uniform for the whole CTA
+    if (threadIdx.x == 0) atomicExch(p.err, (int)LR_ERR_UNSUPPORTED);
+    return;
+  }
+  Aux* aux = reinterpret_cast<Aux*>(smem_raw);
+  uint8_t* q_s = smem_raw + kAuxBytes;
+  uint8_t* ring = q_s + p.q_bytes;
   uint8_t* p_s = ring + p.nslot * kSlotBytes;
-  Aux* aux = reinterpret_cast<Aux*>(p_s + 2 * kPBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, b = blockIdx.y;
@@ -145,14 +155,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&aux->slot_empty[s], 1);
     }
     ptx::mbar_init(&aux->q_full, 1);
-    ptx::mbar_init(&aux->o_done, 1);
+    ptx::mbar_init(&aux->s_full, 1);
+    ptx::mbar_init(&aux->s_empty, 128);
+    ptx::mbar_init(&aux->p_full, 128);
+    ptx::mbar_init(&aux->p_empty, 1);
     ptx::mbar_init(&aux->o_final, 1);
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(&aux->s_full[i], 1);
-      ptx::mbar_init(&aux->s_empty[i], 128);
-      ptx::mbar_init(&aux->p_full[i], 128);
-      ptx::mbar_init(&aux->p_empty[i], 1);
-    }
     aux->abort_flag = 0;
     for (int j = 0; j < 32; ++j) aux->m_s[j] = -INFINITY;
     ptx::fence_mbar_init();
@@ -188,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = 0; u < per_tile; ++u) {
           const int pos = i * per_tile + u;
           const int slot = pos % p.nslot, round = pos / p.nslot;
-          if (pos >= p.ck && !q_issued) {
+          if (!q_issued && (pos >= p.ck || round > 0)) {
             pdl_wait();
             ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
             for (int sb = 0; sb < p.kb_k; ++sb)
@@ -216,7 +223,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
         for (int sb = 0; sb < p.kb_k; ++sb)
           ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
-        q_issued = true;
       }
       if (!ok) {
         drain_wait(&aux->q_full, 0);
@@ -227,21 +233,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0 && ntiles > 0) {
-      const uint32_t id1 = ptx::idesc_f16(1, 0, 0, 128, 64);
-      const uint32_t id2 = ptx::idesc_f16(1, 1, 1, 128, 64);
+      const uint32_t id = ptx::idesc_f16(1, 0, 0, 128, 32);    // GEMM1: K-major x K-major, N = 32
+      const uint32_t id2 = ptx::idesc_f16(1, 1, 1, 128, 32);   // GEMM2: MN-major x MN-major, N = 32
       const uint32_t q_addr = ptx::smem_u32(q_s), ring_addr = ptx::smem_u32(ring), p_addr = ptx::smem_u32(p_s);
       bool ok = wait_b(&aux->q_full, 0, aux, p.err);
       ptx::tc_fence_after();
       trace_stamp(p, 2);
-      auto gemm1 = [&](int i) -> bool {
-        const int buf = i & 1;
-        if (i >= 2 && !wait_b(&aux->s_empty[buf], ((i - 2) >> 1) & 1, aux, p.err)) return false;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        // GEMM1: S = Z_k q~_hi^T + Z_k q~_lo^T (the two halves accumulate in place)
+        if (i >= 1 && !(ok = wait_b(&aux->s_empty, (i - 1) & 1, aux, p.err))) break;
         ptx::tc_fence_after();
-        const uint32_t d = tmem + buf * 64;
-        for (int c = 0; c < p.ck; ++c) {
+        for (int c = 0; c < p.ck && ok; ++c) {
           const int pos = i * per_tile + c;
           const int slot = pos % p.nslot;
-          if (!wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err)) return false;
+          if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
           ptx::tc_fence_after();
           const uint32_t sa = ring_addr + slot * kSlotBytes;
 #pragma unroll
@@ -251,53 +256,39 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int k0 = c * 128 + sb * 64 + kk * 16;
               if (k0 < p.r_k) {
                 const uint64_t ad = ptx::smem_desc(sa + sb * kSubBytes + kk * 32, 16, 1024, 2);
-                const uint64_t bd = ptx::smem_desc(q_addr + (c * 2 + sb) * kQSubBytes + kk * 32, 16, 1024, 2);
-                ptx::mma_f16(d, ad, bd, id1, k0 > 0 ? 1u : 0u);
+                const uint32_t qb = q_addr + (c * 2 + sb) * kQSubBytes + kk * 32;
+                ptx::mma_f16(tmem + kSCol, ad, ptx::smem_desc(qb, 16, 1024, 2), id, k0 > 0 ? 1u : 0u);
+                ptx::mma_f16(tmem + kSCol, ad, ptx::smem_desc(qb + kQLoOffset, 16, 1024, 2), id, 1u);
               }
             }
           }
           ptx::mma_commit(&aux->slot_empty[slot]);
         }
-        ptx::mma_commit(&aux->s_full[buf]);
+        if (!ok) break;
+        ptx::mma_commit(&aux->s_full);
         if (i < 16) trace_stamp(p, 3 + 4 * i);
-        return true;
-      };
-      auto gemm2 = [&](int i) -> bool {
-        const int buf = i & 1;
-        if (!wait_b(&aux->p_full[buf], (i >> 1) & 1, aux, p.err)) return false;
+        // GEMM2: O~ += Z_v^T P_hi + Z_v^T P_lo
+        if (!(ok = wait_b(&aux->p_full, i & 1, aux, p.err))) break;
         ptx::tc_fence_after();
-        for (int c = 0; c < p.cv; ++c) {
+        for (int c = 0; c < p.cv && ok; ++c) {
           const int pos = i * per_tile + p.ck + c;
           const int slot = pos % p.nslot;
-          if (!wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err)) return false;
+          if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
           ptx::tc_fence_after();
           const uint32_t sa = ring_addr + slot * kSlotBytes;
 #pragma unroll
           for (int kt = 0; kt < 8; ++kt) {
             const uint64_t ad = ptx::smem_desc(sa + kt * 2048, kSubBytes, 1024, 2);
-            const uint64_t bd = ptx::smem_desc(p_addr + buf * kPBytes + kt * 256, 128, 2048, 0);
-            ptx::mma_f16(tmem + kOCol + c * kOColsPerChunk, ad, bd, id2, (i > 0 || kt > 0) ? 1u : 0u);
+            const uint32_t pb = p_addr + kt * 256;
+            ptx::mma_f16(tmem + kOCol + c * 32, ad, ptx::smem_desc(pb, 128, 2048, 0), id2,
+                         (i > 0 || kt > 0) ? 1u : 0u);
+            ptx::mma_f16(tmem + kOCol + c * 32, ad, ptx::smem_desc(pb + kPHalfBytes, 128, 2048, 0), id2, 1u);
           }
           ptx::mma_commit(&aux->slot_empty[slot]);
         }
-        ptx::mma_commit(&aux->p_empty[buf]);
-        ptx::mma_commit(&aux->o_done);
+        if (!ok) break;
+        ptx::mma_commit(&aux->p_empty);
         if (i < 16) trace_stamp(p, 6 + 4 * i);
-        return true;
-      };
-      if (ok) {
-        if (p.lookahead) {
-          ok = gemm1(0);
-          for (int i = 0; i < ntiles && ok; ++i) {
-            if (i + 1 < ntiles) ok = gemm1(i + 1);
-            if (ok) ok = gemm2(i);
-          }
-        } else {
-          for (int i = 0; i < ntiles && ok; ++i) {
-            ok = gemm1(i);
-            if (ok) ok = gemm2(i);
-          }
-        }
       }
       ptx::mma_commit(&aux->o_final);
       if (!ok) drain_wait(&aux->o_final, 0);
@@ -308,43 +299,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qd = warp & 3;
     const int row = qd * 32 + lane;
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    float m[32], l[32];
+    float l[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      m[j] = -INFINITY;
-      l[j] = 0.f;
-    }
+    for (int j = 0; j < 32; ++j) l[j] = 0.f;
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
-      const int buf = i & 1;
       const bool valid = tok_begin + i * kTile + row < tok_end;
-      ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full[buf], (i >> 1) & 1, aux, p.err));
+      ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full, i & 1, aux, p.err));
       if (!ok) break;
       ptx::tc_fence_after();
       if (i < 16 && threadIdx.x == 64) trace_stamp(p, 4 + 4 * i);
-      uint32_t hi[32], lo[32];
-      ptx::tmem_ld32(tmem + lane_off + buf * 64, hi);
-      ptx::tmem_ld32(tmem + lane_off + buf * 64 + 32, lo);
+      uint32_t sv[32];
+      ptx::tmem_ld32(tmem + lane_off + kSCol, sv);
       ptx::tmem_wait_ld();
       float s[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(hi[j]) + __uint_as_float(lo[j]) : -INFINITY;
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&aux->s_empty[buf]);
+      for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
 
       bool ex = false;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) ex |= s[j] > m[j] + kLazy;
+      for (int j = 0; j < 32; ++j) ex |= s[j] > aux->m_s[j] + kLazy;
       ex = ptx::named_bar_or(1, 128, ex);
-      if (i >= 2) {
-        ok = ptx::named_bar_and(1, 128, wait_b(&aux->p_empty[buf], ((i - 2) >> 1) & 1, aux, p.err));
+      if (i >= 1) {   // the previous value mix has completed: P may be rewritten, O~ rescaled
+        ok = ptx::named_bar_and(1, 128, wait_b(&aux->p_empty, (i - 1) & 1, aux, p.err));
         if (!ok) break;
+        ptx::tc_fence_after();
       }
       if (ex) {
-        float v[32];
+        // reduce in place, then read the scores again (S stays intact until s_empty)
+        aux->red[qd][lane] = warp_reduce_scatter32<true>(s, lane);
+        ptx::tmem_ld32(tmem + lane_off + kSCol, sv);
+        ptx::tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = s[j];
-        aux->red[qd][lane] = warp_reduce_scatter32<true>(v, lane);
+        for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
         ptx::named_bar_sync(1, 128);
         if (qd == 0) {
           const float mt = fmaxf(fmaxf(aux->red[0][lane], aux->red[1][lane]), fmaxf(aux->red[2][lane], aux->red[3][lane]));
@@ -354,51 +341,53 @@ __global__ void __launch_bounds__(kThreads, 1)
           aux->m_s[lane] = mn;
         }
         ptx::named_bar_sync(1, 128);
-        float alpha[32];
         bool need_o = false;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          m[j] = aux->m_s[j];
-          alpha[j] = aux->alpha_s[j];
-          l[j] *= alpha[j];
-          need_o |= alpha[j] < 1.f;
+          const float a = aux->alpha_s[j];
+          l[j] *= a;
+          need_o |= a < 1.f;
         }
         if (need_o && i > 0) {
-          ok = ptx::named_bar_and(1, 128, wait_b(&aux->o_done, (i - 1) & 1, aux, p.err));
-          if (!ok) break;
-          ptx::tc_fence_after();
-          for (int c = 0; c < 2 * p.cv; ++c) {
+          for (int c = 0; c < p.cv; ++c) {
             uint32_t v2[32];
             ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v2[j] = __float_as_uint(__uint_as_float(v2[j]) * alpha[j]);
+            for (int j = 0; j < 32; ++j) v2[j] = __float_as_uint(__uint_as_float(v2[j]) * aux->alpha_s[j]);
             ptx::tmem_st32(tmem + lane_off + kOCol + c * 32, v2);
           }
           ptx::tmem_wait_st();
         }
       }
-      uint32_t pk[32];   // [0..15] hi pairs, [16..31] lo pairs
+      // probabilities in two bf16 halves: p = hi + lo, hi = bf16(p), lo = bf16(p - hi)
+      const uint32_t prow = ptx::smem_u32(p_s + row * 16);
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const float p0 = exp2f(s[2 * jj] - m[2 * jj]);
-        const float p1 = exp2f(s[2 * jj + 1] - m[2 * jj + 1]);
-        const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(p0 - __low2float(h), p1 - __high2float(h));
-        l[2 * jj] += p0;
-        l[2 * jj + 1] += p1;
-        pk[jj] = *reinterpret_cast<const uint32_t*>(&h);
-        pk[16 + jj] = *reinterpret_cast<const uint32_t*>(&lo2);
-      }
-      const uint32_t prow = ptx::smem_u32(p_s + buf * kPBytes + row * 16);
+      for (int hg = 0; hg < 4; ++hg) {
+        uint32_t hw[4], lw[4];
 #pragma unroll
-      for (int hg = 0; hg < 8; ++hg)
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + hg * 2048), "r"(pk[4 * hg]),
-                     "r"(pk[4 * hg + 1]), "r"(pk[4 * hg + 2]), "r"(pk[4 * hg + 3])
+        for (int e = 0; e < 4; ++e) {
+          const int j = hg * 8 + 2 * e;
+          const float p0 = exp2f(s[j] - aux->m_s[j]);
+          const float p1 = exp2f(s[j + 1] - aux->m_s[j + 1]);
+          const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+          const __nv_bfloat162 lo2 = __floats2bfloat162_rn(p0 - __low2float(h), p1 - __high2float(h));
+          l[j] += p0;
+          l[j + 1] += p1;
+          hw[e] = *reinterpret_cast<const uint32_t*>(&h);
+          lw[e] = *reinterpret_cast<const uint32_t*>(&lo2);
+        }
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + hg * 2048), "r"(hw[0]), "r"(hw[1]),
+                     "r"(hw[2]), "r"(hw[3])
                      : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + kPHalfBytes + hg * 2048), "r"(lw[0]),
+                     "r"(lw[1]), "r"(lw[2]), "r"(lw[3])
+                     : "memory");
+      }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&aux->p_full[buf]);
+      ptx::mbar_arrive(&aux->s_empty);
+      ptx::mbar_arrive(&aux->p_full);
       if (i < 16 && threadIdx.x == 64) trace_stamp(p, 5 + 4 * i);
     }
     if (ok) ok = ptx::named_bar_and(1, 128, wait_b(&aux->o_final, 0, aux, p.err));
@@ -406,15 +395,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_after();
       const size_t base_out = ((size_t)b * p.n_splits + split) * p.Hq;
       for (int c = 0; c < p.cv; ++c) {
-        uint32_t vh[32], vl[32];
-        ptx::tmem_ld32(tmem + lane_off + kOCol + c * kOColsPerChunk, vh);
-        ptx::tmem_ld32(tmem + lane_off + kOCol + c * kOColsPerChunk + 32, vl);
+        uint32_t v2[32];
+        ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
         ptx::tmem_wait_ld();
         const int e = c * 128 + qd * 32 + lane;
         if (e < p.r_v) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j < p.Hq) p.part_o[(base_out + j) * p.r_v + e] = __uint_as_float(vh[j]) + __uint_as_float(vl[j]);
+            if (j < p.Hq) p.part_o[(base_out + j) * p.r_v + e] = __uint_as_float(v2[j]);
         }
       }
       aux->red[qd][lane] = warp_reduce_scatter32<false>(l, lane);
@@ -465,9 +453,21 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
 
 int q_bytes_for(int r_k) { return ((r_k + 63) / 64) * kQSubBytes; }
 
-int slots_that_fit(const lr_cache_desc* d) {
-  const int fixed = 1024 + q_bytes_for(d->rank_k) + 2 * kPBytes + (int)sizeof(Aux);
-  return std::min(kMaxSlots, (kSmemLimit - fixed) / kSlotBytes);
+size_t smem_for(int r_k, int nslot) { return (size_t)kAuxBytes + q_bytes_for(r_k) + (size_t)nslot * kSlotBytes + kPBytes; }
+
+// Two blocks per SM when the block fits half the SM with a 2-slot ring (the streaming
+// rate of two rings per SM is higher than one deeper ring); otherwise one block with
+// as many slots as fit.
+void choose_slots(const lr_cache_desc* d, int* nslot, int* ctas_per_sm) {
+  if (smem_for(d->rank_k, 2) <= (size_t)kSmemPair) {
+    *nslot = 2;
+    *ctas_per_sm = 2;
+    return;
+  }
+  int n = 0;
+  while (n + 1 <= kMaxSlots && smem_for(d->rank_k, n + 1) <= (size_t)kSmemLimit) ++n;
+  *nslot = n;
+  *ctas_per_sm = 1;
 }
 
 }  // namespace
@@ -475,8 +475,15 @@ int slots_that_fit(const lr_cache_desc* d) {
 bool tc_supported(const lr_cache_desc* d) {
   if (d->dtype != LR_BF16 || d->quant_bits != 0 || d->rope_in_kernel) return false;
   if (d->n_q_heads > 32) return false;
-  const int ck = (d->rank_k + 127) / 128, cv = (d->rank_v + 127) / 128;
-  return slots_that_fit(d) >= std::max(std::max(ck, cv), 2);
+  int nslot, cps;
+  choose_slots(d, &nslot, &cps);
+  return nslot >= 1;
+}
+
+int tc_ctas_per_sm(const lr_cache_desc* d) {
+  int nslot, cps;
+  choose_slots(d, &nslot, &cps);
+  return cps;
 }
 
 cudaError_t tc_prepare(lr_cache* c) {
@@ -509,11 +516,8 @@ cudaError_t tc_prepare(lr_cache* c) {
     if (!make_map(side ? &st->zv : &st->zk, side ? c->z_v : c->z_k, 3, dims, strides, box))
       return cudaErrorInvalidValue;
   }
-  const int ck = (d.rank_k + 127) / 128, cv = (d.rank_v + 127) / 128;
-  st->nslot = slots_that_fit(&d);
-  st->lookahead = st->nslot >= ck + cv ? 1 : 0;
-  if (st->lookahead) st->nslot = std::min(st->nslot, std::max(ck + cv + 1, 4));
-  st->smem = 1024 + q_bytes_for(d.rank_k) + (size_t)st->nslot * kSlotBytes + 2 * kPBytes + sizeof(Aux);
+  choose_slots(&d, &st->nslot, &st->ctas_per_sm);
+  st->smem = smem_for(d.rank_k, st->nslot);
   return cudaSuccess;
 }
 
@@ -532,13 +536,12 @@ cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, 
   p.ck = (d.rank_k + 127) / 128;
   p.cv = (d.rank_v + 127) / 128;
   p.kb_k = (d.rank_k + 63) / 64;
-  p.tmem_cols = (kOCol + p.cv * kOColsPerChunk) <= 256 ? 256 : 512;
+  p.tmem_cols = (kOCol + p.cv * 32) <= 128 ? 128 : 256;
   p.Hq = d.n_q_heads;
   p.hist_len = c->hist_len;
   p.split_tokens = split_tokens;
   p.n_splits = n_splits;
   p.nslot = st->nslot;
-  p.lookahead = st->lookahead;
   p.q_bytes = q_bytes_for(d.rank_k);
   p.part_o = c->part_o;
   p.part_ml = c->part_ml;

@@ -1,0 +1,500 @@
+// The small kernels around the decode: query projection (q~ = s log2(e) B_k,h q), the
+// append of one token (z = k A, stored / quantised, window ring and fold), both fused
+// in one grid for lr_decode_step, and the split merge with the output projection
+// (o = o~ B_v,h / l).
+//
+// Method: TraceKV abstract (latent KV storage, low-rank attention kernels); iS-KV
+// abstract and method section (exact window, folding).
+//
+// These kernels move little data (bases, one token, one query), so they are built for
+// issue efficiency: the element type is a template parameter, shared-memory reads are
+// 16-byte vectors, each thread computes a rank row for every query head of its group,
+// and the bases — which no in-flight kernel writes — are staged with cp.async before
+// the grid-dependency wait, overlapping the preceding kernel.
+#include "lr_internal.cuh"
+#include "k_common.cuh"
+
+#include <algorithm>
+
+namespace {
+
+// ---- element helpers ---------------------------------------------------------------
+template <typename T>
+struct El;
+template <>
+struct El<__nv_bfloat16> {
+  static __device__ __forceinline__ float ld(const void* p, size_t i) {
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  }
+  static __device__ __forceinline__ void st(void* p, size_t i, float v) {
+    reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  }
+  // 8 consecutive elements from 16-byte aligned shared memory
+  static __device__ __forceinline__ void lds8(const uint8_t* s, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(s);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = __uint_as_float(w[k] << 16);
+      v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+  static __device__ __forceinline__ float lds1(const uint8_t* s) {
+    return __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(s)) << 16);
+  }
+};
+template <>
+struct El<float> {
+  static __device__ __forceinline__ float ld(const void* p, size_t i) { return reinterpret_cast<const float*>(p)[i]; }
+  static __device__ __forceinline__ void st(void* p, size_t i, float v) { reinterpret_cast<float*>(p)[i] = v; }
+  static __device__ __forceinline__ void lds8(const uint8_t* s, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(s);
+    const float4 b = *reinterpret_cast<const float4*>(s + 16);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  static __device__ __forceinline__ float lds1(const uint8_t* s) { return *reinterpret_cast<const float*>(s); }
+};
+
+// ---- query projection -----------------------------------------------------------
+// One CTA per (128 rank rows of B_k,h, KV head h, sequence b); thread = rank row i,
+// for every query head j of the group: q~_j[i] = s log2(e) sum_c B_k[i][h d + c] q_j[c].
+// qt16 (tensor-core path): rows [b][j] and [b][32 + j] of a [B][64][r_k] bf16 array get
+// hi = bf16(q~) and lo = bf16(q~ - hi), so that hi + lo carries q~ to ~16 significant bits.
+constexpr int kQRowsCta = 128;
+constexpr int kHB = 8;            // query heads per register block
+
+struct QprojArgs {
+  const void* q; const void* Bk; float* qt; float* qd; __nv_bfloat16* qt16;
+  int Hq, Hkv, d, D, rk;
+  float scale_log2;
+  int want_latent;
+};
+
+template <typename T>
+__device__ __forceinline__ int qproj_pitch(int d) { return d * (int)sizeof(T) + 16; }
+
+template <typename T>
+__device__ __forceinline__ void qproj_stage(const QprojArgs& a, int rchunk, int h, uint8_t* smem) {
+  const int r0 = rchunk * kQRowsCta;
+  const int nr = min(kQRowsCta, a.rk - r0);
+  if (a.want_latent && nr > 0)
+    stage_rows(smem, qproj_pitch<T>(a.d), a.Bk, a.D, sizeof(T), r0, nr, (long long)h * a.d, a.d);
+}
+
+template <typename T>
+__device__ __forceinline__ void qproj_main(const QprojArgs& a, int rchunk, int h, int b, uint8_t* smem) {
+  const int d = a.d, G = a.Hq / a.Hkv, j0 = h * G;
+  const int pitch = qproj_pitch<T>(d);
+  float* qs = reinterpret_cast<float*>(smem + (size_t)kQRowsCta * pitch);   // [G][d]
+  const size_t qoff = ((size_t)b * a.Hq + j0) * d;
+#pragma unroll 4
+  for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) {
+    const float v = El<T>::ld(a.q, qoff + idx);
+    qs[idx] = v;
+    if (a.qd && rchunk == 0) a.qd[qoff + idx] = v * a.scale_log2;
+  }
+  if (!a.want_latent) return;
+  cp_async_wait_all();
+  __syncthreads();
+  const int r0 = rchunk * kQRowsCta;
+  const int nr = min(kQRowsCta, a.rk - r0);
+  for (int t = threadIdx.x; t < nr; t += blockDim.x) {
+    const uint8_t* row = smem + (size_t)t * pitch;
+    const int i = r0 + t;
+    for (int jb = 0; jb < G; jb += kHB) {
+      float acc[kHB];
+#pragma unroll
+      for (int u = 0; u < kHB; ++u) acc[u] = 0.f;
+      for (int c = 0; c < d; c += 8) {
+        float bv[8];
+        El<T>::lds8(row + (size_t)c * sizeof(T), bv);
+#pragma unroll
+        for (int u = 0; u < kHB; ++u) {
+          if (jb + u < G) {
+            const float4 q0 = *reinterpret_cast<const float4*>(qs + (jb + u) * d + c);
+            const float4 q1 = *reinterpret_cast<const float4*>(qs + (jb + u) * d + c + 4);
+            acc[u] = fmaf(bv[0], q0.x, acc[u]);
+            acc[u] = fmaf(bv[1], q0.y, acc[u]);
+            acc[u] = fmaf(bv[2], q0.z, acc[u]);
+            acc[u] = fmaf(bv[3], q0.w, acc[u]);
+            acc[u] = fmaf(bv[4], q1.x, acc[u]);
+            acc[u] = fmaf(bv[5], q1.y, acc[u]);
+            acc[u] = fmaf(bv[6], q1.z, acc[u]);
+            acc[u] = fmaf(bv[7], q1.w, acc[u]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kHB; ++u) {
+        if (jb + u < G) {
+          const int j = j0 + jb + u;
+          const float v = acc[u] * a.scale_log2;
+          a.qt[((size_t)b * a.Hq + j) * a.rk + i] = v;
+          if (a.qt16) {
+            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+            a.qt16[((size_t)b * 64 + j) * a.rk + i] = hi;
+            a.qt16[((size_t)b * 64 + 32 + j) * a.rk + i] = lo;
+          }
+        }
+      }
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) k_qproj(QprojArgs a) {
+  extern __shared__ __align__(16) uint8_t qsm[];
+  qproj_stage<T>(a, blockIdx.x, blockIdx.y, qsm);      // bases: stable data
+  pdl_wait();
+  pdl_trigger();
+  qproj_main<T>(a, blockIdx.x, blockIdx.y, blockIdx.z, qsm);
+}
+
+size_t qproj_smem(const lr_cache_desc& d, size_t es) {
+  return (size_t)kQRowsCta * (d.head_dim * es + 16) + (size_t)(d.n_q_heads / d.n_kv_heads) * d.head_dim * sizeof(float);
+}
+
+// ---- append -----------------------------------------------------------------------
+// One CTA per (32-coordinate chunk of K or V, sequence b): z[i] = sum_c x[c] A[c][i].
+// The chunk's columns of A ([D][32]) are staged before the grid-dependency wait; the
+// source row after it.  The 8 warps take fixed eighths of D and the partial sums are
+// added in a fixed order, so the projection does not depend on the storage kind.
+struct AppendArgs {
+  const void* src_k; const void* src_v;   // rows to project (input or evicted ring rows)
+  long long src_bstride;                  // elements between batch rows of src
+  const void* A_k; const void* A_v;
+  void* Zk; void* Zv; uint32_t* codes_k; uint32_t* codes_v; uint32_t* params_k; uint32_t* params_v;
+  int rk, rv, Gk, Gv, chunks_k, chunks_v;
+  long long cap; int dst_slot; int project;
+  const void* new_k; const void* new_v;   // exact token for the ring, or null
+  void* win_k; void* win_v; int slots; int new_slot;
+  int B, D, kind, dtype;
+};
+
+template <typename T>
+__device__ __forceinline__ void append_stage(const AppendArgs& a, int x, uint8_t* smem) {
+  const int nproj = a.project ? (a.chunks_k + a.chunks_v) : 0;
+  if (x >= nproj) return;
+  const bool is_k = x < a.chunks_k;
+  const int ch = is_k ? x : x - a.chunks_k;
+  const int r = is_k ? a.rk : a.rv;
+  const int ncol = min(32, r - ch * 32);         // 16 or 32 (ranks are multiples of 16)
+  stage_rows(smem, 32 * sizeof(T), is_k ? a.A_k : a.A_v, r, sizeof(T), 0, a.D, (long long)ch * 32, ncol);
+}
+
+template <typename T>
+__device__ __forceinline__ void append_main(const AppendArgs& a, int x, int b, uint8_t* smem, float (*red)[32]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nproj = a.project ? (a.chunks_k + a.chunks_v) : 0;
+  constexpr int es = sizeof(T);
+  if (x < nproj) {
+    const bool is_k = x < a.chunks_k;
+    const int ch = is_k ? x : x - a.chunks_k;
+    const int r = is_k ? a.rk : a.rv;
+    const void* src = is_k ? a.src_k : a.src_v;
+    const int ncol = min(32, r - ch * 32);
+    const uint8_t* As = smem;                            // [D][32]
+    uint8_t* xs = smem + (size_t)a.D * 32 * es;          // [D]
+    const uint8_t* g = reinterpret_cast<const uint8_t*>(src) + (size_t)b * a.src_bstride * es;
+    for (int v = threadIdx.x; v < a.D * es / 16; v += blockDim.x) cp_async16(xs + v * 16, g + v * 16);
+    cp_async_wait_all();
+    __syncthreads();
+    const int per = (((a.D + 7) / 8) + 7) & ~7;          // multiple of 8 (vector reads of x)
+    const int cb = warp * per, ce = min(a.D, cb + per);
+    float z0 = 0.f, z1 = 0.f;
+    if (lane < ncol) {
+      for (int c = cb; c < ce; c += 8) {
+        float xv[8];
+        El<T>::lds8(xs + (size_t)c * es, xv);
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          z0 = fmaf(xv[e], El<T>::lds1(As + ((size_t)(c + e) * 32 + lane) * es), z0);
+          z1 = fmaf(xv[e + 1], El<T>::lds1(As + ((size_t)(c + e + 1) * 32 + lane) * es), z1);
+        }
+      }
+    }
+    red[warp][lane] = z0 + z1;
+    __syncthreads();
+    if (warp == 0) {
+      float z = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) z += red[w][lane];
+      const long long row = (long long)b * a.cap + a.dst_slot;
+      store_latent_chunk(z, ch, r, a.kind, a.dtype, is_k ? a.Zk : a.Zv, is_k ? a.codes_k : a.codes_v,
+                         is_k ? a.params_k : a.params_v, is_k ? a.Gk : a.Gv, row);
+    }
+    return;
+  }
+  // ring write of the exact new token of sequence b
+  const bool is_k = (x - nproj) == 0;
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(is_k ? a.new_k : a.new_v) + (size_t)b * a.D * es;
+  uint8_t* dst = reinterpret_cast<uint8_t*>(is_k ? a.win_k : a.win_v) + ((size_t)b * a.slots + a.new_slot) * a.D * es;
+  for (int v = threadIdx.x; v < a.D * es / 16; v += blockDim.x)
+    reinterpret_cast<uint4*>(dst)[v] = reinterpret_cast<const uint4*>(src)[v];
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_append(AppendArgs a) {
+  extern __shared__ __align__(16) uint8_t asm_[];
+  __shared__ float red[8][32];
+  append_stage<T>(a, blockIdx.x, asm_);                 // bases: stable data
+  pdl_wait();
+  pdl_trigger();
+  append_main<T>(a, blockIdx.x, blockIdx.y, asm_, red);
+}
+
+// The independent first half of a decode step in one grid: CTAs [0, x_app) of each
+// row are the append of the new token, the others the query projection.
+template <typename T>
+__global__ void __launch_bounds__(256) k_step_pre(AppendArgs aa, QprojArgs qa, int x_app, int nchunks_q) {
+  extern __shared__ __align__(16) uint8_t psm[];
+  __shared__ float red[8][32];
+  const int x = blockIdx.x, b = blockIdx.y;
+  const int qx = x - x_app;
+  if (x < x_app) append_stage<T>(aa, x, psm);
+  else qproj_stage<T>(qa, qx % nchunks_q, qx / nchunks_q, psm);
+  pdl_wait();
+  pdl_trigger();
+  if (x < x_app) append_main<T>(aa, x, b, psm, red);
+  else qproj_main<T>(qa, qx % nchunks_q, qx / nchunks_q, b, psm);
+}
+
+// ---- split merge and output projection ------------------------------------------
+// One CTA per (query head j, sequence b); thread = pair of output columns.  The
+// B_v,h slice is staged before the grid-dependency wait; then the split weights
+// (log-sum-exp with the window partial), the combined rank-space output o~ (all S
+// partial loads of a rank issued together), and o = o~ B_v,h / l.
+constexpr int kMergeThreads = 128;
+constexpr size_t kMergeStage = 64 * 1024;    // bytes of B_v,h rows staged in shared memory
+
+template <typename T>
+__global__ void __launch_bounds__(kMergeThreads) k_merge(const float* part_o, const float* part_ml,
+                                                         const float* win_o, const float* win_ml,
+                                                         const void* Bv, void* out, float* lse, int S, int Hq,
+                                                         int Hkv, int d, int D, int rv) {
+  extern __shared__ __align__(16) uint8_t msm[];
+  constexpr int es = sizeof(T);
+  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int h = j / (Hq / Hkv);
+  const int pitch = d * es;
+  const int rows_staged = min(rv, (int)(kMergeStage / pitch));
+  uint8_t* bs = msm;                                                   // [rows_staged][d]
+  float* ot = reinterpret_cast<float*>(msm + (size_t)rows_staged * pitch);   // [rv]
+  float* w_s = ot + rv;                                                // [S]
+  float* hdr = w_s + S;                                                // m*, 1/l, window weight
+  stage_rows(bs, pitch, Bv, D, es, 0, rows_staged, (long long)h * d, d);   // bases: stable data
+  pdl_wait();
+  pdl_trigger();
+  if (tid < 32) {
+    const int lane = tid;
+    float m = -INFINITY;
+    for (int s = lane; s < S; s += 32) m = fmaxf(m, part_ml[(((size_t)b * S + s) * Hq + j) * 2]);
+    const float mw = win_ml ? win_ml[((size_t)b * Hq + j) * 2] : -INFINITY;
+    m = fmaxf(m, mw);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    for (int s = lane; s < S; s += 32) {
+      const size_t e = (((size_t)b * S + s) * Hq + j) * 2;
+      const float ms = part_ml[e];
+      const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - m);
+      w_s[s] = w;
+      l = fmaf(w, part_ml[e + 1], l);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      float ww = 0.f;
+      if (win_ml && mw != -INFINITY) {
+        ww = exp2f(mw - m);
+        l = fmaf(ww, win_ml[((size_t)b * Hq + j) * 2 + 1], l);
+      }
+      hdr[0] = m;
+      hdr[1] = 1.0f / l;
+      hdr[2] = ww;
+      if (lse) lse[(size_t)b * Hq + j] = (m + log2f(l)) * LR_LN2;
+    }
+  }
+  __syncthreads();
+  const size_t sstride = (size_t)Hq * rv;
+  for (int i = tid; i < rv; i += blockDim.x) {
+    const float* src = part_o + ((size_t)b * S * Hq + j) * rv + i;
+    float acc = 0.f;
+    for (int s0 = 0; s0 < S; s0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = (s0 + k < S) ? __ldg(src + k * sstride) : 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (s0 + k < S) acc = fmaf(w_s[s0 + k], v[k], acc);
+      src += 8 * sstride;
+    }
+    ot[i] = acc;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  const size_t ooff = ((size_t)b * Hq + j) * d;
+  for (int c = 2 * tid; c < d; c += 2 * blockDim.x) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int i = 0;
+    for (; i + 4 <= rows_staged; i += 4) {
+      const float4 o4 = *reinterpret_cast<const float4*>(ot + i);
+      const uint8_t* p0 = bs + (size_t)i * pitch + (size_t)c * es;
+      a0 = fmaf(o4.x, El<T>::lds1(p0), a0);
+      a1 = fmaf(o4.x, El<T>::lds1(p0 + es), a1);
+      a2 = fmaf(o4.y, El<T>::lds1(p0 + pitch), a2);
+      a3 = fmaf(o4.y, El<T>::lds1(p0 + pitch + es), a3);
+      a0 = fmaf(o4.z, El<T>::lds1(p0 + 2 * pitch), a0);
+      a1 = fmaf(o4.z, El<T>::lds1(p0 + 2 * pitch + es), a1);
+      a2 = fmaf(o4.w, El<T>::lds1(p0 + 3 * pitch), a2);
+      a3 = fmaf(o4.w, El<T>::lds1(p0 + 3 * pitch + es), a3);
+    }
+    for (; i < rv; ++i) {
+      const float b0 = i < rows_staged ? El<T>::lds1(bs + (size_t)i * pitch + (size_t)c * es)
+                                       : El<T>::ld(Bv, (size_t)i * D + (size_t)h * d + c);
+      const float b1 = i < rows_staged ? El<T>::lds1(bs + (size_t)i * pitch + (size_t)(c + 1) * es)
+                                       : El<T>::ld(Bv, (size_t)i * D + (size_t)h * d + c + 1);
+      a0 = fmaf(ot[i], b0, a0);
+      a1 = fmaf(ot[i], b1, a1);
+    }
+    float o0 = a0 + a2, o1 = a1 + a3;
+    if (win_o) {
+      o0 = fmaf(hdr[2], win_o[ooff + c], o0);
+      o1 = fmaf(hdr[2], win_o[ooff + c + 1], o1);
+    }
+    El<T>::st(out, ooff + c, o0 * hdr[1]);
+    El<T>::st(out, ooff + c + 1, o1 * hdr[1]);
+  }
+}
+
+size_t merge_smem(const lr_cache_desc& d, int S, size_t es) {
+  const size_t pitch = (size_t)d.head_dim * es;
+  const size_t rows = std::min((size_t)d.rank_v, kMergeStage / pitch);
+  return rows * pitch + ((size_t)d.rank_v + S + 4) * sizeof(float);
+}
+
+// ---- argument construction ------------------------------------------------------------
+QprojArgs make_qproj_args(const lr_cache* c, const void* q, bool tc) {
+  const lr_cache_desc& d = c->desc;
+  const bool rope = d.rope_in_kernel != 0;
+  QprojArgs a;
+  a.q = q;
+  a.Bk = c->B_k;
+  a.qt = c->qt;
+  a.qd = (rope || c->win_slots) ? (rope ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k) : nullptr;
+  a.qt16 = tc ? (__nv_bfloat16*)c->qt16 : nullptr;
+  a.Hq = d.n_q_heads; a.Hkv = d.n_kv_heads; a.d = d.head_dim; a.D = c->D; a.rk = d.rank_k;
+  a.scale_log2 = c->scale_log2;
+  a.want_latent = rope ? 0 : 1;
+  return a;
+}
+
+int qproj_chunks(const lr_cache* c) {
+  return c->desc.rope_in_kernel ? 1 : (c->desc.rank_k + kQRowsCta - 1) / kQRowsCta;
+}
+
+AppendArgs make_append_args(const lr_cache* c, const void* k, const void* v) {
+  const lr_cache_desc& d = c->desc;
+  AppendArgs a;
+  const bool win = c->win_slots > 0;
+  const bool fold = win && c->win_len == d.window;
+  a.project = win ? (fold ? 1 : 0) : 1;
+  if (win) {
+    const int old_slot = c->hist_len % c->win_slots;
+    const size_t es = c->esize;
+    a.src_k = (const char*)c->win_k + (size_t)old_slot * c->D * es;
+    a.src_v = (const char*)c->win_v + (size_t)old_slot * c->D * es;
+    a.src_bstride = (long long)c->win_slots * c->D;
+  } else {
+    a.src_k = k; a.src_v = v; a.src_bstride = c->D;
+  }
+  a.A_k = c->A_k; a.A_v = c->A_v;
+  a.Zk = c->z_k; a.Zv = c->z_v; a.codes_k = c->codes_k; a.codes_v = c->codes_v;
+  a.params_k = c->params_k; a.params_v = c->params_v;
+  a.rk = d.rank_k; a.rv = d.rank_v; a.Gk = c->G_k; a.Gv = c->G_v;
+  a.chunks_k = (d.rank_k + 31) / 32; a.chunks_v = (d.rank_v + 31) / 32;
+  a.cap = d.capacity; a.dst_slot = c->hist_len;
+  a.new_k = win ? k : nullptr; a.new_v = win ? v : nullptr;
+  a.win_k = c->win_k; a.win_v = c->win_v; a.slots = c->win_slots;
+  a.new_slot = win ? (c->len % c->win_slots) : 0;
+  a.B = d.batch; a.D = c->D; a.kind = c->latent_kind; a.dtype = d.dtype;
+  return a;
+}
+
+int append_ctas(const AppendArgs& a) { return (a.project ? a.chunks_k + a.chunks_v : 0) + (a.new_k ? 2 : 0); }
+
+size_t append_smem(const lr_cache* c) { return (size_t)c->D * 32 * c->esize + (size_t)c->D * c->esize; }
+
+template <typename T>
+cudaError_t qproj_t(const lr_cache* c, const void* q, cudaStream_t s, bool tc) {
+  const lr_cache_desc& d = c->desc;
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_qproj<T>, optin_done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_qproj<T>, dim3(qproj_chunks(c), d.n_kv_heads, d.batch), dim3(128), qproj_smem(d, sizeof(T)), s,
+                    make_qproj_args(c, q, tc));
+}
+
+template <typename T>
+cudaError_t merge_t(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  const bool win = c->win_slots > 0;
+  const size_t smem = merge_smem(d, n_splits, sizeof(T));
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_merge<T>, optin_done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_merge<T>, dim3(d.n_q_heads, d.batch), dim3(kMergeThreads), smem, s, c->part_o, c->part_ml,
+                    win ? c->win_o : nullptr, win ? c->win_ml : nullptr, c->B_v, out, lse, n_splits, d.n_q_heads,
+                    d.n_kv_heads, d.head_dim, c->D, d.rank_v);
+}
+
+template <typename T>
+cudaError_t append_t(lr_cache* c, const void* k, const void* v, cudaStream_t s) {
+  const AppendArgs a = make_append_args(c, k, v);
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_append<T>, optin_done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_append<T>, dim3(append_ctas(a), c->desc.batch), dim3(256), append_smem(c), s, a);
+}
+
+template <typename T>
+cudaError_t step_pre_t(lr_cache* c, const void* k, const void* v, const void* q, bool tc, cudaStream_t s) {
+  const AppendArgs aa = make_append_args(c, k, v);
+  const QprojArgs qa = make_qproj_args(c, q, tc);
+  const int x_app = append_ctas(aa);
+  const int nq = qproj_chunks(c);
+  const size_t smem = std::max(append_smem(c), qproj_smem(c->desc, sizeof(T)));
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_step_pre<T>, optin_done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_step_pre<T>, dim3(x_app + nq * c->desc.n_kv_heads, c->desc.batch), dim3(256), smem, s, aa, qa,
+                    x_app, nq);
+}
+
+}  // namespace
+
+cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s) {
+  return c->desc.dtype == LR_BF16 ? qproj_t<__nv_bfloat16>(c, q, s, false) : qproj_t<float>(c, q, s, false);
+}
+
+cudaError_t launch_qproj_tc(const lr_cache* c, const void* q, cudaStream_t s) {
+  if (!c->qt16 || c->desc.dtype != LR_BF16) return cudaErrorNotSupported;
+  return qproj_t<__nv_bfloat16>(c, q, s, true);
+}
+
+cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s) {
+  return c->desc.dtype == LR_BF16 ? merge_t<__nv_bfloat16>(c, n_splits, out, lse, s)
+                                  : merge_t<float>(c, n_splits, out, lse, s);
+}
+
+cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s) {
+  return c->desc.dtype == LR_BF16 ? append_t<__nv_bfloat16>(c, k, v, s) : append_t<float>(c, k, v, s);
+}
+
+cudaError_t launch_step_pre(lr_cache* c, const void* k, const void* v, const void* q, bool tc, cudaStream_t s) {
+  if (tc && c->desc.dtype != LR_BF16) return cudaErrorNotSupported;
+  return c->desc.dtype == LR_BF16 ? step_pre_t<__nv_bfloat16>(c, k, v, q, tc, s)
+                                  : step_pre_t<float>(c, k, v, q, false, s);
+}
