@@ -20,17 +20,20 @@
 // thread; warps 2..5 run the softmax (thread = token row = TMEM lane) and the
 // epilogue (thread = rank row).  Every wait is bounded: on timeout the kernel records
 // LR_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
-#include "lr_internal.cuh"
-#include "ptx.cuh"
+#include "tc_common.cuh"
 
-#include <cudaTypedefs.h>
-
-#include <mutex>
+#include <algorithm>
 
 namespace {
 
+using tc::drain_wait;
+using tc::kLazy;
+using tc::kSmemLimit;
+using tc::kTile;
+using tc::kTraceSlots;
+using tc::warp_reduce_scatter32;
+
 constexpr int kThreads = 192;
-constexpr int kTile = 128;                 // tokens per tile
 constexpr int kSubBytes = 128 * 128;       // 128 tokens x 64 ranks x 2 B
 constexpr int kSlotBytes = 2 * kSubBytes;  // 128 tokens x 128 ranks
 constexpr int kQRows = 64;                 // 32 head rows (hi) + 32 head rows (lo)
@@ -42,18 +45,11 @@ constexpr int kAuxBytes = 1024;            // barriers and reduction scratch, fi
 constexpr int kSCol = 0;                   // TMEM: S in columns [0, 32)
 constexpr int kOCol = 32;                  // TMEM: O~ chunk c in columns [32 + 32c, 64 + 32c)
 constexpr int kMaxSlots = 8;
-constexpr float kLazy = 8.0f;              // log2 of the allowed growth before a rescale
-constexpr uint64_t kTimeoutNs = 2000000000ull;
-constexpr int kSmemLimit = 232448;         // 227 KB opt-in per block
 constexpr int kSmemPair = 115712;          // per block when two blocks share an SM (228 KB - 2 x 1 KB)
-constexpr int kTraceSlots = 72;            // 0 start, 1 setup done, 2 query latents in,
-                                           // 3+4i: key tile i consumed, 4+4i: scores of tile i read,
-                                           // 5+4i: probabilities of tile i written,
-                                           // 6+4i: value mix of tile i issued (i < 16), 71 end
 
 struct TcParams {
   int r_k, r_v, ck, cv, kb_k, tmem_cols;
-  int Hq, hist_len, split_tokens, n_splits, nslot;
+  int Hq, hist_len, stable_len, split_tokens, n_splits, nslot;
   uint32_t q_bytes;
   float* part_o;
   float* part_ml;
@@ -81,49 +77,10 @@ struct TcState {
 };
 
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = ptx::globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((it & 31) == 0) {
-      if (*(volatile int*)&aux->abort_flag) return false;
-      if (ptx::globaltimer() - t0 > kTimeoutNs) {
-        *(volatile int*)&aux->abort_flag = 1;
-        atomicExch(err, (int)LR_ERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
+  return tc::wait_b(bar, parity, &aux->abort_flag, err);
 }
 
-__device__ __forceinline__ void trace_stamp(const TcParams& p, int slot) {
-  if (p.trace) p.trace[((size_t)blockIdx.y * gridDim.x + blockIdx.x) * kTraceSlots + slot] = ptx::globaltimer();
-}
-
-// Wait that ignores the abort flag (used to drain in-flight work after an abort).
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = ptx::globaltimer();
-  while (!ptx::mbar_try_wait(bar, parity))
-    if (ptx::globaltimer() - t0 > kTimeoutNs) return;
-}
-
-// Butterfly reduce-scatter over a warp: on return lane l holds op over all lanes of
-// v[l] (v is destroyed).
-template <bool kMax>
-__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane) {
-#pragma unroll
-  for (int w = 16; w >= 1; w >>= 1) {
-    const bool up = (lane & w) != 0;
-#pragma unroll
-    for (int k = 0; k < w; ++k) {
-      const float keep = up ? v[k + w] : v[k];
-      const float send = up ? v[k] : v[k + w];
-      const float got = __shfl_xor_sync(0xffffffffu, send, w);
-      v[k] = kMax ? fmaxf(keep, got) : keep + got;
-    }
-  }
-  return v[0];
-}
+__device__ __forceinline__ void trace_stamp(const TcParams& p, int slot) { tc::trace_stamp(p.trace, slot); }
 
 // Shared memory: [aux 1 KB][q~ hi|lo per 64-rank sub-block][ring of nslot x 32 KB][P hi | P lo].
 // The dynamic shared-memory window starts 1024-byte aligned (checked); the swizzled
@@ -184,9 +141,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0 && ntiles > 0) {
-      // The first tile's key chunks are issued before the grid-dependency wait: the
-      // cache was written by kernels that completed before the preceding (query
-      // projection) kernel allowed this one to start.  The query latents are not.
+      // The first tile's key chunks are issued before the grid-dependency wait when
+      // every token of the tile lies below stable_len: those rows were written by
+      // kernels that completed before the preceding kernel allowed this one to start.
+      // The query latents, and rows the preceding kernel appends, come after the wait.
       int issued = 0;
       bool ok = true;
       bool q_issued = false;
@@ -195,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int u = 0; u < per_tile; ++u) {
           const int pos = i * per_tile + u;
           const int slot = pos % p.nslot, round = pos / p.nslot;
-          if (!q_issued && (pos >= p.ck || round > 0)) {
+          if (!q_issued && (pos >= p.ck || round > 0 || t0 + kTile > p.stable_len)) {
             pdl_wait();
             ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
             for (int sb = 0; sb < p.kb_k; ++sb)
@@ -427,28 +385,9 @@ __global__ void __launch_bounds__(kThreads, 2)
 // host side
 // ---------------------------------------------------------------------------
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
 bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
               const cuuint32_t* box) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return tc::make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, rank, dims, strides, box);
 }
 
 int q_bytes_for(int r_k) { return ((r_k + 63) / 64) * kQSubBytes; }
@@ -473,6 +412,7 @@ void choose_slots(const lr_cache_desc* d, int* nslot, int* ctas_per_sm) {
 }  // namespace
 
 bool tc_supported(const lr_cache_desc* d) {
+  if (d->quant_bits == 4) return tc_i4_supported(d);
   if (d->dtype != LR_BF16 || d->quant_bits != 0 || d->rope_in_kernel) return false;
   if (d->n_q_heads > 32) return false;
   int nslot, cps;
@@ -481,6 +421,7 @@ bool tc_supported(const lr_cache_desc* d) {
 }
 
 int tc_ctas_per_sm(const lr_cache_desc* d) {
+  if (d->quant_bits == 4) return 1;
   int nslot, cps;
   choose_slots(d, &nslot, &cps);
   return cps;
@@ -489,6 +430,7 @@ int tc_ctas_per_sm(const lr_cache_desc* d) {
 cudaError_t tc_prepare(lr_cache* c) {
   const lr_cache_desc& d = c->desc;
   if (!tc_supported(&d)) return cudaSuccess;
+  if (d.quant_bits == 4) return tc_i4_prepare(c);
   TcState* st = reinterpret_cast<TcState*>(c->tc_state);
   if (!st) {
     st = new (std::nothrow) TcState();
@@ -522,12 +464,17 @@ cudaError_t tc_prepare(lr_cache* c) {
 }
 
 void tc_release(lr_cache* c) {
+  if (c->desc.quant_bits == 4) {
+    tc_i4_release(c);
+    return;
+  }
   delete reinterpret_cast<TcState*>(c->tc_state);
   c->tc_state = nullptr;
 }
 
 cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s) {
   const lr_cache_desc& d = c->desc;
+  if (d.quant_bits == 4) return launch_decode_tc_i4(c, n_splits, split_tokens, s);
   const TcState* st = reinterpret_cast<const TcState*>(c->tc_state);
   if (!st) return cudaErrorNotSupported;
   TcParams p;
@@ -539,6 +486,7 @@ cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, 
   p.tmem_cols = (kOCol + p.cv * 32) <= 128 ? 128 : 256;
   p.Hq = d.n_q_heads;
   p.hist_len = c->hist_len;
+  p.stable_len = std::min(c->stable_len, c->hist_len);
   p.split_tokens = split_tokens;
   p.n_splits = n_splits;
   p.nslot = st->nslot;

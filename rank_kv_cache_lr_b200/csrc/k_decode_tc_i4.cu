@@ -1,0 +1,652 @@
+// Tensor-core (tcgen05) split-sequence decode over int4 group-quantised latents.
+//
+// Method: TraceKV abstract (latent KV states stored with quantization, "optimized
+// low-rank attention kernels").  Attention runs in rank space, as in the bf16 kernel:
+//   S[t, j]  = z^_k,t . q~_j            GEMM1: M = 128 tokens, N = 32 heads, K = r_k
+//   p[t, j]  = exp2(S[t, j] - m_j)      online softmax, lazy running max
+//   O~[e, j] += sum_t z^_v,t[e] p[t, j]  GEMM2: M = 128 ranks per chunk, N = 32, K = 128 tokens
+// where z^ = code * scale + zero is expanded in shared memory to fp16 (one rounding of
+// the exact fused product-sum) and q~, p enter the MMAs as fp16 (11 significant bits,
+// so neither needs the hi/lo split of the bf16 kernel).
+//
+// Data flow.  The rows of a 128-token tile are contiguous in the cache, so the producer
+// (warp 0) moves a tile's packed codes and its {scale, zero} words with two plain bulk
+// copies per side into a ring of raw slots.  Six dequantisation warps expand raw tiles
+// into 32 KB operand slots (128 tokens x 128 ranks, fp16, the 128-byte-swizzled
+// K-major layout that GEMM1 reads as A and GEMM2 reads MN-major).  Warp 1 owns TMEM and
+// issues the MMAs from one thread.  Four softmax warps (thread = token row = TMEM lane)
+// turn scores into probabilities and finish with the epilogue (thread = rank row).
+//
+// Pipeline.  Operand slots, raw slots and MMAs all follow the order
+//   K(0), K(1), V(0), K(2), V(1), ..., K(n-1), V(n-2), V(n-1)
+// so GEMM1 of tile s+1 runs while the softmax of tile s is still working: the scores
+// and the probabilities are double-buffered (S in two TMEM column blocks, P in two
+// shared-memory buffers).  When the running max of a head grows by more than 2^8 the
+// softmax first waits for the value mix of the previous tile and rescales O~ in TMEM.
+//
+// Nibble order.  A code word holds elements m = 0..7 of an 8-rank run at bits 4m.  Two
+// masks and one shift give the four fp16 pairs (m0,m4) (m1,m5) (m2,m6) (m3,m7) through
+// the exponent-bias trick (0x6400 | n is 1024 + n; 0x5400 | 16n is 64 + n), so each run
+// sits in shared memory in the order 0,4,1,5,2,6,3,7.  The query latents are stored in
+// the same order (a score is an order-free sum over ranks), and the epilogue maps the
+// rows of O~ back to rank order.
+//
+// Every wait is bounded: on timeout the kernel records LR_ERR_TIMEOUT, drains its own
+// copies and MMAs, frees TMEM and returns.
+#include "tc_common.cuh"
+
+#include <algorithm>
+
+namespace {
+
+using tc::drain_wait;
+using tc::kLazy;
+using tc::kSmemLimit;
+using tc::kTile;
+using tc::kTraceSlots;
+using tc::warp_reduce_scatter32;
+
+constexpr int kThreads = 384;              // 12 warps
+constexpr int kDqThreads = 192;            // warps 2, 3, 8, 9, 10, 11
+constexpr int kSubBytes = 128 * 128;       // 128 tokens x 64 ranks x 2 B
+constexpr int kSlotBytes = 2 * kSubBytes;  // 128 tokens x 128 ranks
+constexpr int kQRows = 32;                 // query heads, padded
+constexpr int kQSubBytes = kQRows * 128;   // 32 rows x 64 ranks x 2 B
+constexpr int kPBytes = 128 * 32 * 2;      // 128 tokens x 32 heads x 2 B
+constexpr int kAuxBytes = 1024;
+constexpr int kSCol = 0;                   // TMEM: S of tile s in columns [32 (s % 2), +32)
+constexpr int kOCol = 64;                  // TMEM: O~ chunk c in columns [64 + 32c, +32)
+constexpr int kMaxSlots = 4;
+constexpr int kMaxRaw = 6;
+
+struct I4Params {
+  const uint32_t* codes_k;
+  const uint32_t* codes_v;
+  const uint32_t* params_k;
+  const uint32_t* params_v;
+  long long cap;
+  int r_k, r_v, G_k, G_v, ck, cv, kb_k, tmem_cols;
+  int Hq, hist_len, stable_len, split_tokens, n_splits, nslot, nraw;
+  uint32_t q_bytes, raw_bytes, raw_codes_bytes;
+  float* part_o;
+  float* part_ml;
+  int* err;
+  unsigned long long* trace;
+};
+
+struct Aux {
+  uint64_t slot_full[kMaxSlots];
+  uint64_t slot_empty[kMaxSlots];
+  uint64_t raw_full[kMaxRaw];
+  uint64_t raw_empty[kMaxRaw];
+  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
+  uint64_t q_full, o_final;
+  uint32_t tmem_base;
+  int abort_flag;
+  float red[4][32];
+  float m_s[32];
+  float alpha_s[32];
+};
+static_assert(sizeof(Aux) <= kAuxBytes, "aux block");
+
+struct I4State {
+  CUtensorMap q;
+  int nslot, nraw;
+  uint32_t raw_bytes, raw_codes_bytes;
+  size_t smem;
+};
+
+__device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
+  return tc::wait_b(bar, parity, &aux->abort_flag, err);
+}
+
+// The k-th unit of the pipeline order: K(k/2 ... ) — unit u is K(tile) or V(tile).
+//   u = 0 -> K(0); u = 2s - 1 -> K(s) for 1 <= s < n; u = 2s -> V(s - 1).  With n tiles
+//   the last unit, u = 2n - 1, is V(n - 1).
+__device__ __forceinline__ void unit_of(int u, int n, int* tile, bool* is_v) {
+  if (u == 0) {
+    *tile = 0;
+    *is_v = false;
+  } else if (u == 2 * n - 1) {
+    *tile = n - 1;
+    *is_v = true;
+  } else if (u & 1) {
+    *tile = (u + 1) >> 1;
+    *is_v = false;
+  } else {
+    *tile = (u >> 1) - 1;
+    *is_v = true;
+  }
+}
+
+// Byte span of the {scale, zero} words of rows [row0, row0 + n) (G words per row),
+// widened to 16-byte boundaries for a bulk copy; `off` is where row0 starts in it.
+__device__ __forceinline__ void param_span(const uint32_t* params, int G, long long row0, int n,
+                                           const uint8_t** src, uint32_t* off, uint32_t* bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(params + row0 * G);
+  const uintptr_t al = a & ~(uintptr_t)15;
+  *src = reinterpret_cast<const uint8_t*>(al);
+  *off = (uint32_t)(a - al);
+  *bytes = (*off + (uint32_t)n * G * 4 + 15u) & ~15u;
+}
+
+// Eight int4 codes of one word -> four fp16 pairs (m0,m4) (m1,m5) (m2,m6) (m3,m7) of
+// code * scale + zero; s2 = (scale, scale), z2 = (zero, zero).
+__device__ __forceinline__ uint4 dequant8(uint32_t w, uint32_t s2, uint32_t z2) {
+  const uint32_t a = (w & 0x000F000Fu) | 0x64006400u;   // 1024 + n
+  const uint32_t b = (w & 0x00F000F0u) | 0x54005400u;   // 64 + n
+  const uint32_t w8 = w >> 8;
+  const uint32_t c = (w8 & 0x000F000Fu) | 0x64006400u;
+  const uint32_t d = (w8 & 0x00F000F0u) | 0x54005400u;
+  uint4 r;
+  asm("{\n\t.reg .b32 t;\n\t"
+      "sub.rn.f16x2 t, %1, %2;\n\t"
+      "fma.rn.f16x2 %0, t, %3, %4;\n\t}"
+      : "=r"(r.x)
+      : "r"(a), "r"(0x64006400u), "r"(s2), "r"(z2));
+  asm("{\n\t.reg .b32 t;\n\t"
+      "sub.rn.f16x2 t, %1, %2;\n\t"
+      "fma.rn.f16x2 %0, t, %3, %4;\n\t}"
+      : "=r"(r.y)
+      : "r"(b), "r"(0x54005400u), "r"(s2), "r"(z2));
+  asm("{\n\t.reg .b32 t;\n\t"
+      "sub.rn.f16x2 t, %1, %2;\n\t"
+      "fma.rn.f16x2 %0, t, %3, %4;\n\t}"
+      : "=r"(r.z)
+      : "r"(c), "r"(0x64006400u), "r"(s2), "r"(z2));
+  asm("{\n\t.reg .b32 t;\n\t"
+      "sub.rn.f16x2 t, %1, %2;\n\t"
+      "fma.rn.f16x2 %0, t, %3, %4;\n\t}"
+      : "=r"(r.w)
+      : "r"(d), "r"(0x54005400u), "r"(s2), "r"(z2));
+  return r;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Shared memory: [aux 1 KB][q~ per 64-rank sub-block][operand ring nslot x 32 KB]
+//                [P double buffer 2 x 8 KB][raw ring nraw x raw_bytes]
+__global__ void __launch_bounds__(kThreads, 1)
+    k_decode_tc_i4(const __grid_constant__ CUtensorMap tm_q, const I4Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (ptx::smem_u32(smem_raw) & 1023) {
+    if (threadIdx.x == 0) atomicExch(p.err, (int)LR_ERR_UNSUPPORTED);
+    return;
+  }
+  Aux* aux = reinterpret_cast<Aux*>(smem_raw);
+  uint8_t* q_s = smem_raw + kAuxBytes;
+  uint8_t* ring = q_s + p.q_bytes;
+  uint8_t* p_s = ring + p.nslot * kSlotBytes;
+  uint8_t* raw = p_s + 2 * kPBytes;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, b = blockIdx.y;
+  const int tok_begin = split * p.split_tokens;
+  const int tok_end = min(p.hist_len, tok_begin + p.split_tokens);
+  const int ntiles = tok_end > tok_begin ? (tok_end - tok_begin + kTile - 1) / kTile : 0;
+  const int nunits = 2 * ntiles;
+
+  if (threadIdx.x == 0) {
+    tc::trace_stamp(p.trace, 0);
+    for (int s = 0; s < p.nslot; ++s) {
+      ptx::mbar_init(&aux->slot_full[s], kDqThreads);
+      ptx::mbar_init(&aux->slot_empty[s], 1);
+    }
+    for (int s = 0; s < p.nraw; ++s) {
+      ptx::mbar_init(&aux->raw_full[s], 1);
+      ptx::mbar_init(&aux->raw_empty[s], kDqThreads);
+    }
+    for (int k = 0; k < 2; ++k) {
+      ptx::mbar_init(&aux->s_full[k], 1);
+      ptx::mbar_init(&aux->s_empty[k], 128);
+      ptx::mbar_init(&aux->p_full[k], 128);
+      ptx::mbar_init(&aux->p_empty[k], 1);
+    }
+    ptx::mbar_init(&aux->q_full, 1);
+    ptx::mbar_init(&aux->o_final, 1);
+    aux->abort_flag = 0;
+    for (int j = 0; j < 32; ++j) aux->m_s[j] = -INFINITY;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) ptx::prefetch_tmap(&tm_q);
+  if (warp == 1) {
+    ptx::tmem_alloc(&aux->tmem_base, p.tmem_cols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = aux->tmem_base;
+  // Only the producer reads memory that the preceding kernel writes (the query latents,
+  // rows at or above stable_len); it waits for that kernel before those copies.  Every
+  // other thread works on shared memory and TMEM behind the producer's barriers, and
+  // the epilogue's writes follow the query latents' arrival.
+  pdl_trigger();
+  if (threadIdx.x == 32) tc::trace_stamp(p.trace, 1);
+
+  const bool is_dq = warp == 2 || warp == 3 || warp >= 8;
+  if (warp == 0) {
+    // ------------------------------------------------------------- bulk-copy producer
+    if (lane == 0 && ntiles > 0) {
+      bool waited = false, ok = true;
+      int issued = 0;
+      for (int u = 0; u < nunits && ok; ++u) {
+        int tile;
+        bool is_v;
+        unit_of(u, ntiles, &tile, &is_v);
+        const int t0 = tok_begin + tile * kTile;
+        const int n = min(kTile, tok_end - t0);
+        const int rs = u % p.nraw, round = u / p.nraw;
+        if (!waited && (round > 0 || t0 + n > p.stable_len)) {
+          pdl_wait();
+          ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
+          for (int sb = 0; sb < p.kb_k; ++sb)
+            ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
+          waited = true;
+        }
+        if (round > 0 && !(ok = wait_b(&aux->raw_empty[rs], (round - 1) & 1, aux, p.err))) break;
+        const int G = is_v ? p.G_v : p.G_k;
+        const long long row0 = (long long)b * p.cap + t0;
+        const uint32_t* codes = is_v ? p.codes_v : p.codes_k;
+        const uint8_t* psrc;
+        uint32_t poff, pbytes;
+        param_span(is_v ? p.params_v : p.params_k, G, row0, n, &psrc, &poff, &pbytes);
+        const uint32_t cbytes = (uint32_t)n * G * 16;
+        uint8_t* dst = raw + rs * p.raw_bytes;
+        ptx::mbar_arrive_expect_tx(&aux->raw_full[rs], cbytes + pbytes);
+        ptx::bulk_load(dst, codes + row0 * G * 4, cbytes, &aux->raw_full[rs]);
+        ptx::bulk_load(dst + p.raw_codes_bytes, psrc, pbytes, &aux->raw_full[rs]);
+        issued = u + 1;
+      }
+      if (!waited) {
+        pdl_wait();
+        ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
+        for (int sb = 0; sb < p.kb_k; ++sb)
+          ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
+      }
+      if (!ok) {
+        drain_wait(&aux->q_full, 0);
+        for (int u = max(0, issued - p.nraw); u < issued; ++u)
+          drain_wait(&aux->raw_full[u % p.nraw], (u / p.nraw) & 1);
+      }
+    }
+  } else if (is_dq) {
+    // ------------------------------------------------------------- dequantisation
+    if (ntiles > 0) {
+      const int dq = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;
+      const uint32_t ring_addr = ptx::smem_u32(ring);
+      bool ok = true;
+      int pos = 0;   // operand-slot sequence number
+      for (int u = 0; u < nunits && ok; ++u) {
+        int tile;
+        bool is_v;
+        unit_of(u, ntiles, &tile, &is_v);
+        const int t0 = tok_begin + tile * kTile;
+        const int n = min(kTile, tok_end - t0);
+        const int rs = u % p.nraw;
+        if (!(ok = wait_b(&aux->raw_full[rs], (u / p.nraw) & 1, aux, p.err))) break;
+        const int G = is_v ? p.G_v : p.G_k;
+        const long long row0 = (long long)b * p.cap + t0;
+        const uint8_t* rb = raw + rs * p.raw_bytes;
+        const uint32_t poff =
+            (uint32_t)(reinterpret_cast<uintptr_t>((is_v ? p.params_v : p.params_k) + row0 * G) & 15u);
+        const uint4* cw = reinterpret_cast<const uint4*>(rb);
+        const uint32_t* pw = reinterpret_cast<const uint32_t*>(rb + p.raw_codes_bytes + poff);
+        const int nch = is_v ? p.cv : p.ck;
+        for (int c = 0; c < nch && ok; ++c, ++pos) {
+          const int slot = pos % p.nslot, round = pos / p.nslot;
+          if (round > 0 && !(ok = wait_b(&aux->slot_empty[slot], (round - 1) & 1, aux, p.err))) break;
+          const uint32_t dst = ring_addr + slot * kSlotBytes;
+          // unit = (token t, group lg of the chunk): four words -> four 16-byte chunks of
+          // row t.  Lanes of a quarter-warp cover 2 tokens x 4 groups; rotating the word
+          // order of groups 2, 3 by two chunks makes each store conflict-free.
+          for (int v = dq; v < kTile * 4; v += kDqThreads) {
+            const int t = v >> 2, lg = v & 3, g = c * 4 + lg;
+            if (g >= G) continue;
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            uint32_t s2 = 0u, z2 = 0u;
+            if (t < n) {
+              w = cw[t * G + g];
+              const uint32_t prm = pw[t * G + g];
+              s2 = __byte_perm(prm, 0u, 0x1010);
+              z2 = __byte_perm(prm, 0u, 0x3232);
+            }
+            const int rot = lg & 2;
+            if (rot) {
+              const uint32_t x0 = w.x, x1 = w.y;
+              w.x = w.z;
+              w.y = w.w;
+              w.z = x0;
+              w.w = x1;
+            }
+            const uint32_t rowa = dst + (lg >> 1) * kSubBytes + t * 128;
+            const int cb = (lg & 1) * 4, sw = t & 7;
+            sts128(rowa + (((cb + (0 ^ rot)) ^ sw) << 4), dequant8(w.x, s2, z2));
+            sts128(rowa + (((cb + (1 ^ rot)) ^ sw) << 4), dequant8(w.y, s2, z2));
+            sts128(rowa + (((cb + (2 ^ rot)) ^ sw) << 4), dequant8(w.z, s2, z2));
+            sts128(rowa + (((cb + (3 ^ rot)) ^ sw) << 4), dequant8(w.w, s2, z2));
+          }
+          ptx::fence_proxy_async_smem();
+          ptx::mbar_arrive(&aux->slot_full[slot]);
+        }
+        if (ok) ptx::mbar_arrive(&aux->raw_empty[rs]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0 && ntiles > 0) {
+      const uint32_t id = ptx::idesc_f16(0, 0, 0, 128, 32);    // GEMM1: fp16, K-major x K-major
+      const uint32_t id2 = ptx::idesc_f16(0, 1, 1, 128, 32);   // GEMM2: fp16, MN-major x MN-major
+      const uint32_t q_addr = ptx::smem_u32(q_s), ring_addr = ptx::smem_u32(ring), p_addr = ptx::smem_u32(p_s);
+      bool ok = wait_b(&aux->q_full, 0, aux, p.err);
+      ptx::tc_fence_after();
+      tc::trace_stamp(p.trace, 2);
+      int pos = 0;
+      for (int u = 0; u < nunits && ok; ++u) {
+        int tile;
+        bool is_v;
+        unit_of(u, ntiles, &tile, &is_v);
+        if (!is_v) {
+          // GEMM1(tile): S[tile % 2] = Z_k q~^T
+          const int sb2 = tile & 1;
+          if (tile >= 2 && !(ok = wait_b(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
+          ptx::tc_fence_after();
+          for (int c = 0; c < p.ck && ok; ++c, ++pos) {
+            const int slot = pos % p.nslot;
+            if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+            ptx::tc_fence_after();
+            const uint32_t sa = ring_addr + slot * kSlotBytes;
+#pragma unroll
+            for (int sb = 0; sb < 2; ++sb) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const int k0 = c * 128 + sb * 64 + kk * 16;
+                if (k0 < p.r_k) {
+                  const uint64_t ad = ptx::smem_desc(sa + sb * kSubBytes + kk * 32, 16, 1024, 2);
+                  const uint64_t bd = ptx::smem_desc(q_addr + (c * 2 + sb) * kQSubBytes + kk * 32, 16, 1024, 2);
+                  ptx::mma_f16(tmem + kSCol + 32 * sb2, ad, bd, id, k0 > 0 ? 1u : 0u);
+                }
+              }
+            }
+            ptx::mma_commit(&aux->slot_empty[slot]);
+          }
+          if (!ok) break;
+          ptx::mma_commit(&aux->s_full[sb2]);
+          if (tile < 16) tc::trace_stamp(p.trace, 3 + 4 * tile);
+        } else {
+          // GEMM2(tile): O~ += Z_v^T P[tile % 2]
+          const int pb2 = tile & 1;
+          if (!(ok = wait_b(&aux->p_full[pb2], (tile >> 1) & 1, aux, p.err))) break;
+          ptx::tc_fence_after();
+          for (int c = 0; c < p.cv && ok; ++c, ++pos) {
+            const int slot = pos % p.nslot;
+            if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+            ptx::tc_fence_after();
+            const uint32_t sa = ring_addr + slot * kSlotBytes;
+#pragma unroll
+            for (int kt = 0; kt < 8; ++kt) {
+              const uint64_t ad = ptx::smem_desc(sa + kt * 2048, kSubBytes, 1024, 2);
+              const uint64_t bd = ptx::smem_desc(p_addr + pb2 * kPBytes + kt * 256, 128, 2048, 0);
+              ptx::mma_f16(tmem + kOCol + c * 32, ad, bd, id2, (tile > 0 || kt > 0) ? 1u : 0u);
+            }
+            ptx::mma_commit(&aux->slot_empty[slot]);
+          }
+          if (!ok) break;
+          ptx::mma_commit(&aux->p_empty[pb2]);
+          if (tile < 16) tc::trace_stamp(p.trace, 6 + 4 * tile);
+        }
+      }
+      ptx::mma_commit(&aux->o_final);
+      if (!ok) drain_wait(&aux->o_final, 0);
+    }
+    __syncwarp();
+  } else if (ntiles > 0) {
+    // ------------------------------------------------------------- softmax / epilogue
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    float l[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) l[j] = 0.f;
+    bool ok = true;
+    for (int i = 0; i < ntiles; ++i) {
+      const int k2 = i & 1;
+      const bool valid = tok_begin + i * kTile + row < tok_end;
+      ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full[k2], (i >> 1) & 1, aux, p.err));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 4 + 4 * i);
+      const uint32_t s_col = tmem + lane_off + kSCol + 32 * k2;
+      uint32_t sv[32];
+      ptx::tmem_ld32(s_col, sv);
+      ptx::tmem_wait_ld();
+      float s[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+
+      bool ex = false;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ex |= s[j] > aux->m_s[j] + kLazy;
+      ex = ptx::named_bar_or(1, 128, ex);
+      if (ex) {
+        // the value mix of the previous tile must be complete before O~ is rescaled
+        if (i >= 1) {
+          ok = ptx::named_bar_and(1, 128, wait_b(&aux->p_empty[(i - 1) & 1], ((i - 1) >> 1) & 1, aux, p.err));
+          if (!ok) break;
+          ptx::tc_fence_after();
+        }
+        aux->red[qd][lane] = warp_reduce_scatter32<true>(s, lane);
+        ptx::tmem_ld32(s_col, sv);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+        ptx::named_bar_sync(1, 128);
+        if (qd == 0) {
+          const float mt =
+              fmaxf(fmaxf(aux->red[0][lane], aux->red[1][lane]), fmaxf(aux->red[2][lane], aux->red[3][lane]));
+          const float mo = aux->m_s[lane];
+          const float mn = fmaxf(mo, mt);
+          aux->alpha_s[lane] = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+          aux->m_s[lane] = mn;
+        }
+        ptx::named_bar_sync(1, 128);
+        bool need_o = false;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float a = aux->alpha_s[j];
+          l[j] *= a;
+          need_o |= a < 1.f;
+        }
+        if (need_o && i > 0) {
+          for (int c = 0; c < p.cv; ++c) {
+            uint32_t v2[32];
+            ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v2[j] = __float_as_uint(__uint_as_float(v2[j]) * aux->alpha_s[j]);
+            ptx::tmem_st32(tmem + lane_off + kOCol + c * 32, v2);
+          }
+          ptx::tmem_wait_st();
+        }
+      }
+      // P[i % 2] is free once the value mix of tile i - 2 has completed
+      if (i >= 2) {
+        ok = ptx::named_bar_and(1, 128, wait_b(&aux->p_empty[k2], ((i - 2) >> 1) & 1, aux, p.err));
+        if (!ok) break;
+      }
+      // probabilities as fp16; l sums the rounded values the MMA uses
+      const uint32_t prow = ptx::smem_u32(p_s + k2 * kPBytes + row * 16);
+#pragma unroll
+      for (int hg = 0; hg < 4; ++hg) {
+        uint32_t hw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = hg * 8 + 2 * e;
+          const __half2 h = __floats2half2_rn(exp2f(s[j] - aux->m_s[j]), exp2f(s[j + 1] - aux->m_s[j + 1]));
+          const float2 f = __half22float2(h);
+          l[j] += f.x;
+          l[j + 1] += f.y;
+          hw[e] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + hg * 2048), "r"(hw[0]), "r"(hw[1]),
+                     "r"(hw[2]), "r"(hw[3])
+                     : "memory");
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&aux->s_empty[k2]);
+      ptx::mbar_arrive(&aux->p_full[k2]);
+      if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 5 + 4 * i);
+    }
+    if (ok) ok = ptx::named_bar_and(1, 128, wait_b(&aux->o_final, 0, aux, p.err));
+    if (ok) {
+      ptx::tc_fence_after();
+      const size_t base_out = ((size_t)b * p.n_splits + split) * p.Hq;
+      // TMEM row m of a chunk holds rank 8 (m / 8) + perm(m % 8), perm = 0,4,1,5,2,6,3,7
+      const int m = qd * 32 + lane;
+      const int e_in = (m & ~7) + ((m & 7) >> 1) + ((m & 1) << 2);
+      for (int c = 0; c < p.cv; ++c) {
+        uint32_t v2[32];
+        ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
+        ptx::tmem_wait_ld();
+        const int e = c * 128 + e_in;
+        if (e < p.r_v) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < p.Hq) p.part_o[(base_out + j) * p.r_v + e] = __uint_as_float(v2[j]);
+        }
+      }
+      aux->red[qd][lane] = warp_reduce_scatter32<false>(l, lane);
+      ptx::named_bar_sync(1, 128);
+      if (qd == 0 && lane < p.Hq) {
+        const float lt = (aux->red[0][lane] + aux->red[1][lane]) + (aux->red[2][lane] + aux->red[3][lane]);
+        p.part_ml[(base_out + lane) * 2] = aux->m_s[lane];
+        p.part_ml[(base_out + lane) * 2 + 1] = lt;
+      }
+      if (threadIdx.x == 128) tc::trace_stamp(p.trace, kTraceSlots - 1);
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+int groups(int r) { return (r + 31) / 32; }
+int q_bytes_for(int r_k) { return ((r_k + 63) / 64) * kQSubBytes; }
+
+struct I4Layout {
+  int nslot, nraw;
+  uint32_t raw_bytes, raw_codes_bytes;
+  size_t smem;
+};
+
+// As many operand slots (up to 4) as leave room for two raw slots, then as many raw
+// slots (up to 6) as fit in 227 KB.
+bool choose_layout(const lr_cache_desc* d, I4Layout* L) {
+  const int G = std::max(groups(d->rank_k), groups(d->rank_v));
+  L->raw_codes_bytes = (uint32_t)kTile * G * 16;
+  L->raw_bytes = ((uint32_t)kTile * G * 20 + 16 + 127) & ~127u;
+  const size_t fixed = (size_t)kAuxBytes + q_bytes_for(d->rank_k) + 2 * kPBytes;
+  int ns = kMaxSlots;
+  while (ns >= 2 && fixed + (size_t)ns * kSlotBytes + 2 * (size_t)L->raw_bytes > (size_t)kSmemLimit) --ns;
+  if (ns < 2) return false;
+  int nr = (int)(((size_t)kSmemLimit - fixed - (size_t)ns * kSlotBytes) / L->raw_bytes);
+  nr = std::min(nr, kMaxRaw);
+  L->nslot = ns;
+  L->nraw = nr;
+  L->smem = fixed + (size_t)ns * kSlotBytes + (size_t)nr * L->raw_bytes;
+  return true;
+}
+
+}  // namespace
+
+bool tc_i4_supported(const lr_cache_desc* d) {
+  if (d->quant_bits != 4 || d->quant_group != 32) return false;
+  if (d->dtype != LR_BF16 || d->rope_in_kernel) return false;
+  if (d->n_q_heads > 32 || d->rank_v > 512) return false;
+  I4Layout L;
+  return choose_layout(d, &L);
+}
+
+cudaError_t tc_i4_prepare(lr_cache* c) {
+  const lr_cache_desc& d = c->desc;
+  I4State* st = reinterpret_cast<I4State*>(c->tc_state);
+  if (!st) {
+    st = new (std::nothrow) I4State();
+    if (!st) return cudaErrorMemoryAllocation;
+    c->tc_state = st;
+  }
+  const size_t qbytes = (size_t)d.batch * kQRows * d.rank_k * 2;
+  if (!c->qt16) {
+    cudaError_t e = cudaMalloc(&c->qt16, qbytes);
+    if (e != cudaSuccess) return e;
+    e = cudaMemset(c->qt16, 0, qbytes);
+    if (e != cudaSuccess) return e;
+  }
+  cuuint64_t dims[2] = {(cuuint64_t)d.rank_k, (cuuint64_t)d.batch * kQRows};
+  cuuint64_t strides[1] = {(cuuint64_t)d.rank_k * 2};
+  cuuint32_t box[2] = {64, kQRows};
+  if (!tc::make_map(&st->q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, c->qt16, 2, dims, strides, box))
+    return cudaErrorInvalidValue;
+  I4Layout L;
+  if (!choose_layout(&d, &L)) return cudaErrorNotSupported;
+  st->nslot = L.nslot;
+  st->nraw = L.nraw;
+  st->raw_bytes = L.raw_bytes;
+  st->raw_codes_bytes = L.raw_codes_bytes;
+  st->smem = L.smem;
+  return cudaSuccess;
+}
+
+void tc_i4_release(lr_cache* c) {
+  delete reinterpret_cast<I4State*>(c->tc_state);
+  c->tc_state = nullptr;
+}
+
+cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  const I4State* st = reinterpret_cast<const I4State*>(c->tc_state);
+  if (!st) return cudaErrorNotSupported;
+  I4Params p;
+  p.codes_k = c->codes_k;
+  p.codes_v = c->codes_v;
+  p.params_k = c->params_k;
+  p.params_v = c->params_v;
+  p.cap = d.capacity;
+  p.r_k = d.rank_k;
+  p.r_v = d.rank_v;
+  p.G_k = c->G_k;
+  p.G_v = c->G_v;
+  p.ck = (d.rank_k + 127) / 128;
+  p.cv = (d.rank_v + 127) / 128;
+  p.kb_k = (d.rank_k + 63) / 64;
+  p.tmem_cols = (kOCol + p.cv * 32) <= 128 ? 128 : 256;
+  p.Hq = d.n_q_heads;
+  p.hist_len = c->hist_len;
+  p.stable_len = std::min(c->stable_len, c->hist_len);
+  p.split_tokens = split_tokens;
+  p.n_splits = n_splits;
+  p.nslot = st->nslot;
+  p.nraw = st->nraw;
+  p.q_bytes = q_bytes_for(d.rank_k);
+  p.raw_bytes = st->raw_bytes;
+  p.raw_codes_bytes = st->raw_codes_bytes;
+  p.part_o = c->part_o;
+  p.part_ml = c->part_ml;
+  p.err = c->dev_err;
+  p.trace = c->trace;
+  static std::atomic<uint32_t> optin_done{0};
+  cudaError_t e = smem_optin(k_decode_tc_i4, optin_done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_decode_tc_i4, dim3(n_splits, d.batch), dim3(kThreads), st->smem, s, st->q, p);
+}

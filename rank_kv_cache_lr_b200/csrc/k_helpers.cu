@@ -58,13 +58,16 @@ struct El<float> {
 // ---- query projection -----------------------------------------------------------
 // One CTA per (128 rank rows of B_k,h, KV head h, sequence b); thread = rank row i,
 // for every query head j of the group: q~_j[i] = s log2(e) sum_c B_k[i][h d + c] q_j[c].
-// qt16 (tensor-core path): rows [b][j] and [b][32 + j] of a [B][64][r_k] bf16 array get
-// hi = bf16(q~) and lo = bf16(q~ - hi), so that hi + lo carries q~ to ~16 significant bits.
+// qt16 (tensor-core path), bf16 latents: rows [b][j] and [b][32 + j] of a [B][64][r_k]
+// bf16 array get hi = bf16(q~) and lo = bf16(q~ - hi), so that hi + lo carries q~ to ~16
+// significant bits.  int4 latents: row [b][j] of a [B][32][r_k] fp16 array gets fp16(q~),
+// each 8-rank run in the order 0,4,1,5,2,6,3,7 in which the int4 kernel expands codes.
 constexpr int kQRowsCta = 128;
 constexpr int kHB = 8;            // query heads per register block
 
 struct QprojArgs {
-  const void* q; const void* Bk; float* qt; float* qd; __nv_bfloat16* qt16;
+  const void* q; const void* Bk; float* qt; float* qd; void* qt16;
+  int qt16_fp16;          // 1: fp16 rows in int4 run order; 0: bf16 hi / lo rows
   int Hq, Hkv, d, D, rk;
   float scale_log2;
   int want_latent;
@@ -130,11 +133,15 @@ __device__ __forceinline__ void qproj_main(const QprojArgs& a, int rchunk, int h
           const int j = j0 + jb + u;
           const float v = acc[u] * a.scale_log2;
           a.qt[((size_t)b * a.Hq + j) * a.rk + i] = v;
-          if (a.qt16) {
+          if (a.qt16 && a.qt16_fp16) {
+            const int pos = (i & ~7) | ((i & 3) << 1) | ((i >> 2) & 1);
+            reinterpret_cast<__half*>(a.qt16)[((size_t)b * 32 + j) * a.rk + pos] = __float2half_rn(v);
+          } else if (a.qt16) {
             const __nv_bfloat16 hi = __float2bfloat16_rn(v);
             const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-            a.qt16[((size_t)b * 64 + j) * a.rk + i] = hi;
-            a.qt16[((size_t)b * 64 + 32 + j) * a.rk + i] = lo;
+            __nv_bfloat16* q16 = reinterpret_cast<__nv_bfloat16*>(a.qt16);
+            q16[((size_t)b * 64 + j) * a.rk + i] = hi;
+            q16[((size_t)b * 64 + 32 + j) * a.rk + i] = lo;
           }
         }
       }
@@ -383,7 +390,8 @@ QprojArgs make_qproj_args(const lr_cache* c, const void* q, bool tc) {
   a.Bk = c->B_k;
   a.qt = c->qt;
   a.qd = (rope || c->win_slots) ? (rope ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k) : nullptr;
-  a.qt16 = tc ? (__nv_bfloat16*)c->qt16 : nullptr;
+  a.qt16 = tc ? c->qt16 : nullptr;
+  a.qt16_fp16 = c->latent_kind == LK_INT4 ? 1 : 0;
   a.Hq = d.n_q_heads; a.Hkv = d.n_kv_heads; a.d = d.head_dim; a.D = c->D; a.rk = d.rank_k;
   a.scale_log2 = c->scale_log2;
   a.want_latent = rope ? 0 : 1;

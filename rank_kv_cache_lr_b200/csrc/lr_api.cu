@@ -173,8 +173,10 @@ lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void
     if (c->latent_kind == LK_INT4) {
       e = dalloc(&c->codes_k, B * cap * c->G_k * 4 * sizeof(uint32_t));
       if (e == cudaSuccess) e = dalloc(&c->codes_v, B * cap * c->G_v * 4 * sizeof(uint32_t));
-      if (e == cudaSuccess) e = dalloc(&c->params_k, B * cap * c->G_k * sizeof(uint32_t));
-      if (e == cudaSuccess) e = dalloc(&c->params_v, B * cap * c->G_v * sizeof(uint32_t));
+      // params get 64 bytes of tail padding: the tensor-core decode copies 16-byte
+      // aligned spans that may reach up to 15 bytes past the last row
+      if (e == cudaSuccess) e = dalloc(&c->params_k, B * cap * c->G_k * sizeof(uint32_t) + 64);
+      if (e == cudaSuccess) e = dalloc(&c->params_v, B * cap * c->G_v * sizeof(uint32_t) + 64);
     } else {
       e = dalloc(&c->z_k, B * cap * d.rank_k * es);
       if (e == cudaSuccess) e = dalloc(&c->z_v, B * cap * d.rank_v * es);
@@ -312,6 +314,7 @@ lr_status lr_attn_decode(lr_cache* c, const void* q, void* out, float* lse, void
   if (st != LR_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
+  c->stable_len = c->hist_len;
   cudaError_t e = p.path == LR_PATH_TC ? launch_qproj_tc(c, q, s) : launch_qproj(c, q, s);
   if (e == cudaSuccess) e = decode_rest(c, p, out, lse, s);
   return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
@@ -336,6 +339,7 @@ lr_status lr_decode_step(lr_cache* c, const void* k, const void* v, const void* 
   c->last_stream = s;
   cudaError_t e = launch_step_pre(c, k, v, q, p.path == LR_PATH_TC, s);   // uses the pre-append counters
   if (e != cudaSuccess) return LR_ERR_CUDA;
+  c->stable_len = c->hist_len;   // the row the append writes (new token or fold) is not stable
   c->hist_len = hist1;
   c->win_len = win1;
   ++c->len;

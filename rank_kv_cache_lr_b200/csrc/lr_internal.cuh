@@ -23,6 +23,9 @@ struct lr_cache {
   int G_k, G_v;          // int4 groups per token (0 when unquantised)
   int win_slots;         // window + 1 (ring), or 0
   int32_t len, hist_len, win_len;
+  int32_t stable_len = 0; // history rows [0, stable_len) were written before the kernel that
+                          // precedes the decode (the decode may read them before its
+                          // grid-dependency wait); set by each decode entry point
   float scale_log2;      // softmax_scale * log2(e)
   int latent_kind;       // LatentKind
   size_t esize;          // bytes per dtype element
@@ -98,6 +101,11 @@ cudaError_t tc_prepare(lr_cache* c);
 void tc_release(lr_cache* c);
 cudaError_t launch_qproj_tc(const lr_cache* c, const void* q, cudaStream_t s);
 cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s);
+// int4 latents on tensor cores (k_decode_tc_i4.cu)
+bool tc_i4_supported(const lr_cache_desc* d);
+cudaError_t tc_i4_prepare(lr_cache* c);
+void tc_i4_release(lr_cache* c);
+cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s);
 
 void lr_count_launch(int n = 1);
 

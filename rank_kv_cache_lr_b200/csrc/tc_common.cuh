@@ -1,0 +1,99 @@
+// Pieces shared by the tensor-core decode kernels (bf16 latents and int4 latents):
+// bounded mbarrier waits with a per-CTA abort flag, the warp butterfly reduce-scatter,
+// the optional per-CTA timeline, and the host-side tensor-map encoder.
+#pragma once
+
+#include "lr_internal.cuh"
+#include "ptx.cuh"
+
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+namespace tc {
+
+constexpr int kTile = 128;                 // tokens per tile (the MMA's M for the scores)
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kSmemLimit = 232448;         // 227 KB opt-in per block
+constexpr int kTraceSlots = LR_TRACE_SLOTS; // 0 start, 1 setup done, 2 query latents in,
+                                           // 3+4i: key tile i consumed, 4+4i: scores of tile i read,
+                                           // 5+4i: probabilities of tile i written,
+                                           // 6+4i: value mix of tile i issued (i < 16), last: end
+constexpr float kLazy = 8.0f;              // log2 of the allowed running-max growth before a rescale
+
+// Wait for phase `parity` of `bar`.  Gives up when another thread of the CTA has
+// aborted, or after kTimeoutNs, in which case it records LR_ERR_TIMEOUT in the device
+// error word and raises the CTA's abort flag.  Returns false when it gave up.
+__device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, int* abort_flag, int* err) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((it & 31) == 0) {
+      if (*(volatile int*)abort_flag) return false;
+      if (ptx::globaltimer() - t0 > kTimeoutNs) {
+        *(volatile int*)abort_flag = 1;
+        atomicExch(err, (int)LR_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Wait that ignores the abort flag (used to drain in-flight copies and MMAs after an
+// abort); still bounded.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait(bar, parity))
+    if (ptx::globaltimer() - t0 > kTimeoutNs) return;
+}
+
+__device__ __forceinline__ void trace_stamp(unsigned long long* trace, int slot) {
+  if (trace) trace[((size_t)blockIdx.y * gridDim.x + blockIdx.x) * kTraceSlots + slot] = ptx::globaltimer();
+}
+
+// Butterfly reduce-scatter over a warp: on return lane l holds op over all lanes of
+// v[l] (v is destroyed).
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool up = (lane & w) != 0;
+#pragma unroll
+    for (int k = 0; k < w; ++k) {
+      const float keep = up ? v[k + w] : v[k];
+      const float send = up ? v[k] : v[k + w];
+      const float got = __shfl_xor_sync(0xffffffffu, send, w);
+      v[k] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return v[0];
+}
+
+// ---- host ------------------------------------------------------------------------
+
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// A tiled map with 128-byte swizzle over 16-bit elements.
+inline bool make_map(CUtensorMap* m, CUtensorMapDataType type, const void* ptr, int rank, const cuuint64_t* dims,
+                     const cuuint64_t* strides, const cuuint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, type, rank, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace tc
