@@ -83,9 +83,15 @@ typedef struct lr_cache_desc {
 typedef struct lr_cache lr_cache;   /* opaque */
 
 /* Device pointers and strides of the cache's storage, for inspection.
- * Int4 latents: codes [B][capacity][groups*4] uint32 (element e of group g in
- * word 4g + e/8, bits 4(e%8)..+3), params [B][capacity][groups] as a pair of
- * fp16 {scale (low half), zero (high half)} in one 32-bit word.
+ * Int4 latents are stored in blocks of 128 tokens, group-major inside a block, so that
+ * one group of one block (128 tokens) is a contiguous 2 KB run of codes and a 512-byte
+ * run of params:
+ *   codes  [B][int4_blocks][groups][128][4] uint32: element e of group g of token t
+ *          of sequence b is in word ((b*int4_blocks + t/128)*groups + g)*512
+ *          + (t%128)*4 + e/8, bits 4(e%8)..+3;
+ *   params [B][int4_blocks][groups][128] uint32: ((b*int4_blocks + t/128)*groups + g)*128
+ *          + t%128, a pair of fp16 {scale (low half), zero (high half)};
+ * with int4_blocks = ceil(capacity / 128).
  * Unquantised latents: z [B][capacity][rank] in dtype.
  * Window ring: [B][window+1][D] in dtype; token t lives in slot t % (window+1). */
 typedef struct lr_cache_view {
@@ -96,6 +102,8 @@ typedef struct lr_cache_view {
   void* A_k; void* B_k; void* A_v; void* B_v;   /* current bases (dtype)         */
   int32_t groups_k, groups_v;           /* ceil(rank/32) for int4 caches, else 0 */
   int32_t capacity, window_slots;
+  int32_t int4_blocks;                  /* 128-token blocks per sequence (int4), else 0 */
+  int32_t reserved;
 } lr_cache_view;
 
 /* Decode plan (host arithmetic only; exposed for tests and tooling). */

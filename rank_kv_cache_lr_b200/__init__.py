@@ -45,7 +45,8 @@ class lr_cache_view(ctypes.Structure):
                 ("A_k", ctypes.c_void_p), ("B_k", ctypes.c_void_p),
                 ("A_v", ctypes.c_void_p), ("B_v", ctypes.c_void_p),
                 ("groups_k", ctypes.c_int32), ("groups_v", ctypes.c_int32),
-                ("capacity", ctypes.c_int32), ("window_slots", ctypes.c_int32)]
+                ("capacity", ctypes.c_int32), ("window_slots", ctypes.c_int32),
+                ("int4_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class lr_plan(ctypes.Structure):

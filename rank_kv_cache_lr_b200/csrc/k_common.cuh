@@ -22,9 +22,9 @@ __device__ __forceinline__ void store_elem(void* p, long long idx, float v, int 
 __device__ __forceinline__ float latent_f(const LatentRef& L, int kind, int dtype,
                                           long long row, int i) {
   if (kind == LK_INT4) {
-    const uint32_t w = L.codes[row * (L.G * 4) + (i >> 3)];
+    const uint32_t w = L.codes[i4_code_index(row, L.G, i >> 5, (i >> 3) & 3)];
     const float code = (float)((w >> (4 * (i & 7))) & 15u);
-    const uint32_t p = L.params[row * L.G + (i >> 5)];
+    const uint32_t p = L.params[i4_param_index(row, L.G, i >> 5)];
     const float scale = __half2float(__ushort_as_half((unsigned short)(p & 0xFFFFu)));
     const float zero = __half2float(__ushort_as_half((unsigned short)(p >> 16)));
     return fmaf(code, scale, zero);
@@ -73,7 +73,7 @@ __device__ __forceinline__ void store_latent_chunk(float z, int ch, int r, int k
   const int i = ch * 32 + lane;
   const bool valid = i < r;
   if (kind == LK_INT4) {
-    quant_group_warp(z, valid, codes + row * (G * 4) + ch * 4, params + row * G + ch);
+    quant_group_warp(z, valid, codes + i4_code_index(row, G, ch, 0), params + i4_param_index(row, G, ch));
   } else if (valid) {
     store_elem(Z, row * r + i, z, dtype);
   }

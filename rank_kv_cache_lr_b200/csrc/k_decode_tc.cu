@@ -193,7 +193,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0 && ntiles > 0) {
       const uint32_t id = ptx::idesc_f16(1, 0, 0, 128, 32);    // GEMM1: K-major x K-major, N = 32
       const uint32_t id2 = ptx::idesc_f16(1, 1, 1, 128, 32);   // GEMM2: MN-major x MN-major, N = 32
-      const uint32_t q_addr = ptx::smem_u32(q_s), ring_addr = ptx::smem_u32(ring), p_addr = ptx::smem_u32(p_s);
+      // Descriptors are built once; a step along K or to another slot adds its byte
+      // offset >> 4 to the start-address field (no carry: shared memory < 256 KB).
+      const uint64_t kdesc0 = ptx::smem_desc(ptx::smem_u32(ring), 16, 1024, 2);
+      const uint64_t qdesc0 = ptx::smem_desc(ptx::smem_u32(q_s), 16, 1024, 2);
+      const uint64_t vdesc0 = ptx::smem_desc(ptx::smem_u32(ring), kSubBytes, 1024, 2);
+      const uint64_t pdesc0 = ptx::smem_desc(ptx::smem_u32(p_s), 128, 2048, 0);
       bool ok = wait_b(&aux->q_full, 0, aux, p.err);
       ptx::tc_fence_after();
       trace_stamp(p, 2);
@@ -206,19 +211,14 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int slot = pos % p.nslot;
           if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
           ptx::tc_fence_after();
-          const uint32_t sa = ring_addr + slot * kSlotBytes;
-#pragma unroll
-          for (int sb = 0; sb < 2; ++sb) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const int k0 = c * 128 + sb * 64 + kk * 16;
-              if (k0 < p.r_k) {
-                const uint64_t ad = ptx::smem_desc(sa + sb * kSubBytes + kk * 32, 16, 1024, 2);
-                const uint32_t qb = q_addr + (c * 2 + sb) * kQSubBytes + kk * 32;
-                ptx::mma_f16(tmem + kSCol, ad, ptx::smem_desc(qb, 16, 1024, 2), id, k0 > 0 ? 1u : 0u);
-                ptx::mma_f16(tmem + kSCol, ad, ptx::smem_desc(qb + kQLoOffset, 16, 1024, 2), id, 1u);
-              }
-            }
+          const uint64_t a0 = kdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+          const uint64_t b0 = qdesc0 + (uint64_t)((c * 2 * kQSubBytes) >> 4);
+          const int nk = min(8, (p.r_k - c * 128) >> 4);
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint64_t ad = a0 + (uint64_t)((kk >> 2) * (kSubBytes >> 4) + (kk & 3) * 2);
+            const uint64_t bd = b0 + (uint64_t)((kk >> 2) * (kQSubBytes >> 4) + (kk & 3) * 2);
+            ptx::mma_f16(tmem + kSCol, ad, bd, id, (c | kk) ? 1u : 0u);
+            ptx::mma_f16(tmem + kSCol, ad, bd + (uint64_t)(kQLoOffset >> 4), id, 1u);
           }
           ptx::mma_commit(&aux->slot_empty[slot]);
         }
@@ -233,14 +233,14 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int slot = pos % p.nslot;
           if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
           ptx::tc_fence_after();
-          const uint32_t sa = ring_addr + slot * kSlotBytes;
+          const uint64_t a0 = vdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+          const uint32_t d_o = tmem + kOCol + c * 32;
 #pragma unroll
           for (int kt = 0; kt < 8; ++kt) {
-            const uint64_t ad = ptx::smem_desc(sa + kt * 2048, kSubBytes, 1024, 2);
-            const uint32_t pb = p_addr + kt * 256;
-            ptx::mma_f16(tmem + kOCol + c * 32, ad, ptx::smem_desc(pb, 128, 2048, 0), id2,
-                         (i > 0 || kt > 0) ? 1u : 0u);
-            ptx::mma_f16(tmem + kOCol + c * 32, ad, ptx::smem_desc(pb + kPHalfBytes, 128, 2048, 0), id2, 1u);
+            const uint64_t ad = a0 + (uint64_t)(kt * 128);
+            const uint64_t bd = pdesc0 + (uint64_t)(kt * 16);
+            ptx::mma_f16(d_o, ad, bd, id2, (i | kt) ? 1u : 0u);
+            ptx::mma_f16(d_o, ad, bd + (uint64_t)(kPHalfBytes >> 4), id2, 1u);
           }
           ptx::mma_commit(&aux->slot_empty[slot]);
         }

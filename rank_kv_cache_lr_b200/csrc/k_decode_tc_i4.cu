@@ -9,13 +9,18 @@
 // the exact fused product-sum) and q~, p enter the MMAs as fp16 (11 significant bits,
 // so neither needs the hi/lo split of the bf16 kernel).
 //
-// Data flow.  The rows of a 128-token tile are contiguous in the cache, so the producer
-// (warp 0) moves a tile's packed codes and its {scale, zero} words with two plain bulk
-// copies per side into a ring of raw slots.  Six dequantisation warps expand raw tiles
-// into 32 KB operand slots (128 tokens x 128 ranks, fp16, the 128-byte-swizzled
-// K-major layout that GEMM1 reads as A and GEMM2 reads MN-major).  Warp 1 owns TMEM and
-// issues the MMAs from one thread.  Four softmax warps (thread = token row = TMEM lane)
-// turn scores into probabilities and finish with the epilogue (thread = rank row).
+// Data flow.  The cache stores int4 latents in 128-token blocks, group-major inside a
+// block, so the codes and the {scale, zero} words of one side (K or V) of one tile are
+// two contiguous runs (G x 2 KB and G x 512 B).  The producer (warp 0) moves each with
+// one plain bulk copy into a ring of raw slots (per-SM copy throughput grows with the
+// copy size; 2-10 KB copies from one stream fall well short of HBM bandwidth).  Eight
+// dequantisation warps (thread = token row x half chunk) expand each 128-rank chunk
+// (4 groups) of a raw slot into a 32 KB operand slot
+// (128 tokens x 128 ranks, fp16, the 128-byte-swizzled K-major layout that GEMM1 reads
+// as A and GEMM2 reads MN-major); lanes walk consecutive tokens, so their shared-memory
+// reads and swizzled writes are free of bank conflicts.  Warp 1 owns TMEM and issues
+// the MMAs from one thread.  Four softmax warps (thread = token row = TMEM lane) turn
+// scores into probabilities and finish with the epilogue (thread = rank row).
 //
 // Pipeline.  Operand slots, raw slots and MMAs all follow the order
 //   K(0), K(1), V(0), K(2), V(1), ..., K(n-1), V(n-2), V(n-1)
@@ -46,18 +51,32 @@ using tc::kTile;
 using tc::kTraceSlots;
 using tc::warp_reduce_scatter32;
 
-constexpr int kThreads = 384;              // 12 warps
-constexpr int kDqThreads = 192;            // warps 2, 3, 8, 9, 10, 11
+// 16 warps in four warpgroups: [producer, MMA, 2 idle] [4 softmax] [dequantisation x 8].
+// A warp runs on sub-partition (warp % 4).  A single thread issuing N = 32 MMAs slows
+// about fivefold when ALU-bound warps share its sub-partition, so the MMA warp (1)
+// shares sub-partition 1 only with the softmax warp that must read TMEM lanes 32..63;
+// the dequantisation work runs on warps 8, 10, 11, 12, 14, 15 (sub-partitions 0, 2, 3)
+// and warps 9, 13 stay idle.  Launched at 128 registers per thread; the warpgroups then
+// rebalance the block's 64K registers with setmaxnreg (the softmax keeps 32 scores and
+// 32 running sums per row).
+constexpr int kThreads = 512;
+constexpr int kDqWarp0 = 8;                // first warp of the dequantisation warpgroups
+constexpr int kDqThreads = 192;            // six working dequantisation warps
+constexpr int kLaunchRegs = 128;
+constexpr int kRegsCtl = 56, kRegsSoftmax = 208, kRegsDq = 104;
+static_assert(128 * kRegsCtl + 128 * kRegsSoftmax + 256 * kRegsDq <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr int kSubBytes = 128 * 128;       // 128 tokens x 64 ranks x 2 B
 constexpr int kSlotBytes = 2 * kSubBytes;  // 128 tokens x 128 ranks
 constexpr int kQRows = 32;                 // query heads, padded
 constexpr int kQSubBytes = kQRows * 128;   // 32 rows x 64 ranks x 2 B
 constexpr int kPBytes = 128 * 32 * 2;      // 128 tokens x 32 heads x 2 B
-constexpr int kAuxBytes = 1024;
+constexpr int kAuxBytes = 2048;
 constexpr int kSCol = 0;                   // TMEM: S of tile s in columns [32 (s % 2), +32)
 constexpr int kOCol = 64;                  // TMEM: O~ chunk c in columns [64 + 32c, +32)
 constexpr int kMaxSlots = 4;
-constexpr int kMaxRaw = 6;
+constexpr int kMaxRaw = 6;                 // raw slot: one side of one tile, codes (G x 2 KB)
+                                           // then {scale, zero} words (G x 512 B)
 
 struct I4Params {
   const uint32_t* codes_k;
@@ -67,7 +86,7 @@ struct I4Params {
   long long cap;
   int r_k, r_v, G_k, G_v, ck, cv, kb_k, tmem_cols;
   int Hq, hist_len, stable_len, split_tokens, n_splits, nslot, nraw;
-  uint32_t q_bytes, raw_bytes, raw_codes_bytes;
+  uint32_t q_bytes, raw_bytes, raw_params;   // raw slot size; offset of its params
   float* part_o;
   float* part_ml;
   int* err;
@@ -92,7 +111,7 @@ static_assert(sizeof(Aux) <= kAuxBytes, "aux block");
 struct I4State {
   CUtensorMap q;
   int nslot, nraw;
-  uint32_t raw_bytes, raw_codes_bytes;
+  uint32_t raw_bytes, raw_params;
   size_t smem;
 };
 
@@ -100,9 +119,9 @@ __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux,
   return tc::wait_b(bar, parity, &aux->abort_flag, err);
 }
 
-// The k-th unit of the pipeline order: K(k/2 ... ) — unit u is K(tile) or V(tile).
-//   u = 0 -> K(0); u = 2s - 1 -> K(s) for 1 <= s < n; u = 2s -> V(s - 1).  With n tiles
-//   the last unit, u = 2n - 1, is V(n - 1).
+// Unit u of the pipeline order (each unit is the K or the V side of one tile):
+//   u = 0 -> K(0); u = 2s - 1 -> K(s) for 1 <= s < n; u = 2s -> V(s - 1); the last
+//   unit, u = 2n - 1, is V(n - 1).
 __device__ __forceinline__ void unit_of(int u, int n, int* tile, bool* is_v) {
   if (u == 0) {
     *tile = 0;
@@ -117,17 +136,6 @@ __device__ __forceinline__ void unit_of(int u, int n, int* tile, bool* is_v) {
     *tile = (u >> 1) - 1;
     *is_v = true;
   }
-}
-
-// Byte span of the {scale, zero} words of rows [row0, row0 + n) (G words per row),
-// widened to 16-byte boundaries for a bulk copy; `off` is where row0 starts in it.
-__device__ __forceinline__ void param_span(const uint32_t* params, int G, long long row0, int n,
-                                           const uint8_t** src, uint32_t* off, uint32_t* bytes) {
-  const uintptr_t a = reinterpret_cast<uintptr_t>(params + row0 * G);
-  const uintptr_t al = a & ~(uintptr_t)15;
-  *src = reinterpret_cast<const uint8_t*>(al);
-  *off = (uint32_t)(a - al);
-  *bytes = (*off + (uint32_t)n * G * 4 + 15u) & ~15u;
 }
 
 // Eight int4 codes of one word -> four fp16 pairs (m0,m4) (m1,m5) (m2,m6) (m3,m7) of
@@ -167,7 +175,7 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
                : "memory");
 }
 
-// Shared memory: [aux 1 KB][q~ per 64-rank sub-block][operand ring nslot x 32 KB]
+// Shared memory: [aux 2 KB][q~ per 64-rank sub-block][operand ring nslot x 32 KB]
 //                [P double buffer 2 x 8 KB][raw ring nraw x raw_bytes]
 __global__ void __launch_bounds__(kThreads, 1)
     k_decode_tc_i4(const __grid_constant__ CUtensorMap tm_q, const I4Params p) {
@@ -227,306 +235,314 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
   if (threadIdx.x == 32) tc::trace_stamp(p.trace, 1);
 
-  const bool is_dq = warp == 2 || warp == 3 || warp >= 8;
-  if (warp == 0) {
-    // ------------------------------------------------------------- bulk-copy producer
-    if (lane == 0 && ntiles > 0) {
-      bool waited = false, ok = true;
-      int issued = 0;
-      for (int u = 0; u < nunits && ok; ++u) {
-        int tile;
-        bool is_v;
-        unit_of(u, ntiles, &tile, &is_v);
-        const int t0 = tok_begin + tile * kTile;
-        const int n = min(kTile, tok_end - t0);
-        const int rs = u % p.nraw, round = u / p.nraw;
-        if (!waited && (round > 0 || t0 + n > p.stable_len)) {
+  // Roles by warpgroup; each sets its register budget first thing in its own branch,
+  // so the compiler allocates that branch within the budget.
+  if (warp < 4) {
+    ptx::setmaxnreg_dec<kRegsCtl>();
+    if (warp == 0) {
+      // ------------------------------------------------------------- bulk-copy producer
+      if (lane == 0 && ntiles > 0) {
+        bool waited = false, ok = true;
+        int issued = 0;
+        for (int u = 0; u < nunits && ok; ++u) {
+          int tile;
+          bool is_v;
+          unit_of(u, ntiles, &tile, &is_v);
+          const int t0 = tok_begin + tile * kTile;
+          const int n = min(kTile, tok_end - t0);
+          const int rs = u % p.nraw, round = u / p.nraw;
+          if (!waited && (round > 0 || t0 + n > p.stable_len)) {
+            pdl_wait();
+            ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
+            for (int sb = 0; sb < p.kb_k; ++sb)
+              ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
+            waited = true;
+          }
+          if (round > 0 && !(ok = wait_b(&aux->raw_empty[rs], (round - 1) & 1, aux, p.err))) break;
+          const int G = is_v ? p.G_v : p.G_k;
+          const long long row0 = (long long)b * p.cap + t0;
+          uint8_t* dst = raw + rs * p.raw_bytes;
+          ptx::mbar_arrive_expect_tx(&aux->raw_full[rs], (uint32_t)G * 2560u);
+          ptx::bulk_load(dst, (is_v ? p.codes_v : p.codes_k) + i4_code_index(row0, G, 0, 0), (uint32_t)G * 2048u,
+                         &aux->raw_full[rs]);
+          ptx::bulk_load(dst + p.raw_params, (is_v ? p.params_v : p.params_k) + i4_param_index(row0, G, 0),
+                         (uint32_t)G * 512u, &aux->raw_full[rs]);
+          issued = u + 1;
+        }
+        if (!waited) {
           pdl_wait();
           ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
           for (int sb = 0; sb < p.kb_k; ++sb)
             ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
-          waited = true;
         }
-        if (round > 0 && !(ok = wait_b(&aux->raw_empty[rs], (round - 1) & 1, aux, p.err))) break;
-        const int G = is_v ? p.G_v : p.G_k;
-        const long long row0 = (long long)b * p.cap + t0;
-        const uint32_t* codes = is_v ? p.codes_v : p.codes_k;
-        const uint8_t* psrc;
-        uint32_t poff, pbytes;
-        param_span(is_v ? p.params_v : p.params_k, G, row0, n, &psrc, &poff, &pbytes);
-        const uint32_t cbytes = (uint32_t)n * G * 16;
-        uint8_t* dst = raw + rs * p.raw_bytes;
-        ptx::mbar_arrive_expect_tx(&aux->raw_full[rs], cbytes + pbytes);
-        ptx::bulk_load(dst, codes + row0 * G * 4, cbytes, &aux->raw_full[rs]);
-        ptx::bulk_load(dst + p.raw_codes_bytes, psrc, pbytes, &aux->raw_full[rs]);
-        issued = u + 1;
+        if (!ok) {
+          drain_wait(&aux->q_full, 0);
+          for (int k = max(0, issued - p.nraw); k < issued; ++k)
+            drain_wait(&aux->raw_full[k % p.nraw], (k / p.nraw) & 1);
+        }
       }
-      if (!waited) {
-        pdl_wait();
-        ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
-        for (int sb = 0; sb < p.kb_k; ++sb)
-          ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------- MMA issuer
+      if (lane == 0 && ntiles > 0) {
+        const uint32_t id = ptx::idesc_f16(0, 0, 0, 128, 32);    // GEMM1: fp16, K-major x K-major
+        const uint32_t id2 = ptx::idesc_f16(0, 1, 1, 128, 32);   // GEMM2: fp16, MN-major x MN-major
+        // Descriptors are built once; a step along K or to another slot adds its byte
+        // offset >> 4 to the start-address field (shared-memory addresses stay below
+        // 256 KB, so the 14-bit field never carries).
+        const uint64_t kdesc0 = ptx::smem_desc(ptx::smem_u32(ring), 16, 1024, 2);       // Z_k, K-major SW128
+        const uint64_t qdesc0 = ptx::smem_desc(ptx::smem_u32(q_s), 16, 1024, 2);        // q~, K-major SW128
+        const uint64_t vdesc0 = ptx::smem_desc(ptx::smem_u32(ring), kSubBytes, 1024, 2); // Z_v, MN-major SW128
+        const uint64_t pdesc0 = ptx::smem_desc(ptx::smem_u32(p_s), 128, 2048, 0);       // P, MN-major
+        bool ok = wait_b(&aux->q_full, 0, aux, p.err);
+        ptx::tc_fence_after();
+        tc::trace_stamp(p.trace, 2);
+        int pos = 0;
+        for (int u = 0; u < nunits && ok; ++u) {
+          int tile;
+          bool is_v;
+          unit_of(u, ntiles, &tile, &is_v);
+          if (!is_v) {
+            // GEMM1(tile): S[tile % 2] = Z_k q~^T
+            const int sb2 = tile & 1;
+            if (tile >= 2 && !(ok = wait_b(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
+            ptx::tc_fence_after();
+            const uint32_t d_s = tmem + kSCol + 32 * sb2;
+            for (int c = 0; c < p.ck && ok; ++c, ++pos) {
+              const int slot = pos % p.nslot;
+              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+              ptx::tc_fence_after();
+              const uint64_t a0 = kdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+              const uint64_t b0 = qdesc0 + (uint64_t)((c * 2 * kQSubBytes) >> 4);
+              const int nk = min(8, (p.r_k - c * 128) >> 4);     // 16-rank K steps in this chunk
+              // step kk: sub-block kk / 4 (16 KB on A, 4 KB on B), 32 bytes per step within it
+              for (int kk = 0; kk < nk; ++kk) {
+                const uint32_t ao = (uint32_t)((kk >> 2) * (kSubBytes >> 4) + (kk & 3) * 2);
+                const uint32_t bo = (uint32_t)((kk >> 2) * (kQSubBytes >> 4) + (kk & 3) * 2);
+                ptx::mma_f16(d_s, a0 + ao, b0 + bo, id, (c | kk) ? 1u : 0u);
+              }
+              ptx::mma_commit(&aux->slot_empty[slot]);
+            }
+            if (!ok) break;
+            ptx::mma_commit(&aux->s_full[sb2]);
+            if (tile < 16) tc::trace_stamp(p.trace, 3 + 4 * tile);
+          } else {
+            // GEMM2(tile): O~ += Z_v^T P[tile % 2]
+            const int pb2 = tile & 1;
+            if (!(ok = wait_b(&aux->p_full[pb2], (tile >> 1) & 1, aux, p.err))) break;
+            ptx::tc_fence_after();
+            const uint64_t b0 = pdesc0 + (uint64_t)((pb2 * kPBytes) >> 4);
+            for (int c = 0; c < p.cv && ok; ++c, ++pos) {
+              const int slot = pos % p.nslot;
+              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+              ptx::tc_fence_after();
+              const uint64_t a0 = vdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+              const uint32_t d_o = tmem + kOCol + c * 32;
+              // K step kt = 16 tokens: 2 KB on A (16 swizzled rows), 256 B on P
+#pragma unroll
+              for (int kt = 0; kt < 8; ++kt)
+                ptx::mma_f16(d_o, a0 + (uint64_t)(kt * 128), b0 + (uint64_t)(kt * 16), id2, (tile | kt) ? 1u : 0u);
+              ptx::mma_commit(&aux->slot_empty[slot]);
+            }
+            if (!ok) break;
+            ptx::mma_commit(&aux->p_empty[pb2]);
+            if (tile < 16) tc::trace_stamp(p.trace, 6 + 4 * tile);
+          }
+        }
+        ptx::mma_commit(&aux->o_final);
+        if (!ok) drain_wait(&aux->o_final, 0);
       }
-      if (!ok) {
-        drain_wait(&aux->q_full, 0);
-        for (int u = max(0, issued - p.nraw); u < issued; ++u)
-          drain_wait(&aux->raw_full[u % p.nraw], (u / p.nraw) & 1);
+      __syncwarp();
+    }
+  } else if (warp < kDqWarp0) {
+    ptx::setmaxnreg_inc<kRegsSoftmax>();
+    if (ntiles > 0) {
+      // ------------------------------------------------------------- softmax / epilogue
+      const int qd = warp & 3;
+      const int row = qd * 32 + lane;
+      const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+      float l[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) l[j] = 0.f;
+      bool ok = true;
+      for (int i = 0; i < ntiles; ++i) {
+        const int k2 = i & 1;
+        const bool valid = tok_begin + i * kTile + row < tok_end;
+        ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full[k2], (i >> 1) & 1, aux, p.err));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 4 + 4 * i);
+        const uint32_t s_col = tmem + lane_off + kSCol + 32 * k2;
+        uint32_t sv[32];
+        ptx::tmem_ld32(s_col, sv);
+        ptx::tmem_wait_ld();
+        float s[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+
+        bool ex = false;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ex |= s[j] > aux->m_s[j] + kLazy;
+        ex = ptx::named_bar_or(1, 128, ex);
+        if (ex) {
+          // the value mix of the previous tile must be complete before O~ is rescaled
+          if (i >= 1) {
+            ok = ptx::named_bar_and(1, 128, wait_b(&aux->p_empty[(i - 1) & 1], ((i - 1) >> 1) & 1, aux, p.err));
+            if (!ok) break;
+            ptx::tc_fence_after();
+          }
+          aux->red[qd][lane] = warp_reduce_scatter32<true>(s, lane);
+          ptx::tmem_ld32(s_col, sv);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+          ptx::named_bar_sync(1, 128);
+          if (qd == 0) {
+            const float mt =
+                fmaxf(fmaxf(aux->red[0][lane], aux->red[1][lane]), fmaxf(aux->red[2][lane], aux->red[3][lane]));
+            const float mo = aux->m_s[lane];
+            const float mn = fmaxf(mo, mt);
+            aux->alpha_s[lane] = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+            aux->m_s[lane] = mn;
+          }
+          ptx::named_bar_sync(1, 128);
+          bool need_o = false;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float a = aux->alpha_s[j];
+            l[j] *= a;
+            need_o |= a < 1.f;
+          }
+          if (need_o && i > 0) {
+            for (int c = 0; c < p.cv; ++c) {
+              uint32_t v2[32];
+              ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v2[j] = __float_as_uint(__uint_as_float(v2[j]) * aux->alpha_s[j]);
+              ptx::tmem_st32(tmem + lane_off + kOCol + c * 32, v2);
+            }
+            ptx::tmem_wait_st();
+          }
+        }
+        // P[i % 2] is free once the value mix of tile i - 2 has completed
+        if (i >= 2) {
+          ok = ptx::named_bar_and(1, 128, wait_b(&aux->p_empty[k2], ((i - 2) >> 1) & 1, aux, p.err));
+          if (!ok) break;
+        }
+        // probabilities as fp16; l sums the rounded values the MMA uses
+        const uint32_t prow = ptx::smem_u32(p_s + k2 * kPBytes + row * 16);
+#pragma unroll
+        for (int hg = 0; hg < 4; ++hg) {
+          uint32_t hw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = hg * 8 + 2 * e;
+            const __half2 h = __floats2half2_rn(exp2f(s[j] - aux->m_s[j]), exp2f(s[j + 1] - aux->m_s[j + 1]));
+            const float2 f = __half22float2(h);
+            l[j] += f.x;
+            l[j + 1] += f.y;
+            hw[e] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + hg * 2048), "r"(hw[0]), "r"(hw[1]),
+                       "r"(hw[2]), "r"(hw[3])
+                       : "memory");
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&aux->s_empty[k2]);
+        ptx::mbar_arrive(&aux->p_full[k2]);
+        if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 5 + 4 * i);
+      }
+      if (ok) ok = ptx::named_bar_and(1, 128, wait_b(&aux->o_final, 0, aux, p.err));
+      if (ok) {
+        ptx::tc_fence_after();
+        const size_t base_out = ((size_t)b * p.n_splits + split) * p.Hq;
+        // TMEM row m of a chunk holds rank 8 (m / 8) + perm(m % 8), perm = 0,4,1,5,2,6,3,7
+        const int m = qd * 32 + lane;
+        const int e_in = (m & ~7) + ((m & 7) >> 1) + ((m & 1) << 2);
+        for (int c = 0; c < p.cv; ++c) {
+          uint32_t v2[32];
+          ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
+          ptx::tmem_wait_ld();
+          const int e = c * 128 + e_in;
+          if (e < p.r_v) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < p.Hq) p.part_o[(base_out + j) * p.r_v + e] = __uint_as_float(v2[j]);
+          }
+        }
+        aux->red[qd][lane] = warp_reduce_scatter32<false>(l, lane);
+        ptx::named_bar_sync(1, 128);
+        if (qd == 0 && lane < p.Hq) {
+          const float lt = (aux->red[0][lane] + aux->red[1][lane]) + (aux->red[2][lane] + aux->red[3][lane]);
+          p.part_ml[(base_out + lane) * 2] = aux->m_s[lane];
+          p.part_ml[(base_out + lane) * 2 + 1] = lt;
+        }
+        if (threadIdx.x == 128) tc::trace_stamp(p.trace, kTraceSlots - 1);
       }
     }
-  } else if (is_dq) {
+  } else {
+    ptx::setmaxnreg_dec<kRegsDq>();
     // ------------------------------------------------------------- dequantisation
     if (ntiles > 0) {
-      const int dq = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;
-      const uint32_t ring_addr = ptx::smem_u32(ring);
-      bool ok = true;
-      int pos = 0;   // operand-slot sequence number
+      // working warps 8, 10, 11, 12, 14, 15 -> dq 0..191; unit v = (token v % 128, group
+      // v / 128 of the chunk) for v = dq, dq + 192, ...; lanes walk consecutive tokens
+      const int wi = warp - kDqWarp0;      // 0..7
+      const bool dq_live = wi != 1 && wi != 5;
+      const int dq = (wi - (wi > 1) - (wi > 5)) * 32 + lane;
+      const uint32_t ring_base = ptx::smem_u32(ring);
+      bool ok = dq_live;
+      int pos = 0;
       for (int u = 0; u < nunits && ok; ++u) {
         int tile;
         bool is_v;
         unit_of(u, ntiles, &tile, &is_v);
-        const int t0 = tok_begin + tile * kTile;
-        const int n = min(kTile, tok_end - t0);
+        const int nvalid = tok_end - (tok_begin + tile * kTile);   // valid token rows of the tile
+        const int G = is_v ? p.G_v : p.G_k;
+        const int nch = is_v ? p.cv : p.ck;
         const int rs = u % p.nraw;
         if (!(ok = wait_b(&aux->raw_full[rs], (u / p.nraw) & 1, aux, p.err))) break;
-        const int G = is_v ? p.G_v : p.G_k;
-        const long long row0 = (long long)b * p.cap + t0;
-        const uint8_t* rb = raw + rs * p.raw_bytes;
-        const uint32_t poff =
-            (uint32_t)(reinterpret_cast<uintptr_t>((is_v ? p.params_v : p.params_k) + row0 * G) & 15u);
-        const uint4* cw = reinterpret_cast<const uint4*>(rb);
-        const uint32_t* pw = reinterpret_cast<const uint32_t*>(rb + p.raw_codes_bytes + poff);
-        const int nch = is_v ? p.cv : p.ck;
-        for (int c = 0; c < nch && ok; ++c, ++pos) {
-          const int slot = pos % p.nslot, round = pos / p.nslot;
-          if (round > 0 && !(ok = wait_b(&aux->slot_empty[slot], (round - 1) & 1, aux, p.err))) break;
-          const uint32_t dst = ring_addr + slot * kSlotBytes;
-          // unit = (token t, group lg of the chunk): four words -> four 16-byte chunks of
-          // row t.  Lanes of a quarter-warp cover 2 tokens x 4 groups; rotating the word
-          // order of groups 2, 3 by two chunks makes each store conflict-free.
-          for (int v = dq; v < kTile * 4; v += kDqThreads) {
-            const int t = v >> 2, lg = v & 3, g = c * 4 + lg;
-            if (g >= G) continue;
-            uint4 w = make_uint4(0u, 0u, 0u, 0u);
-            uint32_t s2 = 0u, z2 = 0u;
-            if (t < n) {
-              w = cw[t * G + g];
-              const uint32_t prm = pw[t * G + g];
-              s2 = __byte_perm(prm, 0u, 0x1010);
-              z2 = __byte_perm(prm, 0u, 0x3232);
+        for (int c = 0; c < nch; ++c, ++pos) {
+          const int slot = pos % p.nslot;
+          if (pos >= p.nslot && !(ok = wait_b(&aux->slot_empty[slot], ((pos / p.nslot) - 1) & 1, aux, p.err)))
+            break;
+          const int ng = min(4, G - 4 * c);
+          const uint8_t* rb = raw + rs * p.raw_bytes + c * 8192;          // codes of groups 4c..
+          const uint32_t* rp = reinterpret_cast<const uint32_t*>(raw + rs * p.raw_bytes + p.raw_params) + c * 512;
+          const uint32_t dst = ring_base + slot * kSlotBytes;
+          // up to three units per thread; all loads first, then the arithmetic and stores
+          constexpr int kU = (4 * kTile + kDqThreads - 1) / kDqThreads;
+          uint4 w[kU];
+          uint32_t prm[kU];
+#pragma unroll
+          for (int k = 0; k < kU; ++k) {
+            const int v = dq + k * kDqThreads, t = v & (kTile - 1), gl = v >> 7;
+            w[k] = make_uint4(0u, 0u, 0u, 0u);
+            prm[k] = 0u;
+            if (v < ng * kTile && t < nvalid) {
+              w[k] = reinterpret_cast<const uint4*>(rb)[gl * kTile + t];
+              prm[k] = rp[gl * kTile + t];
             }
-            const int rot = lg & 2;
-            if (rot) {
-              const uint32_t x0 = w.x, x1 = w.y;
-              w.x = w.z;
-              w.y = w.w;
-              w.z = x0;
-              w.w = x1;
+          }
+#pragma unroll
+          for (int k = 0; k < kU; ++k) {
+            const int v = dq + k * kDqThreads, t = v & (kTile - 1), gl = v >> 7, sw = t & 7;
+            if (v < ng * kTile) {
+              const uint32_t s2 = __byte_perm(prm[k], 0u, 0x1010), z2 = __byte_perm(prm[k], 0u, 0x3232);
+              // group gl = ranks 32 gl.. of the chunk: sub-block gl / 2, 16-byte columns 4 (gl % 2)..
+              const uint32_t rowa = dst + (gl >> 1) * kSubBytes + t * 128;
+              const int cb = (gl & 1) * 4;
+              sts128(rowa + (((cb + 0) ^ sw) << 4), dequant8(w[k].x, s2, z2));
+              sts128(rowa + (((cb + 1) ^ sw) << 4), dequant8(w[k].y, s2, z2));
+              sts128(rowa + (((cb + 2) ^ sw) << 4), dequant8(w[k].z, s2, z2));
+              sts128(rowa + (((cb + 3) ^ sw) << 4), dequant8(w[k].w, s2, z2));
             }
-            const uint32_t rowa = dst + (lg >> 1) * kSubBytes + t * 128;
-            const int cb = (lg & 1) * 4, sw = t & 7;
-            sts128(rowa + (((cb + (0 ^ rot)) ^ sw) << 4), dequant8(w.x, s2, z2));
-            sts128(rowa + (((cb + (1 ^ rot)) ^ sw) << 4), dequant8(w.y, s2, z2));
-            sts128(rowa + (((cb + (2 ^ rot)) ^ sw) << 4), dequant8(w.z, s2, z2));
-            sts128(rowa + (((cb + (3 ^ rot)) ^ sw) << 4), dequant8(w.w, s2, z2));
           }
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(&aux->slot_full[slot]);
         }
         if (ok) ptx::mbar_arrive(&aux->raw_empty[rs]);
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
-    if (lane == 0 && ntiles > 0) {
-      const uint32_t id = ptx::idesc_f16(0, 0, 0, 128, 32);    // GEMM1: fp16, K-major x K-major
-      const uint32_t id2 = ptx::idesc_f16(0, 1, 1, 128, 32);   // GEMM2: fp16, MN-major x MN-major
-      const uint32_t q_addr = ptx::smem_u32(q_s), ring_addr = ptx::smem_u32(ring), p_addr = ptx::smem_u32(p_s);
-      bool ok = wait_b(&aux->q_full, 0, aux, p.err);
-      ptx::tc_fence_after();
-      tc::trace_stamp(p.trace, 2);
-      int pos = 0;
-      for (int u = 0; u < nunits && ok; ++u) {
-        int tile;
-        bool is_v;
-        unit_of(u, ntiles, &tile, &is_v);
-        if (!is_v) {
-          // GEMM1(tile): S[tile % 2] = Z_k q~^T
-          const int sb2 = tile & 1;
-          if (tile >= 2 && !(ok = wait_b(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
-          ptx::tc_fence_after();
-          for (int c = 0; c < p.ck && ok; ++c, ++pos) {
-            const int slot = pos % p.nslot;
-            if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
-            ptx::tc_fence_after();
-            const uint32_t sa = ring_addr + slot * kSlotBytes;
-#pragma unroll
-            for (int sb = 0; sb < 2; ++sb) {
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const int k0 = c * 128 + sb * 64 + kk * 16;
-                if (k0 < p.r_k) {
-                  const uint64_t ad = ptx::smem_desc(sa + sb * kSubBytes + kk * 32, 16, 1024, 2);
-                  const uint64_t bd = ptx::smem_desc(q_addr + (c * 2 + sb) * kQSubBytes + kk * 32, 16, 1024, 2);
-                  ptx::mma_f16(tmem + kSCol + 32 * sb2, ad, bd, id, k0 > 0 ? 1u : 0u);
-                }
-              }
-            }
-            ptx::mma_commit(&aux->slot_empty[slot]);
-          }
-          if (!ok) break;
-          ptx::mma_commit(&aux->s_full[sb2]);
-          if (tile < 16) tc::trace_stamp(p.trace, 3 + 4 * tile);
-        } else {
-          // GEMM2(tile): O~ += Z_v^T P[tile % 2]
-          const int pb2 = tile & 1;
-          if (!(ok = wait_b(&aux->p_full[pb2], (tile >> 1) & 1, aux, p.err))) break;
-          ptx::tc_fence_after();
-          for (int c = 0; c < p.cv && ok; ++c, ++pos) {
-            const int slot = pos % p.nslot;
-            if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
-            ptx::tc_fence_after();
-            const uint32_t sa = ring_addr + slot * kSlotBytes;
-#pragma unroll
-            for (int kt = 0; kt < 8; ++kt) {
-              const uint64_t ad = ptx::smem_desc(sa + kt * 2048, kSubBytes, 1024, 2);
-              const uint64_t bd = ptx::smem_desc(p_addr + pb2 * kPBytes + kt * 256, 128, 2048, 0);
-              ptx::mma_f16(tmem + kOCol + c * 32, ad, bd, id2, (tile > 0 || kt > 0) ? 1u : 0u);
-            }
-            ptx::mma_commit(&aux->slot_empty[slot]);
-          }
-          if (!ok) break;
-          ptx::mma_commit(&aux->p_empty[pb2]);
-          if (tile < 16) tc::trace_stamp(p.trace, 6 + 4 * tile);
-        }
-      }
-      ptx::mma_commit(&aux->o_final);
-      if (!ok) drain_wait(&aux->o_final, 0);
-    }
-    __syncwarp();
-  } else if (ntiles > 0) {
-    // ------------------------------------------------------------- softmax / epilogue
-    const int qd = warp & 3;
-    const int row = qd * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    float l[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) l[j] = 0.f;
-    bool ok = true;
-    for (int i = 0; i < ntiles; ++i) {
-      const int k2 = i & 1;
-      const bool valid = tok_begin + i * kTile + row < tok_end;
-      ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full[k2], (i >> 1) & 1, aux, p.err));
-      if (!ok) break;
-      ptx::tc_fence_after();
-      if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 4 + 4 * i);
-      const uint32_t s_col = tmem + lane_off + kSCol + 32 * k2;
-      uint32_t sv[32];
-      ptx::tmem_ld32(s_col, sv);
-      ptx::tmem_wait_ld();
-      float s[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
-
-      bool ex = false;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) ex |= s[j] > aux->m_s[j] + kLazy;
-      ex = ptx::named_bar_or(1, 128, ex);
-      if (ex) {
-        // the value mix of the previous tile must be complete before O~ is rescaled
-        if (i >= 1) {
-          ok = ptx::named_bar_and(1, 128, wait_b(&aux->p_empty[(i - 1) & 1], ((i - 1) >> 1) & 1, aux, p.err));
-          if (!ok) break;
-          ptx::tc_fence_after();
-        }
-        aux->red[qd][lane] = warp_reduce_scatter32<true>(s, lane);
-        ptx::tmem_ld32(s_col, sv);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
-        ptx::named_bar_sync(1, 128);
-        if (qd == 0) {
-          const float mt =
-              fmaxf(fmaxf(aux->red[0][lane], aux->red[1][lane]), fmaxf(aux->red[2][lane], aux->red[3][lane]));
-          const float mo = aux->m_s[lane];
-          const float mn = fmaxf(mo, mt);
-          aux->alpha_s[lane] = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
-          aux->m_s[lane] = mn;
-        }
-        ptx::named_bar_sync(1, 128);
-        bool need_o = false;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float a = aux->alpha_s[j];
-          l[j] *= a;
-          need_o |= a < 1.f;
-        }
-        if (need_o && i > 0) {
-          for (int c = 0; c < p.cv; ++c) {
-            uint32_t v2[32];
-            ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v2[j] = __float_as_uint(__uint_as_float(v2[j]) * aux->alpha_s[j]);
-            ptx::tmem_st32(tmem + lane_off + kOCol + c * 32, v2);
-          }
-          ptx::tmem_wait_st();
-        }
-      }
-      // P[i % 2] is free once the value mix of tile i - 2 has completed
-      if (i >= 2) {
-        ok = ptx::named_bar_and(1, 128, wait_b(&aux->p_empty[k2], ((i - 2) >> 1) & 1, aux, p.err));
-        if (!ok) break;
-      }
-      // probabilities as fp16; l sums the rounded values the MMA uses
-      const uint32_t prow = ptx::smem_u32(p_s + k2 * kPBytes + row * 16);
-#pragma unroll
-      for (int hg = 0; hg < 4; ++hg) {
-        uint32_t hw[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = hg * 8 + 2 * e;
-          const __half2 h = __floats2half2_rn(exp2f(s[j] - aux->m_s[j]), exp2f(s[j + 1] - aux->m_s[j + 1]));
-          const float2 f = __half22float2(h);
-          l[j] += f.x;
-          l[j + 1] += f.y;
-          hw[e] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + hg * 2048), "r"(hw[0]), "r"(hw[1]),
-                     "r"(hw[2]), "r"(hw[3])
-                     : "memory");
-      }
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&aux->s_empty[k2]);
-      ptx::mbar_arrive(&aux->p_full[k2]);
-      if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 5 + 4 * i);
-    }
-    if (ok) ok = ptx::named_bar_and(1, 128, wait_b(&aux->o_final, 0, aux, p.err));
-    if (ok) {
-      ptx::tc_fence_after();
-      const size_t base_out = ((size_t)b * p.n_splits + split) * p.Hq;
-      // TMEM row m of a chunk holds rank 8 (m / 8) + perm(m % 8), perm = 0,4,1,5,2,6,3,7
-      const int m = qd * 32 + lane;
-      const int e_in = (m & ~7) + ((m & 7) >> 1) + ((m & 1) << 2);
-      for (int c = 0; c < p.cv; ++c) {
-        uint32_t v2[32];
-        ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
-        ptx::tmem_wait_ld();
-        const int e = c * 128 + e_in;
-        if (e < p.r_v) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < p.Hq) p.part_o[(base_out + j) * p.r_v + e] = __uint_as_float(v2[j]);
-        }
-      }
-      aux->red[qd][lane] = warp_reduce_scatter32<false>(l, lane);
-      ptx::named_bar_sync(1, 128);
-      if (qd == 0 && lane < p.Hq) {
-        const float lt = (aux->red[0][lane] + aux->red[1][lane]) + (aux->red[2][lane] + aux->red[3][lane]);
-        p.part_ml[(base_out + lane) * 2] = aux->m_s[lane];
-        p.part_ml[(base_out + lane) * 2 + 1] = lt;
-      }
-      if (threadIdx.x == 128) tc::trace_stamp(p.trace, kTraceSlots - 1);
     }
   }
   ptx::tc_fence_before();
@@ -541,31 +557,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 // host side
 // ---------------------------------------------------------------------------
 
-int groups(int r) { return (r + 31) / 32; }
 int q_bytes_for(int r_k) { return ((r_k + 63) / 64) * kQSubBytes; }
 
 struct I4Layout {
   int nslot, nraw;
-  uint32_t raw_bytes, raw_codes_bytes;
+  uint32_t raw_bytes, raw_params;
   size_t smem;
 };
 
-// As many operand slots (up to 4) as leave room for two raw slots, then as many raw
-// slots (up to 6) as fit in 227 KB.
+// Raw slots hold one side of one tile.  As many operand slots as leave room for two raw
+// slots (up to four: the dequantisation can then run a full 128-rank chunk further ahead
+// of the MMAs), then as many raw slots (up to 6) as fit in 227 KB.
 bool choose_layout(const lr_cache_desc* d, I4Layout* L) {
-  const int G = std::max(groups(d->rank_k), groups(d->rank_v));
-  L->raw_codes_bytes = (uint32_t)kTile * G * 16;
-  L->raw_bytes = ((uint32_t)kTile * G * 20 + 16 + 127) & ~127u;
+  const int G = std::max((d->rank_k + 31) / 32, (d->rank_v + 31) / 32);
+  L->raw_params = (uint32_t)G * 2048u;
+  L->raw_bytes = (uint32_t)G * 2560u;
   const size_t fixed = (size_t)kAuxBytes + q_bytes_for(d->rank_k) + 2 * kPBytes;
-  int ns = kMaxSlots;
-  while (ns >= 2 && fixed + (size_t)ns * kSlotBytes + 2 * (size_t)L->raw_bytes > (size_t)kSmemLimit) --ns;
-  if (ns < 2) return false;
-  int nr = (int)(((size_t)kSmemLimit - fixed - (size_t)ns * kSlotBytes) / L->raw_bytes);
-  nr = std::min(nr, kMaxRaw);
-  L->nslot = ns;
-  L->nraw = nr;
-  L->smem = fixed + (size_t)ns * kSlotBytes + (size_t)nr * L->raw_bytes;
-  return true;
+  for (int ns = kMaxSlots; ns >= 2; --ns) {
+    if (fixed + (size_t)ns * kSlotBytes > (size_t)kSmemLimit) continue;
+    const int nr =
+        std::min(kMaxRaw, (int)(((size_t)kSmemLimit - fixed - (size_t)ns * kSlotBytes) / L->raw_bytes));
+    if (nr >= 2) {
+      L->nslot = ns;
+      L->nraw = nr;
+      L->smem = fixed + (size_t)ns * kSlotBytes + (size_t)nr * L->raw_bytes;
+      return true;
+    }
+  }
+  return false;
 }
 
 }  // namespace
@@ -603,7 +622,7 @@ cudaError_t tc_i4_prepare(lr_cache* c) {
   st->nslot = L.nslot;
   st->nraw = L.nraw;
   st->raw_bytes = L.raw_bytes;
-  st->raw_codes_bytes = L.raw_codes_bytes;
+  st->raw_params = L.raw_params;
   st->smem = L.smem;
   return cudaSuccess;
 }
@@ -622,7 +641,7 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   p.codes_v = c->codes_v;
   p.params_k = c->params_k;
   p.params_v = c->params_v;
-  p.cap = d.capacity;
+  p.cap = c->lat_cap;
   p.r_k = d.rank_k;
   p.r_v = d.rank_v;
   p.G_k = c->G_k;
@@ -640,7 +659,7 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   p.nraw = st->nraw;
   p.q_bytes = q_bytes_for(d.rank_k);
   p.raw_bytes = st->raw_bytes;
-  p.raw_codes_bytes = st->raw_codes_bytes;
+  p.raw_params = st->raw_params;
   p.part_o = c->part_o;
   p.part_ml = c->part_ml;
   p.err = c->dev_err;
@@ -648,5 +667,11 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_decode_tc_i4, optin_done);
   if (e != cudaSuccess) return e;
+  // The register rebalancing assumes the launch allocation the split was sized for.
+  static const int regs = [] {
+    cudaFuncAttributes fa;
+    return cudaFuncGetAttributes(&fa, k_decode_tc_i4) == cudaSuccess ? fa.numRegs : -1;
+  }();
+  if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   return launch_pdl(k_decode_tc_i4, dim3(n_splits, d.batch), dim3(kThreads), st->smem, s, st->q, p);
 }

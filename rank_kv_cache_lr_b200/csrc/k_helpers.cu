@@ -268,117 +268,149 @@ __global__ void __launch_bounds__(256) k_step_pre(AppendArgs aa, QprojArgs qa, i
 }
 
 // ---- split merge and output projection ------------------------------------------
-// One CTA per (query head j, sequence b); thread = pair of output columns.  The
-// B_v,h slice is staged before the grid-dependency wait; then the split weights
-// (log-sum-exp with the window partial), the combined rank-space output o~ (all S
-// partial loads of a rank issued together), and o = o~ B_v,h / l.
-constexpr int kMergeThreads = 128;
-constexpr size_t kMergeStage = 64 * 1024;    // bytes of B_v,h rows staged in shared memory
+// One CTA per (32-column block of the head dimension, KV head h, sequence b), 256
+// threads.  Its columns of B_v,h ([r_v][32], no in-flight kernel writes them) are
+// staged before the grid-dependency wait and reused by every query head of the group.
+// Query heads go through in passes of up to 8: the split weights (log-sum-exp over the
+// splits and the window partial; one warp per head), the combined rank-space output
+// o~_j = sum_s w_s o~_s,j (thread = rank), and o_j = o~_j B_v,h / l_j (thread = 4
+// columns x head x quarter of the ranks, quarters added in a fixed order).
+constexpr int kMergeThreads = 256;
+constexpr int kMergeCols = 32;     // output columns per CTA
+constexpr int kMergeHeads = 8;     // query heads per pass
+
+struct MergeArgs {
+  const float* part_o; const float* part_ml; const float* win_o; const float* win_ml;
+  const void* Bv; void* out; float* lse;
+  int S, Hq, Hkv, d, D, rv;
+};
+
+size_t merge_pitch_f(int rv) { return (size_t)rv + 4; }   // o~ rows, padded against bank conflicts
 
 template <typename T>
-__global__ void __launch_bounds__(kMergeThreads) k_merge(const float* part_o, const float* part_ml,
-                                                         const float* win_o, const float* win_ml,
-                                                         const void* Bv, void* out, float* lse, int S, int Hq,
-                                                         int Hkv, int d, int D, int rv) {
+__global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
   extern __shared__ __align__(16) uint8_t msm[];
   constexpr int es = sizeof(T);
-  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int h = j / (Hq / Hkv);
-  const int pitch = d * es;
-  const int rows_staged = min(rv, (int)(kMergeStage / pitch));
-  uint8_t* bs = msm;                                                   // [rows_staged][d]
-  float* ot = reinterpret_cast<float*>(msm + (size_t)rows_staged * pitch);   // [rv]
-  float* w_s = ot + rv;                                                // [S]
-  float* hdr = w_s + S;                                                // m*, 1/l, window weight
-  stage_rows(bs, pitch, Bv, D, es, 0, rows_staged, (long long)h * d, d);   // bases: stable data
+  const int cb = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int G = a.Hq / a.Hkv, S = a.S, rv = a.rv;
+  const int c0 = cb * kMergeCols, ncols = min(kMergeCols, a.d - c0);
+  const int opitch = rv + 4;
+  uint8_t* bs = msm;                                                          // [rv][ncols]
+  float* ot = reinterpret_cast<float*>(msm + (size_t)rv * kMergeCols * es);   // [8][rv + 4]
+  float* wsm = ot + kMergeHeads * opitch;                                     // [8][S]
+  float* red = wsm + kMergeHeads * S;                                         // [4][8][32]
+  float* hdr = red + 4 * kMergeHeads * kMergeCols;                            // [8][3]
+  stage_rows(bs, ncols * es, a.Bv, a.D, es, 0, rv, (long long)h * a.d + c0, ncols);   // stable data
   pdl_wait();
   pdl_trigger();
-  if (tid < 32) {
-    const int lane = tid;
-    float m = -INFINITY;
-    for (int s = lane; s < S; s += 32) m = fmaxf(m, part_ml[(((size_t)b * S + s) * Hq + j) * 2]);
-    const float mw = win_ml ? win_ml[((size_t)b * Hq + j) * 2] : -INFINITY;
-    m = fmaxf(m, mw);
+  // projection roles: 4 columns x head x quarter of the ranks
+  const int cq = tid & 7, hh = (tid >> 3) & 7, rq = tid >> 6;
+  const int rper = ((rv + 15) / 16) * 4;            // ranks per quarter, multiple of 4
+  const int i0 = rq * rper, i1 = min(rv, i0 + rper);
+  bool staged = false;
+  for (int jb = 0; jb < G; jb += kMergeHeads) {
+    const int nh = min(kMergeHeads, G - jb);
+    // split weights, one warp per head
+    if (warp < nh) {
+      const int j = h * G + jb + warp;
+      float m = -INFINITY;
+      for (int s = lane; s < S; s += 32) m = fmaxf(m, a.part_ml[(((size_t)b * S + s) * a.Hq + j) * 2]);
+      const float mw = a.win_ml ? a.win_ml[((size_t)b * a.Hq + j) * 2] : -INFINITY;
+      m = fmaxf(m, mw);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float l = 0.f;
-    for (int s = lane; s < S; s += 32) {
-      const size_t e = (((size_t)b * S + s) * Hq + j) * 2;
-      const float ms = part_ml[e];
-      const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - m);
-      w_s[s] = w;
-      l = fmaf(w, part_ml[e + 1], l);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) {
-      float ww = 0.f;
-      if (win_ml && mw != -INFINITY) {
-        ww = exp2f(mw - m);
-        l = fmaf(ww, win_ml[((size_t)b * Hq + j) * 2 + 1], l);
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float l = 0.f;
+      for (int s = lane; s < S; s += 32) {
+        const size_t e = (((size_t)b * S + s) * a.Hq + j) * 2;
+        const float ms = a.part_ml[e];
+        const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - m);
+        wsm[warp * S + s] = w;
+        l = fmaf(w, a.part_ml[e + 1], l);
       }
-      hdr[0] = m;
-      hdr[1] = 1.0f / l;
-      hdr[2] = ww;
-      if (lse) lse[(size_t)b * Hq + j] = (m + log2f(l)) * LR_LN2;
-    }
-  }
-  __syncthreads();
-  const size_t sstride = (size_t)Hq * rv;
-  for (int i = tid; i < rv; i += blockDim.x) {
-    const float* src = part_o + ((size_t)b * S * Hq + j) * rv + i;
-    float acc = 0.f;
-    for (int s0 = 0; s0 < S; s0 += 8) {
-      float v[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = (s0 + k < S) ? __ldg(src + k * sstride) : 0.f;
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      if (lane == 0) {
+        float ww = 0.f;
+        if (a.win_ml && mw != -INFINITY) {
+          ww = exp2f(mw - m);
+          l = fmaf(ww, a.win_ml[((size_t)b * a.Hq + j) * 2 + 1], l);
+        }
+        hdr[warp * 3 + 0] = m;
+        hdr[warp * 3 + 1] = 1.0f / l;
+        hdr[warp * 3 + 2] = ww;
+        if (a.lse && cb == 0) a.lse[(size_t)b * a.Hq + j] = (m + log2f(l)) * LR_LN2;
+      }
+    }
+    __syncthreads();
+    // combined rank-space outputs, thread = rank
+    const size_t sstride = (size_t)a.Hq * rv;
+    for (int u = 0; u < nh; ++u) {
+      const int j = h * G + jb + u;
+      for (int i = tid; i < rv; i += kMergeThreads) {
+        const float* src = a.part_o + ((size_t)b * S * a.Hq + j) * rv + i;
+        float acc = 0.f;
+        for (int s0 = 0; s0 < S; s0 += 8) {
+          float v[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (s0 + k < S) acc = fmaf(w_s[s0 + k], v[k], acc);
-      src += 8 * sstride;
+          for (int k = 0; k < 8; ++k) v[k] = (s0 + k < S) ? __ldg(src + k * sstride) : 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (s0 + k < S) acc = fmaf(wsm[u * S + s0 + k], v[k], acc);
+          src += 8 * sstride;
+        }
+        ot[u * opitch + i] = acc;
+      }
     }
-    ot[i] = acc;
-  }
-  cp_async_wait_all();
-  __syncthreads();
-  const size_t ooff = ((size_t)b * Hq + j) * d;
-  for (int c = 2 * tid; c < d; c += 2 * blockDim.x) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    int i = 0;
-    for (; i + 4 <= rows_staged; i += 4) {
-      const float4 o4 = *reinterpret_cast<const float4*>(ot + i);
-      const uint8_t* p0 = bs + (size_t)i * pitch + (size_t)c * es;
-      a0 = fmaf(o4.x, El<T>::lds1(p0), a0);
-      a1 = fmaf(o4.x, El<T>::lds1(p0 + es), a1);
-      a2 = fmaf(o4.y, El<T>::lds1(p0 + pitch), a2);
-      a3 = fmaf(o4.y, El<T>::lds1(p0 + pitch + es), a3);
-      a0 = fmaf(o4.z, El<T>::lds1(p0 + 2 * pitch), a0);
-      a1 = fmaf(o4.z, El<T>::lds1(p0 + 2 * pitch + es), a1);
-      a2 = fmaf(o4.w, El<T>::lds1(p0 + 3 * pitch), a2);
-      a3 = fmaf(o4.w, El<T>::lds1(p0 + 3 * pitch + es), a3);
+    if (!staged) {
+      cp_async_wait_all();
+      staged = true;
     }
-    for (; i < rv; ++i) {
-      const float b0 = i < rows_staged ? El<T>::lds1(bs + (size_t)i * pitch + (size_t)c * es)
-                                       : El<T>::ld(Bv, (size_t)i * D + (size_t)h * d + c);
-      const float b1 = i < rows_staged ? El<T>::lds1(bs + (size_t)i * pitch + (size_t)(c + 1) * es)
-                                       : El<T>::ld(Bv, (size_t)i * D + (size_t)h * d + c + 1);
-      a0 = fmaf(ot[i], b0, a0);
-      a1 = fmaf(ot[i], b1, a1);
+    __syncthreads();
+    // projection partial sums over this thread's quarter of the ranks
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (hh < nh && 4 * cq < ncols) {
+      const float* orow = ot + hh * opitch;
+      for (int i = i0; i < i1; i += 4) {
+        const float4 o4 = *reinterpret_cast<const float4*>(orow + i);
+        const float ov[4] = {o4.x, o4.y, o4.z, o4.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (i + k < i1) {
+            float bv[4];
+            const uint8_t* bp = bs + ((size_t)(i + k) * ncols + 4 * cq) * es;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) bv[e] = El<T>::lds1(bp + e * es);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[e] = fmaf(ov[k], bv[e], acc[e]);
+          }
+        }
+      }
     }
-    float o0 = a0 + a2, o1 = a1 + a3;
-    if (win_o) {
-      o0 = fmaf(hdr[2], win_o[ooff + c], o0);
-      o1 = fmaf(hdr[2], win_o[ooff + c + 1], o1);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) red[(rq * kMergeHeads + hh) * kMergeCols + 4 * cq + e] = acc[e];
+    __syncthreads();
+    // quarters added in order; window partial; normalisation; store
+    {
+      const int u = tid >> 5, c = tid & 31;
+      if (u < nh && c < ncols) {
+        const int j = h * G + jb + u;
+        float o = ((red[(0 * kMergeHeads + u) * kMergeCols + c] + red[(1 * kMergeHeads + u) * kMergeCols + c]) +
+                   red[(2 * kMergeHeads + u) * kMergeCols + c]) +
+                  red[(3 * kMergeHeads + u) * kMergeCols + c];
+        const size_t oi = ((size_t)b * a.Hq + j) * a.d + c0 + c;
+        if (a.win_o) o = fmaf(hdr[u * 3 + 2], a.win_o[oi], o);
+        El<T>::st(a.out, oi, o * hdr[u * 3 + 1]);
+      }
     }
-    El<T>::st(out, ooff + c, o0 * hdr[1]);
-    El<T>::st(out, ooff + c + 1, o1 * hdr[1]);
+    __syncthreads();
   }
 }
 
 size_t merge_smem(const lr_cache_desc& d, int S, size_t es) {
-  const size_t pitch = (size_t)d.head_dim * es;
-  const size_t rows = std::min((size_t)d.rank_v, kMergeStage / pitch);
-  return rows * pitch + ((size_t)d.rank_v + S + 4) * sizeof(float);
+  return (size_t)d.rank_v * kMergeCols * es +
+         ((size_t)kMergeHeads * merge_pitch_f(d.rank_v) + (size_t)kMergeHeads * S +
+          4 * kMergeHeads * kMergeCols + kMergeHeads * 3) * sizeof(float);
 }
 
 // ---- argument construction ------------------------------------------------------------
@@ -422,7 +454,7 @@ AppendArgs make_append_args(const lr_cache* c, const void* k, const void* v) {
   a.params_k = c->params_k; a.params_v = c->params_v;
   a.rk = d.rank_k; a.rv = d.rank_v; a.Gk = c->G_k; a.Gv = c->G_v;
   a.chunks_k = (d.rank_k + 31) / 32; a.chunks_v = (d.rank_v + 31) / 32;
-  a.cap = d.capacity; a.dst_slot = c->hist_len;
+  a.cap = c->lat_cap; a.dst_slot = c->hist_len;
   a.new_k = win ? k : nullptr; a.new_v = win ? v : nullptr;
   a.win_k = c->win_k; a.win_v = c->win_v; a.slots = c->win_slots;
   a.new_slot = win ? (c->len % c->win_slots) : 0;
@@ -453,9 +485,22 @@ cudaError_t merge_t(const lr_cache* c, int n_splits, void* out, float* lse, cuda
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_merge<T>, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_merge<T>, dim3(d.n_q_heads, d.batch), dim3(kMergeThreads), smem, s, c->part_o, c->part_ml,
-                    win ? c->win_o : nullptr, win ? c->win_ml : nullptr, c->B_v, out, lse, n_splits, d.n_q_heads,
-                    d.n_kv_heads, d.head_dim, c->D, d.rank_v);
+  MergeArgs a;
+  a.part_o = c->part_o;
+  a.part_ml = c->part_ml;
+  a.win_o = win ? c->win_o : nullptr;
+  a.win_ml = win ? c->win_ml : nullptr;
+  a.Bv = c->B_v;
+  a.out = out;
+  a.lse = lse;
+  a.S = n_splits;
+  a.Hq = d.n_q_heads;
+  a.Hkv = d.n_kv_heads;
+  a.d = d.head_dim;
+  a.D = c->D;
+  a.rv = d.rank_v;
+  const int cbs = (d.head_dim + kMergeCols - 1) / kMergeCols;
+  return launch_pdl(k_merge<T>, dim3(cbs, d.n_kv_heads, d.batch), dim3(kMergeThreads), smem, s, a);
 }
 
 template <typename T>

@@ -74,6 +74,7 @@ extern "C" lr_status lr_attn_decode_noalloc(const lr_cache_desc* desc, int32_t l
   c.D = desc->n_kv_heads * desc->head_dim;
   c.G_k = c.G_v = 0;
   c.win_slots = 0;
+  c.lat_cap = desc->capacity;
   c.len = c.hist_len = len;
   c.win_len = 0;
   c.esize = desc->dtype == LR_BF16 ? 2 : 4;

@@ -251,7 +251,7 @@ LatentRef latent_ref(const lr_cache* c, bool k) {
   L.params = k ? c->params_k : c->params_v;
   L.r = k ? c->desc.rank_k : c->desc.rank_v;
   L.G = k ? c->G_k : c->G_v;
-  L.cap = c->desc.capacity;
+  L.cap = c->lat_cap;
   return L;
 }
 
@@ -313,7 +313,7 @@ cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, 
   if (e != cudaSuccess) return e;
   return launch_pdl(k_append_latent, grid, dim3(256), 0, s, zk, zv, n, d.batch, d.rank_k, d.rank_v, chunks_k, chunks_v, c->z_k,
                                        c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->G_k,
-                                       c->G_v, d.capacity, c->hist_len, c->latent_kind, d.dtype);
+                                       c->G_v, c->lat_cap, c->hist_len, c->latent_kind, d.dtype);
 }
 
 cudaError_t launch_sync_simt(lr_cache* c, const float* R, int which, cudaStream_t s) {

@@ -160,6 +160,8 @@ lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void
   c->G_k = d.quant_bits == 4 ? (d.rank_k + 31) / 32 : 0;
   c->G_v = d.quant_bits == 4 ? (d.rank_v + 31) / 32 : 0;
   c->win_slots = d.window > 0 ? d.window + 1 : 0;
+  c->lat_cap = c->latent_kind == LK_INT4 ? ((long long)d.capacity + kI4Block - 1) / kI4Block * kI4Block
+                                         : (long long)d.capacity;
   c->len = c->hist_len = c->win_len = 0;
   const float sm_scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / std::sqrt((float)d.head_dim);
   c->scale_log2 = sm_scale * LR_LOG2E;
@@ -171,12 +173,11 @@ lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void
   const size_t B = d.batch, cap = d.capacity, es = c->esize, D = c->D;
   if (e == cudaSuccess) {
     if (c->latent_kind == LK_INT4) {
-      e = dalloc(&c->codes_k, B * cap * c->G_k * 4 * sizeof(uint32_t));
-      if (e == cudaSuccess) e = dalloc(&c->codes_v, B * cap * c->G_v * 4 * sizeof(uint32_t));
-      // params get 64 bytes of tail padding: the tensor-core decode copies 16-byte
-      // aligned spans that may reach up to 15 bytes past the last row
-      if (e == cudaSuccess) e = dalloc(&c->params_k, B * cap * c->G_k * sizeof(uint32_t) + 64);
-      if (e == cudaSuccess) e = dalloc(&c->params_v, B * cap * c->G_v * sizeof(uint32_t) + 64);
+      const size_t rows = B * (size_t)c->lat_cap;
+      e = dalloc(&c->codes_k, rows * c->G_k * 4 * sizeof(uint32_t));
+      if (e == cudaSuccess) e = dalloc(&c->codes_v, rows * c->G_v * 4 * sizeof(uint32_t));
+      if (e == cudaSuccess) e = dalloc(&c->params_k, rows * c->G_k * sizeof(uint32_t));
+      if (e == cudaSuccess) e = dalloc(&c->params_v, rows * c->G_v * sizeof(uint32_t));
     } else {
       e = dalloc(&c->z_k, B * cap * d.rank_k * es);
       if (e == cudaSuccess) e = dalloc(&c->z_v, B * cap * d.rank_v * es);
@@ -392,6 +393,8 @@ lr_status lr_cache_view_get(const lr_cache* c, lr_cache_view* v) {
   v->A_k = c->A_k; v->B_k = c->B_k; v->A_v = c->A_v; v->B_v = c->B_v;
   v->groups_k = c->G_k; v->groups_v = c->G_v;
   v->capacity = c->desc.capacity; v->window_slots = c->win_slots;
+  v->int4_blocks = c->latent_kind == LK_INT4 ? (int32_t)(c->lat_cap / kI4Block) : 0;
+  v->reserved = 0;
   return LR_OK;
 }
 

@@ -17,11 +17,23 @@
 // Latent storage kinds.
 enum LatentKind { LK_F32 = 0, LK_BF16 = 1, LK_INT4 = 2 };
 
+// Int4 storage: blocks of 128 tokens, group-major inside a block.  A latent row is
+// b * lat_cap + slot (lat_cap = capacity rounded up to 128), so row >> 7 is the block
+// and row & 127 the token inside it.
+constexpr int kI4Block = 128;
+__host__ __device__ __forceinline__ long long i4_code_index(long long row, int G, int g, int w) {
+  return ((((row >> 7) * G + g) << 9) + ((row & 127) << 2)) + w;
+}
+__host__ __device__ __forceinline__ long long i4_param_index(long long row, int G, int g) {
+  return (((row >> 7) * G + g) << 7) + (row & 127);
+}
+
 struct lr_cache {
   lr_cache_desc desc;
   int D;                 // n_kv_heads * head_dim
   int G_k, G_v;          // int4 groups per token (0 when unquantised)
   int win_slots;         // window + 1 (ring), or 0
+  long long lat_cap;     // latent rows per sequence: capacity (int4: rounded up to 128)
   int32_t len, hist_len, win_len;
   int32_t stable_len = 0; // history rows [0, stable_len) were written before the kernel that
                           // precedes the decode (the decode may read them before its
@@ -62,8 +74,8 @@ struct lr_cache {
 
 struct LatentRef {
   const void* z;          // unquantised [B][cap][r]
-  const uint32_t* codes;  // int4 [B][cap][G*4]
-  const uint32_t* params; // int4 [B][cap][G]
+  const uint32_t* codes;  // int4, blocked (i4_code_index)
+  const uint32_t* params; // int4, blocked (i4_param_index)
   int r, G;
   long long cap;
 };

@@ -125,6 +125,19 @@ def fill_cache(lr, p: synth.Problem, capacity: Optional[int] = None, chunk: int 
     return c
 
 
+def int4_token_major(lr, view, batch: int, which: str):
+    """Copy a cache's int4 storage of K ("k") or V ("v") to the host and rearrange it from
+    the blocked device layout ([B][blocks][G][128][4] codes, [B][blocks][G][128] params)
+    to token-major ([B][tokens][G*4], [B][tokens][G]), the layout of the oracle's packer."""
+    nb = view.int4_blocks
+    G = view.groups_k if which == "k" else view.groups_v
+    codes = lr.copy_view(view.codes_k if which == "k" else view.codes_v, (batch, nb, G, 128, 4), "<i4")
+    params = lr.copy_view(view.params_k if which == "k" else view.params_v, (batch, nb, G, 128), "<i4")
+    c = codes.cpu().numpy().view(np.uint32).transpose(0, 1, 3, 2, 4).reshape(batch, nb * 128, G * 4)
+    pr = params.cpu().numpy().view(np.uint32).transpose(0, 1, 3, 2).reshape(batch, nb * 128, G)
+    return c, pr
+
+
 def gpu_decode(lr, p: synth.Problem, cache, q: Optional[np.ndarray] = None, with_lse=True):
     import torch
     qd = to_dev(p, p.q if q is None else q)

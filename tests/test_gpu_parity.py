@@ -90,11 +90,8 @@ def test_tiny_from_exact_keys_via_append(lib):
 
 def _read_int4(lib, p, c, n):
     v = lib.lr_cache_view_get(c)
-    cap = v.capacity
-    ck = lib.copy_view(v.codes_k, (p.batch, cap, v.groups_k * 4), "<i4").cpu().numpy().view(np.uint32)
-    pk = lib.copy_view(v.params_k, (p.batch, cap, v.groups_k), "<i4").cpu().numpy().view(np.uint32)
-    cv = lib.copy_view(v.codes_v, (p.batch, cap, v.groups_v * 4), "<i4").cpu().numpy().view(np.uint32)
-    pv = lib.copy_view(v.params_v, (p.batch, cap, v.groups_v), "<i4").cpu().numpy().view(np.uint32)
+    ck, pk = H.int4_token_major(lib, v, p.batch, "k")
+    cv, pv = H.int4_token_major(lib, v, p.batch, "v")
     return ck[:, :n], pk[:, :n], cv[:, :n], pv[:, :n]
 
 
@@ -138,8 +135,8 @@ def test_int4_quantiser_edge_cases_bit_exact(lib):
     zt = torch.from_numpy(z).cuda()
     lib.lr_kv_append_latent(c, zt, zt)
     v = lib.lr_cache_view_get(c)
-    codes = lib.copy_view(v.codes_k, (1, v.capacity, v.groups_k * 4), "<i4").cpu().numpy().view(np.uint32)[:, :n]
-    params = lib.copy_view(v.params_k, (1, v.capacity, v.groups_k), "<i4").cpu().numpy().view(np.uint32)[:, :n]
+    codes, params = H.int4_token_major(lib, v, 1, "k")
+    codes, params = codes[:, :n], params[:, :n]
     w, s, zz = quant.quantize_and_pack(z)
     assert np.array_equal(codes, w)
     assert np.array_equal(params, _params_word(s, zz))
@@ -171,8 +168,8 @@ def test_append_projection_and_quantiser_agree(lib):
     bound = 1e-6 * np.abs(ks).transpose(1, 0, 2) @ np.abs(A) + 1e-30
     assert np.all(np.abs(zk - ref) <= bound * 8)
     vq = lib.lr_cache_view_get(caches[4])
-    codes = lib.copy_view(vq.codes_k, (Bsz, vq.capacity, vq.groups_k * 4), "<i4").cpu().numpy().view(np.uint32)[:, :n]
-    params = lib.copy_view(vq.params_k, (Bsz, vq.capacity, vq.groups_k), "<i4").cpu().numpy().view(np.uint32)[:, :n]
+    codes, params = H.int4_token_major(lib, vq, Bsz, "k")
+    codes, params = codes[:, :n], params[:, :n]
     w, s, zz = quant.quantize_and_pack(zk)
     assert np.array_equal(codes, w) and np.array_equal(params, _params_word(s, zz))
     assert lib.lr_cache_get_len(caches[4]) == (n, n, 0)
