@@ -44,11 +44,24 @@ FALLBACK_HBM_GBS = 6650.0
 WORKLOADS = {
     "qwen4k": dict(desc="Qwen2.5-VL-7B layer: B=16, Hq=28, Hkv=4, d=128, T=4096, r_k=r_v=256 bf16 latents",
                    batch=16, n_q_heads=28, n_kv_heads=4, head_dim=128, rank=256, length=4096,
-                   quant_bits=0),
+                   quant_bits=0, layers=1),
     "qwen16k": dict(desc="Qwen2.5-VL-7B layer: B=16, Hq=28, Hkv=4, d=128, T=16384, r=352 int4 g32 latents",
                     batch=16, n_q_heads=28, n_kv_heads=4, head_dim=128, rank=352, length=16384,
-                    quant_bits=4),
+                    quant_bits=4, layers=1),
+    "qwen32k": dict(desc="28 Qwen2.5-VL-7B layers: B=16, Hq=28, Hkv=4, d=128, T=32768, int4 g32 latents, "
+                         "seeded per-layer ranks in [128, 448] (mean 256), keys stored after RoPE",
+                    batch=16, n_q_heads=28, n_kv_heads=4, head_dim=128, rank=256, length=32768,
+                    quant_bits=4, layers=28),
 }
+
+
+def layer_ranks(workload: str, seed: int = 0):
+    """(r_k, r_v) of every layer of a workload."""
+    import synth
+    W = WORKLOADS[workload]
+    if W["layers"] == 1:
+        return [(W["rank"], W["rank"])]
+    return synth.qwen32k_ranks(seed, W["layers"])
 
 
 def latent_bytes_per_token(rank: int, quant_bits: int) -> int:
@@ -164,30 +177,54 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     W = WORKLOADS[args.workload]
-    Bsz, Hq, Hkv, d, r, T = W["batch"], W["n_q_heads"], W["n_kv_heads"], W["head_dim"], W["rank"], W["length"]
+    Bsz, Hq, Hkv, d, T = W["batch"], W["n_q_heads"], W["n_kv_heads"], W["head_dim"], W["length"]
     qb = W["quant_bits"]
     D = Hkv * d
-
-    # seeded synthetic layer, one seed per rank (independent sequences)
-    p = synth.make_qwen(args.workload, seed=rank, batch=Bsz, length=T - 1, rank=r, quant_bits=qb)
     dev = torch.device("cuda", local)
 
     def to_dev(x):
         return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    desc = lr.make_desc(Bsz, Hq, Hkv, d, r, r, T, quant_bits=qb, dtype=lr.LR_BF16)
-    cache = lr.lr_cache_create(desc, to_dev(p.A_k), to_dev(p.B_k), to_dev(p.A_v), to_dev(p.B_v))
-    chunk = 1024
-    for s in range(0, T - 1, chunk):
-        e = min(T - 1, s + chunk)
-        lr.lr_kv_append_latent(cache, torch.from_numpy(np.ascontiguousarray(p.z_k[:, s:e])).to(dev),
-                               torch.from_numpy(np.ascontiguousarray(p.z_v[:, s:e])).to(dev))
-    kx, vx = synth.hybrid_token(args.workload, rank, T - 1, Bsz, D,
-                                synth.bf16_to_f64(p.B_k), synth.bf16_to_f64(p.B_v))
-    k_h, v_h = synth.bf16_bits(kx), synth.bf16_bits(vx)
-    k_d, v_d, q_d = to_dev(k_h), to_dev(v_h), to_dev(p.q)
-    out = torch.empty_like(q_d)
-    lse = torch.empty((Bsz, Hq), dtype=torch.float32, device=dev)
+    # seeded synthetic layers, one seed per rank (independent sequences).  Single-layer
+    # workloads take their latents from the host generator; the 28-layer one draws them
+    # on the device (same law: N(0,1) x i^-0.7 per rank coordinate) and quantises them
+    # through lr_kv_append_latent.
+    layers = []
+    host_p = None
+    for li, (rk, rv) in enumerate(layer_ranks(args.workload)):
+        hist = T - 1
+        if W["layers"] == 1:
+            p = synth.make_qwen(args.workload, seed=rank, batch=Bsz, length=hist, rank=rk, quant_bits=qb)
+            host_p = p
+        else:
+            p = synth.make_qwen(args.workload, seed=rank, batch=Bsz, length=0, rank=rk, rank_v=rv,
+                                quant_bits=qb, layer=li)
+        desc = lr.make_desc(Bsz, Hq, Hkv, d, rk, rv, T, quant_bits=qb, dtype=lr.LR_BF16)
+        cache = lr.lr_cache_create(desc, to_dev(p.A_k), to_dev(p.B_k), to_dev(p.A_v), to_dev(p.B_v))
+        chunk = 1024 if W["layers"] == 1 else 2048
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1000003 * (rank + 1) + li)
+        sig_k = torch.arange(1, rk + 1, device=dev, dtype=torch.float32).pow(-0.7)
+        sig_v = torch.arange(1, rv + 1, device=dev, dtype=torch.float32).pow(-0.7)
+        for s0 in range(0, hist, chunk):
+            e0 = min(hist, s0 + chunk)
+            if W["layers"] == 1:
+                zk = torch.from_numpy(np.ascontiguousarray(p.z_k[:, s0:e0])).to(dev)
+                zv = torch.from_numpy(np.ascontiguousarray(p.z_v[:, s0:e0])).to(dev)
+            else:
+                zk = torch.randn((Bsz, e0 - s0, rk), generator=gen, device=dev) * sig_k
+                zv = torch.randn((Bsz, e0 - s0, rv), generator=gen, device=dev) * sig_v
+            lr.lr_kv_append_latent(cache, zk, zv)
+        kx, vx = synth.hybrid_token(args.workload, rank * 1000 + li, hist, Bsz, D,
+                                    synth.bf16_to_f64(p.B_k), synth.bf16_to_f64(p.B_v))
+        L = dict(cache=cache, rk=rk, rv=rv, k_h=synth.bf16_bits(kx), v_h=synth.bf16_bits(vx), q_h=p.q)
+        L["k"], L["v"], L["q"] = to_dev(L["k_h"]), to_dev(L["v_h"]), to_dev(L["q_h"])
+        L["out"] = torch.empty_like(L["q"])
+        L["lse"] = torch.empty((Bsz, Hq), dtype=torch.float32, device=dev)
+        L["bytes"] = Bsz * T * (latent_bytes_per_token(rk, qb) + latent_bytes_per_token(rv, qb))
+        layers.append(L)
+    torch.cuda.synchronize()
+    bytes_per_step = sum(L["bytes"] for L in layers)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush_sink = torch.empty((), dtype=torch.int64, device=dev)
 
@@ -197,11 +234,12 @@ def run_ours(args):
         # pays for write-backs of the flush
         flush.zero_()
         torch.sum(flush.view(torch.int64), dim=0, out=flush_sink)
-    plan = lr.lr_cache_plan(cache)
+    plan = lr.lr_cache_plan(layers[0]["cache"])
 
-    def step(kk, vv, qq, oo, ll):
-        lr.lr_decode_step(cache, kk, vv, qq, oo, ll)   # lr_kv_append + lr_attn_decode, fused launches
-        lr.lr_cache_truncate(cache, T - 1)
+    def step():
+        for L in layers:   # lr_kv_append + lr_attn_decode per layer (fused launches)
+            lr.lr_decode_step(L["cache"], L["k"], L["v"], L["q"], L["out"], L["lse"])
+            lr.lr_cache_truncate(L["cache"], T - 1)
 
     def barrier():
         if world > 1:
@@ -210,31 +248,47 @@ def run_ours(args):
 
     for _ in range(args.warmup):
         flush_l2()
-        step(k_d, v_d, q_d, out, lse)
+        step()
     torch.cuda.synchronize()
 
-    # kernel-only events around the main decode kernel (recorded by the library)
-    kev0, kev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    kev0.record(); kev1.record()
+    # Two captures of the same step: `plain` (no event nodes, so consecutive kernels keep
+    # their programmatic-dependent-launch overlap) is timed for the headline value;
+    # `kev` records events around every layer's main decode kernel for the roofline.
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+    for a0, a1 in kev:
+        a0.record(); a1.record()
     torch.cuda.synchronize()
-    lr.lr_cache_set_kernel_events(cache, kev0, kev1)
-    graph = None
     n0 = lr.lr_launch_count()
     if args.graph:
-        # the step is replayed as a CUDA graph: the context is fixed (append at slot T-1,
-        # decode over T tokens, truncate back), so the captured launches are the step
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            step(k_d, v_d, q_d, out, lse)
+        g_plain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_plain):
+            step()
         torch.cuda.synchronize()
-        run = graph.replay
+        launches_per_step = lr.lr_launch_count() - n0
+        for L, (a0, a1) in zip(layers, kev):
+            lr.lr_cache_set_kernel_events(L["cache"], a0, a1)
+        g_kev = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_kev):
+            step()
+        torch.cuda.synchronize()
+        for L in layers:
+            lr.lr_cache_set_kernel_events(L["cache"])
+        run, run_kev = g_plain.replay, g_kev.replay
     else:
-        step(k_d, v_d, q_d, out, lse)
+        step()
         torch.cuda.synchronize()
-        run = lambda: step(k_d, v_d, q_d, out, lse)  # noqa: E731
-    launches_per_step = lr.lr_launch_count() - n0
+        launches_per_step = lr.lr_launch_count() - n0
+
+        def run_kev():
+            for L, (a0, a1) in zip(layers, kev):
+                lr.lr_cache_set_kernel_events(L["cache"], a0, a1)
+            step()
+            for L in layers:
+                lr.lr_cache_set_kernel_events(L["cache"])
+        run = step
     for _ in range(3):
         run()
+        run_kev()
     torch.cuda.synchronize()
 
     uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "")
@@ -242,13 +296,12 @@ def run_ours(args):
     sampler.start()
     t_end = time.time() + args.load_seconds          # sustained load so the sampler sees the
     while time.time() < t_end:                        # clocks of this very step
-        for _ in range(50):
+        for _ in range(max(1, 50 // len(layers))):
             run()
         torch.cuda.synchronize()
 
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    kern_ms = []
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -257,41 +310,49 @@ def run_ours(args):
         ev[i][0].record()
         run()
         ev[i][1].record()
-        kev1.synchronize()
-        kern_ms.append(kev0.elapsed_time(kev1))
     torch.cuda.synchronize()
     barrier()
     launches = launches_per_step * K
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = sum(step_ms)
+    # roofline: the main decode kernel of every layer, timed inside the `kev` capture
+    kern_ms = []
+    for i in range(K):
+        flush_l2()
+        run_kev()
+        torch.cuda.synchronize()
+        kern_ms.append(sum(a0.elapsed_time(a1) for a0, a1 in kev))
 
     # end to end with host buffers (pinned): H2D of the step's inputs, the step through
-    # the public API (replayed graph of lr_kv_append + lr_attn_decode), D2H of the result
-    q_host = torch.from_numpy(np.ascontiguousarray(p.q).view(np.int16)).view(torch.bfloat16).pin_memory()
-    k_host = torch.from_numpy(k_h.view(np.int16)).view(torch.bfloat16).pin_memory()
-    v_host = torch.from_numpy(v_h.view(np.int16)).view(torch.bfloat16).pin_memory()
-    out_host = torch.empty((Bsz, Hq, d), dtype=torch.bfloat16).pin_memory()
-    lse_host = torch.empty((Bsz, Hq), dtype=torch.float32).pin_memory()
+    # the public API (replayed graph of lr_kv_append + lr_attn_decode per layer), D2H of
+    # the results
+    for L in layers:
+        L["q_host"] = torch.from_numpy(np.ascontiguousarray(L["q_h"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        L["k_host"] = torch.from_numpy(L["k_h"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        L["v_host"] = torch.from_numpy(L["v_h"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        L["out_host"] = torch.empty((Bsz, Hq, d), dtype=torch.bfloat16).pin_memory()
+        L["lse_host"] = torch.empty((Bsz, Hq), dtype=torch.float32).pin_memory()
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     torch.cuda.synchronize()
     barrier()
     for i in range(K):
         flush_l2()
         e2e_ev[i][0].record()
-        q_d.copy_(q_host, non_blocking=True)
-        k_d.copy_(k_host, non_blocking=True)
-        v_d.copy_(v_host, non_blocking=True)
+        for L in layers:
+            L["q"].copy_(L["q_host"], non_blocking=True)
+            L["k"].copy_(L["k_host"], non_blocking=True)
+            L["v"].copy_(L["v_host"], non_blocking=True)
         run()
-        out_host.copy_(out, non_blocking=True)
-        lse_host.copy_(lse, non_blocking=True)
+        for L in layers:
+            L["out_host"].copy_(L["out"], non_blocking=True)
+            L["lse_host"].copy_(L["lse"], non_blocking=True)
         e2e_ev[i][1].record()
     torch.cuda.synchronize()
     barrier()
     sampler.stop()
-    lr.lr_cache_set_kernel_events(cache)
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
-    h2d = (q_host.numel() + k_host.numel() + v_host.numel()) * 2
-    d2h = out_host.numel() * 2 + lse_host.numel() * 4
+    h2d = sum((L["q_host"].numel() + L["k_host"].numel() + L["v_host"].numel()) * 2 for L in layers)
+    d2h = sum(L["out_host"].numel() * 2 + L["lse_host"].numel() * 4 for L in layers)
 
     if world > 1:
         import torch.distributed as dist
@@ -299,22 +360,23 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms, e2e_ms = float(t[0]), float(t[1])
 
-    bytes_per_step = Bsz * T * 2 * latent_bytes_per_token(r, qb)
     value = bytes_per_step * K * world / (total_ms * 1e-3) / 1e9
     peaks, peak_src = measured_peaks()
     kern_mean = statistics.mean(kern_ms)
     achieved = bytes_per_step / (kern_mean * 1e-3) / 1e9
-    kname = "decode_tc" if plan.path == lr.LR_PATH_TC else "decode_simt"
-    traf = traffic_record(kname)
+    kname = ("decode_tc_i4" if qb == 4 else "decode_tc") if plan.path == lr.LR_PATH_TC else "decode_simt"
+    traf = traffic_record(f"{kname}:{args.workload}")
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
         "us_per_step": round(1000 * total_ms / K, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int4+bf16" if qb else "bf16",
         "data": "synthetic (seeded; one seed per rank)",
-        "config": {"workload": W["desc"], "batch": Bsz, "context": T, "rank": r,
+        "config": {"workload": W["desc"], "batch": Bsz, "context": T, "layers": len(layers),
+                   "ranks": sorted({rr for L in layers for rr in (L["rk"], L["rv"])}) if len(layers) > 1 else layers[0]["rk"],
                    "quant_bits": qb, "latent_bytes_per_step": bytes_per_step,
-                   "step": "lr_decode_step (= lr_kv_append + lr_attn_decode)", "l2": "flushed before every timed step outside the events (256 MiB written, then read back so L2 holds clean unrelated lines)",
+                   "step": "lr_decode_step (= lr_kv_append + lr_attn_decode) per layer",
+                   "l2": "flushed before every timed step outside the events (256 MiB written, then read back so L2 holds clean unrelated lines)",
                    "parallelism": f"dp{world} (independent sequences per GPU)",
                    "decode_path": "tcgen05" if plan.path == lr.LR_PATH_TC else "simt",
                    "splits": plan.n_splits, "cuda_graph": bool(args.graph),
@@ -323,6 +385,7 @@ def run_ours(args):
                      "peak": peaks.get("hbm_gbs", FALLBACK_HBM_GBS), "peak_source": peak_src,
                      "unit": "GB/s", "frac": round(achieved / peaks.get("hbm_gbs", FALLBACK_HBM_GBS), 4),
                      "kernel_us": round(1000 * kern_mean, 2),
+                     "kernel_timing": "CUDA events around each layer's decode kernel (separate graph capture), summed over layers",
                      "traffic": (traf["bytes_per_launch"] if traf else None)},
         "e2e": {"value": round(bytes_per_step * K * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "us_per_step": round(1000 * e2e_ms / K, 2), "h2d_bytes_per_step": h2d,
@@ -331,11 +394,14 @@ def run_ours(args):
         "clocks": sampler.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(args.workload, p, args.cpu_seconds)
+        res["cpu_baseline"] = cpu_baseline(args.workload, host_p, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(res), flush=True)
-    del graph
-    lr.lr_cache_destroy(cache)
+    run = run_kev = None
+    if args.graph:
+        del g_plain, g_kev
+    for L in layers:
+        lr.lr_cache_destroy(L["cache"])
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -382,22 +448,32 @@ def oracle_step_sample(p, rows, seconds):
             return nbytes / el, el / done, done
 
 
+def host_problem(workload, seed, batch):
+    """A host-side instance of (the first layer of) a workload for the CPU oracle."""
+    import synth
+    W = WORKLOADS[workload]
+    if W["layers"] == 1:
+        return synth.make_qwen(workload, seed=seed, batch=batch, length=W["length"] - 1, rank=W["rank"],
+                               quant_bits=W["quant_bits"])
+    return synth.make_qwen32k_layer(0, seed=seed, batch=batch, length=W["length"] - 1, rope=False)
+
+
 def cpu_baseline(workload, p, seconds):
+    if p is None:
+        p = host_problem(workload, 0, 1)
     bps, s_per_row, n = oracle_step_sample(p, [0], seconds)
     return {"value": round(bps / 1e9, 4), "unit": "GB/s", "cores": _blas_threads(), "kind": "oracle",
             "us_per_step_equiv": round(1e6 * s_per_row * p.batch, 1),
             "sample": f"{n} oracle decodes of batch row 0 (all {p.n_q_heads} heads, T={p.hist_len}) of the "
-                      f"{workload} step, fp64 NumPy; GB/s of latents processed"}
+                      f"{workload} step (first layer), fp64 NumPy; GB/s of latents processed"}
 
 
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    import synth
     W = WORKLOADS[args.workload]
-    p = synth.make_qwen(args.workload, seed=0, batch=W["batch"], length=W["length"] - 1,
-                        rank=W["rank"], quant_bits=W["quant_bits"])
+    p = host_problem(args.workload, 0, 1)
     for _ in range(args.warmup):
         oracle_step_sample(p, [0], 0.0)
     t0 = time.time()

@@ -343,23 +343,34 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
       }
     }
     __syncthreads();
-    // combined rank-space outputs, thread = rank
+    // combined rank-space outputs, thread = rank; two heads at a time with up to 16
+    // splits each in flight, so the L2 round trips overlap
     const size_t sstride = (size_t)a.Hq * rv;
-    for (int u = 0; u < nh; ++u) {
-      const int j = h * G + jb + u;
+    for (int u0 = 0; u0 < nh; u0 += 2) {
+      const bool two = u0 + 1 < nh;
+      const int j0 = h * G + jb + u0;
       for (int i = tid; i < rv; i += kMergeThreads) {
-        const float* src = a.part_o + ((size_t)b * S * a.Hq + j) * rv + i;
-        float acc = 0.f;
-        for (int s0 = 0; s0 < S; s0 += 8) {
-          float v[8];
+        const float* src0 = a.part_o + ((size_t)b * S * a.Hq + j0) * rv + i;
+        const float* src1 = src0 + rv;                       // head j0 + 1
+        float acc0 = 0.f, acc1 = 0.f;
+        for (int s0 = 0; s0 < S; s0 += 16) {
+          float v0[16], v1[16];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) v[k] = (s0 + k < S) ? __ldg(src + k * sstride) : 0.f;
+          for (int k = 0; k < 16; ++k) {
+            const bool in = s0 + k < S;
+            v0[k] = in ? __ldg(src0 + (size_t)(s0 + k) * sstride) : 0.f;
+            v1[k] = (in && two) ? __ldg(src1 + (size_t)(s0 + k) * sstride) : 0.f;
+          }
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if (s0 + k < S) acc = fmaf(wsm[u * S + s0 + k], v[k], acc);
-          src += 8 * sstride;
+          for (int k = 0; k < 16; ++k) {
+            if (s0 + k < S) {
+              acc0 = fmaf(wsm[u0 * S + s0 + k], v0[k], acc0);
+              if (two) acc1 = fmaf(wsm[(u0 + 1) * S + s0 + k], v1[k], acc1);
+            }
+          }
         }
-        ot[u * opitch + i] = acc;
+        ot[u0 * opitch + i] = acc0;
+        if (two) ot[(u0 + 1) * opitch + i] = acc1;
       }
     }
     if (!staged) {
