@@ -7,12 +7,15 @@
 //                                    running max grows by more than 2^8)
 //   O~[e, j] += sum_t z_v,t[e] p[t,j] GEMM2: M = 128 ranks per chunk, N = 64, K = 128 tokens
 // The query latent q~ (scaled by s log2 e) enters GEMM1 as two bf16 halves, hi and
-// lo = q~ - hi, stacked on N (columns 0..31 and 32..63), so the scores carry almost
+// lo = q~ - hi, stacked on N (B rows 0..31 and 32..63), so the scores carry almost
 // fp32 precision while the stored latents stay bf16.  The probabilities enter GEMM2
 // the same way (p = p_hi + p_lo), so the value mix and the normaliser l are both
 // computed from ~fp32 weights; a single bf16 rounding of p would bias l when the
-// weights cluster (near-uniform softmax).  Accumulators live in TMEM: S double-
-// buffered (2 x 64 columns), O~ in ceil(r_v/128) chunks of 64 columns (hi | lo).
+// weights cluster (near-uniform softmax).  One N = 64 MMA costs what an N = 32 MMA
+// costs on this tensor core, so the halves go through N rather than through a second
+// MMA; the softmax and the epilogue add the two 32-column halves of each accumulator.
+// Accumulators live in TMEM: S in 64 columns (hi | lo), O~ in ceil(r_v/128) chunks of
+// 64 columns (hi | lo).
 //
 // Roles (192 threads): warp 0 issues TMA tile loads (128 tokens x 64 ranks boxes,
 // 128-byte swizzle, no multicast) into a ring of 32 KB slots (one 128-rank chunk of
@@ -38,12 +41,11 @@ constexpr int kSubBytes = 128 * 128;       // 128 tokens x 64 ranks x 2 B
 constexpr int kSlotBytes = 2 * kSubBytes;  // 128 tokens x 128 ranks
 constexpr int kQRows = 64;                 // 32 head rows (hi) + 32 head rows (lo)
 constexpr int kQSubBytes = kQRows * 128;   // 64 rows x 64 ranks x 2 B
-constexpr int kQLoOffset = 32 * 128;       // lo rows start 32 rows into each sub-block
 constexpr int kPHalfBytes = 128 * 32 * 2;  // 128 tokens x 32 heads x 2 B (one of hi, lo)
 constexpr int kPBytes = 2 * kPHalfBytes;
 constexpr int kAuxBytes = 1024;            // barriers and reduction scratch, first in smem
-constexpr int kSCol = 0;                   // TMEM: S in columns [0, 32)
-constexpr int kOCol = 32;                  // TMEM: O~ chunk c in columns [32 + 32c, 64 + 32c)
+constexpr int kSCol = 0;                   // TMEM: S in columns [0, 64) (hi | lo)
+constexpr int kOCol = 64;                  // TMEM: O~ chunk c in columns [64 + 64c, 128 + 64c) (hi | lo)
 constexpr int kMaxSlots = 8;
 constexpr int kSmemPair = 115712;          // per block when two blocks share an SM (228 KB - 2 x 1 KB)
 
@@ -75,6 +77,20 @@ struct TcState {
   int ctas_per_sm;
   size_t smem;
 };
+
+// Row `lane_off` of an N = 64 accumulator at column `col`: hi (columns 0..31) + lo
+// (32..63), 16 columns at a time.
+__device__ __forceinline__ void tmem_ld_sum(uint32_t taddr, float (&v)[32]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t a[16], b[16];
+    ptx::tmem_ld16(taddr + 16 * h, a);
+    ptx::tmem_ld16(taddr + 32 + 16 * h, b);
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[16 * h + j] = __uint_as_float(a[j]) + __uint_as_float(b[j]);
+  }
+}
 
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
   return tc::wait_b(bar, parity, &aux->abort_flag, err);
@@ -191,8 +207,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0 && ntiles > 0) {
-      const uint32_t id = ptx::idesc_f16(1, 0, 0, 128, 32);    // GEMM1: K-major x K-major, N = 32
-      const uint32_t id2 = ptx::idesc_f16(1, 1, 1, 128, 32);   // GEMM2: MN-major x MN-major, N = 32
+      const uint32_t id = ptx::idesc_f16(1, 0, 0, 128, 64);    // GEMM1: K-major x K-major, N = 64 (hi | lo)
+      const uint32_t id2 = ptx::idesc_f16(1, 1, 1, 128, 64);   // GEMM2: MN-major x MN-major, N = 64 (hi | lo)
       // Descriptors are built once; a step along K or to another slot adds its byte
       // offset >> 4 to the start-address field (no carry: shared memory < 256 KB).
       const uint64_t kdesc0 = ptx::smem_desc(ptx::smem_u32(ring), 16, 1024, 2);
@@ -218,7 +234,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint64_t ad = a0 + (uint64_t)((kk >> 2) * (kSubBytes >> 4) + (kk & 3) * 2);
             const uint64_t bd = b0 + (uint64_t)((kk >> 2) * (kQSubBytes >> 4) + (kk & 3) * 2);
             ptx::mma_f16(tmem + kSCol, ad, bd, id, (c | kk) ? 1u : 0u);
-            ptx::mma_f16(tmem + kSCol, ad, bd + (uint64_t)(kQLoOffset >> 4), id, 1u);
           }
           ptx::mma_commit(&aux->slot_empty[slot]);
         }
@@ -234,13 +249,12 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
           ptx::tc_fence_after();
           const uint64_t a0 = vdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
-          const uint32_t d_o = tmem + kOCol + c * 32;
+          const uint32_t d_o = tmem + kOCol + c * 64;
 #pragma unroll
           for (int kt = 0; kt < 8; ++kt) {
             const uint64_t ad = a0 + (uint64_t)(kt * 128);
             const uint64_t bd = pdesc0 + (uint64_t)(kt * 16);
             ptx::mma_f16(d_o, ad, bd, id2, (i | kt) ? 1u : 0u);
-            ptx::mma_f16(d_o, ad, bd + (uint64_t)(kPHalfBytes >> 4), id2, 1u);
           }
           ptx::mma_commit(&aux->slot_empty[slot]);
         }
@@ -267,12 +281,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (!ok) break;
       ptx::tc_fence_after();
       if (i < 16 && threadIdx.x == 64) trace_stamp(p, 4 + 4 * i);
-      uint32_t sv[32];
-      ptx::tmem_ld32(tmem + lane_off + kSCol, sv);
-      ptx::tmem_wait_ld();
       float s[32];
+      tmem_ld_sum(tmem + lane_off + kSCol, s);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+      for (int j = 0; j < 32; ++j) s[j] = valid ? s[j] : -INFINITY;
 
       bool ex = false;
 #pragma unroll
@@ -286,10 +298,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (ex) {
         // reduce in place, then read the scores again (S stays intact until s_empty)
         aux->red[qd][lane] = warp_reduce_scatter32<true>(s, lane);
-        ptx::tmem_ld32(tmem + lane_off + kSCol, sv);
-        ptx::tmem_wait_ld();
+        tmem_ld_sum(tmem + lane_off + kSCol, s);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+        for (int j = 0; j < 32; ++j) s[j] = valid ? s[j] : -INFINITY;
         ptx::named_bar_sync(1, 128);
         if (qd == 0) {
           const float mt = fmaxf(fmaxf(aux->red[0][lane], aux->red[1][lane]), fmaxf(aux->red[2][lane], aux->red[3][lane]));
@@ -307,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           need_o |= a < 1.f;
         }
         if (need_o && i > 0) {
-          for (int c = 0; c < p.cv; ++c) {
+          for (int c = 0; c < 2 * p.cv; ++c) {   // both halves of every chunk
             uint32_t v2[32];
             ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
             ptx::tmem_wait_ld();
@@ -352,23 +363,23 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (ok) {
       ptx::tc_fence_after();
       const size_t base_out = ((size_t)b * p.n_splits + split) * p.Hq;
-      for (int c = 0; c < p.cv; ++c) {
-        uint32_t v2[32];
-        ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
-        ptx::tmem_wait_ld();
-        const int e = c * 128 + qd * 32 + lane;
-        if (e < p.r_v) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < p.Hq) p.part_o[(base_out + j) * p.r_v + e] = __uint_as_float(v2[j]);
-        }
-      }
+      // the normaliser first, so its 32 registers are free for the two accumulator halves
       aux->red[qd][lane] = warp_reduce_scatter32<false>(l, lane);
       ptx::named_bar_sync(1, 128);
       if (qd == 0 && lane < p.Hq) {
         const float lt = (aux->red[0][lane] + aux->red[1][lane]) + (aux->red[2][lane] + aux->red[3][lane]);
         p.part_ml[(base_out + lane) * 2] = aux->m_s[lane];
         p.part_ml[(base_out + lane) * 2 + 1] = lt;
+      }
+      for (int c = 0; c < p.cv; ++c) {
+        float o[32];
+        tmem_ld_sum(tmem + lane_off + kOCol + c * 64, o);
+        const int e = c * 128 + qd * 32 + lane;
+        if (e < p.r_v) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < p.Hq) p.part_o[(base_out + j) * p.r_v + e] = o[j];
+        }
       }
       if (threadIdx.x == 64) trace_stamp(p, kTraceSlots - 1);
     }
@@ -397,8 +408,13 @@ size_t smem_for(int r_k, int nslot) { return (size_t)kAuxBytes + q_bytes_for(r_k
 // Two blocks per SM when the block fits half the SM with a 2-slot ring (the streaming
 // rate of two rings per SM is higher than one deeper ring); otherwise one block with
 // as many slots as fit.
+int tmem_cols_for(int r_v) {
+  const int cols = kOCol + 64 * ((r_v + 127) / 128);
+  return cols <= 128 ? 128 : (cols <= 256 ? 256 : 512);
+}
+
 void choose_slots(const lr_cache_desc* d, int* nslot, int* ctas_per_sm) {
-  if (smem_for(d->rank_k, 2) <= (size_t)kSmemPair) {
+  if (smem_for(d->rank_k, 2) <= (size_t)kSmemPair && tmem_cols_for(d->rank_v) <= 256) {
     *nslot = 2;
     *ctas_per_sm = 2;
     return;
@@ -483,7 +499,7 @@ cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, 
   p.ck = (d.rank_k + 127) / 128;
   p.cv = (d.rank_v + 127) / 128;
   p.kb_k = (d.rank_k + 63) / 64;
-  p.tmem_cols = (kOCol + p.cv * 32) <= 128 ? 128 : 256;
+  p.tmem_cols = tmem_cols_for(d.rank_v);
   p.Hq = d.n_q_heads;
   p.hist_len = c->hist_len;
   p.stable_len = std::min(c->stable_len, c->hist_len);

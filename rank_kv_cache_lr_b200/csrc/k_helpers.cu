@@ -56,14 +56,14 @@ struct El<float> {
 };
 
 // ---- query projection -----------------------------------------------------------
-// One CTA per (128 rank rows of B_k,h, KV head h, sequence b); thread = rank row i,
-// for every query head j of the group: q~_j[i] = s log2(e) sum_c B_k[i][h d + c] q_j[c].
+// One CTA per (32 rank rows of B_k,h, KV head h, sequence b), 256 threads; thread =
+// (rank row i, query head j of the group; heads beyond 8 in further passes):
+// q~_j[i] = s log2(e) sum_c B_k[i][h d + c] q_j[c].
 // qt16 (tensor-core path), bf16 latents: rows [b][j] and [b][32 + j] of a [B][64][r_k]
 // bf16 array get hi = bf16(q~) and lo = bf16(q~ - hi), so that hi + lo carries q~ to ~16
 // significant bits.  int4 latents: row [b][j] of a [B][32][r_k] fp16 array gets fp16(q~),
 // each 8-rank run in the order 0,4,1,5,2,6,3,7 in which the int4 kernel expands codes.
-constexpr int kQRowsCta = 128;
-constexpr int kHB = 8;            // query heads per register block
+constexpr int kQRowsCta = 32;
 
 struct QprojArgs {
   const void* q; const void* Bk; float* qt; float* qd; void* qt16;
@@ -101,56 +101,44 @@ __device__ __forceinline__ void qproj_main(const QprojArgs& a, int rchunk, int h
   __syncthreads();
   const int r0 = rchunk * kQRowsCta;
   const int nr = min(kQRowsCta, a.rk - r0);
-  for (int t = threadIdx.x; t < nr; t += blockDim.x) {
-    const uint8_t* row = smem + (size_t)t * pitch;
-    const int i = r0 + t;
-    for (int jb = 0; jb < G; jb += kHB) {
-      float acc[kHB];
-#pragma unroll
-      for (int u = 0; u < kHB; ++u) acc[u] = 0.f;
-      for (int c = 0; c < d; c += 8) {
-        float bv[8];
-        El<T>::lds8(row + (size_t)c * sizeof(T), bv);
-#pragma unroll
-        for (int u = 0; u < kHB; ++u) {
-          if (jb + u < G) {
-            const float4 q0 = *reinterpret_cast<const float4*>(qs + (jb + u) * d + c);
-            const float4 q1 = *reinterpret_cast<const float4*>(qs + (jb + u) * d + c + 4);
-            acc[u] = fmaf(bv[0], q0.x, acc[u]);
-            acc[u] = fmaf(bv[1], q0.y, acc[u]);
-            acc[u] = fmaf(bv[2], q0.z, acc[u]);
-            acc[u] = fmaf(bv[3], q0.w, acc[u]);
-            acc[u] = fmaf(bv[4], q1.x, acc[u]);
-            acc[u] = fmaf(bv[5], q1.y, acc[u]);
-            acc[u] = fmaf(bv[6], q1.z, acc[u]);
-            acc[u] = fmaf(bv[7], q1.w, acc[u]);
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kHB; ++u) {
-        if (jb + u < G) {
-          const int j = j0 + jb + u;
-          const float v = acc[u] * a.scale_log2;
-          a.qt[((size_t)b * a.Hq + j) * a.rk + i] = v;
-          if (a.qt16 && a.qt16_fp16) {
-            const int pos = (i & ~7) | ((i & 3) << 1) | ((i >> 2) & 1);
-            reinterpret_cast<__half*>(a.qt16)[((size_t)b * 32 + j) * a.rk + pos] = __float2half_rn(v);
-          } else if (a.qt16) {
-            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-            __nv_bfloat16* q16 = reinterpret_cast<__nv_bfloat16*>(a.qt16);
-            q16[((size_t)b * 64 + j) * a.rk + i] = hi;
-            q16[((size_t)b * 64 + 32 + j) * a.rk + i] = lo;
-          }
-        }
-      }
+  const int t = threadIdx.x & 31;            // rank row within the chunk
+  const int i = r0 + t;
+  const uint8_t* row = smem + (size_t)t * pitch;
+  for (int u = threadIdx.x >> 5; u < G && t < nr; u += (int)(blockDim.x >> 5)) {
+    const float* qj = qs + u * d;
+    float acc0 = 0.f, acc1 = 0.f;
+    for (int c = 0; c < d; c += 8) {
+      float bv[8];
+      El<T>::lds8(row + (size_t)c * sizeof(T), bv);
+      const float4 q0 = *reinterpret_cast<const float4*>(qj + c);
+      const float4 q1 = *reinterpret_cast<const float4*>(qj + c + 4);
+      acc0 = fmaf(bv[0], q0.x, acc0);
+      acc1 = fmaf(bv[1], q0.y, acc1);
+      acc0 = fmaf(bv[2], q0.z, acc0);
+      acc1 = fmaf(bv[3], q0.w, acc1);
+      acc0 = fmaf(bv[4], q1.x, acc0);
+      acc1 = fmaf(bv[5], q1.y, acc1);
+      acc0 = fmaf(bv[6], q1.z, acc0);
+      acc1 = fmaf(bv[7], q1.w, acc1);
+    }
+    const int j = j0 + u;
+    const float v = (acc0 + acc1) * a.scale_log2;
+    a.qt[((size_t)b * a.Hq + j) * a.rk + i] = v;
+    if (a.qt16 && a.qt16_fp16) {
+      const int pos = (i & ~7) | ((i & 3) << 1) | ((i >> 2) & 1);
+      reinterpret_cast<__half*>(a.qt16)[((size_t)b * 32 + j) * a.rk + pos] = __float2half_rn(v);
+    } else if (a.qt16) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+      __nv_bfloat16* q16 = reinterpret_cast<__nv_bfloat16*>(a.qt16);
+      q16[((size_t)b * 64 + j) * a.rk + i] = hi;
+      q16[((size_t)b * 64 + 32 + j) * a.rk + i] = lo;
     }
   }
 }
 
 template <typename T>
-__global__ void __launch_bounds__(128) k_qproj(QprojArgs a) {
+__global__ void __launch_bounds__(256) k_qproj(QprojArgs a) {
   extern __shared__ __align__(16) uint8_t qsm[];
   qproj_stage<T>(a, blockIdx.x, blockIdx.y, qsm);      // bases: stable data
   pdl_wait();
@@ -483,7 +471,7 @@ cudaError_t qproj_t(const lr_cache* c, const void* q, cudaStream_t s, bool tc) {
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_qproj<T>, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_qproj<T>, dim3(qproj_chunks(c), d.n_kv_heads, d.batch), dim3(128), qproj_smem(d, sizeof(T)), s,
+  return launch_pdl(k_qproj<T>, dim3(qproj_chunks(c), d.n_kv_heads, d.batch), dim3(256), qproj_smem(d, sizeof(T)), s,
                     make_qproj_args(c, q, tc));
 }
 
