@@ -73,9 +73,8 @@ static_assert(sizeof(Aux) <= kAuxBytes, "aux block");
 
 struct TcState {
   CUtensorMap q, zk, zv;
-  int nslot;
-  int ctas_per_sm;
-  size_t smem;
+  int nslot_pair, nslot_single;   // ring slots with two blocks per SM (0: not possible) / with one
+  size_t smem_pair, smem_single;
 };
 
 // Row `lane_off` of an N = 64 accumulator at column `col`: hi (columns 0..31) + lo
@@ -157,10 +156,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0 && ntiles > 0) {
-      // The first tile's key chunks are issued before the grid-dependency wait when
-      // every token of the tile lies below stable_len: those rows were written by
-      // kernels that completed before the preceding kernel allowed this one to start.
-      // The query latents, and rows the preceding kernel appends, come after the wait.
+      // The first round of the ring is issued before the grid-dependency wait when every
+      // token of its tiles lies below stable_len: those rows were written by kernels that
+      // completed before the preceding kernel allowed this one to start.  The query
+      // latents, and rows the preceding kernel appends, come after the wait.
       int issued = 0;
       bool ok = true;
       bool q_issued = false;
@@ -169,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int u = 0; u < per_tile; ++u) {
           const int pos = i * per_tile + u;
           const int slot = pos % p.nslot, round = pos / p.nslot;
-          if (!q_issued && (pos >= p.ck || round > 0 || t0 + kTile > p.stable_len)) {
+          if (!q_issued && (round > 0 || t0 + kTile > p.stable_len)) {
             pdl_wait();
             ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
             for (int sb = 0; sb < p.kb_k; ++sb)
@@ -405,24 +404,20 @@ int q_bytes_for(int r_k) { return ((r_k + 63) / 64) * kQSubBytes; }
 
 size_t smem_for(int r_k, int nslot) { return (size_t)kAuxBytes + q_bytes_for(r_k) + (size_t)nslot * kSlotBytes + kPBytes; }
 
-// Two blocks per SM when the block fits half the SM with a 2-slot ring (the streaming
-// rate of two rings per SM is higher than one deeper ring); otherwise one block with
-// as many slots as fit.
 int tmem_cols_for(int r_v) {
   const int cols = kOCol + 64 * ((r_v + 127) / 128);
   return cols <= 128 ? 128 : (cols <= 256 ? 256 : 512);
 }
 
-void choose_slots(const lr_cache_desc* d, int* nslot, int* ctas_per_sm) {
-  if (smem_for(d->rank_k, 2) <= (size_t)kSmemPair && tmem_cols_for(d->rank_v) <= 256) {
-    *nslot = 2;
-    *ctas_per_sm = 2;
-    return;
-  }
+// Ring slots with two blocks per SM (a 2-slot ring in half the SM; 0 if the block does not
+// fit) and with one block per SM (as many slots as fit).
+int slots_pair(const lr_cache_desc* d) {
+  return (smem_for(d->rank_k, 2) <= (size_t)kSmemPair && tmem_cols_for(d->rank_v) <= 256) ? 2 : 0;
+}
+int slots_single(const lr_cache_desc* d) {
   int n = 0;
   while (n + 1 <= kMaxSlots && smem_for(d->rank_k, n + 1) <= (size_t)kSmemLimit) ++n;
-  *nslot = n;
-  *ctas_per_sm = 1;
+  return n;
 }
 
 }  // namespace
@@ -431,16 +426,17 @@ bool tc_supported(const lr_cache_desc* d) {
   if (d->quant_bits == 4) return tc_i4_supported(d);
   if (d->dtype != LR_BF16 || d->quant_bits != 0 || d->rope_in_kernel) return false;
   if (d->n_q_heads > 32) return false;
-  int nslot, cps;
-  choose_slots(d, &nslot, &cps);
-  return nslot >= 1;
+  return slots_single(d) >= 1;
 }
 
-int tc_ctas_per_sm(const lr_cache_desc* d) {
+// Two blocks per SM whenever they fit: each block's tile chain (scores, softmax, value
+// mix) is serial, and a second block overlaps it on the same SM; measured faster than one
+// block with a deep ring both at 4K and at 16K tokens.
+int tc_ctas_per_sm(const lr_cache_desc* d, int hist_len, int num_sms) {
+  (void)hist_len;
+  (void)num_sms;
   if (d->quant_bits == 4) return 1;
-  int nslot, cps;
-  choose_slots(d, &nslot, &cps);
-  return cps;
+  return slots_pair(d) ? 2 : 1;
 }
 
 cudaError_t tc_prepare(lr_cache* c) {
@@ -474,8 +470,10 @@ cudaError_t tc_prepare(lr_cache* c) {
     if (!make_map(side ? &st->zv : &st->zk, side ? c->z_v : c->z_k, 3, dims, strides, box))
       return cudaErrorInvalidValue;
   }
-  choose_slots(&d, &st->nslot, &st->ctas_per_sm);
-  st->smem = smem_for(d.rank_k, st->nslot);
+  st->nslot_pair = slots_pair(&d);
+  st->nslot_single = slots_single(&d);
+  st->smem_pair = smem_for(d.rank_k, st->nslot_pair);
+  st->smem_single = smem_for(d.rank_k, st->nslot_single);
   return cudaSuccess;
 }
 
@@ -500,12 +498,13 @@ cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, 
   p.cv = (d.rank_v + 127) / 128;
   p.kb_k = (d.rank_k + 63) / 64;
   p.tmem_cols = tmem_cols_for(d.rank_v);
+  const bool pair = tc_ctas_per_sm(&d, c->hist_len, c->num_sms) == 2;
   p.Hq = d.n_q_heads;
   p.hist_len = c->hist_len;
   p.stable_len = std::min(c->stable_len, c->hist_len);
   p.split_tokens = split_tokens;
   p.n_splits = n_splits;
-  p.nslot = st->nslot;
+  p.nslot = pair ? st->nslot_pair : st->nslot_single;
   p.q_bytes = q_bytes_for(d.rank_k);
   p.part_o = c->part_o;
   p.part_ml = c->part_ml;
@@ -514,5 +513,6 @@ cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, 
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_decode_tc, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_decode_tc, dim3(n_splits, d.batch), dim3(kThreads), st->smem, s, st->q, st->zk, st->zv, p);
+  return launch_pdl(k_decode_tc, dim3(n_splits, d.batch), dim3(kThreads), pair ? st->smem_pair : st->smem_single, s,
+                    st->q, st->zk, st->zv, p);
 }

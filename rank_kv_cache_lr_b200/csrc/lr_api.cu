@@ -52,7 +52,7 @@ lr_status plan(const lr_cache_desc* d, int hist_len, int num_sms, int path, int 
   if (splits <= 0) {
     // SIMT: about two CTAs per SM; tensor-core path: one wave of its resident blocks
     const int sms = std::max(num_sms, 1);
-    const int target = (p == LR_PATH_TC) ? std::max(1, tc_ctas_per_sm(d) * sms / d->batch)
+    const int target = (p == LR_PATH_TC) ? std::max(1, tc_ctas_per_sm(d, hist_len, sms) * sms / d->batch)
                                          : std::max(1, (2 * sms + d->batch - 1) / d->batch);
     splits = std::min(tiles, target);
   }

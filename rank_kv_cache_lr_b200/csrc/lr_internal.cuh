@@ -108,7 +108,7 @@ size_t decode_simt_smem(const lr_cache* c);
 
 // tensor-core path (k_decode_tc.cu)
 bool tc_supported(const lr_cache_desc* d);
-int tc_ctas_per_sm(const lr_cache_desc* d);   // resident decode blocks per SM
+int tc_ctas_per_sm(const lr_cache_desc* d, int hist_len, int num_sms);   // decode blocks per SM
 cudaError_t tc_prepare(lr_cache* c);
 void tc_release(lr_cache* c);
 cudaError_t launch_qproj_tc(const lr_cache* c, const void* q, cudaStream_t s);
