@@ -6,6 +6,8 @@
 //   p[t, j]  = exp2(S[t, j] - m_j)   online softmax, lazy max (rescale only when the
 //                                    running max grows by more than 2^8)
 //   O~[e, j] += sum_t z_v,t[e] p[t,j] GEMM2: M = 128 ranks per chunk, N = 64, K = 128 tokens
+// The ring and the MMAs follow the order K(0), K(1), V(0), K(2), V(1), ..., so the scores
+// of tile s+1 are computed while the softmax of tile s runs (S double-buffered in TMEM).
 // The query latent q~ (scaled by s log2 e) enters GEMM1 as two bf16 halves, hi and
 // lo = q~ - hi, stacked on N (B rows 0..31 and 32..63), so the scores carry almost
 // fp32 precision while the stored latents stay bf16.  The probabilities enter GEMM2
@@ -14,8 +16,8 @@
 // weights cluster (near-uniform softmax).  One N = 64 MMA costs what an N = 32 MMA
 // costs on this tensor core, so the halves go through N rather than through a second
 // MMA; the softmax and the epilogue add the two 32-column halves of each accumulator.
-// Accumulators live in TMEM: S in 64 columns (hi | lo), O~ in ceil(r_v/128) chunks of
-// 64 columns (hi | lo).
+// Accumulators live in TMEM: S in two buffers of 64 columns (hi | lo), O~ in
+// ceil(r_v/128) chunks of 64 columns (hi | lo).
 //
 // Roles (192 threads): warp 0 issues TMA tile loads (128 tokens x 64 ranks boxes,
 // 128-byte swizzle, no multicast) into a ring of 32 KB slots (one 128-rank chunk of
@@ -44,8 +46,8 @@ constexpr int kQSubBytes = kQRows * 128;   // 64 rows x 64 ranks x 2 B
 constexpr int kPHalfBytes = 128 * 32 * 2;  // 128 tokens x 32 heads x 2 B (one of hi, lo)
 constexpr int kPBytes = 2 * kPHalfBytes;
 constexpr int kAuxBytes = 1024;            // barriers and reduction scratch, first in smem
-constexpr int kSCol = 0;                   // TMEM: S in columns [0, 64) (hi | lo)
-constexpr int kOCol = 64;                  // TMEM: O~ chunk c in columns [64 + 64c, 128 + 64c) (hi | lo)
+constexpr int kSCol = 0;                   // TMEM: S of tile s in columns [64 (s % 2), +64) (hi | lo)
+constexpr int kOCol = 128;                 // TMEM: O~ chunk c in columns [128 + 64c, +64) (hi | lo)
 constexpr int kMaxSlots = 8;
 constexpr int kSmemPair = 115712;          // per block when two blocks share an SM (228 KB - 2 x 1 KB)
 
@@ -62,7 +64,8 @@ struct TcParams {
 struct Aux {
   uint64_t slot_full[kMaxSlots];
   uint64_t slot_empty[kMaxSlots];
-  uint64_t q_full, s_full, s_empty, p_full, p_empty, o_final;
+  uint64_t s_full[2], s_empty[2];
+  uint64_t q_full, p_full, p_empty, o_final;
   uint32_t tmem_base;
   int abort_flag;
   float red[4][32];
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int tok_begin = split * p.split_tokens;
   const int tok_end = min(p.hist_len, tok_begin + p.split_tokens);
   const int ntiles = tok_end > tok_begin ? (tok_end - tok_begin + kTile - 1) / kTile : 0;
-  const int per_tile = p.ck + p.cv;
+  const int nunits = 2 * ntiles;
 
   if (threadIdx.x == 0) {
     trace_stamp(p, 0);
@@ -127,8 +130,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       ptx::mbar_init(&aux->slot_empty[s], 1);
     }
     ptx::mbar_init(&aux->q_full, 1);
-    ptx::mbar_init(&aux->s_full, 1);
-    ptx::mbar_init(&aux->s_empty, 128);
+    for (int k = 0; k < 2; ++k) {
+      ptx::mbar_init(&aux->s_full[k], 1);
+      ptx::mbar_init(&aux->s_empty[k], 128);
+    }
     ptx::mbar_init(&aux->p_full, 128);
     ptx::mbar_init(&aux->p_empty, 1);
     ptx::mbar_init(&aux->o_final, 1);
@@ -160,13 +165,17 @@ __global__ void __launch_bounds__(kThreads, 2)
       // token of its tiles lies below stable_len: those rows were written by kernels that
       // completed before the preceding kernel allowed this one to start.  The query
       // latents, and rows the preceding kernel appends, come after the wait.
-      int issued = 0;
+      int issued = 0, pos = 0;
       bool ok = true;
       bool q_issued = false;
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const int t0 = tok_begin + i * kTile;
-        for (int u = 0; u < per_tile; ++u) {
-          const int pos = i * per_tile + u;
+      for (int u = 0; u < nunits && ok; ++u) {
+        int tile;
+        bool isv;
+        tc::unit_of(u, ntiles, &tile, &isv);
+        const int t0 = tok_begin + tile * kTile;
+        const int nch = isv ? p.cv : p.ck;
+        const int r = isv ? p.r_v : p.r_k;
+        for (int c = 0; c < nch; ++c, ++pos) {
           const int slot = pos % p.nslot, round = pos / p.nslot;
           if (!q_issued && (round > 0 || t0 + kTile > p.stable_len)) {
             pdl_wait();
@@ -179,14 +188,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             ok = false;
             break;
           }
-          const bool isk = u < p.ck;
-          const int c = isk ? u : u - p.ck;
-          const int r = isk ? p.r_k : p.r_v;
           const int nsub = (c * 128 + 64 < r) ? 2 : 1;
           uint8_t* dst = ring + slot * kSlotBytes;
           ptx::mbar_arrive_expect_tx(&aux->slot_full[slot], nsub * kSubBytes);
           for (int sb = 0; sb < nsub; ++sb)
-            ptx::tma_load_3d(dst + sb * kSubBytes, isk ? &tm_zk : &tm_zv, &aux->slot_full[slot],
+            ptx::tma_load_3d(dst + sb * kSubBytes, isv ? &tm_zv : &tm_zk, &aux->slot_full[slot],
                              c * 128 + sb * 64, t0, b);
           issued = pos + 1;
         }
@@ -217,49 +223,56 @@ __global__ void __launch_bounds__(kThreads, 2)
       bool ok = wait_b(&aux->q_full, 0, aux, p.err);
       ptx::tc_fence_after();
       trace_stamp(p, 2);
-      for (int i = 0; i < ntiles && ok; ++i) {
-        // GEMM1: S = Z_k q~_hi^T + Z_k q~_lo^T (the two halves accumulate in place)
-        if (i >= 1 && !(ok = wait_b(&aux->s_empty, (i - 1) & 1, aux, p.err))) break;
-        ptx::tc_fence_after();
-        for (int c = 0; c < p.ck && ok; ++c) {
-          const int pos = i * per_tile + c;
-          const int slot = pos % p.nslot;
-          if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+      int pos = 0;
+      for (int u = 0; u < nunits && ok; ++u) {
+        int tile;
+        bool isv;
+        tc::unit_of(u, ntiles, &tile, &isv);
+        if (!isv) {
+          // GEMM1(tile): S[tile % 2] = Z_k [q~_hi | q~_lo]^T
+          const int sb2 = tile & 1;
+          if (tile >= 2 && !(ok = wait_b(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
           ptx::tc_fence_after();
-          const uint64_t a0 = kdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
-          const uint64_t b0 = qdesc0 + (uint64_t)((c * 2 * kQSubBytes) >> 4);
-          const int nk = min(8, (p.r_k - c * 128) >> 4);
-          for (int kk = 0; kk < nk; ++kk) {
-            const uint64_t ad = a0 + (uint64_t)((kk >> 2) * (kSubBytes >> 4) + (kk & 3) * 2);
-            const uint64_t bd = b0 + (uint64_t)((kk >> 2) * (kQSubBytes >> 4) + (kk & 3) * 2);
-            ptx::mma_f16(tmem + kSCol, ad, bd, id, (c | kk) ? 1u : 0u);
+          const uint32_t d_s = tmem + kSCol + 64 * sb2;
+          for (int c = 0; c < p.ck && ok; ++c, ++pos) {
+            const int slot = pos % p.nslot;
+            if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+            ptx::tc_fence_after();
+            const uint64_t a0 = kdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+            const uint64_t b0 = qdesc0 + (uint64_t)((c * 2 * kQSubBytes) >> 4);
+            const int nk = min(8, (p.r_k - c * 128) >> 4);
+            for (int kk = 0; kk < nk; ++kk) {
+              const uint64_t ad = a0 + (uint64_t)((kk >> 2) * (kSubBytes >> 4) + (kk & 3) * 2);
+              const uint64_t bd = b0 + (uint64_t)((kk >> 2) * (kQSubBytes >> 4) + (kk & 3) * 2);
+              ptx::mma_f16(d_s, ad, bd, id, (c | kk) ? 1u : 0u);
+            }
+            ptx::mma_commit(&aux->slot_empty[slot]);
           }
-          ptx::mma_commit(&aux->slot_empty[slot]);
-        }
-        if (!ok) break;
-        ptx::mma_commit(&aux->s_full);
-        if (i < 16) trace_stamp(p, 3 + 4 * i);
-        // GEMM2: O~ += Z_v^T P_hi + Z_v^T P_lo
-        if (!(ok = wait_b(&aux->p_full, i & 1, aux, p.err))) break;
-        ptx::tc_fence_after();
-        for (int c = 0; c < p.cv && ok; ++c) {
-          const int pos = i * per_tile + p.ck + c;
-          const int slot = pos % p.nslot;
-          if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+          if (!ok) break;
+          ptx::mma_commit(&aux->s_full[sb2]);
+          if (tile < 16) trace_stamp(p, 3 + 4 * tile);
+        } else {
+          // GEMM2(tile): O~ += Z_v^T [P_hi | P_lo]
+          if (!(ok = wait_b(&aux->p_full, tile & 1, aux, p.err))) break;
           ptx::tc_fence_after();
-          const uint64_t a0 = vdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
-          const uint32_t d_o = tmem + kOCol + c * 64;
+          for (int c = 0; c < p.cv && ok; ++c, ++pos) {
+            const int slot = pos % p.nslot;
+            if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+            ptx::tc_fence_after();
+            const uint64_t a0 = vdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+            const uint32_t d_o = tmem + kOCol + c * 64;
 #pragma unroll
-          for (int kt = 0; kt < 8; ++kt) {
-            const uint64_t ad = a0 + (uint64_t)(kt * 128);
-            const uint64_t bd = pdesc0 + (uint64_t)(kt * 16);
-            ptx::mma_f16(d_o, ad, bd, id2, (i | kt) ? 1u : 0u);
+            for (int kt = 0; kt < 8; ++kt) {
+              const uint64_t ad = a0 + (uint64_t)(kt * 128);
+              const uint64_t bd = pdesc0 + (uint64_t)(kt * 16);
+              ptx::mma_f16(d_o, ad, bd, id2, (tile | kt) ? 1u : 0u);
+            }
+            ptx::mma_commit(&aux->slot_empty[slot]);
           }
-          ptx::mma_commit(&aux->slot_empty[slot]);
+          if (!ok) break;
+          ptx::mma_commit(&aux->p_empty);
+          if (tile < 16) trace_stamp(p, 6 + 4 * tile);
         }
-        if (!ok) break;
-        ptx::mma_commit(&aux->p_empty);
-        if (i < 16) trace_stamp(p, 6 + 4 * i);
       }
       ptx::mma_commit(&aux->o_final);
       if (!ok) drain_wait(&aux->o_final, 0);
@@ -276,12 +289,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
       const bool valid = tok_begin + i * kTile + row < tok_end;
-      ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full, i & 1, aux, p.err));
+      const int k2 = i & 1;
+      const uint32_t s_col = tmem + lane_off + kSCol + 64 * k2;
+      ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full[k2], (i >> 1) & 1, aux, p.err));
       if (!ok) break;
       ptx::tc_fence_after();
       if (i < 16 && threadIdx.x == 64) trace_stamp(p, 4 + 4 * i);
       float s[32];
-      tmem_ld_sum(tmem + lane_off + kSCol, s);
+      tmem_ld_sum(s_col, s);
 #pragma unroll
       for (int j = 0; j < 32; ++j) s[j] = valid ? s[j] : -INFINITY;
 
@@ -289,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int j = 0; j < 32; ++j) ex |= s[j] > aux->m_s[j] + kLazy;
       ex = ptx::named_bar_or(1, 128, ex);
-      if (i >= 1) {   // the previous value mix has completed: P may be rewritten, O~ rescaled
+      if (i >= 1) {   // the value mix of tile i - 1 has completed: P may be rewritten, O~ rescaled
         ok = ptx::named_bar_and(1, 128, wait_b(&aux->p_empty, (i - 1) & 1, aux, p.err));
         if (!ok) break;
         ptx::tc_fence_after();
@@ -297,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (ex) {
         // reduce in place, then read the scores again (S stays intact until s_empty)
         aux->red[qd][lane] = warp_reduce_scatter32<true>(s, lane);
-        tmem_ld_sum(tmem + lane_off + kSCol, s);
+        tmem_ld_sum(s_col, s);
 #pragma unroll
         for (int j = 0; j < 32; ++j) s[j] = valid ? s[j] : -INFINITY;
         ptx::named_bar_sync(1, 128);
@@ -354,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&aux->s_empty);
+      ptx::mbar_arrive(&aux->s_empty[k2]);
       ptx::mbar_arrive(&aux->p_full);
       if (i < 16 && threadIdx.x == 64) trace_stamp(p, 5 + 4 * i);
     }

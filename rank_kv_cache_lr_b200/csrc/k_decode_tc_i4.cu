@@ -119,25 +119,6 @@ __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux,
   return tc::wait_b(bar, parity, &aux->abort_flag, err);
 }
 
-// Unit u of the pipeline order (each unit is the K or the V side of one tile):
-//   u = 0 -> K(0); u = 2s - 1 -> K(s) for 1 <= s < n; u = 2s -> V(s - 1); the last
-//   unit, u = 2n - 1, is V(n - 1).
-__device__ __forceinline__ void unit_of(int u, int n, int* tile, bool* is_v) {
-  if (u == 0) {
-    *tile = 0;
-    *is_v = false;
-  } else if (u == 2 * n - 1) {
-    *tile = n - 1;
-    *is_v = true;
-  } else if (u & 1) {
-    *tile = (u + 1) >> 1;
-    *is_v = false;
-  } else {
-    *tile = (u >> 1) - 1;
-    *is_v = true;
-  }
-}
-
 // Eight int4 codes of one word -> four fp16 pairs (m0,m4) (m1,m5) (m2,m6) (m3,m7) of
 // code * scale + zero; s2 = (scale, scale), z2 = (zero, zero).
 __device__ __forceinline__ uint4 dequant8(uint32_t w, uint32_t s2, uint32_t z2) {
@@ -247,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = 0; u < nunits && ok; ++u) {
           int tile;
           bool is_v;
-          unit_of(u, ntiles, &tile, &is_v);
+          tc::unit_of(u, ntiles, &tile, &is_v);
           const int t0 = tok_begin + tile * kTile;
           const int n = min(kTile, tok_end - t0);
           const int rs = u % p.nraw, round = u / p.nraw;
@@ -300,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = 0; u < nunits && ok; ++u) {
           int tile;
           bool is_v;
-          unit_of(u, ntiles, &tile, &is_v);
+          tc::unit_of(u, ntiles, &tile, &is_v);
           if (!is_v) {
             // GEMM1(tile): S[tile % 2] = Z_k q~^T
             const int sb2 = tile & 1;
@@ -496,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = 0; u < nunits && ok; ++u) {
         int tile;
         bool is_v;
-        unit_of(u, ntiles, &tile, &is_v);
+        tc::unit_of(u, ntiles, &tile, &is_v);
         const int nvalid = tok_end - (tok_begin + tile * kTile);   // valid token rows of the tile
         const int G = is_v ? p.G_v : p.G_k;
         const int nch = is_v ? p.cv : p.ck;

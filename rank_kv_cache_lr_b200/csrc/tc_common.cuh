@@ -52,6 +52,26 @@ __device__ __forceinline__ void trace_stamp(unsigned long long* trace, int slot)
   if (trace) trace[((size_t)blockIdx.y * gridDim.x + blockIdx.x) * kTraceSlots + slot] = ptx::globaltimer();
 }
 
+// Unit u of the pipelined tile order, in which the scores of tile s+1 are computed before
+// the value mix of tile s (each unit is the K or the V side of one tile):
+//   u = 0 -> K(0); u = 2s - 1 -> K(s) for 1 <= s < n; u = 2s -> V(s - 1); the last unit,
+//   u = 2n - 1, is V(n - 1).
+__device__ __forceinline__ void unit_of(int u, int n, int* tile, bool* is_v) {
+  if (u == 0) {
+    *tile = 0;
+    *is_v = false;
+  } else if (u == 2 * n - 1) {
+    *tile = n - 1;
+    *is_v = true;
+  } else if (u & 1) {
+    *tile = (u + 1) >> 1;
+    *is_v = false;
+  } else {
+    *tile = (u >> 1) - 1;
+    *is_v = true;
+  }
+}
+
 // Butterfly reduce-scatter over a warp: on return lane l holds op over all lanes of
 // v[l] (v is destroyed).
 template <bool kMax>
