@@ -81,6 +81,23 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings over all ranks (identity with one process).
+    Multi-GPU numbers are the slowest rank's, never a wall clock."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_rate(bytes_per_step_per_rank: float, steps: int, world: int, total_ms: float) -> float:
+    """Whole-job GB/s: the latent bytes every rank processed over the slowest rank's time."""
+    return bytes_per_step_per_rank * steps * world / (total_ms * 1e-3) / 1e9
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -354,13 +371,8 @@ def run_ours(args):
     h2d = sum((L["q_host"].numel() + L["k_host"].numel() + L["v_host"].numel()) * 2 for L in layers)
     d2h = sum(L["out_host"].numel() * 2 + L["lse_host"].numel() * 4 for L in layers)
 
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms, e2e_ms, max(kern_ms) if kern_ms else 0.0], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
-
-    value = bytes_per_step * K * world / (total_ms * 1e-3) / 1e9
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
+    value = job_rate(bytes_per_step, K, world, total_ms)
     peaks, peak_src = measured_peaks()
     kern_mean = statistics.mean(kern_ms)
     achieved = bytes_per_step / (kern_mean * 1e-3) / 1e9
@@ -387,7 +399,7 @@ def run_ours(args):
                      "kernel_us": round(1000 * kern_mean, 2),
                      "kernel_timing": "CUDA events around each layer's decode kernel (separate graph capture), summed over layers",
                      "traffic": (traf["bytes_per_launch"] if traf else None)},
-        "e2e": {"value": round(bytes_per_step * K * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(job_rate(bytes_per_step, K, world, e2e_ms), 2), "unit": "GB/s",
                 "us_per_step": round(1000 * e2e_ms / K, 2), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
