@@ -132,9 +132,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::mbar_init(&aux->q_full, 1);
     for (int k = 0; k < 2; ++k) {
       ptx::mbar_init(&aux->s_full[k], 1);
-      ptx::mbar_init(&aux->s_empty[k], 128);
+      ptx::mbar_init(&aux->s_empty[k], 4);     // one arrival per softmax warp
     }
-    ptx::mbar_init(&aux->p_full, 128);
+    ptx::mbar_init(&aux->p_full, 4);
     ptx::mbar_init(&aux->p_empty, 1);
     ptx::mbar_init(&aux->o_final, 1);
     aux->abort_flag = 0;
@@ -367,10 +367,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                      "r"(lw[1]), "r"(lw[2]), "r"(lw[3])
                      : "memory");
       }
+      // every lane makes its own P stores visible to the tensor core, then one arrival per warp
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&aux->s_empty[k2]);
-      ptx::mbar_arrive(&aux->p_full);
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(&aux->s_empty[k2]);
+        ptx::mbar_arrive(&aux->p_full);
+      }
       if (i < 16 && threadIdx.x == 64) trace_stamp(p, 5 + 4 * i);
     }
     if (ok) ok = ptx::named_bar_and(1, 128, wait_b(&aux->o_final, 0, aux, p.err));

@@ -62,6 +62,8 @@ using tc::warp_reduce_scatter32;
 constexpr int kThreads = 512;
 constexpr int kDqWarp0 = 8;                // first warp of the dequantisation warpgroups
 constexpr int kDqThreads = 192;            // six working dequantisation warps
+constexpr int kDqWarps = 6;                // arrivals per operand slot / raw slot (one per warp)
+constexpr int kSmWarps = 4;                // softmax warps (one arrival each)
 constexpr int kLaunchRegs = 128;
 constexpr int kRegsCtl = 56, kRegsSoftmax = 208, kRegsDq = 104;
 static_assert(128 * kRegsCtl + 128 * kRegsSoftmax + 256 * kRegsDq <= kThreads * kLaunchRegs,
@@ -181,17 +183,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     tc::trace_stamp(p.trace, 0);
     for (int s = 0; s < p.nslot; ++s) {
-      ptx::mbar_init(&aux->slot_full[s], kDqThreads);
+      ptx::mbar_init(&aux->slot_full[s], kDqWarps);
       ptx::mbar_init(&aux->slot_empty[s], 1);
     }
     for (int s = 0; s < p.nraw; ++s) {
       ptx::mbar_init(&aux->raw_full[s], 1);
-      ptx::mbar_init(&aux->raw_empty[s], kDqThreads);
+      ptx::mbar_init(&aux->raw_empty[s], kDqWarps);
     }
     for (int k = 0; k < 2; ++k) {
       ptx::mbar_init(&aux->s_full[k], 1);
-      ptx::mbar_init(&aux->s_empty[k], 128);
-      ptx::mbar_init(&aux->p_full[k], 128);
+      ptx::mbar_init(&aux->s_empty[k], kSmWarps);
+      ptx::mbar_init(&aux->p_full[k], kSmWarps);
       ptx::mbar_init(&aux->p_empty[k], 1);
     }
     ptx::mbar_init(&aux->q_full, 1);
@@ -428,10 +430,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                        "r"(hw[2]), "r"(hw[3])
                        : "memory");
         }
+        // every lane makes its own P stores visible to the tensor core, then one arrival
+        // per warp
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&aux->s_empty[k2]);
-        ptx::mbar_arrive(&aux->p_full[k2]);
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(&aux->s_empty[k2]);
+          ptx::mbar_arrive(&aux->p_full[k2]);
+        }
         if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 5 + 4 * i);
       }
       if (ok) ok = ptx::named_bar_and(1, 128, wait_b(&aux->o_final, 0, aux, p.err));
@@ -482,10 +489,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int G = is_v ? p.G_v : p.G_k;
         const int nch = is_v ? p.cv : p.ck;
         const int rs = u % p.nraw;
-        if (!(ok = wait_b(&aux->raw_full[rs], (u / p.nraw) & 1, aux, p.err))) break;
+        // waits are made warp-uniform: the warp arrives once, after __syncwarp
+        if (!(ok = __all_sync(0xffffffffu, wait_b(&aux->raw_full[rs], (u / p.nraw) & 1, aux, p.err)))) break;
         for (int c = 0; c < nch; ++c, ++pos) {
           const int slot = pos % p.nslot;
-          if (pos >= p.nslot && !(ok = wait_b(&aux->slot_empty[slot], ((pos / p.nslot) - 1) & 1, aux, p.err)))
+          if (pos >= p.nslot &&
+              !(ok = __all_sync(0xffffffffu, wait_b(&aux->slot_empty[slot], ((pos / p.nslot) - 1) & 1, aux, p.err))))
             break;
           const int ng = min(4, G - 4 * c);
           const uint8_t* rb = raw + rs * p.raw_bytes + c * 8192;          // codes of groups 4c..
@@ -519,10 +528,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               sts128(rowa + (((cb + 3) ^ sw) << 4), dequant8(w[k].w, s2, z2));
             }
           }
+          // each lane fences its own stores for the tensor core; one arrival per warp
           ptx::fence_proxy_async_smem();
-          ptx::mbar_arrive(&aux->slot_full[slot]);
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&aux->slot_full[slot]);
         }
-        if (ok) ptx::mbar_arrive(&aux->raw_empty[rs]);
+        __syncwarp();
+        if (ok && lane == 0) ptx::mbar_arrive(&aux->raw_empty[rs]);
       }
     }
   }
