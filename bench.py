@@ -52,6 +52,12 @@ WORKLOADS = {
                          "seeded per-layer ranks in [128, 448] (mean 256), keys stored after RoPE",
                     batch=16, n_q_heads=28, n_kv_heads=4, head_dim=128, rank=256, length=32768,
                     quant_bits=4, layers=28),
+    "hybrid32k": dict(desc="Qwen3-8B-shaped iS-KV hybrid layer: B=8, Hq=32, Hkv=8, d=128, 32640 history "
+                           "tokens of r=256 bf16 latents + an exact bf16 window of 128; every step appends "
+                           "one token (the oldest window token is folded into history) and decodes; "
+                           "lr_basis_sync every 128 steps, amortised into the step",
+                      batch=8, n_q_heads=32, n_kv_heads=8, head_dim=128, rank=256, length=32768,
+                      quant_bits=0, layers=1, window=128, sync_every=128),
 }
 
 
@@ -208,15 +214,22 @@ def run_ours(args):
     # through lr_kv_append_latent.
     layers = []
     host_p = None
+    win = W.get("window", 0)
     for li, (rk, rv) in enumerate(layer_ranks(args.workload)):
         hist = T - 1
-        if W["layers"] == 1:
+        if win:
+            hist = T - win
+            p = synth.make_hybrid(seed=rank, batch=Bsz, hist_len=hist, window=win, rank=rk,
+                                  n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d)
+            host_p = p
+        elif W["layers"] == 1:
             p = synth.make_qwen(args.workload, seed=rank, batch=Bsz, length=hist, rank=rk, quant_bits=qb)
             host_p = p
         else:
             p = synth.make_qwen(args.workload, seed=rank, batch=Bsz, length=0, rank=rk, rank_v=rv,
                                 quant_bits=qb, layer=li)
-        desc = lr.make_desc(Bsz, Hq, Hkv, d, rk, rv, T, quant_bits=qb, dtype=lr.LR_BF16)
+        desc = lr.make_desc(Bsz, Hq, Hkv, d, rk, rv, T + (8 if win else 0), window=win, quant_bits=qb,
+                            dtype=lr.LR_BF16)
         cache = lr.lr_cache_create(desc, to_dev(p.A_k), to_dev(p.B_k), to_dev(p.A_v), to_dev(p.B_v))
         chunk = 1024 if W["layers"] == 1 else 2048
         gen = torch.Generator(device=dev)
@@ -225,20 +238,27 @@ def run_ours(args):
         sig_v = torch.arange(1, rv + 1, device=dev, dtype=torch.float32).pow(-0.7)
         for s0 in range(0, hist, chunk):
             e0 = min(hist, s0 + chunk)
-            if W["layers"] == 1:
+            if W["layers"] == 1 or win:
                 zk = torch.from_numpy(np.ascontiguousarray(p.z_k[:, s0:e0])).to(dev)
                 zv = torch.from_numpy(np.ascontiguousarray(p.z_v[:, s0:e0])).to(dev)
             else:
                 zk = torch.randn((Bsz, e0 - s0, rk), generator=gen, device=dev) * sig_k
                 zv = torch.randn((Bsz, e0 - s0, rv), generator=gen, device=dev) * sig_v
             lr.lr_kv_append_latent(cache, zk, zv)
-        kx, vx = synth.hybrid_token(args.workload, rank * 1000 + li, hist, Bsz, D,
-                                    synth.bf16_to_f64(p.B_k), synth.bf16_to_f64(p.B_v))
-        L = dict(cache=cache, rk=rk, rv=rv, k_h=synth.bf16_bits(kx), v_h=synth.bf16_bits(vx), q_h=p.q)
+        for t in range(p.win_len if win else 0):   # the exact window, through lr_kv_append
+            lr.lr_kv_append(cache, to_dev(np.ascontiguousarray(p.win_k[:, t])), to_dev(np.ascontiguousarray(p.win_v[:, t])))
+        kx, vx = synth.hybrid_token(args.workload, rank * 1000 + li, T - 1, Bsz, D,
+                                    synth.bf16_to_f64(p.B_k), synth.bf16_to_f64(p.B_v), noise=1e-2 if win else 0.0)
+        L = dict(cache=cache, rk=rk, rv=rv, k_h=synth.bf16_bits(kx), v_h=synth.bf16_bits(vx), q_h=p.q,
+                 len0=lr.lr_cache_get_len(cache)[0])
         L["k"], L["v"], L["q"] = to_dev(L["k_h"]), to_dev(L["v_h"]), to_dev(L["q_h"])
         L["out"] = torch.empty_like(L["q"])
         L["lse"] = torch.empty((Bsz, Hq), dtype=torch.float32, device=dev)
-        L["bytes"] = Bsz * T * (latent_bytes_per_token(rk, qb) + latent_bytes_per_token(rv, qb))
+        if win:   # history latents plus the exact window tokens the step reads
+            L["bytes"] = Bsz * ((T - win) * (latent_bytes_per_token(rk, qb) + latent_bytes_per_token(rv, qb))
+                                + win * 2 * D * 2)
+        else:
+            L["bytes"] = Bsz * T * (latent_bytes_per_token(rk, qb) + latent_bytes_per_token(rv, qb))
         layers.append(L)
     torch.cuda.synchronize()
     bytes_per_step = sum(L["bytes"] for L in layers)
@@ -256,7 +276,7 @@ def run_ours(args):
     def step():
         for L in layers:   # lr_kv_append + lr_attn_decode per layer (fused launches)
             lr.lr_decode_step(L["cache"], L["k"], L["v"], L["q"], L["out"], L["lse"])
-            lr.lr_cache_truncate(L["cache"], T - 1)
+            lr.lr_cache_truncate(L["cache"], L["len0"])   # windowed caches: undo of the last append
 
     def barrier():
         if world > 1:
@@ -371,6 +391,35 @@ def run_ours(args):
     h2d = sum((L["q_host"].numel() + L["k_host"].numel() + L["v_host"].numel()) * 2 for L in layers)
     d2h = sum(L["out_host"].numel() * 2 + L["lse_host"].numel() * 4 for L in layers)
 
+    # basis sync (windowed workloads): seeded Haar rotations, B' = R^T B, A' = A R, timed
+    # alone; its cost is amortised over `sync_every` steps in the headline value
+    sync = None
+    if W.get("sync_every"):
+        L = layers[0]
+        Rk = synth.sync_rotation(rank, 0, L["rk"], "k")
+        Rv = synth.sync_rotation(rank, 0, L["rv"], "v")
+        Bk0, Bv0 = synth.bf16_to_f64(host_p.B_k), synth.bf16_to_f64(host_p.B_v)
+        Ak0, Av0 = synth.bf16_to_f64(host_p.A_k), synth.bf16_to_f64(host_p.A_v)
+        sargs = (torch.from_numpy(Rk.astype(np.float32)).to(dev), torch.from_numpy(Rv.astype(np.float32)).to(dev),
+                 to_dev(synth.bf16_bits(Rk.T @ Bk0)), to_dev(synth.bf16_bits(Rv.T @ Bv0)),
+                 to_dev(synth.bf16_bits(Ak0 @ Rk)), to_dev(synth.bf16_bits(Av0 @ Rv)))
+        lr.lr_basis_sync(L["cache"], *sargs)
+        torch.cuda.synchronize()
+        sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+        for a0, a1 in sev:
+            flush_l2()
+            a0.record()
+            lr.lr_basis_sync(L["cache"], *sargs)
+            a1.record()
+        torch.cuda.synchronize()
+        sync_ms = statistics.median(a0.elapsed_time(a1) for a0, a1 in sev)
+        sync_bytes = 2 * 2 * Bsz * (T - W["window"]) * L["rk"] * 2      # K and V history, read + write
+        sync = {"us_per_call": round(1000 * sync_ms, 2), "every_steps": W["sync_every"],
+                "us_per_step_amortised": round(1000 * sync_ms / W["sync_every"], 3),
+                "GBps": round(sync_bytes / (sync_ms * 1e-3) / 1e9, 1)}
+        total_ms += K * sync_ms / W["sync_every"]
+        e2e_ms += K * sync_ms / W["sync_every"]
+
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
     value = job_rate(bytes_per_step, K, world, total_ms)
     peaks, peak_src = measured_peaks()
@@ -405,6 +454,8 @@ def run_ours(args):
         "gpu_launches": launches,
         "clocks": sampler.summary(),
     }
+    if sync is not None:
+        res["config"]["basis_sync"] = sync
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(args.workload, host_p, args.cpu_seconds)
     if rank == 0:
@@ -452,9 +503,13 @@ def oracle_step_sample(p, rows, seconds):
             qv = (p.q[b:b + 1].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
             Bk = (p.B_k.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
             Bv = (p.B_v.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-            attention.decode(qv, zk[None], zv[None], Bk, Bv, p.n_kv_heads)
+            wk = wv = None
+            if p.win_k is not None and p.win_len:
+                wk = (p.win_k[b:b + 1].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+                wv = (p.win_v[b:b + 1].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            attention.decode(qv, zk[None], zv[None], Bk, Bv, p.n_kv_heads, None, None, wk, wv)
             done += 1
-            nbytes += p.hist_len * 2 * per_tok
+            nbytes += p.hist_len * 2 * per_tok + (p.win_len * 2 * p.kv_dim * 2 if wk is not None else 0)
         el = time.time() - t0
         if el >= seconds:
             return nbytes / el, el / done, done
@@ -464,6 +519,10 @@ def host_problem(workload, seed, batch):
     """A host-side instance of (the first layer of) a workload for the CPU oracle."""
     import synth
     W = WORKLOADS[workload]
+    if W.get("window"):
+        return synth.make_hybrid(seed=seed, batch=batch, hist_len=W["length"] - W["window"], window=W["window"],
+                                 rank=W["rank"], n_q_heads=W["n_q_heads"], n_kv_heads=W["n_kv_heads"],
+                                 head_dim=W["head_dim"])
     if W["layers"] == 1:
         return synth.make_qwen(workload, seed=seed, batch=batch, length=W["length"] - 1, rank=W["rank"],
                                quant_bits=W["quant_bits"])

@@ -209,7 +209,10 @@ lr_status lr_attn_decode_noalloc(const lr_cache_desc* desc, int32_t len, const v
 /* Current total length, history length and window length (host-side counters). */
 lr_status lr_cache_get_len(const lr_cache* cache, int32_t* len, int32_t* hist_len,
                            int32_t* win_len);
-/* Drop tokens at positions >= len (no device work).  Caches without a window only. */
+/* Drop tokens at positions >= len (no device work).  Caches with a window can drop only
+ * the token of the last lr_kv_append / lr_decode_step (len = current length - 1; the
+ * ring's spare slot still holds the token that append folded out of the window);
+ * anything else returns LR_ERR_UNSUPPORTED. */
 lr_status lr_cache_truncate(lr_cache* cache, int32_t len);
 /* Device pointers of the storage (see lr_cache_view). */
 lr_status lr_cache_view_get(const lr_cache* cache, lr_cache_view* out);

@@ -246,7 +246,8 @@ lr_status lr_kv_append(lr_cache* c, const void* k, const void* v, void* stream) 
   cudaError_t e = launch_append(c, k, v, s);
   if (e != cudaSuccess) return LR_ERR_CUDA;
   if (c->win_slots) {
-    if (c->win_len == c->desc.window) ++c->hist_len;
+    c->undo = c->win_len == c->desc.window ? 2 : 1;
+    if (c->undo == 2) ++c->hist_len;
     else ++c->win_len;
   } else {
     ++c->hist_len;
@@ -259,6 +260,7 @@ lr_status lr_kv_append_latent(lr_cache* c, const float* zk, const float* zv, int
   if (!c || !zk || !zv || n < 0) return LR_ERR_INVALID_ARG;
   if (c->win_len > 0) return LR_ERR_INVALID_ARG;
   if ((long long)c->len + n > c->desc.capacity) return LR_ERR_CAPACITY;
+  c->undo = 0;
   if (n == 0) return LR_OK;
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
@@ -341,6 +343,7 @@ lr_status lr_decode_step(lr_cache* c, const void* k, const void* v, const void* 
   cudaError_t e = launch_step_pre(c, k, v, q, p.path == LR_PATH_TC, s);   // uses the pre-append counters
   if (e != cudaSuccess) return LR_ERR_CUDA;
   c->stable_len = c->hist_len;   // the row the append writes (new token or fold) is not stable
+  if (c->win_slots) c->undo = hist1 > c->hist_len ? 2 : 1;
   c->hist_len = hist1;
   c->win_len = win1;
   ++c->len;
@@ -378,7 +381,17 @@ lr_status lr_cache_get_len(const lr_cache* c, int32_t* len, int32_t* hist_len, i
 
 lr_status lr_cache_truncate(lr_cache* c, int32_t len) {
   if (!c || len < 0 || len > c->len) return LR_ERR_INVALID_ARG;
-  if (c->win_slots) return LR_ERR_UNSUPPORTED;
+  if (c->win_slots) {
+    // The ring keeps one slot beyond the window, so the last append can be undone: the
+    // token it folded out of the window is still in its slot.
+    if (len == c->len) return LR_OK;
+    if (len != c->len - 1 || c->undo == 0) return LR_ERR_UNSUPPORTED;
+    if (c->undo == 2) --c->hist_len;
+    else --c->win_len;
+    --c->len;
+    c->undo = 0;
+    return LR_OK;
+  }
   c->len = c->hist_len = len;
   return LR_OK;
 }

@@ -35,6 +35,8 @@ struct lr_cache {
   int win_slots;         // window + 1 (ring), or 0
   long long lat_cap;     // latent rows per sequence: capacity (int4: rounded up to 128)
   int32_t len, hist_len, win_len;
+  int undo = 0;           // windowed caches: 0 = no undo, 1 = the last append only filled
+                          // the window, 2 = it folded the oldest window token into history
   int32_t stable_len = 0; // history rows [0, stable_len) were written before the kernel that
                           // precedes the decode (the decode may read them before its
                           // grid-dependency wait); set by each decode entry point

@@ -420,6 +420,27 @@ def test_truncate_replays_same_step(lib):
     assert np.array_equal(first, again)
 
 
+@pytest.mark.parametrize("win_len", [50, 128])
+def test_truncate_undoes_last_append_with_window(lib, win_len):
+    """A windowed cache can drop the token of its last append (the ring's spare slot keeps
+    the folded token): window not yet full (no fold) and full (fold)."""
+    p = synth.small_variant("hybrid", hist_len=300, win_len=win_len)
+    c = H.fill_cache(lib, p)
+    first, first_lse = H.gpu_decode(lib, p, c)
+    n0 = lib.lr_cache_get_len(c)
+    k, v = synth.hybrid_token("undo", 0, 0, p.batch, p.kv_dim, H.stored_value(p, p.B_k), H.stored_value(p, p.B_v))
+    for _ in range(2):
+        lib.lr_kv_append(c, H.to_dev(p, p.store(k)), H.to_dev(p, p.store(v)))
+        assert lib.lr_cache_get_len(c) != n0
+        lib.lr_cache_truncate(c, n0[0])
+        assert lib.lr_cache_get_len(c) == n0
+        again, again_lse = H.gpu_decode(lib, p, c)
+        assert np.array_equal(first, again) and np.array_equal(first_lse, again_lse)
+    with pytest.raises(lib.LRError) as e:
+        lib.lr_cache_truncate(c, n0[0] - 1)           # nothing left to undo
+    assert e.value.status == lib.LR_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("kind", ["tiny", "qwen4k", "qwen16k", "hybrid"])
 def test_decode_step_equals_append_then_decode(lib, kind):
     """lr_decode_step is lr_kv_append followed by lr_attn_decode, bit for bit."""
