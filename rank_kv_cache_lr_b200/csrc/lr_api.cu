@@ -87,6 +87,7 @@ cudaError_t dalloc(T** p, size_t bytes) {
 void free_all(lr_cache* c) {
   if (!c) return;
   tc_release(c);
+  sync_tc_release(c);
   void* ptrs[] = {c->z_k, c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->win_k, c->win_v,
                   c->A_k, c->B_k, c->A_v, c->B_v, c->rope_cs, c->qt, c->qt16, c->part_o, c->part_ml,
                   c->win_o, c->win_ml, c->dev_err};
@@ -360,8 +361,12 @@ lr_status lr_basis_sync(lr_cache* c, const float* R_k, const float* R_v, const v
   const lr_cache_desc& d = c->desc;
   const size_t es = c->esize, D = c->D;
   cudaError_t e = cudaSuccess;
-  if (R_k) e = launch_sync_simt(c, R_k, 0, s);
-  if (e == cudaSuccess && R_v) e = launch_sync_simt(c, R_v, 1, s);
+  if ((R_k || R_v) && sync_tc_supported(&d) && c->path_force != LR_PATH_SIMT) {
+    e = launch_sync_tc(c, R_k, R_v, s);
+  } else {
+    if (R_k) e = launch_sync_simt(c, R_k, 0, s);
+    if (e == cudaSuccess && R_v) e = launch_sync_simt(c, R_v, 1, s);
+  }
   if (e == cudaSuccess && B_k_new) e = cudaMemcpyAsync(c->B_k, B_k_new, (size_t)d.rank_k * D * es, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess && B_v_new) e = cudaMemcpyAsync(c->B_v, B_v_new, (size_t)d.rank_v * D * es, cudaMemcpyDeviceToDevice, s);
   if (A_k_new || A_v_new) c->has_A = true;

@@ -68,6 +68,7 @@ struct lr_cache {
   int device = 0;
   cudaStream_t last_stream = nullptr;
   void* tc_state = nullptr;    // tensor-core path state (tensor maps), owned
+  void* sync_state = nullptr;  // tensor-core basis sync state (tensor maps, split R), owned
   cudaEvent_t ev_start = nullptr, ev_stop = nullptr;   // caller-owned kernel timing events
   unsigned long long* trace = nullptr;                 // caller-owned decode timeline buffer
 };
@@ -120,6 +121,11 @@ bool tc_i4_supported(const lr_cache_desc* d);
 cudaError_t tc_i4_prepare(lr_cache* c);
 void tc_i4_release(lr_cache* c);
 cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s);
+
+// basis sync on tensor cores (k_sync_tc.cu)
+bool sync_tc_supported(const lr_cache_desc* d);
+cudaError_t launch_sync_tc(lr_cache* c, const float* R_k, const float* R_v, cudaStream_t s);
+void sync_tc_release(lr_cache* c);
 
 void lr_count_launch(int n = 1);
 

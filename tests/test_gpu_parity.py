@@ -292,6 +292,46 @@ def test_sync_identity_is_bit_exact(lib):
     assert np.array_equal(before, after)
 
 
+@pytest.mark.parametrize("which", ["kv", "k", "v"])
+def test_sync_tensor_core_matches_oracle_and_cuda_cores(lib, which):
+    """The tensor-core sync (bf16 latents, r <= 256) against the oracle's rounded fp64
+    Z R and against the CUDA-core sync: several 128-token tiles plus a ragged tail,
+    two sequences, one side or both."""
+    import torch
+    p = synth.small_variant("hybrid", hist_len=700, batch=2)
+    c_tc, c_simt = H.fill_cache(lib, p), H.fill_cache(lib, p)
+    lib.lr_cache_set_path(c_simt, lib.LR_PATH_SIMT)
+    Rk = synth.sync_rotation(0, 3, p.rank_k, "k").astype(np.float32)
+    Rv = synth.sync_rotation(0, 3, p.rank_v, "v").astype(np.float32)
+    rk = torch.from_numpy(Rk).cuda() if "k" in which else None
+    rv = torch.from_numpy(Rv).cuda() if "v" in which else None
+    for c in (c_tc, c_simt):
+        lib.lr_basis_sync(c, rk, rv, None, None, None, None)
+    torch.cuda.synchronize()
+    n = p.hist_len
+    for side, R, on in (("k", Rk, "k" in which), ("v", Rv, "v" in which)):
+        z0 = H.oracle_latents(p, p.z_k if side == "k" else p.z_v)        # stored bf16 values
+        ref = synth.bf16_bits(z0 @ R.astype(np.float64)) if on else synth.bf16_bits(z0)
+        got = []
+        for c in (c_tc, c_simt):
+            v = lib.lr_cache_view_get(c)
+            z = lib.copy_view(v.z_k if side == "k" else v.z_v, (p.batch, v.capacity, p.rank_k), "<i2")
+            got.append(z.cpu().numpy().view(np.uint16)[:, :n])
+        rv64 = synth.bf16_to_f64(ref)
+        ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(rv64), 1e-30))) - 7)   # bf16 spacing at ref
+        # rounding bound of the computed product before its bf16 store: R split into bf16
+        # hi + lo leaves <= 2^-18 |R| per entry, and fp32 accumulation of 2r terms adds
+        # <= 2r 2^-24 sum|z R|; 2^-14 sum_k |z_k| |R_kn| covers both (cancellations near zero
+        # make ulps of the result meaningless there)
+        mag = (np.abs(z0) @ np.abs(R.astype(np.float64))) if on else np.zeros_like(rv64)
+        bound = ulp + 2.0 ** -14 * mag
+        for name, g in zip(("tensor cores", "cuda cores"), got):
+            err = np.abs(synth.bf16_to_f64(g) - rv64)
+            assert np.all(err <= bound), f"{side} {name}: {np.max(err / bound):.2f} x bound"
+            assert np.mean(err > 0) < 0.01, f"{side} {name}: {np.mean(err > 0):.4f} of elements differ"
+    assert lib.lr_device_error(c_tc) == 0
+
+
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("layer", [0, 5, 4])
 def test_decode_parity_int4_postrope(lib, layer):
