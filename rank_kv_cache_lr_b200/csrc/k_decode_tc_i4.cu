@@ -53,16 +53,16 @@ using tc::warp_reduce_scatter32;
 
 // 16 warps in four warpgroups: [producer, MMA, 2 idle] [4 softmax] [dequantisation x 8].
 // A warp runs on sub-partition (warp % 4).  A single thread issuing N = 32 MMAs slows
-// about fivefold when ALU-bound warps share its sub-partition, so the MMA warp (1)
-// shares sub-partition 1 only with the softmax warp that must read TMEM lanes 32..63;
-// the dequantisation work runs on warps 8, 10, 11, 12, 14, 15 (sub-partitions 0, 2, 3)
-// and warps 9, 13 stay idle.  Launched at 128 registers per thread; the warpgroups then
-// rebalance the block's 64K registers with setmaxnreg (the softmax keeps 32 scores and
-// 32 running sums per row).
+// about fivefold when three ALU-bound warps share its sub-partition; with the producer,
+// MMA and two idle warps in the first warpgroup, the MMA warp (1) shares sub-partition 1
+// with one softmax warp and two dequantisation warps.  Measured against leaving those two
+// dequantisation warps idle, the extra dequantisation throughput wins by ~3 %.  Launched
+// at 128 registers per thread; the warpgroups then rebalance the block's 64K registers
+// with setmaxnreg (the softmax keeps 32 scores and 32 running sums per row).
 constexpr int kThreads = 512;
 constexpr int kDqWarp0 = 8;                // first warp of the dequantisation warpgroups
-constexpr int kDqThreads = 192;            // six working dequantisation warps
-constexpr int kDqWarps = 6;                // arrivals per operand slot / raw slot (one per warp)
+constexpr int kDqThreads = 256;            // eight working dequantisation warps
+constexpr int kDqWarps = 8;                // arrivals per operand slot / raw slot (one per warp)
 constexpr int kSmWarps = 4;                // softmax warps (one arrival each)
 constexpr int kLaunchRegs = 128;
 constexpr int kRegsCtl = 56, kRegsSoftmax = 208, kRegsDq = 104;
@@ -473,11 +473,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::setmaxnreg_dec<kRegsDq>();
     // ------------------------------------------------------------- dequantisation
     if (ntiles > 0) {
-      // working warps 8, 10, 11, 12, 14, 15 -> dq 0..191; unit v = (token v % 128, group
-      // v / 128 of the chunk) for v = dq, dq + 192, ...; lanes walk consecutive tokens
+      // warps 8..15 -> dq 0..255; unit v = (token v % 128, group v / 128 of the chunk) for
+      // v = dq, dq + 256, ...; lanes walk consecutive tokens
       const int wi = warp - kDqWarp0;      // 0..7
-      const bool dq_live = wi != 1 && wi != 5;
-      const int dq = (wi - (wi > 1) - (wi > 5)) * 32 + lane;
+      const bool dq_live = true;
+      const int dq = wi * 32 + lane;
       const uint32_t ring_base = ptx::smem_u32(ring);
       bool ok = dq_live;
       int pos = 0;
