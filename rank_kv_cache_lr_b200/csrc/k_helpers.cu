@@ -42,6 +42,14 @@ struct El<__nv_bfloat16> {
   static __device__ __forceinline__ float lds1(const uint8_t* s) {
     return __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(s)) << 16);
   }
+  // 4 consecutive elements from 8-byte aligned shared memory
+  static __device__ __forceinline__ void lds4(const uint8_t* s, float (&v)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2*>(s);
+    v[0] = __uint_as_float(u.x << 16);
+    v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(u.y << 16);
+    v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+  }
 };
 template <>
 struct El<float> {
@@ -53,6 +61,10 @@ struct El<float> {
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   }
   static __device__ __forceinline__ float lds1(const uint8_t* s) { return *reinterpret_cast<const float*>(s); }
+  static __device__ __forceinline__ void lds4(const uint8_t* s, float (&v)[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(s);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  }
 };
 
 // ---- query projection -----------------------------------------------------------
@@ -377,9 +389,7 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
         for (int k = 0; k < 4; ++k) {
           if (i + k < i1) {
             float bv[4];
-            const uint8_t* bp = bs + ((size_t)(i + k) * ncols + 4 * cq) * es;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) bv[e] = El<T>::lds1(bp + e * es);
+            El<T>::lds4(bs + ((size_t)(i + k) * ncols + 4 * cq) * es, bv);
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[e] = fmaf(ov[k], bv[e], acc[e]);
           }
