@@ -49,9 +49,15 @@ WORKLOADS = {
                     batch=16, n_q_heads=28, n_kv_heads=4, head_dim=128, rank=352, length=16384,
                     quant_bits=4, layers=1),
     "qwen32k": dict(desc="28 Qwen2.5-VL-7B layers: B=16, Hq=28, Hkv=4, d=128, T=32768, int4 g32 latents, "
-                         "seeded per-layer ranks in [128, 448] (mean 256), keys stored after RoPE",
+                         "seeded per-layer ranks in [128, 448] (mean 256), keys stored before RoPE "
+                         "(rebuilt and rotated per tile, theta=1e6)",
                     batch=16, n_q_heads=28, n_kv_heads=4, head_dim=128, rank=256, length=32768,
-                    quant_bits=4, layers=28),
+                    quant_bits=4, layers=28, rope=True),
+    "qwen32k_postrope": dict(desc="28 Qwen2.5-VL-7B layers: B=16, Hq=28, Hkv=4, d=128, T=32768, int4 g32 "
+                                  "latents, seeded per-layer ranks in [128, 448] (mean 256), keys stored "
+                                  "after RoPE (scores in rank space)",
+                             batch=16, n_q_heads=28, n_kv_heads=4, head_dim=128, rank=256, length=32768,
+                             quant_bits=4, layers=28, rope=False),
     "hybrid32k": dict(desc="Qwen3-8B-shaped iS-KV hybrid layer: B=8, Hq=32, Hkv=8, d=128, 32640 history "
                            "tokens of r=256 bf16 latents + an exact bf16 window of 128; every step appends "
                            "one token (the oldest window token is folded into history) and decodes; "
@@ -229,7 +235,7 @@ def run_ours(args):
             p = synth.make_qwen(args.workload, seed=rank, batch=Bsz, length=0, rank=rk, rank_v=rv,
                                 quant_bits=qb, layer=li)
         desc = lr.make_desc(Bsz, Hq, Hkv, d, rk, rv, T + (8 if win else 0), window=win, quant_bits=qb,
-                            dtype=lr.LR_BF16)
+                            dtype=lr.LR_BF16, rope_in_kernel=1 if W.get("rope") else 0)
         cache = lr.lr_cache_create(desc, to_dev(p.A_k), to_dev(p.B_k), to_dev(p.A_v), to_dev(p.B_v))
         chunk = 1024 if W["layers"] == 1 else 2048
         gen = torch.Generator(device=dev)
@@ -526,7 +532,7 @@ def host_problem(workload, seed, batch):
     if W["layers"] == 1:
         return synth.make_qwen(workload, seed=seed, batch=batch, length=W["length"] - 1, rank=W["rank"],
                                quant_bits=W["quant_bits"])
-    return synth.make_qwen32k_layer(0, seed=seed, batch=batch, length=W["length"] - 1, rope=False)
+    return synth.make_qwen32k_layer(0, seed=seed, batch=batch, length=W["length"] - 1, rope=bool(W.get("rope")))
 
 
 def cpu_baseline(workload, p, seconds):

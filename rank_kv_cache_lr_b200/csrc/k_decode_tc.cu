@@ -458,10 +458,12 @@ int tc_ctas_per_sm(const lr_cache_desc* d, int hist_len, int num_sms) {
   return slots_pair(d) ? 2 : 1;
 }
 
-cudaError_t tc_prepare(lr_cache* c) {
+int tc_split_ctas(const lr_cache_desc* d) { return d->quant_bits == 4 ? tc_i4_split_ctas(d) : 1; }
+
+cudaError_t tc_prepare(lr_cache* c, cudaStream_t s) {
   const lr_cache_desc& d = c->desc;
   if (!tc_supported(&d)) return cudaSuccess;
-  if (d.quant_bits == 4) return tc_i4_prepare(c);
+  if (d.quant_bits == 4) return tc_i4_prepare(c, s);
   TcState* st = reinterpret_cast<TcState*>(c->tc_state);
   if (!st) {
     st = new (std::nothrow) TcState();

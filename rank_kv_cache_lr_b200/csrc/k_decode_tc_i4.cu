@@ -36,6 +36,18 @@
 // the same order (a score is an order-free sum over ranks), and the epilogue maps the
 // rows of O~ back to rank order.
 //
+// Keys stored before the rotary embedding (kRope).  The score needs the rotated key,
+// which has no rank-space form, so each tile's keys are rebuilt on the tensor cores:
+//   K^_h[t, :] = z^_k,t B_k,h          GEMM0: M = 128 tokens, N = d = 128, K = r_k
+// then rotated (rotate-half RoPE at the token's absolute position, cos / sin from the
+// cache's fp64-derived table) and dotted with the raw query rows on CUDA cores by the
+// softmax warps (thread = token row).  K^ for all four KV heads would need all of TMEM,
+// so a CTA covers a pair of KV heads (grid x), query slots 16 h + jj for query head jj
+// of pair head h; both CTAs of a pair dequantise the same tiles.  B_k enters as an fp16
+// copy, [D rows][ranks] with each 8-rank run in the dequantised order, streamed per
+// (128-rank chunk, head) by TMA from a spare warp (warp 2) through a two-slot ring.  The
+// value mix and the epilogue are those of the rank-space kernel with 32 slots.
+//
 // Every wait is bounded: on timeout the kernel records LR_ERR_TIMEOUT, drains its own
 // copies and MMAs, frees TMEM and returns.
 #include "tc_common.cuh"
@@ -77,6 +89,12 @@ constexpr int kAuxBytes = 2048;
 constexpr int kSCol = 0;                   // TMEM: S of tile s in columns [32 (s % 2), +32)
 constexpr int kOCol = 64;                  // TMEM: O~ chunk c in columns [64 + 32c, +32)
 constexpr int kMaxSlots = 4;
+// keys before RoPE
+constexpr int kRD = 128;                   // head dim of the rebuilt keys
+constexpr int kGHMax = 2;                  // KV heads per CTA (K^ of both fills 256 columns)
+constexpr int kMaxG = 32 / kGHMax;         // query slots per KV head
+constexpr int kOColR = 256;                // TMEM: O~ chunk c in columns [256 + 32c, +32)
+constexpr int kNB = 2;                     // B_k ring slots (128 rows x 128 ranks, fp16)
 constexpr int kMaxRaw = 6;                 // raw slot: one side of one tile, codes (G x 2 KB)
                                            // then {scale, zero} words (G x 512 B)
 
@@ -93,6 +111,11 @@ struct I4Params {
   float* part_ml;
   int* err;
   unsigned long long* trace;
+  // keys before RoPE
+  const float* qf;          // [B][Hq][d] scaled queries, fp32
+  const float2* rope_cs;    // [capacity][d / 2] (cos, sin)
+  int gh, gsz;              // KV heads per CTA, query heads per KV head
+  uint32_t q_load_bytes;    // gh * gsz * d * 4
 };
 
 struct Aux {
@@ -102,6 +125,7 @@ struct Aux {
   uint64_t raw_empty[kMaxRaw];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
   uint64_t q_full, o_final;
+  uint64_t k_full, k_empty, b_full[kNB], b_empty[kNB];   // keys before RoPE
   uint32_t tmem_base;
   int abort_flag;
   float red[4][32];
@@ -112,8 +136,11 @@ static_assert(sizeof(Aux) <= kAuxBytes, "aux block");
 
 struct I4State {
   CUtensorMap q;
+  CUtensorMap bk;           // keys before RoPE: fp16 B_k [D][r_pad], rank runs permuted
+  void* bk16 = nullptr;
+  int r_pad = 0;
   int nslot, nraw;
-  uint32_t raw_bytes, raw_params;
+  uint32_t raw_bytes, raw_params, q_bytes;
   size_t smem;
 };
 
@@ -158,10 +185,13 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
                : "memory");
 }
 
-// Shared memory: [aux 2 KB][q~ per 64-rank sub-block][operand ring nslot x 32 KB]
+// Shared memory: [aux 2 KB][q~ per 64-rank sub-block | fp32 query rows (kRope)]
+//                [B_k ring kNB x 32 KB (kRope)][operand ring nslot x 32 KB]
 //                [P double buffer 2 x 8 KB][raw ring nraw x raw_bytes]
+template <bool kRope>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_decode_tc_i4(const __grid_constant__ CUtensorMap tm_q, const I4Params p) {
+    k_decode_tc_i4(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_b,
+                   const I4Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (ptx::smem_u32(smem_raw) & 1023) {
     if (threadIdx.x == 0) atomicExch(p.err, (int)LR_ERR_UNSUPPORTED);
@@ -169,12 +199,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   Aux* aux = reinterpret_cast<Aux*>(smem_raw);
   uint8_t* q_s = smem_raw + kAuxBytes;
-  uint8_t* ring = q_s + p.q_bytes;
+  uint8_t* bring = q_s + p.q_bytes;
+  uint8_t* ring = bring + (kRope ? kNB * kSlotBytes : 0);
   uint8_t* p_s = ring + p.nslot * kSlotBytes;
   uint8_t* raw = p_s + 2 * kPBytes;
+  constexpr int kOC = kRope ? kOColR : kOCol;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, b = blockIdx.y;
+  const int pair = kRope ? (int)blockIdx.x : 0;
+  const int split = kRope ? blockIdx.y : blockIdx.x, b = kRope ? blockIdx.z : blockIdx.y;
   const int tok_begin = split * p.split_tokens;
   const int tok_end = min(p.hist_len, tok_begin + p.split_tokens);
   const int ntiles = tok_end > tok_begin ? (tok_end - tok_begin + kTile - 1) / kTile : 0;
@@ -198,11 +231,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::mbar_init(&aux->q_full, 1);
     ptx::mbar_init(&aux->o_final, 1);
+    if (kRope) {
+      ptx::mbar_init(&aux->k_full, 1);
+      ptx::mbar_init(&aux->k_empty, kSmWarps);
+      for (int k = 0; k < kNB; ++k) {
+        ptx::mbar_init(&aux->b_full[k], 1);
+        ptx::mbar_init(&aux->b_empty[k], 1);
+      }
+    }
     aux->abort_flag = 0;
     for (int j = 0; j < 32; ++j) aux->m_s[j] = -INFINITY;
     ptx::fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) ptx::prefetch_tmap(&tm_q);
+  if (warp == 0 && lane == 0 && !kRope) ptx::prefetch_tmap(&tm_q);
+  if (warp == 2 && lane == 0 && kRope) ptx::prefetch_tmap(&tm_b);
   if (warp == 1) {
     ptx::tmem_alloc(&aux->tmem_base, p.tmem_cols);
     ptx::tmem_relinquish();
@@ -225,6 +267,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
       // ------------------------------------------------------------- bulk-copy producer
       if (lane == 0 && ntiles > 0) {
+        // the query rows: q~ (fp16, by TMA) or, for keys before RoPE, the pair's fp32 rows
+        auto load_query = [&]() {
+          if (kRope) {
+            ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_load_bytes);
+            ptx::bulk_load(q_s, p.qf + ((size_t)b * p.Hq + (size_t)pair * p.gh * p.gsz) * kRD, p.q_load_bytes,
+                           &aux->q_full);
+          } else {
+            ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
+            for (int sb = 0; sb < p.kb_k; ++sb)
+              ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
+          }
+        };
         bool waited = false, ok = true;
         int issued = 0;
         for (int u = 0; u < nunits && ok; ++u) {
@@ -236,9 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int rs = u % p.nraw, round = u / p.nraw;
           if (!waited && (round > 0 || t0 + n > p.stable_len)) {
             pdl_wait();
-            ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
-            for (int sb = 0; sb < p.kb_k; ++sb)
-              ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
+            load_query();
             waited = true;
           }
           if (round > 0 && !(ok = wait_b(&aux->raw_empty[rs], (round - 1) & 1, aux, p.err))) break;
@@ -254,15 +306,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!waited) {
           pdl_wait();
-          ptx::mbar_arrive_expect_tx(&aux->q_full, p.q_bytes);
-          for (int sb = 0; sb < p.kb_k; ++sb)
-            ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
+          load_query();
         }
         if (!ok) {
           drain_wait(&aux->q_full, 0);
           for (int k = max(0, issued - p.nraw); k < issued; ++k)
             drain_wait(&aux->raw_full[k % p.nraw], (k / p.nraw) & 1);
         }
+      }
+    } else if (kRope && warp == 2) {
+      // ------------------------------------------------------------- B_k producer (kRope)
+      // (tile, chunk c, pair head h) in the MMA's order; B_k is written before the cache
+      // is used, so no grid-dependency wait is needed.
+      if (lane == 0 && ntiles > 0) {
+        const int total = ntiles * p.ck * p.gh;
+        bool ok = true;
+        int issued = 0;
+        for (int k = 0; k < total; ++k) {
+          const int slot = k % kNB;
+          if (k >= kNB && !(ok = wait_b(&aux->b_empty[slot], ((k / kNB) - 1) & 1, aux, p.err))) break;
+          const int h = k % p.gh, c = (k / p.gh) % p.ck;
+          const int row = (pair * p.gh + h) * kRD;
+          uint8_t* dst = bring + slot * kSlotBytes;
+          ptx::mbar_arrive_expect_tx(&aux->b_full[slot], (uint32_t)kSlotBytes);
+          ptx::tma_load_2d(dst, &tm_b, &aux->b_full[slot], c * 128, row);
+          ptx::tma_load_2d(dst + kSubBytes, &tm_b, &aux->b_full[slot], c * 128 + 64, row);
+          issued = k + 1;
+        }
+        if (!ok)
+          for (int k = max(0, issued - kNB); k < issued; ++k) drain_wait(&aux->b_full[k % kNB], (k / kNB) & 1);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------- MMA issuer
@@ -276,15 +348,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t qdesc0 = ptx::smem_desc(ptx::smem_u32(q_s), 16, 1024, 2);        // q~, K-major SW128
         const uint64_t vdesc0 = ptx::smem_desc(ptx::smem_u32(ring), kSubBytes, 1024, 2); // Z_v, MN-major SW128
         const uint64_t pdesc0 = ptx::smem_desc(ptx::smem_u32(p_s), 128, 2048, 0);       // P, MN-major
-        bool ok = wait_b(&aux->q_full, 0, aux, p.err);
+        const uint32_t idk = ptx::idesc_f16(0, 0, 0, 128, kRD);  // GEMM0 (kRope): K-major x K-major
+        const uint64_t bdesc0 = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, 2);      // B_k, K-major SW128
+        bool ok = kRope ? true : wait_b(&aux->q_full, 0, aux, p.err);
         ptx::tc_fence_after();
         tc::trace_stamp(p.trace, 2);
-        int pos = 0;
+        int pos = 0, bpos = 0;
         for (int u = 0; u < nunits && ok; ++u) {
           int tile;
           bool is_v;
           tc::unit_of(u, ntiles, &tile, &is_v);
-          if (!is_v) {
+          if (kRope && !is_v) {
+            // GEMM0(tile): K^_h = Z_k B_k,h for the pair's heads, into columns [128 h, +128)
+            if (tile >= 1 && !(ok = wait_b(&aux->k_empty, (tile - 1) & 1, aux, p.err))) break;
+            ptx::tc_fence_after();
+            for (int c = 0; c < p.ck && ok; ++c, ++pos) {
+              const int slot = pos % p.nslot;
+              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+              ptx::tc_fence_after();
+              const uint64_t a0 = kdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+              const int nk = min(8, (p.r_k - c * 128) >> 4);
+              for (int h = 0; h < p.gh; ++h, ++bpos) {
+                const int bs = bpos % kNB;
+                if (!(ok = wait_b(&aux->b_full[bs], (bpos / kNB) & 1, aux, p.err))) break;
+                ptx::tc_fence_after();
+                const uint64_t b0 = bdesc0 + (uint64_t)((bs * kSlotBytes) >> 4);
+                // A and B share the layout: 64-rank sub-blocks of 16 KB, 32 bytes per step
+                for (int kk = 0; kk < nk; ++kk) {
+                  const uint32_t o = (uint32_t)((kk >> 2) * (kSubBytes >> 4) + (kk & 3) * 2);
+                  ptx::mma_f16(tmem + h * kRD, a0 + o, b0 + o, idk, (c | kk) ? 1u : 0u);
+                }
+                ptx::mma_commit(&aux->b_empty[bs]);
+              }
+              if (!ok) break;
+              ptx::mma_commit(&aux->slot_empty[slot]);
+            }
+            if (!ok) break;
+            ptx::mma_commit(&aux->k_full);
+          } else if (!is_v) {
             // GEMM1(tile): S[tile % 2] = Z_k q~^T
             const int sb2 = tile & 1;
             if (tile >= 2 && !(ok = wait_b(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
@@ -319,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
               const uint64_t a0 = vdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
-              const uint32_t d_o = tmem + kOCol + c * 32;
+              const uint32_t d_o = tmem + kOC + c * 32;
               // K step kt = 16 tokens: 2 KB on A (16 swizzled rows), 256 B on P
 #pragma unroll
               for (int kt = 0; kt < 8; ++kt)
@@ -347,20 +448,91 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < 32; ++j) l[j] = 0.f;
       bool ok = true;
-      for (int i = 0; i < ntiles; ++i) {
+      // keys before RoPE: the query rows are read here, from shared memory
+      if (kRope) ok = ptx::named_bar_and(1, 128, wait_b(&aux->q_full, 0, aux, p.err));
+      const float* q_f = reinterpret_cast<const float*>(q_s);
+      for (int i = 0; i < ntiles && ok; ++i) {
         const int k2 = i & 1;
         const bool valid = tok_begin + i * kTile + row < tok_end;
-        ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full[k2], (i >> 1) & 1, aux, p.err));
-        if (!ok) break;
-        ptx::tc_fence_after();
-        if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 4 + 4 * i);
         const uint32_t s_col = tmem + lane_off + kSCol + 32 * k2;
-        uint32_t sv[32];
-        ptx::tmem_ld32(s_col, sv);
-        ptx::tmem_wait_ld();
         float s[32];
+        if (kRope) {
+          ok = ptx::named_bar_and(1, 128, wait_b(&aux->k_full, i & 1, aux, p.err));
+          if (!ok) break;
+          ptx::tc_fence_after();
+          // score of query slot 16 h + jj: q_jj . RoPE_t(K^_h[t]), pairs (c, c + 64)
+          const int t = tok_begin + i * kTile + row;
+          const float2* cs_row = p.rope_cs + (size_t)(valid ? t : tok_begin) * (kRD / 2);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+          for (int j = 0; j < 32; ++j) s[j] = 0.f;
+#pragma unroll 1
+          for (int c0 = 0; c0 < kRD / 2; c0 += 16) {
+            float cs[32];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float4 v = __ldg(reinterpret_cast<const float4*>(cs_row + c0) + k);
+              cs[4 * k] = v.x;
+              cs[4 * k + 1] = v.y;
+              cs[4 * k + 2] = v.z;
+              cs[4 * k + 3] = v.w;
+            }
+#pragma unroll
+            for (int h = 0; h < kGHMax; ++h) {
+              if (h < p.gh) {
+                uint32_t x1[16], x2[16];
+                ptx::tmem_ld16(tmem + lane_off + h * kRD + c0, x1);
+                ptx::tmem_ld16(tmem + lane_off + h * kRD + kRD / 2 + c0, x2);
+                ptx::tmem_wait_ld();
+                float r1[16], r2[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                  const float a = __uint_as_float(x1[k]), e = __uint_as_float(x2[k]);
+                  r1[k] = a * cs[2 * k] - e * cs[2 * k + 1];
+                  r2[k] = e * cs[2 * k] + a * cs[2 * k + 1];
+                }
+#pragma unroll
+                for (int jj = 0; jj < kMaxG; ++jj) {
+                  if (jj < p.gsz) {
+                    const float* qr = q_f + (size_t)(h * p.gsz + jj) * kRD + c0;
+                    float acc = s[h * kMaxG + jj];
+#pragma unroll
+                    for (int k = 0; k < 16; k += 4) {
+                      const float4 qa = *reinterpret_cast<const float4*>(qr + k);
+                      const float4 qb = *reinterpret_cast<const float4*>(qr + kRD / 2 + k);
+                      acc = fmaf(qa.x, r1[k], acc);
+                      acc = fmaf(qa.y, r1[k + 1], acc);
+                      acc = fmaf(qa.z, r1[k + 2], acc);
+                      acc = fmaf(qa.w, r1[k + 3], acc);
+                      acc = fmaf(qb.x, r2[k], acc);
+                      acc = fmaf(qb.y, r2[k + 1], acc);
+                      acc = fmaf(qb.z, r2[k + 2], acc);
+                      acc = fmaf(qb.w, r2[k + 3], acc);
+                    }
+                    s[h * kMaxG + jj] = acc;
+                  }
+                }
+              }
+            }
+          }
+          // K^ has been read: GEMM0 of the next tile may overwrite it
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&aux->k_empty);
+          if (!valid) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s[j] = -INFINITY;
+          }
+        } else {
+          ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full[k2], (i >> 1) & 1, aux, p.err));
+          if (!ok) break;
+          ptx::tc_fence_after();
+          if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 4 + 4 * i);
+          uint32_t sv[32];
+          ptx::tmem_ld32(s_col, sv);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+        }
 
         bool ex = false;
 #pragma unroll
@@ -373,11 +545,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             ptx::tc_fence_after();
           }
-          aux->red[qd][lane] = warp_reduce_scatter32<true>(s, lane);
-          ptx::tmem_ld32(s_col, sv);
-          ptx::tmem_wait_ld();
+          if (kRope) {
+            float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+            for (int j = 0; j < 32; ++j) v[j] = s[j];
+            aux->red[qd][lane] = warp_reduce_scatter32<true>(v, lane);
+          } else {
+            // the reduction consumes s; it is read again from TMEM
+            aux->red[qd][lane] = warp_reduce_scatter32<true>(s, lane);
+            uint32_t sv[32];
+            ptx::tmem_ld32(s_col, sv);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+          }
           ptx::named_bar_sync(1, 128);
           if (qd == 0) {
             const float mt =
@@ -398,11 +579,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (need_o && i > 0) {
             for (int c = 0; c < p.cv; ++c) {
               uint32_t v2[32];
-              ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
+              ptx::tmem_ld32(tmem + lane_off + kOC + c * 32, v2);
               ptx::tmem_wait_ld();
 #pragma unroll
               for (int j = 0; j < 32; ++j) v2[j] = __float_as_uint(__uint_as_float(v2[j]) * aux->alpha_s[j]);
-              ptx::tmem_st32(tmem + lane_off + kOCol + c * 32, v2);
+              ptx::tmem_st32(tmem + lane_off + kOC + c * 32, v2);
             }
             ptx::tmem_wait_st();
           }
@@ -436,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          ptx::mbar_arrive(&aux->s_empty[k2]);
+          if (!kRope) ptx::mbar_arrive(&aux->s_empty[k2]);
           ptx::mbar_arrive(&aux->p_full[k2]);
         }
         if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 5 + 4 * i);
@@ -448,23 +629,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         // TMEM row m of a chunk holds rank 8 (m / 8) + perm(m % 8), perm = 0,4,1,5,2,6,3,7
         const int m = qd * 32 + lane;
         const int e_in = (m & ~7) + ((m & 7) >> 1) + ((m & 1) << 2);
+        // query head of slot j (-1: padding)
+        auto head_of = [&](int j) -> int {
+          if (!kRope) return j < p.Hq ? j : -1;
+          const int h = j / kMaxG, jj = j % kMaxG;
+          return (h < p.gh && jj < p.gsz) ? (pair * p.gh + h) * p.gsz + jj : -1;
+        };
         for (int c = 0; c < p.cv; ++c) {
           uint32_t v2[32];
-          ptx::tmem_ld32(tmem + lane_off + kOCol + c * 32, v2);
+          ptx::tmem_ld32(tmem + lane_off + kOC + c * 32, v2);
           ptx::tmem_wait_ld();
           const int e = c * 128 + e_in;
           if (e < p.r_v) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < p.Hq) p.part_o[(base_out + j) * p.r_v + e] = __uint_as_float(v2[j]);
+            for (int j = 0; j < 32; ++j) {
+              const int J = head_of(j);
+              if (J >= 0) p.part_o[(base_out + J) * p.r_v + e] = __uint_as_float(v2[j]);
+            }
           }
         }
         aux->red[qd][lane] = warp_reduce_scatter32<false>(l, lane);
         ptx::named_bar_sync(1, 128);
-        if (qd == 0 && lane < p.Hq) {
+        const int J = head_of(lane);
+        if (qd == 0 && J >= 0) {
           const float lt = (aux->red[0][lane] + aux->red[1][lane]) + (aux->red[2][lane] + aux->red[3][lane]);
-          p.part_ml[(base_out + lane) * 2] = aux->m_s[lane];
-          p.part_ml[(base_out + lane) * 2 + 1] = lt;
+          p.part_ml[(base_out + J) * 2] = aux->m_s[lane];
+          p.part_ml[(base_out + J) * 2 + 1] = lt;
         }
         if (threadIdx.x == 128) tc::trace_stamp(p.trace, kTraceSlots - 1);
       }
@@ -546,11 +736,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// B_k as the fp16 B operand of GEMM0: out[n][pos] = B_k[rank(pos)][n] for the D output
+// columns n, where position pos of each 8-rank run holds rank 0,4,1,5,2,6,3,7 (the order
+// of the dequantised latents); ranks >= r_k are zero.  bf16 -> fp16 is exact for values
+// of magnitude 2^-14 .. 65504.
+__global__ void k_prep_bk16(const __nv_bfloat16* Bk, __half* out, int r_k, int r_pad, int D) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)D * r_pad) return;
+  const int n = (int)(idx / r_pad), pos = (int)(idx % r_pad);
+  const int i = (pos & ~7) | ((pos & 1) << 2) | ((pos >> 1) & 3);
+  out[idx] = i < r_k ? __float2half_rn(__bfloat162float(Bk[(size_t)i * D + n])) : __float2half_rn(0.f);
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 
-int q_bytes_for(int r_k) { return ((r_k + 63) / 64) * kQSubBytes; }
+int q_bytes_for(const lr_cache_desc* d) {
+  if (d->rope_in_kernel) {
+    const int gh = d->n_kv_heads % 2 == 0 ? 2 : 1;
+    const int rows = gh * (d->n_q_heads / d->n_kv_heads);
+    return ((rows * kRD * 4 + 1023) / 1024) * 1024;
+  }
+  return ((d->rank_k + 63) / 64) * kQSubBytes;
+}
 
 struct I4Layout {
   int nslot, nraw;
@@ -560,12 +769,14 @@ struct I4Layout {
 
 // Raw slots hold one side of one tile.  As many operand slots as leave room for two raw
 // slots (up to four: the dequantisation can then run a full 128-rank chunk further ahead
-// of the MMAs), then as many raw slots (up to 6) as fit in 227 KB.
+// of the MMAs), then as many raw slots (up to 6) as fit in 227 KB.  Keys before RoPE add
+// the B_k ring.
 bool choose_layout(const lr_cache_desc* d, I4Layout* L) {
   const int G = std::max((d->rank_k + 31) / 32, (d->rank_v + 31) / 32);
   L->raw_params = (uint32_t)G * 2048u;
   L->raw_bytes = (uint32_t)G * 2560u;
-  const size_t fixed = (size_t)kAuxBytes + q_bytes_for(d->rank_k) + 2 * kPBytes;
+  const size_t fixed =
+      (size_t)kAuxBytes + q_bytes_for(d) + (d->rope_in_kernel ? (size_t)kNB * kSlotBytes : 0) + 2 * kPBytes;
   for (int ns = kMaxSlots; ns >= 2; --ns) {
     if (fixed + (size_t)ns * kSlotBytes > (size_t)kSmemLimit) continue;
     const int nr =
@@ -580,17 +791,25 @@ bool choose_layout(const lr_cache_desc* d, I4Layout* L) {
   return false;
 }
 
+int kv_per_cta(const lr_cache_desc* d) {
+  if (!d->rope_in_kernel) return d->n_kv_heads;
+  return d->n_kv_heads % 2 == 0 ? 2 : 1;
+}
+
 }  // namespace
 
 bool tc_i4_supported(const lr_cache_desc* d) {
   if (d->quant_bits != 4 || d->quant_group != 32) return false;
-  if (d->dtype != LR_BF16 || d->rope_in_kernel) return false;
+  if (d->dtype != LR_BF16) return false;
   if (d->n_q_heads > 32 || d->rank_v > 512) return false;
+  if (d->rope_in_kernel && (d->head_dim != kRD || d->n_q_heads / d->n_kv_heads > kMaxG)) return false;
   I4Layout L;
   return choose_layout(d, &L);
 }
 
-cudaError_t tc_i4_prepare(lr_cache* c) {
+int tc_i4_split_ctas(const lr_cache_desc* d) { return d->n_kv_heads / kv_per_cta(d); }
+
+cudaError_t tc_i4_prepare(lr_cache* c, cudaStream_t s) {
   const lr_cache_desc& d = c->desc;
   I4State* st = reinterpret_cast<I4State*>(c->tc_state);
   if (!st) {
@@ -598,30 +817,54 @@ cudaError_t tc_i4_prepare(lr_cache* c) {
     if (!st) return cudaErrorMemoryAllocation;
     c->tc_state = st;
   }
-  const size_t qbytes = (size_t)d.batch * kQRows * d.rank_k * 2;
-  if (!c->qt16) {
-    cudaError_t e = cudaMalloc(&c->qt16, qbytes);
+  if (d.rope_in_kernel) {
+    const int r_pad = ((d.rank_k + 127) / 128) * 128;
+    if (!st->bk16) {
+      cudaError_t e = cudaMalloc(&st->bk16, (size_t)c->D * r_pad * 2);
+      if (e != cudaSuccess) return e;
+      st->r_pad = r_pad;
+    }
+    const long long n = (long long)c->D * r_pad;
+    k_prep_bk16<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(c->B_k),
+                                                            reinterpret_cast<__half*>(st->bk16), d.rank_k, r_pad, c->D);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = cudaMemset(c->qt16, 0, qbytes);
-    if (e != cudaSuccess) return e;
+    cuuint64_t dims[2] = {(cuuint64_t)r_pad, (cuuint64_t)c->D};
+    cuuint64_t strides[1] = {(cuuint64_t)r_pad * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kRD};
+    if (!tc::make_map(&st->bk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, st->bk16, 2, dims, strides, box))
+      return cudaErrorInvalidValue;
+    st->q = st->bk;   // unused by the kRope kernel
+  } else {
+    const size_t qbytes = (size_t)d.batch * kQRows * d.rank_k * 2;
+    if (!c->qt16) {
+      cudaError_t e = cudaMalloc(&c->qt16, qbytes);
+      if (e != cudaSuccess) return e;
+      e = cudaMemset(c->qt16, 0, qbytes);
+      if (e != cudaSuccess) return e;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)d.rank_k, (cuuint64_t)d.batch * kQRows};
+    cuuint64_t strides[1] = {(cuuint64_t)d.rank_k * 2};
+    cuuint32_t box[2] = {64, kQRows};
+    if (!tc::make_map(&st->q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, c->qt16, 2, dims, strides, box))
+      return cudaErrorInvalidValue;
+    st->bk = st->q;   // unused by the rank-space kernel
   }
-  cuuint64_t dims[2] = {(cuuint64_t)d.rank_k, (cuuint64_t)d.batch * kQRows};
-  cuuint64_t strides[1] = {(cuuint64_t)d.rank_k * 2};
-  cuuint32_t box[2] = {64, kQRows};
-  if (!tc::make_map(&st->q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, c->qt16, 2, dims, strides, box))
-    return cudaErrorInvalidValue;
   I4Layout L;
   if (!choose_layout(&d, &L)) return cudaErrorNotSupported;
   st->nslot = L.nslot;
   st->nraw = L.nraw;
   st->raw_bytes = L.raw_bytes;
   st->raw_params = L.raw_params;
+  st->q_bytes = (uint32_t)q_bytes_for(&d);
   st->smem = L.smem;
   return cudaSuccess;
 }
 
 void tc_i4_release(lr_cache* c) {
-  delete reinterpret_cast<I4State*>(c->tc_state);
+  I4State* st = reinterpret_cast<I4State*>(c->tc_state);
+  if (st && st->bk16) cudaFree(st->bk16);
+  delete st;
   c->tc_state = nullptr;
 }
 
@@ -629,6 +872,7 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   const lr_cache_desc& d = c->desc;
   const I4State* st = reinterpret_cast<const I4State*>(c->tc_state);
   if (!st) return cudaErrorNotSupported;
+  const bool rope = d.rope_in_kernel != 0;
   I4Params p;
   p.codes_k = c->codes_k;
   p.codes_v = c->codes_v;
@@ -642,7 +886,7 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   p.ck = (d.rank_k + 127) / 128;
   p.cv = (d.rank_v + 127) / 128;
   p.kb_k = (d.rank_k + 63) / 64;
-  p.tmem_cols = (kOCol + p.cv * 32) <= 128 ? 128 : 256;
+  p.tmem_cols = rope ? 512 : ((kOCol + p.cv * 32) <= 128 ? 128 : 256);
   p.Hq = d.n_q_heads;
   p.hist_len = c->hist_len;
   p.stable_len = std::min(c->stable_len, c->hist_len);
@@ -650,21 +894,34 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   p.n_splits = n_splits;
   p.nslot = st->nslot;
   p.nraw = st->nraw;
-  p.q_bytes = q_bytes_for(d.rank_k);
+  p.q_bytes = st->q_bytes;
   p.raw_bytes = st->raw_bytes;
   p.raw_params = st->raw_params;
   p.part_o = c->part_o;
   p.part_ml = c->part_ml;
   p.err = c->dev_err;
-  p.trace = c->trace;
-  static std::atomic<uint32_t> optin_done{0};
-  cudaError_t e = smem_optin(k_decode_tc_i4, optin_done);
+  p.trace = rope ? nullptr : c->trace;    // the timeline covers the rank-space grid only
+  p.qf = c->qt;
+  p.rope_cs = c->rope_cs;
+  p.gh = kv_per_cta(&d);
+  p.gsz = d.n_q_heads / d.n_kv_heads;
+  p.q_load_bytes = (uint32_t)(p.gh * p.gsz * kRD * 4);
+  auto kern = rope ? k_decode_tc_i4<true> : k_decode_tc_i4<false>;
+  static std::atomic<uint32_t> optin_done[2] = {0, 0};
+  cudaError_t e = smem_optin(kern, optin_done[rope ? 1 : 0]);
   if (e != cudaSuccess) return e;
   // The register rebalancing assumes the launch allocation the split was sized for.
-  static const int regs = [] {
-    cudaFuncAttributes fa;
-    return cudaFuncGetAttributes(&fa, k_decode_tc_i4) == cudaSuccess ? fa.numRegs : -1;
-  }();
-  if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-  return launch_pdl(k_decode_tc_i4, dim3(n_splits, d.batch), dim3(kThreads), st->smem, s, st->q, p);
+  static const int regs[2] = {[] {
+                                cudaFuncAttributes fa;
+                                return cudaFuncGetAttributes(&fa, k_decode_tc_i4<false>) == cudaSuccess ? fa.numRegs
+                                                                                                        : -1;
+                              }(),
+                              [] {
+                                cudaFuncAttributes fa;
+                                return cudaFuncGetAttributes(&fa, k_decode_tc_i4<true>) == cudaSuccess ? fa.numRegs
+                                                                                                       : -1;
+                              }()};
+  if (regs[rope ? 1 : 0] != kLaunchRegs) return cudaErrorInvalidConfiguration;
+  const dim3 grid = rope ? dim3(d.n_kv_heads / p.gh, n_splits, d.batch) : dim3(n_splits, d.batch);
+  return launch_pdl(kern, grid, dim3(kThreads), st->smem, s, st->q, st->bk, p);
 }

@@ -542,7 +542,8 @@ cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s) {
 }
 
 cudaError_t launch_qproj_tc(const lr_cache* c, const void* q, cudaStream_t s) {
-  if (!c->qt16 || c->desc.dtype != LR_BF16) return cudaErrorNotSupported;
+  // keys before RoPE: the decode reads the scaled fp32 queries, no 16-bit latents
+  if (c->desc.dtype != LR_BF16 || (!c->qt16 && !c->desc.rope_in_kernel)) return cudaErrorNotSupported;
   return qproj_t<__nv_bfloat16>(c, q, s, true);
 }
 

@@ -52,8 +52,9 @@ lr_status plan(const lr_cache_desc* d, int hist_len, int num_sms, int path, int 
   if (splits <= 0) {
     // SIMT: about two CTAs per SM; tensor-core path: one wave of its resident blocks
     const int sms = std::max(num_sms, 1);
-    const int target = (p == LR_PATH_TC) ? std::max(1, tc_ctas_per_sm(d, hist_len, sms) * sms / d->batch)
-                                         : std::max(1, (2 * sms + d->batch - 1) / d->batch);
+    const int target =
+        (p == LR_PATH_TC) ? std::max(1, tc_ctas_per_sm(d, hist_len, sms) * sms / (d->batch * tc_split_ctas(d)))
+                          : std::max(1, (2 * sms + d->batch - 1) / d->batch);
     splits = std::min(tiles, target);
   }
   splits = std::max(1, std::min(splits, tiles));
@@ -63,7 +64,7 @@ lr_status plan(const lr_cache_desc* d, int hist_len, int num_sms, int path, int 
   out->n_splits = splits;
   out->tile_tokens = tile;
   out->split_tokens = tiles_per * tile;
-  out->ctas = splits * d->batch;
+  out->ctas = splits * d->batch * (p == LR_PATH_TC ? tc_split_ctas(d) : 1);
   return LR_OK;
 }
 
@@ -219,7 +220,7 @@ lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void
   if (e == cudaSuccess && A_k) e = cudaMemcpyAsync(c->A_k, A_k, D * d.rank_k * es, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess && A_v) e = cudaMemcpyAsync(c->A_v, A_v, D * d.rank_v * es, cudaMemcpyDeviceToDevice, s);
   c->has_A = A_k != nullptr;
-  if (e == cudaSuccess && tc_supported(&d)) e = tc_prepare(c);
+  if (e == cudaSuccess && tc_supported(&d)) e = tc_prepare(c, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     free_all(c);
@@ -372,7 +373,7 @@ lr_status lr_basis_sync(lr_cache* c, const float* R_k, const float* R_v, const v
   if (A_k_new || A_v_new) c->has_A = true;
   if (e == cudaSuccess && A_k_new) e = cudaMemcpyAsync(c->A_k, A_k_new, D * d.rank_k * es, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess && A_v_new) e = cudaMemcpyAsync(c->A_v, A_v_new, D * d.rank_v * es, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess && (B_k_new || B_v_new)) e = tc_prepare(c);
+  if (e == cudaSuccess && (B_k_new || B_v_new)) e = tc_prepare(c, s);
   return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
 }
 

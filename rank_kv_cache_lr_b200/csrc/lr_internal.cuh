@@ -112,13 +112,17 @@ size_t decode_simt_smem(const lr_cache* c);
 // tensor-core path (k_decode_tc.cu)
 bool tc_supported(const lr_cache_desc* d);
 int tc_ctas_per_sm(const lr_cache_desc* d, int hist_len, int num_sms);   // decode blocks per SM
-cudaError_t tc_prepare(lr_cache* c);
+// (re)builds the path's tensor maps and derived operands; kernels it launches go on s
+cudaError_t tc_prepare(lr_cache* c, cudaStream_t s);
+// decode CTAs per (sequence, split): 1, or the KV-head pairs of the keys-before-RoPE grid
+int tc_split_ctas(const lr_cache_desc* d);
 void tc_release(lr_cache* c);
 cudaError_t launch_qproj_tc(const lr_cache* c, const void* q, cudaStream_t s);
 cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s);
 // int4 latents on tensor cores (k_decode_tc_i4.cu)
 bool tc_i4_supported(const lr_cache_desc* d);
-cudaError_t tc_i4_prepare(lr_cache* c);
+cudaError_t tc_i4_prepare(lr_cache* c, cudaStream_t s);
+int tc_i4_split_ctas(const lr_cache_desc* d);
 void tc_i4_release(lr_cache* c);
 cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s);
 

@@ -44,6 +44,39 @@ def fp16_operand_lse_bound(p: synth.Problem, q: np.ndarray) -> np.ndarray:
     return out
 
 
+def fp16_latent_rope_lse_bound(p: synth.Problem, q: np.ndarray) -> np.ndarray:
+    """Worst-case |lse error| [B][Hq] of the keys-before-RoPE decode on tensor cores.  The
+    keys are rebuilt from the fp16 roundings of the dequantised int4 latents x^ (error
+    <= 2^-11 |x^| + 2^-25 each) and of B_k (bf16 -> fp16: exact above 2^-14, else <= 2^-25),
+    accumulated in fp32, rotated and dotted with the fp32 query; the probabilities are fp16
+    as on the rank-space path.  With |.| the Euclidean norm (a rotation keeps it) and
+    b_i = |B_k,h[i, :]|:
+      |d logit_t| <= s |q_j| [ sum_i (2^-11 |x^_t,i| + 2^-25) b_i + sqrt(d) 2^-25 sum_i |x^_t,i|
+                              + (r + d + 8) 2^-24 sum_i |x^_t,i| b_i ],
+      |d lse|     <= max_t |d logit_t| + 2^-10."""
+    qv = stored_value(p, q)
+    Bk = stored_value(p, p.B_k)
+    d, G = p.head_dim, p.n_q_heads // p.n_kv_heads
+    s = 1.0 / math.sqrt(d)
+    rel = 2.0 ** -11 + (p.rank_k + d + 8) * 2.0 ** -24
+    out = np.zeros((p.batch, p.n_q_heads))
+    for b in range(p.batch):
+        X = np.abs(oracle_latents(p, p.z_k[b]))
+        sx = X.sum(axis=1)
+        for h in range(p.n_kv_heads):
+            bn = np.linalg.norm(Bk[:, h * d:(h + 1) * d], axis=1)
+            worst = np.max(rel * (X @ bn) + 2.0 ** -25 * bn.sum() + math.sqrt(d) * 2.0 ** -25 * sx)
+            for j in range(h * G, (h + 1) * G):
+                out[b, j] = s * np.linalg.norm(qv[b, j]) * worst + 2.0 ** -10
+    return out
+
+
+def decode_lse_bound(p: synth.Problem, q: np.ndarray) -> np.ndarray:
+    """The LSE bar of a tensor-core decode over int4 latents: the rank-space bound or the
+    keys-before-RoPE bound."""
+    return fp16_latent_rope_lse_bound(p, q) if p.rope else fp16_operand_lse_bound(p, q)
+
+
 def bf16_bits_to_f64(bits) -> np.ndarray:
     """Oracle-side decoding of stored bf16 bit patterns (input format, not arithmetic)."""
     b = np.ascontiguousarray(np.asarray(bits, dtype=np.uint16)).astype(np.uint32) << 16

@@ -99,6 +99,25 @@ def test_plan_covers_history_exactly(lib, length, batch, path):
     assert p.n_splits * batch <= max(2 * 148 + batch, batch)
 
 
+@pytest.mark.parametrize("n_kv_heads, pairs", [(4, 2), (2, 1), (1, 1), (3, 3)])
+@pytest.mark.parametrize("rank_k", [128, 256, 448])
+def test_plan_keys_before_rope_int4_on_kv_head_pairs(lib, n_kv_heads, pairs, rank_k):
+    """int4 keys before RoPE take the tensor-core path with one CTA per pair of KV heads
+    (or per KV head when their count is odd), within one wave of 148 SMs."""
+    d = _qwen(lib, n_q_heads=7 * n_kv_heads, n_kv_heads=n_kv_heads, rank_k=rank_k, rank_v=448,
+              quant_bits=4, rope_in_kernel=1, capacity=32768)
+    p = lib.lr_plan_decode(d, 32768, 148)
+    assert p.path == lib.LR_PATH_TC
+    assert p.ctas == p.n_splits * d.batch * pairs
+    assert p.ctas <= 148
+    assert (p.n_splits - 1) * p.split_tokens < 32768 <= p.n_splits * p.split_tokens
+
+
+def test_plan_keys_before_rope_other_head_dims_use_cuda_cores(lib):
+    d = _qwen(lib, head_dim=64, quant_bits=4, rope_in_kernel=1)
+    assert lib.lr_plan_decode(d, 4096, 148).path == lib.LR_PATH_SIMT
+
+
 def test_plan_forced_splits_and_window(lib):
     d = _qwen(lib, capacity=8192)
     p = lib.lr_plan_decode(d, 4096, 148, 1, 7)

@@ -46,7 +46,7 @@ def _check(lib, p, count=6, seed=0):
         lse_tol = None
         if plan.path == lib.LR_PATH_TC and p.quant_bits == 4:
             lse_tol = np.full((p.batch, p.n_q_heads), np.nan)
-            bound = H.fp16_operand_lse_bound(_rows_only(p, pairs), q[sorted({b for b, _ in pairs})])
+            bound = H.decode_lse_bound(_rows_only(p, pairs), q[sorted({b for b, _ in pairs})])
             for k, b in enumerate(sorted({b for b, _ in pairs})):
                 lse_tol[b] = bound[k]
         H.compare(p, got, ref, lse, ref_lse, pairs=pairs, tag=f"{p.name} T={p.length} path={plan.path}",
@@ -77,6 +77,14 @@ def test_fullsize_qwen16k_int4(lib):
 def test_fullsize_qwen32k_int4_layer(lib):
     # layer 0 of the 28-layer cache, ranks (256, 384), keys stored after RoPE
     p = synth.make_qwen32k_layer(0, seed=0, batch=16, length=32768, rope=False)
+    plan = _check(lib, p, count=4)
+    assert plan.path == lib.LR_PATH_TC
+
+
+def test_fullsize_qwen32k_int4_layer_prerope(lib):
+    # layer 11 of the 28-layer cache, ranks (448, 256), keys stored before RoPE: the
+    # per-tile rebuild and rotation at positions up to 32767
+    p = synth.make_qwen32k_layer(11, seed=0, batch=16, length=32768, rope=True)
     plan = _check(lib, p, count=4)
     assert plan.path == lib.LR_PATH_TC
 

@@ -28,7 +28,7 @@ def lse_tol_for(lr, p, q, path):
     """The LSE bar: the stated one, or for int4 latents on tensor cores (fp16 operands)
     the rounding bound derived in helpers.fp16_operand_lse_bound."""
     if path == lr.LR_PATH_TC and p.quant_bits == 4:
-        return H.fp16_operand_lse_bound(p, q)
+        return H.decode_lse_bound(p, q)
     return None
 
 
@@ -56,15 +56,21 @@ def test_decode_parity(lib, kind, sharp):
                   lse_tol=lse_tol_for(lib, p, q, path))
 
 
-@pytest.mark.parametrize("layer", [0, 5, 4])
+@pytest.mark.parametrize("layer", [0, 5, 4, 11, 12])
 def test_decode_parity_prerope(lib, layer):
-    # ranks of these layers: (256, 384), (128, 128), (400, 224)
+    """Keys stored before RoPE, rebuilt and rotated per tile (CUDA cores, and tensor cores
+    for each KV-head pair).  Ranks of these layers: (256, 384), (128, 128), (400, 224),
+    (448, 256), (192, 448) — partial last chunks, the largest ranks, r_k != r_v."""
     p = synth.small_variant("qwen32k", layer=layer, length=300)
     c = H.fill_cache(lib, p)
     for q in (p.q, _sharp(p)):
         ref, ref_lse = H.oracle_decode(p, q)
-        got, lse = H.gpu_decode(lib, p, c, q)
-        H.compare(p, got, ref, lse, ref_lse, tag=f"prerope layer={layer}")
+        for path in paths(lib, p):
+            lib.lr_cache_set_path(c, path)
+            got, lse = H.gpu_decode(lib, p, c, q)
+            H.compare(p, got, ref, lse, ref_lse, tag=f"prerope layer={layer} path={path}",
+                      lse_tol=lse_tol_for(lib, p, q, path))
+
 
 
 def test_tiny_from_exact_keys_via_append(lib):
@@ -353,7 +359,7 @@ def test_decode_parity_int4_postrope(lib, layer):
 # ----------------------------------------------------------------------------
 
 
-@pytest.mark.parametrize("kind", ["qwen4k", "qwen16k"])
+@pytest.mark.parametrize("kind", ["qwen4k", "qwen16k", "qwen32k"])
 def test_split_count_invariance(lib, kind):
     p = synth.small_variant(kind, length=1000)
     c = H.fill_cache(lib, p)
@@ -398,6 +404,21 @@ def test_tile_edges_int4(lib, length):
         lib.lr_cache_set_path(c, path)
         got, lse = H.gpu_decode(lib, p, c, q)
         H.compare(p, got, ref, lse, ref_lse, tag=f"int4 T={length} path={path}",
+                  lse_tol=lse_tol_for(lib, p, q, path))
+
+
+@pytest.mark.parametrize("length", [1, 127, 128, 129, 257])
+def test_tile_edges_int4_prerope(lib, length):
+    """Keys before RoPE around the 128-token tile: the rotation positions of ragged tiles
+    and of later splits, zero-filled tail rows."""
+    p = synth.small_variant("qwen32k", layer=0, length=length, batch=3)
+    c = H.fill_cache(lib, p)
+    q = _sharp(p)
+    ref, ref_lse = H.oracle_decode(p, q)
+    for path in paths(lib, p):
+        lib.lr_cache_set_path(c, path)
+        got, lse = H.gpu_decode(lib, p, c, q)
+        H.compare(p, got, ref, lse, ref_lse, tag=f"int4 pre-RoPE T={length} path={path}",
                   lse_tol=lse_tol_for(lib, p, q, path))
 
 
