@@ -45,8 +45,11 @@
 // so a CTA covers a pair of KV heads (grid x), query slots 16 h + jj for query head jj
 // of pair head h; both CTAs of a pair dequantise the same tiles.  B_k enters as an fp16
 // copy, [D rows][ranks] with each 8-rank run in the dequantised order, streamed per
-// (128-rank chunk, head) by TMA from a spare warp (warp 2) through a two-slot ring.  The
-// value mix and the epilogue are those of the rank-space kernel with 32 slots.
+// 64-rank sub-block (both heads' rows, one N = 256 MMA per 16 ranks) by TMA from a spare
+// warp (warp 2) through a ring of up to four slots.  The rotation factors of a row are
+// fetched one 16-pair chunk ahead (the next tile's first chunk during the last one), so
+// their L2 latency stays off the chain rebuild -> rotate -> rebuild.  The value mix and
+// the epilogue are those of the rank-space kernel with 32 slots.
 //
 // Every wait is bounded: on timeout the kernel records LR_ERR_TIMEOUT, drains its own
 // copies and MMAs, frees TMEM and returns.
@@ -94,7 +97,7 @@ constexpr int kRD = 128;                   // head dim of the rebuilt keys
 constexpr int kGHMax = 2;                  // KV heads per CTA (K^ of both fills 256 columns)
 constexpr int kMaxG = 32 / kGHMax;         // query slots per KV head
 constexpr int kOColR = 256;                // TMEM: O~ chunk c in columns [256 + 32c, +32)
-constexpr int kNB = 2;                     // B_k ring slots (128 rows x 128 ranks, fp16)
+constexpr int kNBMax = 4;                  // B_k ring slots (kv heads x 128 rows x 64 ranks, fp16)
 constexpr int kMaxRaw = 6;                 // raw slot: one side of one tile, codes (G x 2 KB)
                                            // then {scale, zero} words (G x 512 B)
 
@@ -116,6 +119,7 @@ struct I4Params {
   const float2* rope_cs;    // [capacity][d / 2] (cos, sin)
   int gh, gsz;              // KV heads per CTA, query heads per KV head
   uint32_t q_load_bytes;    // gh * gsz * d * 4
+  int nb;                   // B_k ring slots of gh * 16 KB
 };
 
 struct Aux {
@@ -125,7 +129,7 @@ struct Aux {
   uint64_t raw_empty[kMaxRaw];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
   uint64_t q_full, o_final;
-  uint64_t k_full, k_empty, b_full[kNB], b_empty[kNB];   // keys before RoPE
+  uint64_t k_full, k_empty, b_full[kNBMax], b_empty[kNBMax];   // keys before RoPE
   uint32_t tmem_base;
   int abort_flag;
   float red[4][32];
@@ -139,7 +143,7 @@ struct I4State {
   CUtensorMap bk;           // keys before RoPE: fp16 B_k [D][r_pad], rank runs permuted
   void* bk16 = nullptr;
   int r_pad = 0;
-  int nslot, nraw;
+  int nslot, nraw, nb = 0;
   uint32_t raw_bytes, raw_params, q_bytes;
   size_t smem;
 };
@@ -186,9 +190,11 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
 }
 
 // Shared memory: [aux 2 KB][q~ per 64-rank sub-block | fp32 query rows (kRope)]
-//                [B_k ring kNB x 32 KB (kRope)][operand ring nslot x 32 KB]
+//                [B_k ring nb x gh x 16 KB (kRope)][operand ring nslot x 32 KB]
 //                [P double buffer 2 x 8 KB][raw ring nraw x raw_bytes]
-template <bool kRope>
+// kG: query heads per KV head (compile time for the keys-before-RoPE dots, so that the
+// kG accumulation chains interleave; 0 for the rank-space kernel).
+template <bool kRope, int kG>
 __global__ void __launch_bounds__(kThreads, 1)
     k_decode_tc_i4(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_b,
                    const I4Params p) {
@@ -200,7 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   Aux* aux = reinterpret_cast<Aux*>(smem_raw);
   uint8_t* q_s = smem_raw + kAuxBytes;
   uint8_t* bring = q_s + p.q_bytes;
-  uint8_t* ring = bring + (kRope ? kNB * kSlotBytes : 0);
+  const uint32_t b_slot_bytes = kRope ? (uint32_t)(p.gh * kSubBytes) : 0u;
+  uint8_t* ring = bring + (kRope ? p.nb * b_slot_bytes : 0);
   uint8_t* p_s = ring + p.nslot * kSlotBytes;
   uint8_t* raw = p_s + 2 * kPBytes;
   constexpr int kOC = kRope ? kOColR : kOCol;
@@ -234,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (kRope) {
       ptx::mbar_init(&aux->k_full, 1);
       ptx::mbar_init(&aux->k_empty, kSmWarps);
-      for (int k = 0; k < kNB; ++k) {
+      for (int k = 0; k < p.nb; ++k) {
         ptx::mbar_init(&aux->b_full[k], 1);
         ptx::mbar_init(&aux->b_empty[k], 1);
       }
@@ -316,25 +323,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (kRope && warp == 2) {
       // ------------------------------------------------------------- B_k producer (kRope)
-      // (tile, chunk c, pair head h) in the MMA's order; B_k is written before the cache
-      // is used, so no grid-dependency wait is needed.
+      // (tile, 64-rank sub-block) in the MMA's order, one box of the pair's gh x 128 rows;
+      // B_k is written before the cache is used, so no grid-dependency wait is needed.
       if (lane == 0 && ntiles > 0) {
-        const int total = ntiles * p.ck * p.gh;
+        const int total = ntiles * p.kb_k;
         bool ok = true;
         int issued = 0;
         for (int k = 0; k < total; ++k) {
-          const int slot = k % kNB;
-          if (k >= kNB && !(ok = wait_b(&aux->b_empty[slot], ((k / kNB) - 1) & 1, aux, p.err))) break;
-          const int h = k % p.gh, c = (k / p.gh) % p.ck;
-          const int row = (pair * p.gh + h) * kRD;
-          uint8_t* dst = bring + slot * kSlotBytes;
-          ptx::mbar_arrive_expect_tx(&aux->b_full[slot], (uint32_t)kSlotBytes);
-          ptx::tma_load_2d(dst, &tm_b, &aux->b_full[slot], c * 128, row);
-          ptx::tma_load_2d(dst + kSubBytes, &tm_b, &aux->b_full[slot], c * 128 + 64, row);
+          const int slot = k % p.nb;
+          if (k >= p.nb && !(ok = wait_b(&aux->b_empty[slot], ((k / p.nb) - 1) & 1, aux, p.err))) break;
+          const int sb = k % p.kb_k;
+          ptx::mbar_arrive_expect_tx(&aux->b_full[slot], b_slot_bytes);
+          ptx::tma_load_2d(bring + slot * b_slot_bytes, &tm_b, &aux->b_full[slot], sb * 64, pair * p.gh * kRD);
           issued = k + 1;
         }
         if (!ok)
-          for (int k = max(0, issued - kNB); k < issued; ++k) drain_wait(&aux->b_full[k % kNB], (k / kNB) & 1);
+          for (int k = max(0, issued - p.nb); k < issued; ++k) drain_wait(&aux->b_full[k % p.nb], (k / p.nb) & 1);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------- MMA issuer
@@ -348,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t qdesc0 = ptx::smem_desc(ptx::smem_u32(q_s), 16, 1024, 2);        // q~, K-major SW128
         const uint64_t vdesc0 = ptx::smem_desc(ptx::smem_u32(ring), kSubBytes, 1024, 2); // Z_v, MN-major SW128
         const uint64_t pdesc0 = ptx::smem_desc(ptx::smem_u32(p_s), 128, 2048, 0);       // P, MN-major
-        const uint32_t idk = ptx::idesc_f16(0, 0, 0, 128, kRD);  // GEMM0 (kRope): K-major x K-major
+        const uint32_t idk = ptx::idesc_f16(0, 0, 0, 128, kRope ? p.gh * kRD : 128);   // GEMM0 (kRope)
         const uint64_t bdesc0 = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, 2);      // B_k, K-major SW128
         bool ok = kRope ? true : wait_b(&aux->q_full, 0, aux, p.err);
         ptx::tc_fence_after();
@@ -359,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bool is_v;
           tc::unit_of(u, ntiles, &tile, &is_v);
           if (kRope && !is_v) {
-            // GEMM0(tile): K^_h = Z_k B_k,h for the pair's heads, into columns [128 h, +128)
+            // GEMM0(tile): [K^_0 | K^_1] = Z_k [B_k,0 | B_k,1], columns [128 h, +128) per head
             if (tile >= 1 && !(ok = wait_b(&aux->k_empty, (tile - 1) & 1, aux, p.err))) break;
             ptx::tc_fence_after();
             for (int c = 0; c < p.ck && ok; ++c, ++pos) {
@@ -367,17 +371,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
               const uint64_t a0 = kdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
-              const int nk = min(8, (p.r_k - c * 128) >> 4);
-              for (int h = 0; h < p.gh; ++h, ++bpos) {
-                const int bs = bpos % kNB;
-                if (!(ok = wait_b(&aux->b_full[bs], (bpos / kNB) & 1, aux, p.err))) break;
+              for (int sb = 0; sb < 2 && c * 128 + sb * 64 < p.r_k; ++sb, ++bpos) {
+                const int bs = bpos % p.nb;
+                if (!(ok = wait_b(&aux->b_full[bs], (bpos / p.nb) & 1, aux, p.err))) break;
                 ptx::tc_fence_after();
-                const uint64_t b0 = bdesc0 + (uint64_t)((bs * kSlotBytes) >> 4);
-                // A and B share the layout: 64-rank sub-blocks of 16 KB, 32 bytes per step
-                for (int kk = 0; kk < nk; ++kk) {
-                  const uint32_t o = (uint32_t)((kk >> 2) * (kSubBytes >> 4) + (kk & 3) * 2);
-                  ptx::mma_f16(tmem + h * kRD, a0 + o, b0 + o, idk, (c | kk) ? 1u : 0u);
-                }
+                const uint64_t b0 = bdesc0 + (uint64_t)((bs * b_slot_bytes) >> 4);
+                // sub-block sb of the A slot (16 KB) against the B slot; 32 bytes per step
+                const int nk = min(4, (p.r_k - c * 128 - sb * 64) >> 4);
+                for (int kk = 0; kk < nk; ++kk)
+                  ptx::mma_f16(tmem, a0 + (uint64_t)(sb * (kSubBytes >> 4) + kk * 2), b0 + (uint64_t)(kk * 2), idk,
+                               (c | sb | kk) ? 1u : 0u);
                 ptx::mma_commit(&aux->b_empty[bs]);
               }
               if (!ok) break;
@@ -385,6 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             ptx::mma_commit(&aux->k_full);
+            if (tile < 16) tc::trace_stamp(p.trace, 3 + 4 * tile);
           } else if (!is_v) {
             // GEMM1(tile): S[tile % 2] = Z_k q~^T
             const int sb2 = tile & 1;
@@ -451,6 +455,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // keys before RoPE: the query rows are read here, from shared memory
       if (kRope) ok = ptx::named_bar_and(1, 128, wait_b(&aux->q_full, 0, aux, p.err));
       const float* q_f = reinterpret_cast<const float*>(q_s);
+      // rotation factors: cs holds the chunk in use, csn the one after it
+      float cs[32], csn[32];
+      auto load_cs = [&](float(&dst)[32], int tile_i, int c0) {
+        const int t = tok_begin + tile_i * kTile + row;
+        const float2* src = p.rope_cs + (size_t)(t < tok_end ? t : tok_begin) * (kRD / 2) + c0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(src) + k);
+          dst[4 * k] = v.x;
+          dst[4 * k + 1] = v.y;
+          dst[4 * k + 2] = v.z;
+          dst[4 * k + 3] = v.w;
+        }
+      };
+      if (kRope) load_cs(cs, 0, 0);
       for (int i = 0; i < ntiles && ok; ++i) {
         const int k2 = i & 1;
         const bool valid = tok_begin + i * kTile + row < tok_end;
@@ -460,22 +479,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = ptx::named_bar_and(1, 128, wait_b(&aux->k_full, i & 1, aux, p.err));
           if (!ok) break;
           ptx::tc_fence_after();
+          if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 4 + 4 * i);
           // score of query slot 16 h + jj: q_jj . RoPE_t(K^_h[t]), pairs (c, c + 64)
-          const int t = tok_begin + i * kTile + row;
-          const float2* cs_row = p.rope_cs + (size_t)(valid ? t : tok_begin) * (kRD / 2);
 #pragma unroll
           for (int j = 0; j < 32; ++j) s[j] = 0.f;
 #pragma unroll 1
           for (int c0 = 0; c0 < kRD / 2; c0 += 16) {
-            float cs[32];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const float4 v = __ldg(reinterpret_cast<const float4*>(cs_row + c0) + k);
-              cs[4 * k] = v.x;
-              cs[4 * k + 1] = v.y;
-              cs[4 * k + 2] = v.z;
-              cs[4 * k + 3] = v.w;
-            }
+            if (c0 + 16 < kRD / 2) load_cs(csn, i, c0 + 16);
+            else if (i + 1 < ntiles) load_cs(csn, i + 1, 0);
 #pragma unroll
             for (int h = 0; h < kGHMax; ++h) {
               if (h < p.gh) {
@@ -491,28 +502,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                   r2[k] = e * cs[2 * k] + a * cs[2 * k + 1];
                 }
 #pragma unroll
-                for (int jj = 0; jj < kMaxG; ++jj) {
-                  if (jj < p.gsz) {
-                    const float* qr = q_f + (size_t)(h * p.gsz + jj) * kRD + c0;
-                    float acc = s[h * kMaxG + jj];
+                for (int k = 0; k < 16; k += 4) {
 #pragma unroll
-                    for (int k = 0; k < 16; k += 4) {
-                      const float4 qa = *reinterpret_cast<const float4*>(qr + k);
-                      const float4 qb = *reinterpret_cast<const float4*>(qr + kRD / 2 + k);
-                      acc = fmaf(qa.x, r1[k], acc);
-                      acc = fmaf(qa.y, r1[k + 1], acc);
-                      acc = fmaf(qa.z, r1[k + 2], acc);
-                      acc = fmaf(qa.w, r1[k + 3], acc);
-                      acc = fmaf(qb.x, r2[k], acc);
-                      acc = fmaf(qb.y, r2[k + 1], acc);
-                      acc = fmaf(qb.z, r2[k + 2], acc);
-                      acc = fmaf(qb.w, r2[k + 3], acc);
-                    }
+                  for (int jj = 0; jj < kG; ++jj) {
+                    const float* qr = q_f + (size_t)(h * kG + jj) * kRD + c0 + k;
+                    const float4 qa = *reinterpret_cast<const float4*>(qr);
+                    const float4 qb = *reinterpret_cast<const float4*>(qr + kRD / 2);
+                    float acc = s[h * kMaxG + jj];
+                    acc = fmaf(qa.x, r1[k], acc);
+                    acc = fmaf(qa.y, r1[k + 1], acc);
+                    acc = fmaf(qa.z, r1[k + 2], acc);
+                    acc = fmaf(qa.w, r1[k + 3], acc);
+                    acc = fmaf(qb.x, r2[k], acc);
+                    acc = fmaf(qb.y, r2[k + 1], acc);
+                    acc = fmaf(qb.z, r2[k + 2], acc);
+                    acc = fmaf(qb.w, r2[k + 3], acc);
                     s[h * kMaxG + jj] = acc;
                   }
                 }
               }
             }
+#pragma unroll
+            for (int k = 0; k < 32; ++k) cs[k] = csn[k];
           }
           // K^ has been read: GEMM0 of the next tile may overwrite it
           ptx::tc_fence_before();
@@ -762,7 +773,7 @@ int q_bytes_for(const lr_cache_desc* d) {
 }
 
 struct I4Layout {
-  int nslot, nraw;
+  int nslot, nraw, nb;
   uint32_t raw_bytes, raw_params;
   size_t smem;
 };
@@ -775,8 +786,22 @@ bool choose_layout(const lr_cache_desc* d, I4Layout* L) {
   const int G = std::max((d->rank_k + 31) / 32, (d->rank_v + 31) / 32);
   L->raw_params = (uint32_t)G * 2048u;
   L->raw_bytes = (uint32_t)G * 2560u;
-  const size_t fixed =
-      (size_t)kAuxBytes + q_bytes_for(d) + (d->rope_in_kernel ? (size_t)kNB * kSlotBytes : 0) + 2 * kPBytes;
+  const size_t fixed = (size_t)kAuxBytes + q_bytes_for(d) + 2 * kPBytes;
+  if (d->rope_in_kernel) {
+    // two operand slots and two raw slots, then B_k slots up to one tile's worth (the next
+    // tile's sub-blocks load while the current one is rotated), then raw slots
+    const size_t bslot = (size_t)(d->n_kv_heads % 2 == 0 ? 2 : 1) * kSubBytes;
+    const int kb = (d->rank_k + 63) / 64;
+    const size_t base = fixed + 2 * (size_t)kSlotBytes + 2 * (size_t)L->raw_bytes;
+    if (base + 2 * bslot > (size_t)kSmemLimit) return false;
+    L->nb = std::min(kNBMax, std::max(2, std::min(kb, (int)(((size_t)kSmemLimit - base) / bslot))));
+    L->nslot = 2;
+    const size_t used = fixed + (size_t)L->nb * bslot + 2 * (size_t)kSlotBytes;
+    L->nraw = std::min(kMaxRaw, (int)(((size_t)kSmemLimit - used) / L->raw_bytes));
+    L->smem = used + (size_t)L->nraw * L->raw_bytes;
+    return true;
+  }
+  L->nb = 0;
   for (int ns = kMaxSlots; ns >= 2; --ns) {
     if (fixed + (size_t)ns * kSlotBytes > (size_t)kSmemLimit) continue;
     const int nr =
@@ -802,7 +827,10 @@ bool tc_i4_supported(const lr_cache_desc* d) {
   if (d->quant_bits != 4 || d->quant_group != 32) return false;
   if (d->dtype != LR_BF16) return false;
   if (d->n_q_heads > 32 || d->rank_v > 512) return false;
-  if (d->rope_in_kernel && (d->head_dim != kRD || d->n_q_heads / d->n_kv_heads > kMaxG)) return false;
+  if (d->rope_in_kernel) {
+    const int g = d->n_q_heads / d->n_kv_heads;
+    if (d->head_dim != kRD || (g != 4 && g != 7 && g != 8)) return false;
+  }
   I4Layout L;
   return choose_layout(d, &L);
 }
@@ -831,7 +859,7 @@ cudaError_t tc_i4_prepare(lr_cache* c, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     cuuint64_t dims[2] = {(cuuint64_t)r_pad, (cuuint64_t)c->D};
     cuuint64_t strides[1] = {(cuuint64_t)r_pad * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)kRD};
+    cuuint32_t box[2] = {64, (cuuint32_t)(kv_per_cta(&d) * kRD)};
     if (!tc::make_map(&st->bk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, st->bk16, 2, dims, strides, box))
       return cudaErrorInvalidValue;
     st->q = st->bk;   // unused by the kRope kernel
@@ -854,6 +882,7 @@ cudaError_t tc_i4_prepare(lr_cache* c, cudaStream_t s) {
   if (!choose_layout(&d, &L)) return cudaErrorNotSupported;
   st->nslot = L.nslot;
   st->nraw = L.nraw;
+  st->nb = L.nb;
   st->raw_bytes = L.raw_bytes;
   st->raw_params = L.raw_params;
   st->q_bytes = (uint32_t)q_bytes_for(&d);
@@ -900,28 +929,31 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   p.part_o = c->part_o;
   p.part_ml = c->part_ml;
   p.err = c->dev_err;
-  p.trace = rope ? nullptr : c->trace;    // the timeline covers the rank-space grid only
+  // the timeline buffer holds S_max CTAs per sequence
+  p.trace = n_splits * tc_i4_split_ctas(&d) <= c->S_max ? c->trace : nullptr;
   p.qf = c->qt;
   p.rope_cs = c->rope_cs;
   p.gh = kv_per_cta(&d);
   p.gsz = d.n_q_heads / d.n_kv_heads;
   p.q_load_bytes = (uint32_t)(p.gh * p.gsz * kRD * 4);
-  auto kern = rope ? k_decode_tc_i4<true> : k_decode_tc_i4<false>;
-  static std::atomic<uint32_t> optin_done[2] = {0, 0};
-  cudaError_t e = smem_optin(kern, optin_done[rope ? 1 : 0]);
+  p.nb = st->nb;
+  // instantiation: 0 rank space; 1, 2, 3 keys before RoPE with 4, 7, 8 query heads per KV head
+  using Kern = void (*)(CUtensorMap, CUtensorMap, I4Params);
+  static const Kern kerns[4] = {k_decode_tc_i4<false, 0>, k_decode_tc_i4<true, 4>, k_decode_tc_i4<true, 7>,
+                                k_decode_tc_i4<true, 8>};
+  const int ki = !rope ? 0 : (p.gsz == 4 ? 1 : (p.gsz == 7 ? 2 : (p.gsz == 8 ? 3 : -1)));
+  if (ki < 0) return cudaErrorNotSupported;
+  const Kern kern = kerns[ki];
+  static std::atomic<uint32_t> optin_done[4] = {0, 0, 0, 0};
+  cudaError_t e = smem_optin(kern, optin_done[ki]);
   if (e != cudaSuccess) return e;
   // The register rebalancing assumes the launch allocation the split was sized for.
-  static const int regs[2] = {[] {
-                                cudaFuncAttributes fa;
-                                return cudaFuncGetAttributes(&fa, k_decode_tc_i4<false>) == cudaSuccess ? fa.numRegs
-                                                                                                        : -1;
-                              }(),
-                              [] {
-                                cudaFuncAttributes fa;
-                                return cudaFuncGetAttributes(&fa, k_decode_tc_i4<true>) == cudaSuccess ? fa.numRegs
-                                                                                                       : -1;
-                              }()};
-  if (regs[rope ? 1 : 0] != kLaunchRegs) return cudaErrorInvalidConfiguration;
+  static std::atomic<int> regs[4] = {0, 0, 0, 0};
+  if (regs[ki].load() == 0) {
+    cudaFuncAttributes fa;
+    regs[ki].store(cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1);
+  }
+  if (regs[ki].load() != kLaunchRegs) return cudaErrorInvalidConfiguration;
   const dim3 grid = rope ? dim3(d.n_kv_heads / p.gh, n_splits, d.batch) : dim3(n_splits, d.batch);
   return launch_pdl(kern, grid, dim3(kThreads), st->smem, s, st->q, st->bk, p);
 }

@@ -49,7 +49,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 __device__ __forceinline__ void trace_stamp(unsigned long long* trace, int slot) {
-  if (trace) trace[((size_t)blockIdx.y * gridDim.x + blockIdx.x) * kTraceSlots + slot] = ptx::globaltimer();
+  if (trace)
+    trace[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * kTraceSlots + slot] =
+        ptx::globaltimer();
 }
 
 // Unit u of the pipelined tile order, in which the scores of tile s+1 are computed before
