@@ -81,7 +81,10 @@ constexpr int kDqWarps = 8;                // arrivals per operand slot / raw sl
 constexpr int kSmWarps = 4;                // softmax warps (one arrival each)
 constexpr int kLaunchRegs = 128;
 constexpr int kRegsCtl = 56, kRegsSoftmax = 208, kRegsDq = 104;
+constexpr int kRegsSoftmaxRope = 216;      // keys before RoPE: rotation and query dots too
 static_assert(128 * kRegsCtl + 128 * kRegsSoftmax + 256 * kRegsDq <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+static_assert(128 * kRegsCtl + 128 * kRegsSoftmaxRope + 256 * kRegsDq <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr int kSubBytes = 128 * 128;       // 128 tokens x 64 ranks x 2 B
 constexpr int kSlotBytes = 2 * kSubBytes;  // 128 tokens x 128 ranks
@@ -187,6 +190,21 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, uint32_t s2, uint32_t z2) 
 __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
+}
+
+// Two fp32 lanes in one 64-bit register for the paired FMA: d = a * b + c per lane,
+// each rounded once (IEEE fma).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi2(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
 }
 
 // Shared memory: [aux 2 KB][q~ per 64-rank sub-block | fp32 query rows (kRope)]
@@ -442,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     }
   } else if (warp < kDqWarp0) {
-    ptx::setmaxnreg_inc<kRegsSoftmax>();
+    ptx::setmaxnreg_inc<kRope ? kRegsSoftmaxRope : kRegsSoftmax>();
     if (ntiles > 0) {
       // ------------------------------------------------------------- softmax / epilogue
       const int qd = warp & 3;
@@ -501,25 +519,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                   r1[k] = a * cs[2 * k] - e * cs[2 * k + 1];
                   r2[k] = e * cs[2 * k] + a * cs[2 * k + 1];
                 }
+                // paired fp32 FMAs over adjacent elements (two partial sums per score,
+                // folded at the end of the chunk)
+                uint64_t acc[kG > 0 ? kG : 1];
+#pragma unroll
+                for (int jj = 0; jj < kG; ++jj) acc[jj] = pack2(s[h * kMaxG + jj], 0.f);
 #pragma unroll
                 for (int k = 0; k < 16; k += 4) {
+                  const uint64_t ra = pack2(r1[k], r1[k + 1]), rb = pack2(r1[k + 2], r1[k + 3]);
+                  const uint64_t rc = pack2(r2[k], r2[k + 1]), rd = pack2(r2[k + 2], r2[k + 3]);
 #pragma unroll
                   for (int jj = 0; jj < kG; ++jj) {
                     const float* qr = q_f + (size_t)(h * kG + jj) * kRD + c0 + k;
                     const float4 qa = *reinterpret_cast<const float4*>(qr);
                     const float4 qb = *reinterpret_cast<const float4*>(qr + kRD / 2);
-                    float acc = s[h * kMaxG + jj];
-                    acc = fmaf(qa.x, r1[k], acc);
-                    acc = fmaf(qa.y, r1[k + 1], acc);
-                    acc = fmaf(qa.z, r1[k + 2], acc);
-                    acc = fmaf(qa.w, r1[k + 3], acc);
-                    acc = fmaf(qb.x, r2[k], acc);
-                    acc = fmaf(qb.y, r2[k + 1], acc);
-                    acc = fmaf(qb.z, r2[k + 2], acc);
-                    acc = fmaf(qb.w, r2[k + 3], acc);
-                    s[h * kMaxG + jj] = acc;
+                    acc[jj] = ffma2(pack2(qa.x, qa.y), ra, acc[jj]);
+                    acc[jj] = ffma2(pack2(qa.z, qa.w), rb, acc[jj]);
+                    acc[jj] = ffma2(pack2(qb.x, qb.y), rc, acc[jj]);
+                    acc[jj] = ffma2(pack2(qb.z, qb.w), rd, acc[jj]);
                   }
                 }
+#pragma unroll
+                for (int jj = 0; jj < kG; ++jj) s[h * kMaxG + jj] = lo2(acc[jj]) + hi2(acc[jj]);
               }
             }
 #pragma unroll
