@@ -58,8 +58,8 @@ typedef enum lr_path {
   LR_PATH_AUTO = 0,   /* tensor-core path where supported, else SIMT           */
   LR_PATH_SIMT = 1,   /* fp32 CUDA-core path (every configuration)             */
   LR_PATH_TC = 2      /* tcgen05 path: bf16 / int4 latents with keys after RoPE;
-                         int4 latents with keys before RoPE when head_dim = 128
-                         and Hq/Hkv is 4, 7 or 8 (keys rebuilt per tile)        */
+                         int4 latents with keys before RoPE when head_dim = 128,
+                         Hq = 7 Hkv and Hkv is even (keys rebuilt per tile)     */
 } lr_path;
 
 /* Cache description.  All counts are per layer; one cache holds one layer. */

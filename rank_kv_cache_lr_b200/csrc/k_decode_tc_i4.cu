@@ -100,6 +100,7 @@ constexpr int kRD = 128;                   // head dim of the rebuilt keys
 constexpr int kGHMax = 2;                  // KV heads per CTA (K^ of both fills 256 columns)
 constexpr int kMaxG = 32 / kGHMax;         // query slots per KV head
 constexpr int kOColR = 256;                // TMEM: O~ chunk c in columns [256 + 32c, +32)
+constexpr int kRopeG = 7;                  // query heads per KV head of the instantiated variant
 constexpr int kNBMax = 4;                  // B_k ring slots (kv heads x 128 rows x 64 ranks, fp16)
 constexpr int kMaxRaw = 6;                 // raw slot: one side of one tile, codes (G x 2 KB)
                                            // then {scale, zero} words (G x 512 B)
@@ -211,7 +212,8 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
 //                [B_k ring nb x gh x 16 KB (kRope)][operand ring nslot x 32 KB]
 //                [P double buffer 2 x 8 KB][raw ring nraw x raw_bytes]
 // kG: query heads per KV head (compile time for the keys-before-RoPE dots, so that the
-// kG accumulation chains interleave; 0 for the rank-space kernel).
+// kG accumulation chains interleave; 0 for the rank-space kernel).  A runtime count with a
+// guard inside the unrolled loop serialised the chains (13 us per tile instead of 7).
 template <bool kRope, int kG>
 __global__ void __launch_bounds__(kThreads, 1)
     k_decode_tc_i4(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_b,
@@ -848,10 +850,11 @@ bool tc_i4_supported(const lr_cache_desc* d) {
   if (d->quant_bits != 4 || d->quant_group != 32) return false;
   if (d->dtype != LR_BF16) return false;
   if (d->n_q_heads > 32 || d->rank_v > 512) return false;
-  if (d->rope_in_kernel) {
-    const int g = d->n_q_heads / d->n_kv_heads;
-    if (d->head_dim != kRD || (g != 4 && g != 7 && g != 8)) return false;
-  }
+  // keys before RoPE: instantiated for the shape the parity tests cover (d = 128, seven
+  // query heads per KV head, KV heads in pairs); other shapes take the CUDA-core path
+  if (d->rope_in_kernel &&
+      (d->head_dim != kRD || d->n_q_heads != kRopeG * d->n_kv_heads || d->n_kv_heads % kGHMax != 0))
+    return false;
   I4Layout L;
   return choose_layout(d, &L);
 }
@@ -958,18 +961,17 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   p.gsz = d.n_q_heads / d.n_kv_heads;
   p.q_load_bytes = (uint32_t)(p.gh * p.gsz * kRD * 4);
   p.nb = st->nb;
-  // instantiation: 0 rank space; 1, 2, 3 keys before RoPE with 4, 7, 8 query heads per KV head
+  // instantiation: 0 rank space; 1 keys before RoPE
   using Kern = void (*)(CUtensorMap, CUtensorMap, I4Params);
-  static const Kern kerns[4] = {k_decode_tc_i4<false, 0>, k_decode_tc_i4<true, 4>, k_decode_tc_i4<true, 7>,
-                                k_decode_tc_i4<true, 8>};
-  const int ki = !rope ? 0 : (p.gsz == 4 ? 1 : (p.gsz == 7 ? 2 : (p.gsz == 8 ? 3 : -1)));
-  if (ki < 0) return cudaErrorNotSupported;
+  static const Kern kerns[2] = {k_decode_tc_i4<false, 0>, k_decode_tc_i4<true, kRopeG>};
+  if (rope && (p.gsz != kRopeG || p.gh != kGHMax)) return cudaErrorNotSupported;
+  const int ki = rope ? 1 : 0;
   const Kern kern = kerns[ki];
-  static std::atomic<uint32_t> optin_done[4] = {0, 0, 0, 0};
+  static std::atomic<uint32_t> optin_done[2] = {0, 0};
   cudaError_t e = smem_optin(kern, optin_done[ki]);
   if (e != cudaSuccess) return e;
   // The register rebalancing assumes the launch allocation the split was sized for.
-  static std::atomic<int> regs[4] = {0, 0, 0, 0};
+  static std::atomic<int> regs[2] = {0, 0};
   if (regs[ki].load() == 0) {
     cudaFuncAttributes fa;
     regs[ki].store(cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1);

@@ -99,11 +99,11 @@ def test_plan_covers_history_exactly(lib, length, batch, path):
     assert p.n_splits * batch <= max(2 * 148 + batch, batch)
 
 
-@pytest.mark.parametrize("n_kv_heads, pairs", [(4, 2), (2, 1), (1, 1), (3, 3)])
+@pytest.mark.parametrize("n_kv_heads, pairs", [(4, 2), (2, 1)])
 @pytest.mark.parametrize("rank_k", [128, 256, 448])
 def test_plan_keys_before_rope_int4_on_kv_head_pairs(lib, n_kv_heads, pairs, rank_k):
-    """int4 keys before RoPE take the tensor-core path with one CTA per pair of KV heads
-    (or per KV head when their count is odd), within one wave of 148 SMs."""
+    """int4 keys before RoPE take the tensor-core path with one CTA per pair of KV heads,
+    within one wave of 148 SMs."""
     d = _qwen(lib, n_q_heads=7 * n_kv_heads, n_kv_heads=n_kv_heads, rank_k=rank_k, rank_v=448,
               quant_bits=4, rope_in_kernel=1, capacity=32768)
     p = lib.lr_plan_decode(d, 32768, 148)
@@ -113,8 +113,12 @@ def test_plan_keys_before_rope_int4_on_kv_head_pairs(lib, n_kv_heads, pairs, ran
     assert (p.n_splits - 1) * p.split_tokens < 32768 <= p.n_splits * p.split_tokens
 
 
-def test_plan_keys_before_rope_other_head_dims_use_cuda_cores(lib):
-    d = _qwen(lib, head_dim=64, quant_bits=4, rope_in_kernel=1)
+@pytest.mark.parametrize("shape", [dict(head_dim=64), dict(n_q_heads=16, n_kv_heads=4),
+                                   dict(n_q_heads=7, n_kv_heads=1), dict(n_q_heads=21, n_kv_heads=3)])
+def test_plan_keys_before_rope_other_shapes_use_cuda_cores(lib, shape):
+    """The tensor-core keys-before-RoPE variant exists for d = 128, seven query heads per KV
+    head and KV heads in pairs; every other shape decodes on CUDA cores."""
+    d = _qwen(lib, quant_bits=4, rope_in_kernel=1, **shape)
     assert lib.lr_plan_decode(d, 4096, 148).path == lib.LR_PATH_SIMT
 
 
