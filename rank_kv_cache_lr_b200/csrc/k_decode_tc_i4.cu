@@ -126,6 +126,24 @@ struct I4Params {
   int nb;                   // B_k ring slots of gh * 16 KB
 };
 
+// Barriers (arrival count; who arrives -> who waits).  Every ring is used in the unit order
+// K(0), K(1), V(0), K(2), ..., and phase k of a barrier is waited with parity k & 1.
+//   raw_full[nraw]    1 + tx   producer's two bulk copies -> dequantisation warps
+//   raw_empty[nraw]   8        dequantisation warps -> producer
+//   slot_full[nslot]  8        dequantisation warps (fenced stores) -> MMA issuer
+//   slot_empty[nslot] 1        MMA commit -> dequantisation warps
+//   q_full            1 + tx   producer (after the grid-dependency wait) -> MMA issuer, or
+//                              the softmax warps for keys before RoPE
+//   s_full[2]         1        MMA commit of GEMM1 -> softmax warps
+//   s_empty[2]        4        softmax warps (scores read) -> MMA issuer
+//   p_full[2]         4        softmax warps (fenced P stores) -> MMA issuer
+//   p_empty[2]        1        MMA commit of GEMM2 -> softmax warps (P reuse, O~ rescale)
+//   o_final           1        MMA commit after the last unit -> softmax warps (epilogue)
+//   keys before RoPE, in place of s_full / s_empty:
+//   k_full            1        MMA commit of GEMM0 -> softmax warps
+//   k_empty           4        softmax warps (K^ read) -> MMA issuer (next GEMM0)
+//   b_full[nb]        1 + tx   B_k producer (warp 2) -> MMA issuer
+//   b_empty[nb]       1        MMA commit -> B_k producer
 struct Aux {
   uint64_t slot_full[kMaxSlots];
   uint64_t slot_empty[kMaxSlots];
@@ -133,7 +151,7 @@ struct Aux {
   uint64_t raw_empty[kMaxRaw];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
   uint64_t q_full, o_final;
-  uint64_t k_full, k_empty, b_full[kNBMax], b_empty[kNBMax];   // keys before RoPE
+  uint64_t k_full, k_empty, b_full[kNBMax], b_empty[kNBMax];
   uint32_t tmem_base;
   int abort_flag;
   float red[4][32];
