@@ -61,6 +61,15 @@ struct TcParams {
   unsigned long long* trace;   // optional per-CTA timeline (kTraceSlots stamps per CTA), or null
 };
 
+// Barriers (arrival count; who arrives -> who waits); phase k is waited with parity k & 1.
+//   slot_full[nslot]  1 + tx   producer's TMA boxes of one 128-rank chunk -> MMA issuer
+//   slot_empty[nslot] 1        MMA commit -> producer
+//   q_full            1 + tx   producer (after the grid-dependency wait) -> MMA issuer
+//   s_full[2]         1        MMA commit of GEMM1 -> softmax warps
+//   s_empty[2]        4        softmax warps (scores read) -> MMA issuer
+//   p_full            4        softmax warps (fenced P stores) -> MMA issuer
+//   p_empty           1        MMA commit of GEMM2 -> softmax warps (P reuse, O~ rescale)
+//   o_final           1        MMA commit after the last unit -> softmax warps (epilogue)
 struct Aux {
   uint64_t slot_full[kMaxSlots];
   uint64_t slot_empty[kMaxSlots];

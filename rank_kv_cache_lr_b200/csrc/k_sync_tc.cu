@@ -37,6 +37,13 @@ struct SyncParams {
   int* err;
 };
 
+// Barriers (arrival count; who arrives -> who waits); phase k is waited with parity k & 1.
+//   z_full      1 + tx   producer's TMA boxes of one Z tile -> MMA issuer
+//   z_empty     1        the storing thread, once its TMA store has read the tile -> producer
+//   r_full[2]   1 + tx   producer's R chunk (hi and lo rows) -> MMA issuer
+//   r_empty[2]  1        MMA commit -> producer
+//   d_full      1        MMA commit of a tile's product -> epilogue warps
+//   d_empty     4        epilogue warps (product read from TMEM) -> MMA issuer
 struct Aux {
   uint64_t z_full, z_empty, d_full, d_empty;
   uint64_t r_full[2], r_empty[2];
