@@ -32,6 +32,12 @@ def test_library_exports_every_declared_symbol(lib):
     assert not missing, missing
 
 
+def test_binding_keeps_every_declared_name(lib):
+    """The Python binding exposes each C call under its own name."""
+    missing = [n for n in declared_functions() if not callable(getattr(lib, n, None))]
+    assert not missing, missing
+
+
 def test_struct_sizes_match_binding(lib):
     assert lib.lr_abi_struct_sizes() == (ctypes.sizeof(lib.lr_cache_desc),
                                          ctypes.sizeof(lib.lr_cache_view),
