@@ -171,6 +171,30 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.rows)}
 
 
+def roofline_entry(kname: str, bytes_per_step: float, flops_per_step: float, kern_ms: float,
+                   peaks: dict, peak_src: str, traf) -> dict:
+    """The `roofline` object of the bench line for the main decode kernel (summed over the
+    step's layers, `kern_ms` per step).  HBM-bound kernels: latent bytes against the measured
+    copy rate.  With `flops_per_step` > 0 (keys rebuilt per tile on the tensor cores) the
+    bound is the contraction, against the sustained bf16 rate (fp16 operands run at the same
+    nominal rate), with the HBM view alongside."""
+    gbs = bytes_per_step / (kern_ms * 1e-3) / 1e9
+    timing = "CUDA events around each layer's decode kernel (separate graph capture), summed over layers"
+    traffic = traf["bytes_per_launch"] if traf else None
+    if flops_per_step <= 0:
+        peak = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
+        return {"bound": "hbm", "kernel": kname, "achieved": round(gbs, 1), "peak": peak,
+                "peak_source": peak_src, "unit": "GB/s", "frac": round(gbs / peak, 4),
+                "kernel_us": round(1000 * kern_ms, 2), "kernel_timing": timing, "traffic": traffic}
+    tflops = flops_per_step / (kern_ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_TFLOPS_SUSTAINED)
+    return {"bound": "tensor", "kernel": kname, "achieved": round(tflops, 1), "peak": peak,
+            "peak_source": peak_src + " (bf16 sustained; fp16 operands run at the same rate)",
+            "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "flops_per_step": flops_per_step,
+            "hbm_gbs": round(gbs, 1), "kernel_us": round(1000 * kern_ms, 2), "kernel_timing": timing,
+            "traffic": traffic}
+
+
 def traffic_record(kernel: str):
     """DRAM traffic per launch from a committed ncu summary, valid only while the kernel
     source is unchanged (matched by hash)."""
@@ -431,7 +455,6 @@ def run_ours(args):
     value = job_rate(bytes_per_step, K, world, total_ms)
     peaks, peak_src = measured_peaks()
     kern_mean = statistics.mean(kern_ms)
-    achieved = bytes_per_step / (kern_mean * 1e-3) / 1e9
     kname = ("decode_tc_i4" if qb == 4 else "decode_tc") if plan.path == lr.LR_PATH_TC else "decode_simt"
     rope = bool(W.get("rope"))
     if rope:
@@ -457,23 +480,7 @@ def run_ours(args):
                    "decode_path": "tcgen05" if plan.path == lr.LR_PATH_TC else "simt",
                    "splits": plan.n_splits, "cuda_graph": bool(args.graph),
                    "launches_per_step": launches_per_step},
-        "roofline": ({"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
-                      "peak": peaks.get("hbm_gbs", FALLBACK_HBM_GBS), "peak_source": peak_src,
-                      "unit": "GB/s", "frac": round(achieved / peaks.get("hbm_gbs", FALLBACK_HBM_GBS), 4),
-                      "kernel_us": round(1000 * kern_mean, 2),
-                      "kernel_timing": "CUDA events around each layer's decode kernel (separate graph capture), summed over layers",
-                      "traffic": (traf["bytes_per_launch"] if traf else None)} if not rope else
-                     {"bound": "tensor", "kernel": kname,
-                      "achieved": round(roof_flops / (kern_mean * 1e-3) / 1e12, 1),
-                      "peak": peaks.get("bf16_tflops_sustained", FALLBACK_TFLOPS_SUSTAINED),
-                      "peak_source": peak_src + " (bf16 sustained; fp16 operands run at the same rate)",
-                      "unit": "TFLOP/s",
-                      "frac": round(roof_flops / (kern_mean * 1e-3) / 1e12
-                                    / peaks.get("bf16_tflops_sustained", FALLBACK_TFLOPS_SUSTAINED), 4),
-                      "flops_per_step": roof_flops, "hbm_gbs": round(achieved, 1),
-                      "kernel_us": round(1000 * kern_mean, 2),
-                      "kernel_timing": "CUDA events around each layer's decode kernel (separate graph capture), summed over layers",
-                      "traffic": (traf["bytes_per_launch"] if traf else None)}),
+        "roofline": roofline_entry(kname, bytes_per_step, roof_flops, kern_mean, peaks, peak_src, traf),
         "e2e": {"value": round(job_rate(bytes_per_step, K, world, e2e_ms), 2), "unit": "GB/s",
                 "us_per_step": round(1000 * e2e_ms / K, 2), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
