@@ -1,5 +1,6 @@
-"""The bench line's `roofline` object, on the CPU: the HBM form for the rank-space kernels and
-the tensor-pipe form for the keys-before-RoPE kernel, from fixed timings."""
+"""Host-side pieces of the bench line, on the CPU: the `roofline` object (the HBM form for
+the rank-space kernels, the tensor-pipe form for the keys-before-RoPE kernel) from fixed
+timings, and the clock record built from nvidia-smi samples."""
 import os
 import sys
 
@@ -35,3 +36,26 @@ def test_fallback_peaks():
     assert r["peak"] == bench.FALLBACK_HBM_GBS
     r = bench.roofline_entry("decode_tc_i4_rope", 1e9, 1e12, 1.0, {}, "fallback", None)
     assert r["peak"] == bench.FALLBACK_TFLOPS_SUSTAINED
+
+
+def test_clock_summary_filters_gpu_and_reports_reasons():
+    class FakeProc:
+        stdout = [
+            "GPU-aaa, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active\n",
+            "GPU-bbb, 300, 1965, 90.0, 0x0, Active, Not Active, Not Active, Not Active\n",
+            "GPU-aaa, 1890, 1965, 998.0, 0x4, Not Active, Not Active, Not Active, Active\n",
+            "GPU-aaa, 1950, 1965, 980.0, 0x0, Not Active, Not Active, Not Active, Not Active\n",
+            "malformed line\n",
+        ]
+    cs = bench.ClockSampler("GPU-aaa")
+    cs.proc = FakeProc()
+    cs._read()
+    s = cs.summary()
+    assert s["samples"] == 3                       # the other GPU's row and the malformed one are dropped
+    assert s["sm_mhz"] == 1950.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]        # another GPU's hw_slowdown is not ours
+
+
+def test_clock_summary_without_samples():
+    s = bench.ClockSampler("GPU-aaa").summary()
+    assert s["samples"] == 0 and s["reasons"] == ["unsampled"]
