@@ -24,9 +24,10 @@ Modules:
   iskv       step simulator for the windowed cache: append with fold, basis
              sync, decode.
   svd        truncated SVD bases and the Eckart-Young error.
+  incsvd     block-incremental SVD update of the basis, with the sync rotation.
 
 Every function is pinned by a `-m "not gpu"` test against closed forms,
 invariants, special cases or brute force (tests/test_oracle_pins.py).
 """
 
-from . import attention, iskv, quant, svd  # noqa: F401
+from . import attention, incsvd, iskv, quant, svd  # noqa: F401
