@@ -7,10 +7,12 @@ lr_attn_decode over the full context (query projection, split-sequence latent
 attention, split merge and output projection).  The context is held fixed by truncating the appended
 token after each step (host bookkeeping only).
 
-Default workload: one Qwen2.5-VL-7B-shaped layer, batch 16, 28 query heads over
-4 KV heads, head_dim 128, 4096 tokens of bf16 rank-256 latents (the latency
-setup of TraceKV, "Perspective" section of the ai4snews digest: batch 16,
-context 4K-32K).  Inputs are seeded synthetic data resident in HBM; L2 is
+By default every workload is measured and printed as its own JSON line, in the order
+qwen4k, qwen16k, hybrid32k, qwen32k, qwen32k_postrope; the last line is the headline,
+batch 16 at 32K context with int4 latents (the latency setup of TraceKV, "Perspective"
+section of the ai4snews digest: Qwen2.5-VL-7B, batch 16, context 4K-32K), keys stored
+after RoPE so that the scores run in rank space.  Inputs are seeded synthetic data
+resident in HBM; L2 is
 flushed before every timed step, outside the timed events (256 MiB written, then
 read back, so the step neither finds its data in L2 nor pays the write-back of
 dirty flush lines).
@@ -25,6 +27,7 @@ sample of the same workload and prints the same JSON line with impl=reference.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -59,6 +62,11 @@ WORKLOADS = {
                                   "after RoPE (scores in rank space)",
                              batch=16, n_q_heads=28, n_kv_heads=4, head_dim=128, rank=256, length=32768,
                              quant_bits=4, layers=28, rope=False),
+    "qwen4k_perhead": dict(desc="Qwen2.5-VL-7B layer with one latent per KV head: B=16, Hq=28, Hkv=4, d=128, "
+                                "T=4096, 4 groups of r=64 bf16 latents (the same 512 B of latents per token "
+                                "as qwen4k)",
+                           batch=16, n_q_heads=28, n_kv_heads=4, head_dim=128, rank=64, length=4096,
+                           quant_bits=0, layers=1, groups=4),
     "hybrid32k": dict(desc="Qwen3-8B-shaped iS-KV hybrid layer: B=8, Hq=32, Hkv=8, d=128, 32640 history "
                            "tokens of r=256 bf16 latents + an exact bf16 window of 128; every step appends "
                            "one token (the oldest window token is folded into history) and decodes; "
@@ -68,12 +76,19 @@ WORKLOADS = {
 }
 
 
+# The default run measures every workload, one JSON line each; the last line is the
+# headline: batch 16 at 32K with the keys stored after RoPE (scores in rank space), the
+# HBM-bound case of the 32K configuration.
+ORDER = ["qwen4k", "qwen4k_perhead", "qwen16k", "hybrid32k", "qwen32k", "qwen32k_postrope"]
+
+
 def layer_ranks(workload: str, seed: int = 0):
-    """(r_k, r_v) of every layer of a workload."""
+    """(r_k, r_v) of every layer of a workload (the stored rank: groups x the group rank)."""
     import synth
     W = WORKLOADS[workload]
     if W["layers"] == 1:
-        return [(W["rank"], W["rank"])]
+        g = W.get("groups", 1)
+        return [(g * W["rank"], g * W["rank"])]
     return synth.qwen32k_ranks(seed, W["layers"])
 
 
@@ -82,6 +97,38 @@ def latent_bytes_per_token(rank: int, quant_bits: int) -> int:
         g = (rank + 31) // 32
         return g * 16 + g * 4
     return rank * 2
+
+
+def r_full_A(B_full, r):
+    """A = r B^T of a block-diagonal basis (the generator's A for every group)."""
+    return r * B_full.T
+
+
+def workload_bytes(workload: str) -> int:
+    """Latent (and exact-window) bytes one step reads, summed over the workload's layers."""
+    W = WORKLOADS[workload]
+    Bsz, T, qb = W["batch"], W["length"], W["quant_bits"]
+    D = W["n_kv_heads"] * W["head_dim"]
+    win = W.get("window", 0)
+    total = 0
+    for rk, rv in layer_ranks(workload):
+        per_tok = latent_bytes_per_token(rk, qb) + latent_bytes_per_token(rv, qb)
+        total += Bsz * ((T - win) * per_tok + win * 2 * D * 2) if win else Bsz * T * per_tok
+    return total
+
+
+def static_config(workload: str, world: int) -> dict:
+    """The `config` object of a bench line: the workload alone, identical for both arms."""
+    W = WORKLOADS[workload]
+    ranks = layer_ranks(workload)
+    return {"workload": W["desc"], "name": workload, "batch": W["batch"], "context": W["length"],
+            "layers": len(ranks),
+            "ranks": sorted({r for rr in ranks for r in rr}) if len(ranks) > 1 else ranks[0][0],
+            "quant_bits": W["quant_bits"], "latent_bytes_per_step": workload_bytes(workload),
+            "step": "lr_decode_step (= lr_kv_append + lr_attn_decode) per layer",
+            "l2": "flushed before every timed step outside the events (256 MiB written, then read back "
+                  "so L2 holds clean unrelated lines)",
+            "parallelism": f"dp{world} (independent sequences per GPU)"}
 
 
 # ----------------------------------------------------------------------------
@@ -217,11 +264,7 @@ def traffic_record(kernel: str):
 
 
 def run_ours(args):
-    import numpy as np
     import torch
-
-    import rank_kv_cache_lr_b200 as lr
-    import synth
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -230,7 +273,27 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    W = WORKLOADS[args.workload]
+    for wl in workloads_of(args):
+        run_workload(args, wl)
+        torch.cuda.empty_cache()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def workloads_of(args):
+    return ORDER if args.workload == "all" else [args.workload]
+
+
+def run_workload(args, workload):
+    import numpy as np
+    import torch
+
+    import rank_kv_cache_lr_b200 as lr
+    import synth
+
+    rank, world, local = dist_env()
+    W = WORKLOADS[workload]
     Bsz, Hq, Hkv, d, T = W["batch"], W["n_q_heads"], W["n_kv_heads"], W["head_dim"], W["length"]
     qb = W["quant_bits"]
     D = Hkv * d
@@ -246,7 +309,7 @@ def run_ours(args):
     layers = []
     host_p = None
     win = W.get("window", 0)
-    for li, (rk, rv) in enumerate(layer_ranks(args.workload)):
+    for li, (rk, rv) in enumerate(layer_ranks(workload)):
         hist = T - 1
         if win:
             hist = T - win
@@ -254,13 +317,22 @@ def run_ours(args):
                                   n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d)
             host_p = p
         elif W["layers"] == 1:
-            p = synth.make_qwen(args.workload, seed=rank, batch=Bsz, length=hist, rank=rk, quant_bits=qb)
+            p = synth.make_qwen(workload, seed=rank, batch=Bsz, length=hist, rank=rk, quant_bits=qb)
             host_p = p
+            if W.get("groups"):   # per-group bases; the latents keep the layout [g r] per token
+                g = W["groups"]
+                Ak_c, Bk_c, Av_c, Bv_c, Bk_f, Bv_f = synth.grouped_bases(workload, rank, g, W["rank"], D)
+                p = dataclasses.replace(p, A_k=Ak_c, B_k=Bk_c, A_v=Av_c, B_v=Bv_c)
+                host_p = dataclasses.replace(p, A_k=synth.bf16_bits(r_full_A(Bk_f, W["rank"])),
+                                             B_k=synth.bf16_bits(Bk_f),
+                                             A_v=synth.bf16_bits(r_full_A(Bv_f, W["rank"])),
+                                             B_v=synth.bf16_bits(Bv_f))
         else:
-            p = synth.make_qwen(args.workload, seed=rank, batch=Bsz, length=0, rank=rk, rank_v=rv,
+            p = synth.make_qwen(workload, seed=rank, batch=Bsz, length=0, rank=rk, rank_v=rv,
                                 quant_bits=qb, layer=li)
-        desc = lr.make_desc(Bsz, Hq, Hkv, d, rk, rv, T + (8 if win else 0), window=win, quant_bits=qb,
-                            dtype=lr.LR_BF16, rope_in_kernel=1 if W.get("rope") else 0)
+        g = W.get("groups", 1)
+        desc = lr.make_desc(Bsz, Hq, Hkv, d, rk // g, rv // g, T + (8 if win else 0), window=win, quant_bits=qb,
+                            dtype=lr.LR_BF16, rope_in_kernel=1 if W.get("rope") else 0, latent_groups=g)
         cache = lr.lr_cache_create(desc, to_dev(p.A_k), to_dev(p.B_k), to_dev(p.A_v), to_dev(p.B_v))
         chunk = 1024 if W["layers"] == 1 else 2048
         gen = torch.Generator(device=dev)
@@ -278,8 +350,9 @@ def run_ours(args):
             lr.lr_kv_append_latent(cache, zk, zv)
         for t in range(p.win_len if win else 0):   # the exact window, through lr_kv_append
             lr.lr_kv_append(cache, to_dev(np.ascontiguousarray(p.win_k[:, t])), to_dev(np.ascontiguousarray(p.win_v[:, t])))
-        kx, vx = synth.hybrid_token(args.workload, rank * 1000 + li, T - 1, Bsz, D,
-                                    synth.bf16_to_f64(p.B_k), synth.bf16_to_f64(p.B_v), noise=1e-2 if win else 0.0)
+        hp = host_p if (host_p is not None and W.get("groups")) else p
+        kx, vx = synth.hybrid_token(workload, rank * 1000 + li, T - 1, Bsz, D,
+                                    synth.bf16_to_f64(hp.B_k), synth.bf16_to_f64(hp.B_v), noise=1e-2 if win else 0.0)
         L = dict(cache=cache, rk=rk, rv=rv, k_h=synth.bf16_bits(kx), v_h=synth.bf16_bits(vx), q_h=p.q,
                  len0=lr.lr_cache_get_len(cache)[0])
         L["k"], L["v"], L["q"] = to_dev(L["k_h"]), to_dev(L["v_h"]), to_dev(L["q_h"])
@@ -459,27 +532,23 @@ def run_ours(args):
     rope = bool(W.get("rope"))
     if rope:
         kname += "_rope"
-    traf = traffic_record(f"{kname}:{args.workload}")
+    traf = traffic_record(f"{kname}:{workload}")
     # Keys stored before RoPE are rebuilt per tile on the tensor cores: the contraction
     # (2 r_k D per token for the keys, 2 r_v Hq for the value mix) bounds that kernel, not
     # HBM; fp16 operands run at the bf16 rate, and the kernel runs inside a long step
     # (sustained peak).
     roof_flops = sum(Bsz * T * (2 * L["rk"] * D + 2 * L["rv"] * Hq) for L in layers) if rope else 0.0
+    assert bytes_per_step == workload_bytes(workload)
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
         "us_per_step": round(1000 * total_ms / K, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int4+bf16" if qb else "bf16",
         "data": "synthetic (seeded; one seed per rank)",
-        "config": {"workload": W["desc"], "batch": Bsz, "context": T, "layers": len(layers),
-                   "ranks": sorted({rr for L in layers for rr in (L["rk"], L["rv"])}) if len(layers) > 1 else layers[0]["rk"],
-                   "quant_bits": qb, "latent_bytes_per_step": bytes_per_step,
-                   "step": "lr_decode_step (= lr_kv_append + lr_attn_decode) per layer",
-                   "l2": "flushed before every timed step outside the events (256 MiB written, then read back so L2 holds clean unrelated lines)",
-                   "parallelism": f"dp{world} (independent sequences per GPU)",
-                   "decode_path": "tcgen05" if plan.path == lr.LR_PATH_TC else "simt",
-                   "splits": plan.n_splits, "cuda_graph": bool(args.graph),
-                   "launches_per_step": launches_per_step},
+        "config": static_config(workload, world),
+        "run": {"decode_path": "tcgen05" if plan.path == lr.LR_PATH_TC else "simt",
+                "splits": plan.n_splits, "cuda_graph": bool(args.graph),
+                "launches_per_step": launches_per_step},
         "roofline": roofline_entry(kname, bytes_per_step, roof_flops, kern_mean, peaks, peak_src, traf),
         "e2e": {"value": round(job_rate(bytes_per_step, K, world, e2e_ms), 2), "unit": "GB/s",
                 "us_per_step": round(1000 * e2e_ms / K, 2), "h2d_bytes_per_step": h2d,
@@ -488,9 +557,9 @@ def run_ours(args):
         "clocks": sampler.summary(),
     }
     if sync is not None:
-        res["config"]["basis_sync"] = sync
+        res["run"]["basis_sync"] = sync
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(args.workload, host_p, args.cpu_seconds)
+        res["cpu_baseline"] = cpu_baseline(workload, host_p, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(res), flush=True)
     run = run_kev = None
@@ -498,9 +567,6 @@ def run_ours(args):
         del g_plain, g_kev
     for L in layers:
         lr.lr_cache_destroy(L["cache"])
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
 
 
 # ----------------------------------------------------------------------------
@@ -531,16 +597,17 @@ def oracle_step_sample(p, rows, seconds):
             if p.quant_bits == 4:
                 c, s, z = quant.quantize_int4(p.z_k[b]); zk = quant.dequantize_int4(c, s, z, p.rank_k)
                 c, s, z = quant.quantize_int4(p.z_v[b]); zv = quant.dequantize_int4(c, s, z, p.rank_v)
-            else:
+            elif p.dtype == "bf16":
                 zk = quant.round_to_bf16(p.z_k[b]); zv = quant.round_to_bf16(p.z_v[b])
-            qv = (p.q[b:b + 1].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-            Bk = (p.B_k.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-            Bv = (p.B_v.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            else:
+                zk = np.asarray(p.z_k[b], np.float64); zv = np.asarray(p.z_v[b], np.float64)
+            qv = p.to_f64(p.q[b:b + 1])
+            Bk, Bv = p.to_f64(p.B_k), p.to_f64(p.B_v)
             wk = wv = None
             if p.win_k is not None and p.win_len:
-                wk = (p.win_k[b:b + 1].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-                wv = (p.win_v[b:b + 1].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-            attention.decode(qv, zk[None], zv[None], Bk, Bv, p.n_kv_heads, None, None, wk, wv)
+                wk, wv = p.to_f64(p.win_k[b:b + 1]), p.to_f64(p.win_v[b:b + 1])
+            attention.decode(qv, zk[None], zv[None], Bk, Bv, p.n_kv_heads, None,
+                             p.rope_theta if p.rope else None, wk, wv)
             done += 1
             nbytes += p.hist_len * 2 * per_tok + (p.win_len * 2 * p.kv_dim * 2 if wk is not None else 0)
         el = time.time() - t0
@@ -557,27 +624,56 @@ def host_problem(workload, seed, batch):
                                  rank=W["rank"], n_q_heads=W["n_q_heads"], n_kv_heads=W["n_kv_heads"],
                                  head_dim=W["head_dim"])
     if W["layers"] == 1:
-        return synth.make_qwen(workload, seed=seed, batch=batch, length=W["length"] - 1, rank=W["rank"],
-                               quant_bits=W["quant_bits"])
+        g = W.get("groups", 1)
+        p = synth.make_qwen(workload, seed=seed, batch=batch, length=W["length"] - 1, rank=g * W["rank"],
+                            quant_bits=W["quant_bits"])
+        if g > 1:   # the block-diagonal bases of the per-group ones
+            D = W["n_kv_heads"] * W["head_dim"]
+            *_, Bk_f, Bv_f = synth.grouped_bases(workload, seed, g, W["rank"], D)
+            p = dataclasses.replace(p, A_k=synth.bf16_bits(r_full_A(Bk_f, W["rank"])), B_k=synth.bf16_bits(Bk_f),
+                                    A_v=synth.bf16_bits(r_full_A(Bv_f, W["rank"])), B_v=synth.bf16_bits(Bv_f))
+        return p
     return synth.make_qwen32k_layer(0, seed=seed, batch=batch, length=W["length"] - 1, rope=bool(W.get("rope")))
+
+
+def single_core_timings(seconds):
+    """The oracle on one host core for the two small configurations (the tiny fp32 case
+    and the 4K bf16 layer): one batch row, all heads; bounded to `seconds` in total."""
+    import synth
+    from threadpoolctl import threadpool_limits
+    out = {}
+    with threadpool_limits(limits=1):
+        for name, p in (("tiny", synth.make_tiny()), ("qwen4k", host_problem("qwen4k", 0, 1))):
+            bps, s_per_row, n = oracle_step_sample(p, [0], seconds / 2)
+            out[name] = {"GBps": round(bps / 1e9, 5), "ms_per_row": round(1e3 * s_per_row, 3), "rows": n,
+                         "cores": 1}
+    return out
 
 
 def cpu_baseline(workload, p, seconds):
     if p is None:
         p = host_problem(workload, 0, 1)
     bps, s_per_row, n = oracle_step_sample(p, [0], seconds)
-    return {"value": round(bps / 1e9, 4), "unit": "GB/s", "cores": _blas_threads(), "kind": "oracle",
-            "us_per_step_equiv": round(1e6 * s_per_row * p.batch, 1),
-            "sample": f"{n} oracle decodes of batch row 0 (all {p.n_q_heads} heads, T={p.hist_len}) of the "
-                      f"{workload} step (first layer), fp64 NumPy; GB/s of latents processed"}
+    res = {"value": round(bps / 1e9, 4), "unit": "GB/s", "cores": _blas_threads(), "kind": "oracle",
+           "us_per_step_equiv": round(1e6 * s_per_row * p.batch, 1),
+           "sample": f"{n} oracle decodes of batch row 0 (all {p.n_q_heads} heads, T={p.hist_len}) of the "
+                     f"{workload} step (first layer), fp64 NumPy; GB/s of latents processed"}
+    if workload == "qwen4k":
+        res["single_core"] = single_core_timings(min(seconds, 8.0))
+    return res
 
 
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    W = WORKLOADS[args.workload]
-    p = host_problem(args.workload, 0, 1)
+    for wl in workloads_of(args):
+        run_reference_workload(args, wl, world)
+
+
+def run_reference_workload(args, workload, world):
+    W = WORKLOADS[workload]
+    p = host_problem(workload, 0, 1)
     for _ in range(args.warmup):
         oracle_step_sample(p, [0], 0.0)
     t0 = time.time()
@@ -594,7 +690,7 @@ def run_reference(args):
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(us_step / 1000, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": W["desc"], "batch": W["batch"], "context": W["length"], "rank": W["rank"]},
+           "config": static_config(workload, world),
            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                             "sample": "each step: repeated oracle decodes of batch row 0 (all heads) for a "
                                       f"bounded {per:.1f} s; value = latent bytes processed per second"},
@@ -609,9 +705,10 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="qwen4k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="all", choices=["all"] + sorted(WORKLOADS),
+                    help="one workload, or all of them (one line each, the 32K rank-space headline last)")
     ap.add_argument("--load-seconds", type=float, default=1.5)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch the step's calls directly instead of replaying a CUDA graph")

@@ -79,21 +79,30 @@ typedef struct lr_cache_desc {
                              each reconstructed key at its absolute position        */
   double rope_theta;      /* RoPE base, e.g. 1e6                                   */
   float softmax_scale;    /* 0 -> 1/sqrt(head_dim)                                 */
-  int32_t reserved[5];    /* must be zero                                          */
+  int32_t latent_groups;  /* 0 or 1: one latent group spans all KV heads; g > 1 (dividing
+                             n_kv_heads): g groups of n_kv_heads / g heads, each with its own
+                             latents of rank_k / rank_v and its own bases, so g = n_kv_heads
+                             is one latent per KV head.  g * rank_k and g * rank_v <= 512.  */
+  int32_t reserved[4];    /* must be zero                                          */
 } lr_cache_desc;
 
 typedef struct lr_cache lr_cache;   /* opaque */
 
 /* Device pointers and strides of the cache's storage, for inspection.
- * Int4 latents are stored in blocks of 128 tokens, group-major inside a block, so that
- * one group of one block (128 tokens) is a contiguous 2 KB run of codes and a 512-byte
- * run of params:
- *   codes  [B][int4_blocks][groups][128][4] uint32: element e of group g of token t
- *          of sequence b is in word ((b*int4_blocks + t/128)*groups + g)*512
- *          + (t%128)*4 + e/8, bits 4(e%8)..+3;
- *   params [B][int4_blocks][groups][128] uint32: ((b*int4_blocks + t/128)*groups + g)*128
- *          + t%128, a pair of fp16 {scale (low half), zero (high half)};
- * with int4_blocks = ceil(capacity / 128).
+ * Int4 latents are stored in blocks of 128 tokens (int4_blocks = ceil(capacity / 128) per
+ * sequence; block k of sequence b is block n = b*int4_blocks + k), each side's block being
+ * one contiguous run of groups*2 KB of codes and one of groups*512 B of params.
+ * Keys, token-major inside a block (group-major):
+ *   codes_k  [B][int4_blocks][groups][128][4] uint32: element e of group g of token t is
+ *            in word (n*groups + g)*512 + (t%128)*4 + e/8, bits 4(e%8)..+3;
+ *   params_k [B][int4_blocks][groups][128] uint32: word (n*groups + g)*128 + t%128, a pair
+ *            of fp16 {scale (low half), zero (high half)}.
+ * Values, rank-major inside a block:
+ *   codes_v  [B][int4_blocks][groups*32][16] uint32: rank i (= 32g + e) of token t (u = t%128)
+ *            is in word (n*groups*32 + i)*16 + 4*((u/32) ^ ((i/2)%4)) + (u%32)/8,
+ *            bits 4m..+3 with m = 4*(u%2) + (u/2)%4 (tokens 2k and 2k+1 in nibbles k, k+4);
+ *   params_v [B][int4_blocks][groups][256] fp16 (same bytes as params_k): half
+ *            (n*groups + g)*256 + u is the scale, half (n*groups + g)*256 + 128 + u the zero.
  * Unquantised latents: z [B][capacity][rank] in dtype.
  * Window ring: [B][window+1][D] in dtype; token t lives in slot t % (window+1). */
 typedef struct lr_cache_view {
@@ -120,6 +129,11 @@ typedef struct lr_plan {
 /* ---- lifetime -------------------------------------------------------------
  * lr_cache_create — allocate a cache for `desc` and copy the bases.
  *   A_k [D][r_k], B_k [r_k][D], A_v [D][r_v], B_v [r_v][D], device, dtype.
+ *   With g = latent_groups > 1 the bases are given per group: A_k [g][D/g][r_k],
+ *   B_k [g][r_k][D/g] (group i covers KV heads i*Hkv/g .. and ranks i*r_k ..); the cache
+ *   stores them as one block-diagonal basis of rank g*r_k (A [D][g r_k], B [g r_k][D], zero
+ *   outside the blocks), and every latent row holds the g groups' latents one after another
+ *   ([g*r_k]).  Latent fills (lr_kv_append_latent) and the view then use the rank g*r_k.
  *   A_* may be NULL when the caller only fills latents (lr_kv_append then
  *   returns LR_ERR_INVALID_ARG).  Returns LR_ERR_INVALID_ARG / LR_ERR_UNSUPPORTED
  *   for bad descriptions before touching the device, LR_ERR_OOM if allocation
@@ -161,6 +175,37 @@ lr_status lr_kv_append_latent(lr_cache* cache, const float* z_k, const float* z_
  *   LR_ERR_INVALID_ARG. */
 lr_status lr_attn_decode(lr_cache* cache, const void* q, void* out, float* lse, void* stream);
 
+/* lr_attn_decode_varlen — lr_attn_decode for a batch whose rows hold different numbers of
+ *   tokens (a serving batch of sequences at different lengths): row b attends to its first
+ *   row_len[b] history tokens only.  row_len: [B] int32, device, each in
+ *   1..history length (values outside are clamped to that range); the cache itself is
+ *   filled up to its common length, and the tokens of a row beyond its row_len are not
+ *   read.  The sequence splits are planned for the longest row; splits past a row's end
+ *   carry zero weight.  Caches with an exact window return LR_ERR_UNSUPPORTED. */
+lr_status lr_attn_decode_varlen(lr_cache* cache, const void* q, void* out, float* lse,
+                                const int32_t* row_len, void* stream);
+
+/* ---- context sharding (SURVEY-style split of the context over GPUs; the pages'
+ *      workload, TraceKV digest Perspective: batch 16 at up to 32K tokens) -----------
+ * Several caches (typically one per GPU) hold consecutive slices of the same sequences'
+ * context, with the same bases and query.  Each computes a partial result over its slice;
+ * the partials are exchanged (e.g. an all-gather over NCCL) and merged by the log-sum-exp
+ * rule, then projected once through B_v.  Caches with a window or with keys before RoPE
+ * return LR_ERR_UNSUPPORTED (their tokens' positions are not the slice's own).
+ * lr_attn_decode_partial — the decode of this cache's tokens up to, not including, the
+ *   output projection: part_o [B][Hq][r_v] fp32 = sum_t 2^(s_t - m) z_v,t, part_ml
+ *   [B][Hq][2] fp32 = (m, l = sum_t 2^(s_t - m)) with s_t = log2(e) * softmax_scale *
+ *   q . k_t (the rank-space form of one slice's softmax).  len >= 1 (else
+ *   LR_ERR_INVALID_ARG).
+ * lr_merge_partials — out [B][Hq][d] (dtype) and lse [B][Hq] (natural log, or NULL) of the
+ *   whole context from n partials: part_o [n][B][Hq][r_v], part_ml [n][B][Hq][2] fp32,
+ *   device, as lr_attn_decode_partial writes them (shard order does not matter).  Uses this
+ *   cache's B_v; n <= the cache's partial capacity (LR_ERR_CAPACITY). */
+lr_status lr_attn_decode_partial(lr_cache* cache, const void* q, float* part_o, float* part_ml,
+                                 void* stream);
+lr_status lr_merge_partials(lr_cache* cache, int32_t n, const float* part_o, const float* part_ml,
+                            void* out, float* lse, void* stream);
+
 /* lr_decode_step — one whole decode step: lr_kv_append(k, v) then lr_attn_decode(q,
  *   out, lse), with identical arguments, results and errors, but with the projection
  *   of the new token and the projection of the query run in one launch. */
@@ -170,7 +215,8 @@ lr_status lr_decode_step(lr_cache* cache, const void* k, const void* v, const vo
 /* ---- basis sync (iS-KV abstract: historical coordinates synchronised with the
  *      updated basis) ---------------------------------------------------------
  * lr_basis_sync — Z_hist <- Z_hist R for the history latents of every sequence,
- *   then install new bases.  R_k [r_k][r_k], R_v [r_v][r_v] fp32 device, or NULL
+ *   then install new bases.  R_k [r_k][r_k], R_v [r_v][r_v] fp32 device (per group,
+ *   [g][r_k][r_k] and the bases in the per-group form of lr_cache_create), or NULL
  *   to leave that side's latents unchanged; B_k_new, B_v_new, A_k_new, A_v_new
  *   (dtype) or NULL to keep the current basis.  For orthogonal R, passing
  *   B' = R^T B keeps every reconstructed key/value unchanged.  The window is
@@ -193,7 +239,9 @@ lr_status lr_basis_sync(lr_cache* cache, const float* R_k, const float* R_v,
  *     (otherwise LR_ERR_UNSUPPORTED); len: tokens to attend, 1..capacity.
  *   z_k [B][capacity][r_k], z_v [B][capacity][r_v]: latents in the cache layout;
  *   B_k [r_k][D], B_v [r_v][D], q [B][Hq][d], out [B][Hq][d]: dtype, device;
- *   lse [B][Hq] fp32 or NULL.
+ *   B_k and B_v 16-byte aligned (else LR_ERR_INVALID_ARG, before any launch);
+ *   lse [B][Hq] fp32 or NULL.  The first kernel starts only after the work before the
+ *   call on `stream` has completed, so that work may write the bases and the query.
  *   Uses fewer sequence splits when needed to fit the array, and returns
  *   LR_ERR_CAPACITY when even one split's working set exceeds it
  *   (4 * B * Hq * (r_k + r_v + 2) bytes > LR_NOALLOC_SCRATCH_BYTES).
@@ -235,14 +283,42 @@ lr_status lr_device_error(lr_cache* cache, int32_t* code);
  * timed; both NULL to stop.  The events must stay valid while set. */
 lr_status lr_cache_set_kernel_events(lr_cache* cache, void* ev_start, void* ev_stop);
 /* Timeline trace of the tensor-core decode kernel: when buf (device, capacity_words
- * 64-bit words >= LR_TRACE_SLOTS * batch * max splits) is set, every CTA of each
- * following decode writes %globaltimer stamps (ns) to
+ * 64-bit words >= LR_TRACE_SLOTS * batch * max splits + LR_TRACE_SPAN_WORDS) is set, every
+ * CTA of each following decode writes %globaltimer stamps (ns) to
  * buf[((b * n_splits) + split) * LR_TRACE_SLOTS + slot]: 0 start, 1 set-up done,
  * 2 query latents in shared memory, 3+4i key tile i consumed, 4+4i its scores read,
  * 5+4i its probabilities written, 6+4i its value mix issued (tiles i < 16), 71 end.
+ * The last LR_TRACE_SPAN_WORDS words hold kernel spans, as pairs (earliest CTA start,
+ * latest CTA end) for: 0 the append / query projection kernel, 1 the split-sequence decode,
+ * 2 the exact window, 3 the split merge; the caller sets each pair to (~0, 0) before a call
+ * whose spans it wants.  (The max split count is the larger of 64 and two CTAs per SM
+ * spread over the batch, capped at one split per 16 tokens of capacity.)
  * NULL stops tracing.  LR_ERR_CAPACITY if buf is too small. */
 #define LR_TRACE_SLOTS 72
+#define LR_TRACE_SPAN_WORDS 8
 lr_status lr_cache_set_trace(lr_cache* cache, uint64_t* buf, int64_t capacity_words);
+/* ---- failure testing (no counterpart on the pages) ----------------------------
+ * lr_cache_set_wait_limit — limit, in nanoseconds, of every bounded wait inside this
+ *   cache's tensor-core kernels (decode and basis sync); 0 restores the default (2 s).
+ *   A wait that gives up makes its kernel record LR_ERR_TIMEOUT in the device error word
+ *   (lr_device_error), finish its own copies and MMAs, free its tensor memory and return;
+ *   that call's outputs are then undefined, the cache's contents are untouched.  For
+ *   tests of that path: a limit of a few nanoseconds makes the first wait that is not
+ *   already satisfied give up.  LR_ERR_INVALID_ARG for ns < 0. */
+lr_status lr_cache_set_wait_limit(lr_cache* cache, int64_t ns);
+
+/* lr_debug_inject_fault — make the library's next-but-`after` device allocation
+ *   (kind LR_FAULT_ALLOC) or kernel launch (LR_FAULT_LAUNCH) fail without allocating or
+ *   launching: `after` operations of that kind still succeed, the one after them fails,
+ *   then the fault disarms itself; after = -1 disarms.  Process-wide.  The failing call
+ *   returns LR_ERR_OOM (allocation) or LR_ERR_CUDA (launch); lr_cache_create frees what
+ *   it had allocated.  A failed launch inside lr_decode_step can leave the appended token
+ *   in the cache (its length then counts it).  LR_ERR_INVALID_ARG for another kind or
+ *   after < -1. */
+#define LR_FAULT_ALLOC 0
+#define LR_FAULT_LAUNCH 1
+lr_status lr_debug_inject_fault(int32_t kind, int64_t after);
+
 /* sizeof(lr_cache_desc), sizeof(lr_cache_view), sizeof(lr_plan) as compiled (binding checks). */
 void lr_abi_struct_sizes(int32_t* desc_size, int32_t* view_size, int32_t* plan_size);
 /* Human-readable name of a status. */

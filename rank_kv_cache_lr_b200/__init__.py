@@ -10,7 +10,8 @@ Functions keep the C names: lr_cache_create, lr_cache_destroy, lr_kv_append, lr_
 lr_kv_append_latent, lr_attn_decode, lr_basis_sync, lr_cache_get_len,
 lr_cache_truncate, lr_cache_view_get, lr_cache_set_path, lr_cache_plan,
 lr_plan_decode, lr_cache_set_kernel_events, lr_cache_set_trace, lr_device_error, lr_abi_struct_sizes,
-lr_status_string, lr_launch_count, lr_attn_decode_noalloc.
+lr_status_string, lr_launch_count, lr_attn_decode_noalloc, lr_cache_set_wait_limit,
+lr_debug_inject_fault, lr_attn_decode_varlen, lr_attn_decode_partial, lr_merge_partials.
 """
 from __future__ import annotations
 
@@ -34,7 +35,7 @@ class lr_cache_desc(ctypes.Structure):
                 ("quant_bits", ctypes.c_int32), ("quant_group", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("rope_in_kernel", ctypes.c_int32),
                 ("rope_theta", ctypes.c_double), ("softmax_scale", ctypes.c_float),
-                ("reserved", ctypes.c_int32 * 5)]
+                ("latent_groups", ctypes.c_int32), ("reserved", ctypes.c_int32 * 4)]
 
 
 class lr_cache_view(ctypes.Structure):
@@ -84,6 +85,11 @@ def _load() -> ctypes.CDLL:
         "lr_device_error": [vp, ctypes.POINTER(i32)],
         "lr_cache_set_kernel_events": [vp, vp, vp],
         "lr_cache_set_trace": [vp, vp, ctypes.c_int64],
+        "lr_cache_set_wait_limit": [vp, ctypes.c_int64],
+        "lr_attn_decode_varlen": [vp, vp, vp, vp, vp, vp],
+        "lr_attn_decode_partial": [vp, vp, vp, vp, vp],
+        "lr_merge_partials": [vp, i32, vp, vp, vp, vp, vp],
+        "lr_debug_inject_fault": [i32, ctypes.c_int64],
         "lr_attn_decode_noalloc": [ctypes.POINTER(lr_cache_desc), i32, vp, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
@@ -121,10 +127,11 @@ def lr_launch_count() -> int:
 def make_desc(batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int, rank_k: int,
               rank_v: int, capacity: int, window: int = 0, quant_bits: int = 0,
               dtype: int = LR_BF16, rope_in_kernel: int = 0, rope_theta: float = 1e6,
-              softmax_scale: float = 0.0, quant_group: int = 32) -> lr_cache_desc:
+              softmax_scale: float = 0.0, quant_group: int = 32,
+              latent_groups: int = 0) -> lr_cache_desc:
     return lr_cache_desc(batch, n_q_heads, n_kv_heads, head_dim, rank_k, rank_v, capacity,
                          window, quant_bits, quant_group, dtype, rope_in_kernel, rope_theta,
-                         softmax_scale)
+                         softmax_scale, latent_groups)
 
 
 # ---------------------------------------------------------------------------
@@ -178,15 +185,26 @@ class Cache:
             self.handle = None
 
 
+def _groups(desc) -> int:
+    return desc.latent_groups if desc.latent_groups > 1 else 1
+
+
+def _basis_shapes(desc, r):
+    """(A shape, B shape) of the bases a caller passes: [D][r], [r][D], or per group."""
+    D, g = desc.n_kv_heads * desc.head_dim, _groups(desc)
+    if g == 1:
+        return (D, r), (r, D)
+    return (g, D // g, r), (g, r, D // g)
+
+
 def lr_cache_create(desc: lr_cache_desc, A_k, B_k, A_v, B_v, stream=None) -> Cache:
     dt = _torch_dtype(desc.dtype)
-    D = desc.n_kv_heads * desc.head_dim
+    ak, bk = _basis_shapes(desc, desc.rank_k)
+    av, bv = _basis_shapes(desc, desc.rank_v)
     out = ctypes.c_void_p()
     _check(_lib.lr_cache_create(ctypes.byref(desc),
-                                _ptr(A_k, dt, (D, desc.rank_k), "A_k", True),
-                                _ptr(B_k, dt, (desc.rank_k, D), "B_k"),
-                                _ptr(A_v, dt, (D, desc.rank_v), "A_v", True),
-                                _ptr(B_v, dt, (desc.rank_v, D), "B_v"),
+                                _ptr(A_k, dt, ak, "A_k", True), _ptr(B_k, dt, bk, "B_k"),
+                                _ptr(A_v, dt, av, "A_v", True), _ptr(B_v, dt, bv, "B_v"),
                                 _stream(stream), ctypes.byref(out)), "lr_cache_create")
     return Cache(out, desc)
 
@@ -206,10 +224,11 @@ def lr_kv_append(cache: Cache, k, v, stream=None) -> None:
 def lr_kv_append_latent(cache: Cache, z_k, z_v, stream=None) -> None:
     import torch
     d = cache.desc
+    g = _groups(d)
     n = z_k.shape[1] if z_k.dim() == 3 else -1
     _check(_lib.lr_kv_append_latent(cache.handle,
-                                    _ptr(z_k, torch.float32, (d.batch, n, d.rank_k), "z_k"),
-                                    _ptr(z_v, torch.float32, (d.batch, n, d.rank_v), "z_v"),
+                                    _ptr(z_k, torch.float32, (d.batch, n, g * d.rank_k), "z_k"),
+                                    _ptr(z_v, torch.float32, (d.batch, n, g * d.rank_v), "z_v"),
                                     n, _stream(stream)), "lr_kv_append_latent")
 
 
@@ -220,6 +239,42 @@ def lr_attn_decode(cache: Cache, q, out, lse=None, stream=None) -> None:
     _check(_lib.lr_attn_decode(cache.handle, _ptr(q, dt, shp, "q"), _ptr(out, dt, shp, "out"),
                                _ptr(lse, torch.float32, (d.batch, d.n_q_heads), "lse", True),
                                _stream(stream)), "lr_attn_decode")
+
+
+def lr_attn_decode_varlen(cache: Cache, q, out, row_len, lse=None, stream=None) -> None:
+    """row_len: int32 CUDA tensor [batch], tokens of history each row attends to."""
+    import torch
+    d, dt = cache.desc, _torch_dtype(cache.desc.dtype)
+    shp = (d.batch, d.n_q_heads, d.head_dim)
+    _check(_lib.lr_attn_decode_varlen(cache.handle, _ptr(q, dt, shp, "q"), _ptr(out, dt, shp, "out"),
+                                      _ptr(lse, torch.float32, (d.batch, d.n_q_heads), "lse", True),
+                                      _ptr(row_len, torch.int32, (d.batch,), "row_len"),
+                                      _stream(stream)), "lr_attn_decode_varlen")
+
+
+def lr_attn_decode_partial(cache: Cache, q, part_o, part_ml, stream=None) -> None:
+    """part_o: fp32 CUDA tensor [batch][Hq][r_v], part_ml: [batch][Hq][2]."""
+    import torch
+    d, dt = cache.desc, _torch_dtype(cache.desc.dtype)
+    rv = _groups(d) * d.rank_v
+    _check(_lib.lr_attn_decode_partial(cache.handle, _ptr(q, dt, (d.batch, d.n_q_heads, d.head_dim), "q"),
+                                       _ptr(part_o, torch.float32, (d.batch, d.n_q_heads, rv), "part_o"),
+                                       _ptr(part_ml, torch.float32, (d.batch, d.n_q_heads, 2), "part_ml"),
+                                       _stream(stream)), "lr_attn_decode_partial")
+
+
+def lr_merge_partials(cache: Cache, part_o, part_ml, out, lse=None, stream=None) -> None:
+    """part_o: fp32 [n][batch][Hq][r_v], part_ml: [n][batch][Hq][2] (n shards' partials)."""
+    import torch
+    d, dt = cache.desc, _torch_dtype(cache.desc.dtype)
+    rv = _groups(d) * d.rank_v
+    n = part_o.shape[0]
+    _check(_lib.lr_merge_partials(cache.handle, int(n),
+                                  _ptr(part_o, torch.float32, (n, d.batch, d.n_q_heads, rv), "part_o"),
+                                  _ptr(part_ml, torch.float32, (n, d.batch, d.n_q_heads, 2), "part_ml"),
+                                  _ptr(out, dt, (d.batch, d.n_q_heads, d.head_dim), "out"),
+                                  _ptr(lse, torch.float32, (d.batch, d.n_q_heads), "lse", True),
+                                  _stream(stream)), "lr_merge_partials")
 
 
 def lr_decode_step(cache: Cache, k, v, q, out, lse=None, stream=None) -> None:
@@ -237,30 +292,39 @@ def lr_basis_sync(cache: Cache, R_k=None, R_v=None, B_k_new=None, B_v_new=None, 
                   A_v_new=None, stream=None) -> None:
     import torch
     d, dt = cache.desc, _torch_dtype(cache.desc.dtype)
-    D = cache.D
+    g = _groups(d)
+    ak, bk = _basis_shapes(d, d.rank_k)
+    av, bv = _basis_shapes(d, d.rank_v)
+    rk = (d.rank_k, d.rank_k) if g == 1 else (g, d.rank_k, d.rank_k)
+    rv = (d.rank_v, d.rank_v) if g == 1 else (g, d.rank_v, d.rank_v)
     _check(_lib.lr_basis_sync(cache.handle,
-                              _ptr(R_k, torch.float32, (d.rank_k, d.rank_k), "R_k", True),
-                              _ptr(R_v, torch.float32, (d.rank_v, d.rank_v), "R_v", True),
-                              _ptr(B_k_new, dt, (d.rank_k, D), "B_k_new", True),
-                              _ptr(B_v_new, dt, (d.rank_v, D), "B_v_new", True),
-                              _ptr(A_k_new, dt, (D, d.rank_k), "A_k_new", True),
-                              _ptr(A_v_new, dt, (D, d.rank_v), "A_v_new", True),
+                              _ptr(R_k, torch.float32, rk, "R_k", True),
+                              _ptr(R_v, torch.float32, rv, "R_v", True),
+                              _ptr(B_k_new, dt, bk, "B_k_new", True),
+                              _ptr(B_v_new, dt, bv, "B_v_new", True),
+                              _ptr(A_k_new, dt, ak, "A_k_new", True),
+                              _ptr(A_v_new, dt, av, "A_v_new", True),
                               _stream(stream)), "lr_basis_sync")
 
 
 LR_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 
-def lr_attn_decode_noalloc(desc: lr_cache_desc, length: int, z_k: int, z_v: int, B_k: int, B_v: int,
+def _addr(x) -> ctypes.c_void_p:
+    """Device address of a CUDA tensor, or an address given as an int."""
+    return ctypes.c_void_p(x.data_ptr() if hasattr(x, "data_ptr") else int(x))
+
+
+def lr_attn_decode_noalloc(desc: lr_cache_desc, length: int, z_k, z_v, B_k, B_v,
                            q, out, lse=None, stream=None) -> None:
     """Decode without device allocation (working memory in the library's static device
-    array).  z_k, z_v, B_k, B_v: device addresses (ints) of caller-owned buffers in the
-    cache layout; q, out (and lse) are CUDA tensors."""
+    array).  z_k, z_v, B_k, B_v: caller-owned device buffers in the cache layout (CUDA
+    tensors or device addresses as ints); q, out (and lse) are CUDA tensors."""
     import torch
     dt = _torch_dtype(desc.dtype)
     shp = (desc.batch, desc.n_q_heads, desc.head_dim)
-    _check(_lib.lr_attn_decode_noalloc(ctypes.byref(desc), int(length), ctypes.c_void_p(z_k),
-                                       ctypes.c_void_p(z_v), ctypes.c_void_p(B_k), ctypes.c_void_p(B_v),
+    _check(_lib.lr_attn_decode_noalloc(ctypes.byref(desc), int(length), _addr(z_k),
+                                       _addr(z_v), _addr(B_k), _addr(B_v),
                                        _ptr(q, dt, shp, "q"), _ptr(out, dt, shp, "out"),
                                        _ptr(lse, torch.float32, (desc.batch, desc.n_q_heads), "lse", True),
                                        _stream(stream)), "lr_attn_decode_noalloc")
@@ -324,6 +388,17 @@ def lr_abi_struct_sizes():
     a, b, c = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
     _lib.lr_abi_struct_sizes(ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
     return a.value, b.value, c.value
+
+
+LR_FAULT_ALLOC, LR_FAULT_LAUNCH = 0, 1
+
+
+def lr_cache_set_wait_limit(cache: Cache, ns: int = 0) -> None:
+    _check(_lib.lr_cache_set_wait_limit(cache.handle, int(ns)), "lr_cache_set_wait_limit")
+
+
+def lr_debug_inject_fault(kind: int, after: int) -> None:
+    _check(_lib.lr_debug_inject_fault(int(kind), int(after)), "lr_debug_inject_fault")
 
 
 def lr_device_error(cache: Cache) -> int:

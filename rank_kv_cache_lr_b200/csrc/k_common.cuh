@@ -21,6 +21,13 @@ __device__ __forceinline__ void store_elem(void* p, long long idx, float v, int 
 // product is exact in fp32, so this is the fp32 rounding of the exact value).
 __device__ __forceinline__ float latent_f(const LatentRef& L, int kind, int dtype,
                                           long long row, int i) {
+  if (kind == LK_INT4 && L.rank_major) {
+    const uint32_t w = L.codes[i4v_code_index(row, L.G, i)];
+    const float code = (float)((w >> (4 * i4v_nibble(row))) & 15u);
+    const unsigned short* h = reinterpret_cast<const unsigned short*>(L.params);
+    const long long si = i4v_scale_index(row, L.G, i >> 5);
+    return fmaf(code, __half2float(__ushort_as_half(h[si])), __half2float(__ushort_as_half(h[si + 128])));
+  }
   if (kind == LK_INT4) {
     const uint32_t w = L.codes[i4_code_index(row, L.G, i >> 5, (i >> 3) & 3)];
     const float code = (float)((w >> (4 * (i & 7))) & 15u);
@@ -37,9 +44,11 @@ __device__ __forceinline__ float latent_f(const LatentRef& L, int kind, int dtyp
 // none): zero = fp16(min), scale = fp16((max - min) / 15) in fp32, code =
 // clamp(rint((x - zero) / scale), 0, 15) in IEEE fp32, 0 if scale == 0; a zero
 // point of -0 is stored as +0.  Writes 4 packed words and the {scale, zero} word.
-__device__ __forceinline__ void quant_group_warp(float x, bool valid, uint32_t* words,
-                                                 uint32_t* param) {
-  const int lane = threadIdx.x & 31;
+struct QuantOut {
+  uint32_t code;           // this lane's code (0 for padding lanes)
+  unsigned short sh, zh;   // fp16 bits of the group's scale and zero
+};
+__device__ __forceinline__ QuantOut quant_group_codes(float x, bool valid) {
   float mn = valid ? x : INFINITY;
   float mx = valid ? x : -INFINITY;
 #pragma unroll
@@ -57,22 +66,57 @@ __device__ __forceinline__ void quant_group_warp(float x, bool valid, uint32_t* 
     t = fminf(fmaxf(t, 0.0f), 15.0f);
     code = (uint32_t)t;
   }
-  uint32_t v = code << (4 * (lane & 7));
+  QuantOut q;
+  q.code = code;
+  q.sh = __half_as_ushort(sh);
+  q.zh = __half_as_ushort(zh);
+  return q;
+}
+
+// Token-major packing of one quantised group (keys): 4 words and the {scale, zero} word.
+__device__ __forceinline__ void quant_group_warp(float x, bool valid, uint32_t* words,
+                                                 uint32_t* param) {
+  const int lane = threadIdx.x & 31;
+  const QuantOut q = quant_group_codes(x, valid);
+  uint32_t v = q.code << (4 * (lane & 7));
   v |= __shfl_xor_sync(0xffffffffu, v, 1);
   v |= __shfl_xor_sync(0xffffffffu, v, 2);
   v |= __shfl_xor_sync(0xffffffffu, v, 4);
   if ((lane & 7) == 0) words[lane >> 3] = v;
-  if (lane == 0) *param = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
+  if (lane == 0) *param = (uint32_t)q.sh | ((uint32_t)q.zh << 16);
 }
 
-// Store one warp's 32-coordinate chunk `ch` of a latent row (lane = coordinate).
+// Rank-major store of one quantised group of one value token (lane = rank 32 g + lane):
+// each lane replaces its token's nibble in its rank's word.  The words are shared with
+// seven other tokens, which other warps of the same launch may be writing, so the nibble
+// is cleared and set with atomics (the two touch only this token's bits).
+__device__ __forceinline__ void quant_group_warp_v(float x, bool valid, uint32_t* codes, uint32_t* params,
+                                                   int G, int g, long long row) {
+  const int lane = threadIdx.x & 31;
+  const QuantOut q = quant_group_codes(x, valid);
+  const int sh = 4 * i4v_nibble(row);
+  uint32_t* w = codes + i4v_code_index(row, G, g * 32 + lane);
+  atomicAnd(w, ~(15u << sh));
+  if (q.code) atomicOr(w, q.code << sh);
+  if (lane == 0) {
+    unsigned short* h = reinterpret_cast<unsigned short*>(params);
+    const long long si = i4v_scale_index(row, G, g);
+    h[si] = q.sh;
+    h[si + 128] = q.zh;
+  }
+}
+
+// Store one warp's 32-coordinate chunk `ch` of a latent row (lane = coordinate); int4
+// values (rank_major) take the rank-major block layout.
 __device__ __forceinline__ void store_latent_chunk(float z, int ch, int r, int kind, int dtype,
                                                    void* Z, uint32_t* codes, uint32_t* params,
-                                                   int G, long long row) {
+                                                   int G, long long row, bool rank_major = false) {
   const int lane = threadIdx.x & 31;
   const int i = ch * 32 + lane;
   const bool valid = i < r;
-  if (kind == LK_INT4) {
+  if (kind == LK_INT4 && rank_major) {
+    quant_group_warp_v(z, valid, codes, params, G, ch, row);
+  } else if (kind == LK_INT4) {
     quant_group_warp(z, valid, codes + i4_code_index(row, G, ch, 0), params + i4_param_index(row, G, ch));
   } else if (valid) {
     store_elem(Z, row * r + i, z, dtype);

@@ -52,6 +52,9 @@ constexpr int kMaxSlots = 8;
 constexpr int kSmemPair = 115712;          // per block when two blocks share an SM (228 KB - 2 x 1 KB)
 
 struct TcParams {
+  unsigned long long wait_ns;   // bounded-wait limit (0: the default)
+  const int32_t* row_len;       // per-row history lengths (device), or null
+  unsigned long long* span;     // timeline span, or null
   int r_k, r_v, ck, cv, kb_k, tmem_cols;
   int Hq, hist_len, stable_len, split_tokens, n_splits, nslot;
   uint32_t q_bytes;
@@ -77,6 +80,7 @@ struct Aux {
   uint64_t q_full, p_full, p_empty, o_final;
   uint32_t tmem_base;
   int abort_flag;
+  unsigned long long wait_ns;   // this launch's wait limit
   float red[4][32];
   float m_s[32];
   float alpha_s[32];
@@ -104,7 +108,7 @@ __device__ __forceinline__ void tmem_ld_sum(uint32_t taddr, float (&v)[32]) {
 }
 
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
-  return tc::wait_b(bar, parity, &aux->abort_flag, err);
+  return tc::wait_b(bar, parity, &aux->abort_flag, err, aux->wait_ns);
 }
 
 __device__ __forceinline__ void trace_stamp(const TcParams& p, int slot) { tc::trace_stamp(p.trace, slot); }
@@ -120,6 +124,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (threadIdx.x == 0) atomicExch(p.err, (int)LR_ERR_UNSUPPORTED);
     return;
   }
+  span_begin(p.span);
   Aux* aux = reinterpret_cast<Aux*>(smem_raw);
   uint8_t* q_s = smem_raw + kAuxBytes;
   uint8_t* ring = q_s + p.q_bytes;
@@ -128,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, b = blockIdx.y;
   const int tok_begin = split * p.split_tokens;
-  const int tok_end = min(p.hist_len, tok_begin + p.split_tokens);
+  const int tok_end = min(row_hist(p.row_len, b, p.hist_len), tok_begin + p.split_tokens);
   const int ntiles = tok_end > tok_begin ? (tok_end - tok_begin + kTile - 1) / kTile : 0;
   const int nunits = 2 * ntiles;
 
@@ -147,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::mbar_init(&aux->p_empty, 1);
     ptx::mbar_init(&aux->o_final, 1);
     aux->abort_flag = 0;
+    aux->wait_ns = tc::wait_limit(p.wait_ns);
     for (int j = 0; j < 32; ++j) aux->m_s[j] = -INFINITY;
     ptx::fence_mbar_init();
   }
@@ -212,11 +218,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int sb = 0; sb < p.kb_k; ++sb)
           ptx::tma_load_2d(q_s + sb * kQSubBytes, &tm_q, &aux->q_full, sb * 64, b * kQRows);
       }
-      if (!ok) {
-        drain_wait(&aux->q_full, 0);
-        for (int pos = max(0, issued - p.nslot); pos < issued; ++pos)
-          drain_wait(&aux->slot_full[pos % p.nslot], (pos / p.nslot) & 1);
-      }
+      // Every copy this thread issued has landed before the CTA can exit: after an abort
+      // (here or in another role, which may come after this loop) the consumers stop
+      // waiting for them.  In a normal run these are the phases the consumers already
+      // waited for, so the waits return at once.
+      drain_wait(&aux->q_full, 0);
+      for (int pos = max(0, issued - p.nslot); pos < issued; ++pos)
+        drain_wait(&aux->slot_full[pos % p.nslot], (pos / p.nslot) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -284,7 +292,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       ptx::mma_commit(&aux->o_final);
-      if (!ok) drain_wait(&aux->o_final, 0);
+      // the MMAs have completed before TMEM is freed, even if the epilogue aborted
+      drain_wait(&aux->o_final, 0);
     }
     __syncwarp();
   } else if (ntiles > 0) {
@@ -410,6 +419,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (threadIdx.x == 64) trace_stamp(p, kTraceSlots - 1);
     }
+  } else if (warp == 2) {
+    // a split that starts beyond its row's length: zero weight in the merge
+    const size_t base_out = ((size_t)b * p.n_splits + split) * p.Hq;
+    if (lane < p.Hq) {
+      p.part_ml[(base_out + lane) * 2] = -INFINITY;
+      p.part_ml[(base_out + lane) * 2 + 1] = 0.f;
+    }
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -417,6 +433,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, p.tmem_cols);
   }
+  span_end(p.span);
 }
 
 // ---------------------------------------------------------------------------
@@ -480,7 +497,7 @@ cudaError_t tc_prepare(lr_cache* c, cudaStream_t s) {
     c->tc_state = st;
   }
   if (!c->qt16) {
-    cudaError_t e = cudaMalloc(&c->qt16, (size_t)d.batch * kQRows * d.rank_k * 2);
+    cudaError_t e = lr_dev_malloc(&c->qt16, (size_t)d.batch * kQRows * d.rank_k * 2);
     if (e != cudaSuccess) return e;
     e = cudaMemset(c->qt16, 0, (size_t)d.batch * kQRows * d.rank_k * 2);
     if (e != cudaSuccess) return e;
@@ -522,6 +539,9 @@ cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, 
   const TcState* st = reinterpret_cast<const TcState*>(c->tc_state);
   if (!st) return cudaErrorNotSupported;
   TcParams p;
+  p.wait_ns = c->wait_ns;
+  p.row_len = c->row_len;
+  p.span = span_of(c->spans, SPAN_DECODE);
   p.r_k = d.rank_k;
   p.r_v = d.rank_v;
   p.ck = (d.rank_k + 127) / 128;

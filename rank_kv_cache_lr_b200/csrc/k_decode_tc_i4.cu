@@ -5,51 +5,64 @@
 //   S[t, j]  = z^_k,t . q~_j            GEMM1: M = 128 tokens, N = 32 heads, K = r_k
 //   p[t, j]  = exp2(S[t, j] - m_j)      online softmax, lazy running max
 //   O~[e, j] += sum_t z^_v,t[e] p[t, j]  GEMM2: M = 128 ranks per chunk, N = 32, K = 128 tokens
-// where z^ = code * scale + zero is expanded in shared memory to fp16 (one rounding of
-// the exact fused product-sum) and q~, p enter the MMAs as fp16 (11 significant bits,
-// so neither needs the hi/lo split of the bf16 kernel).
+// where z^ = code * scale + zero is expanded to fp16 (one rounding of the exact fused
+// product-sum) and q~, p enter the MMAs as fp16 (11 significant bits, so neither needs the
+// hi/lo split of the bf16 kernel).
 //
-// Data flow.  The cache stores int4 latents in 128-token blocks, group-major inside a
-// block, so the codes and the {scale, zero} words of one side (K or V) of one tile are
-// two contiguous runs (G x 2 KB and G x 512 B).  The producer (warp 0) moves each with
-// one plain bulk copy into a ring of raw slots (per-SM copy throughput grows with the
-// copy size; 2-10 KB copies from one stream fall well short of HBM bandwidth).  Eight
-// dequantisation warps (thread = token row x half chunk) expand each 128-rank chunk
-// (4 groups) of a raw slot into a 32 KB operand slot
-// (128 tokens x 128 ranks, fp16, the 128-byte-swizzled K-major layout that GEMM1 reads
-// as A and GEMM2 reads MN-major); lanes walk consecutive tokens, so their shared-memory
-// reads and swizzled writes are free of bank conflicts.  Warp 1 owns TMEM and issues
-// the MMAs from one thread.  Four softmax warps (thread = token row = TMEM lane) turn
-// scores into probabilities and finish with the epilogue (thread = rank row).
+// Operands in tensor memory.  An M = 128 MMA with N = 32 that reads its A operand (128 x 16
+// fp16 = 4 KB) from shared memory is bound by the shared-memory bandwidth (128 B per
+// clock): the expanded latents would be written to and read back from shared memory once
+// each, 256 KB per 128-token tile at r = 256.  Here the dequantisation warps write the
+// expanded latents straight into tensor memory with tcgen05.st, and both GEMMs take their
+// A operand from there (A in TMEM: lane = row, column c = K elements 2c, 2c + 1).  Shared
+// memory carries only the packed codes (bulk copies), q~ and P.
+//   GEMM1 A = z^_k tile: lane = token, K = ranks.  A dequantisation thread owns one token
+//     row and expands its code words (keys are stored token-major).
+//   GEMM2 A = z^_v chunk transposed: lane = rank, K = tokens.  Values are stored
+//     rank-major (see lr_internal.cuh), so a thread owns one rank row and expands eight
+//     tokens per word, each pair with its own fp16 {scale, zero}.
+// A tcgen05.st reaches only the 32 lanes of the writing warp's sub-partition, so the eight
+// dequantisation warps are two per sub-partition (warp % 4 = lane quarter), splitting the
+// columns of a chunk between them.
+//
+// Data flow.  The producer (warp 0) moves the codes and the {scale, zero} words of one side
+// (K or V) of one 128-token tile with two plain bulk copies into a ring of raw slots.  The
+// dequantisation warps expand each 128-rank chunk of a raw slot into a 64-column operand
+// slot of a TMEM ring.  Warp 1 issues the MMAs from one thread.  Four softmax warps (thread
+// = token row = TMEM lane) turn scores into probabilities and finish with the epilogue
+// (thread = rank row).
 //
 // Pipeline.  Operand slots, raw slots and MMAs all follow the order
 //   K(0), K(1), V(0), K(2), V(1), ..., K(n-1), V(n-2), V(n-1)
 // so GEMM1 of tile s+1 runs while the softmax of tile s is still working: the scores
 // and the probabilities are double-buffered (S in two TMEM column blocks, P in two
-// shared-memory buffers).  When the running max of a head grows by more than 2^8 the
-// softmax first waits for the value mix of the previous tile and rescales O~ in TMEM.
+// shared-memory buffers).  The K steps of GEMM1 alternate between two accumulators, so
+// consecutive MMAs do not wait on each other's accumulation; the softmax adds the two.
+// When the running max of a head grows by more than 2^8 the softmax first waits for the
+// value mix of the previous tile and rescales O~ in TMEM.
 //
-// Nibble order.  A code word holds elements m = 0..7 of an 8-rank run at bits 4m.  Two
+// Nibble order.  A key code word holds elements m = 0..7 of an 8-rank run at bits 4m.  Two
 // masks and one shift give the four fp16 pairs (m0,m4) (m1,m5) (m2,m6) (m3,m7) through
 // the exponent-bias trick (0x6400 | n is 1024 + n; 0x5400 | 16n is 64 + n), so each run
-// sits in shared memory in the order 0,4,1,5,2,6,3,7.  The query latents are stored in
-// the same order (a score is an order-free sum over ranks), and the epilogue maps the
-// rows of O~ back to rank order.
+// sits in TMEM in the order 0,4,1,5,2,6,3,7.  The query latents are stored in the same
+// order (a score is an order-free sum over ranks).  A value word holds eight tokens, with
+// tokens 2m and 2m + 1 in nibbles m and m + 4, so the same four pairs come out in token
+// order, matching the probabilities.
 //
 // Keys stored before the rotary embedding (kRope).  The score needs the rotated key,
 // which has no rank-space form, so each tile's keys are rebuilt on the tensor cores:
 //   K^_h[t, :] = z^_k,t B_k,h          GEMM0: M = 128 tokens, N = d = 128, K = r_k
-// then rotated (rotate-half RoPE at the token's absolute position, cos / sin from the
-// cache's fp64-derived table) and dotted with the raw query rows on CUDA cores by the
-// softmax warps (thread = token row).  K^ for all four KV heads would need all of TMEM,
-// so a CTA covers a pair of KV heads (grid x), query slots 16 h + jj for query head jj
-// of pair head h; both CTAs of a pair dequantise the same tiles.  B_k enters as an fp16
-// copy, [D rows][ranks] with each 8-rank run in the dequantised order, streamed per
-// 64-rank sub-block (both heads' rows, one N = 256 MMA per 16 ranks) by TMA from a spare
-// warp (warp 2) through a ring of up to four slots.  The rotation factors of a row are
-// fetched one 16-pair chunk ahead (the next tile's first chunk during the last one), so
-// their L2 latency stays off the chain rebuild -> rotate -> rebuild.  The value mix and
-// the epilogue are those of the rank-space kernel with 32 slots.
+// (A = the same token-row operand as GEMM1) then rotated (rotate-half RoPE at the token's
+// absolute position, cos / sin from the cache's fp64-derived table) and dotted with the
+// raw query rows on CUDA cores by the softmax warps (thread = token row).  K^ for all four
+// KV heads would need all of TMEM, so a CTA covers a pair of KV heads (grid x), query slots
+// 16 h + jj for query head jj of pair head h; both CTAs of a pair dequantise the same
+// tiles.  B_k enters as an fp16 copy, [D rows][ranks] with each 8-rank run in the
+// dequantised order, streamed per 64-rank sub-block (both heads' rows, one N = 256 MMA per
+// 16 ranks) by TMA from a spare warp (warp 2) through a ring of up to four slots.  The
+// rotation factors of a row are fetched one 16-pair chunk ahead (the next tile's first
+// chunk during the last one), so their L2 latency stays off the chain rebuild -> rotate
+// -> rebuild.  The value mix and the epilogue are those of the rank-space kernel.
 //
 // Every wait is bounded: on timeout the kernel records LR_ERR_TIMEOUT, drains its own
 // copies and MMAs, frees TMEM and returns.
@@ -66,53 +79,59 @@ using tc::kTile;
 using tc::kTraceSlots;
 using tc::warp_reduce_scatter32;
 
-// 16 warps in four warpgroups: [producer, MMA, 2 idle] [4 softmax] [dequantisation x 8].
-// A warp runs on sub-partition (warp % 4).  A single thread issuing N = 32 MMAs slows
-// about fivefold when three ALU-bound warps share its sub-partition; with the producer,
-// MMA and two idle warps in the first warpgroup, the MMA warp (1) shares sub-partition 1
-// with one softmax warp and two dequantisation warps.  Measured against leaving those two
-// dequantisation warps idle, the extra dequantisation throughput wins by ~3 %.  Launched
-// at 128 registers per thread; the warpgroups then rebalance the block's 64K registers
-// with setmaxnreg (the softmax keeps 32 scores and 32 running sums per row).
+// 16 warps in four warpgroups: [producer, MMA, B_k producer / idle, idle] [4 softmax]
+// [dequantisation x 8].  A warp runs on sub-partition (warp % 4), and a tcgen05.ld / st
+// reaches TMEM lanes 32 (warp % 4) .. + 31.  Launched at 128 registers per thread; the
+// warpgroups then rebalance the block's 64K registers with setmaxnreg (the softmax keeps
+// 32 scores and 32 running sums per row).
 constexpr int kThreads = 512;
 constexpr int kDqWarp0 = 8;                // first warp of the dequantisation warpgroups
-constexpr int kDqThreads = 256;            // eight working dequantisation warps
 constexpr int kDqWarps = 8;                // arrivals per operand slot / raw slot (one per warp)
 constexpr int kSmWarps = 4;                // softmax warps (one arrival each)
 constexpr int kLaunchRegs = 128;
-constexpr int kRegsCtl = 56, kRegsSoftmax = 208, kRegsDq = 104;
-constexpr int kRegsSoftmaxRope = 216;      // keys before RoPE: rotation and query dots too
-static_assert(128 * kRegsCtl + 128 * kRegsSoftmax + 256 * kRegsDq <= kThreads * kLaunchRegs,
+// Per-warpgroup register budgets of each variant (the smallest that ptxas fits without
+// spilling; multiples of 8): control, softmax / epilogue, dequantisation.
+template <bool kRope> struct Regs;
+template <> struct Regs<false> { static constexpr int ctl = 56, softmax = 208, dq = 112; };
+template <> struct Regs<true> { static constexpr int ctl = 64, softmax = 240, dq = 104; };
+static_assert(128 * Regs<false>::ctl + 128 * Regs<false>::softmax + 256 * Regs<false>::dq <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-static_assert(128 * kRegsCtl + 128 * kRegsSoftmaxRope + 256 * kRegsDq <= kThreads * kLaunchRegs,
+static_assert(128 * Regs<true>::ctl + 128 * Regs<true>::softmax + 256 * Regs<true>::dq <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr int kSubBytes = 128 * 128;       // 128 tokens x 64 ranks x 2 B
-constexpr int kSlotBytes = 2 * kSubBytes;  // 128 tokens x 128 ranks
+constexpr int kSubBytes = 128 * 128;       // B_k ring: 128 rows x 64 ranks x 2 B per KV head
 constexpr int kQRows = 32;                 // query heads, padded
 constexpr int kQSubBytes = kQRows * 128;   // 32 rows x 64 ranks x 2 B
 constexpr int kPBytes = 128 * 32 * 2;      // 128 tokens x 32 heads x 2 B
 constexpr int kAuxBytes = 2048;
-constexpr int kSCol = 0;                   // TMEM: S of tile s in columns [32 (s % 2), +32)
-constexpr int kOCol = 64;                  // TMEM: O~ chunk c in columns [64 + 32c, +32)
-constexpr int kMaxSlots = 4;
-// keys before RoPE
+// TMEM columns, rank space: S of tile s in [64 (s % 2), +64) as two accumulators of 32
+// (K steps alternate), O~ chunk c in [128 + 32 c, +32), operand slots of 64 columns from 256
+constexpr int kSCol = 0;
+constexpr int kOCol = 128;
+constexpr int kACol = 256;
+// keys before RoPE: K^ of the pair in [0, 256), O~ in [256, 384), operand slots from 384
+constexpr int kOColR = 256;
+constexpr int kAColR = 384;
+constexpr int kASlotCols = 64;             // one operand slot: 128 lanes x 128 fp16 K elements
+constexpr int kMaxASlots = 4;
 constexpr int kRD = 128;                   // head dim of the rebuilt keys
 constexpr int kGHMax = 2;                  // KV heads per CTA (K^ of both fills 256 columns)
-constexpr int kMaxG = 32 / kGHMax;         // query slots per KV head
-constexpr int kOColR = 256;                // TMEM: O~ chunk c in columns [256 + 32c, +32)
-constexpr int kRopeG = 7;                  // query heads per KV head of the instantiated variant
+constexpr int kMaxG = 32 / kGHMax;         // query slots per KV head (the N of the score MMA)
+constexpr int kQbHeadBytes = 2 * kMaxG * 128;   // fp16 query rows of one KV head: 2 sub-blocks x 16 x 128 B
 constexpr int kNBMax = 4;                  // B_k ring slots (kv heads x 128 rows x 64 ranks, fp16)
-constexpr int kMaxRaw = 6;                 // raw slot: one side of one tile, codes (G x 2 KB)
+constexpr int kMaxRaw = 8;                 // raw slot: one side of one tile, codes (G x 2 KB)
                                            // then {scale, zero} words (G x 512 B)
 
 struct I4Params {
+  unsigned long long wait_ns;   // bounded-wait limit (0: the default)
+  const int32_t* row_len;       // per-row history lengths (device), or null
+  unsigned long long* span;     // timeline span, or null
   const uint32_t* codes_k;
   const uint32_t* codes_v;
   const uint32_t* params_k;
   const uint32_t* params_v;
   long long cap;
-  int r_k, r_v, G_k, G_v, ck, cv, kb_k, tmem_cols;
-  int Hq, hist_len, stable_len, split_tokens, n_splits, nslot, nraw;
+  int r_k, r_v, G_k, G_v, ck, cv, kb_k;
+  int Hq, hist_len, stable_len, split_tokens, n_splits, nas, nraw;
   uint32_t q_bytes, raw_bytes, raw_params;   // raw slot size; offset of its params
   float* part_o;
   float* part_ml;
@@ -120,9 +139,10 @@ struct I4Params {
   unsigned long long* trace;
   // keys before RoPE
   const float* qf;          // [B][Hq][d] scaled queries, fp32
-  const float2* rope_cs;    // [capacity][d / 2] (cos, sin)
+  const float2* rope_cs;    // (cos, sin), rope_cs_index layout
   int gh, gsz;              // KV heads per CTA, query heads per KV head
   uint32_t q_load_bytes;    // gh * gsz * d * 4
+  uint32_t qf_bytes;        // the fp32 rows' block, rounded up to 1024 (the fp16 operand follows)
   int nb;                   // B_k ring slots of gh * 16 KB
 };
 
@@ -130,8 +150,8 @@ struct I4Params {
 // K(0), K(1), V(0), K(2), ..., and phase k of a barrier is waited with parity k & 1.
 //   raw_full[nraw]    1 + tx   producer's two bulk copies -> dequantisation warps
 //   raw_empty[nraw]   8        dequantisation warps -> producer
-//   slot_full[nslot]  8        dequantisation warps (fenced stores) -> MMA issuer
-//   slot_empty[nslot] 1        MMA commit -> dequantisation warps
+//   slot_full[nas]    8        dequantisation warps (TMEM stores waited and fenced) -> MMA issuer
+//   slot_empty[nas]   1        MMA commit -> dequantisation warps
 //   q_full            1 + tx   producer (after the grid-dependency wait) -> MMA issuer, or
 //                              the softmax warps for keys before RoPE
 //   s_full[2]         1        MMA commit of GEMM1 -> softmax warps
@@ -139,21 +159,25 @@ struct I4Params {
 //   p_full[2]         4        softmax warps (fenced P stores) -> MMA issuer
 //   p_empty[2]        1        MMA commit of GEMM2 -> softmax warps (P reuse, O~ rescale)
 //   o_final           1        MMA commit after the last unit -> softmax warps (epilogue)
-//   keys before RoPE, in place of s_full / s_empty:
+//   keys before RoPE, in place of s_empty:
 //   k_full            1        MMA commit of GEMM0 -> softmax warps
-//   k_empty           4        softmax warps (K^ read) -> MMA issuer (next GEMM0)
+//   krot_full         4        softmax warps (rotated fp16 keys stored, waited, fenced) -> MMA issuer
+//   s_full[0]         1        MMA commit of the score MMAs -> softmax warps
+//   k_empty           4        softmax warps (scores read) -> MMA issuer (next GEMM0)
+//   qb_full           4        softmax warps (fp16 query operand stored, fenced) -> MMA issuer
 //   b_full[nb]        1 + tx   B_k producer (warp 2) -> MMA issuer
 //   b_empty[nb]       1        MMA commit -> B_k producer
 struct Aux {
-  uint64_t slot_full[kMaxSlots];
-  uint64_t slot_empty[kMaxSlots];
+  uint64_t slot_full[kMaxASlots];
+  uint64_t slot_empty[kMaxASlots];
   uint64_t raw_full[kMaxRaw];
   uint64_t raw_empty[kMaxRaw];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
   uint64_t q_full, o_final;
-  uint64_t k_full, k_empty, b_full[kNBMax], b_empty[kNBMax];
+  uint64_t k_full, k_empty, krot_full, qb_full, b_full[kNBMax], b_empty[kNBMax];
   uint32_t tmem_base;
   int abort_flag;
+  unsigned long long wait_ns;   // this launch's wait limit
   float red[4][32];
   float m_s[32];
   float alpha_s[32];
@@ -165,74 +189,85 @@ struct I4State {
   CUtensorMap bk;           // keys before RoPE: fp16 B_k [D][r_pad], rank runs permuted
   void* bk16 = nullptr;
   int r_pad = 0;
-  int nslot, nraw, nb = 0;
+  int nraw, nb = 0;
   uint32_t raw_bytes, raw_params, q_bytes;
   size_t smem;
 };
 
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
-  return tc::wait_b(bar, parity, &aux->abort_flag, err);
+  return tc::wait_b(bar, parity, &aux->abort_flag, err, aux->wait_ns);
+}
+
+// D[tmem] (+)= A[tmem] x B[smem desc], kind::f16: the A operand is read from tensor memory
+// (lane = row, 32-bit column c = K elements 2c, 2c + 1; K-major).
+__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// One fp16 pair of int4 codes: (lo, hi) = n - bias, then * scale + zero (one rounding).
+__device__ __forceinline__ uint32_t dq_pair(uint32_t biased, uint32_t bias, uint32_t s2, uint32_t z2) {
+  uint32_t r;
+  asm("{\n\t.reg .b32 t;\n\t"
+      "sub.rn.f16x2 t, %1, %2;\n\t"
+      "fma.rn.f16x2 %0, t, %3, %4;\n\t}"
+      : "=r"(r)
+      : "r"(biased), "r"(bias), "r"(s2), "r"(z2));
+  return r;
 }
 
 // Eight int4 codes of one word -> four fp16 pairs (m0,m4) (m1,m5) (m2,m6) (m3,m7) of
-// code * scale + zero; s2 = (scale, scale), z2 = (zero, zero).
-__device__ __forceinline__ uint4 dequant8(uint32_t w, uint32_t s2, uint32_t z2) {
+// code * scale + zero, pair k with its own scale and zero pairs (s2.k, z2.k).
+__device__ __forceinline__ uint4 dequant8(uint32_t w, const uint4& s2, const uint4& z2) {
   const uint32_t a = (w & 0x000F000Fu) | 0x64006400u;   // 1024 + n
   const uint32_t b = (w & 0x00F000F0u) | 0x54005400u;   // 64 + n
   const uint32_t w8 = w >> 8;
   const uint32_t c = (w8 & 0x000F000Fu) | 0x64006400u;
   const uint32_t d = (w8 & 0x00F000F0u) | 0x54005400u;
   uint4 r;
-  asm("{\n\t.reg .b32 t;\n\t"
-      "sub.rn.f16x2 t, %1, %2;\n\t"
-      "fma.rn.f16x2 %0, t, %3, %4;\n\t}"
-      : "=r"(r.x)
-      : "r"(a), "r"(0x64006400u), "r"(s2), "r"(z2));
-  asm("{\n\t.reg .b32 t;\n\t"
-      "sub.rn.f16x2 t, %1, %2;\n\t"
-      "fma.rn.f16x2 %0, t, %3, %4;\n\t}"
-      : "=r"(r.y)
-      : "r"(b), "r"(0x54005400u), "r"(s2), "r"(z2));
-  asm("{\n\t.reg .b32 t;\n\t"
-      "sub.rn.f16x2 t, %1, %2;\n\t"
-      "fma.rn.f16x2 %0, t, %3, %4;\n\t}"
-      : "=r"(r.z)
-      : "r"(c), "r"(0x64006400u), "r"(s2), "r"(z2));
-  asm("{\n\t.reg .b32 t;\n\t"
-      "sub.rn.f16x2 t, %1, %2;\n\t"
-      "fma.rn.f16x2 %0, t, %3, %4;\n\t}"
-      : "=r"(r.w)
-      : "r"(d), "r"(0x54005400u), "r"(s2), "r"(z2));
+  r.x = dq_pair(a, 0x64006400u, s2.x, z2.x);
+  r.y = dq_pair(b, 0x54005400u, s2.y, z2.y);
+  r.z = dq_pair(c, 0x64006400u, s2.z, z2.z);
+  r.w = dq_pair(d, 0x54005400u, s2.w, z2.w);
   return r;
 }
-
-__device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
+__device__ __forceinline__ void put4(uint32_t (&v)[32], int at, const uint4& r) {
+  v[at] = r.x;
+  v[at + 1] = r.y;
+  v[at + 2] = r.z;
+  v[at + 3] = r.w;
 }
 
-// Two fp32 lanes in one 64-bit register for the paired FMA: d = a * b + c per lane,
-// each rounded once (IEEE fma).
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
 }
-__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float((uint32_t)v); }
-__device__ __forceinline__ float hi2(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 
-// Shared memory: [aux 2 KB][q~ per 64-rank sub-block | fp32 query rows (kRope)]
-//                [B_k ring nb x gh x 16 KB (kRope)][operand ring nslot x 32 KB]
-//                [P double buffer 2 x 8 KB][raw ring nraw x raw_bytes]
-// kG: query heads per KV head (compile time for the keys-before-RoPE dots, so that the
-// kG accumulation chains interleave; 0 for the rank-space kernel).  A runtime count with a
-// guard inside the unrolled loop serialised the chains (13 us per tile instead of 7).
-template <bool kRope, int kG>
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Shared memory: [aux 2 KB][q~ per 64-rank sub-block | fp32 query rows, then the fp16
+//                query operand of the score MMAs (kRope)]
+//                [B_k ring nb x gh x 16 KB (kRope)][P double buffer 2 x 8 KB]
+//                [raw ring nraw x raw_bytes]
+template <bool kRope>
 __global__ void __launch_bounds__(kThreads, 1)
     k_decode_tc_i4(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_b,
                    const I4Params p) {
@@ -241,26 +276,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) atomicExch(p.err, (int)LR_ERR_UNSUPPORTED);
     return;
   }
+  span_begin(p.span);
   Aux* aux = reinterpret_cast<Aux*>(smem_raw);
   uint8_t* q_s = smem_raw + kAuxBytes;
   uint8_t* bring = q_s + p.q_bytes;
   const uint32_t b_slot_bytes = kRope ? (uint32_t)(p.gh * kSubBytes) : 0u;
-  uint8_t* ring = bring + (kRope ? p.nb * b_slot_bytes : 0);
-  uint8_t* p_s = ring + p.nslot * kSlotBytes;
+  uint8_t* p_s = bring + (kRope ? p.nb * b_slot_bytes : 0);
   uint8_t* raw = p_s + 2 * kPBytes;
   constexpr int kOC = kRope ? kOColR : kOCol;
+  constexpr int kAC = kRope ? kAColR : kACol;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = kRope ? (int)blockIdx.x : 0;
   const int split = kRope ? blockIdx.y : blockIdx.x, b = kRope ? blockIdx.z : blockIdx.y;
   const int tok_begin = split * p.split_tokens;
-  const int tok_end = min(p.hist_len, tok_begin + p.split_tokens);
+  const int tok_end = min(row_hist(p.row_len, b, p.hist_len), tok_begin + p.split_tokens);
   const int ntiles = tok_end > tok_begin ? (tok_end - tok_begin + kTile - 1) / kTile : 0;
   const int nunits = 2 * ntiles;
+  // query head of score / output slot j (-1: padding)
+  auto head_of = [&](int j) -> int {
+    if (!kRope) return j < p.Hq ? j : -1;
+    const int h = j / kMaxG, jj = j % kMaxG;
+    return (h < p.gh && jj < p.gsz) ? (pair * p.gh + h) * p.gsz + jj : -1;
+  };
 
   if (threadIdx.x == 0) {
     tc::trace_stamp(p.trace, 0);
-    for (int s = 0; s < p.nslot; ++s) {
+    for (int s = 0; s < p.nas; ++s) {
       ptx::mbar_init(&aux->slot_full[s], kDqWarps);
       ptx::mbar_init(&aux->slot_empty[s], 1);
     }
@@ -279,19 +321,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (kRope) {
       ptx::mbar_init(&aux->k_full, 1);
       ptx::mbar_init(&aux->k_empty, kSmWarps);
+      ptx::mbar_init(&aux->krot_full, kSmWarps);
+      ptx::mbar_init(&aux->qb_full, kSmWarps);
       for (int k = 0; k < p.nb; ++k) {
         ptx::mbar_init(&aux->b_full[k], 1);
         ptx::mbar_init(&aux->b_empty[k], 1);
       }
     }
     aux->abort_flag = 0;
+    aux->wait_ns = tc::wait_limit(p.wait_ns);
     for (int j = 0; j < 32; ++j) aux->m_s[j] = -INFINITY;
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0 && !kRope) ptx::prefetch_tmap(&tm_q);
   if (warp == 2 && lane == 0 && kRope) ptx::prefetch_tmap(&tm_b);
   if (warp == 1) {
-    ptx::tmem_alloc(&aux->tmem_base, p.tmem_cols);
+    ptx::tmem_alloc(&aux->tmem_base, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -308,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Roles by warpgroup; each sets its register budget first thing in its own branch,
   // so the compiler allocates that branch within the budget.
   if (warp < 4) {
-    ptx::setmaxnreg_dec<kRegsCtl>();
+    ptx::setmaxnreg_dec<Regs<kRope>::ctl>();
     if (warp == 0) {
       // ------------------------------------------------------------- bulk-copy producer
       if (lane == 0 && ntiles > 0) {
@@ -342,6 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int G = is_v ? p.G_v : p.G_k;
           const long long row0 = (long long)b * p.cap + t0;
           uint8_t* dst = raw + rs * p.raw_bytes;
+          // one block of one side: G x 2 KB of codes and G x 512 B of params, at the same
+          // offsets for the token-major keys and the rank-major values
           ptx::mbar_arrive_expect_tx(&aux->raw_full[rs], (uint32_t)G * 2560u);
           ptx::bulk_load(dst, (is_v ? p.codes_v : p.codes_k) + i4_code_index(row0, G, 0, 0), (uint32_t)G * 2048u,
                          &aux->raw_full[rs]);
@@ -353,11 +400,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           pdl_wait();
           load_query();
         }
-        if (!ok) {
-          drain_wait(&aux->q_full, 0);
-          for (int k = max(0, issued - p.nraw); k < issued; ++k)
-            drain_wait(&aux->raw_full[k % p.nraw], (k / p.nraw) & 1);
-        }
+        // Every copy this thread issued has landed before the CTA can exit: after an abort
+        // (here or in another role, which may come after this loop) the consumers stop
+        // waiting for them.  In a normal run these are the phases the consumers already
+        // waited for, so the waits return at once.
+        drain_wait(&aux->q_full, 0);
+        for (int k = max(0, issued - p.nraw); k < issued; ++k)
+          drain_wait(&aux->raw_full[k % p.nraw], (k / p.nraw) & 1);
       }
     } else if (kRope && warp == 2) {
       // ------------------------------------------------------------- B_k producer (kRope)
@@ -375,23 +424,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tma_load_2d(bring + slot * b_slot_bytes, &tm_b, &aux->b_full[slot], sb * 64, pair * p.gh * kRD);
           issued = k + 1;
         }
-        if (!ok)
-          for (int k = max(0, issued - p.nb); k < issued; ++k) drain_wait(&aux->b_full[k % p.nb], (k / p.nb) & 1);
+        (void)ok;   // drained whether or not the CTA aborted (see the producer above)
+        for (int k = max(0, issued - p.nb); k < issued; ++k) drain_wait(&aux->b_full[k % p.nb], (k / p.nb) & 1);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------- MMA issuer
       if (lane == 0 && ntiles > 0) {
-        const uint32_t id = ptx::idesc_f16(0, 0, 0, 128, 32);    // GEMM1: fp16, K-major x K-major
-        const uint32_t id2 = ptx::idesc_f16(0, 1, 1, 128, 32);   // GEMM2: fp16, MN-major x MN-major
+        const uint32_t id = ptx::idesc_f16(0, 0, 0, 128, 32);    // GEMM1: fp16, A (TMEM) x K-major B
+        const uint32_t id2 = ptx::idesc_f16(0, 0, 1, 128, 32);   // GEMM2: fp16, A (TMEM) x MN-major B
         // Descriptors are built once; a step along K or to another slot adds its byte
         // offset >> 4 to the start-address field (shared-memory addresses stay below
         // 256 KB, so the 14-bit field never carries).
-        const uint64_t kdesc0 = ptx::smem_desc(ptx::smem_u32(ring), 16, 1024, 2);       // Z_k, K-major SW128
         const uint64_t qdesc0 = ptx::smem_desc(ptx::smem_u32(q_s), 16, 1024, 2);        // q~, K-major SW128
-        const uint64_t vdesc0 = ptx::smem_desc(ptx::smem_u32(ring), kSubBytes, 1024, 2); // Z_v, MN-major SW128
         const uint64_t pdesc0 = ptx::smem_desc(ptx::smem_u32(p_s), 128, 2048, 0);       // P, MN-major
         const uint32_t idk = ptx::idesc_f16(0, 0, 0, 128, kRope ? p.gh * kRD : 128);   // GEMM0 (kRope)
         const uint64_t bdesc0 = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, 2);      // B_k, K-major SW128
+        const uint32_t idq = ptx::idesc_f16(0, 0, 0, 128, kMaxG);                        // scores (kRope)
+        const uint64_t qbdesc0 = ptx::smem_desc(ptx::smem_u32(q_s + p.qf_bytes), 16, 1024, 2);   // fp16 q, SW128
         bool ok = kRope ? true : wait_b(&aux->q_full, 0, aux, p.err);
         ptx::tc_fence_after();
         tc::trace_stamp(p.trace, 2);
@@ -405,20 +454,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (tile >= 1 && !(ok = wait_b(&aux->k_empty, (tile - 1) & 1, aux, p.err))) break;
             ptx::tc_fence_after();
             for (int c = 0; c < p.ck && ok; ++c, ++pos) {
-              const int slot = pos % p.nslot;
-              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+              const int slot = pos % p.nas;
+              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nas) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
-              const uint64_t a0 = kdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+              const uint32_t a0 = tmem + kAC + slot * kASlotCols;
               for (int sb = 0; sb < 2 && c * 128 + sb * 64 < p.r_k; ++sb, ++bpos) {
                 const int bs = bpos % p.nb;
                 if (!(ok = wait_b(&aux->b_full[bs], (bpos / p.nb) & 1, aux, p.err))) break;
                 ptx::tc_fence_after();
                 const uint64_t b0 = bdesc0 + (uint64_t)((bs * b_slot_bytes) >> 4);
-                // sub-block sb of the A slot (16 KB) against the B slot; 32 bytes per step
+                // K step kk of the sub-block: 8 TMEM columns on A, 32 bytes on B
                 const int nk = min(4, (p.r_k - c * 128 - sb * 64) >> 4);
                 for (int kk = 0; kk < nk; ++kk)
-                  ptx::mma_f16(tmem, a0 + (uint64_t)(sb * (kSubBytes >> 4) + kk * 2), b0 + (uint64_t)(kk * 2), idk,
-                               (c | sb | kk) ? 1u : 0u);
+                  mma_f16_ta(tmem, a0 + (uint32_t)(sb * 32 + kk * 8), b0 + (uint64_t)(kk * 2), idk,
+                             (c | sb | kk) ? 1u : 0u);
                 ptx::mma_commit(&aux->b_empty[bs]);
               }
               if (!ok) break;
@@ -427,24 +476,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             ptx::mma_commit(&aux->k_full);
             if (tile < 16) tc::trace_stamp(p.trace, 3 + 4 * tile);
+            // scores of the pair's query heads against the rotated fp16 keys the softmax warps
+            // wrote back over K^: per head, M = 128 tokens, N = 16 query slots, K = d
+            if (tile == 0 && !(ok = wait_b(&aux->qb_full, 0, aux, p.err))) break;
+            if (!(ok = wait_b(&aux->krot_full, tile & 1, aux, p.err))) break;
+            ptx::tc_fence_after();
+            for (int h = 0; h < p.gh; ++h)
+              for (int kk = 0; kk < kRD / 16; ++kk)
+                mma_f16_ta(tmem + h * kRD + kRD / 2, tmem + h * kRD + kk * 8,
+                           qbdesc0 + (uint64_t)((h * kQbHeadBytes + (kk >> 2) * (kQbHeadBytes / 2)) >> 4) +
+                               (uint64_t)((kk & 3) * 2),
+                           idq, kk ? 1u : 0u);
+            ptx::mma_commit(&aux->s_full[0]);
           } else if (!is_v) {
-            // GEMM1(tile): S[tile % 2] = Z_k q~^T
+            // GEMM1(tile): S[tile % 2] = Z_k q~^T, K steps alternating between the buffer's
+            // two accumulators
             const int sb2 = tile & 1;
             if (tile >= 2 && !(ok = wait_b(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
             ptx::tc_fence_after();
-            const uint32_t d_s = tmem + kSCol + 32 * sb2;
+            const uint32_t d_s = tmem + kSCol + 64 * sb2;
             for (int c = 0; c < p.ck && ok; ++c, ++pos) {
-              const int slot = pos % p.nslot;
-              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+              const int slot = pos % p.nas;
+              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nas) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
-              const uint64_t a0 = kdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+              const uint32_t a0 = tmem + kAC + slot * kASlotCols;
               const uint64_t b0 = qdesc0 + (uint64_t)((c * 2 * kQSubBytes) >> 4);
               const int nk = min(8, (p.r_k - c * 128) >> 4);     // 16-rank K steps in this chunk
-              // step kk: sub-block kk / 4 (16 KB on A, 4 KB on B), 32 bytes per step within it
+              // step kk: 8 TMEM columns on A; sub-block kk / 4 (4 KB), 32 bytes per step on B
               for (int kk = 0; kk < nk; ++kk) {
-                const uint32_t ao = (uint32_t)((kk >> 2) * (kSubBytes >> 4) + (kk & 3) * 2);
                 const uint32_t bo = (uint32_t)((kk >> 2) * (kQSubBytes >> 4) + (kk & 3) * 2);
-                ptx::mma_f16(d_s, a0 + ao, b0 + bo, id, (c | kk) ? 1u : 0u);
+                mma_f16_ta(d_s + 32 * (kk & 1), a0 + (uint32_t)(kk * 8), b0 + bo, id, (c | (kk >> 1)) ? 1u : 0u);
               }
               ptx::mma_commit(&aux->slot_empty[slot]);
             }
@@ -458,15 +519,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             const uint64_t b0 = pdesc0 + (uint64_t)((pb2 * kPBytes) >> 4);
             for (int c = 0; c < p.cv && ok; ++c, ++pos) {
-              const int slot = pos % p.nslot;
-              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+              const int slot = pos % p.nas;
+              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nas) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
-              const uint64_t a0 = vdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
+              const uint32_t a0 = tmem + kAC + slot * kASlotCols;
               const uint32_t d_o = tmem + kOC + c * 32;
-              // K step kt = 16 tokens: 2 KB on A (16 swizzled rows), 256 B on P
+              // K step kt = 16 tokens: 8 TMEM columns on A, 256 B on P
 #pragma unroll
               for (int kt = 0; kt < 8; ++kt)
-                ptx::mma_f16(d_o, a0 + (uint64_t)(kt * 128), b0 + (uint64_t)(kt * 16), id2, (tile | kt) ? 1u : 0u);
+                mma_f16_ta(d_o, a0 + (uint32_t)(kt * 8), b0 + (uint64_t)(kt * 16), id2, (tile | kt) ? 1u : 0u);
               ptx::mma_commit(&aux->slot_empty[slot]);
             }
             if (!ok) break;
@@ -475,52 +536,88 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         ptx::mma_commit(&aux->o_final);
-        if (!ok) drain_wait(&aux->o_final, 0);
+        // the MMAs have completed before TMEM is freed, even if the epilogue aborted
+        drain_wait(&aux->o_final, 0);
       }
       __syncwarp();
     }
   } else if (warp < kDqWarp0) {
-    ptx::setmaxnreg_inc<kRope ? kRegsSoftmaxRope : kRegsSoftmax>();
+    ptx::setmaxnreg_inc<Regs<kRope>::softmax>();
     if (ntiles > 0) {
       // ------------------------------------------------------------- softmax / epilogue
       const int qd = warp & 3;
       const int row = qd * 32 + lane;
       const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+      // the second score accumulator holds the odd K steps (none when r_k = 16)
+      const bool two_acc = p.r_k > 16;
       float l[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) l[j] = 0.f;
       bool ok = true;
-      // keys before RoPE: the query rows are read here, from shared memory
-      if (kRope) ok = ptx::named_bar_and(1, 128, wait_b(&aux->q_full, 0, aux, p.err));
-      const float* q_f = reinterpret_cast<const float*>(q_s);
+      if (kRope) {
+        // keys before RoPE: the fp32 query rows become the fp16 B operand of the score MMAs,
+        // [head][2 sub-blocks of 64 K][16 query slots][128 B] with the 128-byte swizzle;
+        // K element 2m holds dimension m and 2m + 1 dimension m + 64 (the order in which the
+        // rotated keys are stored), slots >= the group size are zero
+        ok = ptx::named_bar_and(1, 128, wait_b(&aux->q_full, 0, aux, p.err));
+        if (ok) {
+          const float* q_f = reinterpret_cast<const float*>(q_s);
+          uint8_t* qb = q_s + p.qf_bytes;
+          for (int idx = threadIdx.x - 128; idx < p.gh * kMaxG * kRD; idx += 128) {
+            const int hh = idx / (kMaxG * kRD), n = (idx / kRD) % kMaxG, k = idx % kRD;
+            const int dim = (k & 1) ? (k >> 1) + kRD / 2 : (k >> 1);
+            const float v = n < p.gsz ? q_f[(hh * p.gsz + n) * kRD + dim] : 0.f;
+            const int sb = k >> 6, ch = (k & 63) >> 3;
+            *reinterpret_cast<__half*>(qb + hh * kQbHeadBytes + sb * (kQbHeadBytes / 2) + n * 128 +
+                                       ((ch ^ (n & 7)) << 4) + (k & 7) * 2) = __float2half_rn(v);
+          }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&aux->qb_full);
+        }
+      }
       // rotation factors: cs holds the chunk in use, csn the one after it
       float cs[32], csn[32];
       auto load_cs = [&](float(&dst)[32], int tile_i, int c0) {
+        // pairs c0 .. c0 + 15 of this row's token; lanes own consecutive tokens, so each
+        // pair is one coalesced 256-byte read per warp
         const int t = tok_begin + tile_i * kTile + row;
-        const float2* src = p.rope_cs + (size_t)(t < tok_end ? t : tok_begin) * (kRD / 2) + c0;
+        const float2* src = p.rope_cs + rope_cs_index(t < tok_end ? t : tok_begin, c0, kRD / 2);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float4 v = __ldg(reinterpret_cast<const float4*>(src) + k);
-          dst[4 * k] = v.x;
-          dst[4 * k + 1] = v.y;
-          dst[4 * k + 2] = v.z;
-          dst[4 * k + 3] = v.w;
+        for (int k = 0; k < 16; ++k) {
+          const float2 v = __ldg(src + k * 128);
+          dst[2 * k] = v.x;
+          dst[2 * k + 1] = v.y;
+        }
+      };
+      // scores of tile buffer k2: the sum of the two accumulators
+      auto load_s = [&](int k2, bool valid, float(&s)[32]) {
+        const uint32_t s_col = tmem + lane_off + kSCol + 64 * k2;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t sv[16], sw[16];
+          ptx::tmem_ld16(s_col + 16 * hh, sv);
+          if (two_acc) ptx::tmem_ld16(s_col + 32 + 16 * hh, sw);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            s[16 * hh + j] = valid ? (two_acc ? __uint_as_float(sv[j]) + __uint_as_float(sw[j]) : __uint_as_float(sv[j]))
+                                   : -INFINITY;
         }
       };
       if (kRope) load_cs(cs, 0, 0);
       for (int i = 0; i < ntiles && ok; ++i) {
         const int k2 = i & 1;
         const bool valid = tok_begin + i * kTile + row < tok_end;
-        const uint32_t s_col = tmem + lane_off + kSCol + 32 * k2;
         float s[32];
         if (kRope) {
           ok = ptx::named_bar_and(1, 128, wait_b(&aux->k_full, i & 1, aux, p.err));
           if (!ok) break;
           ptx::tc_fence_after();
           if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 4 + 4 * i);
-          // score of query slot 16 h + jj: q_jj . RoPE_t(K^_h[t]), pairs (c, c + 64)
-#pragma unroll
-          for (int j = 0; j < 32; ++j) s[j] = 0.f;
+          // rotate-half RoPE of each row's keys at the token's position, written back over
+          // K^ as fp16: pair (c, c + 64) of chunk c0 goes to column h * 128 + c (K elements
+          // 2c, 2c + 1); a chunk's columns were read before they are written
 #pragma unroll 1
           for (int c0 = 0; c0 < kRD / 2; c0 += 16) {
             if (c0 + 16 < kRD / 2) load_cs(csn, i, c0 + 16);
@@ -532,41 +629,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_ld16(tmem + lane_off + h * kRD + c0, x1);
                 ptx::tmem_ld16(tmem + lane_off + h * kRD + kRD / 2 + c0, x2);
                 ptx::tmem_wait_ld();
-                float r1[16], r2[16];
+                uint32_t w[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                   const float a = __uint_as_float(x1[k]), e = __uint_as_float(x2[k]);
-                  r1[k] = a * cs[2 * k] - e * cs[2 * k + 1];
-                  r2[k] = e * cs[2 * k] + a * cs[2 * k + 1];
+                  const __half2 hv = __floats2half2_rn(a * cs[2 * k] - e * cs[2 * k + 1], e * cs[2 * k] + a * cs[2 * k + 1]);
+                  w[k] = *reinterpret_cast<const uint32_t*>(&hv);
                 }
-                // paired fp32 FMAs over adjacent elements (two partial sums per score,
-                // folded at the end of the chunk)
-                uint64_t acc[kG > 0 ? kG : 1];
-#pragma unroll
-                for (int jj = 0; jj < kG; ++jj) acc[jj] = pack2(s[h * kMaxG + jj], 0.f);
-#pragma unroll
-                for (int k = 0; k < 16; k += 4) {
-                  const uint64_t ra = pack2(r1[k], r1[k + 1]), rb = pack2(r1[k + 2], r1[k + 3]);
-                  const uint64_t rc = pack2(r2[k], r2[k + 1]), rd = pack2(r2[k + 2], r2[k + 3]);
-#pragma unroll
-                  for (int jj = 0; jj < kG; ++jj) {
-                    const float* qr = q_f + (size_t)(h * kG + jj) * kRD + c0 + k;
-                    const float4 qa = *reinterpret_cast<const float4*>(qr);
-                    const float4 qb = *reinterpret_cast<const float4*>(qr + kRD / 2);
-                    acc[jj] = ffma2(pack2(qa.x, qa.y), ra, acc[jj]);
-                    acc[jj] = ffma2(pack2(qa.z, qa.w), rb, acc[jj]);
-                    acc[jj] = ffma2(pack2(qb.x, qb.y), rc, acc[jj]);
-                    acc[jj] = ffma2(pack2(qb.z, qb.w), rd, acc[jj]);
-                  }
-                }
-#pragma unroll
-                for (int jj = 0; jj < kG; ++jj) s[h * kMaxG + jj] = lo2(acc[jj]) + hi2(acc[jj]);
+                tmem_st16(tmem + lane_off + h * kRD + c0, w);
               }
             }
 #pragma unroll
             for (int k = 0; k < 32; ++k) cs[k] = csn[k];
           }
-          // K^ has been read: GEMM0 of the next tile may overwrite it
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&aux->krot_full);
+          // the scores of the pair's query slots: head h's 16 slots in columns h * 128 + 64
+          ok = ptx::named_bar_and(1, 128, wait_b(&aux->s_full[0], i & 1, aux, p.err));
+          if (!ok) break;
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int h = 0; h < kGHMax; ++h) {
+            uint32_t sv[16];
+            if (h < p.gh) {
+              ptx::tmem_ld16(tmem + lane_off + h * kRD + kRD / 2, sv);
+              ptx::tmem_wait_ld();
+            }
+#pragma unroll
+            for (int jj = 0; jj < kMaxG; ++jj) s[h * kMaxG + jj] = h < p.gh ? __uint_as_float(sv[jj]) : 0.f;
+          }
+          // the scores have been read: GEMM0 of the next tile may overwrite the region
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&aux->k_empty);
@@ -579,11 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           ptx::tc_fence_after();
           if (i < 16 && threadIdx.x == 128) tc::trace_stamp(p.trace, 4 + 4 * i);
-          uint32_t sv[32];
-          ptx::tmem_ld32(s_col, sv);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+          load_s(k2, valid, s);
         }
 
         bool ex = false;
@@ -605,11 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             // the reduction consumes s; it is read again from TMEM
             aux->red[qd][lane] = warp_reduce_scatter32<true>(s, lane);
-            uint32_t sv[32];
-            ptx::tmem_ld32(s_col, sv);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+            load_s(k2, valid, s);
           }
           ptx::named_bar_sync(1, 128);
           if (qd == 0) {
@@ -678,20 +764,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         ptx::tc_fence_after();
         const size_t base_out = ((size_t)b * p.n_splits + split) * p.Hq;
-        // TMEM row m of a chunk holds rank 8 (m / 8) + perm(m % 8), perm = 0,4,1,5,2,6,3,7
+        // TMEM row m of chunk c holds rank 128 c + m (values are expanded in rank order)
         const int m = qd * 32 + lane;
-        const int e_in = (m & ~7) + ((m & 7) >> 1) + ((m & 1) << 2);
-        // query head of slot j (-1: padding)
-        auto head_of = [&](int j) -> int {
-          if (!kRope) return j < p.Hq ? j : -1;
-          const int h = j / kMaxG, jj = j % kMaxG;
-          return (h < p.gh && jj < p.gsz) ? (pair * p.gh + h) * p.gsz + jj : -1;
-        };
         for (int c = 0; c < p.cv; ++c) {
           uint32_t v2[32];
           ptx::tmem_ld32(tmem + lane_off + kOC + c * 32, v2);
           ptx::tmem_wait_ld();
-          const int e = c * 128 + e_in;
+          const int e = c * 128 + m;
           if (e < p.r_v) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -710,68 +789,95 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (threadIdx.x == 128) tc::trace_stamp(p.trace, kTraceSlots - 1);
       }
+    } else if (warp == 4) {
+      // a split that starts beyond its row's length: zero weight in the merge
+      const int J = head_of(lane);
+      if (J >= 0) {
+        const size_t base_out = ((size_t)b * p.n_splits + split) * p.Hq;
+        p.part_ml[(base_out + J) * 2] = -INFINITY;
+        p.part_ml[(base_out + J) * 2 + 1] = 0.f;
+      }
     }
   } else {
-    ptx::setmaxnreg_dec<kRegsDq>();
+    ptx::setmaxnreg_dec<Regs<kRope>::dq>();
     // ------------------------------------------------------------- dequantisation
     if (ntiles > 0) {
-      // warps 8..15 -> dq 0..255; unit v = (token v % 128, group v / 128 of the chunk) for
-      // v = dq, dq + 256, ...; lanes walk consecutive tokens
-      const int wi = warp - kDqWarp0;      // 0..7
-      const bool dq_live = true;
-      const int dq = wi * 32 + lane;
-      const uint32_t ring_base = ptx::smem_u32(ring);
-      bool ok = dq_live;
+      // warp (quarter qd = warp % 4, half h): TMEM lanes 32 qd .. + 31 of each operand slot,
+      // columns [32 h, +32) of it.  Keys: token 32 qd + lane, ranks 64 h .. + 63 of the
+      // chunk (groups 4c + 2h, + 1).  Values: rank 128 c + 32 qd + lane (group 4c + qd),
+      // tokens 64 h .. + 63.
+      const int qd = warp & 3, h = (warp - kDqWarp0) >> 2;
+      const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+      const uint32_t raw_base = ptx::smem_u32(raw);
+      bool ok = true;
       int pos = 0;
       for (int u = 0; u < nunits && ok; ++u) {
         int tile;
         bool is_v;
         tc::unit_of(u, ntiles, &tile, &is_v);
-        const int nvalid = tok_end - (tok_begin + tile * kTile);   // valid token rows of the tile
         const int G = is_v ? p.G_v : p.G_k;
         const int nch = is_v ? p.cv : p.ck;
         const int rs = u % p.nraw;
+        const uint32_t rb = raw_base + rs * p.raw_bytes;
         // waits are made warp-uniform: the warp arrives once, after __syncwarp
         if (!(ok = __all_sync(0xffffffffu, wait_b(&aux->raw_full[rs], (u / p.nraw) & 1, aux, p.err)))) break;
         for (int c = 0; c < nch; ++c, ++pos) {
-          const int slot = pos % p.nslot;
-          if (pos >= p.nslot &&
-              !(ok = __all_sync(0xffffffffu, wait_b(&aux->slot_empty[slot], ((pos / p.nslot) - 1) & 1, aux, p.err))))
+          const int slot = pos % p.nas;
+          if (pos >= p.nas &&
+              !(ok = __all_sync(0xffffffffu, wait_b(&aux->slot_empty[slot], ((pos / p.nas) - 1) & 1, aux, p.err))))
             break;
-          const int ng = min(4, G - 4 * c);
-          const uint8_t* rb = raw + rs * p.raw_bytes + c * 8192;          // codes of groups 4c..
-          const uint32_t* rp = reinterpret_cast<const uint32_t*>(raw + rs * p.raw_bytes + p.raw_params) + c * 512;
-          const uint32_t dst = ring_base + slot * kSlotBytes;
-          // up to three units per thread; all loads first, then the arithmetic and stores
-          constexpr int kU = (4 * kTile + kDqThreads - 1) / kDqThreads;
-          uint4 w[kU];
-          uint32_t prm[kU];
+          ptx::tc_fence_after();
+          uint32_t v[32];
+          bool any = false;
+          if (!is_v) {
+            const int t = qd * 32 + lane;
+            const int g0 = 4 * c + 2 * h;
+            any = g0 < G;
 #pragma unroll
-          for (int k = 0; k < kU; ++k) {
-            const int v = dq + k * kDqThreads, t = v & (kTile - 1), gl = v >> 7;
-            w[k] = make_uint4(0u, 0u, 0u, 0u);
-            prm[k] = 0u;
-            if (v < ng * kTile && t < nvalid) {
-              w[k] = reinterpret_cast<const uint4*>(rb)[gl * kTile + t];
-              prm[k] = rp[gl * kTile + t];
+            for (int gi = 0; gi < 2; ++gi) {
+              const int g = g0 + gi;
+              if (g < G) {
+                const uint4 w = lds128(rb + (uint32_t)(g * 2048 + t * 16));
+                const uint32_t prm = lds32(rb + p.raw_params + (uint32_t)((g * 128 + t) * 4));
+                const uint32_t s2 = __byte_perm(prm, 0u, 0x1010), z2 = __byte_perm(prm, 0u, 0x3232);
+                const uint4 ss = make_uint4(s2, s2, s2, s2), zz = make_uint4(z2, z2, z2, z2);
+                put4(v, 16 * gi + 0, dequant8(w.x, ss, zz));
+                put4(v, 16 * gi + 4, dequant8(w.y, ss, zz));
+                put4(v, 16 * gi + 8, dequant8(w.z, ss, zz));
+                put4(v, 16 * gi + 12, dequant8(w.w, ss, zz));
+              } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) v[16 * gi + k] = 0u;
+              }
+            }
+          } else {
+            const int g = 4 * c + qd;
+            any = g < G;
+            if (any) {
+              const int i = c * 128 + qd * 32 + lane;
+              const uint32_t rowa = rb + (uint32_t)(i * 64);
+              const uint32_t sc = rb + p.raw_params + (uint32_t)(g * 512 + h * 128);   // scales of tokens 64h..
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                const int lc = 2 * h + half;                                   // 32-token column
+                const uint4 w = lds128(rowa + (uint32_t)(((lc ^ ((i >> 1) & 3))) * 16));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  // tokens 64 h + 32 half + 8 k .. + 7: scale and zero pairs (broadcast reads)
+                  const uint32_t off = (uint32_t)((half * 32 + 8 * k) * 2);
+                  const uint4 sp = lds128(sc + off), zp = lds128(sc + 256 + off);
+                  const uint32_t wk = k == 0 ? w.x : (k == 1 ? w.y : (k == 2 ? w.z : w.w));
+                  put4(v, 16 * half + 4 * k, dequant8(wk, sp, zp));
+                }
+              }
             }
           }
-#pragma unroll
-          for (int k = 0; k < kU; ++k) {
-            const int v = dq + k * kDqThreads, t = v & (kTile - 1), gl = v >> 7, sw = t & 7;
-            if (v < ng * kTile) {
-              const uint32_t s2 = __byte_perm(prm[k], 0u, 0x1010), z2 = __byte_perm(prm[k], 0u, 0x3232);
-              // group gl = ranks 32 gl.. of the chunk: sub-block gl / 2, 16-byte columns 4 (gl % 2)..
-              const uint32_t rowa = dst + (gl >> 1) * kSubBytes + t * 128;
-              const int cb = (gl & 1) * 4;
-              sts128(rowa + (((cb + 0) ^ sw) << 4), dequant8(w[k].x, s2, z2));
-              sts128(rowa + (((cb + 1) ^ sw) << 4), dequant8(w[k].y, s2, z2));
-              sts128(rowa + (((cb + 2) ^ sw) << 4), dequant8(w[k].z, s2, z2));
-              sts128(rowa + (((cb + 3) ^ sw) << 4), dequant8(w[k].w, s2, z2));
-            }
+          if (any) {
+            ptx::tmem_st32(tmem + lane_off + (uint32_t)(kAC + slot * kASlotCols + 32 * h), v);
+            ptx::tmem_wait_st();
           }
-          // each lane fences its own stores for the tensor core; one arrival per warp
-          ptx::fence_proxy_async_smem();
+          // each thread's TMEM stores are complete; order them before the arrival
+          ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&aux->slot_full[slot]);
         }
@@ -784,8 +890,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, p.tmem_cols);
+    ptx::tmem_dealloc(tmem, 512);
   }
+  span_end(p.span);
 }
 
 // B_k as the fp16 B operand of GEMM0: out[n][pos] = B_k[rank(pos)][n] for the D output
@@ -804,57 +911,46 @@ __global__ void k_prep_bk16(const __nv_bfloat16* Bk, __half* out, int r_k, int r
 // host side
 // ---------------------------------------------------------------------------
 
+// keys before RoPE: the pair's fp32 query rows (rounded up to 1 KB), then the fp16 operand
+int qf_bytes_for(const lr_cache_desc* d) {
+  const int gh = d->n_kv_heads % 2 == 0 ? 2 : 1;
+  const int rows = gh * (d->n_q_heads / d->n_kv_heads);
+  return ((rows * kRD * 4 + 1023) / 1024) * 1024;
+}
+
 int q_bytes_for(const lr_cache_desc* d) {
-  if (d->rope_in_kernel) {
-    const int gh = d->n_kv_heads % 2 == 0 ? 2 : 1;
-    const int rows = gh * (d->n_q_heads / d->n_kv_heads);
-    return ((rows * kRD * 4 + 1023) / 1024) * 1024;
-  }
+  if (d->rope_in_kernel) return qf_bytes_for(d) + kGHMax * kQbHeadBytes;
   return ((d->rank_k + 63) / 64) * kQSubBytes;
 }
 
 struct I4Layout {
-  int nslot, nraw, nb;
+  int nraw, nb;
   uint32_t raw_bytes, raw_params;
   size_t smem;
 };
 
-// Raw slots hold one side of one tile.  As many operand slots as leave room for two raw
-// slots (up to four: the dequantisation can then run a full 128-rank chunk further ahead
-// of the MMAs), then as many raw slots (up to 6) as fit in 227 KB.  Keys before RoPE add
-// the B_k ring.
+// Raw slots hold one side of one tile; as many as fit in 227 KB (up to 8) after the query
+// rows and P, and for keys before RoPE the B_k ring (up to one tile's worth of sub-blocks,
+// so the next tile's load while the current one is rotated).  The operand slots are in TMEM.
 bool choose_layout(const lr_cache_desc* d, I4Layout* L) {
   const int G = std::max((d->rank_k + 31) / 32, (d->rank_v + 31) / 32);
   L->raw_params = (uint32_t)G * 2048u;
   L->raw_bytes = (uint32_t)G * 2560u;
-  const size_t fixed = (size_t)kAuxBytes + q_bytes_for(d) + 2 * kPBytes;
+  size_t fixed = (size_t)kAuxBytes + q_bytes_for(d) + 2 * kPBytes;
+  L->nb = 0;
   if (d->rope_in_kernel) {
-    // two operand slots and two raw slots, then B_k slots up to one tile's worth (the next
-    // tile's sub-blocks load while the current one is rotated), then raw slots
     const size_t bslot = (size_t)(d->n_kv_heads % 2 == 0 ? 2 : 1) * kSubBytes;
     const int kb = (d->rank_k + 63) / 64;
-    const size_t base = fixed + 2 * (size_t)kSlotBytes + 2 * (size_t)L->raw_bytes;
+    const size_t base = fixed + 2 * (size_t)L->raw_bytes;
     if (base + 2 * bslot > (size_t)kSmemLimit) return false;
     L->nb = std::min(kNBMax, std::max(2, std::min(kb, (int)(((size_t)kSmemLimit - base) / bslot))));
-    L->nslot = 2;
-    const size_t used = fixed + (size_t)L->nb * bslot + 2 * (size_t)kSlotBytes;
-    L->nraw = std::min(kMaxRaw, (int)(((size_t)kSmemLimit - used) / L->raw_bytes));
-    L->smem = used + (size_t)L->nraw * L->raw_bytes;
-    return true;
+    fixed += (size_t)L->nb * bslot;
   }
-  L->nb = 0;
-  for (int ns = kMaxSlots; ns >= 2; --ns) {
-    if (fixed + (size_t)ns * kSlotBytes > (size_t)kSmemLimit) continue;
-    const int nr =
-        std::min(kMaxRaw, (int)(((size_t)kSmemLimit - fixed - (size_t)ns * kSlotBytes) / L->raw_bytes));
-    if (nr >= 2) {
-      L->nslot = ns;
-      L->nraw = nr;
-      L->smem = fixed + (size_t)ns * kSlotBytes + (size_t)nr * L->raw_bytes;
-      return true;
-    }
-  }
-  return false;
+  const int nr = std::min(kMaxRaw, (int)(((size_t)kSmemLimit - fixed) / L->raw_bytes));
+  if (nr < 2) return false;
+  L->nraw = nr;
+  L->smem = fixed + (size_t)nr * L->raw_bytes;
+  return true;
 }
 
 int kv_per_cta(const lr_cache_desc* d) {
@@ -867,12 +963,12 @@ int kv_per_cta(const lr_cache_desc* d) {
 bool tc_i4_supported(const lr_cache_desc* d) {
   if (d->quant_bits != 4 || d->quant_group != 32) return false;
   if (d->dtype != LR_BF16) return false;
-  if (d->n_q_heads > 32 || d->rank_v > 512) return false;
-  // keys before RoPE: instantiated for the shape the parity tests cover (d = 128, seven
-  // query heads per KV head, KV heads in pairs); other shapes take the CUDA-core path
-  if (d->rope_in_kernel &&
-      (d->head_dim != kRD || d->n_q_heads != kRopeG * d->n_kv_heads || d->n_kv_heads % kGHMax != 0))
-    return false;
+  if (d->rank_v > 512) return false;
+  if (!d->rope_in_kernel && d->n_q_heads > 32) return false;   // all query heads in one N = 32 MMA
+  // keys before RoPE: d = 128 (the rotation pairs and the score MMA's K) and at most 16
+  // query heads per KV head (the score MMA's N); other shapes take the CUDA-core path
+  if (d->rope_in_kernel && (d->head_dim != kRD || d->n_q_heads / d->n_kv_heads > kMaxG)) return false;
+  // keys before RoPE keep O~ in 128 TMEM columns next to K^: r_v <= 512 fits
   I4Layout L;
   return choose_layout(d, &L);
 }
@@ -890,14 +986,14 @@ cudaError_t tc_i4_prepare(lr_cache* c, cudaStream_t s) {
   if (d.rope_in_kernel) {
     const int r_pad = ((d.rank_k + 127) / 128) * 128;
     if (!st->bk16) {
-      cudaError_t e = cudaMalloc(&st->bk16, (size_t)c->D * r_pad * 2);
+      cudaError_t e = lr_dev_malloc(&st->bk16, (size_t)c->D * r_pad * 2);
       if (e != cudaSuccess) return e;
       st->r_pad = r_pad;
     }
     const long long n = (long long)c->D * r_pad;
-    k_prep_bk16<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(c->B_k),
-                                                            reinterpret_cast<__half*>(st->bk16), d.rank_k, r_pad, c->D);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_serial(k_prep_bk16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s,
+                                  reinterpret_cast<const __nv_bfloat16*>(c->B_k), reinterpret_cast<__half*>(st->bk16),
+                                  d.rank_k, r_pad, c->D);
     if (e != cudaSuccess) return e;
     cuuint64_t dims[2] = {(cuuint64_t)r_pad, (cuuint64_t)c->D};
     cuuint64_t strides[1] = {(cuuint64_t)r_pad * 2};
@@ -908,7 +1004,7 @@ cudaError_t tc_i4_prepare(lr_cache* c, cudaStream_t s) {
   } else {
     const size_t qbytes = (size_t)d.batch * kQRows * d.rank_k * 2;
     if (!c->qt16) {
-      cudaError_t e = cudaMalloc(&c->qt16, qbytes);
+      cudaError_t e = lr_dev_malloc(&c->qt16, qbytes);
       if (e != cudaSuccess) return e;
       e = cudaMemset(c->qt16, 0, qbytes);
       if (e != cudaSuccess) return e;
@@ -922,7 +1018,6 @@ cudaError_t tc_i4_prepare(lr_cache* c, cudaStream_t s) {
   }
   I4Layout L;
   if (!choose_layout(&d, &L)) return cudaErrorNotSupported;
-  st->nslot = L.nslot;
   st->nraw = L.nraw;
   st->nb = L.nb;
   st->raw_bytes = L.raw_bytes;
@@ -945,6 +1040,9 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   if (!st) return cudaErrorNotSupported;
   const bool rope = d.rope_in_kernel != 0;
   I4Params p;
+  p.wait_ns = c->wait_ns;
+  p.row_len = c->row_len;
+  p.span = span_of(c->spans, SPAN_DECODE);
   p.codes_k = c->codes_k;
   p.codes_v = c->codes_v;
   p.params_k = c->params_k;
@@ -957,13 +1055,12 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   p.ck = (d.rank_k + 127) / 128;
   p.cv = (d.rank_v + 127) / 128;
   p.kb_k = (d.rank_k + 63) / 64;
-  p.tmem_cols = rope ? 512 : ((kOCol + p.cv * 32) <= 128 ? 128 : 256);
   p.Hq = d.n_q_heads;
   p.hist_len = c->hist_len;
   p.stable_len = std::min(c->stable_len, c->hist_len);
   p.split_tokens = split_tokens;
   p.n_splits = n_splits;
-  p.nslot = st->nslot;
+  p.nas = rope ? (512 - kAColR) / kASlotCols : (512 - kACol) / kASlotCols;
   p.nraw = st->nraw;
   p.q_bytes = st->q_bytes;
   p.raw_bytes = st->raw_bytes;
@@ -978,11 +1075,12 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   p.gh = kv_per_cta(&d);
   p.gsz = d.n_q_heads / d.n_kv_heads;
   p.q_load_bytes = (uint32_t)(p.gh * p.gsz * kRD * 4);
+  p.qf_bytes = rope ? (uint32_t)qf_bytes_for(&d) : 0u;
   p.nb = st->nb;
   // instantiation: 0 rank space; 1 keys before RoPE
   using Kern = void (*)(CUtensorMap, CUtensorMap, I4Params);
-  static const Kern kerns[2] = {k_decode_tc_i4<false, 0>, k_decode_tc_i4<true, kRopeG>};
-  if (rope && (p.gsz != kRopeG || p.gh != kGHMax)) return cudaErrorNotSupported;
+  static const Kern kerns[2] = {k_decode_tc_i4<false>, k_decode_tc_i4<true>};
+  if (rope && p.gsz > kMaxG) return cudaErrorNotSupported;
   const int ki = rope ? 1 : 0;
   const Kern kern = kerns[ki];
   static std::atomic<uint32_t> optin_done[2] = {0, 0};

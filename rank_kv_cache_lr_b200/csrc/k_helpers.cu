@@ -83,6 +83,7 @@ struct QprojArgs {
   int Hq, Hkv, d, D, rk;
   float scale_log2;
   int want_latent;
+  unsigned long long* span;   // timeline span, or null
 };
 
 template <typename T>
@@ -152,10 +153,12 @@ __device__ __forceinline__ void qproj_main(const QprojArgs& a, int rchunk, int h
 template <typename T>
 __global__ void __launch_bounds__(256) k_qproj(QprojArgs a) {
   extern __shared__ __align__(16) uint8_t qsm[];
+  span_begin(a.span);
   qproj_stage<T>(a, blockIdx.x, blockIdx.y, qsm);      // bases: stable data
   pdl_wait();
   pdl_trigger();
   qproj_main<T>(a, blockIdx.x, blockIdx.y, blockIdx.z, qsm);
+  span_end(a.span);
 }
 
 size_t qproj_smem(const lr_cache_desc& d, size_t es) {
@@ -176,6 +179,7 @@ struct AppendArgs {
   long long cap; int dst_slot; int project;
   const void* new_k; const void* new_v;   // exact token for the ring, or null
   void* win_k; void* win_v; int slots; int new_slot;
+  unsigned long long* span;   // timeline span, or null
   int B, D, kind, dtype;
 };
 
@@ -229,7 +233,7 @@ __device__ __forceinline__ void append_main(const AppendArgs& a, int x, int b, u
       for (int w = 0; w < 8; ++w) z += red[w][lane];
       const long long row = (long long)b * a.cap + a.dst_slot;
       store_latent_chunk(z, ch, r, a.kind, a.dtype, is_k ? a.Zk : a.Zv, is_k ? a.codes_k : a.codes_v,
-                         is_k ? a.params_k : a.params_v, is_k ? a.Gk : a.Gv, row);
+                         is_k ? a.params_k : a.params_v, is_k ? a.Gk : a.Gv, row, !is_k);
     }
     return;
   }
@@ -245,10 +249,12 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_append(AppendArgs a) {
   extern __shared__ __align__(16) uint8_t asm_[];
   __shared__ float red[8][32];
+  span_begin(a.span);
   append_stage<T>(a, blockIdx.x, asm_);                 // bases: stable data
   pdl_wait();
   pdl_trigger();
   append_main<T>(a, blockIdx.x, blockIdx.y, asm_, red);
+  span_end(a.span);
 }
 
 // The independent first half of a decode step in one grid: CTAs [0, x_app) of each
@@ -259,12 +265,14 @@ __global__ void __launch_bounds__(256) k_step_pre(AppendArgs aa, QprojArgs qa, i
   __shared__ float red[8][32];
   const int x = blockIdx.x, b = blockIdx.y;
   const int qx = x - x_app;
+  span_begin(aa.span);
   if (x < x_app) append_stage<T>(aa, x, psm);
   else qproj_stage<T>(qa, qx % nchunks_q, qx / nchunks_q, psm);
   pdl_wait();
   pdl_trigger();
   if (x < x_app) append_main<T>(aa, x, b, psm, red);
   else qproj_main<T>(qa, qx % nchunks_q, qx / nchunks_q, b, psm);
+  span_end(aa.span);
 }
 
 // ---- split merge and output projection ------------------------------------------
@@ -283,6 +291,14 @@ struct MergeArgs {
   const float* part_o; const float* part_ml; const float* win_o; const float* win_ml;
   const void* Bv; void* out; float* lse;
   int S, Hq, Hkv, d, D, rv;
+  // partial (b, s) starts at head row (b * b_stride + s * s_stride) * Hq of part_o / part_ml:
+  // the cache's [B][S][Hq] has b_stride = S, s_stride = 1; gathered shards [S][B][Hq] have
+  // b_stride = 1, s_stride = B
+  long long b_stride, s_stride;
+  // rank-space output instead of the projection (one column block): the merged o~ relative
+  // to the merged max, [B][Hq][rv], and (m, l) [B][Hq][2]; or null
+  float* rs_o; float* rs_ml;
+  unsigned long long* span;   // timeline span, or null
 };
 
 size_t merge_pitch_f(int rv) { return (size_t)rv + 4; }   // o~ rows, padded against bank conflicts
@@ -300,7 +316,8 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
   float* ot = reinterpret_cast<float*>(msm + (size_t)rv * kMergeCols * es);   // [8][rv + 4]
   float* wsm = ot + kMergeHeads * opitch;                                     // [8][S]
   float* red = wsm + kMergeHeads * S;                                         // [4][8][32]
-  float* hdr = red + 4 * kMergeHeads * kMergeCols;                            // [8][3]
+  float* hdr = red + 4 * kMergeHeads * kMergeCols;                            // [8][4]
+  span_begin(a.span);
   stage_rows(bs, ncols * es, a.Bv, a.D, es, 0, rv, (long long)h * a.d + c0, ncols);   // stable data
   pdl_wait();
   pdl_trigger();
@@ -315,14 +332,15 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
     if (warp < nh) {
       const int j = h * G + jb + warp;
       float m = -INFINITY;
-      for (int s = lane; s < S; s += 32) m = fmaxf(m, a.part_ml[(((size_t)b * S + s) * a.Hq + j) * 2]);
+      for (int s = lane; s < S; s += 32)
+        m = fmaxf(m, a.part_ml[(((size_t)b * a.b_stride + (size_t)s * a.s_stride) * a.Hq + j) * 2]);
       const float mw = a.win_ml ? a.win_ml[((size_t)b * a.Hq + j) * 2] : -INFINITY;
       m = fmaxf(m, mw);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       float l = 0.f;
       for (int s = lane; s < S; s += 32) {
-        const size_t e = (((size_t)b * S + s) * a.Hq + j) * 2;
+        const size_t e = (((size_t)b * a.b_stride + (size_t)s * a.s_stride) * a.Hq + j) * 2;
         const float ms = a.part_ml[e];
         const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - m);
         wsm[warp * S + s] = w;
@@ -336,21 +354,22 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
           ww = exp2f(mw - m);
           l = fmaf(ww, a.win_ml[((size_t)b * a.Hq + j) * 2 + 1], l);
         }
-        hdr[warp * 3 + 0] = m;
-        hdr[warp * 3 + 1] = 1.0f / l;
-        hdr[warp * 3 + 2] = ww;
+        hdr[warp * 4 + 0] = m;
+        hdr[warp * 4 + 1] = 1.0f / l;
+        hdr[warp * 4 + 2] = ww;
+        hdr[warp * 4 + 3] = l;
         if (a.lse && cb == 0) a.lse[(size_t)b * a.Hq + j] = (m + log2f(l)) * LR_LN2;
       }
     }
     __syncthreads();
     // combined rank-space outputs, thread = rank; two heads at a time with up to 16
     // splits each in flight, so the L2 round trips overlap
-    const size_t sstride = (size_t)a.Hq * rv;
+    const size_t sstride = (size_t)a.s_stride * a.Hq * rv;
     for (int u0 = 0; u0 < nh; u0 += 2) {
       const bool two = u0 + 1 < nh;
       const int j0 = h * G + jb + u0;
       for (int i = tid; i < rv; i += kMergeThreads) {
-        const float* src0 = a.part_o + ((size_t)b * S * a.Hq + j0) * rv + i;
+        const float* src0 = a.part_o + ((size_t)b * a.b_stride * a.Hq + j0) * rv + i;
         const float* src1 = src0 + rv;                       // head j0 + 1
         float acc0 = 0.f, acc1 = 0.f;
         for (int s0 = 0; s0 < S; s0 += 16) {
@@ -364,8 +383,13 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             if (s0 + k < S) {
-              acc0 = fmaf(wsm[u0 * S + s0 + k], v0[k], acc0);
-              if (two) acc1 = fmaf(wsm[(u0 + 1) * S + s0 + k], v1[k], acc1);
+              // a split with no tokens has weight 0 and an unwritten output: skipped
+              const float w0 = wsm[u0 * S + s0 + k];
+              if (w0 != 0.f) acc0 = fmaf(w0, v0[k], acc0);
+              if (two) {
+                const float w1 = wsm[(u0 + 1) * S + s0 + k];
+                if (w1 != 0.f) acc1 = fmaf(w1, v1[k], acc1);
+              }
             }
           }
         }
@@ -378,6 +402,19 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
       staged = true;
     }
     __syncthreads();
+    if (a.rs_o) {
+      // rank-space partial of this shard: the merged o~ (relative to m) and (m, l)
+      for (int idx = tid; idx < nh * rv; idx += kMergeThreads) {
+        const int u = idx / rv, i = idx % rv;
+        a.rs_o[((size_t)b * a.Hq + h * G + jb + u) * rv + i] = ot[u * opitch + i];
+      }
+      if (tid < nh) {
+        a.rs_ml[((size_t)b * a.Hq + h * G + jb + tid) * 2] = hdr[tid * 4 + 0];
+        a.rs_ml[((size_t)b * a.Hq + h * G + jb + tid) * 2 + 1] = hdr[tid * 4 + 3];
+      }
+      __syncthreads();
+      continue;
+    }
     // projection partial sums over this thread's quarter of the ranks
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     if (hh < nh && 4 * cq < ncols) {
@@ -408,18 +445,19 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
                    red[(2 * kMergeHeads + u) * kMergeCols + c]) +
                   red[(3 * kMergeHeads + u) * kMergeCols + c];
         const size_t oi = ((size_t)b * a.Hq + j) * a.d + c0 + c;
-        if (a.win_o) o = fmaf(hdr[u * 3 + 2], a.win_o[oi], o);
-        El<T>::st(a.out, oi, o * hdr[u * 3 + 1]);
+        if (a.win_o) o = fmaf(hdr[u * 4 + 2], a.win_o[oi], o);
+        El<T>::st(a.out, oi, o * hdr[u * 4 + 1]);
       }
     }
     __syncthreads();
   }
+  span_end(a.span);
 }
 
 size_t merge_smem(const lr_cache_desc& d, int S, size_t es) {
   return (size_t)d.rank_v * kMergeCols * es +
          ((size_t)kMergeHeads * merge_pitch_f(d.rank_v) + (size_t)kMergeHeads * S +
-          4 * kMergeHeads * kMergeCols + kMergeHeads * 3) * sizeof(float);
+          4 * kMergeHeads * kMergeCols + kMergeHeads * 4) * sizeof(float);
 }
 
 // ---- argument construction ------------------------------------------------------------
@@ -436,6 +474,7 @@ QprojArgs make_qproj_args(const lr_cache* c, const void* q, bool tc) {
   a.Hq = d.n_q_heads; a.Hkv = d.n_kv_heads; a.d = d.head_dim; a.D = c->D; a.rk = d.rank_k;
   a.scale_log2 = c->scale_log2;
   a.want_latent = rope ? 0 : 1;
+  a.span = span_of(c->spans, SPAN_PRE);
   return a;
 }
 
@@ -468,6 +507,7 @@ AppendArgs make_append_args(const lr_cache* c, const void* k, const void* v) {
   a.win_k = c->win_k; a.win_v = c->win_v; a.slots = c->win_slots;
   a.new_slot = win ? (c->len % c->win_slots) : 0;
   a.B = d.batch; a.D = c->D; a.kind = c->latent_kind; a.dtype = d.dtype;
+  a.span = span_of(c->spans, SPAN_PRE);
   return a;
 }
 
@@ -476,27 +516,33 @@ int append_ctas(const AppendArgs& a) { return (a.project ? a.chunks_k + a.chunks
 size_t append_smem(const lr_cache* c) { return (size_t)c->D * 32 * c->esize + (size_t)c->D * c->esize; }
 
 template <typename T>
-cudaError_t qproj_t(const lr_cache* c, const void* q, cudaStream_t s, bool tc) {
+cudaError_t qproj_t(const lr_cache* c, const void* q, cudaStream_t s, bool tc, bool pdl = true) {
   const lr_cache_desc& d = c->desc;
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_qproj<T>, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_qproj<T>, dim3(qproj_chunks(c), d.n_kv_heads, d.batch), dim3(256), qproj_smem(d, sizeof(T)), s,
-                    make_qproj_args(c, q, tc));
+  const dim3 grid(qproj_chunks(c), d.n_kv_heads, d.batch);
+  if (!pdl) return launch_serial(k_qproj<T>, grid, dim3(256), qproj_smem(d, sizeof(T)), s, make_qproj_args(c, q, tc));
+  return launch_pdl(k_qproj<T>, grid, dim3(256), qproj_smem(d, sizeof(T)), s, make_qproj_args(c, q, tc));
 }
 
 template <typename T>
-cudaError_t merge_t(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s) {
+cudaError_t merge_t(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s,
+                    const MergeSource* src = nullptr) {
   const lr_cache_desc& d = c->desc;
-  const bool win = c->win_slots > 0;
+  const bool win = c->win_slots > 0 && !src;
   const size_t smem = merge_smem(d, n_splits, sizeof(T));
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_merge<T>, optin_done);
   if (e != cudaSuccess) return e;
   MergeArgs a;
-  a.part_o = c->part_o;
-  a.part_ml = c->part_ml;
+  a.part_o = src ? src->part_o : c->part_o;
+  a.part_ml = src ? src->part_ml : c->part_ml;
+  a.b_stride = src ? src->b_stride : n_splits;
+  a.s_stride = src ? src->s_stride : 1;
+  a.rs_o = src ? src->rs_o : nullptr;
+  a.rs_ml = src ? src->rs_ml : nullptr;
   a.win_o = win ? c->win_o : nullptr;
   a.win_ml = win ? c->win_ml : nullptr;
   a.Bv = c->B_v;
@@ -508,7 +554,8 @@ cudaError_t merge_t(const lr_cache* c, int n_splits, void* out, float* lse, cuda
   a.d = d.head_dim;
   a.D = c->D;
   a.rv = d.rank_v;
-  const int cbs = (d.head_dim + kMergeCols - 1) / kMergeCols;
+  a.span = span_of(c->spans, SPAN_MERGE);
+  const int cbs = a.rs_o ? 1 : (d.head_dim + kMergeCols - 1) / kMergeCols;
   return launch_pdl(k_merge<T>, dim3(cbs, d.n_kv_heads, d.batch), dim3(kMergeThreads), smem, s, a);
 }
 
@@ -537,8 +584,9 @@ cudaError_t step_pre_t(lr_cache* c, const void* k, const void* v, const void* q,
 
 }  // namespace
 
-cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s) {
-  return c->desc.dtype == LR_BF16 ? qproj_t<__nv_bfloat16>(c, q, s, false) : qproj_t<float>(c, q, s, false);
+cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s, bool pdl) {
+  return c->desc.dtype == LR_BF16 ? qproj_t<__nv_bfloat16>(c, q, s, false, pdl)
+                                  : qproj_t<float>(c, q, s, false, pdl);
 }
 
 cudaError_t launch_qproj_tc(const lr_cache* c, const void* q, cudaStream_t s) {
@@ -547,9 +595,10 @@ cudaError_t launch_qproj_tc(const lr_cache* c, const void* q, cudaStream_t s) {
   return qproj_t<__nv_bfloat16>(c, q, s, true);
 }
 
-cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s) {
-  return c->desc.dtype == LR_BF16 ? merge_t<__nv_bfloat16>(c, n_splits, out, lse, s)
-                                  : merge_t<float>(c, n_splits, out, lse, s);
+cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s,
+                         const MergeSource* src) {
+  return c->desc.dtype == LR_BF16 ? merge_t<__nv_bfloat16>(c, n_splits, out, lse, s, src)
+                                  : merge_t<float>(c, n_splits, out, lse, s, src);
 }
 
 cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s) {

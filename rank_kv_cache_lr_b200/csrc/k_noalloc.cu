@@ -49,7 +49,10 @@ extern "C" lr_status lr_attn_decode_noalloc(const lr_cache_desc* desc, int32_t l
                                             const void* z_v, const void* B_k, const void* B_v, const void* q,
                                             void* out, float* lse, void* stream) {
   if (!desc || !z_k || !z_v || !B_k || !B_v || !q || !out) return LR_ERR_INVALID_ARG;
-  if (desc->window != 0 || desc->quant_bits != 0 || desc->rope_in_kernel != 0) return LR_ERR_UNSUPPORTED;
+  // the bases are staged into shared memory with 16-byte copies
+  if ((reinterpret_cast<uintptr_t>(B_k) | reinterpret_cast<uintptr_t>(B_v)) & 15) return LR_ERR_INVALID_ARG;
+  if (desc->window != 0 || desc->quant_bits != 0 || desc->rope_in_kernel != 0 || desc->latent_groups > 1)
+    return LR_ERR_UNSUPPORTED;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess) return LR_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LR_ERR_CUDA;
@@ -96,7 +99,11 @@ extern "C" lr_status lr_attn_decode_noalloc(const lr_cache_desc* desc, int32_t l
   if (decode_simt_smem(&c) > 227 * 1024) return LR_ERR_UNSUPPORTED;
 
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = launch_qproj(&c, q, s);
+  // The bases belong to the caller, and the kernel just before this call may have written
+  // them; the query projection stages B_k in its prologue, so it starts only after that
+  // work has completed (no programmatic overlap).  The kernels after it follow their own
+  // predecessor, which writes neither basis.
+  cudaError_t e = launch_qproj(&c, q, s, /*pdl=*/false);
   if (e == cudaSuccess) e = launch_decode_simt(&c, plan.n_splits, plan.split_tokens, s);
   if (e == cudaSuccess) e = launch_merge(&c, plan.n_splits, out, lse, s);
   return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;

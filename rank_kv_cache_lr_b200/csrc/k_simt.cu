@@ -26,6 +26,7 @@ constexpr int kSyncRows = 16;     // rows per CTA in the SIMT basis sync
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind) {
   extern __shared__ float sm[];
+  span_begin(a.span);
   pdl_wait();
   pdl_trigger();
   const int split = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
@@ -50,7 +51,7 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind)
 
   const int group = Hq / a.Hkv;
   const int t_begin = split * a.split_tokens;
-  const int t_end = min(a.hist_len, t_begin + a.split_tokens);
+  const int t_end = min(row_hist(a.row_len, b, a.hist_len), t_begin + a.split_tokens);
   for (int t0 = t_begin; t0 < t_end; t0 += kTileSimt) {
     const int n = min(kTileSimt, t_end - t0);
     const long long row0 = (long long)b * a.k.cap + t0;
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind)
         const int t = idx / (a.Hkv * half);
         const int rem = idx % (a.Hkv * half);
         const int h = rem / half, i = rem % half;
-        const float2 cs = a.rope_cs[(long long)(t0 + t) * half + i];
+        const float2 cs = a.rope_cs[rope_cs_index(t0 + t, i, half)];
         float* row = kh + t * a.D + h * a.d;
         const float x1 = row[i], x2 = row[i + half];
         row[i] = x1 * cs.x - x2 * cs.y;
@@ -134,6 +135,7 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind)
     a.part_ml[(base + j) * 2] = m_s[j];
     a.part_ml[(base + j) * 2 + 1] = l_s[j];
   }
+  span_end(a.span);
 }
 
 // ---------------------------------------------------------------------------
@@ -142,11 +144,13 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) k_window(const void* win_k, const void* win_v, const float* qd,
                                                 float* win_o, float* win_ml, int Hq, int Hkv, int d,
-                                                int D, int slots, int hist_len, int win_len, int dtype) {
+                                                int D, int slots, int hist_len, int win_len, int dtype,
+                                                unsigned long long* span) {
   extern __shared__ float wsm[];
   float* q_s = wsm;           // [d]
   float* p_s = wsm + d;       // [win_len]
   __shared__ float red[2];
+  span_begin(span);
   pdl_wait();
   pdl_trigger();
   const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
@@ -189,6 +193,7 @@ __global__ void __launch_bounds__(128) k_window(const void* win_k, const void* w
     win_ml[((long long)b * Hq + j) * 2] = red[0];
     win_ml[((long long)b * Hq + j) * 2 + 1] = red[1];
   }
+  span_end(span);
 }
 
 // bulk latent fill: one warp per (token, 32-coordinate chunk)
@@ -207,6 +212,7 @@ __global__ void __launch_bounds__(256) k_append_latent(const float* zk, const fl
   if (pi >= (long long)n * per_tok) return;
   const int t = (int)(pi / per_tok), c = (int)(pi % per_tok);
   const bool is_k = c < chunks_k;
+  if (!is_k && kind == LK_INT4) return;   // int4 values: k_append_latent_v
   const int ch = is_k ? c : c - chunks_k;
   const int r = is_k ? rk : rv;
   const float* src = is_k ? zk : zv;
@@ -215,6 +221,48 @@ __global__ void __launch_bounds__(256) k_append_latent(const float* zk, const fl
   const long long row = (long long)b * cap + slot0 + t;
   store_latent_chunk(z, ch, r, kind, dtype, is_k ? Zk : Zv, is_k ? codes_k : codes_v,
                      is_k ? params_k : params_v, is_k ? Gk : Gv, row);
+}
+
+// bulk fill of int4 values in the rank-major layout: one warp per (8-token word, group),
+// lane = rank.  The warp quantises the word's tokens one after another and writes each
+// rank's word once; a word the fill covers only in part (the ends of the range) keeps its
+// other tokens' nibbles (cleared and set with atomics, which touch only the filled bits).
+__global__ void __launch_bounds__(256) k_append_latent_v(const float* zv, int n, int rv, int Gv, uint32_t* codes,
+                                                         uint32_t* params, long long cap, int slot0) {
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int w0 = slot0 >> 3, nwords = ((slot0 + n - 1) >> 3) - w0 + 1;
+  const long long pi = (long long)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (pi >= (long long)nwords * Gv) return;
+  const int wq = w0 + (int)(pi / Gv), g = (int)(pi % Gv);
+  const int b = blockIdx.y;
+  const int i = g * 32 + lane;
+  const bool valid = i < rv;
+  uint32_t word = 0, mask = 0;
+  unsigned short* h = reinterpret_cast<unsigned short*>(params);
+  for (int k = 0; k < 8; ++k) {
+    const int t = wq * 8 + k;
+    if (t < slot0 || t >= slot0 + n) continue;   // warp-uniform
+    const float z = valid ? zv[((long long)b * n + (t - slot0)) * rv + i] : 0.f;
+    const QuantOut q = quant_group_codes(z, valid);
+    const long long row = (long long)b * cap + t;
+    const int sh = 4 * i4v_nibble(row);
+    word |= q.code << sh;
+    mask |= 15u << sh;
+    if (lane == 0) {
+      const long long si = i4v_scale_index(row, Gv, g);
+      h[si] = q.sh;
+      h[si + 128] = q.zh;
+    }
+  }
+  uint32_t* w = codes + i4v_code_index((long long)b * cap + wq * 8, Gv, i);
+  if (mask == 0xFFFFFFFFu) {
+    *w = word;
+  } else {
+    atomicAnd(w, ~mask);
+    if (word) atomicOr(w, word);
+  }
 }
 
 // basis sync on CUDA cores: Z[b][t][:] <- Z[b][t][:] R for t < hist_len (in place)
@@ -252,6 +300,7 @@ LatentRef latent_ref(const lr_cache* c, bool k) {
   L.r = k ? c->desc.rank_k : c->desc.rank_v;
   L.G = k ? c->G_k : c->G_v;
   L.cap = c->lat_cap;
+  L.rank_major = (!k && c->latent_kind == LK_INT4) ? 1 : 0;
   return L;
 }
 
@@ -283,6 +332,8 @@ cudaError_t launch_decode_simt(const lr_cache* c, int n_splits, int split_tokens
   a.Hq = d.n_q_heads; a.Hkv = d.n_kv_heads; a.d = d.head_dim; a.D = c->D;
   a.hist_len = c->hist_len; a.split_tokens = split_tokens; a.n_splits = n_splits;
   a.rope = d.rope_in_kernel; a.dtype = d.dtype;
+  a.row_len = c->row_len;
+  a.span = span_of(c->spans, SPAN_DECODE);
   const size_t smem = decode_simt_smem(c);
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_decode_simt, optin_done);
@@ -300,7 +351,8 @@ cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
   cudaError_t e = smem_optin(k_window, optin_done);
   if (e != cudaSuccess) return e;
   return launch_pdl(k_window, grid, dim3(128), smem, s, c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads, d.n_kv_heads,
-                                   d.head_dim, c->D, c->win_slots, c->hist_len, c->win_len, d.dtype);
+                                   d.head_dim, c->D, c->win_slots, c->hist_len, c->win_len, d.dtype,
+                                   span_of(c->spans, SPAN_WINDOW));
 }
 
 cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, int n, cudaStream_t s) {
@@ -311,9 +363,17 @@ cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, 
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_append_latent, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_append_latent, grid, dim3(256), 0, s, zk, zv, n, d.batch, d.rank_k, d.rank_v, chunks_k, chunks_v, c->z_k,
-                                       c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->G_k,
-                                       c->G_v, c->lat_cap, c->hist_len, c->latent_kind, d.dtype);
+  e = launch_pdl(k_append_latent, grid, dim3(256), 0, s, zk, zv, n, d.batch, d.rank_k, d.rank_v, chunks_k, chunks_v,
+                 c->z_k, c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->G_k, c->G_v, c->lat_cap,
+                 c->hist_len, c->latent_kind, d.dtype);
+  if (e != cudaSuccess || c->latent_kind != LK_INT4 || n == 0) return e;
+  const int slot0 = c->hist_len;
+  const long long units = (long long)(((slot0 + n - 1) >> 3) - (slot0 >> 3) + 1) * c->G_v;
+  static std::atomic<uint32_t> optin_v{0};
+  e = smem_optin(k_append_latent_v, optin_v);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_append_latent_v, dim3((unsigned)((units + 7) / 8), d.batch), dim3(256), 0, s, zv, n, d.rank_v,
+                    c->G_v, c->codes_v, c->params_v, c->lat_cap, slot0);
 }
 
 cudaError_t launch_sync_simt(lr_cache* c, const float* R, int which, cudaStream_t s) {

@@ -32,6 +32,7 @@ constexpr int kRBox = 64 * 128;           // R box: 64 k-rows x 64 n-columns x 2
 constexpr int kAuxBytes = 1024;
 
 struct SyncParams {
+  unsigned long long wait_ns;   // bounded-wait limit (0: the default)
   int r, kb, B, ntile, units, hist;
   uint32_t z_bytes, r_half, r_slot;   // tile bytes; bytes of one of hi/lo per chunk; slot bytes
   int* err;
@@ -47,8 +48,10 @@ struct SyncParams {
 struct Aux {
   uint64_t z_full, z_empty, d_full, d_empty;
   uint64_t r_full[2], r_empty[2];
+  uint64_t fin;                 // one MMA commit after the last unit: every MMA has completed
   uint32_t tmem_base;
   int abort_flag;
+  unsigned long long wait_ns;   // this launch's wait limit
 };
 static_assert(sizeof(Aux) <= kAuxBytes, "aux block");
 
@@ -59,7 +62,7 @@ struct SyncState {
 };
 
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
-  return tc::wait_b(bar, parity, &aux->abort_flag, err);
+  return tc::wait_b(bar, parity, &aux->abort_flag, err, aux->wait_ns);
 }
 
 // unit u -> (side, sequence, first token)
@@ -92,11 +95,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(&aux->z_empty, 1);
     ptx::mbar_init(&aux->d_full, 1);
     ptx::mbar_init(&aux->d_empty, 4);   // one arrival per epilogue warp
+    ptx::mbar_init(&aux->fin, 1);
     for (int k = 0; k < 2; ++k) {
       ptx::mbar_init(&aux->r_full[k], 1);
       ptx::mbar_init(&aux->r_empty[k], 1);
     }
     aux->abort_flag = 0;
+    aux->wait_ns = tc::wait_limit(p.wait_ns);
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -141,10 +146,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           r_issued = rpos + 1;
         }
       }
-      if (!ok) {
-        for (int i = std::max(0, z_issued - 1); i < z_issued; ++i) drain_wait(&aux->z_full, i & 1);
-        for (int k = std::max(0, r_issued - 2); k < r_issued; ++k) drain_wait(&aux->r_full[k & 1], (k >> 1) & 1);
-      }
+      // Every copy this thread issued has landed before the CTA can exit, whether or not
+      // the CTA aborted (an abort in another role may come after this loop); in a normal
+      // run these phases have been waited already and the waits return at once.
+      (void)ok;
+      for (int i = std::max(0, z_issued - 1); i < z_issued; ++i) drain_wait(&aux->z_full, i & 1);
+      for (int k = std::max(0, r_issued - 2); k < r_issued; ++k) drain_wait(&aux->r_full[k & 1], (k >> 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -176,10 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mma_commit(&aux->d_full);
         ++dcommits;
       }
-      if (!ok) {   // every MMA issued so far completes before TMEM is freed
-        ptx::mma_commit(&aux->d_full);
-        drain_wait(&aux->d_full, dcommits & 1);
-      }
+      // every MMA issued so far completes before TMEM is freed, even if the epilogue aborted
+      (void)dcommits;
+      ptx::mma_commit(&aux->fin);
+      drain_wait(&aux->fin, 0);
     }
     __syncwarp();
   } else if (my_units > 0) {
@@ -282,9 +289,12 @@ cudaError_t launch_sync_tc(lr_cache* c, const float* R_k, const float* R_v, cuda
   if (!st) {
     st = new (std::nothrow) SyncState();
     if (!st) return cudaErrorMemoryAllocation;
+    cudaError_t e = lr_dev_malloc(&st->rbuf, (size_t)2 * 2 * r * r * sizeof(__nv_bfloat16));
+    if (e != cudaSuccess) {   // nothing is kept, so the next call starts over
+      delete st;
+      return e;
+    }
     c->sync_state = st;
-    cudaError_t e = cudaMalloc(&st->rbuf, (size_t)2 * 2 * r * r * sizeof(__nv_bfloat16));
-    if (e != cudaSuccess) return e;
     st->r = r;
     const cuuint64_t cap = d.capacity, B = d.batch;
     cuuint64_t zdims[3] = {(cuuint64_t)r, cap, B};
@@ -302,17 +312,12 @@ cudaError_t launch_sync_tc(lr_cache* c, const float* R_k, const float* R_v, cuda
   const int ntile = (c->hist_len + kTile - 1) / kTile;
   if (ntile == 0 || (!R_k && !R_v)) return cudaSuccess;
   cudaError_t e = cudaSuccess;
-  if (R_k) {
-    k_sync_prep<<<std::min(256, (r * r + 255) / 256), 256, 0, s>>>(R_k, st->rbuf, r);
-    lr_count_launch();
-  }
-  if (R_v) {
-    k_sync_prep<<<std::min(256, (r * r + 255) / 256), 256, 0, s>>>(R_v, st->rbuf + (size_t)2 * r * r, r);
-    lr_count_launch();
-  }
-  e = cudaGetLastError();
+  const dim3 pgrid(std::min(256, (r * r + 255) / 256));
+  if (R_k) e = launch_serial(k_sync_prep, pgrid, dim3(256), 0, s, R_k, st->rbuf, r);
+  if (e == cudaSuccess && R_v) e = launch_serial(k_sync_prep, pgrid, dim3(256), 0, s, R_v, st->rbuf + (size_t)2 * r * r, r);
   if (e != cudaSuccess) return e;
   SyncParams p;
+  p.wait_ns = c->wait_ns;
   p.r = r;
   p.kb = (r + 63) / 64;
   p.B = d.batch;

@@ -12,8 +12,41 @@
 namespace {
 
 std::atomic<long long> g_launches{0};
+// Armed faults: the number of operations of each kind still to succeed before one fails
+// (-1: none armed).
+std::atomic<long long> g_fault_left[2] = {{-1}, {-1}};
+
+bool fault_fires(int kind) {
+  long long left = g_fault_left[kind].load();
+  while (left >= 0) {
+    if (g_fault_left[kind].compare_exchange_weak(left, left - 1)) return left == 0;
+  }
+  return false;
+}
+
+int groups_of(const lr_cache_desc* d) { return d->latent_groups > 1 ? d->latent_groups : 1; }
+
+// The description the kernels see: g latent groups of rank r stored as one block-diagonal
+// latent of rank g r.
+lr_cache_desc effective_desc(const lr_cache_desc* d) {
+  lr_cache_desc e = *d;
+  e.rank_k *= groups_of(d);
+  e.rank_v *= groups_of(d);
+  return e;
+}
+
+lr_status validate_user_desc(const lr_cache_desc* d);
 
 lr_status validate_desc(const lr_cache_desc* d) {
+  if (!d) return LR_ERR_INVALID_ARG;
+  if (d->latent_groups < 0) return LR_ERR_INVALID_ARG;
+  if (d->latent_groups > 1 && (d->n_kv_heads % d->latent_groups)) return LR_ERR_INVALID_ARG;
+  if (d->rank_k < 16 || d->rank_k % 16 || d->rank_v < 16 || d->rank_v % 16) return LR_ERR_INVALID_ARG;
+  const lr_cache_desc e = effective_desc(d);
+  return validate_user_desc(&e);
+}
+
+lr_status validate_user_desc(const lr_cache_desc* d) {
   if (!d) return LR_ERR_INVALID_ARG;
   if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1) return LR_ERR_INVALID_ARG;
   if (d->n_q_heads % d->n_kv_heads) return LR_ERR_INVALID_ARG;
@@ -28,7 +61,7 @@ lr_status validate_desc(const lr_cache_desc* d) {
   if (d->rope_in_kernel && !(d->rope_theta > 0.0)) return LR_ERR_INVALID_ARG;
   if (d->rope_in_kernel && d->window > 0) return LR_ERR_UNSUPPORTED;
   if (!(d->softmax_scale >= 0.0f) || std::isinf(d->softmax_scale)) return LR_ERR_INVALID_ARG;
-  for (int i = 0; i < 5; ++i)
+  for (int i = 0; i < 4; ++i)
     if (d->reserved[i] != 0) return LR_ERR_INVALID_ARG;
   if ((long long)d->n_kv_heads * d->head_dim > 4096) return LR_ERR_UNSUPPORTED;
   if (d->n_q_heads > 128 || d->n_q_heads / d->n_kv_heads > 64) return LR_ERR_UNSUPPORTED;
@@ -80,7 +113,7 @@ template <typename T>
 cudaError_t dalloc(T** p, size_t bytes) {
   *p = nullptr;
   if (bytes == 0) return cudaSuccess;
-  cudaError_t e = cudaMalloc((void**)p, bytes);
+  cudaError_t e = lr_dev_malloc((void**)p, bytes);
   if (e != cudaSuccess) return e;
   return cudaMemset(*p, 0, bytes);
 }
@@ -91,7 +124,7 @@ void free_all(lr_cache* c) {
   sync_tc_release(c);
   void* ptrs[] = {c->z_k, c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->win_k, c->win_v,
                   c->A_k, c->B_k, c->A_v, c->B_v, c->rope_cs, c->qt, c->qt16, c->part_o, c->part_ml,
-                  c->win_o, c->win_ml, c->dev_err};
+                  c->win_o, c->win_ml, c->dev_err, c->r_full};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -106,6 +139,29 @@ cudaError_t record_event(cudaEvent_t ev, cudaStream_t s) {
   return cudaEventRecord(ev, s);
 }
 
+// dst [g rows][g cols] (zero outside the blocks) <- the g diagonal blocks src [g][rows][cols],
+// elements of `es` bytes.
+cudaError_t expand_blockdiag(void* dst, const void* src, int g, size_t rows, size_t cols, size_t es,
+                             cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < g && e == cudaSuccess; ++i)
+    e = cudaMemcpy2DAsync(static_cast<char*>(dst) + (i * rows * g * cols + i * cols) * es, g * cols * es,
+                          static_cast<const char*>(src) + i * rows * cols * es, cols * es, cols * es, rows,
+                          cudaMemcpyDeviceToDevice, s);
+  return e;
+}
+
+// Copy a caller's basis into the cache: A [D][r] / B [r][D] as they are, or, with latent
+// groups, the per-group blocks A [g][D/g][r/g] / B [g][r/g][D/g] onto the diagonal of the
+// block-diagonal basis (its other entries stay zero from the allocation).
+cudaError_t install_basis(lr_cache* c, void* dst, const void* src, bool is_A, bool is_k, cudaStream_t s) {
+  const lr_cache_desc& d = c->desc;
+  const size_t r = is_k ? d.rank_k : d.rank_v, D = c->D, es = c->esize;
+  const int g = c->groups;
+  if (g == 1) return cudaMemcpyAsync(dst, src, r * D * es, cudaMemcpyDeviceToDevice, s);
+  return is_A ? expand_blockdiag(dst, src, g, D / g, r / g, es, s) : expand_blockdiag(dst, src, g, r / g, D / g, es, s);
+}
+
 lr_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return LR_OK;
   if (e == cudaErrorMemoryAllocation) return LR_ERR_OOM;
@@ -115,6 +171,8 @@ lr_status cuda_status(cudaError_t e) {
 }  // namespace
 
 void lr_count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+bool lr_fault_alloc() { return fault_fires(0); }
+bool lr_fault_launch() { return fault_fires(1); }
 
 extern "C" {
 
@@ -140,7 +198,8 @@ lr_status lr_plan_decode(const lr_cache_desc* desc, int32_t len, int32_t num_sms
   if (!out || len < 0 || len > desc->capacity || num_sms < 1) return LR_ERR_INVALID_ARG;
   if (path < 0 || path > 2 || n_splits < 0) return LR_ERR_INVALID_ARG;
   const int hist = desc->window > 0 ? std::max(0, len - desc->window) : len;
-  return plan(desc, hist, num_sms, path, n_splits, out);
+  const lr_cache_desc e = effective_desc(desc);
+  return plan(&e, hist, num_sms, path, n_splits, out);
 }
 
 lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void* B_k, const void* A_v,
@@ -154,7 +213,8 @@ lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void
 
   lr_cache* c = new (std::nothrow) lr_cache();
   if (!c) return LR_ERR_OOM;
-  c->desc = *desc;
+  c->desc = effective_desc(desc);
+  c->groups = groups_of(desc);
   const lr_cache_desc& d = c->desc;
   c->D = d.n_kv_heads * d.head_dim;
   c->esize = d.dtype == LR_BF16 ? 2 : 4;
@@ -203,22 +263,23 @@ lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void
   if (e == cudaSuccess) e = dalloc(&c->dev_err, sizeof(int));
   if (e == cudaSuccess && d.rope_in_kernel) {
     const int half = d.head_dim / 2;
-    std::vector<float2> cs((size_t)cap * half);
+    const size_t cap128 = (cap + 127) / 128 * 128;
+    std::vector<float2> cs(cap128 * half);
     std::vector<double> omega(half);
     for (int i = 0; i < half; ++i) omega[i] = std::pow(d.rope_theta, -2.0 * i / d.head_dim);
-    for (size_t t = 0; t < cap; ++t)
+    for (size_t t = 0; t < cap128; ++t)
       for (int i = 0; i < half; ++i) {
         const double ang = (double)t * omega[i];
-        cs[t * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+        cs[rope_cs_index((long long)t, i, half)] = make_float2((float)std::cos(ang), (float)std::sin(ang));
       }
     e = dalloc(&c->rope_cs, cs.size() * sizeof(float2));
     if (e == cudaSuccess) e = cudaMemcpy(c->rope_cs, cs.data(), cs.size() * sizeof(float2), cudaMemcpyHostToDevice);
   }
   cudaStream_t s = (cudaStream_t)stream;
-  if (e == cudaSuccess) e = cudaMemcpyAsync(c->B_k, B_k, (size_t)d.rank_k * D * es, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(c->B_v, B_v, (size_t)d.rank_v * D * es, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess && A_k) e = cudaMemcpyAsync(c->A_k, A_k, D * d.rank_k * es, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess && A_v) e = cudaMemcpyAsync(c->A_v, A_v, D * d.rank_v * es, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = install_basis(c, c->B_k, B_k, false, true, s);
+  if (e == cudaSuccess) e = install_basis(c, c->B_v, B_v, false, false, s);
+  if (e == cudaSuccess && A_k) e = install_basis(c, c->A_k, A_k, true, true, s);
+  if (e == cudaSuccess && A_v) e = install_basis(c, c->A_v, A_v, true, false, s);
   c->has_A = A_k != nullptr;
   if (e == cudaSuccess && tc_supported(&d)) e = tc_prepare(c, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -325,6 +386,59 @@ lr_status lr_attn_decode(lr_cache* c, const void* q, void* out, float* lse, void
   return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
 }
 
+lr_status lr_attn_decode_partial(lr_cache* c, const void* q, float* part_o, float* part_ml, void* stream) {
+  if (!c || !q || !part_o || !part_ml) return LR_ERR_INVALID_ARG;
+  if (c->win_slots || c->desc.rope_in_kernel) return LR_ERR_UNSUPPORTED;
+  if (c->len == 0) return LR_ERR_INVALID_ARG;
+  lr_plan p;
+  lr_status st = decode_plan(c, c->hist_len, &p);
+  if (st != LR_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  c->stable_len = c->hist_len;
+  cudaError_t e = p.path == LR_PATH_TC ? launch_qproj_tc(c, q, s) : launch_qproj(c, q, s);
+  if (e == cudaSuccess && c->ev_start) e = record_event(c->ev_start, s);
+  if (e == cudaSuccess)
+    e = p.path == LR_PATH_TC ? launch_decode_tc(c, p.n_splits, p.split_tokens, s)
+                             : launch_decode_simt(c, p.n_splits, p.split_tokens, s);
+  if (e == cudaSuccess && c->ev_stop) e = record_event(c->ev_stop, s);
+  if (e == cudaSuccess) {
+    MergeSource src{c->part_o, c->part_ml, p.n_splits, 1, part_o, part_ml};
+    e = launch_merge(c, p.n_splits, nullptr, nullptr, s, &src);
+  }
+  return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
+}
+
+lr_status lr_merge_partials(lr_cache* c, int32_t n, const float* part_o, const float* part_ml, void* out,
+                            float* lse, void* stream) {
+  if (!c || !part_o || !part_ml || !out || n < 1) return LR_ERR_INVALID_ARG;
+  if (c->win_slots || c->desc.rope_in_kernel) return LR_ERR_UNSUPPORTED;
+  if (n > c->S_max) return LR_ERR_CAPACITY;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  MergeSource src{part_o, part_ml, 1, c->desc.batch, nullptr, nullptr};
+  cudaError_t e = launch_merge(c, n, out, lse, s, &src);
+  return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
+}
+
+lr_status lr_attn_decode_varlen(lr_cache* c, const void* q, void* out, float* lse, const int32_t* row_len,
+                                void* stream) {
+  if (!c || !q || !out || !row_len) return LR_ERR_INVALID_ARG;
+  if (c->win_slots) return LR_ERR_UNSUPPORTED;
+  if (c->len == 0) return LR_ERR_INVALID_ARG;
+  lr_plan p;
+  lr_status st = decode_plan(c, c->hist_len, &p);
+  if (st != LR_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  c->stable_len = c->hist_len;
+  c->row_len = row_len;
+  cudaError_t e = p.path == LR_PATH_TC ? launch_qproj_tc(c, q, s) : launch_qproj(c, q, s);
+  if (e == cudaSuccess) e = decode_rest(c, p, out, lse, s);
+  c->row_len = nullptr;
+  return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
+}
+
 lr_status lr_decode_step(lr_cache* c, const void* k, const void* v, const void* q, void* out, float* lse,
                          void* stream) {
   if (!c || !k || !v || !q || !out || !c->has_A) return LR_ERR_INVALID_ARG;
@@ -360,19 +474,37 @@ lr_status lr_basis_sync(lr_cache* c, const float* R_k, const float* R_v, const v
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
   const lr_cache_desc& d = c->desc;
-  const size_t es = c->esize, D = c->D;
   cudaError_t e = cudaSuccess;
+  if (c->groups > 1 && (R_k || R_v)) {
+    // per-group rotations onto the diagonal of one block-diagonal rotation per side
+    const size_t rk = d.rank_k, rv = d.rank_v;
+    if (!c->r_full) {
+      e = lr_dev_malloc(&c->r_full, (rk * rk + rv * rv) * sizeof(float));
+      if (e == cudaSuccess) e = cudaMemsetAsync(c->r_full, 0, (rk * rk + rv * rv) * sizeof(float), s);
+      if (e != cudaSuccess) {
+        if (c->r_full) cudaFree(c->r_full);
+        c->r_full = nullptr;
+        return cuda_status(e);
+      }
+    }
+    const int g = c->groups;
+    if (R_k) e = expand_blockdiag(c->r_full, R_k, g, rk / g, rk / g, sizeof(float), s);
+    if (e == cudaSuccess && R_v) e = expand_blockdiag(c->r_full + rk * rk, R_v, g, rv / g, rv / g, sizeof(float), s);
+    if (e != cudaSuccess) return LR_ERR_CUDA;
+    R_k = R_k ? c->r_full : nullptr;
+    R_v = R_v ? c->r_full + rk * rk : nullptr;
+  }
   if ((R_k || R_v) && sync_tc_supported(&d) && c->path_force != LR_PATH_SIMT) {
     e = launch_sync_tc(c, R_k, R_v, s);
   } else {
     if (R_k) e = launch_sync_simt(c, R_k, 0, s);
     if (e == cudaSuccess && R_v) e = launch_sync_simt(c, R_v, 1, s);
   }
-  if (e == cudaSuccess && B_k_new) e = cudaMemcpyAsync(c->B_k, B_k_new, (size_t)d.rank_k * D * es, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess && B_v_new) e = cudaMemcpyAsync(c->B_v, B_v_new, (size_t)d.rank_v * D * es, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && B_k_new) e = install_basis(c, c->B_k, B_k_new, false, true, s);
+  if (e == cudaSuccess && B_v_new) e = install_basis(c, c->B_v, B_v_new, false, false, s);
   if (A_k_new || A_v_new) c->has_A = true;
-  if (e == cudaSuccess && A_k_new) e = cudaMemcpyAsync(c->A_k, A_k_new, D * d.rank_k * es, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess && A_v_new) e = cudaMemcpyAsync(c->A_v, A_v_new, D * d.rank_v * es, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && A_k_new) e = install_basis(c, c->A_k, A_k_new, true, true, s);
+  if (e == cudaSuccess && A_v_new) e = install_basis(c, c->A_v, A_v_new, true, false, s);
   if (e == cudaSuccess && (B_k_new || B_v_new)) e = tc_prepare(c, s);
   return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
 }
@@ -435,8 +567,10 @@ lr_status lr_cache_set_kernel_events(lr_cache* c, void* ev_start, void* ev_stop)
 
 lr_status lr_cache_set_trace(lr_cache* c, uint64_t* buf, int64_t capacity_words) {
   if (!c) return LR_ERR_INVALID_ARG;
-  if (buf && capacity_words < (int64_t)LR_TRACE_SLOTS * c->desc.batch * c->S_max) return LR_ERR_CAPACITY;
+  const int64_t cta_words = (int64_t)LR_TRACE_SLOTS * c->desc.batch * c->S_max;
+  if (buf && capacity_words < cta_words + LR_TRACE_SPAN_WORDS) return LR_ERR_CAPACITY;
   c->trace = reinterpret_cast<unsigned long long*>(buf);
+  c->spans = buf ? c->trace + cta_words : nullptr;
   return LR_OK;
 }
 
@@ -444,6 +578,19 @@ void lr_abi_struct_sizes(int32_t* desc_size, int32_t* view_size, int32_t* plan_s
   if (desc_size) *desc_size = (int32_t)sizeof(lr_cache_desc);
   if (view_size) *view_size = (int32_t)sizeof(lr_cache_view);
   if (plan_size) *plan_size = (int32_t)sizeof(lr_plan);
+}
+
+lr_status lr_debug_inject_fault(int32_t kind, int64_t after) {
+  if (kind != LR_FAULT_ALLOC && kind != LR_FAULT_LAUNCH) return LR_ERR_INVALID_ARG;
+  if (after < -1) return LR_ERR_INVALID_ARG;
+  g_fault_left[kind].store(after);
+  return LR_OK;
+}
+
+lr_status lr_cache_set_wait_limit(lr_cache* c, int64_t ns) {
+  if (!c || ns < 0) return LR_ERR_INVALID_ARG;
+  c->wait_ns = (unsigned long long)ns;
+  return LR_OK;
 }
 
 lr_status lr_device_error(lr_cache* c, int32_t* code) {

@@ -27,6 +27,32 @@ __host__ __device__ __forceinline__ long long i4_code_index(long long row, int G
 __host__ __device__ __forceinline__ long long i4_param_index(long long row, int G, int g) {
   return (((row >> 7) * G + g) << 7) + (row & 127);
 }
+// Values (V) are stored rank-major inside a block, so that the decode's value-mix operand
+// (rank rows, token columns) is read one rank row per thread: rank i of a block holds 16
+// words, each with eight tokens' codes; the 16-byte column c of the row holds tokens
+// 32 (c ^ ((i / 2) % 4)) .. +31 (the XOR spreads the rows of consecutive ranks over the
+// shared-memory banks), and token t sits in nibble ((t & 1) << 2) | ((t >> 1) & 3) of its
+// word, so that the two nibbles (m, m + 4) of a word are two consecutive tokens.  The
+// params of one (block, group) are 128 fp16 scales (tokens 0..127) then 128 fp16 zeros.
+__host__ __device__ __forceinline__ long long i4v_code_index(long long row, int G, int i) {
+  const int t = (int)(row & 127);
+  return ((((row >> 7) * G) << 5) + i) * 16 + ((((t >> 5) ^ ((i >> 1) & 3))) << 2) + ((t & 31) >> 3);
+}
+__host__ __device__ __forceinline__ int i4v_nibble(long long row) {
+  const int t = (int)(row & 127);
+  return ((t & 1) << 2) | ((t >> 1) & 3);
+}
+// index of the fp16 scale of token `row` in group g (the zero is 128 halves further on)
+__host__ __device__ __forceinline__ long long i4v_scale_index(long long row, int G, int g) {
+  return (((row >> 7) * G + g) << 8) + (row & 127);
+}
+
+// RoPE factors (cos, sin) of position t and frequency pair i (of d/2), fp32 from fp64
+// angles, stored in 128-token tiles, pair-major inside a tile: the 128 tokens of one pair are
+// contiguous, so threads that own consecutive tokens read one coalesced run per pair.
+__host__ __device__ __forceinline__ long long rope_cs_index(long long t, int i, int half) {
+  return (((t >> 7) * half + i) << 7) + (t & 127);
+}
 
 struct lr_cache {
   lr_cache_desc desc;
@@ -35,6 +61,8 @@ struct lr_cache {
   int win_slots;         // window + 1 (ring), or 0
   long long lat_cap;     // latent rows per sequence: capacity (int4: rounded up to 128)
   int32_t len, hist_len, win_len;
+  int groups = 1;         // latent groups (desc ranks are the block-diagonal total g r)
+  float* r_full = nullptr; // block-diagonal sync rotations (latent groups), [r_k^2 + r_v^2]
   int undo = 0;           // windowed caches: 0 = no undo, 1 = the last append only filled
                           // the window, 2 = it folded the oldest window token into history
   int32_t stable_len = 0; // history rows [0, stable_len) were written before the kernel that
@@ -50,7 +78,7 @@ struct lr_cache {
   uint32_t* params_k = nullptr; uint32_t* params_v = nullptr;
   void* win_k = nullptr; void* win_v = nullptr;
   void* A_k = nullptr; void* B_k = nullptr; void* A_v = nullptr; void* B_v = nullptr;
-  float2* rope_cs = nullptr;   // [capacity][head_dim/2] (cos, sin), fp32 from fp64 angles
+  float2* rope_cs = nullptr;   // (cos, sin) per (position, pair), rope_cs_index; fp32 from fp64 angles
 
   // scratch
   float* qt = nullptr;         // [B][Hq][r_k] fp32 scaled query latents (or [B][Hq][d] for RoPE)
@@ -60,6 +88,8 @@ struct lr_cache {
   float* win_o = nullptr;      // [B][Hq][d]
   float* win_ml = nullptr;     // [B][Hq][2]
   int* dev_err = nullptr;      // device error word
+  unsigned long long wait_ns = 0;   // bounded-wait limit of the tensor-core kernels (0: default)
+  const int32_t* row_len = nullptr; // per-row history lengths of the decode in flight (device), or null
   int S_max = 1;
 
   bool has_A = false;         // projections given at creation (needed by lr_kv_append)
@@ -71,15 +101,17 @@ struct lr_cache {
   void* sync_state = nullptr;  // tensor-core basis sync state (tensor maps, split R), owned
   cudaEvent_t ev_start = nullptr, ev_stop = nullptr;   // caller-owned kernel timing events
   unsigned long long* trace = nullptr;                 // caller-owned decode timeline buffer
+  unsigned long long* spans = nullptr;                 // its kernel spans (SPAN_KINDS pairs), or null
 };
 
 // ---- argument blocks --------------------------------------------------------
 
 struct LatentRef {
   const void* z;          // unquantised [B][cap][r]
-  const uint32_t* codes;  // int4, blocked (i4_code_index)
-  const uint32_t* params; // int4, blocked (i4_param_index)
+  const uint32_t* codes;  // int4, blocked (i4_code_index; values: i4v_code_index)
+  const uint32_t* params; // int4, blocked (i4_param_index; values: i4v_scale_index)
   int r, G;
+  int rank_major;         // int4 values: the rank-major block layout
   long long cap;
 };
 
@@ -87,20 +119,38 @@ struct DecodeSimtArgs {
   LatentRef k, v;
   const float* qs;        // [B][Hq][r_k] (latent path) or [B][Hq][d] (RoPE path), pre-scaled
   const void* B_k;        // RoPE path: [r_k][D]
-  const float2* rope_cs;  // RoPE path: [cap][d/2]
+  const float2* rope_cs;  // RoPE path: rope_cs_index layout
   float* part_o;          // [B][S][Hq][r_v]
   float* part_ml;         // [B][S][Hq][2]
   int Hq, Hkv, d, D;
   int hist_len, split_tokens, n_splits;
   int rope;
   int dtype;
+  const int32_t* row_len;  // per-row history lengths (device), or null: every row has hist_len
+  unsigned long long* span;  // timeline span of this kernel, or null
 };
 
+// History tokens row b attends to: its own length, clamped to [1, hist_len], or hist_len.
+__device__ __forceinline__ int row_hist(const int32_t* row_len, int b, int hist_len) {
+  return row_len ? min(max(row_len[b], 1), hist_len) : hist_len;
+}
+
 // ---- launchers (return cudaGetLastError) ------------------------------------
-cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s);
+// pdl = false: launched after the preceding work completes (for bases the caller owns,
+// which the kernel just before may have written)
+cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s, bool pdl = true);
 cudaError_t launch_decode_simt(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s);
 cudaError_t launch_window(const lr_cache* c, cudaStream_t s);
-cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s);
+// Where the merge reads its partials and what it writes: by default the cache's own split
+// partials ([B][S][Hq]) merged and projected to `out`; with a MergeSource, partials at other
+// addresses / strides, and (rs_o set) a rank-space result instead of the projection.
+struct MergeSource {
+  const float* part_o; const float* part_ml;
+  long long b_stride, s_stride;   // head-row blocks: (b, s) at (b * b_stride + s * s_stride) * Hq
+  float* rs_o; float* rs_ml;      // rank-space output [B][Hq][r_v], [B][Hq][2], or null
+};
+cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s,
+                         const MergeSource* src = nullptr);
 cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s);
 // append (with the cache's current counters) and query projection in one grid
 cudaError_t launch_step_pre(lr_cache* c, const void* k, const void* v, const void* q, bool tc, cudaStream_t s);
@@ -133,6 +183,23 @@ void sync_tc_release(lr_cache* c);
 
 void lr_count_launch(int n = 1);
 
+// Host-side fault injection (lr_debug_inject_fault): true when this device allocation or
+// kernel launch is the one armed to fail; the caller then fails without allocating or
+// launching.
+bool lr_fault_alloc();
+bool lr_fault_launch();
+
+// Every device allocation of the library goes through here.
+inline cudaError_t lr_dev_malloc(void** p, size_t bytes) {
+  *p = nullptr;
+  if (lr_fault_alloc()) return cudaErrorMemoryAllocation;
+  return cudaMalloc(p, bytes);
+}
+template <typename T>
+inline cudaError_t lr_dev_malloc(T** p, size_t bytes) {
+  return lr_dev_malloc(reinterpret_cast<void**>(p), bytes);
+}
+
 // Programmatic dependent launch.  Every kernel of the library does its prologue on data
 // no in-flight kernel writes, then pdl_wait() (the preceding grid has completed and its
 // memory is visible), then pdl_trigger() (the next grid may start its own prologue).
@@ -140,6 +207,28 @@ void lr_count_launch(int n = 1);
 // kernel has completed whenever a prologue runs.  Both are no-ops without the attribute.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Kernel spans of the timeline trace (lr_cache_set_trace): for span kind k, word 2k holds
+// the earliest CTA start and word 2k + 1 the latest CTA end of the kernels of that kind, in
+// %globaltimer nanoseconds (the caller initialises the words to ~0 and 0).  A null pointer
+// disables the stamps.  span_end synchronises the block, so every thread must reach it.
+enum SpanKind { SPAN_PRE = 0, SPAN_DECODE = 1, SPAN_WINDOW = 2, SPAN_MERGE = 3, SPAN_KINDS = 4 };
+__device__ __forceinline__ unsigned long long span_now() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void span_begin(unsigned long long* sp) {
+  if (sp && threadIdx.x == 0) atomicMin(sp, span_now());
+}
+__device__ __forceinline__ void span_end(unsigned long long* sp) {
+  if (!sp) return;
+  __syncthreads();
+  if (threadIdx.x == 0) atomicMax(sp + 1, span_now());
+}
+__host__ __device__ __forceinline__ unsigned long long* span_of(unsigned long long* spans, int kind) {
+  return spans ? spans + 2 * kind : nullptr;
+}
 
 // Launch with the programmatic-stream-serialization attribute; returns the launch error.
 template <typename... KArgs, typename... Args>
@@ -155,6 +244,24 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (lr_fault_launch()) return cudaErrorLaunchFailure;
+  lr_count_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Launch without the attribute: the kernel starts only after the preceding work on the
+// stream has completed, so its prologue may read anything that work wrote.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_serial(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                 Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  if (lr_fault_launch()) return cudaErrorLaunchFailure;
   lr_count_launch();
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }

@@ -21,17 +21,22 @@ constexpr int kTraceSlots = LR_TRACE_SLOTS; // 0 start, 1 setup done, 2 query la
                                            // 6+4i: value mix of tile i issued (i < 16), last: end
 constexpr float kLazy = 8.0f;              // log2 of the allowed running-max growth before a rescale
 
+// The wait limit of a launch: the cache's test setting (lr_cache_set_wait_limit), or
+// kTimeoutNs when that is 0.
+__host__ __device__ __forceinline__ uint64_t wait_limit(unsigned long long ns) { return ns ? ns : kTimeoutNs; }
+
 // Wait for phase `parity` of `bar`.  Gives up when another thread of the CTA has
-// aborted, or after kTimeoutNs, in which case it records LR_ERR_TIMEOUT in the device
+// aborted, or after `limit_ns`, in which case it records LR_ERR_TIMEOUT in the device
 // error word and raises the CTA's abort flag.  Returns false when it gave up.
-__device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, int* abort_flag, int* err) {
+__device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, int* abort_flag, int* err,
+                                       uint64_t limit_ns = kTimeoutNs) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if ((it & 31) == 0) {
       if (*(volatile int*)abort_flag) return false;
-      if (ptx::globaltimer() - t0 > kTimeoutNs) {
+      if (ptx::globaltimer() - t0 > limit_ns) {
         *(volatile int*)abort_flag = 1;
         atomicExch(err, (int)LR_ERR_TIMEOUT);
         return false;
@@ -41,7 +46,8 @@ __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, int* abor
 }
 
 // Wait that ignores the abort flag (used to drain in-flight copies and MMAs after an
-// abort); still bounded.
+// abort); still bounded, always by kTimeoutNs (a short test limit applies only to the
+// waits above).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = ptx::globaltimer();
   while (!ptx::mbar_try_wait(bar, parity))

@@ -220,6 +220,24 @@ def _qwen_bases(name: str, seed: int, r_k: int, r_v: int, D: int, dtype: str, la
     return _store(dtype, Ak), _store(dtype, Bk), _store(dtype, Av), _store(dtype, Bv)
 
 
+def grouped_bases(name: str, seed: int, g: int, r: int, D: int, dtype: str = "bf16"):
+    """Per-group bases of a cache with g latent groups of rank r: B_i with Haar orthonormal
+    rows scaled by 1/sqrt(r) over the group's D/g coordinates, A_i = r B_i^T.  Returns the
+    compact forms (A [g][D/g][r], B [g][r][D/g], for K then V) and the block-diagonal
+    B_k, B_v ([g r][D], fp64) they stand for."""
+    Dg = D // g
+    out = []
+    for side in ("k", "v"):
+        rng = rng_for(name, f"B_{side}/groups{g}", seed)
+        Bs = np.stack([haar_orthonormal(rng, r, Dg) / np.sqrt(r) for _ in range(g)])
+        full = np.zeros((g * r, D))
+        for i in range(g):
+            full[i * r:(i + 1) * r, i * Dg:(i + 1) * Dg] = Bs[i]
+        out.append((_store(dtype, r * Bs.transpose(0, 2, 1)), _store(dtype, Bs), full))
+    (Ak, Bk, Bk_full), (Av, Bv, Bv_full) = out
+    return Ak, Bk, Av, Bv, Bk_full, Bv_full
+
+
 def _latents(name: str, tensor: str, seed: int, B: int, T: int, r: int, power: float) -> np.ndarray:
     g = rng_for(name, tensor, seed).standard_normal((B, T, r))
     return (g * spectrum(r, power)[None, None, :]).astype(np.float32)

@@ -48,26 +48,30 @@ def fp16_latent_rope_lse_bound(p: synth.Problem, q: np.ndarray) -> np.ndarray:
     """Worst-case |lse error| [B][Hq] of the keys-before-RoPE decode on tensor cores.  The
     keys are rebuilt from the fp16 roundings of the dequantised int4 latents x^ (error
     <= 2^-11 |x^| + 2^-25 each) and of B_k (bf16 -> fp16: exact above 2^-14, else <= 2^-25),
-    accumulated in fp32, rotated and dotted with the fp32 query; the probabilities are fp16
-    as on the rank-space path.  With |.| the Euclidean norm (a rotation keeps it) and
-    b_i = |B_k,h[i, :]|:
-      |d logit_t| <= s |q_j| [ sum_i (2^-11 |x^_t,i| + 2^-25) b_i + sqrt(d) 2^-25 sum_i |x^_t,i|
-                              + (r + d + 8) 2^-24 sum_i |x^_t,i| b_i ],
+    accumulated in fp32 and rotated with the fp32 table; the rotated keys and the scaled
+    query enter the score MMA as fp16 (each <= 2^-11 relative + 2^-25 absolute per element)
+    with fp32 accumulation; the probabilities are fp16 as on the rank-space path.  With |.|
+    the Euclidean norm (a rotation keeps it), b_i = |B_k,h[i, :]| and
+    K_t = sum_i |x^_t,i| b_i (>= |k^_t|):
+      E_t         = (3 2^-11 + (r + d + 8) 2^-24) K_t + 2^-25 sum_i b_i
+                    + sqrt(d) 2^-25 (sum_i |x^_t,i| + 1),
+      |d logit_t| <= s |q_j| E_t + sqrt(d) 2^-25 K_t,
       |d lse|     <= max_t |d logit_t| + 2^-10."""
     qv = stored_value(p, q)
     Bk = stored_value(p, p.B_k)
     d, G = p.head_dim, p.n_q_heads // p.n_kv_heads
     s = 1.0 / math.sqrt(d)
-    rel = 2.0 ** -11 + (p.rank_k + d + 8) * 2.0 ** -24
+    rel = 3 * 2.0 ** -11 + (p.rank_k + d + 8) * 2.0 ** -24
     out = np.zeros((p.batch, p.n_q_heads))
     for b in range(p.batch):
         X = np.abs(oracle_latents(p, p.z_k[b]))
         sx = X.sum(axis=1)
         for h in range(p.n_kv_heads):
             bn = np.linalg.norm(Bk[:, h * d:(h + 1) * d], axis=1)
-            worst = np.max(rel * (X @ bn) + 2.0 ** -25 * bn.sum() + math.sqrt(d) * 2.0 ** -25 * sx)
+            K = X @ bn
+            E = rel * K + 2.0 ** -25 * bn.sum() + math.sqrt(d) * 2.0 ** -25 * (sx + 1.0)
             for j in range(h * G, (h + 1) * G):
-                out[b, j] = s * np.linalg.norm(qv[b, j]) * worst + 2.0 ** -10
+                out[b, j] = np.max(s * np.linalg.norm(qv[b, j]) * E + math.sqrt(d) * 2.0 ** -25 * K) + 2.0 ** -10
     return out
 
 
@@ -158,16 +162,54 @@ def fill_cache(lr, p: synth.Problem, capacity: Optional[int] = None, chunk: int 
     return c
 
 
+def _value_layout_maps():
+    """For the rank-major value blocks: word index within a rank row [32 ranks mod 8 ...] and
+    nibble of token t, as the header defines them (XOR-rotated 16-byte columns; tokens
+    2m, 2m+1 in nibbles m, m + 4)."""
+    i = np.arange(256)[:, None]           # rank (only i // 2 % 4 matters)
+    t = np.arange(128)[None, :]
+    widx = (((t >> 5) ^ ((i >> 1) & 3)) << 2) + ((t & 31) >> 3)
+    nib = ((t & 1) << 2) | ((t >> 1) & 3)
+    return widx, nib[0]
+
+
 def int4_token_major(lr, view, batch: int, which: str):
     """Copy a cache's int4 storage of K ("k") or V ("v") to the host and rearrange it from
-    the blocked device layout ([B][blocks][G][128][4] codes, [B][blocks][G][128] params)
-    to token-major ([B][tokens][G*4], [B][tokens][G]), the layout of the oracle's packer."""
+    the blocked device layout to token-major ([B][tokens][G*4] code words, [B][tokens][G]
+    {scale, zero} words), the layout of the oracle's packer.  Keys: [B][blocks][G][128][4]
+    codes and [B][blocks][G][128] params.  Values: rank-major blocks [B][blocks][G*32][16]
+    and per (block, group) 128 fp16 scales then 128 fp16 zeros."""
     nb = view.int4_blocks
-    G = view.groups_k if which == "k" else view.groups_v
-    codes = lr.copy_view(view.codes_k if which == "k" else view.codes_v, (batch, nb, G, 128, 4), "<i4")
-    params = lr.copy_view(view.params_k if which == "k" else view.params_v, (batch, nb, G, 128), "<i4")
-    c = codes.cpu().numpy().view(np.uint32).transpose(0, 1, 3, 2, 4).reshape(batch, nb * 128, G * 4)
-    pr = params.cpu().numpy().view(np.uint32).transpose(0, 1, 3, 2).reshape(batch, nb * 128, G)
+    if which == "k":
+        G = view.groups_k
+        codes = lr.copy_view(view.codes_k, (batch, nb, G, 128, 4), "<i4")
+        params = lr.copy_view(view.params_k, (batch, nb, G, 128), "<i4")
+        c = codes.cpu().numpy().view(np.uint32).transpose(0, 1, 3, 2, 4).reshape(batch, nb * 128, G * 4)
+        pr = params.cpu().numpy().view(np.uint32).transpose(0, 1, 3, 2).reshape(batch, nb * 128, G)
+        return c, pr
+    G = view.groups_v
+    raw = lr.copy_view(view.codes_v, (batch, nb, G * 32, 16), "<i4").cpu().numpy().view(np.uint32)
+    halves = lr.copy_view(view.params_v, (batch, nb, G, 128), "<i4").cpu().numpy().view(np.uint16)
+    return value_blocks_to_token_major(raw, halves.reshape(batch, nb, G, 256))
+
+
+def value_blocks_to_token_major(raw: np.ndarray, halves: np.ndarray):
+    """raw [B][nb][G*32][16] u32 rank-major code rows, halves [B][nb][G][256] u16 (scales,
+    then zeros) -> token-major code words [B][nb*128][G*4] and params [B][nb*128][G]."""
+    batch, nb, R, _ = raw.shape
+    G = R // 32
+    widx, nib = _value_layout_maps()
+    i_idx = np.arange(G * 32)[:, None]
+    words = raw[:, :, i_idx, widx[(np.arange(G * 32) % 8)][:, :]]      # [B][nb][G*32][128]
+    codes = (words >> (4 * nib[None, None, None, :]).astype(np.uint32)) & 15
+    # token-major packing: element e of group g at word g*4 + e//8, nibble e%8
+    codes = codes.transpose(0, 1, 3, 2).reshape(batch, nb * 128, G * 4, 8)
+    c = np.zeros((batch, nb * 128, G * 4), np.uint32)
+    for m in range(8):
+        c |= codes[..., m].astype(np.uint32) << np.uint32(4 * m)
+    sc = halves[..., :128].astype(np.uint32)
+    zr = halves[..., 128:].astype(np.uint32)
+    pr = (sc | (zr << 16)).transpose(0, 1, 3, 2).reshape(batch, nb * 128, G)
     return c, pr
 
 

@@ -119,11 +119,23 @@ def test_plan_keys_before_rope_int4_on_kv_head_pairs(lib, n_kv_heads, pairs, ran
     assert (p.n_splits - 1) * p.split_tokens < 32768 <= p.n_splits * p.split_tokens
 
 
-@pytest.mark.parametrize("shape", [dict(head_dim=64), dict(n_q_heads=16, n_kv_heads=4),
-                                   dict(n_q_heads=7, n_kv_heads=1), dict(n_q_heads=21, n_kv_heads=3)])
+@pytest.mark.parametrize("shape", [dict(n_q_heads=16, n_kv_heads=4), dict(n_q_heads=7, n_kv_heads=1),
+                                   dict(n_q_heads=21, n_kv_heads=3), dict(n_q_heads=64, n_kv_heads=4)])
+def test_plan_keys_before_rope_on_tensor_cores_for_head_groups_up_to_16(lib, shape):
+    """The tensor-core keys-before-RoPE variant takes d = 128 with up to 16 query heads per
+    KV head (the score MMA's N), one CTA per pair of KV heads, or per KV head when their
+    number is odd."""
+    d = _qwen(lib, quant_bits=4, rope_in_kernel=1, **shape)
+    p = lib.lr_plan_decode(d, 4096, 148)
+    assert p.path == lib.LR_PATH_TC
+    per = 2 if shape["n_kv_heads"] % 2 == 0 else 1
+    assert p.ctas == p.n_splits * d.batch * (shape["n_kv_heads"] // per)
+
+
+@pytest.mark.parametrize("shape", [dict(head_dim=64), dict(n_q_heads=20, n_kv_heads=1),
+                                   dict(n_q_heads=68, n_kv_heads=2)])
 def test_plan_keys_before_rope_other_shapes_use_cuda_cores(lib, shape):
-    """The tensor-core keys-before-RoPE variant exists for d = 128, seven query heads per KV
-    head and KV heads in pairs; every other shape decodes on CUDA cores."""
+    """Other head dimensions, and more than 16 query heads per KV head, decode on CUDA cores."""
     d = _qwen(lib, quant_bits=4, rope_in_kernel=1, **shape)
     assert lib.lr_plan_decode(d, 4096, 148).path == lib.LR_PATH_SIMT
 
@@ -136,3 +148,31 @@ def test_plan_forced_splits_and_window(lib):
     p = lib.lr_plan_decode(dw, 32768, 148, 1)
     assert p.n_splits * p.split_tokens >= 32768 - 128
     assert (p.n_splits - 1) * p.split_tokens < 32768 - 128
+
+
+def test_fault_injection_arguments(lib):
+    """Arming and disarming the host fault injection is host-only bookkeeping."""
+    assert lib.raw_status("lr_debug_inject_fault", 2, 0) == lib.LR_ERR_INVALID_ARG
+    assert lib.raw_status("lr_debug_inject_fault", lib.LR_FAULT_ALLOC, -2) == lib.LR_ERR_INVALID_ARG
+    for kind in (lib.LR_FAULT_ALLOC, lib.LR_FAULT_LAUNCH):
+        assert lib.raw_status("lr_debug_inject_fault", kind, 3) == lib.LR_OK
+        assert lib.raw_status("lr_debug_inject_fault", kind, -1) == lib.LR_OK
+
+
+def test_wait_limit_rejects_bad_arguments(lib):
+    assert lib.raw_status("lr_cache_set_wait_limit", None, 10) == lib.LR_ERR_INVALID_ARG
+
+
+def test_latent_groups_validation_and_plan(lib):
+    """Latent groups must divide the KV heads, and the ranks they add up to stay within the
+    512 limit; the plan is that of the block-diagonal cache of rank g * r."""
+    def status(**kw):
+        d = _qwen(lib, **kw)
+        return lib.raw_status("lr_plan_decode", ctypes.byref(d), 4096, 148, 0, 0, ctypes.byref(lib.lr_plan()))
+    assert status(latent_groups=3) == lib.LR_ERR_INVALID_ARG            # 4 KV heads
+    assert status(latent_groups=-1) == lib.LR_ERR_INVALID_ARG
+    assert status(latent_groups=4, rank_k=160, rank_v=64) == lib.LR_ERR_INVALID_ARG   # 640 > 512
+    assert status(latent_groups=4, rank_k=64, rank_v=64) == lib.LR_OK
+    grouped = lib.lr_plan_decode(_qwen(lib, latent_groups=4, rank_k=64, rank_v=64), 4096, 148)
+    shared = lib.lr_plan_decode(_qwen(lib, rank_k=256, rank_v=256), 4096, 148)
+    assert (grouped.path, grouped.n_splits, grouped.ctas) == (shared.path, shared.n_splits, shared.ctas)

@@ -57,7 +57,8 @@ def _emulate_rank_space(p: synth.Problem, q: np.ndarray, head_shift: int = 0) ->
 
 def _emulate_rope(p: synth.Problem, q: np.ndarray, sin_sign: float = 1.0, head_shift: int = 0) -> np.ndarray:
     """int4 latents, keys before RoPE: K^ = fp16(x^) fp16(B_k) in fp32, rotate-half with an
-    fp32 cos / sin table, fp32 dots with the scaled query."""
+    fp32 cos / sin table, the rotated keys and the scaled query rounded to fp16, dots
+    accumulated in fp32."""
     d, Hq, Hkv = p.head_dim, p.n_q_heads, p.n_kv_heads
     G, half = Hq // Hkv, p.head_dim // 2
     B16 = _fp16(H.stored_value(p, p.B_k))
@@ -73,8 +74,8 @@ def _emulate_rope(p: synth.Problem, q: np.ndarray, sin_sign: float = 1.0, head_s
         for j in range(Hq):
             h = (j // G + head_shift) % Hkv
             k1, k2 = K[:, h * d:h * d + half], K[:, h * d + half:(h + 1) * d]
-            kr = np.concatenate([k1 * cos - k2 * sin, k2 * cos + k1 * sin], axis=1)
-            lse[b, j] = _lse_from_log2_logits(kr @ qs[b, j])
+            kr = _fp16(np.concatenate([k1 * cos - k2 * sin, k2 * cos + k1 * sin], axis=1))
+            lse[b, j] = _lse_from_log2_logits(kr @ _fp16(qs[b, j]))
     return lse
 
 

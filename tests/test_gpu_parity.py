@@ -522,3 +522,22 @@ def test_decode_step_equals_append_then_decode(lib, kind):
         torch.cuda.synchronize()
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
         assert lib.lr_cache_get_len(c1) == lib.lr_cache_get_len(c2)
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 2), (12, 3), (16, 1), (28, 4)])
+def test_decode_parity_prerope_head_shapes(lib, hq, hkv):
+    """Keys before RoPE on tensor cores for other group sizes and KV-head counts: pairs of KV
+    heads (Hkv even) or single heads (Hkv odd), up to 16 query heads per KV head (the
+    score MMA's N); against the oracle, with the CUDA-core path alongside."""
+    p = synth.make_qwen("qwen32k", seed=3, batch=2, length=300, rank=192, quant_bits=4, rope=True,
+                        n_q_heads=hq, n_kv_heads=hkv, rank_v=160)
+    c = H.fill_cache(lib, p)
+    assert lib.LR_PATH_TC in paths(lib, p)
+    for q in (p.q, _sharp(p)):
+        ref, ref_lse = H.oracle_decode(p, q)
+        for path in paths(lib, p):
+            lib.lr_cache_set_path(c, path)
+            got, lse = H.gpu_decode(lib, p, c, q)
+            H.compare(p, got, ref, lse, ref_lse, tag=f"prerope Hq={hq} Hkv={hkv} path={path}",
+                      lse_tol=lse_tol_for(lib, p, q, path))
+    lib.lr_cache_destroy(c)
