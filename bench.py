@@ -104,27 +104,31 @@ def r_full_A(B_full, r):
     return r * B_full.T
 
 
-def workload_bytes(workload: str) -> int:
-    """Latent (and exact-window) bytes one step reads, summed over the workload's layers."""
+def workload_bytes(workload: str, layers: int = 0) -> int:
+    """Latent (and exact-window) bytes one step reads, summed over the workload's layers
+    (the first `layers` of them when given)."""
     W = WORKLOADS[workload]
     Bsz, T, qb = W["batch"], W["length"], W["quant_bits"]
     D = W["n_kv_heads"] * W["head_dim"]
     win = W.get("window", 0)
     total = 0
-    for rk, rv in layer_ranks(workload):
+    ranks = layer_ranks(workload)
+    for rk, rv in (ranks[:layers] if layers else ranks):
         per_tok = latent_bytes_per_token(rk, qb) + latent_bytes_per_token(rv, qb)
         total += Bsz * ((T - win) * per_tok + win * 2 * D * 2) if win else Bsz * T * per_tok
     return total
 
 
-def static_config(workload: str, world: int) -> dict:
+def static_config(workload: str, world: int, layers: int = 0) -> dict:
     """The `config` object of a bench line: the workload alone, identical for both arms."""
     W = WORKLOADS[workload]
     ranks = layer_ranks(workload)
+    if layers:
+        ranks = ranks[:layers]
     return {"workload": W["desc"], "name": workload, "batch": W["batch"], "context": W["length"],
             "layers": len(ranks),
             "ranks": sorted({r for rr in ranks for r in rr}) if len(ranks) > 1 else ranks[0][0],
-            "quant_bits": W["quant_bits"], "latent_bytes_per_step": workload_bytes(workload),
+            "quant_bits": W["quant_bits"], "latent_bytes_per_step": workload_bytes(workload, layers),
             "step": "lr_decode_step (= lr_kv_append + lr_attn_decode) per layer",
             "l2": "flushed before every timed step outside the events (256 MiB written, then read back "
                   "so L2 holds clean unrelated lines)",
@@ -309,7 +313,10 @@ def run_workload(args, workload):
     layers = []
     host_p = None
     win = W.get("window", 0)
-    for li, (rk, rv) in enumerate(layer_ranks(workload)):
+    ranks = layer_ranks(workload)
+    if args.layers:
+        ranks = ranks[:args.layers]
+    for li, (rk, rv) in enumerate(ranks):
         hist = T - 1
         if win:
             hist = T - win
@@ -538,14 +545,14 @@ def run_workload(args, workload):
     # HBM; fp16 operands run at the bf16 rate, and the kernel runs inside a long step
     # (sustained peak).
     roof_flops = sum(Bsz * T * (2 * L["rk"] * D + 2 * L["rv"] * Hq) for L in layers) if rope else 0.0
-    assert bytes_per_step == workload_bytes(workload)
+    assert bytes_per_step == workload_bytes(workload, len(layers))
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
         "us_per_step": round(1000 * total_ms / K, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int4+bf16" if qb else "bf16",
         "data": "synthetic (seeded; one seed per rank)",
-        "config": static_config(workload, world),
+        "config": static_config(workload, world, args.layers),
         "run": {"decode_path": "tcgen05" if plan.path == lr.LR_PATH_TC else "simt",
                 "splits": plan.n_splits, "cuda_graph": bool(args.graph),
                 "launches_per_step": launches_per_step},
@@ -690,7 +697,7 @@ def run_reference_workload(args, workload, world):
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(us_step / 1000, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": static_config(workload, world),
+           "config": static_config(workload, world, args.layers),
            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                             "sample": "each step: repeated oracle decodes of batch row 0 (all heads) for a "
                                       f"bounded {per:.1f} s; value = latent bytes processed per second"},
@@ -707,6 +714,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="all", choices=["all"] + sorted(WORKLOADS),
                     help="one workload, or all of them (one line each, the 32K rank-space headline last)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="only the first N layers of a multi-layer workload (profiling runs; 0 = all)")
     ap.add_argument("--load-seconds", type=float, default=1.5)
     ap.add_argument("--cpu-seconds", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

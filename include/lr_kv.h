@@ -156,6 +156,16 @@ lr_status lr_cache_destroy(lr_cache* cache);
  *   LR_ERR_CAPACITY when len == capacity. */
 lr_status lr_kv_append(lr_cache* cache, const void* k, const void* v, void* stream);
 
+/* lr_kv_prefill — append n tokens per sequence from their exact keys and values (a prompt).
+ *   k, v: [B][n][D] in dtype, 16-byte aligned (else LR_ERR_INVALID_ARG).  Each token's latents
+ *   z = k A_k, z_v = v A_v are computed in fp32 and stored at slots len .. len + n - 1
+ *   (rounded to dtype, or int4-quantised), as n calls of lr_kv_append would store them up to
+ *   the summation order of the fp32 projection.  bf16 caches with D a multiple of 64 compute
+ *   the projection as one tensor-core GEMM per 128-token tile; others append token by token
+ *   on CUDA cores.  Caches with a window return LR_ERR_UNSUPPORTED; LR_ERR_CAPACITY when
+ *   len + n > capacity. */
+lr_status lr_kv_prefill(lr_cache* cache, const void* k, const void* v, int32_t n, void* stream);
+
 /* lr_kv_append_latent — bulk fill of n history tokens from given latents.
  *   z_k [B][n][r_k], z_v [B][n][r_v] fp32, device.  Stored rounded to dtype or
  *   int4-quantised (group 32, fp16 scale/zero; reading stated in the oracle).

@@ -11,7 +11,8 @@ lr_kv_append_latent, lr_attn_decode, lr_basis_sync, lr_cache_get_len,
 lr_cache_truncate, lr_cache_view_get, lr_cache_set_path, lr_cache_plan,
 lr_plan_decode, lr_cache_set_kernel_events, lr_cache_set_trace, lr_device_error, lr_abi_struct_sizes,
 lr_status_string, lr_launch_count, lr_attn_decode_noalloc, lr_cache_set_wait_limit,
-lr_debug_inject_fault, lr_attn_decode_varlen, lr_attn_decode_partial, lr_merge_partials.
+lr_debug_inject_fault, lr_attn_decode_varlen, lr_attn_decode_partial, lr_merge_partials,
+lr_kv_prefill.
 """
 from __future__ import annotations
 
@@ -88,6 +89,7 @@ def _load() -> ctypes.CDLL:
         "lr_cache_set_wait_limit": [vp, ctypes.c_int64],
         "lr_attn_decode_varlen": [vp, vp, vp, vp, vp, vp],
         "lr_attn_decode_partial": [vp, vp, vp, vp, vp],
+        "lr_kv_prefill": [vp, vp, vp, i32, vp],
         "lr_merge_partials": [vp, i32, vp, vp, vp, vp, vp],
         "lr_debug_inject_fault": [i32, ctypes.c_int64],
         "lr_attn_decode_noalloc": [ctypes.POINTER(lr_cache_desc), i32, vp, vp, vp, vp, vp, vp, vp, vp],
@@ -219,6 +221,14 @@ def lr_kv_append(cache: Cache, k, v, stream=None) -> None:
     d, dt = cache.desc, _torch_dtype(cache.desc.dtype)
     _check(_lib.lr_kv_append(cache.handle, _ptr(k, dt, (d.batch, cache.D), "k"),
                              _ptr(v, dt, (d.batch, cache.D), "v"), _stream(stream)), "lr_kv_append")
+
+
+def lr_kv_prefill(cache: Cache, k, v, stream=None) -> None:
+    """k, v: CUDA tensors [batch][n][D] in the cache dtype."""
+    d, dt = cache.desc, _torch_dtype(cache.desc.dtype)
+    n = k.shape[1] if k.dim() == 3 else -1
+    _check(_lib.lr_kv_prefill(cache.handle, _ptr(k, dt, (d.batch, n, cache.D), "k"),
+                              _ptr(v, dt, (d.batch, n, cache.D), "v"), n, _stream(stream)), "lr_kv_prefill")
 
 
 def lr_kv_append_latent(cache: Cache, z_k, z_v, stream=None) -> None:

@@ -276,21 +276,23 @@ __global__ void __launch_bounds__(256) k_step_pre(AppendArgs aa, QprojArgs qa, i
 }
 
 // ---- split merge and output projection ------------------------------------------
-// One CTA per (32-column block of the head dimension, KV head h, sequence b), 256
-// threads.  Its columns of B_v,h ([r_v][32], no in-flight kernel writes them) are
-// staged before the grid-dependency wait and reused by every query head of the group.
-// Query heads go through in passes of up to 8: the split weights (log-sum-exp over the
-// splits and the window partial; one warp per head), the combined rank-space output
-// o~_j = sum_s w_s o~_s,j (thread = rank), and o_j = o~_j B_v,h / l_j (thread = 4
-// columns x head x quarter of the ranks, quarters added in a fixed order).
-constexpr int kMergeThreads = 256;
-constexpr int kMergeCols = 32;     // output columns per CTA
-constexpr int kMergeHeads = 8;     // query heads per pass
+// One CTA per (column block of the head dimension, KV head h, sequence b), 512 threads; the
+// column block is the whole head dimension whenever B_v,h fits in shared memory (bf16 up to
+// r_v = 384), so the split partials of a (KV head, sequence) are read once.  Its columns of
+// B_v,h ([r_v][cols], no in-flight kernel writes them) are staged before the grid-dependency
+// wait.  Query heads go through in passes of up to 8: the split weights (log-sum-exp over
+// the splits and the window partial; one warp per head), the combined rank-space outputs
+// o~_j = sum_s w_s o~_s,j (thread = (head, rank) element, each with all its splits' loads in
+// flight), and o_j = o~_j B_v,h / l_j (thread = column x quarter of the ranks, all heads of
+// the pass; quarters added in a fixed order).
+constexpr int kMergeThreads = 512;
+constexpr int kMergeHeads = 8;       // query heads per pass
+constexpr int kMergeBvBytes = 96 * 1024;   // shared-memory budget for the B_v,h columns
 
 struct MergeArgs {
   const float* part_o; const float* part_ml; const float* win_o; const float* win_ml;
   const void* Bv; void* out; float* lse;
-  int S, Hq, Hkv, d, D, rv;
+  int S, Hq, Hkv, d, D, rv, cols;   // cols: output columns per CTA (multiple of 32, or d)
   // partial (b, s) starts at head row (b * b_stride + s * s_stride) * Hq of part_o / part_ml:
   // the cache's [B][S][Hq] has b_stride = S, s_stride = 1; gathered shards [S][B][Hq] have
   // b_stride = 1, s_stride = B
@@ -301,6 +303,12 @@ struct MergeArgs {
   unsigned long long* span;   // timeline span, or null
 };
 
+int merge_cols(int d, int rv, size_t es) {
+  int cols = (int)(kMergeBvBytes / ((size_t)rv * es)) / 32 * 32;
+  cols = std::max(32, cols);
+  return cols >= d ? d : cols;
+}
+
 size_t merge_pitch_f(int rv) { return (size_t)rv + 4; }   // o~ rows, padded against bank conflicts
 
 template <typename T>
@@ -310,21 +318,22 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
   const int cb = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int G = a.Hq / a.Hkv, S = a.S, rv = a.rv;
-  const int c0 = cb * kMergeCols, ncols = min(kMergeCols, a.d - c0);
+  const int c0 = cb * a.cols, ncols = min(a.cols, a.d - c0);
   const int opitch = rv + 4;
-  uint8_t* bs = msm;                                                          // [rv][ncols]
-  float* ot = reinterpret_cast<float*>(msm + (size_t)rv * kMergeCols * es);   // [8][rv + 4]
-  float* wsm = ot + kMergeHeads * opitch;                                     // [8][S]
-  float* red = wsm + kMergeHeads * S;                                         // [4][8][32]
-  float* hdr = red + 4 * kMergeHeads * kMergeCols;                            // [8][4]
+  uint8_t* bs = msm;                                                               // [rv][ncols]
+  float* ot = reinterpret_cast<float*>(msm + ((size_t)rv * a.cols * es + 15) / 16 * 16);  // [8][rv + 4]
+  float* wsm = ot + kMergeHeads * opitch;                                          // [8][S]
+  float* red = wsm + kMergeHeads * S;                                              // [nq][8][cols]
+  float* hdr = red + kMergeHeads * kMergeThreads;                                  // [8][4]
   span_begin(a.span);
-  stage_rows(bs, ncols * es, a.Bv, a.D, es, 0, rv, (long long)h * a.d + c0, ncols);   // stable data
+  if (!a.rs_o) stage_rows(bs, ncols * es, a.Bv, a.D, es, 0, rv, (long long)h * a.d + c0, ncols);   // stable data
   pdl_wait();
   pdl_trigger();
-  // projection roles: 4 columns x head x quarter of the ranks
-  const int cq = tid & 7, hh = (tid >> 3) & 7, rq = tid >> 6;
-  const int rper = ((rv + 15) / 16) * 4;            // ranks per quarter, multiple of 4
-  const int i0 = rq * rper, i1 = min(rv, i0 + rper);
+  // projection roles: column c of the block, quarter rq of the ranks
+  const int c = tid % a.cols, rq = tid / a.cols;
+  const int nq = kMergeThreads / a.cols;            // rank quarters (4 when cols = 128)
+  const int rper = ((rv + 4 * nq - 1) / (4 * nq)) * 4;   // ranks per quarter, multiple of 4
+  const int i0 = min(rv, rq * rper), i1 = min(rv, i0 + rper);
   bool staged = false;
   for (int jb = 0; jb < G; jb += kMergeHeads) {
     const int nh = min(kMergeHeads, G - jb);
@@ -362,40 +371,25 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
       }
     }
     __syncthreads();
-    // combined rank-space outputs, thread = rank; two heads at a time with up to 16
-    // splits each in flight, so the L2 round trips overlap
+    // combined rank-space outputs: thread = (head u, rank i) element, its splits' loads
+    // issued 16 at a time before the arithmetic
     const size_t sstride = (size_t)a.s_stride * a.Hq * rv;
-    for (int u0 = 0; u0 < nh; u0 += 2) {
-      const bool two = u0 + 1 < nh;
-      const int j0 = h * G + jb + u0;
-      for (int i = tid; i < rv; i += kMergeThreads) {
-        const float* src0 = a.part_o + ((size_t)b * a.b_stride * a.Hq + j0) * rv + i;
-        const float* src1 = src0 + rv;                       // head j0 + 1
-        float acc0 = 0.f, acc1 = 0.f;
-        for (int s0 = 0; s0 < S; s0 += 16) {
-          float v0[16], v1[16];
+    for (int idx = tid; idx < nh * rv; idx += kMergeThreads) {
+      const int u = idx / rv, i = idx - (idx / rv) * rv;
+      const float* src = a.part_o + ((size_t)b * a.b_stride * a.Hq + h * G + jb + u) * rv + i;
+      float acc = 0.f;
+      for (int s0 = 0; s0 < S; s0 += 16) {
+        float v[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const bool in = s0 + k < S;
-            v0[k] = in ? __ldg(src0 + (size_t)(s0 + k) * sstride) : 0.f;
-            v1[k] = (in && two) ? __ldg(src1 + (size_t)(s0 + k) * sstride) : 0.f;
-          }
+        for (int k = 0; k < 16; ++k) v[k] = s0 + k < S ? __ldg(src + (size_t)(s0 + k) * sstride) : 0.f;
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            if (s0 + k < S) {
-              // a split with no tokens has weight 0 and an unwritten output: skipped
-              const float w0 = wsm[u0 * S + s0 + k];
-              if (w0 != 0.f) acc0 = fmaf(w0, v0[k], acc0);
-              if (two) {
-                const float w1 = wsm[(u0 + 1) * S + s0 + k];
-                if (w1 != 0.f) acc1 = fmaf(w1, v1[k], acc1);
-              }
-            }
-          }
+        for (int k = 0; k < 16; ++k) {
+          // a split with no tokens has weight 0 and an unwritten output: skipped
+          const float w = s0 + k < S ? wsm[u * S + s0 + k] : 0.f;
+          if (w != 0.f) acc = fmaf(w, v[k], acc);
         }
-        ot[u0 * opitch + i] = acc0;
-        if (two) ot[(u0 + 1) * opitch + i] = acc1;
       }
+      ot[u * opitch + i] = acc;
     }
     if (!staged) {
       cp_async_wait_all();
@@ -415,39 +409,38 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
       __syncthreads();
       continue;
     }
-    // projection partial sums over this thread's quarter of the ranks
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (hh < nh && 4 * cq < ncols) {
-      const float* orow = ot + hh * opitch;
+    // projection partial sums over this thread's quarter of the ranks, for every head
+    float acc[kMergeHeads];
+#pragma unroll
+    for (int u = 0; u < kMergeHeads; ++u) acc[u] = 0.f;
+    if (c < ncols && rq < nq) {
       for (int i = i0; i < i1; i += 4) {
-        const float4 o4 = *reinterpret_cast<const float4*>(orow + i);
-        const float ov[4] = {o4.x, o4.y, o4.z, o4.w};
+        float bv[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (i + k < i1) {
-            float bv[4];
-            El<T>::lds4(bs + ((size_t)(i + k) * ncols + 4 * cq) * es, bv);
+        for (int k = 0; k < 4; ++k) bv[k] = i + k < i1 ? El<T>::lds1(bs + ((size_t)(i + k) * ncols + c) * es) : 0.f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[e] = fmaf(ov[k], bv[e], acc[e]);
+        for (int u = 0; u < kMergeHeads; ++u) {
+          if (u < nh) {
+            const float4 o4 = *reinterpret_cast<const float4*>(ot + u * opitch + i);
+            acc[u] = fmaf(o4.x, bv[0], acc[u]);
+            acc[u] = fmaf(o4.y, bv[1], acc[u]);
+            acc[u] = fmaf(o4.z, bv[2], acc[u]);
+            acc[u] = fmaf(o4.w, bv[3], acc[u]);
           }
         }
       }
+      for (int u = 0; u < nh; ++u) red[(rq * kMergeHeads + u) * a.cols + c] = acc[u];
     }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) red[(rq * kMergeHeads + hh) * kMergeCols + 4 * cq + e] = acc[e];
     __syncthreads();
     // quarters added in order; window partial; normalisation; store
-    {
-      const int u = tid >> 5, c = tid & 31;
-      if (u < nh && c < ncols) {
-        const int j = h * G + jb + u;
-        float o = ((red[(0 * kMergeHeads + u) * kMergeCols + c] + red[(1 * kMergeHeads + u) * kMergeCols + c]) +
-                   red[(2 * kMergeHeads + u) * kMergeCols + c]) +
-                  red[(3 * kMergeHeads + u) * kMergeCols + c];
-        const size_t oi = ((size_t)b * a.Hq + j) * a.d + c0 + c;
-        if (a.win_o) o = fmaf(hdr[u * 4 + 2], a.win_o[oi], o);
-        El<T>::st(a.out, oi, o * hdr[u * 4 + 1]);
-      }
+    for (int idx = tid; idx < nh * ncols; idx += kMergeThreads) {
+      const int u = idx / ncols, cc = idx - (idx / ncols) * ncols;
+      float o = red[u * a.cols + cc];
+      for (int q = 1; q < nq; ++q) o += red[(q * kMergeHeads + u) * a.cols + cc];
+      const int j = h * G + jb + u;
+      const size_t oi = ((size_t)b * a.Hq + j) * a.d + c0 + cc;
+      if (a.win_o) o = fmaf(hdr[u * 4 + 2], a.win_o[oi], o);
+      El<T>::st(a.out, oi, o * hdr[u * 4 + 1]);
     }
     __syncthreads();
   }
@@ -455,9 +448,10 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
 }
 
 size_t merge_smem(const lr_cache_desc& d, int S, size_t es) {
-  return (size_t)d.rank_v * kMergeCols * es +
-         ((size_t)kMergeHeads * merge_pitch_f(d.rank_v) + (size_t)kMergeHeads * S +
-          4 * kMergeHeads * kMergeCols + kMergeHeads * 4) * sizeof(float);
+  const int cols = merge_cols(d.head_dim, d.rank_v, es);
+  return ((size_t)d.rank_v * cols * es + 15) / 16 * 16 +
+         ((size_t)kMergeHeads * merge_pitch_f(d.rank_v) + (size_t)kMergeHeads * S + kMergeHeads * kMergeThreads +
+          kMergeHeads * 4) * sizeof(float);
 }
 
 // ---- argument construction ------------------------------------------------------------
@@ -554,14 +548,16 @@ cudaError_t merge_t(const lr_cache* c, int n_splits, void* out, float* lse, cuda
   a.d = d.head_dim;
   a.D = c->D;
   a.rv = d.rank_v;
+  a.cols = merge_cols(d.head_dim, d.rank_v, sizeof(T));
   a.span = span_of(c->spans, SPAN_MERGE);
-  const int cbs = a.rs_o ? 1 : (d.head_dim + kMergeCols - 1) / kMergeCols;
+  const int cbs = a.rs_o ? 1 : (d.head_dim + a.cols - 1) / a.cols;
   return launch_pdl(k_merge<T>, dim3(cbs, d.n_kv_heads, d.batch), dim3(kMergeThreads), smem, s, a);
 }
 
 template <typename T>
-cudaError_t append_t(lr_cache* c, const void* k, const void* v, cudaStream_t s) {
-  const AppendArgs a = make_append_args(c, k, v);
+cudaError_t append_t(lr_cache* c, const void* k, const void* v, cudaStream_t s, long long bstride) {
+  AppendArgs a = make_append_args(c, k, v);
+  if (bstride && !c->win_slots) a.src_bstride = bstride;
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_append<T>, optin_done);
   if (e != cudaSuccess) return e;
@@ -601,8 +597,8 @@ cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse,
                                   : merge_t<float>(c, n_splits, out, lse, s, src);
 }
 
-cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s) {
-  return c->desc.dtype == LR_BF16 ? append_t<__nv_bfloat16>(c, k, v, s) : append_t<float>(c, k, v, s);
+cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s, long long bstride) {
+  return c->desc.dtype == LR_BF16 ? append_t<__nv_bfloat16>(c, k, v, s, bstride) : append_t<float>(c, k, v, s, bstride);
 }
 
 cudaError_t launch_step_pre(lr_cache* c, const void* k, const void* v, const void* q, bool tc, cudaStream_t s) {

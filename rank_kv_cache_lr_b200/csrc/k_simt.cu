@@ -139,59 +139,101 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind)
 }
 
 // ---------------------------------------------------------------------------
-// exact window (iS-KV): attention of each query head over the window tokens of
-// its KV head, as one more partial (in head space, relative to its own max)
+// exact window (iS-KV): attention of the query heads of each KV head over that head's
+// window tokens, as one more partial (in head space, relative to its own max).  One CTA per
+// (KV head, sequence), 256 threads: the window is read once per KV head, staged through
+// shared memory kWinChunk tokens at a time, with an online softmax per query head (warp per
+// head for the max and sum; thread per (head, token) for the scores and per (head, column)
+// for the outputs).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) k_window(const void* win_k, const void* win_v, const float* qd,
+constexpr int kWinChunk = 32;
+
+size_t window_smem(int G, int d) {
+  return ((size_t)G * d * 2 + 2 * (size_t)kWinChunk * (d + 1) + (size_t)G * kWinChunk + 3 * (size_t)G) *
+         sizeof(float);
+}
+
+__global__ void __launch_bounds__(256) k_window(const void* win_k, const void* win_v, const float* qd,
                                                 float* win_o, float* win_ml, int Hq, int Hkv, int d,
                                                 int D, int slots, int hist_len, int win_len, int dtype,
                                                 unsigned long long* span) {
   extern __shared__ float wsm[];
-  float* q_s = wsm;           // [d]
-  float* p_s = wsm + d;       // [win_len]
-  __shared__ float red[2];
+  const int G = Hq / Hkv;
+  const int kp = d + 1;                   // padded row pitch of the staged keys and values
+  float* q_s = wsm;                       // [G][d]
+  float* o_s = q_s + G * d;               // [G][d]
+  float* k_s = o_s + G * d;               // [kWinChunk][d + 1]
+  float* v_s = k_s + kWinChunk * kp;      // [kWinChunk][d + 1]
+  float* p_s = v_s + kWinChunk * kp;      // [G][kWinChunk]
+  float* m_s = p_s + G * kWinChunk;       // [G]
+  float* l_s = m_s + G;                   // [G]
+  float* a_s = l_s + G;                   // [G]
   span_begin(span);
   pdl_wait();
   pdl_trigger();
-  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int h = j / (Hq / Hkv);
-  const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
-  for (int c = tid; c < d; c += blockDim.x) q_s[c] = qd[((long long)b * Hq + j) * d + c];
-  __syncthreads();
-  for (int t = warp; t < win_len; t += nw) {
-    const int slot = (hist_len + t) % slots;
-    const long long off = ((long long)b * slots + slot) * D + (long long)h * d;
-    float s = 0.f;
-    for (int c = lane; c < d; c += 32) s = fmaf(q_s[c], elem_f(win_k, off + c, dtype), s);
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
+  const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
+  for (int idx = tid; idx < G * d; idx += nt) {
+    q_s[idx] = qd[((long long)b * Hq + h * G) * d + idx];
+    o_s[idx] = 0.f;
+  }
+  for (int u = tid; u < G; u += nt) {
+    m_s[u] = -INFINITY;
+    l_s[u] = 0.f;
+  }
+  for (int t0 = 0; t0 < win_len; t0 += kWinChunk) {
+    const int n = min(kWinChunk, win_len - t0);
+    __syncthreads();
+    for (int idx = tid; idx < n * d; idx += nt) {
+      const int t = idx / d, c = idx - (idx / d) * d;
+      const long long off = ((long long)b * slots + (hist_len + t0 + t) % slots) * D + (long long)h * d + c;
+      k_s[t * kp + c] = elem_f(win_k, off, dtype);
+      v_s[t * kp + c] = elem_f(win_v, off, dtype);
+    }
+    __syncthreads();
+    for (int idx = tid; idx < G * n; idx += nt) {
+      const int u = idx / n, t = idx - (idx / n) * n;
+      const float* qv = q_s + u * d;
+      const float* kv = k_s + t * kp;
+      float s0 = 0.f, s1 = 0.f;
+      for (int c = 0; c + 1 < d; c += 2) {
+        s0 = fmaf(qv[c], kv[c], s0);
+        s1 = fmaf(qv[c + 1], kv[c + 1], s1);
+      }
+      p_s[u * kWinChunk + t] = s0 + s1;
+    }
+    __syncthreads();
+    for (int u = warp; u < G; u += nw) {
+      const float sc = lane < n ? p_s[u * kWinChunk + lane] : -INFINITY;
+      float mx = sc;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) p_s[t] = s;
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float mo = m_s[u], mn = fmaxf(mo, mx);
+      const float pv = lane < n ? exp2f(sc - mn) : 0.f;
+      float sum = pv;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane < n) p_s[u * kWinChunk + lane] = pv;
+      if (lane == 0) {
+        const float alpha = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+        a_s[u] = alpha;
+        l_s[u] = l_s[u] * alpha + sum;
+        m_s[u] = mn;
+      }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < G * d; idx += nt) {
+      const int u = idx / d, c = idx - (idx / d) * d;
+      float o = o_s[idx] * a_s[u];
+      for (int t = 0; t < n; ++t) o = fmaf(p_s[u * kWinChunk + t], v_s[t * kp + c], o);
+      o_s[idx] = o;
+    }
   }
   __syncthreads();
-  if (tid == 0) {
-    float m = -INFINITY;
-    for (int t = 0; t < win_len; ++t) m = fmaxf(m, p_s[t]);
-    float l = 0.f;
-    for (int t = 0; t < win_len; ++t) {
-      const float p = exp2f(p_s[t] - m);
-      p_s[t] = p;
-      l += p;
-    }
-    red[0] = m;
-    red[1] = l;
-  }
-  __syncthreads();
-  for (int c = tid; c < d; c += blockDim.x) {
-    float o = 0.f;
-    for (int t = 0; t < win_len; ++t) {
-      const int slot = (hist_len + t) % slots;
-      o = fmaf(p_s[t], elem_f(win_v, ((long long)b * slots + slot) * D + (long long)h * d + c, dtype), o);
-    }
-    win_o[((long long)b * Hq + j) * d + c] = o;
-  }
-  if (tid == 0) {
-    win_ml[((long long)b * Hq + j) * 2] = red[0];
-    win_ml[((long long)b * Hq + j) * 2 + 1] = red[1];
+  for (int idx = tid; idx < G * d; idx += nt) win_o[((long long)b * Hq + h * G) * d + idx] = o_s[idx];
+  for (int u = tid; u < G; u += nt) {
+    win_ml[((long long)b * Hq + h * G + u) * 2] = m_s[u];
+    win_ml[((long long)b * Hq + h * G + u) * 2 + 1] = l_s[u];
   }
   span_end(span);
 }
@@ -345,12 +387,13 @@ cudaError_t launch_decode_simt(const lr_cache* c, int n_splits, int split_tokens
 cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
   const lr_cache_desc& d = c->desc;
   const float* qd = d.rope_in_kernel ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k;
-  const size_t smem = (size_t)(d.head_dim + c->win_len + 1) * sizeof(float);
-  dim3 grid(d.n_q_heads, d.batch);
+  const size_t smem = window_smem(d.n_q_heads / d.n_kv_heads, d.head_dim);
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+  dim3 grid(d.n_kv_heads, d.batch);
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_window, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_window, grid, dim3(128), smem, s, c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads, d.n_kv_heads,
+  return launch_pdl(k_window, grid, dim3(256), smem, s, c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads, d.n_kv_heads,
                                    d.head_dim, c->D, c->win_slots, c->hist_len, c->win_len, d.dtype,
                                    span_of(c->spans, SPAN_WINDOW));
 }

@@ -319,6 +319,35 @@ lr_status lr_kv_append(lr_cache* c, const void* k, const void* v, void* stream) 
   return LR_OK;
 }
 
+lr_status lr_kv_prefill(lr_cache* c, const void* k, const void* v, int32_t n, void* stream) {
+  if (!c || !k || !v || n < 0 || !c->has_A) return LR_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15) return LR_ERR_INVALID_ARG;
+  if (c->win_slots) return LR_ERR_UNSUPPORTED;
+  if ((long long)c->len + n > c->desc.capacity) return LR_ERR_CAPACITY;
+  c->undo = 0;
+  if (n == 0) return LR_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  cudaError_t e = cudaSuccess;
+  if (prefill_tc_supported(&c->desc, c->D)) {
+    e = launch_prefill_tc(c, k, v, n, s);
+    if (e != cudaSuccess) return LR_ERR_CUDA;
+    c->hist_len += n;
+    c->len += n;
+    return LR_OK;
+  }
+  // other dtypes and shapes: one append launch per token (CUDA cores)
+  const size_t row = (size_t)c->D * c->esize;
+  for (int t = 0; t < n; ++t) {
+    e = launch_append(c, static_cast<const char*>(k) + t * row, static_cast<const char*>(v) + t * row, s,
+                      (long long)n * c->D);
+    if (e != cudaSuccess) return LR_ERR_CUDA;
+    ++c->hist_len;
+    ++c->len;
+  }
+  return LR_OK;
+}
+
 lr_status lr_kv_append_latent(lr_cache* c, const float* zk, const float* zv, int32_t n, void* stream) {
   if (!c || !zk || !zv || n < 0) return LR_ERR_INVALID_ARG;
   if (c->win_len > 0) return LR_ERR_INVALID_ARG;

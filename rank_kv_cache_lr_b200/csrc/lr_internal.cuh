@@ -151,7 +151,11 @@ struct MergeSource {
 };
 cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s,
                          const MergeSource* src = nullptr);
-cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s);
+// bstride: elements between the batch rows of k and v (0: D, rows of one token per sequence)
+cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s, long long bstride = 0);
+// bulk prefill on tensor cores (k_prefill_tc.cu): n tokens per sequence, k / v [B][n][D]
+bool prefill_tc_supported(const lr_cache_desc* d, int D);
+cudaError_t launch_prefill_tc(lr_cache* c, const void* k, const void* v, int n, cudaStream_t s);
 // append (with the cache's current counters) and query projection in one grid
 cudaError_t launch_step_pre(lr_cache* c, const void* k, const void* v, const void* q, bool tc, cudaStream_t s);
 cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, int n,
