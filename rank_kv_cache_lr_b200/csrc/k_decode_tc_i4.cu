@@ -79,7 +79,7 @@ using tc::kTile;
 using tc::kTraceSlots;
 using tc::warp_reduce_scatter32;
 
-// 16 warps in four warpgroups: [producer, MMA, B_k producer / idle, idle] [4 softmax]
+// 16 warps in four warpgroups: [producer, key MMAs, B_k producer / idle, value MMAs] [4 softmax]
 // [dequantisation x 8].  A warp runs on sub-partition (warp % 4), and a tcgen05.ld / st
 // reaches TMEM lanes 32 (warp % 4) .. + 31.  Launched at 128 registers per thread; the
 // warpgroups then rebalance the block's 64K registers with setmaxnreg (the softmax keeps
@@ -158,7 +158,8 @@ struct I4Params {
 //   s_empty[2]        4        softmax warps (scores read) -> MMA issuer
 //   p_full[2]         4        softmax warps (fenced P stores) -> MMA issuer
 //   p_empty[2]        1        MMA commit of GEMM2 -> softmax warps (P reuse, O~ rescale)
-//   o_final           1        MMA commit after the last unit -> softmax warps (epilogue)
+//   o_final           1        value issuer's commit after its last unit -> softmax warps (epilogue)
+//   k_fin             1        key issuer's commit after its last unit -> itself (drain before exit)
 //   keys before RoPE, in place of s_empty:
 //   k_full            1        MMA commit of GEMM0 -> softmax warps
 //   krot_full         4        softmax warps (rotated fp16 keys stored, waited, fenced) -> MMA issuer
@@ -173,7 +174,7 @@ struct Aux {
   uint64_t raw_full[kMaxRaw];
   uint64_t raw_empty[kMaxRaw];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
-  uint64_t q_full, o_final;
+  uint64_t q_full, o_final, k_fin;
   uint64_t k_full, k_empty, krot_full, qb_full, b_full[kNBMax], b_empty[kNBMax];
   uint32_t tmem_base;
   int abort_flag;
@@ -318,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::mbar_init(&aux->q_full, 1);
     ptx::mbar_init(&aux->o_final, 1);
+    ptx::mbar_init(&aux->k_fin, 1);
     if (kRope) {
       ptx::mbar_init(&aux->k_full, 1);
       ptx::mbar_init(&aux->k_empty, kSmWarps);
@@ -427,8 +429,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         (void)ok;   // drained whether or not the CTA aborted (see the producer above)
         for (int k = max(0, issued - p.nb); k < issued; ++k) drain_wait(&aux->b_full[k % p.nb], (k / p.nb) & 1);
       }
-    } else if (warp == 1) {
-      // ------------------------------------------------------------- MMA issuer
+    } else if (warp == 1 || warp == 3) {
+      // ------------------------------------------------------------- MMA issuers
+      // The issue of one MMA from a thread costs ~100 cycles on this tensor core whatever
+      // its N, which at N = 32 is the pace of the whole kernel; two issuers on different
+      // sub-partitions double the rate: warp 1 issues the key side (GEMM1, or GEMM0 and
+      // the score MMAs), warp 3 the value mix (GEMM2).  Both walk the units in order to
+      // keep the operand-slot positions; each commits its own MMAs.
+      const bool kside = warp == 1;
       if (lane == 0 && ntiles > 0) {
         const uint32_t id = ptx::idesc_f16(0, 0, 0, 128, 32);    // GEMM1: fp16, A (TMEM) x K-major B
         const uint32_t id2 = ptx::idesc_f16(0, 0, 1, 128, 32);   // GEMM2: fp16, A (TMEM) x MN-major B
@@ -441,14 +449,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bdesc0 = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, 2);      // B_k, K-major SW128
         const uint32_t idq = ptx::idesc_f16(0, 0, 0, 128, kMaxG);                        // scores (kRope)
         const uint64_t qbdesc0 = ptx::smem_desc(ptx::smem_u32(q_s + p.qf_bytes), 16, 1024, 2);   // fp16 q, SW128
-        bool ok = kRope ? true : wait_b(&aux->q_full, 0, aux, p.err);
+        bool ok = (kRope || !kside) ? true : wait_b(&aux->q_full, 0, aux, p.err);
         ptx::tc_fence_after();
-        tc::trace_stamp(p.trace, 2);
+        if (kside) tc::trace_stamp(p.trace, 2);
         int pos = 0, bpos = 0;
         for (int u = 0; u < nunits && ok; ++u) {
           int tile;
           bool is_v;
           tc::unit_of(u, ntiles, &tile, &is_v);
+          if (is_v == kside) {          // the other issuer's unit: its operand slots only
+            pos += is_v ? p.cv : p.ck;
+            continue;
+          }
           if (kRope && !is_v) {
             // GEMM0(tile): [K^_0 | K^_1] = Z_k [B_k,0 | B_k,1], columns [128 h, +128) per head
             if (tile >= 1 && !(ok = wait_b(&aux->k_empty, (tile - 1) & 1, aux, p.err))) break;
@@ -535,9 +547,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (tile < 16) tc::trace_stamp(p.trace, 6 + 4 * tile);
           }
         }
-        ptx::mma_commit(&aux->o_final);
-        // the MMAs have completed before TMEM is freed, even if the epilogue aborted
-        drain_wait(&aux->o_final, 0);
+        // the value issuer's last commit releases the epilogue; each issuer's MMAs have
+        // completed before TMEM is freed, even if the epilogue aborted
+        uint64_t* fin = kside ? &aux->k_fin : &aux->o_final;
+        ptx::mma_commit(fin);
+        drain_wait(fin, 0);
       }
       __syncwarp();
     }

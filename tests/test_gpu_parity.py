@@ -529,8 +529,9 @@ def test_decode_parity_prerope_head_shapes(lib, hq, hkv):
     """Keys before RoPE on tensor cores for other group sizes and KV-head counts: pairs of KV
     heads (Hkv even) or single heads (Hkv odd), up to 16 query heads per KV head (the
     score MMA's N); against the oracle, with the CUDA-core path alongside."""
-    p = synth.make_qwen("qwen32k", seed=3, batch=2, length=300, rank=192, quant_bits=4, rope=True,
-                        n_q_heads=hq, n_kv_heads=hkv, rank_v=160)
+    D = hkv * 128
+    p = synth.make_qwen("qwen32k", seed=3, batch=2, length=300, rank=min(192, D), quant_bits=4, rope=True,
+                        n_q_heads=hq, n_kv_heads=hkv, rank_v=min(160, D - 16))
     c = H.fill_cache(lib, p)
     assert lib.LR_PATH_TC in paths(lib, p)
     for q in (p.q, _sharp(p)):
