@@ -152,6 +152,9 @@ struct I4Params {
 //   raw_empty[nraw]   8        dequantisation warps -> producer
 //   slot_full[nas]    8        dequantisation warps (TMEM stores waited and fenced) -> MMA issuer
 //   slot_empty[nas]   1        MMA commit -> dequantisation warps
+//                              (slots [0, nas/2) hold key chunks, [nas/2, nas) value chunks: two
+//                              rings, each consumed by one issuer in order, so a consumer never
+//                              waits on a phase more than one ahead of its barrier)
 //   q_full            1 + tx   producer (after the grid-dependency wait) -> MMA issuer, or
 //                              the softmax warps for keys before RoPE
 //   s_full[2]         1        MMA commit of GEMM1 -> softmax warps
@@ -452,22 +455,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = (kRope || !kside) ? true : wait_b(&aux->q_full, 0, aux, p.err);
         ptx::tc_fence_after();
         if (kside) tc::trace_stamp(p.trace, 2);
+        // this issuer's operand-slot ring: the key ring is slots [0, nks), the value ring
+        // [nks, nas); each ring has one consumer, so its barriers' phases are waited in order
+        const int nks = p.nas / 2, ring0 = kside ? 0 : nks, nring = kside ? nks : p.nas - nks;
         int pos = 0, bpos = 0;
         for (int u = 0; u < nunits && ok; ++u) {
           int tile;
           bool is_v;
           tc::unit_of(u, ntiles, &tile, &is_v);
-          if (is_v == kside) {          // the other issuer's unit: its operand slots only
-            pos += is_v ? p.cv : p.ck;
-            continue;
-          }
+          if (is_v == kside) continue;   // the other issuer's unit
           if (kRope && !is_v) {
             // GEMM0(tile): [K^_0 | K^_1] = Z_k [B_k,0 | B_k,1], columns [128 h, +128) per head
             if (tile >= 1 && !(ok = wait_b(&aux->k_empty, (tile - 1) & 1, aux, p.err))) break;
             ptx::tc_fence_after();
             for (int c = 0; c < p.ck && ok; ++c, ++pos) {
-              const int slot = pos % p.nas;
-              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nas) & 1, aux, p.err))) break;
+              const int slot = ring0 + pos % nring;
+              if (!(ok = wait_b(&aux->slot_full[slot], (pos / nring) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
               const uint32_t a0 = tmem + kAC + slot * kASlotCols;
               for (int sb = 0; sb < 2 && c * 128 + sb * 64 < p.r_k; ++sb, ++bpos) {
@@ -508,8 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             const uint32_t d_s = tmem + kSCol + 64 * sb2;
             for (int c = 0; c < p.ck && ok; ++c, ++pos) {
-              const int slot = pos % p.nas;
-              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nas) & 1, aux, p.err))) break;
+              const int slot = ring0 + pos % nring;
+              if (!(ok = wait_b(&aux->slot_full[slot], (pos / nring) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
               const uint32_t a0 = tmem + kAC + slot * kASlotCols;
               const uint64_t b0 = qdesc0 + (uint64_t)((c * 2 * kQSubBytes) >> 4);
@@ -531,8 +534,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             const uint64_t b0 = pdesc0 + (uint64_t)((pb2 * kPBytes) >> 4);
             for (int c = 0; c < p.cv && ok; ++c, ++pos) {
-              const int slot = pos % p.nas;
-              if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nas) & 1, aux, p.err))) break;
+              const int slot = ring0 + pos % nring;
+              if (!(ok = wait_b(&aux->slot_full[slot], (pos / nring) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
               const uint32_t a0 = tmem + kAC + slot * kASlotCols;
               const uint32_t d_o = tmem + kOC + c * 32;
@@ -824,7 +827,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
       const uint32_t raw_base = ptx::smem_u32(raw);
       bool ok = true;
-      int pos = 0;
+      // operand-slot rings of the key side ([0, nks)) and the value side ([nks, nas)), each
+      // filled in unit order and consumed by one MMA issuer
+      const int nks = p.nas / 2;
+      int posk = 0, posv = 0;
       for (int u = 0; u < nunits && ok; ++u) {
         int tile;
         bool is_v;
@@ -833,12 +839,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nch = is_v ? p.cv : p.ck;
         const int rs = u % p.nraw;
         const uint32_t rb = raw_base + rs * p.raw_bytes;
+        const int ring0 = is_v ? nks : 0, nring = is_v ? p.nas - nks : nks;
+        int& pos = is_v ? posv : posk;
         // waits are made warp-uniform: the warp arrives once, after __syncwarp
         if (!(ok = __all_sync(0xffffffffu, wait_b(&aux->raw_full[rs], (u / p.nraw) & 1, aux, p.err)))) break;
         for (int c = 0; c < nch; ++c, ++pos) {
-          const int slot = pos % p.nas;
-          if (pos >= p.nas &&
-              !(ok = __all_sync(0xffffffffu, wait_b(&aux->slot_empty[slot], ((pos / p.nas) - 1) & 1, aux, p.err))))
+          const int slot = ring0 + pos % nring;
+          if (pos >= nring &&
+              !(ok = __all_sync(0xffffffffu, wait_b(&aux->slot_empty[slot], ((pos / nring) - 1) & 1, aux, p.err))))
             break;
           ptx::tc_fence_after();
           uint32_t v[32];
