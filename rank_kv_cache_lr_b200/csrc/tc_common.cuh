@@ -28,20 +28,21 @@ __host__ __device__ __forceinline__ uint64_t wait_limit(unsigned long long ns) {
 // Wait for phase `parity` of `bar`.  Gives up when another thread of the CTA has
 // aborted, or after `limit_ns`, in which case it records LR_ERR_TIMEOUT in the device
 // error word and raises the CTA's abort flag.  Returns false when it gave up.
+// (A phase already complete passes the first, non-blocking test; after that every round of
+// the loop checks the abort flag and the clock, then waits with the blocking try_wait, which
+// may suspend the thread for a while on its own.)
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, int* abort_flag, int* err,
                                        uint64_t limit_ns = kTimeoutNs) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+  if (ptx::mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((it & 31) == 0) {
-      if (*(volatile int*)abort_flag) return false;
-      if (ptx::globaltimer() - t0 > limit_ns) {
-        *(volatile int*)abort_flag = 1;
-        atomicExch(err, (int)LR_ERR_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (*(volatile int*)abort_flag) return false;
+    if (ptx::globaltimer() - t0 > limit_ns) {
+      *(volatile int*)abort_flag = 1;
+      atomicExch(err, (int)LR_ERR_TIMEOUT);
+      return false;
     }
+    if (ptx::mbar_try_wait(bar, parity)) return true;
   }
 }
 

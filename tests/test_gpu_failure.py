@@ -47,8 +47,11 @@ def test_wait_timeout_is_reported_and_the_cache_recovers(lib, kind, kw):
 
 
 def _free_bytes():
+    """Free device memory with torch's cached blocks returned (the test's own tensors
+    would otherwise keep 2 MB blocks of the caching allocator)."""
     import torch
     torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     return torch.cuda.mem_get_info()[0]
 
 
