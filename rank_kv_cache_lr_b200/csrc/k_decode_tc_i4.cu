@@ -902,9 +902,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&aux->slot_full[slot]);
+          if (u == 0 && c == 0 && threadIdx.x == kDqWarp0 * 32) tc::trace_stamp(p.trace, 67);
         }
         __syncwarp();
         if (ok && lane == 0) ptx::mbar_arrive(&aux->raw_empty[rs]);
+        if (threadIdx.x == kDqWarp0 * 32 && u < 3) tc::trace_stamp(p.trace, 68 + (u == 2));
+        if (threadIdx.x == kDqWarp0 * 32 && u == nunits - 1) tc::trace_stamp(p.trace, 70);
       }
     }
   }
