@@ -21,25 +21,27 @@
 //   GEMM2 A = z^_v chunk transposed: lane = rank, K = tokens.  Values are stored
 //     rank-major (see lr_internal.cuh), so a thread owns one rank row and expands eight
 //     tokens per word, each pair with its own fp16 {scale, zero}.
-// A tcgen05.st reaches only the 32 lanes of the writing warp's sub-partition, so the eight
-// dequantisation warps are two per sub-partition (warp % 4 = lane quarter), splitting the
-// columns of a chunk between them.
+// A tcgen05.st reaches only the 32 lanes of the writing warp's sub-partition, so each side
+// has four dequantisation warps, one per sub-partition (warp % 4 = lane quarter), each
+// expanding all 64 columns of its 32 lanes.
 //
 // Data flow.  The producer (warp 0) moves the codes and the {scale, zero} words of one side
-// (K or V) of one 128-token tile with two plain bulk copies into a ring of raw slots.  The
-// dequantisation warps expand each 128-rank chunk of a raw slot into a 64-column operand
-// slot of a TMEM ring.  Warp 1 issues the MMAs from one thread.  Four softmax warps (thread
-// = token row = TMEM lane) turn scores into probabilities and finish with the epilogue
-// (thread = rank row).
+// (K or V) of one 128-token tile with two plain bulk copies into that side's ring of raw
+// slots.  The four key warps expand each 128-rank chunk of a key slot into a 64-column
+// operand slot of the key ring in TMEM, the four value warps do the same for the values
+// into the value ring.  Warp 1 issues the key-side MMAs and warp 3 the value mix, each from
+// one thread.  Four softmax warps (thread = token row = TMEM lane) turn scores into
+// probabilities and finish with the epilogue (thread = rank row).
 //
-// Pipeline.  Operand slots, raw slots and MMAs all follow the order
+// Pipeline.  The producer issues the copies in the order
 //   K(0), K(1), V(0), K(2), V(1), ..., K(n-1), V(n-2), V(n-1)
-// so GEMM1 of tile s+1 runs while the softmax of tile s is still working: the scores
-// and the probabilities are double-buffered (S in two TMEM column blocks, P in two
-// shared-memory buffers).  The K steps of GEMM1 alternate between two accumulators, so
-// consecutive MMAs do not wait on each other's accumulation; the softmax adds the two.
-// When the running max of a head grows by more than 2^8 the softmax first waits for the
-// value mix of the previous tile and rescales O~ in TMEM.
+// so the keys of tile s+1 arrive before the values of tile s.  Each side's warps, rings and
+// issuer then run on their own: the key side up to two tiles ahead of the softmax (the
+// scores and the probabilities are double-buffered: S in two TMEM column blocks, P in two
+// shared-memory buffers), the value side behind it, never holding up the keys of the next
+// tile while a value chunk waits for its probabilities.  When the running max of a head
+// grows by more than 2^8 the softmax first waits for the value mix of the previous tile and
+// rescales O~ in TMEM.
 //
 // Nibble order.  A key code word holds elements m = 0..7 of an 8-rank run at bits 4m.  Two
 // masks and one shift give the four fp16 pairs (m0,m4) (m1,m5) (m2,m6) (m3,m7) through
@@ -80,19 +82,19 @@ using tc::kTraceSlots;
 using tc::warp_reduce_scatter32;
 
 // 16 warps in four warpgroups: [producer, key MMAs, B_k producer / idle, value MMAs] [4 softmax]
-// [dequantisation x 8].  A warp runs on sub-partition (warp % 4), and a tcgen05.ld / st
+// [4 key dequantisation] [4 value dequantisation].  A warp runs on sub-partition (warp % 4), and a tcgen05.ld / st
 // reaches TMEM lanes 32 (warp % 4) .. + 31.  Launched at 128 registers per thread; the
 // warpgroups then rebalance the block's 64K registers with setmaxnreg (the softmax keeps
 // 32 scores and 32 running sums per row).
 constexpr int kThreads = 512;
 constexpr int kDqWarp0 = 8;                // first warp of the dequantisation warpgroups
-constexpr int kDqWarps = 8;                // arrivals per operand slot / raw slot (one per warp)
+constexpr int kDqSide = 4;                 // arrivals per operand slot / raw slot (the side's warps)
 constexpr int kSmWarps = 4;                // softmax warps (one arrival each)
 constexpr int kLaunchRegs = 128;
 // Per-warpgroup register budgets of each variant (the smallest that ptxas fits without
 // spilling; multiples of 8): control, softmax / epilogue, dequantisation.
 template <bool kRope> struct Regs;
-template <> struct Regs<false> { static constexpr int ctl = 56, softmax = 208, dq = 112; };
+template <> struct Regs<false> { static constexpr int ctl = 64, softmax = 184, dq = 120; };
 template <> struct Regs<true> { static constexpr int ctl = 64, softmax = 240, dq = 104; };
 static_assert(128 * Regs<false>::ctl + 128 * Regs<false>::softmax + 256 * Regs<false>::dq <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
@@ -103,16 +105,16 @@ constexpr int kQRows = 32;                 // query heads, padded
 constexpr int kQSubBytes = kQRows * 128;   // 32 rows x 64 ranks x 2 B
 constexpr int kPBytes = 128 * 32 * 2;      // 128 tokens x 32 heads x 2 B
 constexpr int kAuxBytes = 2048;
-// TMEM columns, rank space: S of tile s in [64 (s % 2), +64) as two accumulators of 32
-// (K steps alternate), O~ chunk c in [128 + 32 c, +32), operand slots of 64 columns from 256
+// TMEM columns, rank space: S of tile s in [32 (s % 2), +32), O~ chunk c in [64 + 32 c, +32),
+// operand slots of 64 columns from 192 (two for keys, three for values)
 constexpr int kSCol = 0;
-constexpr int kOCol = 128;
-constexpr int kACol = 256;
+constexpr int kOCol = 64;
+constexpr int kACol = 192;
 // keys before RoPE: K^ of the pair in [0, 256), O~ in [256, 384), operand slots from 384
 constexpr int kOColR = 256;
 constexpr int kAColR = 384;
 constexpr int kASlotCols = 64;             // one operand slot: 128 lanes x 128 fp16 K elements
-constexpr int kMaxASlots = 4;
+constexpr int kMaxASlots = 5;
 constexpr int kRD = 128;                   // head dim of the rebuilt keys
 constexpr int kGHMax = 2;                  // KV heads per CTA (K^ of both fills 256 columns)
 constexpr int kMaxG = 32 / kGHMax;         // query slots per KV head (the N of the score MMA)
@@ -131,7 +133,9 @@ struct I4Params {
   const uint32_t* params_v;
   long long cap;
   int r_k, r_v, G_k, G_v, ck, cv, kb_k;
-  int Hq, hist_len, stable_len, split_tokens, n_splits, nas, nraw;
+  int Hq, hist_len, stable_len, split_tokens, n_splits;
+  int nks, nvs;                 // operand slots of the key ring [0, nks) and the value ring [nks, +nvs)
+  int nrk, nrv;                 // raw slots of the key ring [0, nrk) and the value ring [nrk, +nrv)
   uint32_t q_bytes, raw_bytes, raw_params;   // raw slot size; offset of its params
   float* part_o;
   float* part_ml;
@@ -146,15 +150,17 @@ struct I4Params {
   int nb;                   // B_k ring slots of gh * 16 KB
 };
 
-// Barriers (arrival count; who arrives -> who waits).  Every ring is used in the unit order
-// K(0), K(1), V(0), K(2), ..., and phase k of a barrier is waited with parity k & 1.
-//   raw_full[nraw]    1 + tx   producer's two bulk copies -> dequantisation warps
-//   raw_empty[nraw]   8        dequantisation warps -> producer
-//   slot_full[nas]    8        dequantisation warps (TMEM stores waited and fenced) -> MMA issuer
-//   slot_empty[nas]   1        MMA commit -> dequantisation warps
-//                              (slots [0, nas/2) hold key chunks, [nas/2, nas) value chunks: two
-//                              rings, each consumed by one issuer in order, so a consumer never
-//                              waits on a phase more than one ahead of its barrier)
+// Barriers (arrival count; who arrives -> who waits).  Phase k of a barrier is waited with
+// parity k & 1.
+//   raw_full[]        1 + tx   producer's two bulk copies -> the side's dequantisation warps
+//   raw_empty[]       4        the side's dequantisation warps -> producer
+//   slot_full[]       4        the side's dequantisation warps (TMEM stores waited and fenced)
+//                              -> the side's MMA issuer
+//   slot_empty[]      1        MMA commit -> the side's dequantisation warps
+//                              (raw slots [0, nrk) and operand slots [0, nks) hold keys, the
+//                              rest values: each ring has one producer and one consumer that
+//                              walk it in tile order, so no wait is on a phase more than one
+//                              ahead of its barrier)
 //   q_full            1 + tx   producer (after the grid-dependency wait) -> MMA issuer, or
 //                              the softmax warps for keys before RoPE
 //   s_full[2]         1        MMA commit of GEMM1 -> softmax warps
@@ -183,7 +189,7 @@ struct Aux {
   int abort_flag;
   unsigned long long wait_ns;   // this launch's wait limit
   float red[4][32];
-  float m_s[32];
+  alignas(16) float m_s[32];
   float alpha_s[32];
 };
 static_assert(sizeof(Aux) <= kAuxBytes, "aux block");
@@ -306,13 +312,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     tc::trace_stamp(p.trace, 0);
-    for (int s = 0; s < p.nas; ++s) {
-      ptx::mbar_init(&aux->slot_full[s], kDqWarps);
+    for (int s = 0; s < p.nks + p.nvs; ++s) {
+      ptx::mbar_init(&aux->slot_full[s], kDqSide);
       ptx::mbar_init(&aux->slot_empty[s], 1);
     }
-    for (int s = 0; s < p.nraw; ++s) {
+    for (int s = 0; s < p.nrk + p.nrv; ++s) {
       ptx::mbar_init(&aux->raw_full[s], 1);
-      ptx::mbar_init(&aux->raw_empty[s], kDqWarps);
+      ptx::mbar_init(&aux->raw_empty[s], kDqSide);
     }
     for (int k = 0; k < 2; ++k) {
       ptx::mbar_init(&aux->s_full[k], 1);
@@ -375,14 +381,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         };
         bool waited = false, ok = true;
-        int issued = 0;
+        int issued_k = 0, issued_v = 0;   // tiles whose copies were issued, per side
         for (int u = 0; u < nunits && ok; ++u) {
           int tile;
           bool is_v;
           tc::unit_of(u, ntiles, &tile, &is_v);
           const int t0 = tok_begin + tile * kTile;
           const int n = min(kTile, tok_end - t0);
-          const int rs = u % p.nraw, round = u / p.nraw;
+          const int nr = is_v ? p.nrv : p.nrk;
+          const int rs = (is_v ? p.nrk : 0) + tile % nr, round = tile / nr;
           if (!waited && (round > 0 || t0 + n > p.stable_len)) {
             pdl_wait();
             load_query();
@@ -399,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          &aux->raw_full[rs]);
           ptx::bulk_load(dst + p.raw_params, (is_v ? p.params_v : p.params_k) + i4_param_index(row0, G, 0),
                          (uint32_t)G * 512u, &aux->raw_full[rs]);
-          issued = u + 1;
+          (is_v ? issued_v : issued_k) = tile + 1;
         }
         if (!waited) {
           pdl_wait();
@@ -410,8 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // waiting for them.  In a normal run these are the phases the consumers already
         // waited for, so the waits return at once.
         drain_wait(&aux->q_full, 0);
-        for (int k = max(0, issued - p.nraw); k < issued; ++k)
-          drain_wait(&aux->raw_full[k % p.nraw], (k / p.nraw) & 1);
+        for (int k = max(0, issued_k - p.nrk); k < issued_k; ++k) drain_wait(&aux->raw_full[k % p.nrk], (k / p.nrk) & 1);
+        for (int k = max(0, issued_v - p.nrv); k < issued_v; ++k)
+          drain_wait(&aux->raw_full[p.nrk + k % p.nrv], (k / p.nrv) & 1);
       }
     } else if (kRope && warp == 2) {
       // ------------------------------------------------------------- B_k producer (kRope)
@@ -456,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_after();
         if (kside) tc::trace_stamp(p.trace, 2);
         // this issuer's operand-slot ring: the key ring is slots [0, nks), the value ring
-        // [nks, nas); each ring has one consumer, so its barriers' phases are waited in order
-        const int nks = p.nas / 2, ring0 = kside ? 0 : nks, nring = kside ? nks : p.nas - nks;
+        // [nks, nks + nvs)
+        const int ring0 = kside ? 0 : p.nks, nring = kside ? p.nks : p.nvs;
         int pos = 0, bpos = 0;
         for (int u = 0; u < nunits && ok; ++u) {
           int tile;
@@ -504,12 +512,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                            idq, kk ? 1u : 0u);
             ptx::mma_commit(&aux->s_full[0]);
           } else if (!is_v) {
-            // GEMM1(tile): S[tile % 2] = Z_k q~^T, K steps alternating between the buffer's
-            // two accumulators
+            // GEMM1(tile): S[tile % 2] = Z_k q~^T (consecutive MMAs into one accumulator issue
+            // at the same rate as into alternating ones)
             const int sb2 = tile & 1;
             if (tile >= 2 && !(ok = wait_b(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
             ptx::tc_fence_after();
-            const uint32_t d_s = tmem + kSCol + 64 * sb2;
+            const uint32_t d_s = tmem + kSCol + 32 * sb2;
             for (int c = 0; c < p.ck && ok; ++c, ++pos) {
               const int slot = ring0 + pos % nring;
               if (!(ok = wait_b(&aux->slot_full[slot], (pos / nring) & 1, aux, p.err))) break;
@@ -520,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               // step kk: 8 TMEM columns on A; sub-block kk / 4 (4 KB), 32 bytes per step on B
               for (int kk = 0; kk < nk; ++kk) {
                 const uint32_t bo = (uint32_t)((kk >> 2) * (kQSubBytes >> 4) + (kk & 3) * 2);
-                mma_f16_ta(d_s + 32 * (kk & 1), a0 + (uint32_t)(kk * 8), b0 + bo, id, (c | (kk >> 1)) ? 1u : 0u);
+                mma_f16_ta(d_s, a0 + (uint32_t)(kk * 8), b0 + bo, id, (c | kk) ? 1u : 0u);
               }
               ptx::mma_commit(&aux->slot_empty[slot]);
             }
@@ -565,8 +573,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qd = warp & 3;
       const int row = qd * 32 + lane;
       const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-      // the second score accumulator holds the odd K steps (none when r_k = 16)
-      const bool two_acc = p.r_k > 16;
       float l[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) l[j] = 0.f;
@@ -607,19 +613,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           dst[2 * k + 1] = v.y;
         }
       };
-      // scores of tile buffer k2: the sum of the two accumulators
+      // scores of tile buffer k2
       auto load_s = [&](int k2, bool valid, float(&s)[32]) {
-        const uint32_t s_col = tmem + lane_off + kSCol + 64 * k2;
+        const uint32_t s_col = tmem + lane_off + kSCol + 32 * k2;
+        uint32_t sv[16], sw[16];
+        ptx::tmem_ld16(s_col, sv);
+        ptx::tmem_ld16(s_col + 16, sw);
+        ptx::tmem_wait_ld();
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t sv[16], sw[16];
-          ptx::tmem_ld16(s_col + 16 * hh, sv);
-          if (two_acc) ptx::tmem_ld16(s_col + 32 + 16 * hh, sw);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            s[16 * hh + j] = valid ? (two_acc ? __uint_as_float(sv[j]) + __uint_as_float(sw[j]) : __uint_as_float(sv[j]))
-                                   : -INFINITY;
+        for (int j = 0; j < 16; ++j) {
+          s[j] = valid ? __uint_as_float(sv[j]) : -INFINITY;
+          s[16 + j] = valid ? __uint_as_float(sw[j]) : -INFINITY;
         }
       };
       if (kRope) load_cs(cs, 0, 0);
@@ -695,7 +699,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         bool ex = false;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ex |= s[j] > aux->m_s[j] + kLazy;
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 mv = reinterpret_cast<const float4*>(aux->m_s)[j4];   // broadcast reads
+          ex |= (s[4 * j4] > mv.x + kLazy) | (s[4 * j4 + 1] > mv.y + kLazy) | (s[4 * j4 + 2] > mv.z + kLazy) |
+                (s[4 * j4 + 3] > mv.w + kLazy);
+        }
         ex = ptx::named_bar_or(1, 128, ex);
         if (ex) {
           // the value mix of the previous tile must be complete before O~ is rescaled
@@ -753,10 +761,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int hg = 0; hg < 4; ++hg) {
           uint32_t hw[4];
+          const float4 ma = reinterpret_cast<const float4*>(aux->m_s)[2 * hg];
+          const float4 mb = reinterpret_cast<const float4*>(aux->m_s)[2 * hg + 1];
+          const float mh[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int j = hg * 8 + 2 * e;
-            const __half2 h = __floats2half2_rn(exp2f(s[j] - aux->m_s[j]), exp2f(s[j + 1] - aux->m_s[j + 1]));
+            const __half2 h = __floats2half2_rn(exp2f(s[j] - mh[2 * e]), exp2f(s[j + 1] - mh[2 * e + 1]));
             const float2 f = __half22float2(h);
             l[j] += f.x;
             l[j + 1] += f.y;
@@ -819,95 +830,97 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::setmaxnreg_dec<Regs<kRope>::dq>();
     // ------------------------------------------------------------- dequantisation
     if (ntiles > 0) {
-      // warp (quarter qd = warp % 4, half h): TMEM lanes 32 qd .. + 31 of each operand slot,
-      // columns [32 h, +32) of it.  Keys: token 32 qd + lane, ranks 64 h .. + 63 of the
-      // chunk (groups 4c + 2h, + 1).  Values: rank 128 c + 32 qd + lane (group 4c + qd),
-      // tokens 64 h .. + 63.
-      const int qd = warp & 3, h = (warp - kDqWarp0) >> 2;
+      // side = 0 (warps 8..11): keys; side = 1 (warps 12..15): values.  Warp quarter
+      // qd = warp % 4 owns TMEM lanes 32 qd .. + 31 of every operand slot of its side and
+      // fills all 64 columns, in two halves h of 32 columns.  Keys: token 32 qd + lane, ranks
+      // 64 h .. + 63 of the chunk (groups 4c + 2h, + 1).  Values: rank 128 c + 32 qd + lane
+      // (group 4c + qd), tokens 64 h .. + 63.
+      const int qd = warp & 3;
+      const bool is_v = warp >= kDqWarp0 + 4;
       const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
       const uint32_t raw_base = ptx::smem_u32(raw);
+      const int G = is_v ? p.G_v : p.G_k;
+      const int nch = is_v ? p.cv : p.ck;
+      const int nr = is_v ? p.nrv : p.nrk, r0 = is_v ? p.nrk : 0;
+      const int ring0 = is_v ? p.nks : 0, nring = is_v ? p.nvs : p.nks;
+      const bool tracer = lane == 0 && qd == 0;
       bool ok = true;
-      // operand-slot rings of the key side ([0, nks)) and the value side ([nks, nas)), each
-      // filled in unit order and consumed by one MMA issuer
-      const int nks = p.nas / 2;
-      int posk = 0, posv = 0;
-      for (int u = 0; u < nunits && ok; ++u) {
-        int tile;
-        bool is_v;
-        tc::unit_of(u, ntiles, &tile, &is_v);
-        const int G = is_v ? p.G_v : p.G_k;
-        const int nch = is_v ? p.cv : p.ck;
-        const int rs = u % p.nraw;
+      int pos = 0;
+      for (int tile = 0; tile < ntiles && ok; ++tile) {
+        const int rs = r0 + tile % nr;
         const uint32_t rb = raw_base + rs * p.raw_bytes;
-        const int ring0 = is_v ? nks : 0, nring = is_v ? p.nas - nks : nks;
-        int& pos = is_v ? posv : posk;
         // waits are made warp-uniform: the warp arrives once, after __syncwarp
-        if (!(ok = __all_sync(0xffffffffu, wait_b(&aux->raw_full[rs], (u / p.nraw) & 1, aux, p.err)))) break;
+        if (!(ok = __all_sync(0xffffffffu, wait_b(&aux->raw_full[rs], (tile / nr) & 1, aux, p.err)))) break;
         for (int c = 0; c < nch; ++c, ++pos) {
           const int slot = ring0 + pos % nring;
           if (pos >= nring &&
               !(ok = __all_sync(0xffffffffu, wait_b(&aux->slot_empty[slot], ((pos / nring) - 1) & 1, aux, p.err))))
             break;
           ptx::tc_fence_after();
-          uint32_t v[32];
-          bool any = false;
-          if (!is_v) {
-            const int t = qd * 32 + lane;
-            const int g0 = 4 * c + 2 * h;
-            any = g0 < G;
+          bool stored = false;
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            uint32_t v[32];
+            bool any = false;
+            if (!is_v) {
+              const int t = qd * 32 + lane;
+              const int g0 = 4 * c + 2 * h;
+              any = g0 < G;
 #pragma unroll
-            for (int gi = 0; gi < 2; ++gi) {
-              const int g = g0 + gi;
-              if (g < G) {
-                const uint4 w = lds128(rb + (uint32_t)(g * 2048 + t * 16));
-                const uint32_t prm = lds32(rb + p.raw_params + (uint32_t)((g * 128 + t) * 4));
-                const uint32_t s2 = __byte_perm(prm, 0u, 0x1010), z2 = __byte_perm(prm, 0u, 0x3232);
-                const uint4 ss = make_uint4(s2, s2, s2, s2), zz = make_uint4(z2, z2, z2, z2);
-                put4(v, 16 * gi + 0, dequant8(w.x, ss, zz));
-                put4(v, 16 * gi + 4, dequant8(w.y, ss, zz));
-                put4(v, 16 * gi + 8, dequant8(w.z, ss, zz));
-                put4(v, 16 * gi + 12, dequant8(w.w, ss, zz));
-              } else {
+              for (int gi = 0; gi < 2; ++gi) {
+                const int g = g0 + gi;
+                if (g < G) {
+                  const uint4 w = lds128(rb + (uint32_t)(g * 2048 + t * 16));
+                  const uint32_t prm = lds32(rb + p.raw_params + (uint32_t)((g * 128 + t) * 4));
+                  const uint32_t s2 = __byte_perm(prm, 0u, 0x1010), z2 = __byte_perm(prm, 0u, 0x3232);
+                  const uint4 ss = make_uint4(s2, s2, s2, s2), zz = make_uint4(z2, z2, z2, z2);
+                  put4(v, 16 * gi + 0, dequant8(w.x, ss, zz));
+                  put4(v, 16 * gi + 4, dequant8(w.y, ss, zz));
+                  put4(v, 16 * gi + 8, dequant8(w.z, ss, zz));
+                  put4(v, 16 * gi + 12, dequant8(w.w, ss, zz));
+                } else {
 #pragma unroll
-                for (int k = 0; k < 16; ++k) v[16 * gi + k] = 0u;
+                  for (int k = 0; k < 16; ++k) v[16 * gi + k] = 0u;
+                }
               }
-            }
-          } else {
-            const int g = 4 * c + qd;
-            any = g < G;
-            if (any) {
-              const int i = c * 128 + qd * 32 + lane;
-              const uint32_t rowa = rb + (uint32_t)(i * 64);
-              const uint32_t sc = rb + p.raw_params + (uint32_t)(g * 512 + h * 128);   // scales of tokens 64h..
+            } else {
+              const int g = 4 * c + qd;
+              any = g < G;
+              if (any) {
+                const int i = c * 128 + qd * 32 + lane;
+                const uint32_t rowa = rb + (uint32_t)(i * 64);
+                const uint32_t sc = rb + p.raw_params + (uint32_t)(g * 512 + h * 128);   // scales of tokens 64h..
 #pragma unroll
-              for (int half = 0; half < 2; ++half) {
-                const int lc = 2 * h + half;                                   // 32-token column
-                const uint4 w = lds128(rowa + (uint32_t)(((lc ^ ((i >> 1) & 3))) * 16));
+                for (int half = 0; half < 2; ++half) {
+                  const int lc = 2 * h + half;                                   // 32-token column
+                  const uint4 w = lds128(rowa + (uint32_t)(((lc ^ ((i >> 1) & 3))) * 16));
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  // tokens 64 h + 32 half + 8 k .. + 7: scale and zero pairs (broadcast reads)
-                  const uint32_t off = (uint32_t)((half * 32 + 8 * k) * 2);
-                  const uint4 sp = lds128(sc + off), zp = lds128(sc + 256 + off);
-                  const uint32_t wk = k == 0 ? w.x : (k == 1 ? w.y : (k == 2 ? w.z : w.w));
-                  put4(v, 16 * half + 4 * k, dequant8(wk, sp, zp));
+                  for (int k = 0; k < 4; ++k) {
+                    // tokens 64 h + 32 half + 8 k .. + 7: scale and zero pairs (broadcast reads)
+                    const uint32_t off = (uint32_t)((half * 32 + 8 * k) * 2);
+                    const uint4 sp = lds128(sc + off), zp = lds128(sc + 256 + off);
+                    const uint32_t wk = k == 0 ? w.x : (k == 1 ? w.y : (k == 2 ? w.z : w.w));
+                    put4(v, 16 * half + 4 * k, dequant8(wk, sp, zp));
+                  }
                 }
               }
             }
+            if (any) {
+              ptx::tmem_st32(tmem + lane_off + (uint32_t)(kAC + slot * kASlotCols + 32 * h), v);
+              stored = true;
+            }
           }
-          if (any) {
-            ptx::tmem_st32(tmem + lane_off + (uint32_t)(kAC + slot * kASlotCols + 32 * h), v);
-            ptx::tmem_wait_st();
-          }
+          if (stored) ptx::tmem_wait_st();
           // each thread's TMEM stores are complete; order them before the arrival
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&aux->slot_full[slot]);
-          if (u == 0 && c == 0 && threadIdx.x == kDqWarp0 * 32) tc::trace_stamp(p.trace, 67);
+          if (!is_v && tile == 0 && c == 0 && tracer) tc::trace_stamp(p.trace, 67);
         }
         __syncwarp();
         if (ok && lane == 0) ptx::mbar_arrive(&aux->raw_empty[rs]);
-        if (threadIdx.x == kDqWarp0 * 32 && u < 3) tc::trace_stamp(p.trace, 68 + (u == 2));
-        if (threadIdx.x == kDqWarp0 * 32 && u == nunits - 1) tc::trace_stamp(p.trace, 70);
+        if (tracer && tile == (is_v ? 0 : 1)) tc::trace_stamp(p.trace, is_v ? 69 : 68);
+        if (tracer && is_v && tile == ntiles - 1) tc::trace_stamp(p.trace, 70);
       }
     }
   }
@@ -949,12 +962,13 @@ int q_bytes_for(const lr_cache_desc* d) {
 }
 
 struct I4Layout {
-  int nraw, nb;
+  int nraw, nb;   // raw slots (split evenly between the key and the value ring); B_k slots
   uint32_t raw_bytes, raw_params;
   size_t smem;
 };
 
-// Raw slots hold one side of one tile; as many as fit in 227 KB (up to 8) after the query
+// Raw slots hold one side of one tile; as many as fit in 227 KB (up to 8, at least one per
+// side; the keys get the smaller half) after the query
 // rows and P, and for keys before RoPE the B_k ring (up to one tile's worth of sub-blocks,
 // so the next tile's load while the current one is rotated).  The operand slots are in TMEM.
 bool choose_layout(const lr_cache_desc* d, I4Layout* L) {
@@ -1085,8 +1099,12 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   p.stable_len = std::min(c->stable_len, c->hist_len);
   p.split_tokens = split_tokens;
   p.n_splits = n_splits;
-  p.nas = rope ? (512 - kAColR) / kASlotCols : (512 - kACol) / kASlotCols;
-  p.nraw = st->nraw;
+  // operand slots: keys before RoPE 1 + 1 (K^ fills half of TMEM); rank space 2 + 3 (the
+  // values' ring holds a whole tile for r_v <= 384)
+  p.nks = rope ? 1 : 2;
+  p.nvs = rope ? 1 : 3;
+  p.nrk = st->nraw / 2;
+  p.nrv = st->nraw - p.nrk;
   p.q_bytes = st->q_bytes;
   p.raw_bytes = st->raw_bytes;
   p.raw_params = st->raw_params;

@@ -28,13 +28,16 @@ __host__ __device__ __forceinline__ uint64_t wait_limit(unsigned long long ns) {
 // Wait for phase `parity` of `bar`.  Gives up when another thread of the CTA has
 // aborted, or after `limit_ns`, in which case it records LR_ERR_TIMEOUT in the device
 // error word and raises the CTA's abort flag.  Returns false when it gave up.
-// (A phase already complete passes the first, non-blocking test; after that every round of
-// the loop checks the abort flag and the clock, then waits with the blocking try_wait, which
-// may suspend the thread for a while on its own.)
+// (A phase already complete passes the first, non-blocking test.  After that every round of
+// the loop checks the abort flag and the clock, then sleeps in the barrier until the phase
+// completes or kSuspendNs pass: a waiting thread costs no issue slots that the working warps
+// of its sub-partition need, and still sees an abort or its limit within kSuspendNs.)
+constexpr uint32_t kSuspendNs = 20000;
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, int* abort_flag, int* err,
                                        uint64_t limit_ns = kTimeoutNs) {
   if (ptx::mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
+  const uint32_t hint = limit_ns < kSuspendNs ? (uint32_t)limit_ns : kSuspendNs;
   for (;;) {
     if (*(volatile int*)abort_flag) return false;
     if (ptx::globaltimer() - t0 > limit_ns) {
@@ -42,7 +45,7 @@ __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, int* abor
       atomicExch(err, (int)LR_ERR_TIMEOUT);
       return false;
     }
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_try_wait_hint(bar, parity, hint)) return true;
   }
 }
 
@@ -51,7 +54,7 @@ __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, int* abor
 // waits above).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = ptx::globaltimer();
-  while (!ptx::mbar_try_wait(bar, parity))
+  while (!ptx::mbar_try_wait_hint(bar, parity, kSuspendNs))
     if (ptx::globaltimer() - t0 > kTimeoutNs) return;
 }
 
