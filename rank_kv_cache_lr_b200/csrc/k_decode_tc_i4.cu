@@ -207,17 +207,9 @@ struct I4State {
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
   return tc::wait_b(bar, parity, &aux->abort_flag, err, aux->wait_ns);
 }
-
-// D[tmem] (+)= A[tmem] x B[smem desc], kind::f16: the A operand is read from tensor memory
-// (lane = row, 32-bit column c = K elements 2c, 2c + 1; K-major).
-__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+// The same, by a whole warp with one verdict for all its lanes.
+__device__ __forceinline__ bool wait_w(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
+  return __all_sync(0xffffffffu, wait_b(bar, parity, aux, err));
 }
 
 // One fp16 pair of int4 codes: (lo, hi) = n - bias, then * scale + zero (one rounding).
@@ -442,13 +434,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 1 || warp == 3) {
       // ------------------------------------------------------------- MMA issuers
-      // The issue of one MMA from a thread costs ~100 cycles on this tensor core whatever
-      // its N, which at N = 32 is the pace of the whole kernel; two issuers on different
-      // sub-partitions double the rate: warp 1 issues the key side (GEMM1, or GEMM0 and
-      // the score MMAs), warp 3 the value mix (GEMM2).  Both walk the units in order to
-      // keep the operand-slot positions; each commits its own MMAs.
+      // Warp 1 issues the key side (GEMM1, or GEMM0 and the score MMAs), warp 3 the value
+      // mix (GEMM2); each commits its own MMAs.  The whole warp runs its loop (operands
+      // warp-uniform, K steps unrolled) and one elected lane issues: an MMA every ~18
+      // cycles, the tensor core's pace at N = 32, where one lane alone needs ~50-80.
       const bool kside = warp == 1;
-      if (lane == 0 && ntiles > 0) {
+      if (ntiles > 0) {
         const uint32_t id = ptx::idesc_f16(0, 0, 0, 128, 32);    // GEMM1: fp16, A (TMEM) x K-major B
         const uint32_t id2 = ptx::idesc_f16(0, 0, 1, 128, 32);   // GEMM2: fp16, A (TMEM) x MN-major B
         // Descriptors are built once; a step along K or to another slot adds its byte
@@ -460,9 +451,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bdesc0 = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, 2);      // B_k, K-major SW128
         const uint32_t idq = ptx::idesc_f16(0, 0, 0, 128, kMaxG);                        // scores (kRope)
         const uint64_t qbdesc0 = ptx::smem_desc(ptx::smem_u32(q_s + p.qf_bytes), 16, 1024, 2);   // fp16 q, SW128
-        bool ok = (kRope || !kside) ? true : wait_b(&aux->q_full, 0, aux, p.err);
+        bool ok = (kRope || !kside) ? true : wait_w(&aux->q_full, 0, aux, p.err);
         ptx::tc_fence_after();
-        if (kside) tc::trace_stamp(p.trace, 2);
+        if (kside && lane == 0) tc::trace_stamp(p.trace, 2);
         // this issuer's operand-slot ring: the key ring is slots [0, nks), the value ring
         // [nks, nks + nvs)
         const int ring0 = kside ? 0 : p.nks, nring = kside ? p.nks : p.nvs;
@@ -474,94 +465,98 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (is_v == kside) continue;   // the other issuer's unit
           if (kRope && !is_v) {
             // GEMM0(tile): [K^_0 | K^_1] = Z_k [B_k,0 | B_k,1], columns [128 h, +128) per head
-            if (tile >= 1 && !(ok = wait_b(&aux->k_empty, (tile - 1) & 1, aux, p.err))) break;
+            if (tile >= 1 && !(ok = wait_w(&aux->k_empty, (tile - 1) & 1, aux, p.err))) break;
             ptx::tc_fence_after();
             for (int c = 0; c < p.ck && ok; ++c, ++pos) {
               const int slot = ring0 + pos % nring;
-              if (!(ok = wait_b(&aux->slot_full[slot], (pos / nring) & 1, aux, p.err))) break;
+              if (!(ok = wait_w(&aux->slot_full[slot], (pos / nring) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
               const uint32_t a0 = tmem + kAC + slot * kASlotCols;
               for (int sb = 0; sb < 2 && c * 128 + sb * 64 < p.r_k; ++sb, ++bpos) {
                 const int bs = bpos % p.nb;
-                if (!(ok = wait_b(&aux->b_full[bs], (bpos / p.nb) & 1, aux, p.err))) break;
+                if (!(ok = wait_w(&aux->b_full[bs], (bpos / p.nb) & 1, aux, p.err))) break;
                 ptx::tc_fence_after();
                 const uint64_t b0 = bdesc0 + (uint64_t)((bs * b_slot_bytes) >> 4);
                 // K step kk of the sub-block: 8 TMEM columns on A, 32 bytes on B
                 const int nk = min(4, (p.r_k - c * 128 - sb * 64) >> 4);
-                for (int kk = 0; kk < nk; ++kk)
-                  mma_f16_ta(tmem, a0 + (uint32_t)(sb * 32 + kk * 8), b0 + (uint64_t)(kk * 2), idk,
-                             (c | sb | kk) ? 1u : 0u);
-                ptx::mma_commit(&aux->b_empty[bs]);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  if (kk < nk)
+                    ptx::mma_f16_ta_elect(tmem, a0 + (uint32_t)(sb * 32 + kk * 8), b0 + (uint64_t)(kk * 2), idk,
+                                     (c | sb | kk) ? 1u : 0u);
+                ptx::mma_commit_elect(&aux->b_empty[bs]);
               }
               if (!ok) break;
-              ptx::mma_commit(&aux->slot_empty[slot]);
+              ptx::mma_commit_elect(&aux->slot_empty[slot]);
             }
             if (!ok) break;
-            ptx::mma_commit(&aux->k_full);
-            if (tile < 16) tc::trace_stamp(p.trace, 3 + 4 * tile);
+            ptx::mma_commit_elect(&aux->k_full);
+            if (tile < 16 && lane == 0) tc::trace_stamp(p.trace, 3 + 4 * tile);
             // scores of the pair's query heads against the rotated fp16 keys the softmax warps
             // wrote back over K^: per head, M = 128 tokens, N = 16 query slots, K = d
-            if (tile == 0 && !(ok = wait_b(&aux->qb_full, 0, aux, p.err))) break;
-            if (!(ok = wait_b(&aux->krot_full, tile & 1, aux, p.err))) break;
+            if (tile == 0 && !(ok = wait_w(&aux->qb_full, 0, aux, p.err))) break;
+            if (!(ok = wait_w(&aux->krot_full, tile & 1, aux, p.err))) break;
             ptx::tc_fence_after();
             for (int h = 0; h < p.gh; ++h)
+#pragma unroll
               for (int kk = 0; kk < kRD / 16; ++kk)
-                mma_f16_ta(tmem + h * kRD + kRD / 2, tmem + h * kRD + kk * 8,
+                ptx::mma_f16_ta_elect(tmem + h * kRD + kRD / 2, tmem + h * kRD + kk * 8,
                            qbdesc0 + (uint64_t)((h * kQbHeadBytes + (kk >> 2) * (kQbHeadBytes / 2)) >> 4) +
                                (uint64_t)((kk & 3) * 2),
                            idq, kk ? 1u : 0u);
-            ptx::mma_commit(&aux->s_full[0]);
+            ptx::mma_commit_elect(&aux->s_full[0]);
           } else if (!is_v) {
             // GEMM1(tile): S[tile % 2] = Z_k q~^T (consecutive MMAs into one accumulator issue
             // at the same rate as into alternating ones)
             const int sb2 = tile & 1;
-            if (tile >= 2 && !(ok = wait_b(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
+            if (tile >= 2 && !(ok = wait_w(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
             ptx::tc_fence_after();
             const uint32_t d_s = tmem + kSCol + 32 * sb2;
             for (int c = 0; c < p.ck && ok; ++c, ++pos) {
               const int slot = ring0 + pos % nring;
-              if (!(ok = wait_b(&aux->slot_full[slot], (pos / nring) & 1, aux, p.err))) break;
+              if (!(ok = wait_w(&aux->slot_full[slot], (pos / nring) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
               const uint32_t a0 = tmem + kAC + slot * kASlotCols;
               const uint64_t b0 = qdesc0 + (uint64_t)((c * 2 * kQSubBytes) >> 4);
               const int nk = min(8, (p.r_k - c * 128) >> 4);     // 16-rank K steps in this chunk
               // step kk: 8 TMEM columns on A; sub-block kk / 4 (4 KB), 32 bytes per step on B
-              for (int kk = 0; kk < nk; ++kk) {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t bo = (uint32_t)((kk >> 2) * (kQSubBytes >> 4) + (kk & 3) * 2);
-                mma_f16_ta(d_s, a0 + (uint32_t)(kk * 8), b0 + bo, id, (c | kk) ? 1u : 0u);
+                if (kk < nk) ptx::mma_f16_ta_elect(d_s, a0 + (uint32_t)(kk * 8), b0 + bo, id, (c | kk) ? 1u : 0u);
               }
-              ptx::mma_commit(&aux->slot_empty[slot]);
+              ptx::mma_commit_elect(&aux->slot_empty[slot]);
             }
             if (!ok) break;
-            ptx::mma_commit(&aux->s_full[sb2]);
-            if (tile < 16) tc::trace_stamp(p.trace, 3 + 4 * tile);
+            ptx::mma_commit_elect(&aux->s_full[sb2]);
+            if (tile < 16 && lane == 0) tc::trace_stamp(p.trace, 3 + 4 * tile);
           } else {
             // GEMM2(tile): O~ += Z_v^T P[tile % 2]
             const int pb2 = tile & 1;
-            if (!(ok = wait_b(&aux->p_full[pb2], (tile >> 1) & 1, aux, p.err))) break;
+            if (!(ok = wait_w(&aux->p_full[pb2], (tile >> 1) & 1, aux, p.err))) break;
             ptx::tc_fence_after();
             const uint64_t b0 = pdesc0 + (uint64_t)((pb2 * kPBytes) >> 4);
             for (int c = 0; c < p.cv && ok; ++c, ++pos) {
               const int slot = ring0 + pos % nring;
-              if (!(ok = wait_b(&aux->slot_full[slot], (pos / nring) & 1, aux, p.err))) break;
+              if (!(ok = wait_w(&aux->slot_full[slot], (pos / nring) & 1, aux, p.err))) break;
               ptx::tc_fence_after();
               const uint32_t a0 = tmem + kAC + slot * kASlotCols;
               const uint32_t d_o = tmem + kOC + c * 32;
               // K step kt = 16 tokens: 8 TMEM columns on A, 256 B on P
 #pragma unroll
               for (int kt = 0; kt < 8; ++kt)
-                mma_f16_ta(d_o, a0 + (uint32_t)(kt * 8), b0 + (uint64_t)(kt * 16), id2, (tile | kt) ? 1u : 0u);
-              ptx::mma_commit(&aux->slot_empty[slot]);
+                ptx::mma_f16_ta_elect(d_o, a0 + (uint32_t)(kt * 8), b0 + (uint64_t)(kt * 16), id2, (tile | kt) ? 1u : 0u);
+              ptx::mma_commit_elect(&aux->slot_empty[slot]);
             }
             if (!ok) break;
-            ptx::mma_commit(&aux->p_empty[pb2]);
-            if (tile < 16) tc::trace_stamp(p.trace, 6 + 4 * tile);
+            ptx::mma_commit_elect(&aux->p_empty[pb2]);
+            if (tile < 16 && lane == 0) tc::trace_stamp(p.trace, 6 + 4 * tile);
           }
         }
         // the value issuer's last commit releases the epilogue; each issuer's MMAs have
         // completed before TMEM is freed, even if the epilogue aborted
         uint64_t* fin = kside ? &aux->k_fin : &aux->o_final;
-        ptx::mma_commit(fin);
+        ptx::mma_commit_elect(fin);
         drain_wait(fin, 0);
       }
       __syncwarp();

@@ -276,84 +276,133 @@ __global__ void __launch_bounds__(256) k_step_pre(AppendArgs aa, QprojArgs qa, i
 }
 
 // ---- split merge and output projection ------------------------------------------
-// One CTA per (column block of the head dimension, KV head h, sequence b), 512 threads; the
-// column block is the whole head dimension whenever B_v,h fits in shared memory (bf16 up to
-// r_v = 384), so the split partials of a (KV head, sequence) are read once.  Its columns of
-// B_v,h ([r_v][cols], no in-flight kernel writes them) are staged before the grid-dependency
-// wait.  Query heads go through in passes of up to 8: the split weights (log-sum-exp over
-// the splits and the window partial; one warp per head), the combined rank-space outputs
-// o~_j = sum_s w_s o~_s,j (thread = (head, rank) element, each with all its splits' loads in
-// flight), and o_j = o~_j B_v,h / l_j (thread = column x quarter of the ranks, all heads of
-// the pass; quarters added in a fixed order).
-constexpr int kMergeThreads = 512;
+// A cluster of ncb = ceil(d / 32) CTAs per (KV head h, sequence b), 128 threads each; CTA p
+// of the cluster owns output columns [32 p, +32) of the group's heads and ranks
+// [p rp, +rp) of the merge.  Per pass of up to 8 query heads:
+//   1. the split weights (log-sum-exp over the splits and the window partial; a warp per
+//      head in turn) while each thread's first split loads are already in flight;
+//   2. the merged rank-space outputs o~_j = sum_s w_s o~_s,j of the CTA's ranks (thread =
+//      (head, 4 ranks), float4 loads of up to 16 splits in flight);
+//   3. the parts are exchanged through distributed shared memory, so every CTA holds the
+//      whole o~_j of the pass, and projected: o_j = o~_j B_v,h / l_j for its columns
+//      (thread = column x quarter of the ranks, quarters added in a fixed order).
+// The columns of B_v,h (no in-flight kernel writes them) are staged before the
+// grid-dependency wait.  The exchange keeps every load of the partials issued once per
+// cluster and the dependent global-load rounds at two (the (m, l) pairs and the partials,
+// issued together).
+constexpr int kMergeThreads = 128;
 constexpr int kMergeHeads = 8;       // query heads per pass
-constexpr int kMergeBvBytes = 96 * 1024;   // shared-memory budget for the B_v,h columns
+constexpr int kMergeCols = 32;       // output columns per CTA
+constexpr int kMergeLoads = 16;      // split loads in flight per thread
 
 struct MergeArgs {
   const float* part_o; const float* part_ml; const float* win_o; const float* win_ml;
   const void* Bv; void* out; float* lse;
-  int S, Hq, Hkv, d, D, rv, cols;   // cols: output columns per CTA (multiple of 32, or d)
+  int S, Hq, Hkv, d, D, rv;
+  int ncb, rp;                // CTAs per cluster; ranks per CTA (multiple of 4)
   // partial (b, s) starts at head row (b * b_stride + s * s_stride) * Hq of part_o / part_ml:
   // the cache's [B][S][Hq] has b_stride = S, s_stride = 1; gathered shards [S][B][Hq] have
   // b_stride = 1, s_stride = B
   long long b_stride, s_stride;
-  // rank-space output instead of the projection (one column block): the merged o~ relative
-  // to the merged max, [B][Hq][rv], and (m, l) [B][Hq][2]; or null
+  // rank-space output instead of the projection: the merged o~ (relative to the merged
+  // max) [B][Hq][rv] and (m, l) [B][Hq][2]; or null
   float* rs_o; float* rs_ml;
   unsigned long long* span;   // timeline span, or null
 };
 
-int merge_cols(int d, int rv, size_t es) {
-  int cols = (int)(kMergeBvBytes / ((size_t)rv * es)) / 32 * 32;
-  cols = std::max(32, cols);
-  return cols >= d ? d : cols;
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_addr(const void* smem_ptr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(r)
+               : "r"((uint32_t)__cvta_generic_to_shared(smem_ptr)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 
-size_t merge_pitch_f(int rv) { return (size_t)rv + 4; }   // o~ rows, padded against bank conflicts
+struct MergeSmem {
+  size_t bs, otp, otf, mls, wsm, red, hdr, total;
+};
+__host__ __device__ inline MergeSmem merge_layout(int rv, int rp, int S, int es) {
+  MergeSmem L;
+  size_t o = 0;
+  L.bs = o;  o += ((size_t)rv * kMergeCols * es + 15) / 16 * 16;            // [rv][ncols] B_v columns
+  L.otp = o; o += (size_t)kMergeHeads * (rp + 4) * 4;                        // [8][rp + 4] this part
+  L.otf = o; o += (size_t)kMergeHeads * (rv + 4) * 4;                        // [8][rv + 4] whole o~
+  L.mls = o; o += (size_t)kMergeHeads * S * 8;                               // [8][S] (m, l)
+  L.wsm = o; o += ((size_t)kMergeHeads * S * 4 + 15) / 16 * 16;              // [8][S] weights
+  L.red = o; o += (size_t)4 * kMergeHeads * kMergeCols * 4;                  // [4][8][32]
+  L.hdr = o; o += (size_t)kMergeHeads * 4 * 4;                               // [8]{m, 1/l, w_win, l}
+  L.total = o;
+  return L;
+}
 
 template <typename T>
-__global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
+__global__ void __launch_bounds__(kMergeThreads, 1) k_merge(MergeArgs a) {
   extern __shared__ __align__(16) uint8_t msm[];
   constexpr int es = sizeof(T);
-  const int cb = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int p = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int G = a.Hq / a.Hkv, S = a.S, rv = a.rv;
-  const int c0 = cb * a.cols, ncols = min(a.cols, a.d - c0);
-  const int opitch = rv + 4;
-  uint8_t* bs = msm;                                                               // [rv][ncols]
-  float* ot = reinterpret_cast<float*>(msm + ((size_t)rv * a.cols * es + 15) / 16 * 16);  // [8][rv + 4]
-  float* wsm = ot + kMergeHeads * opitch;                                          // [8][S]
-  float* red = wsm + kMergeHeads * S;                                              // [nq][8][cols]
-  float* hdr = red + kMergeHeads * kMergeThreads;                                  // [8][4]
+  const int G = a.Hq / a.Hkv, S = a.S, rv = a.rv, rp = a.rp;
+  const int c0 = p * kMergeCols, ncols = min(kMergeCols, a.d - c0);
+  const int i0 = min(rv, p * rp), np = min(rv, i0 + rp) - i0;   // this CTA's ranks
+  const MergeSmem L = merge_layout(rv, rp, S, es);
+  uint8_t* bs = msm + L.bs;
+  float* otp = reinterpret_cast<float*>(msm + L.otp);
+  float* otf = reinterpret_cast<float*>(msm + L.otf);
+  float2* mls = reinterpret_cast<float2*>(msm + L.mls);
+  float* wsm = reinterpret_cast<float*>(msm + L.wsm);
+  float* red = reinterpret_cast<float*>(msm + L.red);
+  float* hdr = reinterpret_cast<float*>(msm + L.hdr);
+  const bool project = a.rs_o == nullptr;
   span_begin(a.span);
-  if (!a.rs_o) stage_rows(bs, ncols * es, a.Bv, a.D, es, 0, rv, (long long)h * a.d + c0, ncols);   // stable data
+  if (project) stage_rows(bs, ncols * es, a.Bv, a.D, es, 0, rv, (long long)h * a.d + c0, ncols);   // stable data
   pdl_wait();
   pdl_trigger();
-  // projection roles: column c of the block, quarter rq of the ranks
-  const int c = tid % a.cols, rq = tid / a.cols;
-  const int nq = kMergeThreads / a.cols;            // rank quarters (4 when cols = 128)
-  const int rper = ((rv + 4 * nq - 1) / (4 * nq)) * 4;   // ranks per quarter, multiple of 4
-  const int i0 = min(rv, rq * rper), i1 = min(rv, i0 + rper);
+  const size_t sstride = (size_t)a.s_stride * a.Hq * rv;   // floats between splits of one head row
+  auto row_of = [&](int s) -> size_t { return (size_t)b * a.b_stride + (size_t)s * a.s_stride; };
+  const int nq = np / 4;                                    // rank quads of this CTA
   bool staged = false;
   for (int jb = 0; jb < G; jb += kMergeHeads) {
     const int nh = min(kMergeHeads, G - jb);
-    // split weights, one warp per head
-    if (warp < nh) {
-      const int j = h * G + jb + warp;
+    const int nitems = nh * nq;
+    // 1. this thread's first item: its first kMergeLoads split loads go out now
+    const int u0 = tid < nitems ? tid / nq : 0, q0 = tid < nitems ? tid - u0 * nq : 0;
+    const float* src0 = a.part_o + ((size_t)b * a.b_stride * a.Hq + h * G + jb + u0) * rv + i0 + 4 * q0;
+    float4 v[kMergeLoads];
+#pragma unroll
+    for (int k = 0; k < kMergeLoads; ++k)
+      v[k] = (tid < nitems && k < S) ? __ldg(reinterpret_cast<const float4*>(src0 + (size_t)k * sstride))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = tid; e < nh * S; e += kMergeThreads) {
+      const int u = e / S, s = e - (e / S) * S;
+      mls[e] = __ldg(reinterpret_cast<const float2*>(a.part_ml) + row_of(s) * a.Hq + h * G + jb + u);
+    }
+    __syncthreads();
+    for (int u = warp; u < nh; u += kMergeThreads / 32) {
+      // split weights of head u (a split with no tokens has m = -inf: weight 0)
+      const int j = h * G + jb + u;
       float m = -INFINITY;
-      for (int s = lane; s < S; s += 32)
-        m = fmaxf(m, a.part_ml[(((size_t)b * a.b_stride + (size_t)s * a.s_stride) * a.Hq + j) * 2]);
+      for (int s = lane; s < S; s += 32) m = fmaxf(m, mls[u * S + s].x);
       const float mw = a.win_ml ? a.win_ml[((size_t)b * a.Hq + j) * 2] : -INFINITY;
       m = fmaxf(m, mw);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       float l = 0.f;
       for (int s = lane; s < S; s += 32) {
-        const size_t e = (((size_t)b * a.b_stride + (size_t)s * a.s_stride) * a.Hq + j) * 2;
-        const float ms = a.part_ml[e];
-        const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - m);
-        wsm[warp * S + s] = w;
-        l = fmaf(w, a.part_ml[e + 1], l);
+        const float2 ml = mls[u * S + s];
+        const float w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - m);
+        wsm[u * S + s] = w;
+        l = fmaf(w, ml.y, l);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -363,80 +412,109 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
           ww = exp2f(mw - m);
           l = fmaf(ww, a.win_ml[((size_t)b * a.Hq + j) * 2 + 1], l);
         }
-        hdr[warp * 4 + 0] = m;
-        hdr[warp * 4 + 1] = 1.0f / l;
-        hdr[warp * 4 + 2] = ww;
-        hdr[warp * 4 + 3] = l;
-        if (a.lse && cb == 0) a.lse[(size_t)b * a.Hq + j] = (m + log2f(l)) * LR_LN2;
+        hdr[u * 4 + 0] = m;
+        hdr[u * 4 + 1] = 1.0f / l;
+        hdr[u * 4 + 2] = ww;
+        hdr[u * 4 + 3] = l;
+        if (a.lse && p == 0) a.lse[(size_t)b * a.Hq + j] = (m + log2f(l)) * LR_LN2;
       }
     }
     __syncthreads();
-    // combined rank-space outputs: thread = (head u, rank i) element, its splits' loads
-    // issued 16 at a time before the arithmetic
-    const size_t sstride = (size_t)a.s_stride * a.Hq * rv;
-    for (int idx = tid; idx < nh * rv; idx += kMergeThreads) {
-      const int u = idx / rv, i = idx - (idx / rv) * rv;
-      const float* src = a.part_o + ((size_t)b * a.b_stride * a.Hq + h * G + jb + u) * rv + i;
-      float acc = 0.f;
-      for (int s0 = 0; s0 < S; s0 += 16) {
-        float v[16];
+    // 2. merged o~ of this CTA's ranks; splits in a fixed order, zero-weight splits skipped
+    //    (their outputs are not written)
+    for (int it = tid; it < nitems; it += kMergeThreads) {
+      const int u = it / nq, q = it - (it / nq) * nq;
+      const float* src = a.part_o + ((size_t)b * a.b_stride * a.Hq + h * G + jb + u) * rv + i0 + 4 * q;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = 0; s0 < S; s0 += kMergeLoads) {
+        if (it != tid || s0 > 0) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = s0 + k < S ? __ldg(src + (size_t)(s0 + k) * sstride) : 0.f;
+          for (int k = 0; k < kMergeLoads; ++k)
+            v[k] = s0 + k < S ? __ldg(reinterpret_cast<const float4*>(src + (size_t)(s0 + k) * sstride))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          // a split with no tokens has weight 0 and an unwritten output: skipped
+        for (int k = 0; k < kMergeLoads; ++k) {
           const float w = s0 + k < S ? wsm[u * S + s0 + k] : 0.f;
-          if (w != 0.f) acc = fmaf(w, v[k], acc);
+          if (w != 0.f) {
+            acc.x = fmaf(w, v[k].x, acc.x);
+            acc.y = fmaf(w, v[k].y, acc.y);
+            acc.z = fmaf(w, v[k].z, acc.z);
+            acc.w = fmaf(w, v[k].w, acc.w);
+          }
         }
       }
-      ot[u * opitch + i] = acc;
+      *reinterpret_cast<float4*>(otp + u * (rp + 4) + 4 * q) = acc;
     }
-    if (!staged) {
-      cp_async_wait_all();
-      staged = true;
-    }
-    __syncthreads();
-    if (a.rs_o) {
+    if (!project) {
       // rank-space partial of this shard: the merged o~ (relative to m) and (m, l)
-      for (int idx = tid; idx < nh * rv; idx += kMergeThreads) {
-        const int u = idx / rv, i = idx % rv;
-        a.rs_o[((size_t)b * a.Hq + h * G + jb + u) * rv + i] = ot[u * opitch + i];
+      __syncthreads();
+      for (int it = tid; it < nitems; it += kMergeThreads) {
+        const int u = it / nq, q = it - (it / nq) * nq;
+        *reinterpret_cast<float4*>(a.rs_o + ((size_t)b * a.Hq + h * G + jb + u) * rv + i0 + 4 * q) =
+            *reinterpret_cast<const float4*>(otp + u * (rp + 4) + 4 * q);
       }
-      if (tid < nh) {
+      if (p == 0 && tid < nh) {
         a.rs_ml[((size_t)b * a.Hq + h * G + jb + tid) * 2] = hdr[tid * 4 + 0];
         a.rs_ml[((size_t)b * a.Hq + h * G + jb + tid) * 2 + 1] = hdr[tid * 4 + 3];
       }
       __syncthreads();
       continue;
     }
-    // projection partial sums over this thread's quarter of the ranks, for every head
-    float acc[kMergeHeads];
+    // 3. every CTA gathers the whole o~ of the pass from the cluster's parts
+    cluster_sync_all();
+    for (int part = 0; part < a.ncb; ++part) {
+      const int pi0 = min(rv, part * rp), pnq = (min(rv, pi0 + rp) - pi0) / 4;
+      const uint32_t base = cluster_addr(otp, (uint32_t)part);
+      for (int it = tid; it < nh * pnq; it += kMergeThreads) {
+        const int u = it / pnq, q = it - (it / pnq) * pnq;
+        *reinterpret_cast<float4*>(otf + u * (rv + 4) + pi0 + 4 * q) =
+            ld_cluster_f4(base + (uint32_t)((u * (rp + 4) + 4 * q) * 4));
+      }
+    }
+    if (!staged) {
+      cp_async_wait_all();
+      staged = true;
+    }
+    // the parts have been read everywhere before any CTA overwrites its own (next pass) or
+    // exits; the gathered rows and the staged columns are visible to the whole CTA
+    cluster_sync_all();
+    // projection partial sums: column c, quarter rq of the ranks, every head of the pass
+    {
+      const int c = tid & 31, rq = tid >> 5;
+      const int rql = ((rv + 15) / 16) * 4;                  // ranks per quarter, multiple of 4
+      const int r0 = min(rv, rq * rql), r1 = min(rv, r0 + rql);
+      float acc[kMergeHeads];
 #pragma unroll
-    for (int u = 0; u < kMergeHeads; ++u) acc[u] = 0.f;
-    if (c < ncols && rq < nq) {
-      for (int i = i0; i < i1; i += 4) {
-        float bv[4];
+      for (int u = 0; u < kMergeHeads; ++u) acc[u] = 0.f;
+      if (c < ncols) {
+        for (int i = r0; i < r1; i += 4) {
+          float bv[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) bv[k] = i + k < i1 ? El<T>::lds1(bs + ((size_t)(i + k) * ncols + c) * es) : 0.f;
+          for (int k = 0; k < 4; ++k) bv[k] = El<T>::lds1(bs + ((size_t)(i + k) * ncols + c) * es);
 #pragma unroll
-        for (int u = 0; u < kMergeHeads; ++u) {
-          if (u < nh) {
-            const float4 o4 = *reinterpret_cast<const float4*>(ot + u * opitch + i);
-            acc[u] = fmaf(o4.x, bv[0], acc[u]);
-            acc[u] = fmaf(o4.y, bv[1], acc[u]);
-            acc[u] = fmaf(o4.z, bv[2], acc[u]);
-            acc[u] = fmaf(o4.w, bv[3], acc[u]);
+          for (int u = 0; u < kMergeHeads; ++u) {
+            if (u < nh) {
+              const float4 o4 = *reinterpret_cast<const float4*>(otf + u * (rv + 4) + i);
+              acc[u] = fmaf(o4.x, bv[0], acc[u]);
+              acc[u] = fmaf(o4.y, bv[1], acc[u]);
+              acc[u] = fmaf(o4.z, bv[2], acc[u]);
+              acc[u] = fmaf(o4.w, bv[3], acc[u]);
+            }
           }
         }
       }
-      for (int u = 0; u < nh; ++u) red[(rq * kMergeHeads + u) * a.cols + c] = acc[u];
+#pragma unroll
+      for (int u = 0; u < kMergeHeads; ++u) red[(rq * kMergeHeads + u) * kMergeCols + c] = acc[u];
     }
     __syncthreads();
     // quarters added in order; window partial; normalisation; store
-    for (int idx = tid; idx < nh * ncols; idx += kMergeThreads) {
-      const int u = idx / ncols, cc = idx - (idx / ncols) * ncols;
-      float o = red[u * a.cols + cc];
-      for (int q = 1; q < nq; ++q) o += red[(q * kMergeHeads + u) * a.cols + cc];
+    for (int e = tid; e < nh * kMergeCols; e += kMergeThreads) {
+      const int u = e / kMergeCols, cc = e % kMergeCols;
+      if (cc >= ncols) continue;
+      float o = red[u * kMergeCols + cc];
+#pragma unroll
+      for (int q = 1; q < 4; ++q) o += red[(q * kMergeHeads + u) * kMergeCols + cc];
       const int j = h * G + jb + u;
       const size_t oi = ((size_t)b * a.Hq + j) * a.d + c0 + cc;
       if (a.win_o) o = fmaf(hdr[u * 4 + 2], a.win_o[oi], o);
@@ -444,14 +522,18 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(MergeArgs a) {
     }
     __syncthreads();
   }
+  if (!staged) cp_async_wait_all();
   span_end(a.span);
 }
 
+// Ranks per CTA of the merge cluster: the rank range split evenly over the column blocks, in
+// multiples of 4 (ranks are multiples of 16).
+int merge_ncb(int d) { return (d + kMergeCols - 1) / kMergeCols; }
+int merge_rp(int rv, int ncb) { return ((rv + 4 * ncb - 1) / (4 * ncb)) * 4; }
+
 size_t merge_smem(const lr_cache_desc& d, int S, size_t es) {
-  const int cols = merge_cols(d.head_dim, d.rank_v, es);
-  return ((size_t)d.rank_v * cols * es + 15) / 16 * 16 +
-         ((size_t)kMergeHeads * merge_pitch_f(d.rank_v) + (size_t)kMergeHeads * S + kMergeHeads * kMergeThreads +
-          kMergeHeads * 4) * sizeof(float);
+  const int ncb = merge_ncb(d.head_dim);
+  return merge_layout(d.rank_v, merge_rp(d.rank_v, ncb), S, (int)es).total;
 }
 
 // ---- argument construction ------------------------------------------------------------
@@ -548,10 +630,10 @@ cudaError_t merge_t(const lr_cache* c, int n_splits, void* out, float* lse, cuda
   a.d = d.head_dim;
   a.D = c->D;
   a.rv = d.rank_v;
-  a.cols = merge_cols(d.head_dim, d.rank_v, sizeof(T));
+  a.ncb = merge_ncb(d.head_dim);
+  a.rp = merge_rp(d.rank_v, a.ncb);
   a.span = span_of(c->spans, SPAN_MERGE);
-  const int cbs = a.rs_o ? 1 : (d.head_dim + a.cols - 1) / a.cols;
-  return launch_pdl(k_merge<T>, dim3(cbs, d.n_kv_heads, d.batch), dim3(kMergeThreads), smem, s, a);
+  return launch_pdl_cluster(k_merge<T>, dim3(a.ncb, d.n_kv_heads, d.batch), dim3(kMergeThreads), a.ncb, smem, s, a);
 }
 
 template <typename T>
