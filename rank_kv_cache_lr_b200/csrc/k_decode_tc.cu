@@ -110,6 +110,10 @@ __device__ __forceinline__ void tmem_ld_sum(uint32_t taddr, float (&v)[32]) {
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
   return tc::wait_b(bar, parity, &aux->abort_flag, err, aux->wait_ns);
 }
+// The same, by a whole warp with one verdict for all its lanes.
+__device__ __forceinline__ bool wait_w(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
+  return __all_sync(0xffffffffu, wait_b(bar, parity, aux, err));
+}
 
 __device__ __forceinline__ void trace_stamp(const TcParams& p, int slot) { tc::trace_stamp(p.trace, slot); }
 
@@ -228,7 +232,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0 && ntiles > 0) {
+    // The whole warp runs the loop (operands warp-uniform, K steps unrolled) and one
+    // elected lane issues each MMA: far faster issue than a loop run by one lane.
+    if (ntiles > 0) {
       const uint32_t id = ptx::idesc_f16(1, 0, 0, 128, 64);    // GEMM1: K-major x K-major, N = 64 (hi | lo)
       const uint32_t id2 = ptx::idesc_f16(1, 1, 1, 128, 64);   // GEMM2: MN-major x MN-major, N = 64 (hi | lo)
       // Descriptors are built once; a step along K or to another slot adds its byte
@@ -237,9 +243,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint64_t qdesc0 = ptx::smem_desc(ptx::smem_u32(q_s), 16, 1024, 2);
       const uint64_t vdesc0 = ptx::smem_desc(ptx::smem_u32(ring), kSubBytes, 1024, 2);
       const uint64_t pdesc0 = ptx::smem_desc(ptx::smem_u32(p_s), 128, 2048, 0);
-      bool ok = wait_b(&aux->q_full, 0, aux, p.err);
+      bool ok = wait_w(&aux->q_full, 0, aux, p.err);
       ptx::tc_fence_after();
-      trace_stamp(p, 2);
+      if (lane == 0) trace_stamp(p, 2);
       int pos = 0;
       for (int u = 0; u < nunits && ok; ++u) {
         int tile;
@@ -248,33 +254,34 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!isv) {
           // GEMM1(tile): S[tile % 2] = Z_k [q~_hi | q~_lo]^T
           const int sb2 = tile & 1;
-          if (tile >= 2 && !(ok = wait_b(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
+          if (tile >= 2 && !(ok = wait_w(&aux->s_empty[sb2], ((tile - 2) >> 1) & 1, aux, p.err))) break;
           ptx::tc_fence_after();
           const uint32_t d_s = tmem + kSCol + 64 * sb2;
           for (int c = 0; c < p.ck && ok; ++c, ++pos) {
             const int slot = pos % p.nslot;
-            if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+            if (!(ok = wait_w(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
             ptx::tc_fence_after();
             const uint64_t a0 = kdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
             const uint64_t b0 = qdesc0 + (uint64_t)((c * 2 * kQSubBytes) >> 4);
             const int nk = min(8, (p.r_k - c * 128) >> 4);
-            for (int kk = 0; kk < nk; ++kk) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
               const uint64_t ad = a0 + (uint64_t)((kk >> 2) * (kSubBytes >> 4) + (kk & 3) * 2);
               const uint64_t bd = b0 + (uint64_t)((kk >> 2) * (kQSubBytes >> 4) + (kk & 3) * 2);
-              ptx::mma_f16(d_s, ad, bd, id, (c | kk) ? 1u : 0u);
+              if (kk < nk) ptx::mma_f16_elect(d_s, ad, bd, id, (c | kk) ? 1u : 0u);
             }
-            ptx::mma_commit(&aux->slot_empty[slot]);
+            ptx::mma_commit_elect(&aux->slot_empty[slot]);
           }
           if (!ok) break;
-          ptx::mma_commit(&aux->s_full[sb2]);
-          if (tile < 16) trace_stamp(p, 3 + 4 * tile);
+          ptx::mma_commit_elect(&aux->s_full[sb2]);
+          if (tile < 16 && lane == 0) trace_stamp(p, 3 + 4 * tile);
         } else {
           // GEMM2(tile): O~ += Z_v^T [P_hi | P_lo]
-          if (!(ok = wait_b(&aux->p_full, tile & 1, aux, p.err))) break;
+          if (!(ok = wait_w(&aux->p_full, tile & 1, aux, p.err))) break;
           ptx::tc_fence_after();
           for (int c = 0; c < p.cv && ok; ++c, ++pos) {
             const int slot = pos % p.nslot;
-            if (!(ok = wait_b(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
+            if (!(ok = wait_w(&aux->slot_full[slot], (pos / p.nslot) & 1, aux, p.err))) break;
             ptx::tc_fence_after();
             const uint64_t a0 = vdesc0 + (uint64_t)((slot * kSlotBytes) >> 4);
             const uint32_t d_o = tmem + kOCol + c * 64;
@@ -282,16 +289,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int kt = 0; kt < 8; ++kt) {
               const uint64_t ad = a0 + (uint64_t)(kt * 128);
               const uint64_t bd = pdesc0 + (uint64_t)(kt * 16);
-              ptx::mma_f16(d_o, ad, bd, id2, (tile | kt) ? 1u : 0u);
+              ptx::mma_f16_elect(d_o, ad, bd, id2, (tile | kt) ? 1u : 0u);
             }
-            ptx::mma_commit(&aux->slot_empty[slot]);
+            ptx::mma_commit_elect(&aux->slot_empty[slot]);
           }
           if (!ok) break;
-          ptx::mma_commit(&aux->p_empty);
-          if (tile < 16) trace_stamp(p, 6 + 4 * tile);
+          ptx::mma_commit_elect(&aux->p_empty);
+          if (tile < 16 && lane == 0) trace_stamp(p, 6 + 4 * tile);
         }
       }
-      ptx::mma_commit(&aux->o_final);
+      ptx::mma_commit_elect(&aux->o_final);
       // the MMAs have completed before TMEM is freed, even if the epilogue aborted
       drain_wait(&aux->o_final, 0);
     }

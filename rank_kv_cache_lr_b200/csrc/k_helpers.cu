@@ -68,19 +68,21 @@ struct El<float> {
 };
 
 // ---- query projection -----------------------------------------------------------
-// One CTA per (32 rank rows of B_k,h, KV head h, sequence b), 256 threads; thread =
-// (rank row i, query head j of the group; heads beyond 8 in further passes):
-// q~_j[i] = s log2(e) sum_c B_k[i][h d + c] q_j[c].
+// One CTA per (32 rank rows of B_k,h, KV head h, group of kRows sequences), 256 threads;
+// thread = (rank row i, query head j of the group; heads beyond 8 in further passes), each
+// for every sequence of the CTA: q~_j[i] = s log2(e) sum_c B_k[i][h d + c] q_j[c].  The rows
+// of B_k are staged once for the CTA's sequences.
 // qt16 (tensor-core path), bf16 latents: rows [b][j] and [b][32 + j] of a [B][64][r_k]
 // bf16 array get hi = bf16(q~) and lo = bf16(q~ - hi), so that hi + lo carries q~ to ~16
 // significant bits.  int4 latents: row [b][j] of a [B][32][r_k] fp16 array gets fp16(q~),
 // each 8-rank run in the order 0,4,1,5,2,6,3,7 in which the int4 kernel expands codes.
 constexpr int kQRowsCta = 32;
+constexpr int kRows = 4;   // sequences per CTA of the small kernels
 
 struct QprojArgs {
   const void* q; const void* Bk; float* qt; float* qd; void* qt16;
   int qt16_fp16;          // 1: fp16 rows in int4 run order; 0: bf16 hi / lo rows
-  int Hq, Hkv, d, D, rk;
+  int Hq, Hkv, d, D, rk, B;
   float scale_log2;
   int want_latent;
   unsigned long long* span;   // timeline span, or null
@@ -98,20 +100,24 @@ __device__ __forceinline__ void qproj_stage(const QprojArgs& a, int rchunk, int 
 }
 
 template <typename T>
-__device__ __forceinline__ void qproj_main(const QprojArgs& a, int rchunk, int h, int b, uint8_t* smem) {
+__device__ __forceinline__ void qproj_main(const QprojArgs& a, int rchunk, int h, int b0, int B, uint8_t* smem) {
   const int d = a.d, G = a.Hq / a.Hkv, j0 = h * G;
   const int pitch = qproj_pitch<T>(d);
-  float* qs = reinterpret_cast<float*>(smem + (size_t)kQRowsCta * pitch);   // [G][d]
-  const size_t qoff = ((size_t)b * a.Hq + j0) * d;
-#pragma unroll 4
-  for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) {
-    const float v = El<T>::ld(a.q, qoff + idx);
-    qs[idx] = v;
-    if (a.qd && rchunk == 0) a.qd[qoff + idx] = v * a.scale_log2;
+  const int nb = min(kRows, B - b0);
+  float* qs_all = reinterpret_cast<float*>(smem + (size_t)kQRowsCta * pitch);   // [nb][G][d]
+  for (int idx = threadIdx.x; idx < nb * G * d; idx += blockDim.x) {
+    const int bb = idx / (G * d), e = idx - bb * (G * d);
+    const size_t qoff = ((size_t)(b0 + bb) * a.Hq + j0) * d + e;
+    const float v = El<T>::ld(a.q, qoff);
+    qs_all[idx] = v;
+    if (a.qd && rchunk == 0) a.qd[qoff] = v * a.scale_log2;
   }
   if (!a.want_latent) return;
   cp_async_wait_all();
   __syncthreads();
+  for (int bb = 0; bb < nb; ++bb) {
+  const int b = b0 + bb;
+  const float* qs = qs_all + (size_t)bb * G * d;
   const int r0 = rchunk * kQRowsCta;
   const int nr = min(kQRowsCta, a.rk - r0);
   const int t = threadIdx.x & 31;            // rank row within the chunk
@@ -148,6 +154,7 @@ __device__ __forceinline__ void qproj_main(const QprojArgs& a, int rchunk, int h
       q16[((size_t)b * 64 + 32 + j) * a.rk + i] = lo;
     }
   }
+  }
 }
 
 template <typename T>
@@ -157,19 +164,22 @@ __global__ void __launch_bounds__(256) k_qproj(QprojArgs a) {
   qproj_stage<T>(a, blockIdx.x, blockIdx.y, qsm);      // bases: stable data
   pdl_wait();
   pdl_trigger();
-  qproj_main<T>(a, blockIdx.x, blockIdx.y, blockIdx.z, qsm);
+  qproj_main<T>(a, blockIdx.x, blockIdx.y, blockIdx.z * kRows, a.B, qsm);
   span_end(a.span);
 }
 
 size_t qproj_smem(const lr_cache_desc& d, size_t es) {
-  return (size_t)kQRowsCta * (d.head_dim * es + 16) + (size_t)(d.n_q_heads / d.n_kv_heads) * d.head_dim * sizeof(float);
+  return (size_t)kQRowsCta * (d.head_dim * es + 16) +
+         (size_t)kRows * (d.n_q_heads / d.n_kv_heads) * d.head_dim * sizeof(float);
 }
 
 // ---- append -----------------------------------------------------------------------
-// One CTA per (32-coordinate chunk of K or V, sequence b): z[i] = sum_c x[c] A[c][i].
-// The chunk's columns of A ([D][32]) are staged before the grid-dependency wait; the
-// source row after it.  The 8 warps take fixed eighths of D and the partial sums are
-// added in a fixed order, so the projection does not depend on the storage kind.
+// One CTA per (32-coordinate chunk of K or V, group of kRows sequences):
+// z_b[i] = sum_c x_b[c] A[c][i].  The chunk's columns of A ([D][32]) are staged before the
+// grid-dependency wait (once for the CTA's sequences), the source rows after it.  The 8
+// warps take fixed eighths of D, each A element read once for all the rows, and the
+// partial sums are added in a fixed order, so the projection does not depend on the
+// storage kind.
 struct AppendArgs {
   const void* src_k; const void* src_v;   // rows to project (input or evicted ring rows)
   long long src_bstride;                  // elements between batch rows of src
@@ -195,9 +205,11 @@ __device__ __forceinline__ void append_stage(const AppendArgs& a, int x, uint8_t
 }
 
 template <typename T>
-__device__ __forceinline__ void append_main(const AppendArgs& a, int x, int b, uint8_t* smem, float (*red)[32]) {
+__device__ __forceinline__ void append_main(const AppendArgs& a, int x, int b0, uint8_t* smem,
+                                            float (*red)[kRows][32]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nproj = a.project ? (a.chunks_k + a.chunks_v) : 0;
+  const int nb = min(kRows, a.B - b0);
   constexpr int es = sizeof(T);
   if (x < nproj) {
     const bool is_k = x < a.chunks_k;
@@ -206,54 +218,71 @@ __device__ __forceinline__ void append_main(const AppendArgs& a, int x, int b, u
     const void* src = is_k ? a.src_k : a.src_v;
     const int ncol = min(32, r - ch * 32);
     const uint8_t* As = smem;                            // [D][32]
-    uint8_t* xs = smem + (size_t)a.D * 32 * es;          // [D]
-    const uint8_t* g = reinterpret_cast<const uint8_t*>(src) + (size_t)b * a.src_bstride * es;
-    for (int v = threadIdx.x; v < a.D * es / 16; v += blockDim.x) cp_async16(xs + v * 16, g + v * 16);
+    uint8_t* xs = smem + (size_t)a.D * 32 * es;          // [nb][D]
+    const int vrow = a.D * es / 16;
+    for (int v = threadIdx.x; v < nb * vrow; v += blockDim.x) {
+      const int bb = v / vrow, vv = v - bb * vrow;
+      const uint8_t* g = reinterpret_cast<const uint8_t*>(src) + (size_t)(b0 + bb) * a.src_bstride * es;
+      cp_async16(xs + (size_t)bb * a.D * es + vv * 16, g + vv * 16);
+    }
     cp_async_wait_all();
     __syncthreads();
     const int per = (((a.D + 7) / 8) + 7) & ~7;          // multiple of 8 (vector reads of x)
     const int cb = warp * per, ce = min(a.D, cb + per);
-    float z0 = 0.f, z1 = 0.f;
+    float z[kRows];
+#pragma unroll
+    for (int bb = 0; bb < kRows; ++bb) z[bb] = 0.f;
     if (lane < ncol) {
       for (int c = cb; c < ce; c += 8) {
-        float xv[8];
-        El<T>::lds8(xs + (size_t)c * es, xv);
+        float av[8];
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          z0 = fmaf(xv[e], El<T>::lds1(As + ((size_t)(c + e) * 32 + lane) * es), z0);
-          z1 = fmaf(xv[e + 1], El<T>::lds1(As + ((size_t)(c + e + 1) * 32 + lane) * es), z1);
+        for (int e = 0; e < 8; ++e) av[e] = El<T>::lds1(As + ((size_t)(c + e) * 32 + lane) * es);
+#pragma unroll
+        for (int bb = 0; bb < kRows; ++bb) {
+          if (bb < nb) {
+            float xv[8];
+            El<T>::lds8(xs + ((size_t)bb * a.D + c) * es, xv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) z[bb] = fmaf(xv[e], av[e], z[bb]);
+          }
         }
       }
     }
-    red[warp][lane] = z0 + z1;
-    __syncthreads();
-    if (warp == 0) {
-      float z = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) z += red[w][lane];
-      const long long row = (long long)b * a.cap + a.dst_slot;
-      store_latent_chunk(z, ch, r, a.kind, a.dtype, is_k ? a.Zk : a.Zv, is_k ? a.codes_k : a.codes_v,
+    for (int bb = 0; bb < kRows; ++bb) red[warp][bb][lane] = z[bb];
+    __syncthreads();
+    // warp w stores row w (the quantiser works on the 32 lanes of one chunk)
+    if (warp < nb) {
+      float zz = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) zz += red[w][warp][lane];
+      const long long row = (long long)(b0 + warp) * a.cap + a.dst_slot;
+      store_latent_chunk(zz, ch, r, a.kind, a.dtype, is_k ? a.Zk : a.Zv, is_k ? a.codes_k : a.codes_v,
                          is_k ? a.params_k : a.params_v, is_k ? a.Gk : a.Gv, row, !is_k);
     }
     return;
   }
-  // ring write of the exact new token of sequence b
+  // ring write of the exact new token of each sequence
   const bool is_k = (x - nproj) == 0;
-  const uint8_t* src = reinterpret_cast<const uint8_t*>(is_k ? a.new_k : a.new_v) + (size_t)b * a.D * es;
-  uint8_t* dst = reinterpret_cast<uint8_t*>(is_k ? a.win_k : a.win_v) + ((size_t)b * a.slots + a.new_slot) * a.D * es;
-  for (int v = threadIdx.x; v < a.D * es / 16; v += blockDim.x)
-    reinterpret_cast<uint4*>(dst)[v] = reinterpret_cast<const uint4*>(src)[v];
+  const int vrow = a.D * es / 16;
+  for (int v = threadIdx.x; v < nb * vrow; v += blockDim.x) {
+    const int bb = v / vrow, vv = v - bb * vrow;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(is_k ? a.new_k : a.new_v) + (size_t)(b0 + bb) * a.D * es;
+    uint8_t* dst =
+        reinterpret_cast<uint8_t*>(is_k ? a.win_k : a.win_v) + ((size_t)(b0 + bb) * a.slots + a.new_slot) * a.D * es;
+    reinterpret_cast<uint4*>(dst)[vv] = reinterpret_cast<const uint4*>(src)[vv];
+  }
 }
 
 template <typename T>
 __global__ void __launch_bounds__(256) k_append(AppendArgs a) {
   extern __shared__ __align__(16) uint8_t asm_[];
-  __shared__ float red[8][32];
+  __shared__ float red[8][kRows][32];
   span_begin(a.span);
   append_stage<T>(a, blockIdx.x, asm_);                 // bases: stable data
   pdl_wait();
   pdl_trigger();
-  append_main<T>(a, blockIdx.x, blockIdx.y, asm_, red);
+  append_main<T>(a, blockIdx.x, blockIdx.y * kRows, asm_, red);
   span_end(a.span);
 }
 
@@ -262,16 +291,16 @@ __global__ void __launch_bounds__(256) k_append(AppendArgs a) {
 template <typename T>
 __global__ void __launch_bounds__(256) k_step_pre(AppendArgs aa, QprojArgs qa, int x_app, int nchunks_q) {
   extern __shared__ __align__(16) uint8_t psm[];
-  __shared__ float red[8][32];
-  const int x = blockIdx.x, b = blockIdx.y;
+  __shared__ float red[8][kRows][32];
+  const int x = blockIdx.x, b0 = blockIdx.y * kRows;
   const int qx = x - x_app;
   span_begin(aa.span);
   if (x < x_app) append_stage<T>(aa, x, psm);
   else qproj_stage<T>(qa, qx % nchunks_q, qx / nchunks_q, psm);
   pdl_wait();
   pdl_trigger();
-  if (x < x_app) append_main<T>(aa, x, b, psm, red);
-  else qproj_main<T>(qa, qx % nchunks_q, qx / nchunks_q, b, psm);
+  if (x < x_app) append_main<T>(aa, x, b0, psm, red);
+  else qproj_main<T>(qa, qx % nchunks_q, qx / nchunks_q, b0, qa.B, psm);
   span_end(aa.span);
 }
 
@@ -547,7 +576,7 @@ QprojArgs make_qproj_args(const lr_cache* c, const void* q, bool tc) {
   a.qd = (rope || c->win_slots) ? (rope ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k) : nullptr;
   a.qt16 = tc ? c->qt16 : nullptr;
   a.qt16_fp16 = c->latent_kind == LK_INT4 ? 1 : 0;
-  a.Hq = d.n_q_heads; a.Hkv = d.n_kv_heads; a.d = d.head_dim; a.D = c->D; a.rk = d.rank_k;
+  a.Hq = d.n_q_heads; a.Hkv = d.n_kv_heads; a.d = d.head_dim; a.D = c->D; a.rk = d.rank_k; a.B = d.batch;
   a.scale_log2 = c->scale_log2;
   a.want_latent = rope ? 0 : 1;
   a.span = span_of(c->spans, SPAN_PRE);
@@ -589,7 +618,7 @@ AppendArgs make_append_args(const lr_cache* c, const void* k, const void* v) {
 
 int append_ctas(const AppendArgs& a) { return (a.project ? a.chunks_k + a.chunks_v : 0) + (a.new_k ? 2 : 0); }
 
-size_t append_smem(const lr_cache* c) { return (size_t)c->D * 32 * c->esize + (size_t)c->D * c->esize; }
+size_t append_smem(const lr_cache* c) { return (size_t)c->D * 32 * c->esize + (size_t)kRows * c->D * c->esize; }
 
 template <typename T>
 cudaError_t qproj_t(const lr_cache* c, const void* q, cudaStream_t s, bool tc, bool pdl = true) {
@@ -597,7 +626,7 @@ cudaError_t qproj_t(const lr_cache* c, const void* q, cudaStream_t s, bool tc, b
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_qproj<T>, optin_done);
   if (e != cudaSuccess) return e;
-  const dim3 grid(qproj_chunks(c), d.n_kv_heads, d.batch);
+  const dim3 grid(qproj_chunks(c), d.n_kv_heads, (d.batch + kRows - 1) / kRows);
   if (!pdl) return launch_serial(k_qproj<T>, grid, dim3(256), qproj_smem(d, sizeof(T)), s, make_qproj_args(c, q, tc));
   return launch_pdl(k_qproj<T>, grid, dim3(256), qproj_smem(d, sizeof(T)), s, make_qproj_args(c, q, tc));
 }
@@ -643,7 +672,7 @@ cudaError_t append_t(lr_cache* c, const void* k, const void* v, cudaStream_t s, 
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_append<T>, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_append<T>, dim3(append_ctas(a), c->desc.batch), dim3(256), append_smem(c), s, a);
+  return launch_pdl(k_append<T>, dim3(append_ctas(a), (c->desc.batch + kRows - 1) / kRows), dim3(256), append_smem(c), s, a);
 }
 
 template <typename T>
@@ -656,7 +685,8 @@ cudaError_t step_pre_t(lr_cache* c, const void* k, const void* v, const void* q,
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_step_pre<T>, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_step_pre<T>, dim3(x_app + nq * c->desc.n_kv_heads, c->desc.batch), dim3(256), smem, s, aa, qa,
+  return launch_pdl(k_step_pre<T>, dim3(x_app + nq * c->desc.n_kv_heads, (c->desc.batch + kRows - 1) / kRows), dim3(256),
+                    smem, s, aa, qa,
                     x_app, nq);
 }
 

@@ -57,6 +57,10 @@ static_assert(sizeof(Aux) <= kAuxBytes, "aux block");
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
   return tc::wait_b(bar, parity, &aux->abort_flag, err, aux->wait_ns);
 }
+// The same, by a whole warp with one verdict for all its lanes.
+__device__ __forceinline__ bool wait_w(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
+  return __all_sync(0xffffffffu, wait_b(bar, parity, aux, err));
+}
 
 __device__ __forceinline__ uint32_t tmem_cols_for(int r) { return r <= 256 ? 256u : 512u; }
 
@@ -128,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    {   // the whole warp runs the loop; an elected lane issues
       // N per MMA: the whole rank, or 256 then the rest above 256 (the second MMA's B starts
       // at the fifth 64-rank box, its D at TMEM column 256)
       const int nh = r > 256 ? 2 : 1;
@@ -139,18 +143,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int k = 0; k < kb && ok; ++k) {
         const int s = k % p.nstage;
-        if (!(ok = wait_b(&aux->full[s], (k / p.nstage) & 1, aux, p.err))) break;
+        if (!(ok = wait_w(&aux->full[s], (k / p.nstage) & 1, aux, p.err))) break;
         ptx::tc_fence_after();
         const uint64_t xs = xdesc0 + (uint64_t)((s * stage_bytes) >> 4);
         const uint64_t as = adesc0 + (uint64_t)((s * stage_bytes) >> 4);
         for (int kk = 0; kk < 4; ++kk) {                // 16 dims per MMA: 32 B on X, 16 rows on A
           for (int hh = 0; hh < nh; ++hh)
-            ptx::mma_f16(tmem + hh * 256, xs + (uint64_t)(kk * 2),
+            ptx::mma_f16_elect(tmem + hh * 256, xs + (uint64_t)(kk * 2),
                          as + (uint64_t)((hh * 4 * kWBox + kk * 16 * 128) >> 4), hh ? id1 : id0, (k | kk) ? 1u : 0u);
         }
-        ptx::mma_commit(&aux->empty[s]);
+        ptx::mma_commit_elect(&aux->empty[s]);
       }
-      ptx::mma_commit(&aux->d_full);
+      ptx::mma_commit_elect(&aux->d_full);
       drain_wait(&aux->d_full, 0);                      // every MMA done before TMEM is freed
     }
     __syncwarp();

@@ -141,38 +141,58 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind)
 // ---------------------------------------------------------------------------
 // exact window (iS-KV): attention of the query heads of each KV head over that head's
 // window tokens, as one more partial (in head space, relative to its own max).  One CTA per
-// (KV head, sequence), 256 threads: the window is read once per KV head, staged through
-// shared memory kWinChunk tokens at a time, with an online softmax per query head (warp per
-// head for the max and sum; thread per (head, token) for the scores and per (head, column)
-// for the outputs).
+// (KV head, sequence), 256 threads.  The window is read once per KV head, kWinTok tokens at
+// a time: every key and value row of the round is in flight at once (16-byte cp.async into
+// padded rows), then thread per (head, token) for the scores, a warp per head for the
+// online max and sum, and thread per (head, column pair) for the outputs.
 // ---------------------------------------------------------------------------
-constexpr int kWinChunk = 32;
+constexpr int kWinTok = 64;
 
-size_t window_smem(int G, int d) {
-  return ((size_t)G * d * 2 + 2 * (size_t)kWinChunk * (d + 1) + (size_t)G * kWinChunk + 3 * (size_t)G) *
-         sizeof(float);
+__host__ __device__ inline int window_pitch(int d, int es) { return d * es + 16; }   // staged row, bytes
+
+size_t window_smem(int G, int d, int es) {
+  return (size_t)2 * G * d * sizeof(float) + (size_t)2 * kWinTok * window_pitch(d, es) +
+         ((size_t)G * kWinTok + 3 * (size_t)G) * sizeof(float);
+}
+
+__device__ __forceinline__ void load8(const uint8_t* s, int dtype, float (&v)[8]) {
+  if (dtype == LR_BF16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(s);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = __uint_as_float(w[k] << 16);
+      v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(s);
+    const float4 b = *reinterpret_cast<const float4*>(s + 16);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
 }
 
 __global__ void __launch_bounds__(256) k_window(const void* win_k, const void* win_v, const float* qd,
                                                 float* win_o, float* win_ml, int Hq, int Hkv, int d,
                                                 int D, int slots, int hist_len, int win_len, int dtype,
                                                 unsigned long long* span) {
-  extern __shared__ float wsm[];
+  extern __shared__ __align__(16) uint8_t wsm_raw[];
   const int G = Hq / Hkv;
-  const int kp = d + 1;                   // padded row pitch of the staged keys and values
-  float* q_s = wsm;                       // [G][d]
-  float* o_s = q_s + G * d;               // [G][d]
-  float* k_s = o_s + G * d;               // [kWinChunk][d + 1]
-  float* v_s = k_s + kWinChunk * kp;      // [kWinChunk][d + 1]
-  float* p_s = v_s + kWinChunk * kp;      // [G][kWinChunk]
-  float* m_s = p_s + G * kWinChunk;       // [G]
-  float* l_s = m_s + G;                   // [G]
-  float* a_s = l_s + G;                   // [G]
+  const int es = dtype == LR_BF16 ? 2 : 4;
+  const int pitch = window_pitch(d, es);
+  float* q_s = reinterpret_cast<float*>(wsm_raw);          // [G][d]
+  float* o_s = q_s + G * d;                                // [G][d]
+  uint8_t* k_s = reinterpret_cast<uint8_t*>(o_s + G * d);  // [kWinTok] rows of `pitch` bytes
+  uint8_t* v_s = k_s + kWinTok * pitch;
+  float* p_s = reinterpret_cast<float*>(v_s + kWinTok * pitch);   // [G][kWinTok]
+  float* m_s = p_s + G * kWinTok;                          // [G]
+  float* l_s = m_s + G;                                    // [G]
+  float* a_s = l_s + G;                                    // [G]
   span_begin(span);
   pdl_wait();
   pdl_trigger();
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
   const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
+  const int vpr = d * es / 16;                             // 16-byte vectors per row
   for (int idx = tid; idx < G * d; idx += nt) {
     q_s[idx] = qd[((long long)b * Hq + h * G) * d + idx];
     o_s[idx] = 0.f;
@@ -181,39 +201,52 @@ __global__ void __launch_bounds__(256) k_window(const void* win_k, const void* w
     m_s[u] = -INFINITY;
     l_s[u] = 0.f;
   }
-  for (int t0 = 0; t0 < win_len; t0 += kWinChunk) {
-    const int n = min(kWinChunk, win_len - t0);
-    __syncthreads();
-    for (int idx = tid; idx < n * d; idx += nt) {
-      const int t = idx / d, c = idx - (idx / d) * d;
-      const long long off = ((long long)b * slots + (hist_len + t0 + t) % slots) * D + (long long)h * d + c;
-      k_s[t * kp + c] = elem_f(win_k, off, dtype);
-      v_s[t * kp + c] = elem_f(win_v, off, dtype);
+  for (int t0 = 0; t0 < win_len; t0 += kWinTok) {
+    const int n = min(kWinTok, win_len - t0);
+    __syncthreads();   // the previous round's rows and weights are no longer read
+    for (int idx = tid; idx < 2 * n * vpr; idx += nt) {
+      const int kv = idx / (n * vpr), r = idx - kv * (n * vpr);
+      const int t = r / vpr, v = r - (r / vpr) * vpr;
+      const long long row = (long long)b * slots + (hist_len + t0 + t) % slots;
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(kv ? win_v : win_k) + (row * D + (long long)h * d) * es;
+      cp_async16((kv ? v_s : k_s) + t * pitch + v * 16, src + v * 16);
     }
+    cp_async_wait_all();
     __syncthreads();
+    // scores: thread per (head u, token t)
     for (int idx = tid; idx < G * n; idx += nt) {
       const int u = idx / n, t = idx - (idx / n) * n;
       const float* qv = q_s + u * d;
-      const float* kv = k_s + t * kp;
+      const uint8_t* kr = k_s + t * pitch;
       float s0 = 0.f, s1 = 0.f;
-      for (int c = 0; c + 1 < d; c += 2) {
-        s0 = fmaf(qv[c], kv[c], s0);
-        s1 = fmaf(qv[c + 1], kv[c + 1], s1);
+      for (int c = 0; c < d; c += 8) {
+        float kf[8];
+        load8(kr + c * es, dtype, kf);
+        const float4 qa = *reinterpret_cast<const float4*>(qv + c);
+        const float4 qb = *reinterpret_cast<const float4*>(qv + c + 4);
+        s0 = fmaf(qa.x, kf[0], s0); s1 = fmaf(qa.y, kf[1], s1);
+        s0 = fmaf(qa.z, kf[2], s0); s1 = fmaf(qa.w, kf[3], s1);
+        s0 = fmaf(qb.x, kf[4], s0); s1 = fmaf(qb.y, kf[5], s1);
+        s0 = fmaf(qb.z, kf[6], s0); s1 = fmaf(qb.w, kf[7], s1);
       }
-      p_s[u * kWinChunk + t] = s0 + s1;
+      p_s[u * kWinTok + t] = s0 + s1;
     }
     __syncthreads();
+    // online max and sum, a warp per head (two tokens per lane)
     for (int u = warp; u < G; u += nw) {
-      const float sc = lane < n ? p_s[u * kWinChunk + lane] : -INFINITY;
-      float mx = sc;
+      const float sa = lane < n ? p_s[u * kWinTok + lane] : -INFINITY;
+      const float sb = lane + 32 < n ? p_s[u * kWinTok + lane + 32] : -INFINITY;
+      float mx = fmaxf(sa, sb);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       const float mo = m_s[u], mn = fmaxf(mo, mx);
-      const float pv = lane < n ? exp2f(sc - mn) : 0.f;
-      float sum = pv;
+      const float pa = lane < n ? exp2f(sa - mn) : 0.f;
+      const float pb = lane + 32 < n ? exp2f(sb - mn) : 0.f;
+      float sum = pa + pb;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane < n) p_s[u * kWinChunk + lane] = pv;
+      if (lane < n) p_s[u * kWinTok + lane] = pa;
+      if (lane + 32 < n) p_s[u * kWinTok + lane + 32] = pb;
       if (lane == 0) {
         const float alpha = mo == -INFINITY ? 0.f : exp2f(mo - mn);
         a_s[u] = alpha;
@@ -222,11 +255,28 @@ __global__ void __launch_bounds__(256) k_window(const void* win_k, const void* w
       }
     }
     __syncthreads();
-    for (int idx = tid; idx < G * d; idx += nt) {
-      const int u = idx / d, c = idx - (idx / d) * d;
-      float o = o_s[idx] * a_s[u];
-      for (int t = 0; t < n; ++t) o = fmaf(p_s[u * kWinChunk + t], v_s[t * kp + c], o);
-      o_s[idx] = o;
+    // outputs: thread per (head u, column pair c)
+    for (int idx = tid; idx < G * (d / 2); idx += nt) {
+      const int u = idx / (d / 2), c = 2 * (idx - (idx / (d / 2)) * (d / 2));
+      const float a = a_s[u];
+      float o0 = o_s[u * d + c] * a, o1 = o_s[u * d + c + 1] * a;
+      const float* pu = p_s + u * kWinTok;
+      for (int t = 0; t < n; ++t) {
+        float v0, v1;
+        if (dtype == LR_BF16) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(v_s + t * pitch + c * 2);
+          v0 = __uint_as_float(w << 16);
+          v1 = __uint_as_float(w & 0xFFFF0000u);
+        } else {
+          const float2 f = *reinterpret_cast<const float2*>(v_s + t * pitch + c * 4);
+          v0 = f.x;
+          v1 = f.y;
+        }
+        o0 = fmaf(pu[t], v0, o0);
+        o1 = fmaf(pu[t], v1, o1);
+      }
+      o_s[u * d + c] = o0;
+      o_s[u * d + c + 1] = o1;
     }
   }
   __syncthreads();
@@ -387,7 +437,7 @@ cudaError_t launch_decode_simt(const lr_cache* c, int n_splits, int split_tokens
 cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
   const lr_cache_desc& d = c->desc;
   const float* qd = d.rope_in_kernel ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k;
-  const size_t smem = window_smem(d.n_q_heads / d.n_kv_heads, d.head_dim);
+  const size_t smem = window_smem(d.n_q_heads / d.n_kv_heads, d.head_dim, (int)c->esize);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   dim3 grid(d.n_kv_heads, d.batch);
   static std::atomic<uint32_t> optin_done{0};

@@ -64,6 +64,10 @@ struct SyncState {
 __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
   return tc::wait_b(bar, parity, &aux->abort_flag, err, aux->wait_ns);
 }
+// The same, by a whole warp with one verdict for all its lanes.
+__device__ __forceinline__ bool wait_w(uint64_t* bar, uint32_t parity, Aux* aux, int* err) {
+  return __all_sync(0xffffffffu, wait_b(bar, parity, aux, err));
+}
 
 // unit u -> (side, sequence, first token)
 __device__ __forceinline__ void unit_of(const SyncParams& p, int u, int* side, int* b, int* t0) {
@@ -155,37 +159,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0 && my_units > 0) {
+    if (my_units > 0) {   // the whole warp runs the loop; an elected lane issues
       const uint32_t id = ptx::idesc_f16(1, 0, 1, 128, (uint32_t)p.r);   // bf16; A K-major, B MN-major
       const uint64_t adesc0 = ptx::smem_desc(ptx::smem_u32(z_s), 16, 1024, 2);
       const uint64_t bdesc0 = ptx::smem_desc(ptx::smem_u32(r_s), kRBox, 1024, 2);
       bool ok = true;
       int rpos = 0, dcommits = 0;
       for (int i = 0; i < my_units && ok; ++i) {
-        if (!(ok = wait_b(&aux->z_full, i & 1, aux, p.err))) break;
-        if (i > 0 && !(ok = wait_b(&aux->d_empty, (i - 1) & 1, aux, p.err))) break;
+        if (!(ok = wait_w(&aux->z_full, i & 1, aux, p.err))) break;
+        if (i > 0 && !(ok = wait_w(&aux->d_empty, (i - 1) & 1, aux, p.err))) break;
         ptx::tc_fence_after();
         for (int kc = 0; kc < p.kb && ok; ++kc, ++rpos) {
           const int slot = rpos & 1;
-          if (!(ok = wait_b(&aux->r_full[slot], (rpos >> 1) & 1, aux, p.err))) break;
+          if (!(ok = wait_w(&aux->r_full[slot], (rpos >> 1) & 1, aux, p.err))) break;
           ptx::tc_fence_after();
           const uint64_t bs = bdesc0 + (uint64_t)((slot * p.r_slot) >> 4);
           const int nk = std::min(4, (p.r - kc * 64) >> 4);
           for (int kk = 0; kk < nk; ++kk) {
             const uint64_t ad = adesc0 + (uint64_t)((kc * kSubBytes + kk * 32) >> 4);
             const uint64_t bd = bs + (uint64_t)((kk * 2048) >> 4);   // 16 k-rows of 128 B
-            ptx::mma_f16(tmem, ad, bd, id, (kc | kk) ? 1u : 0u);
-            ptx::mma_f16(tmem, ad, bd + (uint64_t)(p.r_half >> 4), id, 1u);
+            ptx::mma_f16_elect(tmem, ad, bd, id, (kc | kk) ? 1u : 0u);
+            ptx::mma_f16_elect(tmem, ad, bd + (uint64_t)(p.r_half >> 4), id, 1u);
           }
-          ptx::mma_commit(&aux->r_empty[slot]);
+          ptx::mma_commit_elect(&aux->r_empty[slot]);
         }
         if (!ok) break;
-        ptx::mma_commit(&aux->d_full);
+        ptx::mma_commit_elect(&aux->d_full);
         ++dcommits;
       }
       // every MMA issued so far completes before TMEM is freed, even if the epilogue aborted
       (void)dcommits;
-      ptx::mma_commit(&aux->fin);
+      ptx::mma_commit_elect(&aux->fin);
       drain_wait(&aux->fin, 0);
     }
     __syncwarp();
