@@ -105,12 +105,46 @@ __device__ __forceinline__ void qproj_main(const QprojArgs& a, int rchunk, int h
   const int pitch = qproj_pitch<T>(d);
   const int nb = min(kRows, B - b0);
   float* qs_all = reinterpret_cast<float*>(smem + (size_t)kQRowsCta * pitch);   // [nb][G][d]
-  for (int idx = threadIdx.x; idx < nb * G * d; idx += blockDim.x) {
-    const int bb = idx / (G * d), e = idx - bb * (G * d);
-    const size_t qoff = ((size_t)(b0 + bb) * a.Hq + j0) * d + e;
-    const float v = El<T>::ld(a.q, qoff);
-    qs_all[idx] = v;
-    if (a.qd && rchunk == 0) a.qd[qoff] = v * a.scale_log2;
+  // the query rows of the group, 16-byte vectors, all of a thread's loads issued before its
+  // first store (a store between dependent loads would serialise their latencies)
+  {
+    constexpr int kVec = 16 / sizeof(T);                // elements per vector
+    constexpr int kPer = 4;                             // vectors in flight per thread
+    const int nvec = nb * G * d / kVec;                 // G d is a multiple of 8
+    for (int v0 = threadIdx.x; v0 < nvec; v0 += kPer * blockDim.x) {
+      uint4 raw[kPer];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int v = v0 + k * blockDim.x;
+        if (v < nvec) {
+          const int e0 = v * kVec, bb = e0 / (G * d), e = e0 - bb * (G * d);
+          raw[k] = __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + ((size_t)(b0 + bb) * a.Hq + j0) * d + e));
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int v = v0 + k * blockDim.x;
+        if (v < nvec) {
+          const int e0 = v * kVec, bb = e0 / (G * d), e = e0 - bb * (G * d);
+          float f[8];
+          if constexpr (sizeof(T) == 2) {
+            El<T>::lds8(reinterpret_cast<const uint8_t*>(&raw[k]), f);
+          } else {
+            f[0] = __uint_as_float(raw[k].x);
+            f[1] = __uint_as_float(raw[k].y);
+            f[2] = __uint_as_float(raw[k].z);
+            f[3] = __uint_as_float(raw[k].w);
+          }
+#pragma unroll
+          for (int m = 0; m < kVec; ++m) qs_all[e0 + m] = f[m];
+          if (a.qd && rchunk == 0) {
+            float* qd = a.qd + ((size_t)(b0 + bb) * a.Hq + j0) * d + e;
+#pragma unroll
+            for (int m = 0; m < kVec; ++m) qd[m] = f[m] * a.scale_log2;
+          }
+        }
+      }
+    }
   }
   if (!a.want_latent) return;
   cp_async_wait_all();

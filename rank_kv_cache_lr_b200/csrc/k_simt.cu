@@ -193,10 +193,9 @@ __global__ void __launch_bounds__(256) k_window(const void* win_k, const void* w
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
   const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
   const int vpr = d * es / 16;                             // 16-byte vectors per row
-  for (int idx = tid; idx < G * d; idx += nt) {
-    q_s[idx] = qd[((long long)b * Hq + h * G) * d + idx];
-    o_s[idx] = 0.f;
-  }
+  // the scaled queries of the group (fp32, 16-byte vectors) come in with the first round's rows
+  for (int v = tid; v < G * d / 4; v += nt) cp_async16(q_s + 4 * v, qd + ((long long)b * Hq + h * G) * d + 4 * v);
+  for (int idx = tid; idx < G * d; idx += nt) o_s[idx] = 0.f;
   for (int u = tid; u < G; u += nt) {
     m_s[u] = -INFINITY;
     l_s[u] = 0.f;
@@ -279,6 +278,7 @@ __global__ void __launch_bounds__(256) k_window(const void* win_k, const void* w
       o_s[u * d + c + 1] = o1;
     }
   }
+  cp_async_wait_all();   // (no window tokens: the query copies still complete)
   __syncthreads();
   for (int idx = tid; idx < G * d; idx += nt) win_o[((long long)b * Hq + h * G) * d + idx] = o_s[idx];
   for (int u = tid; u < G; u += nt) {
