@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(256) k_step_pre(AppendArgs aa, QprojArgs qa, i
 }
 
 // ---- split merge and output projection ------------------------------------------
-// A cluster of ncb = ceil(d / 32) CTAs per (KV head h, sequence b), 128 threads each; CTA p
+// A cluster of ncb = ceil(d / 32) CTAs per (KV head h, sequence b), 256 threads each; CTA p
 // of the cluster owns output columns [32 p, +32) of the group's heads and ranks
 // [p rp, +rp) of the merge.  Per pass of up to 8 query heads:
 //   1. the split weights (log-sum-exp over the splits and the window partial; a warp per
@@ -348,15 +348,15 @@ __global__ void __launch_bounds__(256) k_step_pre(AppendArgs aa, QprojArgs qa, i
 //      (head, 4 ranks), float4 loads of up to 16 splits in flight);
 //   3. the parts are exchanged through distributed shared memory, so every CTA holds the
 //      whole o~_j of the pass, and projected: o_j = o~_j B_v,h / l_j for its columns
-//      (thread = column x quarter of the ranks, quarters added in a fixed order).
+//      (thread = column x eighth of the ranks, eighths added in a fixed order).
 // The columns of B_v,h (no in-flight kernel writes them) are staged before the
 // grid-dependency wait.  The exchange keeps every load of the partials issued once per
 // cluster and the dependent global-load rounds at two (the (m, l) pairs and the partials,
 // issued together).
-constexpr int kMergeThreads = 128;
+constexpr int kMergeThreads = 256;
 constexpr int kMergeHeads = 8;       // query heads per pass
 constexpr int kMergeCols = 32;       // output columns per CTA
-constexpr int kMergeLoads = 16;      // split loads in flight per thread
+constexpr int kMergeLoads = 12;      // split loads in flight per thread
 
 struct MergeArgs {
   const float* part_o; const float* part_ml; const float* win_o; const float* win_ml;
@@ -403,14 +403,14 @@ __host__ __device__ inline MergeSmem merge_layout(int rv, int rp, int S, int es)
   L.otf = o; o += (size_t)kMergeHeads * (rv + 4) * 4;                        // [8][rv + 4] whole o~
   L.mls = o; o += (size_t)kMergeHeads * S * 8;                               // [8][S] (m, l)
   L.wsm = o; o += ((size_t)kMergeHeads * S * 4 + 15) / 16 * 16;              // [8][S] weights
-  L.red = o; o += (size_t)4 * kMergeHeads * kMergeCols * 4;                  // [4][8][32]
+  L.red = o; o += (size_t)(kMergeThreads / 32) * kMergeHeads * kMergeCols * 4;   // [8][8][32]
   L.hdr = o; o += (size_t)kMergeHeads * 4 * 4;                               // [8]{m, 1/l, w_win, l}
   L.total = o;
   return L;
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kMergeThreads, 1) k_merge(MergeArgs a) {
+__global__ void __launch_bounds__(kMergeThreads, 2) k_merge(MergeArgs a) {
   extern __shared__ __align__(16) uint8_t msm[];
   constexpr int es = sizeof(T);
   const int p = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
@@ -542,10 +542,11 @@ __global__ void __launch_bounds__(kMergeThreads, 1) k_merge(MergeArgs a) {
     // the parts have been read everywhere before any CTA overwrites its own (next pass) or
     // exits; the gathered rows and the staged columns are visible to the whole CTA
     cluster_sync_all();
-    // projection partial sums: column c, quarter rq of the ranks, every head of the pass
+    // projection partial sums: column c, eighth rq of the ranks, every head of the pass
     {
+      constexpr int kParts = kMergeThreads / 32;
       const int c = tid & 31, rq = tid >> 5;
-      const int rql = ((rv + 15) / 16) * 4;                  // ranks per quarter, multiple of 4
+      const int rql = ((rv + 4 * kParts - 1) / (4 * kParts)) * 4;   // ranks per part, multiple of 4
       const int r0 = min(rv, rq * rql), r1 = min(rv, r0 + rql);
       float acc[kMergeHeads];
 #pragma unroll
@@ -571,13 +572,13 @@ __global__ void __launch_bounds__(kMergeThreads, 1) k_merge(MergeArgs a) {
       for (int u = 0; u < kMergeHeads; ++u) red[(rq * kMergeHeads + u) * kMergeCols + c] = acc[u];
     }
     __syncthreads();
-    // quarters added in order; window partial; normalisation; store
+    // parts added in order; window partial; normalisation; store
     for (int e = tid; e < nh * kMergeCols; e += kMergeThreads) {
       const int u = e / kMergeCols, cc = e % kMergeCols;
       if (cc >= ncols) continue;
       float o = red[u * kMergeCols + cc];
 #pragma unroll
-      for (int q = 1; q < 4; ++q) o += red[(q * kMergeHeads + u) * kMergeCols + cc];
+      for (int q = 1; q < kMergeThreads / 32; ++q) o += red[(q * kMergeHeads + u) * kMergeCols + cc];
       const int j = h * G + jb + u;
       const size_t oi = ((size_t)b * a.Hq + j) * a.d + c0 + cc;
       if (a.win_o) o = fmaf(hdr[u * 4 + 2], a.win_o[oi], o);

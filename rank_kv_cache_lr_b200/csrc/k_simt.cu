@@ -139,20 +139,22 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind)
 }
 
 // ---------------------------------------------------------------------------
-// exact window (iS-KV): attention of the query heads of each KV head over that head's
-// window tokens, as one more partial (in head space, relative to its own max).  One CTA per
-// (KV head, sequence), 256 threads.  The window is read once per KV head, kWinTok tokens at
-// a time: every key and value row of the round is in flight at once (16-byte cp.async into
-// padded rows), then thread per (head, token) for the scores, a warp per head for the
-// online max and sum, and thread per (head, column pair) for the outputs.
+// exact window (iS-KV): attention of each query head over its KV head's window tokens, as
+// one more partial (in head space, relative to its own max).  One CTA per (KV head,
+// sequence, query head of the group), 128 threads; the window rows come kWinTok tokens at a
+// time with every row of the round in flight at once (16-byte cp.async into padded rows),
+// then thread per token for the scores, a block-wide max and sum, and thread per column
+// for the output.
 // ---------------------------------------------------------------------------
-constexpr int kWinTok = 64;
+constexpr int kWinTok = 128;
+constexpr int kWinThreads = 128;
 
 __host__ __device__ inline int window_pitch(int d, int es) { return d * es + 16; }   // staged row, bytes
 
 size_t window_smem(int G, int d, int es) {
-  return (size_t)2 * G * d * sizeof(float) + (size_t)2 * kWinTok * window_pitch(d, es) +
-         ((size_t)G * kWinTok + 3 * (size_t)G) * sizeof(float);
+  (void)G;
+  return (size_t)2 * d * sizeof(float) + (size_t)2 * kWinTok * window_pitch(d, es) +
+         (size_t)(kWinTok + 16) * sizeof(float);
 }
 
 __device__ __forceinline__ void load8(const uint8_t* s, int dtype, float (&v)[8]) {
@@ -171,39 +173,36 @@ __device__ __forceinline__ void load8(const uint8_t* s, int dtype, float (&v)[8]
   }
 }
 
-__global__ void __launch_bounds__(256) k_window(const void* win_k, const void* win_v, const float* qd,
-                                                float* win_o, float* win_ml, int Hq, int Hkv, int d,
-                                                int D, int slots, int hist_len, int win_len, int dtype,
-                                                unsigned long long* span) {
+__global__ void __launch_bounds__(kWinThreads) k_window(const void* win_k, const void* win_v, const float* qd,
+                                                        float* win_o, float* win_ml, int Hq, int Hkv, int d,
+                                                        int D, int slots, int hist_len, int win_len, int dtype,
+                                                        unsigned long long* span) {
   extern __shared__ __align__(16) uint8_t wsm_raw[];
   const int G = Hq / Hkv;
   const int es = dtype == LR_BF16 ? 2 : 4;
   const int pitch = window_pitch(d, es);
-  float* q_s = reinterpret_cast<float*>(wsm_raw);          // [G][d]
-  float* o_s = q_s + G * d;                                // [G][d]
-  uint8_t* k_s = reinterpret_cast<uint8_t*>(o_s + G * d);  // [kWinTok] rows of `pitch` bytes
+  float* q_s = reinterpret_cast<float*>(wsm_raw);          // [d]
+  float* o_s = q_s + d;                                    // [d] (unused slot kept for alignment)
+  uint8_t* k_s = reinterpret_cast<uint8_t*>(o_s + d);      // [kWinTok] rows of `pitch` bytes
   uint8_t* v_s = k_s + kWinTok * pitch;
-  float* p_s = reinterpret_cast<float*>(v_s + kWinTok * pitch);   // [G][kWinTok]
-  float* m_s = p_s + G * kWinTok;                          // [G]
-  float* l_s = m_s + G;                                    // [G]
-  float* a_s = l_s + G;                                    // [G]
+  float* p_s = reinterpret_cast<float*>(v_s + kWinTok * pitch);   // [kWinTok]
+  float* red = p_s + kWinTok;                              // [8]: warp maxima, then warp sums
   span_begin(span);
   pdl_wait();
   pdl_trigger();
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
-  const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
+  const int h = blockIdx.x, b = blockIdx.y, u = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  constexpr int nw = kWinThreads / 32;
+  const int j = h * G + u;                                 // query head
   const int vpr = d * es / 16;                             // 16-byte vectors per row
-  // the scaled queries of the group (fp32, 16-byte vectors) come in with the first round's rows
-  for (int v = tid; v < G * d / 4; v += nt) cp_async16(q_s + 4 * v, qd + ((long long)b * Hq + h * G) * d + 4 * v);
-  for (int idx = tid; idx < G * d; idx += nt) o_s[idx] = 0.f;
-  for (int u = tid; u < G; u += nt) {
-    m_s[u] = -INFINITY;
-    l_s[u] = 0.f;
-  }
+  for (int v = tid; v < d / 4; v += kWinThreads) cp_async16(q_s + 4 * v, qd + ((long long)b * Hq + j) * d + 4 * v);
+  float m = -INFINITY, l = 0.f;
+  float o = 0.f;                                           // output column tid (d <= 128 here: tid < d)
+  float o2 = 0.f;                                          // column tid + 128 (d > 128)
   for (int t0 = 0; t0 < win_len; t0 += kWinTok) {
     const int n = min(kWinTok, win_len - t0);
     __syncthreads();   // the previous round's rows and weights are no longer read
-    for (int idx = tid; idx < 2 * n * vpr; idx += nt) {
+    for (int idx = tid; idx < 2 * n * vpr; idx += kWinThreads) {
       const int kv = idx / (n * vpr), r = idx - kv * (n * vpr);
       const int t = r / vpr, v = r - (r / vpr) * vpr;
       const long long row = (long long)b * slots + (hist_len + t0 + t) % slots;
@@ -212,78 +211,67 @@ __global__ void __launch_bounds__(256) k_window(const void* win_k, const void* w
     }
     cp_async_wait_all();
     __syncthreads();
-    // scores: thread per (head u, token t)
-    for (int idx = tid; idx < G * n; idx += nt) {
-      const int u = idx / n, t = idx - (idx / n) * n;
-      const float* qv = q_s + u * d;
-      const uint8_t* kr = k_s + t * pitch;
+    // score of token tid (kWinTok = blockDim: one token per thread)
+    float sc = -INFINITY;
+    if (tid < n) {
+      const uint8_t* kr = k_s + tid * pitch;
       float s0 = 0.f, s1 = 0.f;
       for (int c = 0; c < d; c += 8) {
         float kf[8];
         load8(kr + c * es, dtype, kf);
-        const float4 qa = *reinterpret_cast<const float4*>(qv + c);
-        const float4 qb = *reinterpret_cast<const float4*>(qv + c + 4);
+        const float4 qa = *reinterpret_cast<const float4*>(q_s + c);
+        const float4 qb = *reinterpret_cast<const float4*>(q_s + c + 4);
         s0 = fmaf(qa.x, kf[0], s0); s1 = fmaf(qa.y, kf[1], s1);
         s0 = fmaf(qa.z, kf[2], s0); s1 = fmaf(qa.w, kf[3], s1);
         s0 = fmaf(qb.x, kf[4], s0); s1 = fmaf(qb.y, kf[5], s1);
         s0 = fmaf(qb.z, kf[6], s0); s1 = fmaf(qb.w, kf[7], s1);
       }
-      p_s[u * kWinTok + t] = s0 + s1;
+      sc = s0 + s1;
     }
-    __syncthreads();
-    // online max and sum, a warp per head (two tokens per lane)
-    for (int u = warp; u < G; u += nw) {
-      const float sa = lane < n ? p_s[u * kWinTok + lane] : -INFINITY;
-      const float sb = lane + 32 < n ? p_s[u * kWinTok + lane + 32] : -INFINITY;
-      float mx = fmaxf(sa, sb);
+    // block max, weights, block sum (every thread keeps the same m and l)
+    float mx = sc;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float mo = m_s[u], mn = fmaxf(mo, mx);
-      const float pa = lane < n ? exp2f(sa - mn) : 0.f;
-      const float pb = lane + 32 < n ? exp2f(sb - mn) : 0.f;
-      float sum = pa + pb;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane < n) p_s[u * kWinTok + lane] = pa;
-      if (lane + 32 < n) p_s[u * kWinTok + lane + 32] = pb;
-      if (lane == 0) {
-        const float alpha = mo == -INFINITY ? 0.f : exp2f(mo - mn);
-        a_s[u] = alpha;
-        l_s[u] = l_s[u] * alpha + sum;
-        m_s[u] = mn;
-      }
-    }
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) red[warp] = mx;
     __syncthreads();
-    // outputs: thread per (head u, column pair c)
-    for (int idx = tid; idx < G * (d / 2); idx += nt) {
-      const int u = idx / (d / 2), c = 2 * (idx - (idx / (d / 2)) * (d / 2));
-      const float a = a_s[u];
-      float o0 = o_s[u * d + c] * a, o1 = o_s[u * d + c + 1] * a;
-      const float* pu = p_s + u * kWinTok;
-      for (int t = 0; t < n; ++t) {
-        float v0, v1;
-        if (dtype == LR_BF16) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(v_s + t * pitch + c * 2);
-          v0 = __uint_as_float(w << 16);
-          v1 = __uint_as_float(w & 0xFFFF0000u);
-        } else {
-          const float2 f = *reinterpret_cast<const float2*>(v_s + t * pitch + c * 4);
-          v0 = f.x;
-          v1 = f.y;
-        }
-        o0 = fmaf(pu[t], v0, o0);
-        o1 = fmaf(pu[t], v1, o1);
-      }
-      o_s[u * d + c] = o0;
-      o_s[u * d + c + 1] = o1;
+    mx = red[0];
+#pragma unroll
+    for (int w = 1; w < nw; ++w) mx = fmaxf(mx, red[w]);
+    const float mn = fmaxf(m, mx);
+    const float pv = tid < n ? exp2f(sc - mn) : 0.f;
+    p_s[tid] = pv;
+    float sum = pv;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    __syncthreads();   // red[] maxima read by everyone; p_s complete
+    if (lane == 0) red[nw + warp] = sum;
+    __syncthreads();
+    float st = red[nw];
+#pragma unroll
+    for (int w = 1; w < nw; ++w) st += red[nw + w];
+    const float alpha = m == -INFINITY ? 0.f : exp2f(m - mn);
+    l = l * alpha + st;
+    m = mn;
+    // output columns tid (and tid + 128)
+    o *= alpha;
+    o2 *= alpha;
+    for (int t = 0; t < n; ++t) {
+      const float p = p_s[t];
+      const uint8_t* vr = v_s + t * pitch;
+      if (tid < d) o = fmaf(p, dtype == LR_BF16 ? __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(vr + tid * 2)) << 16)
+                                                : *reinterpret_cast<const float*>(vr + tid * 4), o);
+      if (tid + kWinThreads < d)
+        o2 = fmaf(p, dtype == LR_BF16 ? __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(vr + (tid + kWinThreads) * 2)) << 16)
+                                      : *reinterpret_cast<const float*>(vr + (tid + kWinThreads) * 4), o2);
     }
   }
   cp_async_wait_all();   // (no window tokens: the query copies still complete)
-  __syncthreads();
-  for (int idx = tid; idx < G * d; idx += nt) win_o[((long long)b * Hq + h * G) * d + idx] = o_s[idx];
-  for (int u = tid; u < G; u += nt) {
-    win_ml[((long long)b * Hq + h * G + u) * 2] = m_s[u];
-    win_ml[((long long)b * Hq + h * G + u) * 2 + 1] = l_s[u];
+  const long long ob = ((long long)b * Hq + j) * d;
+  if (tid < d) win_o[ob + tid] = o;
+  if (tid + kWinThreads < d) win_o[ob + tid + kWinThreads] = o2;
+  if (tid == 0) {
+    win_ml[((long long)b * Hq + j) * 2] = m;
+    win_ml[((long long)b * Hq + j) * 2 + 1] = l;
   }
   span_end(span);
 }
@@ -439,11 +427,11 @@ cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
   const float* qd = d.rope_in_kernel ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k;
   const size_t smem = window_smem(d.n_q_heads / d.n_kv_heads, d.head_dim, (int)c->esize);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
-  dim3 grid(d.n_kv_heads, d.batch);
+  dim3 grid(d.n_kv_heads, d.batch, d.n_q_heads / d.n_kv_heads);
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_window, optin_done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_window, grid, dim3(256), smem, s, c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads, d.n_kv_heads,
+  return launch_pdl(k_window, grid, dim3(kWinThreads), smem, s, c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads, d.n_kv_heads,
                                    d.head_dim, c->D, c->win_slots, c->hist_len, c->win_len, d.dtype,
                                    span_of(c->spans, SPAN_WINDOW));
 }
