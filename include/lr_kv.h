@@ -235,6 +235,26 @@ lr_status lr_basis_sync(lr_cache* cache, const float* R_k, const float* R_v,
                         const void* B_k_new, const void* B_v_new, const void* A_k_new,
                         const void* A_v_new, void* stream);
 
+/* ---- basis update (iS-KV title and method section: a dynamically updated low-rank
+ *      basis kept current by a block-incremental SVD) ----------------------------------
+ * lr_basis_update — one block update of a truncated SVD, the textbook form of the step the
+ *   pages name: with the current basis rows B [r][D] of `side` (0 keys, 1 values) and the
+ *   Gram matrix S = Z^T Z of the history coordinates (Z = K_hist B^T), and a block of exact
+ *   rows K [n][D]: Y = K B^T, the residual P = K - Y B with orthonormal rows Q^T spanning it
+ *   (numerical rank: directions below 1e-6 of the block's largest row norm are dropped),
+ *   G = [[S + Y^T Y, Y^T Rp^T], [Rp Y, Rp Rp^T]] with Rp^T = P Q, and its r leading
+ *   eigenpairs (lam, V):  B' = V^T [B; Q^T],  R = V[:r, :],  S' = diag(lam).
+ *   B' spans the leading right singular subspace of [Z B; K] (Eckart-Young).
+ *   blk [n][D] dtype device, 16-byte aligned, 1 <= n <= 128 (else LR_ERR_INVALID_ARG).
+ *   gram [r][r] fp32 device: S on entry, S' on return.  R_out [r][r] fp32 device: the
+ *   history sync Z <- Z R, to be passed to lr_basis_sync with B' (and A').  B_new [r][D]
+ *   and A_new = B'^T [D][r] in dtype, device, or NULL.  The current basis must have
+ *   orthonormal rows (A = B^T).  Computed in fp64 on the GPU; the cache's latents are not
+ *   touched.  One latent group only (else LR_ERR_UNSUPPORTED).  Eigenvector signs follow a
+ *   fixed rule (the largest-magnitude entry of each column of V positive). */
+lr_status lr_basis_update(lr_cache* cache, int32_t side, const void* blk, int32_t n, float* gram,
+                          float* R_out, void* B_new, void* A_new, void* stream);
+
 /* ---- decode without device allocation ----------------------------------------
  * (No counterpart on the pages; this entry point exists for callers that cannot
  * allocate device memory at decode time: serving engines that reserve almost all HBM

@@ -7,7 +7,7 @@ and passed by pointer.  There is no fallback: if the library is missing,
 importing this package raises.
 
 Functions keep the C names: lr_cache_create, lr_cache_destroy, lr_kv_append, lr_decode_step,
-lr_kv_append_latent, lr_attn_decode, lr_basis_sync, lr_cache_get_len,
+lr_kv_append_latent, lr_attn_decode, lr_basis_sync, lr_basis_update, lr_cache_get_len,
 lr_cache_truncate, lr_cache_view_get, lr_cache_set_path, lr_cache_plan,
 lr_plan_decode, lr_cache_set_kernel_events, lr_cache_set_trace, lr_device_error, lr_abi_struct_sizes,
 lr_status_string, lr_launch_count, lr_attn_decode_noalloc, lr_cache_set_wait_limit,
@@ -77,6 +77,7 @@ def _load() -> ctypes.CDLL:
         "lr_attn_decode": [vp, vp, vp, vp, vp],
         "lr_decode_step": [vp, vp, vp, vp, vp, vp, vp],
         "lr_basis_sync": [vp, vp, vp, vp, vp, vp, vp, vp],
+        "lr_basis_update": [vp, i32, vp, i32, vp, vp, vp, vp, vp],
         "lr_cache_get_len": [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)],
         "lr_cache_truncate": [vp, i32],
         "lr_cache_view_get": [vp, ctypes.POINTER(lr_cache_view)],
@@ -315,6 +316,24 @@ def lr_basis_sync(cache: Cache, R_k=None, R_v=None, B_k_new=None, B_v_new=None, 
                               _ptr(A_k_new, dt, ak, "A_k_new", True),
                               _ptr(A_v_new, dt, av, "A_v_new", True),
                               _stream(stream)), "lr_basis_sync")
+
+
+def lr_basis_update(cache: Cache, side: int, blk, gram, R_out, B_new=None, A_new=None, stream=None) -> None:
+    """Block-incremental SVD update of the keys' (side 0) or values' (side 1) basis from the
+    block blk [n][D] (cache dtype): gram [r][r] fp32 in S, out S'; R_out [r][r] fp32 the
+    history sync; B_new [r][D], A_new [D][r] (cache dtype) the new basis, or None."""
+    import torch
+    d, dt = cache.desc, _torch_dtype(cache.desc.dtype)
+    r = d.rank_k if side == 0 else d.rank_v
+    D = d.n_kv_heads * d.head_dim
+    if blk is None or blk.dim() != 2 or blk.shape[1] != D:
+        raise ValueError(f"blk must be [n][{D}]")
+    _check(_lib.lr_basis_update(cache.handle, int(side), _ptr(blk, dt, None, "blk"), int(blk.shape[0]),
+                                _ptr(gram, torch.float32, (r, r), "gram"),
+                                _ptr(R_out, torch.float32, (r, r), "R_out"),
+                                _ptr(B_new, dt, (r, D), "B_new", True),
+                                _ptr(A_new, dt, (D, r), "A_new", True),
+                                _stream(stream)), "lr_basis_update")
 
 
 LR_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024

@@ -122,6 +122,7 @@ void free_all(lr_cache* c) {
   if (!c) return;
   tc_release(c);
   sync_tc_release(c);
+  isvd_release(c);
   void* ptrs[] = {c->z_k, c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->win_k, c->win_v,
                   c->A_k, c->B_k, c->A_v, c->B_v, c->rope_cs, c->qt, c->qt16, c->part_o, c->part_ml,
                   c->win_o, c->win_ml, c->dev_err, c->r_full};
@@ -536,6 +537,18 @@ lr_status lr_basis_sync(lr_cache* c, const float* R_k, const float* R_v, const v
   if (e == cudaSuccess && A_v_new) e = install_basis(c, c->A_v, A_v_new, true, false, s);
   if (e == cudaSuccess && (B_k_new || B_v_new)) e = tc_prepare(c, s);
   return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
+}
+
+lr_status lr_basis_update(lr_cache* c, int32_t side, const void* blk, int32_t n, float* gram, float* R_out,
+                          void* B_new, void* A_new, void* stream) {
+  if (!c || !blk || !gram || !R_out || (side != 0 && side != 1)) return LR_ERR_INVALID_ARG;
+  if (n < 1 || n > 128) return LR_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(blk) & 15) return LR_ERR_INVALID_ARG;
+  if (c->groups > 1) return LR_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  cudaError_t e = launch_basis_update(c, side, blk, n, gram, R_out, B_new, A_new, s);
+  return e == cudaSuccess ? LR_OK : cuda_status(e);
 }
 
 lr_status lr_cache_get_len(const lr_cache* c, int32_t* len, int32_t* hist_len, int32_t* win_len) {

@@ -99,6 +99,7 @@ struct lr_cache {
   cudaStream_t last_stream = nullptr;
   void* tc_state = nullptr;    // tensor-core path state (tensor maps), owned
   void* sync_state = nullptr;  // tensor-core basis sync state (tensor maps, split R), owned
+  void* isvd_state = nullptr;  // block-incremental SVD working memory, owned
   cudaEvent_t ev_start = nullptr, ev_stop = nullptr;   // caller-owned kernel timing events
   unsigned long long* trace = nullptr;                 // caller-owned decode timeline buffer
   unsigned long long* spans = nullptr;                 // its kernel spans (SPAN_KINDS pairs), or null
@@ -151,6 +152,10 @@ struct MergeSource {
 };
 cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse, cudaStream_t s,
                          const MergeSource* src = nullptr);
+// block-incremental SVD update of one side's basis (k_incsvd.cu)
+cudaError_t launch_basis_update(lr_cache* c, int side, const void* blk, int n, float* gram, float* R_out,
+                                void* B_out, void* A_out, cudaStream_t s);
+void isvd_release(lr_cache* c);
 // bstride: elements between the batch rows of k and v (0: D, rows of one token per sequence)
 cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s, long long bstride = 0);
 // bulk prefill on tensor cores (k_prefill_tc.cu): n tokens per sequence, k / v [B][n][D]
