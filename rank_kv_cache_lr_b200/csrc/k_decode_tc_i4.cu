@@ -96,6 +96,14 @@ constexpr int kLaunchRegs = 128;
 template <bool kRope> struct Regs;
 template <> struct Regs<false> { static constexpr int ctl = 64, softmax = 184, dq = 120; };
 template <> struct Regs<true> { static constexpr int ctl = 64, softmax = 240, dq = 104; };
+// Move this warpgroup from the launch allocation to `kTo` registers per thread: setmaxnreg.inc
+// when raising, .dec when lowering (a .dec above the current count is an illegal instruction).
+template <int kTo>
+__device__ __forceinline__ void set_regs() {
+  static_assert(kTo % 8 == 0 && kTo >= 24 && kTo <= 256, "setmaxnreg range");
+  if constexpr (kTo > kLaunchRegs) ptx::setmaxnreg_inc<kTo>();
+  else if constexpr (kTo < kLaunchRegs) ptx::setmaxnreg_dec<kTo>();
+}
 static_assert(128 * Regs<false>::ctl + 128 * Regs<false>::softmax + 256 * Regs<false>::dq <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 static_assert(128 * Regs<true>::ctl + 128 * Regs<true>::softmax + 256 * Regs<true>::dq <= kThreads * kLaunchRegs,
@@ -356,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Roles by warpgroup; each sets its register budget first thing in its own branch,
   // so the compiler allocates that branch within the budget.
   if (warp < 4) {
-    ptx::setmaxnreg_dec<Regs<kRope>::ctl>();
+    set_regs<Regs<kRope>::ctl>();
     if (warp == 0) {
       // ------------------------------------------------------------- bulk-copy producer
       if (lane == 0 && ntiles > 0) {
@@ -562,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     }
   } else if (warp < kDqWarp0) {
-    ptx::setmaxnreg_inc<Regs<kRope>::softmax>();
+    set_regs<Regs<kRope>::softmax>();
     if (ntiles > 0) {
       // ------------------------------------------------------------- softmax / epilogue
       const int qd = warp & 3;
@@ -822,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    ptx::setmaxnreg_dec<Regs<kRope>::dq>();
+    set_regs<Regs<kRope>::dq>();
     // ------------------------------------------------------------- dequantisation
     if (ntiles > 0) {
       // side = 0 (warps 8..11): keys; side = 1 (warps 12..15): values.  Warp quarter
