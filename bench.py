@@ -246,6 +246,39 @@ def roofline_entry(kname: str, bytes_per_step: float, flops_per_step: float, ker
             "traffic": traffic}
 
 
+def basis_update_timing(L, Bsz, Hq, Hkv, d, n, dev) -> dict:
+    """Median time of lr_basis_update (keys side) for one block of n rows, on a bf16 cache
+    of the workload's shape whose basis rows are orthonormal (seeded)."""
+    import numpy as np
+    import torch
+    import statistics
+    import rank_kv_cache_lr_b200 as lr
+    import synth
+    r, D = L["rk"], Hkv * d
+    rng = synth.rng_for("basis_update", "B", 0)
+    B = synth.haar_orthonormal(rng, r, D)
+    to = lambda x: torch.from_numpy(synth.bf16_bits(x).view(np.int16)).view(torch.bfloat16).to(dev)
+    desc = lr.make_desc(1, Hq, Hkv, d, r, r, n + 8)
+    c = lr.lr_cache_create(desc, to(B.T), to(B), to(B.T), to(B))
+    blk = to(rng.standard_normal((n, D)) * 0.05)
+    g0 = torch.from_numpy(np.diag(synth.spectrum(r, 0.7) ** 2 * 1000.0).astype(np.float32)).to(dev)
+    R = torch.empty((r, r), dtype=torch.float32, device=dev)
+    Bn = torch.empty((r, D), dtype=torch.bfloat16, device=dev)
+    times = []
+    for i in range(4):
+        g = g0.clone()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lr.lr_basis_update(c, 0, blk, g, R, Bn)
+        e1.record()
+        torch.cuda.synchronize()
+        if i:
+            times.append(e0.elapsed_time(e1))
+    lr.lr_cache_destroy(c)
+    return {"us_per_call": round(1000 * statistics.median(times), 1), "rank": r, "D": D, "block_rows": n,
+            "timing": "CUDA events around the call, median of 3 after one warm-up"}
+
+
 def traffic_record(kernel: str):
     """DRAM traffic per launch from a committed ncu summary, valid only while the kernel
     source is unchanged (matched by hash)."""
@@ -530,6 +563,13 @@ def run_workload(args, workload):
                 "GBps": round(sync_bytes / (sync_ms * 1e-3) / 1e9, 1)}
         total_ms += K * sync_ms / W["sync_every"]
         e2e_ms += K * sync_ms / W["sync_every"]
+        # the basis update that produces R and the new basis from a folded block of
+        # `sync_every` exact key rows (lr_basis_update, fp64 on the GPU), timed on a cache of
+        # the same shape with an orthonormal basis; reported beside the decode, not in it
+        upd = basis_update_timing(L, Bsz, Hq, Hkv, d, W["sync_every"], dev)
+        upd["every_steps"] = W["sync_every"]
+        upd["us_per_step_amortised"] = round(upd["us_per_call"] / W["sync_every"], 2)
+        sync["basis_update"] = upd
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
     value = job_rate(bytes_per_step, K, world, total_ms)
