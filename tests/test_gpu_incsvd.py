@@ -50,7 +50,7 @@ def _update(lib, c, side, blk, S, r, D, dev):
         Bn.cpu().numpy().astype(np.float64), An.cpu().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("D_heads,r,n", [(2, 32, 16), (4, 128, 128), (4, 256, 64)])
+@pytest.mark.parametrize("D_heads,r,n", [(2, 32, 16), (4, 128, 128), (4, 256, 64), (8, 400, 100), (2, 16, 1)])
 def test_update_matches_oracle(lib, D_heads, r, n):
     c, K, B0, S0, D, dev = _setup(lib, D_heads, r, 600, seed=r + n)
     blk = K[600:600 + n]
@@ -70,6 +70,37 @@ def test_update_matches_oracle(lib, D_heads, r, n):
     assert np.abs(Bn @ Bn.T - np.eye(r)).max() < 1e-5
     assert np.array_equal(An, Bn.T)
     assert np.abs(R - B0.astype(np.float64) @ Bn.T).max() < 1e-5
+    lib.lr_cache_destroy(c)
+
+
+def test_update_on_a_bf16_cache(lib):
+    """bf16 basis and block: the GPU and the oracle take the same bf16 values (the basis rows
+    then orthonormal only to bf16 precision); the new basis comes back in bf16."""
+    import torch
+    rng = np.random.default_rng(21)
+    D_heads, r, n = 4, 64, 48
+    D = D_heads * 128
+    K = _keys(rng, 700, D, 0.985)
+    B0, _, _ = incsvd.initial_basis(K[:600], r)
+    B0b = synth.bf16_to_f64(synth.bf16_bits(B0))
+    blk = synth.bf16_to_f64(synth.bf16_bits(K[600:600 + n]))
+    Z0 = K[:600] @ B0b.T
+    S = (Z0.T @ Z0).astype(np.float32).astype(np.float64)
+    desc = lib.make_desc(1, 2 * D_heads, D_heads, 128, r, r, 700)
+    tob = lambda x: torch.from_numpy(synth.bf16_bits(x).view(np.int16)).view(torch.bfloat16).cuda()
+    c = lib.lr_cache_create(desc, tob(B0b.T), tob(B0b), tob(B0b.T), tob(B0b))
+    gram = torch.from_numpy(S.astype(np.float32)).cuda()
+    R = torch.empty((r, r), dtype=torch.float32, device="cuda")
+    Bn = torch.empty((r, D), dtype=torch.bfloat16, device="cuda")
+    lib.lr_basis_update(c, 1, tob(blk), gram, R, Bn)
+    torch.cuda.synchronize()
+    want = incsvd.block_update(B0b, S, blk)
+    got = synth.bf16_to_f64(Bn.cpu().view(torch.int16).numpy().view(np.uint16))
+    sg = np.sign(np.sum(got * want["B_new"], axis=1))
+    # one bf16 rounding of each entry (plus the fp64 differences of the two factorisations)
+    assert np.all(np.abs(got - sg[:, None] * want["B_new"]) <= 2.0 ** -8 * np.abs(want["B_new"]) + 1e-6)
+    lam = want["lam"][:r]
+    assert np.allclose(np.diag(gram.cpu().numpy()), lam, rtol=1e-5, atol=1e-6 * lam[0])
     lib.lr_cache_destroy(c)
 
 
