@@ -77,7 +77,7 @@ struct El<float> {
 // significant bits.  int4 latents: row [b][j] of a [B][32][r_k] fp16 array gets fp16(q~),
 // each 8-rank run in the order 0,4,1,5,2,6,3,7 in which the int4 kernel expands codes.
 constexpr int kQRowsCta = 32;
-constexpr int kRows = 4;   // sequences per CTA of the small kernels
+constexpr int kRows = 2;   // sequences per CTA of the small kernels
 
 struct QprojArgs {
   const void* q; const void* Bk; float* qt; float* qd; void* qt16;
