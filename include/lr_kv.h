@@ -83,7 +83,14 @@ typedef struct lr_cache_desc {
                              n_kv_heads): g groups of n_kv_heads / g heads, each with its own
                              latents of rank_k / rank_v and its own bases, so g = n_kv_heads
                              is one latent per KV head.  g * rank_k and g * rank_v <= 512.  */
-  int32_t reserved[4];    /* must be zero                                          */
+  int32_t page_tokens;    /* 0: each sequence's latents are one contiguous run of rows;
+                             128: paged latents (a pool of n_pages pages of 128 token rows,
+                             sequence b's token t in page table[b][t / 128], row t % 128;
+                             lr_cache_set_block_table).  Paged caches need capacity % 128 == 0
+                             and window == 0.                                       */
+  int32_t n_pages;        /* paged: pages in the pool, >= 1 (0: batch * capacity / 128);
+                             must be 0 when page_tokens is 0                         */
+  int32_t reserved[2];    /* must be zero                                          */
 } lr_cache_desc;
 
 typedef struct lr_cache lr_cache;   /* opaque */
@@ -104,6 +111,9 @@ typedef struct lr_cache lr_cache;   /* opaque */
  *   params_v [B][int4_blocks][groups][256] fp16 (same bytes as params_k): half
  *            (n*groups + g)*256 + u is the scale, half (n*groups + g)*256 + 128 + u the zero.
  * Unquantised latents: z [B][capacity][rank] in dtype.
+ * Paged caches (n_pages > 0): the B sequences of the layouts above become one pool of
+ * n_pages pages (z [n_pages][128][rank]; int4: block n = page n), and token t of sequence b
+ * is token t % 128 of page table[b][t / 128] (lr_cache_set_block_table).
  * Window ring: [B][window+1][D] in dtype; token t lives in slot t % (window+1). */
 typedef struct lr_cache_view {
   void* z_k; void* z_v;                 /* unquantised latents or NULL            */
@@ -114,7 +124,7 @@ typedef struct lr_cache_view {
   int32_t groups_k, groups_v;           /* ceil(rank/32) for int4 caches, else 0 */
   int32_t capacity, window_slots;
   int32_t int4_blocks;                  /* 128-token blocks per sequence (int4), else 0 */
-  int32_t reserved;
+  int32_t n_pages;                      /* pages of a paged cache's pool, else 0  */
 } lr_cache_view;
 
 /* Decode plan (host arithmetic only; exposed for tests and tooling). */
@@ -265,8 +275,8 @@ lr_status lr_basis_update(lr_cache* cache, int32_t side, const void* blk, int32_
  *   working memory (query latents and per-split partial results) is one static device
  *   array of LR_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
  *   process exit.
- *   desc: as for lr_cache_create, with window 0, quant_bits 0 and rope_in_kernel 0
- *     (otherwise LR_ERR_UNSUPPORTED); len: tokens to attend, 1..capacity.
+ *   desc: as for lr_cache_create, with window 0, quant_bits 0, rope_in_kernel 0, one
+ *     latent group and page_tokens 0 (otherwise LR_ERR_UNSUPPORTED); len: tokens to attend, 1..capacity.
  *   z_k [B][capacity][r_k], z_v [B][capacity][r_v]: latents in the cache layout;
  *   B_k [r_k][D], B_v [r_v][D], q [B][Hq][d], out [B][Hq][d]: dtype, device;
  *   B_k and B_v 16-byte aligned (else LR_ERR_INVALID_ARG, before any launch);
@@ -296,6 +306,24 @@ lr_status lr_cache_get_len(const lr_cache* cache, int32_t* len, int32_t* hist_le
 lr_status lr_cache_truncate(lr_cache* cache, int32_t len);
 /* Device pointers of the storage (see lr_cache_view). */
 lr_status lr_cache_view_get(const lr_cache* cache, lr_cache_view* out);
+/* lr_cache_set_block_table — the page of every 128-token span of every sequence of a paged
+ *   cache (page_tokens = 128).  Paging is a storage layout only (the method fixes what is
+ *   computed per token, not where a token's latent row lives): every result equals that
+ *   of a contiguous cache holding the same latents.
+ *   table: host, [batch][capacity / 128] int32, each entry in [0, n_pages); the library
+ *   checks every entry (LR_ERR_INVALID_ARG, nothing changed, if one is out of range or
+ *   table is NULL) and copies the table to the device on `stream` (ordered after the work
+ *   before the call there, so a decode queued earlier still reads the old table); the
+ *   caller's array is no longer read once the call returns.  Not capturable in a CUDA
+ *   graph (a copy from pageable memory).
+ *   Sequences may share pages (a common prefix); an append into a shared page writes it
+ *   for every sequence that maps it.  The rows of a page keep their contents when the
+ *   table changes.  A new cache's table maps span j of sequence b to page
+ *   (b * capacity / 128 + j) % n_pages.  LR_ERR_UNSUPPORTED for a cache that is not paged.
+ *   With paging, lr_kv_prefill, lr_kv_append_latent, lr_decode_step and every decode call
+ *   work as for contiguous caches; lr_basis_sync rotates every row of the pool (each page
+ *   once, whatever maps it). */
+lr_status lr_cache_set_block_table(lr_cache* cache, const int32_t* table, void* stream);
 /* Force a decode path (LR_PATH_*) and/or a split count (0 = automatic). */
 lr_status lr_cache_set_path(lr_cache* cache, int32_t path, int32_t n_splits);
 /* The plan lr_attn_decode would use at the current length. */

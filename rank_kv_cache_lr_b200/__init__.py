@@ -12,7 +12,7 @@ lr_cache_truncate, lr_cache_view_get, lr_cache_set_path, lr_cache_plan,
 lr_plan_decode, lr_cache_set_kernel_events, lr_cache_set_trace, lr_device_error, lr_abi_struct_sizes,
 lr_status_string, lr_launch_count, lr_attn_decode_noalloc, lr_cache_set_wait_limit,
 lr_debug_inject_fault, lr_attn_decode_varlen, lr_attn_decode_partial, lr_merge_partials,
-lr_kv_prefill.
+lr_kv_prefill, lr_cache_set_block_table.
 """
 from __future__ import annotations
 
@@ -36,7 +36,8 @@ class lr_cache_desc(ctypes.Structure):
                 ("quant_bits", ctypes.c_int32), ("quant_group", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("rope_in_kernel", ctypes.c_int32),
                 ("rope_theta", ctypes.c_double), ("softmax_scale", ctypes.c_float),
-                ("latent_groups", ctypes.c_int32), ("reserved", ctypes.c_int32 * 4)]
+                ("latent_groups", ctypes.c_int32), ("page_tokens", ctypes.c_int32),
+                ("n_pages", ctypes.c_int32), ("reserved", ctypes.c_int32 * 2)]
 
 
 class lr_cache_view(ctypes.Structure):
@@ -48,7 +49,7 @@ class lr_cache_view(ctypes.Structure):
                 ("A_v", ctypes.c_void_p), ("B_v", ctypes.c_void_p),
                 ("groups_k", ctypes.c_int32), ("groups_v", ctypes.c_int32),
                 ("capacity", ctypes.c_int32), ("window_slots", ctypes.c_int32),
-                ("int4_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("int4_blocks", ctypes.c_int32), ("n_pages", ctypes.c_int32)]
 
 
 class lr_plan(ctypes.Structure):
@@ -81,6 +82,7 @@ def _load() -> ctypes.CDLL:
         "lr_cache_get_len": [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)],
         "lr_cache_truncate": [vp, i32],
         "lr_cache_view_get": [vp, ctypes.POINTER(lr_cache_view)],
+        "lr_cache_set_block_table": [vp, vp, vp],
         "lr_cache_set_path": [vp, i32, i32],
         "lr_cache_plan": [vp, ctypes.POINTER(lr_plan)],
         "lr_plan_decode": [ctypes.POINTER(lr_cache_desc), i32, i32, i32, i32, ctypes.POINTER(lr_plan)],
@@ -131,10 +133,10 @@ def make_desc(batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int, rank_k
               rank_v: int, capacity: int, window: int = 0, quant_bits: int = 0,
               dtype: int = LR_BF16, rope_in_kernel: int = 0, rope_theta: float = 1e6,
               softmax_scale: float = 0.0, quant_group: int = 32,
-              latent_groups: int = 0) -> lr_cache_desc:
+              latent_groups: int = 0, page_tokens: int = 0, n_pages: int = 0) -> lr_cache_desc:
     return lr_cache_desc(batch, n_q_heads, n_kv_heads, head_dim, rank_k, rank_v, capacity,
                          window, quant_bits, quant_group, dtype, rope_in_kernel, rope_theta,
-                         softmax_scale, latent_groups)
+                         softmax_scale, latent_groups, page_tokens, n_pages)
 
 
 # ---------------------------------------------------------------------------
@@ -374,6 +376,18 @@ def lr_cache_view_get(cache: Cache) -> lr_cache_view:
     v = lr_cache_view()
     _check(_lib.lr_cache_view_get(cache.handle, ctypes.byref(v)), "lr_cache_view_get")
     return v
+
+
+def lr_cache_set_block_table(cache: Cache, table, stream=None) -> None:
+    """table: host array-like of int32, [batch][capacity / 128], the page of each 128-token
+    span of each sequence of a paged cache."""
+    import numpy as np
+    d = cache.desc
+    t = np.ascontiguousarray(np.asarray(table), dtype=np.int32)
+    if t.shape != (d.batch, d.capacity // 128):
+        raise ValueError(f"table must be [{d.batch}][{d.capacity // 128}], got {t.shape}")
+    _check(_lib.lr_cache_set_block_table(cache.handle, t.ctypes.data_as(ctypes.c_void_p), _stream(stream)),
+           "lr_cache_set_block_table")
 
 
 def lr_cache_set_path(cache: Cache, path: int = LR_PATH_AUTO, n_splits: int = 0) -> None:

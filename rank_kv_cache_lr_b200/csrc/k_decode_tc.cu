@@ -55,6 +55,8 @@ struct TcParams {
   unsigned long long wait_ns;   // bounded-wait limit (0: the default)
   const int32_t* row_len;       // per-row history lengths (device), or null
   unsigned long long* span;     // timeline span, or null
+  const int32_t* table;         // paged caches: block table [B][pps] (maps address pages), else null
+  int pps;
   int r_k, r_v, ck, cv, kb_k, tmem_cols;
   int Hq, hist_len, stable_len, split_tokens, n_splits, nslot;
   uint32_t q_bytes;
@@ -192,6 +194,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         bool isv;
         tc::unit_of(u, ntiles, &tile, &isv);
         const int t0 = tok_begin + tile * kTile;
+        // box origin: (token, sequence), or (0, page) in a paged pool (a tile is one page)
+        const int ty = p.table ? 0 : t0;
+        const int tz = p.table ? __ldg(p.table + (long long)b * p.pps + (t0 >> 7)) : b;
         const int nch = isv ? p.cv : p.ck;
         const int r = isv ? p.r_v : p.r_k;
         for (int c = 0; c < nch; ++c, ++pos) {
@@ -212,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           ptx::mbar_arrive_expect_tx(&aux->slot_full[slot], nsub * kSubBytes);
           for (int sb = 0; sb < nsub; ++sb)
             ptx::tma_load_3d(dst + sb * kSubBytes, isv ? &tm_zv : &tm_zk, &aux->slot_full[slot],
-                             c * 128 + sb * 64, t0, b);
+                             c * 128 + sb * 64, ty, tz);
           issued = pos + 1;
         }
       }
@@ -509,7 +514,9 @@ cudaError_t tc_prepare(lr_cache* c, cudaStream_t s) {
     e = cudaMemset(c->qt16, 0, (size_t)d.batch * kQRows * d.rank_k * 2);
     if (e != cudaSuccess) return e;
   }
-  const cuuint64_t cap = d.capacity, B = d.batch;
+  // latent maps: [B][capacity][r], or the paged pool [n_pages][128][r]
+  const cuuint64_t B = d.batch;
+  const cuuint64_t rows = c->ptable ? kPageTokens : d.capacity, seqs = c->ptable ? c->n_pages : B;
   {
     cuuint64_t dims[2] = {(cuuint64_t)d.rank_k, B * kQRows};
     cuuint64_t strides[1] = {(cuuint64_t)d.rank_k * 2};
@@ -518,8 +525,8 @@ cudaError_t tc_prepare(lr_cache* c, cudaStream_t s) {
   }
   for (int side = 0; side < 2; ++side) {
     const int r = side ? d.rank_v : d.rank_k;
-    cuuint64_t dims[3] = {(cuuint64_t)r, cap, B};
-    cuuint64_t strides[2] = {(cuuint64_t)r * 2, cap * r * 2};
+    cuuint64_t dims[3] = {(cuuint64_t)r, rows, seqs};
+    cuuint64_t strides[2] = {(cuuint64_t)r * 2, rows * r * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
     if (!make_map(side ? &st->zv : &st->zk, side ? c->z_v : c->z_k, 3, dims, strides, box))
       return cudaErrorInvalidValue;
@@ -549,6 +556,8 @@ cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, 
   p.wait_ns = c->wait_ns;
   p.row_len = c->row_len;
   p.span = span_of(c->spans, SPAN_DECODE);
+  p.table = c->ptable;
+  p.pps = c->pps;
   p.r_k = d.rank_k;
   p.r_v = d.rank_v;
   p.ck = (d.rank_k + 127) / 128;

@@ -139,7 +139,7 @@ struct I4Params {
   const uint32_t* codes_v;
   const uint32_t* params_k;
   const uint32_t* params_v;
-  long long cap;
+  RowMap map;                   // token -> latent row (block)
   int r_k, r_v, G_k, G_v, ck, cv, kb_k;
   int Hq, hist_len, stable_len, split_tokens, n_splits;
   int nks, nvs;                 // operand slots of the key ring [0, nks) and the value ring [nks, +nvs)
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (round > 0 && !(ok = wait_b(&aux->raw_empty[rs], (round - 1) & 1, aux, p.err))) break;
           const int G = is_v ? p.G_v : p.G_k;
-          const long long row0 = (long long)b * p.cap + t0;
+          const long long row0 = p.map.row(b, t0);   // a whole block: one page
           uint8_t* dst = raw + rs * p.raw_bytes;
           // one block of one side: G x 2 KB of codes and G x 512 B of params, at the same
           // offsets for the token-major keys and the rank-major values
@@ -1089,7 +1089,7 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
   p.codes_v = c->codes_v;
   p.params_k = c->params_k;
   p.params_v = c->params_v;
-  p.cap = c->lat_cap;
+  p.map = row_map(c);
   p.r_k = d.rank_k;
   p.r_v = d.rank_v;
   p.G_k = c->G_k;

@@ -220,7 +220,7 @@ struct AppendArgs {
   const void* A_k; const void* A_v;
   void* Zk; void* Zv; uint32_t* codes_k; uint32_t* codes_v; uint32_t* params_k; uint32_t* params_v;
   int rk, rv, Gk, Gv, chunks_k, chunks_v;
-  long long cap; int dst_slot; int project;
+  RowMap map; int dst_slot; int project;
   const void* new_k; const void* new_v;   // exact token for the ring, or null
   void* win_k; void* win_v; int slots; int new_slot;
   unsigned long long* span;   // timeline span, or null
@@ -290,7 +290,7 @@ __device__ __forceinline__ void append_main(const AppendArgs& a, int x, int b0, 
       float zz = 0.f;
 #pragma unroll
       for (int w = 0; w < 8; ++w) zz += red[w][warp][lane];
-      const long long row = (long long)(b0 + warp) * a.cap + a.dst_slot;
+      const long long row = a.map.row(b0 + warp, a.dst_slot);
       store_latent_chunk(zz, ch, r, a.kind, a.dtype, is_k ? a.Zk : a.Zv, is_k ? a.codes_k : a.codes_v,
                          is_k ? a.params_k : a.params_v, is_k ? a.Gk : a.Gv, row, !is_k);
     }
@@ -642,7 +642,7 @@ AppendArgs make_append_args(const lr_cache* c, const void* k, const void* v) {
   a.params_k = c->params_k; a.params_v = c->params_v;
   a.rk = d.rank_k; a.rv = d.rank_v; a.Gk = c->G_k; a.Gv = c->G_v;
   a.chunks_k = (d.rank_k + 31) / 32; a.chunks_v = (d.rank_v + 31) / 32;
-  a.cap = c->lat_cap; a.dst_slot = c->hist_len;
+  a.map = row_map(c); a.dst_slot = c->hist_len;
   a.new_k = win ? k : nullptr; a.new_v = win ? v : nullptr;
   a.win_k = c->win_k; a.win_v = c->win_v; a.slots = c->win_slots;
   a.new_slot = win ? (c->len % c->win_slots) : 0;

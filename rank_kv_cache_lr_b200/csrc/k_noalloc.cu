@@ -51,7 +51,8 @@ extern "C" lr_status lr_attn_decode_noalloc(const lr_cache_desc* desc, int32_t l
   if (!desc || !z_k || !z_v || !B_k || !B_v || !q || !out) return LR_ERR_INVALID_ARG;
   // the bases are staged into shared memory with 16-byte copies
   if ((reinterpret_cast<uintptr_t>(B_k) | reinterpret_cast<uintptr_t>(B_v)) & 15) return LR_ERR_INVALID_ARG;
-  if (desc->window != 0 || desc->quant_bits != 0 || desc->rope_in_kernel != 0 || desc->latent_groups > 1)
+  if (desc->window != 0 || desc->quant_bits != 0 || desc->rope_in_kernel != 0 || desc->latent_groups > 1 ||
+      desc->page_tokens != 0)
     return LR_ERR_UNSUPPORTED;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess) return LR_ERR_CUDA;

@@ -37,7 +37,7 @@ constexpr int kMaxStages = 4;
 struct PfParams {
   unsigned long long wait_ns;
   int n, D, r_k, r_v, G_k, G_v, slot0, kind, nstage;
-  long long cap;
+  RowMap map;                              // token -> latent row
   void* Zk; void* Zv;                      // bf16 latents (kind LK_BF16)
   uint32_t* codes_k; uint32_t* codes_v; uint32_t* params_k; uint32_t* params_v;
   int* err;
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const int t = tile * kTile + m;
     const bool valid = t < p.n;
-    const long long row = (long long)b * p.cap + p.slot0 + t;
+    const long long row = valid ? p.map.row(b, p.slot0 + t) : 0;   // the table has no row past n
     const bool ok = ptx::named_bar_and(1, 128, wait_b(&aux->d_full, 0, aux, p.err));
     if (ok) {
       ptx::tc_fence_after();
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Tokens past n contribute 0 (their slots hold no data); a word whose first token
             // is past n is not stored at all (its slots may lie beyond the storage).
             const int tb = t & ~7;
-            const long long row_w = (long long)b * p.cap + p.slot0 + tb;
+            const long long row_w = tb < p.n ? p.map.row(b, p.slot0 + tb) : 0;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               uint32_t w = valid ? code[e] << sh4 : 0u;
@@ -305,7 +305,7 @@ cudaError_t launch_prefill_tc(lr_cache* c, const void* k, const void* v, int n, 
   p.G_v = c->G_v;
   p.slot0 = c->hist_len;
   p.kind = c->latent_kind;
-  p.cap = c->lat_cap;
+  p.map = row_map(c);
   p.Zk = c->z_k;
   p.Zv = c->z_v;
   p.codes_k = c->codes_k;

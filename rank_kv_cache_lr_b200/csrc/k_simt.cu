@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(256) k_decode_simt(DecodeSimtArgs a, int kind)
   const int t_end = min(row_hist(a.row_len, b, a.hist_len), t_begin + a.split_tokens);
   for (int t0 = t_begin; t0 < t_end; t0 += kTileSimt) {
     const int n = min(kTileSimt, t_end - t0);
-    const long long row0 = (long long)b * a.k.cap + t0;
+    const long long row0 = a.k.map.row(b, t0);   // a 16-token tile lies inside one page
     for (int idx = tid; idx < n * rk; idx += nt) {
       const int t = idx / rk, i = idx % rk;
       zk_s[t * rk + i] = latent_f(a.k, kind, a.dtype, row0 + t, i);
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(256) k_append_latent(const float* zk, const fl
                                                        void* Zk, void* Zv, uint32_t* codes_k,
                                                        uint32_t* codes_v, uint32_t* params_k,
                                                        uint32_t* params_v, int Gk, int Gv,
-                                                       long long cap, int slot0, int kind, int dtype) {
+                                                       RowMap map, int slot0, int kind, int dtype) {
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(256) k_append_latent(const float* zk, const fl
   const float* src = is_k ? zk : zv;
   const int i = ch * 32 + lane;
   const float z = i < r ? src[((long long)b * n + t) * r + i] : 0.f;
-  const long long row = (long long)b * cap + slot0 + t;
+  const long long row = map.row(b, slot0 + t);
   store_latent_chunk(z, ch, r, kind, dtype, is_k ? Zk : Zv, is_k ? codes_k : codes_v,
                      is_k ? params_k : params_v, is_k ? Gk : Gv, row);
 }
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(256) k_append_latent(const float* zk, const fl
 // rank's word once; a word the fill covers only in part (the ends of the range) keeps its
 // other tokens' nibbles (cleared and set with atomics, which touch only the filled bits).
 __global__ void __launch_bounds__(256) k_append_latent_v(const float* zv, int n, int rv, int Gv, uint32_t* codes,
-                                                         uint32_t* params, long long cap, int slot0) {
+                                                         uint32_t* params, RowMap map, int slot0) {
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(256) k_append_latent_v(const float* zv, int n,
     if (t < slot0 || t >= slot0 + n) continue;   // warp-uniform
     const float z = valid ? zv[((long long)b * n + (t - slot0)) * rv + i] : 0.f;
     const QuantOut q = quant_group_codes(z, valid);
-    const long long row = (long long)b * cap + t;
+    const long long row = map.row(b, t);
     const int sh = 4 * i4v_nibble(row);
     word |= q.code << sh;
     mask |= 15u << sh;
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(256) k_append_latent_v(const float* zv, int n,
       h[si + 128] = q.zh;
     }
   }
-  uint32_t* w = codes + i4v_code_index((long long)b * cap + wq * 8, Gv, i);
+  uint32_t* w = codes + i4v_code_index(map.row(b, wq * 8), Gv, i);   // 8 tokens: one page
   if (mask == 0xFFFFFFFFu) {
     *w = word;
   } else {
@@ -379,7 +379,7 @@ LatentRef latent_ref(const lr_cache* c, bool k) {
   L.params = k ? c->params_k : c->params_v;
   L.r = k ? c->desc.rank_k : c->desc.rank_v;
   L.G = k ? c->G_k : c->G_v;
-  L.cap = c->lat_cap;
+  L.map = row_map(c);
   L.rank_major = (!k && c->latent_kind == LK_INT4) ? 1 : 0;
   return L;
 }
@@ -445,7 +445,7 @@ cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, 
   cudaError_t e = smem_optin(k_append_latent, optin_done);
   if (e != cudaSuccess) return e;
   e = launch_pdl(k_append_latent, grid, dim3(256), 0, s, zk, zv, n, d.batch, d.rank_k, d.rank_v, chunks_k, chunks_v,
-                 c->z_k, c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->G_k, c->G_v, c->lat_cap,
+                 c->z_k, c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->G_k, c->G_v, row_map(c),
                  c->hist_len, c->latent_kind, d.dtype);
   if (e != cudaSuccess || c->latent_kind != LK_INT4 || n == 0) return e;
   const int slot0 = c->hist_len;
@@ -454,18 +454,22 @@ cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, 
   e = smem_optin(k_append_latent_v, optin_v);
   if (e != cudaSuccess) return e;
   return launch_pdl(k_append_latent_v, dim3((unsigned)((units + 7) / 8), d.batch), dim3(256), 0, s, zv, n, d.rank_v,
-                    c->G_v, c->codes_v, c->params_v, c->lat_cap, slot0);
+                    c->G_v, c->codes_v, c->params_v, row_map(c), slot0);
 }
 
 cudaError_t launch_sync_simt(lr_cache* c, const float* R, int which, cudaStream_t s) {
   const lr_cache_desc& d = c->desc;
   const int r = which == 0 ? d.rank_k : d.rank_v;
   void* Z = which == 0 ? c->z_k : c->z_v;
-  if (c->hist_len == 0) return cudaSuccess;
+  // a paged pool is rotated whole, as one run of rows: every page once, whatever maps it
+  const int rows = c->ptable ? c->n_pages * kPageTokens : c->hist_len;
+  const int nseq = c->ptable ? 1 : d.batch;
+  if (rows == 0) return cudaSuccess;
   const size_t smem = (size_t)kSyncRows * r * sizeof(float);
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_sync_simt, optin_done);
   if (e != cudaSuccess) return e;
-  dim3 grid((c->hist_len + kSyncRows - 1) / kSyncRows, d.batch);
-  return launch_pdl(k_sync_simt, grid, dim3(256), smem, s, Z, R, r, d.capacity, c->hist_len, d.dtype);
+  dim3 grid((rows + kSyncRows - 1) / kSyncRows, nseq);
+  return launch_pdl(k_sync_simt, grid, dim3(256), smem, s, Z, R, r, (long long)(c->ptable ? rows : d.capacity), rows,
+                    d.dtype);
 }

@@ -300,7 +300,9 @@ cudaError_t launch_sync_tc(lr_cache* c, const float* R_k, const float* R_v, cuda
     }
     c->sync_state = st;
     st->r = r;
-    const cuuint64_t cap = d.capacity, B = d.batch;
+    // [B][capacity][r], or a paged pool as one run of n_pages * 128 rows
+    const cuuint64_t cap = c->ptable ? (cuuint64_t)c->n_pages * kPageTokens : d.capacity;
+    const cuuint64_t B = c->ptable ? 1 : d.batch;
     cuuint64_t zdims[3] = {(cuuint64_t)r, cap, B};
     cuuint64_t zstr[2] = {(cuuint64_t)r * 2, cap * r * 2};
     cuuint32_t zbox[3] = {64, (cuuint32_t)kTile, 1};
@@ -313,7 +315,10 @@ cudaError_t launch_sync_tc(lr_cache* c, const float* R_k, const float* R_v, cuda
         !map_bf16(&st->rv, st->rbuf + (size_t)2 * r * r, 2, rdims, rstr, rbox))
       return cudaErrorInvalidValue;
   }
-  const int ntile = (c->hist_len + kTile - 1) / kTile;
+  // a paged pool is rotated whole: every page once, whatever maps it
+  const int rows = c->ptable ? c->n_pages * kPageTokens : c->hist_len;
+  const int nseq = c->ptable ? 1 : d.batch;
+  const int ntile = (rows + kTile - 1) / kTile;
   if (ntile == 0 || (!R_k && !R_v)) return cudaSuccess;
   cudaError_t e = cudaSuccess;
   const dim3 pgrid(std::min(256, (r * r + 255) / 256));
@@ -324,16 +329,16 @@ cudaError_t launch_sync_tc(lr_cache* c, const float* R_k, const float* R_v, cuda
   p.wait_ns = c->wait_ns;
   p.r = r;
   p.kb = (r + 63) / 64;
-  p.B = d.batch;
+  p.B = nseq;
   p.ntile = ntile;
-  p.hist = c->hist_len;
+  p.hist = rows;
   p.z_bytes = (uint32_t)p.kb * kSubBytes;
   p.r_half = (uint32_t)p.kb * kRBox;
   p.r_slot = 2 * p.r_half;
   p.err = c->dev_err;
   // units: the K side first (if R_k), then the V side (if R_v)
   const int sides = (R_k ? 1 : 0) + (R_v ? 1 : 0);
-  p.units = sides * d.batch * ntile;
+  p.units = sides * nseq * ntile;
   CUtensorMap zk = st->zk, zv = st->zv, rk = st->rk, rv = st->rv;
   if (!R_k) {   // V only: unit side 0 must address the value latents
     zk = st->zv;

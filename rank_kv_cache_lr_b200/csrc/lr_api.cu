@@ -61,8 +61,14 @@ lr_status validate_user_desc(const lr_cache_desc* d) {
   if (d->rope_in_kernel && !(d->rope_theta > 0.0)) return LR_ERR_INVALID_ARG;
   if (d->rope_in_kernel && d->window > 0) return LR_ERR_UNSUPPORTED;
   if (!(d->softmax_scale >= 0.0f) || std::isinf(d->softmax_scale)) return LR_ERR_INVALID_ARG;
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 2; ++i)
     if (d->reserved[i] != 0) return LR_ERR_INVALID_ARG;
+  if (d->page_tokens != 0 && d->page_tokens != kPageTokens) return LR_ERR_INVALID_ARG;
+  if (d->page_tokens == 0 && d->n_pages != 0) return LR_ERR_INVALID_ARG;
+  if (d->n_pages < 0 || d->n_pages > (1 << 22)) return LR_ERR_INVALID_ARG;
+  if (d->page_tokens && (d->capacity % kPageTokens || d->window > 0)) return LR_ERR_UNSUPPORTED;
+  if (d->page_tokens && d->n_pages == 0 && (long long)d->batch * (d->capacity / kPageTokens) > (1 << 22))
+    return LR_ERR_INVALID_ARG;
   if ((long long)d->n_kv_heads * d->head_dim > 4096) return LR_ERR_UNSUPPORTED;
   if (d->n_q_heads > 128 || d->n_q_heads / d->n_kv_heads > 64) return LR_ERR_UNSUPPORTED;
   return LR_OK;
@@ -125,7 +131,7 @@ void free_all(lr_cache* c) {
   isvd_release(c);
   void* ptrs[] = {c->z_k, c->z_v, c->codes_k, c->codes_v, c->params_k, c->params_v, c->win_k, c->win_v,
                   c->A_k, c->B_k, c->A_v, c->B_v, c->rope_cs, c->qt, c->qt16, c->part_o, c->part_ml,
-                  c->win_o, c->win_ml, c->dev_err, c->r_full};
+                  c->win_o, c->win_ml, c->dev_err, c->r_full, c->ptable};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -225,6 +231,10 @@ lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void
   c->win_slots = d.window > 0 ? d.window + 1 : 0;
   c->lat_cap = c->latent_kind == LK_INT4 ? ((long long)d.capacity + kI4Block - 1) / kI4Block * kI4Block
                                          : (long long)d.capacity;
+  if (d.page_tokens) {
+    c->pps = d.capacity / kPageTokens;
+    c->n_pages = d.n_pages ? d.n_pages : d.batch * c->pps;
+  }
   c->len = c->hist_len = c->win_len = 0;
   const float sm_scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / std::sqrt((float)d.head_dim);
   c->scale_log2 = sm_scale * LR_LOG2E;
@@ -236,15 +246,23 @@ lr_status lr_cache_create(const lr_cache_desc* desc, const void* A_k, const void
   const size_t B = d.batch, cap = d.capacity, es = c->esize, D = c->D;
   if (e == cudaSuccess) {
     if (c->latent_kind == LK_INT4) {
-      const size_t rows = B * (size_t)c->lat_cap;
+      const size_t rows = c->n_pages ? (size_t)c->n_pages * kPageTokens : B * (size_t)c->lat_cap;
       e = dalloc(&c->codes_k, rows * c->G_k * 4 * sizeof(uint32_t));
       if (e == cudaSuccess) e = dalloc(&c->codes_v, rows * c->G_v * 4 * sizeof(uint32_t));
       if (e == cudaSuccess) e = dalloc(&c->params_k, rows * c->G_k * sizeof(uint32_t));
       if (e == cudaSuccess) e = dalloc(&c->params_v, rows * c->G_v * sizeof(uint32_t));
     } else {
-      e = dalloc(&c->z_k, B * cap * d.rank_k * es);
-      if (e == cudaSuccess) e = dalloc(&c->z_v, B * cap * d.rank_v * es);
+      const size_t rows = c->n_pages ? (size_t)c->n_pages * kPageTokens : B * cap;
+      e = dalloc(&c->z_k, rows * d.rank_k * es);
+      if (e == cudaSuccess) e = dalloc(&c->z_v, rows * d.rank_v * es);
     }
+  }
+  if (e == cudaSuccess && c->n_pages) {
+    // the initial table: span j of sequence b in page (b * pps + j) % n_pages
+    std::vector<int32_t> tab((size_t)d.batch * c->pps);
+    for (size_t i = 0; i < tab.size(); ++i) tab[i] = (int32_t)(i % (size_t)c->n_pages);
+    e = dalloc(&c->ptable, tab.size() * sizeof(int32_t));
+    if (e == cudaSuccess) e = cudaMemcpy(c->ptable, tab.data(), tab.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
   }
   if (e == cudaSuccess && c->win_slots) {
     e = dalloc(&c->win_k, B * c->win_slots * D * es);
@@ -587,8 +605,25 @@ lr_status lr_cache_view_get(const lr_cache* c, lr_cache_view* v) {
   v->groups_k = c->G_k; v->groups_v = c->G_v;
   v->capacity = c->desc.capacity; v->window_slots = c->win_slots;
   v->int4_blocks = c->latent_kind == LK_INT4 ? (int32_t)(c->lat_cap / kI4Block) : 0;
-  v->reserved = 0;
+  v->n_pages = c->n_pages;
   return LR_OK;
+}
+
+lr_status lr_cache_set_block_table(lr_cache* c, const int32_t* table, void* stream) {
+  if (!c) return LR_ERR_INVALID_ARG;
+  if (!c->ptable) return LR_ERR_UNSUPPORTED;
+  if (!table) return LR_ERR_INVALID_ARG;
+  const size_t n = (size_t)c->desc.batch * c->pps;
+  for (size_t i = 0; i < n; ++i)
+    if (table[i] < 0 || table[i] >= c->n_pages) return LR_ERR_INVALID_ARG;
+  // The copy goes from the library's own pageable buffer, which the runtime stages before
+  // cudaMemcpyAsync returns: the caller's table (pinned or not) is free on return.
+  c->host_table.assign(table, table + n);
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  const cudaError_t e =
+      cudaMemcpyAsync(c->ptable, c->host_table.data(), n * sizeof(int32_t), cudaMemcpyHostToDevice, s);
+  return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
 }
 
 lr_status lr_cache_set_path(lr_cache* c, int32_t path, int32_t n_splits) {

@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <vector>
 
 #include "lr_kv.h"
 
@@ -47,6 +48,21 @@ __host__ __device__ __forceinline__ long long i4v_scale_index(long long row, int
   return (((row >> 7) * G + g) << 8) + (row & 127);
 }
 
+// Where token t of sequence b is stored: row b * cap + t of the latent arrays, or, in a
+// paged cache, row page * 128 + t % 128 of the page pool, with page = table[b][t / 128].
+// Pages are as long as the tensor-core tile and the int4 block, so a tile or a block never
+// straddles two pages.
+constexpr int kPageTokens = 128;
+struct RowMap {
+  const int32_t* table;   // paged: [B][pps] page of each 128-token span (device), else null
+  long long cap;          // contiguous: rows per sequence
+  int pps;                // paged: pages per sequence
+  __device__ __forceinline__ long long row(int b, int t) const {
+    return table ? ((long long)__ldg(table + (long long)b * pps + (t >> 7)) << 7) + (t & 127)
+                 : (long long)b * cap + t;
+  }
+};
+
 // RoPE factors (cos, sin) of position t and frequency pair i (of d/2), fp32 from fp64
 // angles, stored in 128-token tiles, pair-major inside a tile: the 128 tokens of one pair are
 // contiguous, so threads that own consecutive tokens read one coalesced run per pair.
@@ -60,6 +76,10 @@ struct lr_cache {
   int G_k, G_v;          // int4 groups per token (0 when unquantised)
   int win_slots;         // window + 1 (ring), or 0
   long long lat_cap;     // latent rows per sequence: capacity (int4: rounded up to 128)
+  int32_t* ptable = nullptr;  // paged caches: the device block table [B][pps], else null
+  int pps = 0;           // paged: pages per sequence (capacity / 128)
+  int n_pages = 0;       // paged: pages in the pool
+  std::vector<int32_t> host_table;   // paged: staging copy of the last table set
   int32_t len, hist_len, win_len;
   int groups = 1;         // latent groups (desc ranks are the block-diagonal total g r)
   float* r_full = nullptr; // block-diagonal sync rotations (latent groups), [r_k^2 + r_v^2]
@@ -113,7 +133,7 @@ struct LatentRef {
   const uint32_t* params; // int4, blocked (i4_param_index; values: i4v_scale_index)
   int r, G;
   int rank_major;         // int4 values: the rank-major block layout
-  long long cap;
+  RowMap map;             // token -> latent row
 };
 
 struct DecodeSimtArgs {
@@ -195,6 +215,15 @@ void lr_count_launch(int n = 1);
 // Host-side fault injection (lr_debug_inject_fault): true when this device allocation or
 // kernel launch is the one armed to fail; the caller then fails without allocating or
 // launching.
+// The row map of a cache's latents (paged or contiguous).
+inline RowMap row_map(const lr_cache* c) {
+  RowMap m;
+  m.table = c->ptable;
+  m.cap = c->lat_cap;
+  m.pps = c->pps;
+  return m;
+}
+
 bool lr_fault_alloc();
 bool lr_fault_launch();
 

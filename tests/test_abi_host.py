@@ -81,10 +81,41 @@ def test_rope_with_window_is_unsupported(lib):
 
 
 def test_reserved_fields_must_be_zero(lib):
+    for i in range(2):
+        d = _qwen(lib)
+        d.reserved[i] = 1
+        with pytest.raises(lib.LRError):
+            lib.lr_plan_decode(d, 10, 148)
+
+
+@pytest.mark.parametrize("page_tokens, n_pages, capacity, window, status", [
+    (128, 0, 4096, 0, 0),        # default pool: batch * capacity / 128 pages
+    (128, 5, 4096, 0, 0),        # a pool smaller than the table (pages shared or unused)
+    (64, 0, 4096, 0, 1),         # pages are 128 tokens
+    (0, 8, 4096, 0, 1),          # a pool size without paging
+    (128, -1, 4096, 0, 1),
+    (128, 1 << 23, 4096, 0, 1),  # above the pool limit
+    (128, 0, 4000, 0, 2),        # capacity not a whole number of pages
+    (128, 0, 4096, 128, 2),      # no exact window in a paged cache
+])
+def test_paged_desc_validation(lib, page_tokens, n_pages, capacity, window, status):
+    d = _qwen(lib, capacity=capacity, window=window)
+    d.page_tokens, d.n_pages = page_tokens, n_pages
+    if status == 0:
+        lib.lr_plan_decode(d, 100, 148)
+    else:
+        with pytest.raises(lib.LRError) as e:
+            lib.lr_plan_decode(d, 100, 148)
+        assert e.value.status == status
+
+
+def test_noalloc_refuses_paged_desc_before_any_device_call(lib):
     d = _qwen(lib)
-    d.reserved[2] = 1
-    with pytest.raises(lib.LRError):
-        lib.lr_plan_decode(d, 10, 148)
+    d.page_tokens = 128
+    dummy = ctypes.c_void_p(256)
+    st = lib.raw_status("lr_attn_decode_noalloc", ctypes.byref(d), 100, dummy, dummy, dummy, dummy, dummy,
+                        dummy, None, None)
+    assert st == lib.LR_ERR_UNSUPPORTED
 
 
 def test_null_arguments(lib):
