@@ -173,13 +173,21 @@ __device__ __forceinline__ void load8(const uint8_t* s, int dtype, float (&v)[8]
   }
 }
 
+template <typename T> __device__ __forceinline__ float win_elem(const uint8_t* p);
+template <> __device__ __forceinline__ float win_elem<float>(const uint8_t* p) { return *reinterpret_cast<const float*>(p); }
+template <> __device__ __forceinline__ float win_elem<__nv_bfloat16>(const uint8_t* p) {
+  return __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(p)) << 16);
+}
+
+template <typename T>
 __global__ void __launch_bounds__(kWinThreads) k_window(const void* win_k, const void* win_v, const float* qd,
                                                         float* win_o, float* win_ml, int Hq, int Hkv, int d,
-                                                        int D, int slots, int hist_len, int win_len, int dtype,
+                                                        int D, int slots, int hist_len, int win_len,
                                                         unsigned long long* span) {
   extern __shared__ __align__(16) uint8_t wsm_raw[];
+  constexpr int es = sizeof(T);
+  constexpr int dtype = es == 2 ? LR_BF16 : LR_F32;
   const int G = Hq / Hkv;
-  const int es = dtype == LR_BF16 ? 2 : 4;
   const int pitch = window_pitch(d, es);
   float* q_s = reinterpret_cast<float*>(wsm_raw);          // [d]
   float* o_s = q_s + d;                                    // [d] (unused slot kept for alignment)
@@ -195,19 +203,38 @@ __global__ void __launch_bounds__(kWinThreads) k_window(const void* win_k, const
   constexpr int nw = kWinThreads / 32;
   const int j = h * G + u;                                 // query head
   const int vpr = d * es / 16;                             // 16-byte vectors per row
+  // copy positions: with vpr dividing the block, a thread keeps one vector column and steps
+  // over rows (no division per copy); otherwise (odd head dims) the general walk
+  const bool fixed = (kWinThreads % vpr) == 0;
+  const int rstep = fixed ? kWinThreads / vpr : 0;
   for (int v = tid; v < d / 4; v += kWinThreads) cp_async16(q_s + 4 * v, qd + ((long long)b * Hq + j) * d + 4 * v);
   float m = -INFINITY, l = 0.f;
   float o = 0.f;                                           // output column tid (d <= 128 here: tid < d)
   float o2 = 0.f;                                          // column tid + 128 (d > 128)
+  const uint8_t* gk = reinterpret_cast<const uint8_t*>(win_k) + ((long long)b * slots * D + (long long)h * d) * es;
+  const uint8_t* gv = reinterpret_cast<const uint8_t*>(win_v) + ((long long)b * slots * D + (long long)h * d) * es;
   for (int t0 = 0; t0 < win_len; t0 += kWinTok) {
     const int n = min(kWinTok, win_len - t0);
     __syncthreads();   // the previous round's rows and weights are no longer read
-    for (int idx = tid; idx < 2 * n * vpr; idx += kWinThreads) {
-      const int kv = idx / (n * vpr), r = idx - kv * (n * vpr);
-      const int t = r / vpr, v = r - (r / vpr) * vpr;
-      const long long row = (long long)b * slots + (hist_len + t0 + t) % slots;
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(kv ? win_v : win_k) + (row * D + (long long)h * d) * es;
-      cp_async16((kv ? v_s : k_s) + t * pitch + v * 16, src + v * 16);
+    if (fixed) {
+      const int v = tid % vpr;
+      int t = tid / vpr;
+      int slot = (hist_len + t0 + t) % slots;               // ring slot of token t0 + t
+      const int sstep = rstep % slots;
+      for (; t < n; t += rstep) {
+        const long long off = (long long)slot * D * es + v * 16;
+        cp_async16(k_s + t * pitch + v * 16, gk + off);
+        cp_async16(v_s + t * pitch + v * 16, gv + off);
+        slot += sstep;
+        if (slot >= slots) slot -= slots;
+      }
+    } else {
+      for (int idx = tid; idx < n * vpr; idx += kWinThreads) {
+        const int t = idx / vpr, v = idx - (idx / vpr) * vpr;
+        const long long off = (long long)((hist_len + t0 + t) % slots) * D * es + v * 16;
+        cp_async16(k_s + t * pitch + v * 16, gk + off);
+        cp_async16(v_s + t * pitch + v * 16, gv + off);
+      }
     }
     cp_async_wait_all();
     __syncthreads();
@@ -252,18 +279,24 @@ __global__ void __launch_bounds__(kWinThreads) k_window(const void* win_k, const
     const float alpha = m == -INFINITY ? 0.f : exp2f(m - mn);
     l = l * alpha + st;
     m = mn;
-    // output columns tid (and tid + 128)
+    // output columns tid (and tid + 128): tokens in order, four per step
     o *= alpha;
     o2 *= alpha;
-    for (int t = 0; t < n; ++t) {
-      const float p = p_s[t];
-      const uint8_t* vr = v_s + t * pitch;
-      if (tid < d) o = fmaf(p, dtype == LR_BF16 ? __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(vr + tid * 2)) << 16)
-                                                : *reinterpret_cast<const float*>(vr + tid * 4), o);
-      if (tid + kWinThreads < d)
-        o2 = fmaf(p, dtype == LR_BF16 ? __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(vr + (tid + kWinThreads) * 2)) << 16)
-                                      : *reinterpret_cast<const float*>(vr + (tid + kWinThreads) * 4), o2);
+    const uint8_t* vc = v_s + tid * es;
+    const uint8_t* vc2 = v_s + (tid + kWinThreads) * es;
+    if (tid < d) {
+      int t = 0;
+      for (; t + 4 <= n; t += 4) {
+        const float4 p4 = *reinterpret_cast<const float4*>(p_s + t);
+        o = fmaf(p4.x, win_elem<T>(vc + (t + 0) * pitch), o);
+        o = fmaf(p4.y, win_elem<T>(vc + (t + 1) * pitch), o);
+        o = fmaf(p4.z, win_elem<T>(vc + (t + 2) * pitch), o);
+        o = fmaf(p4.w, win_elem<T>(vc + (t + 3) * pitch), o);
+      }
+      for (; t < n; ++t) o = fmaf(p_s[t], win_elem<T>(vc + t * pitch), o);
     }
+    if (tid + kWinThreads < d)
+      for (int t = 0; t < n; ++t) o2 = fmaf(p_s[t], win_elem<T>(vc2 + t * pitch), o2);
   }
   cp_async_wait_all();   // (no window tokens: the query copies still complete)
   const long long ob = ((long long)b * Hq + j) * d;
@@ -428,12 +461,16 @@ cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
   const size_t smem = window_smem(d.n_q_heads / d.n_kv_heads, d.head_dim, (int)c->esize);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   dim3 grid(d.n_kv_heads, d.batch, d.n_q_heads / d.n_kv_heads);
-  static std::atomic<uint32_t> optin_done{0};
-  cudaError_t e = smem_optin(k_window, optin_done);
+  using Kern = void (*)(const void*, const void*, const float*, float*, float*, int, int, int, int, int, int, int,
+                       unsigned long long*);
+  const bool bf = d.dtype == LR_BF16;
+  const Kern kern = bf ? k_window<__nv_bfloat16> : k_window<float>;
+  static std::atomic<uint32_t> optin_done[2] = {0, 0};
+  cudaError_t e = smem_optin(kern, optin_done[bf ? 1 : 0]);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_window, grid, dim3(kWinThreads), smem, s, c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads, d.n_kv_heads,
-                                   d.head_dim, c->D, c->win_slots, c->hist_len, c->win_len, d.dtype,
-                                   span_of(c->spans, SPAN_WINDOW));
+  return launch_pdl(kern, grid, dim3(kWinThreads), smem, s, c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads,
+                    d.n_kv_heads, d.head_dim, c->D, c->win_slots, c->hist_len, c->win_len,
+                    span_of(c->spans, SPAN_WINDOW));
 }
 
 cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, int n, cudaStream_t s) {
