@@ -438,15 +438,34 @@ __global__ void __launch_bounds__(kMergeThreads, 2) k_merge(MergeArgs a) {
   for (int jb = 0; jb < G; jb += kMergeHeads) {
     const int nh = min(kMergeHeads, G - jb);
     const int nitems = nh * nq;
-    // 1. this thread's first item: its first kMergeLoads split loads go out now
-    const int u0 = tid < nitems ? tid / nq : 0, q0 = tid < nitems ? tid - u0 * nq : 0;
+    // 1. this thread's first item: its first kMergeLoads split loads go out now.  An item
+    //    (head, 4 ranks) is shared by tpi adjacent threads (the CTA's threads spread over
+    //    the items), thread `sub` of them taking splits sub, sub + tpi, ...
+    const int tpi = nitems * 4 <= kMergeThreads ? 4 : (nitems * 2 <= kMergeThreads ? 2 : 1);
+    const int sub = tid & (tpi - 1), it0 = tid / tpi, it_step = kMergeThreads / tpi;
+    const int u0 = it0 < nitems ? it0 / nq : 0, q0 = it0 < nitems ? it0 - u0 * nq : 0;
     const float* src0 = a.part_o + ((size_t)b * a.b_stride * a.Hq + h * G + jb + u0) * rv + i0 + 4 * q0;
+    // the (m, l) pairs first: the weights wait only for them, the partials keep coming
+    float2 mlv[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = tid + k * kMergeThreads;
+      if (e < nh * S) {
+        const int u = e / S, s = e - (e / S) * S;
+        mlv[k] = __ldg(reinterpret_cast<const float2*>(a.part_ml) + row_of(s) * a.Hq + h * G + jb + u);
+      }
+    }
     float4 v[kMergeLoads];
 #pragma unroll
-    for (int k = 0; k < kMergeLoads; ++k)
-      v[k] = (tid < nitems && k < S) ? __ldg(reinterpret_cast<const float4*>(src0 + (size_t)k * sstride))
+    for (int k = 0; k < kMergeLoads; ++k) {
+      const int s = sub + k * tpi;
+      v[k] = (it0 < nitems && s < S) ? __ldg(reinterpret_cast<const float4*>(src0 + (size_t)s * sstride))
                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int e = tid; e < nh * S; e += kMergeThreads) {
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      if (tid + k * kMergeThreads < nh * S) mls[tid + k * kMergeThreads] = mlv[k];
+    for (int e = tid + 2 * kMergeThreads; e < nh * S; e += kMergeThreads) {
       const int u = e / S, s = e - (e / S) * S;
       mls[e] = __ldg(reinterpret_cast<const float2*>(a.part_ml) + row_of(s) * a.Hq + h * G + jb + u);
     }
@@ -483,22 +502,26 @@ __global__ void __launch_bounds__(kMergeThreads, 2) k_merge(MergeArgs a) {
       }
     }
     __syncthreads();
-    // 2. merged o~ of this CTA's ranks; splits in a fixed order, zero-weight splits skipped
-    //    (their outputs are not written)
-    for (int it = tid; it < nitems; it += kMergeThreads) {
+    // 2. merged o~ of this CTA's ranks: each thread sums its splits in a fixed order
+    //    (zero-weight splits skipped: their outputs are not written), then the item's tpi
+    //    threads add their sums (lanes sub ^ 1, then sub ^ 2)
+    for (int it = it0; it < nitems; it += it_step) {
       const int u = it / nq, q = it - (it / nq) * nq;
       const float* src = a.part_o + ((size_t)b * a.b_stride * a.Hq + h * G + jb + u) * rv + i0 + 4 * q;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = 0; s0 < S; s0 += kMergeLoads) {
-        if (it != tid || s0 > 0) {
+      for (int s0 = 0; s0 < S; s0 += kMergeLoads * tpi) {
+        if (it != it0 || s0 > 0) {
 #pragma unroll
-          for (int k = 0; k < kMergeLoads; ++k)
-            v[k] = s0 + k < S ? __ldg(reinterpret_cast<const float4*>(src + (size_t)(s0 + k) * sstride))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int k = 0; k < kMergeLoads; ++k) {
+            const int s = s0 + sub + k * tpi;
+            v[k] = s < S ? __ldg(reinterpret_cast<const float4*>(src + (size_t)s * sstride))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
         }
 #pragma unroll
         for (int k = 0; k < kMergeLoads; ++k) {
-          const float w = s0 + k < S ? wsm[u * S + s0 + k] : 0.f;
+          const int s = s0 + sub + k * tpi;
+          const float w = s < S ? wsm[u * S + s] : 0.f;
           if (w != 0.f) {
             acc.x = fmaf(w, v[k].x, acc.x);
             acc.y = fmaf(w, v[k].y, acc.y);
@@ -507,7 +530,16 @@ __global__ void __launch_bounds__(kMergeThreads, 2) k_merge(MergeArgs a) {
           }
         }
       }
-      *reinterpret_cast<float4*>(otp + u * (rp + 4) + 4 * q) = acc;
+      if (tpi > 1) {
+        const unsigned mask = ((1u << tpi) - 1u) << (lane & ~(tpi - 1));
+        for (int o = 1; o < tpi; o <<= 1) {
+          acc.x += __shfl_xor_sync(mask, acc.x, o);
+          acc.y += __shfl_xor_sync(mask, acc.y, o);
+          acc.z += __shfl_xor_sync(mask, acc.z, o);
+          acc.w += __shfl_xor_sync(mask, acc.w, o);
+        }
+      }
+      if (sub == 0) *reinterpret_cast<float4*>(otp + u * (rp + 4) + 4 * q) = acc;
     }
     if (!project) {
       // rank-space partial of this shard: the merged o~ (relative to m) and (m, l)
@@ -526,13 +558,31 @@ __global__ void __launch_bounds__(kMergeThreads, 2) k_merge(MergeArgs a) {
     }
     // 3. every CTA gathers the whole o~ of the pass from the cluster's parts
     cluster_sync_all();
-    for (int part = 0; part < a.ncb; ++part) {
-      const int pi0 = min(rv, part * rp), pnq = (min(rv, pi0 + rp) - pi0) / 4;
-      const uint32_t base = cluster_addr(otp, (uint32_t)part);
-      for (int it = tid; it < nh * pnq; it += kMergeThreads) {
-        const int u = it / pnq, q = it - (it / pnq) * pnq;
-        *reinterpret_cast<float4*>(otf + u * (rv + 4) + pi0 + 4 * q) =
-            ld_cluster_f4(base + (uint32_t)((u * (rp + 4) + 4 * q) * 4));
+    {
+      // items (part, head, 4 ranks), kGather remote loads in flight per thread before the
+      // stores (a part's last quads may lie past rv: skipped)
+      constexpr int kGather = 4;
+      const int rq = rp / 4, per_part = nh * rq, total = a.ncb * per_part;
+      for (int ib = tid; ib < total; ib += kGather * kMergeThreads) {
+        float4 g[kGather];
+        int dst[kGather];
+#pragma unroll
+        for (int k = 0; k < kGather; ++k) {
+          const int it = ib + k * kMergeThreads;
+          dst[k] = -1;
+          if (it < total) {
+            const int part = it / per_part, r = it - part * per_part;
+            const int u = r / rq, q = r - (r / rq) * rq;
+            const int i = part * rp + 4 * q;
+            if (i < rv) {
+              g[k] = ld_cluster_f4(cluster_addr(otp, (uint32_t)part) + (uint32_t)((u * (rp + 4) + 4 * q) * 4));
+              dst[k] = u * (rv + 4) + i;
+            }
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kGather; ++k)
+          if (dst[k] >= 0) *reinterpret_cast<float4*>(otf + dst[k]) = g[k];
       }
     }
     if (!staged) {
