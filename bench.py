@@ -157,6 +157,17 @@ def max_over_ranks(values, device=None):
     return [float(v) for v in t.tolist()]
 
 
+def percentile(values, q: float) -> float:
+    """The q-th percentile (linear interpolation between order statistics)."""
+    v = sorted(values)
+    if not v:
+        return float("nan")
+    x = (len(v) - 1) * q / 100.0
+    i = int(x)
+    j = min(i + 1, len(v) - 1)
+    return v[i] + (v[j] - v[i]) * (x - i)
+
+
 def job_rate(bytes_per_step_per_rank: float, steps: int, world: int, total_ms: float) -> float:
     """Whole-job GB/s: the latent bytes every rank processed over the slowest rank's time."""
     return bytes_per_step_per_rank * steps * world / (total_ms * 1e-3) / 1e9
@@ -277,6 +288,48 @@ def basis_update_timing(L, Bsz, Hq, Hkv, d, n, dev) -> dict:
     lr.lr_cache_destroy(c)
     return {"us_per_call": round(1000 * statistics.median(times), 1), "rank": r, "D": D, "block_rows": n,
             "timing": "CUDA events around the call, median of 3 after one warm-up"}
+
+
+def paged_timing(L, p, W, dev, flush_l2) -> dict:
+    """The decode kernel on the same layer held in a paged cache (128-token pages, a seeded
+    random permutation of the pool as block table) beside the contiguous cache: CUDA events
+    around the kernel, lr_attn_decode, L2 flushed before each call, median of 10 after 3."""
+    import numpy as np
+    import torch
+    import statistics
+    import rank_kv_cache_lr_b200 as lr
+    Bsz, Hq, Hkv, d, T = W["batch"], W["n_q_heads"], W["n_kv_heads"], W["head_dim"], W["length"]
+    to_dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(dev)
+    desc = lr.make_desc(Bsz, Hq, Hkv, d, L["rk"], L["rv"], T, quant_bits=W["quant_bits"], dtype=lr.LR_BF16,
+                        page_tokens=128)
+    c = lr.lr_cache_create(desc, to_dev(p.A_k), to_dev(p.B_k), to_dev(p.A_v), to_dev(p.B_v))
+    pps = T // 128
+    table = np.random.default_rng(12345).permutation(Bsz * pps).astype(np.int32).reshape(Bsz, pps)
+    lr.lr_cache_set_block_table(c, table)
+    for s0 in range(0, p.hist_len, 1024):
+        e0 = min(p.hist_len, s0 + 1024)
+        lr.lr_kv_append_latent(c, torch.from_numpy(np.ascontiguousarray(p.z_k[:, s0:e0])).to(dev),
+                               torch.from_numpy(np.ascontiguousarray(p.z_v[:, s0:e0])).to(dev))
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(); ev1.record()
+    res = {}
+    for name, cache in (("paged", c), ("contiguous", L["cache"])):
+        ts = []
+        for i in range(13):
+            flush_l2()
+            lr.lr_cache_set_kernel_events(cache, ev0, ev1)
+            lr.lr_attn_decode(cache, L["q"], L["out"], L["lse"])
+            lr.lr_cache_set_kernel_events(cache)
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(ev0.elapsed_time(ev1))
+        res[name] = statistics.median(ts)
+    lr.lr_cache_destroy(c)
+    return {"decode_kernel_us": round(1000 * res["paged"], 2),
+            "contiguous_decode_kernel_us": round(1000 * res["contiguous"], 2),
+            "table": f"random permutation of the {Bsz * pps} pages of 128 tokens",
+            "timing": "CUDA events around the decode kernel of lr_attn_decode, L2 flushed before each, "
+                      "median of 10 after 3"}
 
 
 def traffic_record(kernel: str):
@@ -514,6 +567,14 @@ def run_workload(args, workload):
     launches = launches_per_step * K
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = sum(step_ms)
+    # the same step with a warm L2 (no flush between steps): labelled, not the graded value
+    wev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        wev[i][0].record()
+        run()
+        wev[i][1].record()
+    torch.cuda.synchronize()
+    warm_ms = [a.elapsed_time(b) for a, b in wev]
     # roofline: the main decode kernel of every layer, timed inside the `kev` capture
     kern_ms = []
     for i in range(K):
@@ -605,7 +666,14 @@ def run_workload(args, workload):
         "config": static_config(workload, world, args.layers),
         "run": {"decode_path": "tcgen05" if plan.path == lr.LR_PATH_TC else "simt",
                 "splits": plan.n_splits, "cuda_graph": bool(args.graph),
-                "launches_per_step": launches_per_step},
+                "launches_per_step": launches_per_step,
+                "step_us": {"median": round(1000 * statistics.median(step_ms), 2),
+                            "p10": round(1000 * percentile(step_ms, 10), 2),
+                            "p90": round(1000 * percentile(step_ms, 90), 2),
+                            "of": "this rank's timed steps, L2 flushed before each"},
+                "warm_l2_step_us": {"median": round(1000 * statistics.median(warm_ms), 2),
+                                    "note": "the same step replayed back to back without the L2 flush "
+                                            "(latents partly or wholly L2-resident); not the graded value"}},
         "roofline": roofline_entry(kname, bytes_per_step, roof_flops, kern_mean, peaks, peak_src, traf),
         "e2e": {"value": round(job_rate(bytes_per_step, K, world, e2e_ms), 2), "unit": "GB/s",
                 "us_per_step": round(1000 * e2e_ms / K, 2), "h2d_bytes_per_step": h2d,
@@ -615,6 +683,9 @@ def run_workload(args, workload):
     }
     if sync is not None:
         res["run"]["basis_sync"] = sync
+    if W["layers"] == 1 and not win and not W.get("groups") and world == 1:
+        # the same layer in a paged cache: paging moves no bytes and adds no work
+        res["run"]["paged"] = paged_timing(layers[0], host_p, W, dev, flush_l2)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(workload, host_p, args.cpu_seconds)
     if rank == 0:

@@ -59,3 +59,12 @@ def test_clock_summary_filters_gpu_and_reports_reasons():
 def test_clock_summary_without_samples():
     s = bench.ClockSampler("GPU-aaa").summary()
     assert s["samples"] == 0 and s["reasons"] == ["unsampled"]
+
+
+def test_percentile_matches_numpy_linear():
+    import numpy as np
+    rng = np.random.default_rng(0)
+    for n in (1, 2, 5, 20, 51):
+        v = list(rng.standard_normal(n))
+        for q in (0, 10, 50, 90, 100):
+            assert abs(bench.percentile(v, q) - float(np.percentile(v, q))) < 1e-12

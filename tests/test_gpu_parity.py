@@ -1,6 +1,8 @@
 """Parity of the CUDA library (through the C ABI) with the CPU oracle, on seeded synthetic
 inputs at sizes the oracle finishes in seconds: several tiles, ragged tails, every
 workload family, both decode paths, and the edge cases of the method."""
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -445,6 +447,21 @@ def test_window_only_and_history_only(lib):
     ref, ref_lse = H.oracle_decode(p2)
     got, lse = H.gpu_decode(lib, p2, c2)
     H.compare(p2, got, ref, lse, ref_lse, tag="history only")
+
+
+@pytest.mark.parametrize("head_dim,rank", [(24, 32), (40, 64), (256, 64), (64, 64)])
+def test_window_head_dims(lib, head_dim, rank):
+    """The exact window at head dims whose 16-byte row vectors do or do not divide the
+    window kernel's block (its two copy walks), with columns past 128 (d = 256) and a ring
+    that wraps (the window starts at slot hist_len mod (W + 1))."""
+    p = synth.make_hybrid(batch=2, hist_len=150, window=100, rank=rank, n_q_heads=4, n_kv_heads=2,
+                          head_dim=head_dim)
+    p = dataclasses.replace(p, q=p.store(H.stored_value(p, p.q) * H.sharp_factor(p)))
+    c = H.fill_cache(lib, p)
+    ref, ref_lse = H.oracle_decode(p)
+    got, lse = H.gpu_decode(lib, p, c)
+    H.compare(p, got, ref, lse, ref_lse, tag=f"window d={head_dim}")
+    lib.lr_cache_destroy(c)
 
 
 def test_capacity_and_argument_errors(lib):
