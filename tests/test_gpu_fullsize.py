@@ -93,3 +93,38 @@ def test_fullsize_hybrid(lib):
     p = synth.make_hybrid(seed=0, batch=8, hist_len=32640)
     plan = _check(lib, p, count=4)
     assert plan.path == lib.LR_PATH_TC
+
+
+@pytest.mark.parametrize("kind", ["qwen4k", "qwen16k"])
+def test_fullsize_paged_equals_contiguous(lib, kind):
+    """The bench's layers held in a paged cache (a seeded random permutation of every
+    128-token page as block table) decode bit for bit like the contiguous cache, with the
+    automatic plan the bench uses."""
+    import torch
+    if kind == "qwen4k":
+        p = synth.make_qwen("qwen4k", seed=0, batch=16, length=4095, rank=256)
+        cap = 4096
+    else:
+        p = synth.make_qwen("qwen16k", seed=0, batch=16, length=16383, rank=352, quant_bits=4)
+        cap = 16384
+    caches = []
+    for paged in (False, True):
+        d = H.desc_for(lib, p, cap)
+        if paged:
+            d.page_tokens = 128
+        c = lib.lr_cache_create(d, H.to_dev(p, p.A_k), H.to_dev(p, p.B_k), H.to_dev(p, p.A_v), H.to_dev(p, p.B_v))
+        if paged:
+            pps = cap // 128
+            table = np.random.default_rng(7).permutation(p.batch * pps).astype(np.int32).reshape(p.batch, pps)
+            lib.lr_cache_set_block_table(c, table)
+        for s0 in range(0, p.hist_len, 2048):
+            e0 = min(p.hist_len, s0 + 2048)
+            lib.lr_kv_append_latent(c, torch.from_numpy(np.ascontiguousarray(p.z_k[:, s0:e0])).cuda(),
+                                    torch.from_numpy(np.ascontiguousarray(p.z_v[:, s0:e0])).cuda())
+        caches.append(c)
+    q = p.store(H.stored_value(p, p.q) * H.sharp_factor(p))
+    (a, la), (b, lb) = (H.gpu_decode(lib, p, c, q) for c in caches)
+    assert lib.lr_cache_plan(caches[1]).n_splits == lib.lr_cache_plan(caches[0]).n_splits
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+    for c in caches:
+        lib.lr_cache_destroy(c)
