@@ -324,6 +324,14 @@ lr_status lr_cache_view_get(const lr_cache* cache, lr_cache_view* out);
  *   work as for contiguous caches; lr_basis_sync rotates every row of the pool (each page
  *   once, whatever maps it). */
 lr_status lr_cache_set_block_table(lr_cache* cache, const int32_t* table, void* stream);
+/* lr_cache_set_block_table_device — the same from a DEVICE array (int32, any alignment),
+ *   copied device to device on `stream`, so that a serving loop can update the
+ *   table inside a captured CUDA graph.  The library cannot check the entries without a host
+ *   round trip: every kernel clamps a page index outside [0, n_pages) into the pool, so a bad
+ *   entry gives wrong outputs for its sequence but never an access outside the cache's
+ *   storage.  The caller's array must stay valid until the copy has run.
+ *   LR_ERR_UNSUPPORTED for a cache that is not paged; LR_ERR_INVALID_ARG for NULL. */
+lr_status lr_cache_set_block_table_device(lr_cache* cache, const int32_t* table, void* stream);
 /* Force a decode path (LR_PATH_*) and/or a split count (0 = automatic). */
 lr_status lr_cache_set_path(lr_cache* cache, int32_t path, int32_t n_splits);
 /* The plan lr_attn_decode would use at the current length. */

@@ -12,7 +12,7 @@ lr_cache_truncate, lr_cache_view_get, lr_cache_set_path, lr_cache_plan,
 lr_plan_decode, lr_cache_set_kernel_events, lr_cache_set_trace, lr_device_error, lr_abi_struct_sizes,
 lr_status_string, lr_launch_count, lr_attn_decode_noalloc, lr_cache_set_wait_limit,
 lr_debug_inject_fault, lr_attn_decode_varlen, lr_attn_decode_partial, lr_merge_partials,
-lr_kv_prefill, lr_cache_set_block_table.
+lr_kv_prefill, lr_cache_set_block_table, lr_cache_set_block_table_device.
 """
 from __future__ import annotations
 
@@ -83,6 +83,7 @@ def _load() -> ctypes.CDLL:
         "lr_cache_truncate": [vp, i32],
         "lr_cache_view_get": [vp, ctypes.POINTER(lr_cache_view)],
         "lr_cache_set_block_table": [vp, vp, vp],
+        "lr_cache_set_block_table_device": [vp, vp, vp],
         "lr_cache_set_path": [vp, i32, i32],
         "lr_cache_plan": [vp, ctypes.POINTER(lr_plan)],
         "lr_plan_decode": [ctypes.POINTER(lr_cache_desc), i32, i32, i32, i32, ctypes.POINTER(lr_plan)],
@@ -388,6 +389,16 @@ def lr_cache_set_block_table(cache: Cache, table, stream=None) -> None:
         raise ValueError(f"table must be [{d.batch}][{d.capacity // 128}], got {t.shape}")
     _check(_lib.lr_cache_set_block_table(cache.handle, t.ctypes.data_as(ctypes.c_void_p), _stream(stream)),
            "lr_cache_set_block_table")
+
+
+def lr_cache_set_block_table_device(cache: Cache, table, stream=None) -> None:
+    """table: int32 CUDA tensor [batch][capacity / 128] (entries are not checked; the kernels
+    clamp them into the pool)."""
+    import torch
+    d = cache.desc
+    _check(_lib.lr_cache_set_block_table_device(cache.handle, _ptr(table, torch.int32, (d.batch, d.capacity // 128),
+                                                                   "table"), _stream(stream)),
+           "lr_cache_set_block_table_device")
 
 
 def lr_cache_set_path(cache: Cache, path: int = LR_PATH_AUTO, n_splits: int = 0) -> None:

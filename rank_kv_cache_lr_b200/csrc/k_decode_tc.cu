@@ -55,8 +55,7 @@ struct TcParams {
   unsigned long long wait_ns;   // bounded-wait limit (0: the default)
   const int32_t* row_len;       // per-row history lengths (device), or null
   unsigned long long* span;     // timeline span, or null
-  const int32_t* table;         // paged caches: block table [B][pps] (maps address pages), else null
-  int pps;
+  RowMap map;                   // paged caches: the block table (maps address pages), else table null
   int r_k, r_v, ck, cv, kb_k, tmem_cols;
   int Hq, hist_len, stable_len, split_tokens, n_splits, nslot;
   uint32_t q_bytes;
@@ -195,8 +194,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc::unit_of(u, ntiles, &tile, &isv);
         const int t0 = tok_begin + tile * kTile;
         // box origin: (token, sequence), or (0, page) in a paged pool (a tile is one page)
-        const int ty = p.table ? 0 : t0;
-        const int tz = p.table ? __ldg(p.table + (long long)b * p.pps + (t0 >> 7)) : b;
+        const int ty = p.map.table ? 0 : t0;
+        const int tz = p.map.table ? p.map.page(b, t0) : b;
         const int nch = isv ? p.cv : p.ck;
         const int r = isv ? p.r_v : p.r_k;
         for (int c = 0; c < nch; ++c, ++pos) {
@@ -556,8 +555,7 @@ cudaError_t launch_decode_tc(const lr_cache* c, int n_splits, int split_tokens, 
   p.wait_ns = c->wait_ns;
   p.row_len = c->row_len;
   p.span = span_of(c->spans, SPAN_DECODE);
-  p.table = c->ptable;
-  p.pps = c->pps;
+  p.map = row_map(c);
   p.r_k = d.rank_k;
   p.r_v = d.rank_v;
   p.ck = (d.rank_k + 127) / 128;

@@ -626,6 +626,19 @@ lr_status lr_cache_set_block_table(lr_cache* c, const int32_t* table, void* stre
   return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
 }
 
+lr_status lr_cache_set_block_table_device(lr_cache* c, const int32_t* table, void* stream) {
+  if (!c) return LR_ERR_INVALID_ARG;
+  if (!c->ptable) return LR_ERR_UNSUPPORTED;
+  if (!table) return LR_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  // a copy, not a kernel: the next kernel on the stream starts only after it has completed,
+  // so no dependent launch reads the table early
+  const cudaError_t e = cudaMemcpyAsync(c->ptable, table, (size_t)c->desc.batch * c->pps * sizeof(int32_t),
+                                        cudaMemcpyDeviceToDevice, s);
+  return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
+}
+
 lr_status lr_cache_set_path(lr_cache* c, int32_t path, int32_t n_splits) {
   if (!c || path < 0 || path > 2 || n_splits < 0) return LR_ERR_INVALID_ARG;
   if (path == LR_PATH_TC && !tc_supported(&c->desc)) return LR_ERR_UNSUPPORTED;

@@ -57,9 +57,14 @@ struct RowMap {
   const int32_t* table;   // paged: [B][pps] page of each 128-token span (device), else null
   long long cap;          // contiguous: rows per sequence
   int pps;                // paged: pages per sequence
+  int n_pages;            // paged: pages in the pool (table entries are clamped to it)
   __device__ __forceinline__ long long row(int b, int t) const {
-    return table ? ((long long)__ldg(table + (long long)b * pps + (t >> 7)) << 7) + (t & 127)
-                 : (long long)b * cap + t;
+    return table ? ((long long)page(b, t) << 7) + (t & 127) : (long long)b * cap + t;
+  }
+  // the page of token t of sequence b; an entry outside [0, n_pages) (a device-side table
+  // the library did not check) is clamped, so every access stays inside the pool
+  __device__ __forceinline__ int page(int b, int t) const {
+    return min(max(__ldg(table + (long long)b * pps + (t >> 7)), 0), n_pages - 1);
   }
 };
 
@@ -221,6 +226,7 @@ inline RowMap row_map(const lr_cache* c) {
   m.table = c->ptable;
   m.cap = c->lat_cap;
   m.pps = c->pps;
+  m.n_pages = c->n_pages;
   return m;
 }
 

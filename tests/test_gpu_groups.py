@@ -115,3 +115,30 @@ def test_grouped_sync_with_per_group_rotations_keeps_outputs(lib):
     # bf16 rounding of the rotated latents and of the new bases: the stated bars still hold
     H.compare(p, got, ref, lse, ref_lse, tag="groups after sync")
     lib.lr_cache_destroy(c)
+
+
+@pytest.mark.parametrize("quant_bits", [0, 4])
+def test_grouped_paged_equals_contiguous(lib, quant_bits):
+    """Latent groups in a paged cache (shuffled block table): bit-identical to the contiguous
+    grouped cache."""
+    import torch
+    g, r = 4, 64
+    p, compact = grouped_problem(g, r, quant_bits, batch=3, length=600)
+    cap = 640
+    caches = []
+    for paged in (False, True):
+        desc = lib.make_desc(p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim, r, r, cap,
+                             quant_bits=quant_bits, latent_groups=g, page_tokens=128 if paged else 0,
+                             n_pages=p.batch * (cap // 128) + 2 if paged else 0)
+        c = lib.lr_cache_create(desc, *(H.to_dev(p, compact[k]) for k in ("A_k", "B_k", "A_v", "B_v")))
+        if paged:
+            perm = np.random.default_rng(4).permutation(p.batch * (cap // 128) + 2)[:p.batch * (cap // 128)]
+            lib.lr_cache_set_block_table(c, perm.astype(np.int32).reshape(p.batch, cap // 128))
+        lib.lr_kv_append_latent(c, torch.from_numpy(np.ascontiguousarray(p.z_k)).cuda(),
+                                torch.from_numpy(np.ascontiguousarray(p.z_v)).cuda())
+        caches.append(c)
+    q = p.store(H.stored_value(p, p.q) * H.sharp_factor(p))
+    (a, la), (b, lb) = (H.gpu_decode(lib, p, c, q) for c in caches)
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+    for c in caches:
+        lib.lr_cache_destroy(c)

@@ -205,3 +205,62 @@ def test_block_table_refusals(lib):
     _same(before, _decode(lib, p, c0, q), "paged against contiguous")
     for c in (c0, c1):
         lib.lr_cache_destroy(c)
+
+
+def test_device_table_matches_host_table_and_clamps(lib):
+    """A block table set from device memory decodes like the same table set from the host;
+    entries outside the pool are clamped into it by the kernels (no error, no access outside
+    the storage): the result equals the host table with the clamped entries."""
+    import torch
+    p = synth.small_variant("qwen16k", batch=3, length=700)
+    cap = 768
+    n_pages, table = _shuffled_table(p, cap, spare=2, seed=9)
+    c = _create(lib, p, cap, True, n_pages, table)
+    q = p.store(H.stored_value(p, p.q) * H.sharp_factor(p))
+    host = _decode(lib, p, c, q)
+    lib.lr_cache_set_block_table_device(c, torch.from_numpy(table).cuda())
+    _same(host, _decode(lib, p, c, q), "device table")
+    bad = table.copy()
+    bad[1, 0], bad[2, 3] = -5, n_pages + 3
+    lib.lr_cache_set_block_table_device(c, torch.from_numpy(bad).cuda())
+    got = _decode(lib, p, c, q)
+    assert lib.lr_device_error(c) == 0
+    lib.lr_cache_set_block_table(c, np.clip(bad, 0, n_pages - 1))
+    _same(got, _decode(lib, p, c, q), "clamped entries")
+    lib.lr_cache_destroy(c)
+
+
+def test_device_table_update_inside_a_cuda_graph(lib):
+    """The device-side table update is capturable: a graph of (table update, decode) replayed
+    after the table's device buffer changes decodes with the new table."""
+    import torch
+    p = synth.small_variant("qwen4k", batch=2, length=600)
+    cap = 640
+    n_pages, table = _shuffled_table(p, cap, spare=0, seed=2)
+    c = _create(lib, p, cap, True, n_pages, table)
+    q = p.store(H.stored_value(p, p.q) * H.sharp_factor(p))
+    qd = H.to_dev(p, q)
+    out = torch.empty_like(qd)
+    tdev = torch.from_numpy(table).cuda()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        lib.lr_cache_set_block_table_device(c, tdev, stream=s)
+        lib.lr_attn_decode(c, qd, out, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        lib.lr_cache_set_block_table_device(c, tdev)
+        lib.lr_attn_decode(c, qd, out)
+    torch.cuda.synchronize()
+    for tab in (table[::-1].copy(), table):   # swapped rows, then the original
+        tdev.copy_(torch.from_numpy(tab))
+        g.replay()
+        torch.cuda.synchronize()
+        got = out.float().cpu().numpy()
+        lib.lr_cache_set_block_table(c, tab)
+        want, _ = _decode(lib, p, c, q)
+        assert np.array_equal(got, want)
+    del g
+    lib.lr_cache_destroy(c)
