@@ -382,10 +382,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         bool waited = false, ok = true;
         int issued_k = 0, issued_v = 0;   // tiles whose copies were issued, per side
+        // the latent row (block) of each unit is read one unit ahead, so that a paged cache's
+        // table read overlaps the waits and copies of the unit before
+        auto row_of_unit = [&](int u) -> long long {
+          int tl;
+          bool iv;
+          tc::unit_of(u, ntiles, &tl, &iv);
+          return p.map.row(b, tok_begin + tl * kTile);
+        };
+        long long row_next = nunits > 0 ? row_of_unit(0) : 0;
         for (int u = 0; u < nunits && ok; ++u) {
           int tile;
           bool is_v;
           tc::unit_of(u, ntiles, &tile, &is_v);
+          const long long row0 = row_next;   // a whole block: one page
+          if (u + 1 < nunits) row_next = row_of_unit(u + 1);
           const int t0 = tok_begin + tile * kTile;
           const int n = min(kTile, tok_end - t0);
           const int nr = is_v ? p.nrv : p.nrk;
@@ -397,7 +408,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (round > 0 && !(ok = wait_b(&aux->raw_empty[rs], (round - 1) & 1, aux, p.err))) break;
           const int G = is_v ? p.G_v : p.G_k;
-          const long long row0 = p.map.row(b, t0);   // a whole block: one page
           uint8_t* dst = raw + rs * p.raw_bytes;
           // one block of one side: G x 2 KB of codes and G x 512 B of params, at the same
           // offsets for the token-major keys and the rank-major values
