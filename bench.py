@@ -332,6 +332,47 @@ def paged_timing(L, p, W, dev, flush_l2) -> dict:
                       "median of 10 after 3"}
 
 
+def prefill_timing(L, p, W, dev, flush_l2, peaks) -> dict:
+    """lr_kv_prefill of the workload's whole context (B sequences x T tokens of exact keys and
+    values) into an empty cache of the layer's shape: CUDA events around the call, L2 flushed
+    before each, median of 5 after 2.  Bytes: the keys and values read plus the latents
+    written; flops: 2 D r per token and side."""
+    import numpy as np
+    import torch
+    import statistics
+    import rank_kv_cache_lr_b200 as lr
+    Bsz, Hq, Hkv, d, T = W["batch"], W["n_q_heads"], W["n_kv_heads"], W["head_dim"], W["length"]
+    D, qb = Hkv * d, W["quant_bits"]
+    to_dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(dev)
+    desc = lr.make_desc(Bsz, Hq, Hkv, d, L["rk"], L["rv"], T, quant_bits=qb, dtype=lr.LR_BF16)
+    c = lr.lr_cache_create(desc, to_dev(p.A_k), to_dev(p.B_k), to_dev(p.A_v), to_dev(p.B_v))
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    kx = (torch.randn((Bsz, T, D), generator=g, device=dev) * 0.05).to(torch.bfloat16)
+    vx = (torch.randn((Bsz, T, D), generator=g, device=dev) * 0.05).to(torch.bfloat16)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for i in range(7):
+        lr.lr_cache_truncate(c, 0)
+        flush_l2()
+        ev0.record()
+        lr.lr_kv_prefill(c, kx, vx)
+        ev1.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            ts.append(ev0.elapsed_time(ev1))
+    lr.lr_cache_destroy(c)
+    ms = statistics.median(ts)
+    nbytes = 2 * Bsz * T * D * 2 + Bsz * T * (latent_bytes_per_token(L["rk"], qb) + latent_bytes_per_token(L["rv"], qb))
+    flops = 2.0 * Bsz * T * D * (L["rk"] + L["rv"])
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    tfs = flops / (ms * 1e-3) / 1e12
+    return {"tokens": Bsz * T, "us_per_call": round(1000 * ms, 1), "GBps": round(gbs, 1),
+            "TFLOPs": round(tfs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 3),
+            "timing": "CUDA events around lr_kv_prefill of B x T tokens into an empty cache, L2 flushed before "
+                      "each, median of 5 after 2; bytes = keys and values read + latents written"}
+
+
 def traffic_record(kernel: str):
     """DRAM traffic per launch from a committed ncu summary, valid only while the kernel
     source is unchanged (matched by hash)."""
@@ -705,6 +746,8 @@ def run_workload(args, workload):
     if W["layers"] == 1 and not win and not W.get("groups") and world == 1:
         # the same layer in a paged cache: paging moves no bytes and adds no work
         res["run"]["paged"] = paged_timing(layers[0], host_p, W, dev, flush_l2)
+        # bulk prefill of the layer's whole context (the cache fill from exact keys / values)
+        res["run"]["prefill"] = prefill_timing(layers[0], host_p, W, dev, flush_l2, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(workload, host_p, args.cpu_seconds)
     if rank == 0:

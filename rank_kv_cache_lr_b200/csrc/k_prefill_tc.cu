@@ -43,6 +43,18 @@ struct PfParams {
   int* err;
 };
 
+// The code min(max(rint(x / sf), 0), 15) with the quotient rounded to fp32 as the division
+// rounds it (the append path's quantiser), at the cost of a multiply: y = x * (1/sf) lies within
+// 3 ulp of that rounded quotient, so it rounds to the same integer unless it is within a few
+// ulp of a half-integer, where the division itself decides.  |y| <= 20 keeps 4 ulp below
+// 1e-5; beyond that the clamp decides whatever the rounding.
+__device__ __forceinline__ uint32_t quant_code(float x, float sf, float rs) {
+  const float y = x * rs;
+  const float half_off = fabsf(y - floorf(y) - 0.5f);
+  const float q = half_off < 1e-5f ? rintf(__fdiv_rn(x, sf)) : rintf(y);
+  return (uint32_t)fminf(fmaxf(q, 0.0f), 15.0f);
+}
+
 //   full[s]   1 + tx   producer's TMA boxes of stage s -> MMA issuer
 //   empty[s]  1        MMA commit -> producer
 //   d_full    1        MMA commit after the last K block -> epilogue warps
@@ -205,17 +217,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (__half2float(zh) == 0.0f) zh = __ushort_as_half((unsigned short)0);
         const __half sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
         const float zf = __half2float(zh), sf = __half2float(sh);
+        const float rs = sf != 0.0f ? __frcp_rn(sf) : 0.0f;
         uint32_t code[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          uint32_t cval = 0;
-          if (e < nvalid && sf != 0.0f) {
-            float q = rintf(__fdiv_rn(__fsub_rn(__uint_as_float(v[e]), zf), sf));
-            q = fminf(fmaxf(q, 0.0f), 15.0f);
-            cval = (uint32_t)q;
-          }
-          code[e] = cval;
-        }
+        for (int e = 0; e < 32; ++e)
+          code[e] = (e < nvalid && sf != 0.0f) ? quant_code(__fsub_rn(__uint_as_float(v[e]), zf), sf, rs) : 0u;
         const int G_s = is_v ? p.G_v : p.G_k;
         if (!is_v) {
           if (valid) {
