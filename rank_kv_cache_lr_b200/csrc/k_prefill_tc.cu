@@ -9,8 +9,8 @@
 // One CTA per (128-token tile, sequence, side): warp 0 TMA-loads the tile's X (K-major,
 // 128-byte swizzle) and the matching rows of A (MN-major: 64 ranks per 128-byte row) per
 // 64-wide slice of D through a ring of stages; warp 1 issues the MMAs (bf16, fp32
-// accumulation in TMEM); four epilogue warps (thread = token row = TMEM lane) read each
-// 32-rank group of the row and store it: bf16 rows, or the int4 group quantiser of the
+// accumulation in TMEM); the epilogue warps (kEpiPerQuarter per TMEM lane quarter, taking
+// 32-rank groups in turn; thread = token row = TMEM lane) read each 32-rank group of the row and store it: bf16 rows, or the int4 group quantiser of the
 // append path (the same fp32 operations, so a given fp32 latent gets the same codes) in the
 // token-major key layout or the rank-major value layout (eight tokens' nibbles of one rank
 // gathered across eight lanes with shuffles).
@@ -28,7 +28,8 @@ using tc::drain_wait;
 using tc::kSmemLimit;
 using tc::kTile;
 
-constexpr int kThreads = 192;              // producer, MMA, 4 epilogue warps
+constexpr int kEpiPerQuarter = 4;          // epilogue warps per TMEM lane quarter
+constexpr int kThreads = 64 + 128 * kEpiPerQuarter;   // producer, MMA, the epilogue warps
 constexpr int kAuxBytes = 1024;
 constexpr int kXBytes = 128 * 128;         // X stage: 128 tokens x 64 dims x 2 B
 constexpr int kWBox = 64 * 128;            // A box: 64 dims (rows) x 64 ranks x 2 B
@@ -172,18 +173,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------- epilogue
+    // kEpiPerQuarter warps per TMEM lane quarter, taking 32-rank groups in turn: one warp
+    // per sub-partition left the epilogue's dependent chains (shuffles, index arithmetic)
+    // without another warp to hide their latency
     const int qd = warp & 3;
+    const int part = (warp - 2) >> 2;
     const int m = qd * 32 + lane;                       // token row of the tile
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const int t = tile * kTile + m;
     const bool valid = t < p.n;
     const long long row = valid ? p.map.row(b, p.slot0 + t) : 0;   // the table has no row past n
-    const bool ok = ptx::named_bar_and(1, 128, wait_b(&aux->d_full, 0, aux, p.err));
+    const bool ok = ptx::named_bar_and(1, 128 * kEpiPerQuarter, wait_b(&aux->d_full, 0, aux, p.err));
     if (ok) {
       ptx::tc_fence_after();
       const int G = (r + 31) / 32;
       const bool aligned = (p.slot0 & 7) == 0;
-      for (int g = 0; g < G; ++g) {
+      for (int g = part; g < G; g += kEpiPerQuarter) {
         uint32_t v[32];
         ptx::tmem_ld32(tmem + lane_off + g * 32, v);
         ptx::tmem_wait_ld();
@@ -259,11 +264,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else if (valid) {
             // a fill that starts inside a word shares it with older tokens: this token's
-            // nibbles only (the two atomics touch only its bits)
-            for (int e = 0; e < nvalid; ++e) {
-              uint32_t* w = p.codes_v + i4v_code_index(row, G_s, g * 32 + e);
-              atomicAnd(w, ~(15u << sh4));
-              if (code[e]) atomicOr(w, code[e] << sh4);
+            // nibbles only (the two atomics touch only its bits).  The loop runs to 32 with a
+            // guard so that code[] keeps constant indices and stays in registers.
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (e < nvalid) {
+                uint32_t* w = p.codes_v + i4v_code_index(row, G_s, g * 32 + e);
+                atomicAnd(w, ~(15u << sh4));
+                if (code[e]) atomicOr(w, code[e] << sh4);
+              }
             }
           }
         }
