@@ -253,6 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // is past n is not stored at all (its slots may lie beyond the storage).
             const int tb = t & ~7;
             const long long row_w = tb < p.n ? p.map.row(b, p.slot0 + tb) : 0;
+            // the word of rank g * 32 + e: its rank row's base, then the 16-byte column
+            // (token quarter ^ ((e / 2) % 4)) and the word in it (g * 32 is a multiple of 8,
+            // so the rotation depends on e alone)
+            uint32_t* vrow = p.codes_v + i4v_code_index(row_w, G_s, g * 32) - ((((row_w & 127) >> 5)) << 2);
+            const uint32_t tq = (uint32_t)((row_w & 127) >> 5);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               uint32_t w = valid ? code[e] << sh4 : 0u;
@@ -260,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               w |= __shfl_xor_sync(0xffffffffu, w, 2);
               w |= __shfl_xor_sync(0xffffffffu, w, 4);
               if ((lane & 7) == (e & 7) && e < nvalid && tb < p.n)
-                p.codes_v[i4v_code_index(row_w, G_s, g * 32 + e)] = w;
+                vrow[e * 16 + ((tq ^ (uint32_t)((e >> 1) & 3)) << 2)] = w;
             }
           } else if (valid) {
             // a fill that starts inside a word shares it with older tokens: this token's

@@ -30,7 +30,7 @@ def _tokens(p, n, seed):
     return p.store(k), p.store(v)
 
 
-@pytest.mark.parametrize("quant_bits,rank", [(0, 256), (4, 352), (0, 448), (4, 128)])
+@pytest.mark.parametrize("quant_bits,rank", [(0, 256), (4, 352), (0, 448), (4, 128), (0, 48), (4, 48)])
 @pytest.mark.parametrize("cuts", [[300], [13, 300], [64, 200]])
 def test_prefill_matches_oracle_projection(lib, quant_bits, rank, cuts):
     import torch
