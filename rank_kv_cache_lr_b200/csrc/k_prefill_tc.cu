@@ -258,14 +258,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             // so the rotation depends on e alone)
             uint32_t* vrow = p.codes_v + i4v_code_index(row_w, G_s, g * 32) - ((((row_w & 127) >> 5)) << 2);
             const uint32_t tq = (uint32_t)((row_w & 127) >> 5);
+            // per block of 8 ranks, a butterfly reduce-scatter over the word's 8 lanes: lane
+            // m of the word ends with the OR of all 8 lanes' nibbles of rank 8 jb + m (seven
+            // shuffles per block instead of three per rank)
+            const int m8 = lane & 7;
+            uint32_t* vlane = vrow + m8 * 16 + ((tq ^ (uint32_t)((m8 >> 1) & 3)) << 2);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              uint32_t w = valid ? code[e] << sh4 : 0u;
-              w |= __shfl_xor_sync(0xffffffffu, w, 1);
-              w |= __shfl_xor_sync(0xffffffffu, w, 2);
-              w |= __shfl_xor_sync(0xffffffffu, w, 4);
-              if ((lane & 7) == (e & 7) && e < nvalid && tb < p.n)
-                vrow[e * 16 + ((tq ^ (uint32_t)((e >> 1) & 3)) << 2)] = w;
+            for (int jb = 0; jb < 4; ++jb) {
+              uint32_t x[8];
+#pragma unroll
+              for (int m = 0; m < 8; ++m) x[m] = valid ? code[8 * jb + m] << sh4 : 0u;
+#pragma unroll
+              for (int dd = 4; dd >= 1; dd >>= 1) {
+                const bool up = (lane & dd) != 0;
+#pragma unroll
+                for (int k = 0; k < dd; ++k) {
+                  const uint32_t keep = up ? x[k + dd] : x[k];
+                  const uint32_t send = up ? x[k] : x[k + dd];
+                  x[k] = keep | __shfl_xor_sync(0xffffffffu, send, dd);
+                }
+              }
+              if (8 * jb + m8 < nvalid && tb < p.n) vlane[jb * 128] = x[0];
             }
           } else if (valid) {
             // a fill that starts inside a word shares it with older tokens: this token's
