@@ -81,32 +81,41 @@ using tc::kTile;
 using tc::kTraceSlots;
 using tc::warp_reduce_scatter32;
 
-// 16 warps in four warpgroups: [producer, key MMAs, B_k producer / idle, value MMAs] [4 softmax]
-// [4 key dequantisation] [4 value dequantisation].  A warp runs on sub-partition (warp % 4), and a tcgen05.ld / st
-// reaches TMEM lanes 32 (warp % 4) .. + 31.  Launched at 128 registers per thread; the
-// warpgroups then rebalance the block's 64K registers with setmaxnreg (the softmax keeps
-// 32 scores and 32 running sums per row).
-constexpr int kThreads = 512;
+// Warpgroups: [producer, key MMAs, B_k producer / idle, value MMAs] [4 softmax] [key
+// dequantisation] [value dequantisation], with 4 or 8 warps per dequantisation side (Cfg).  A
+// warp runs on sub-partition (warp % 4), and a tcgen05.ld / st reaches TMEM lanes
+// 32 (warp % 4) .. + 31.  The warpgroups rebalance the launch's registers with setmaxnreg
+// (the softmax keeps 32 scores and 32 running sums per row).
 constexpr int kDqWarp0 = 8;                // first warp of the dequantisation warpgroups
-constexpr int kDqSide = 4;                 // arrivals per operand slot / raw slot (the side's warps)
 constexpr int kSmWarps = 4;                // softmax warps (one arrival each)
-constexpr int kLaunchRegs = 128;
-// Per-warpgroup register budgets of each variant (the smallest that ptxas fits without
-// spilling; multiples of 8): control, softmax / epilogue, dequantisation.
-template <bool kRope> struct Regs;
-template <> struct Regs<false> { static constexpr int ctl = 64, softmax = 184, dq = 120; };
-template <> struct Regs<true> { static constexpr int ctl = 64, softmax = 240, dq = 104; };
+// Per variant: dequantisation warps per TMEM lane quarter and side (rank space: two, each
+// expanding one 32-column half of every chunk, so that a sub-partition holds two warps of each
+// side to hide each other's latency; keys before RoPE: one, expanding both halves), the block
+// size, the launch allocation, and the per-warpgroup register budgets (multiples of 8):
+// control, softmax / epilogue, dequantisation.  The budgets fill the launch allocation.
+template <bool kRope> struct Cfg;
+template <> struct Cfg<false> {
+  static constexpr int dq_per_quarter = 2, threads = 256 + 256 * dq_per_quarter, launch_regs = 80;
+  static constexpr int ctl = 48, softmax = 176, dq = 64;
+};
+template <> struct Cfg<true> {
+  static constexpr int dq_per_quarter = 1, threads = 256 + 256 * dq_per_quarter, launch_regs = 128;
+  static constexpr int ctl = 64, softmax = 240, dq = 104;
+};
+template <bool kRope> using Regs = Cfg<kRope>;
 // Move this warpgroup from the launch allocation to `kTo` registers per thread: setmaxnreg.inc
 // when raising, .dec when lowering (a .dec above the current count is an illegal instruction).
-template <int kTo>
+template <int kTo, int kFrom>
 __device__ __forceinline__ void set_regs() {
   static_assert(kTo % 8 == 0 && kTo >= 24 && kTo <= 256, "setmaxnreg range");
-  if constexpr (kTo > kLaunchRegs) ptx::setmaxnreg_inc<kTo>();
-  else if constexpr (kTo < kLaunchRegs) ptx::setmaxnreg_dec<kTo>();
+  if constexpr (kTo > kFrom) ptx::setmaxnreg_inc<kTo>();
+  else if constexpr (kTo < kFrom) ptx::setmaxnreg_dec<kTo>();
 }
-static_assert(128 * Regs<false>::ctl + 128 * Regs<false>::softmax + 256 * Regs<false>::dq <= kThreads * kLaunchRegs,
+static_assert(128 * Cfg<false>::ctl + 128 * Cfg<false>::softmax + 256 * Cfg<false>::dq_per_quarter * Cfg<false>::dq <=
+                  Cfg<false>::threads * Cfg<false>::launch_regs,
               "register split exceeds the launch allocation");
-static_assert(128 * Regs<true>::ctl + 128 * Regs<true>::softmax + 256 * Regs<true>::dq <= kThreads * kLaunchRegs,
+static_assert(128 * Cfg<true>::ctl + 128 * Cfg<true>::softmax + 256 * Cfg<true>::dq_per_quarter * Cfg<true>::dq <=
+                  Cfg<true>::threads * Cfg<true>::launch_regs,
               "register split exceeds the launch allocation");
 constexpr int kSubBytes = 128 * 128;       // B_k ring: 128 rows x 64 ranks x 2 B per KV head
 constexpr int kQRows = 32;                 // query heads, padded
@@ -278,7 +287,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 //                [B_k ring nb x gh x 16 KB (kRope)][P double buffer 2 x 8 KB]
 //                [raw ring nraw x raw_bytes]
 template <bool kRope>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<kRope>::threads, 1)
     k_decode_tc_i4(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_b,
                    const I4Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -313,12 +322,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     tc::trace_stamp(p.trace, 0);
     for (int s = 0; s < p.nks + p.nvs; ++s) {
-      ptx::mbar_init(&aux->slot_full[s], kDqSide);
+      ptx::mbar_init(&aux->slot_full[s], 4 * Cfg<kRope>::dq_per_quarter);
       ptx::mbar_init(&aux->slot_empty[s], 1);
     }
     for (int s = 0; s < p.nrk + p.nrv; ++s) {
       ptx::mbar_init(&aux->raw_full[s], 1);
-      ptx::mbar_init(&aux->raw_empty[s], kDqSide);
+      ptx::mbar_init(&aux->raw_empty[s], 4 * Cfg<kRope>::dq_per_quarter);
     }
     for (int k = 0; k < 2; ++k) {
       ptx::mbar_init(&aux->s_full[k], 1);
@@ -364,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Roles by warpgroup; each sets its register budget first thing in its own branch,
   // so the compiler allocates that branch within the budget.
   if (warp < 4) {
-    set_regs<Regs<kRope>::ctl>();
+    set_regs<Regs<kRope>::ctl, Cfg<kRope>::launch_regs>();
     if (warp == 0) {
       // ------------------------------------------------------------- bulk-copy producer
       if (lane == 0 && ntiles > 0) {
@@ -580,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     }
   } else if (warp < kDqWarp0) {
-    set_regs<Regs<kRope>::softmax>();
+    set_regs<Regs<kRope>::softmax, Cfg<kRope>::launch_regs>();
     if (ntiles > 0) {
       // ------------------------------------------------------------- softmax / epilogue
       const int qd = warp & 3;
@@ -840,16 +849,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    set_regs<Regs<kRope>::dq>();
+    set_regs<Regs<kRope>::dq, Cfg<kRope>::launch_regs>();
     // ------------------------------------------------------------- dequantisation
     if (ntiles > 0) {
-      // side = 0 (warps 8..11): keys; side = 1 (warps 12..15): values.  Warp quarter
-      // qd = warp % 4 owns TMEM lanes 32 qd .. + 31 of every operand slot of its side and
-      // fills all 64 columns, in two halves h of 32 columns.  Keys: token 32 qd + lane, ranks
+      // side = 0: keys (warps 8 .. 8 + 4 kDqPQ - 1), side = 1: values (the next 4 kDqPQ).
+      // Warp quarter qd = warp % 4 owns TMEM lanes 32 qd .. + 31 of every operand slot of its
+      // side and fills its 64 columns in two halves h of 32 columns (both halves, or with
+      // two warps per quarter one half each).  Keys: token 32 qd + lane, ranks
       // 64 h .. + 63 of the chunk (groups 4c + 2h, + 1).  Values: rank 128 c + 32 qd + lane
       // (group 4c + qd), tokens 64 h .. + 63.
       const int qd = warp & 3;
-      const bool is_v = warp >= kDqWarp0 + 4;
+      constexpr int kDqPQ = Cfg<kRope>::dq_per_quarter;
+      const int dqj = warp - kDqWarp0;                   // [0, 8 kDqPQ): the side's warps, keys first
+      const bool is_v = dqj >= 4 * kDqPQ;
+      // with two warps per quarter, warp (dqj / 4) % 2 of the side expands half h of each chunk
+      const int h_beg = kDqPQ == 2 ? (dqj >> 2) & 1 : 0, h_end = kDqPQ == 2 ? h_beg + 1 : 2;
       const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
       const uint32_t raw_base = ptx::smem_u32(raw);
       const int G = is_v ? p.G_v : p.G_k;
@@ -872,7 +886,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tc_fence_after();
           bool stored = false;
 #pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
+          for (int h = h_beg; h < h_end; ++h) {
             uint32_t v[32];
             bool any = false;
             if (!is_v) {
@@ -1148,7 +1162,8 @@ cudaError_t launch_decode_tc_i4(const lr_cache* c, int n_splits, int split_token
     cudaFuncAttributes fa;
     regs[ki].store(cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1);
   }
-  if (regs[ki].load() != kLaunchRegs) return cudaErrorInvalidConfiguration;
+  if (regs[ki].load() != (rope ? Cfg<true>::launch_regs : Cfg<false>::launch_regs))
+    return cudaErrorInvalidConfiguration;
   const dim3 grid = rope ? dim3(d.n_kv_heads / p.gh, n_splits, d.batch) : dim3(n_splits, d.batch);
-  return launch_pdl(kern, grid, dim3(kThreads), st->smem, s, st->q, st->bk, p);
+  return launch_pdl(kern, grid, dim3(rope ? Cfg<true>::threads : Cfg<false>::threads), st->smem, s, st->q, st->bk, p);
 }
