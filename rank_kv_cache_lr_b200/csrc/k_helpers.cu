@@ -149,45 +149,55 @@ __device__ __forceinline__ void qproj_main(const QprojArgs& a, int rchunk, int h
   if (!a.want_latent) return;
   cp_async_wait_all();
   __syncthreads();
-  for (int bb = 0; bb < nb; ++bb) {
-  const int b = b0 + bb;
-  const float* qs = qs_all + (size_t)bb * G * d;
+  // thread = (rank row, query head); each 8-element run of the B_k row is read and converted
+  // once for the CTA's sequences (the per-output sums keep their order)
   const int r0 = rchunk * kQRowsCta;
   const int nr = min(kQRowsCta, a.rk - r0);
   const int t = threadIdx.x & 31;            // rank row within the chunk
   const int i = r0 + t;
   const uint8_t* row = smem + (size_t)t * pitch;
   for (int u = threadIdx.x >> 5; u < G && t < nr; u += (int)(blockDim.x >> 5)) {
-    const float* qj = qs + u * d;
-    float acc0 = 0.f, acc1 = 0.f;
+    float acc0[kRows], acc1[kRows];
+#pragma unroll
+    for (int bb = 0; bb < kRows; ++bb) acc0[bb] = acc1[bb] = 0.f;
     for (int c = 0; c < d; c += 8) {
       float bv[8];
       El<T>::lds8(row + (size_t)c * sizeof(T), bv);
-      const float4 q0 = *reinterpret_cast<const float4*>(qj + c);
-      const float4 q1 = *reinterpret_cast<const float4*>(qj + c + 4);
-      acc0 = fmaf(bv[0], q0.x, acc0);
-      acc1 = fmaf(bv[1], q0.y, acc1);
-      acc0 = fmaf(bv[2], q0.z, acc0);
-      acc1 = fmaf(bv[3], q0.w, acc1);
-      acc0 = fmaf(bv[4], q1.x, acc0);
-      acc1 = fmaf(bv[5], q1.y, acc1);
-      acc0 = fmaf(bv[6], q1.z, acc0);
-      acc1 = fmaf(bv[7], q1.w, acc1);
+#pragma unroll
+      for (int bb = 0; bb < kRows; ++bb) {
+        if (bb < nb) {
+          const float* qj = qs_all + ((size_t)bb * G + u) * d;
+          const float4 q0 = *reinterpret_cast<const float4*>(qj + c);
+          const float4 q1 = *reinterpret_cast<const float4*>(qj + c + 4);
+          acc0[bb] = fmaf(bv[0], q0.x, acc0[bb]);
+          acc1[bb] = fmaf(bv[1], q0.y, acc1[bb]);
+          acc0[bb] = fmaf(bv[2], q0.z, acc0[bb]);
+          acc1[bb] = fmaf(bv[3], q0.w, acc1[bb]);
+          acc0[bb] = fmaf(bv[4], q1.x, acc0[bb]);
+          acc1[bb] = fmaf(bv[5], q1.y, acc1[bb]);
+          acc0[bb] = fmaf(bv[6], q1.z, acc0[bb]);
+          acc1[bb] = fmaf(bv[7], q1.w, acc1[bb]);
+        }
+      }
     }
     const int j = j0 + u;
-    const float v = (acc0 + acc1) * a.scale_log2;
-    a.qt[((size_t)b * a.Hq + j) * a.rk + i] = v;
-    if (a.qt16 && a.qt16_fp16) {
-      const int pos = (i & ~7) | ((i & 3) << 1) | ((i >> 2) & 1);
-      reinterpret_cast<__half*>(a.qt16)[((size_t)b * 32 + j) * a.rk + pos] = __float2half_rn(v);
-    } else if (a.qt16) {
-      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-      __nv_bfloat16* q16 = reinterpret_cast<__nv_bfloat16*>(a.qt16);
-      q16[((size_t)b * 64 + j) * a.rk + i] = hi;
-      q16[((size_t)b * 64 + 32 + j) * a.rk + i] = lo;
+#pragma unroll
+    for (int bb = 0; bb < kRows; ++bb) {
+      if (bb >= nb) continue;
+      const int b = b0 + bb;
+      const float v = (acc0[bb] + acc1[bb]) * a.scale_log2;
+      a.qt[((size_t)b * a.Hq + j) * a.rk + i] = v;
+      if (a.qt16 && a.qt16_fp16) {
+        const int pos = (i & ~7) | ((i & 3) << 1) | ((i >> 2) & 1);
+        reinterpret_cast<__half*>(a.qt16)[((size_t)b * 32 + j) * a.rk + pos] = __float2half_rn(v);
+      } else if (a.qt16) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+        __nv_bfloat16* q16 = reinterpret_cast<__nv_bfloat16*>(a.qt16);
+        q16[((size_t)b * 64 + j) * a.rk + i] = hi;
+        q16[((size_t)b * 64 + 32 + j) * a.rk + i] = lo;
+      }
     }
-  }
   }
 }
 
