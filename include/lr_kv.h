@@ -166,6 +166,18 @@ lr_status lr_cache_destroy(lr_cache* cache);
  *   LR_ERR_CAPACITY when len == capacity. */
 lr_status lr_kv_append(lr_cache* cache, const void* k, const void* v, void* stream);
 
+/* lr_kv_append_rows — append one token per sequence, each row at its own slot (a serving
+ *   batch whose sequences are at different lengths; read with lr_attn_decode_varlen).
+ *   k, v: [B][D] in dtype, 16-byte aligned (else LR_ERR_INVALID_ARG).  pos: [B] int32,
+ *   device: row b's latents z = k_b A_k, z_v = v_b A_v are stored (as lr_kv_append stores
+ *   them) at history slot pos[b]; a row whose pos lies outside [0, capacity) writes nothing,
+ *   and the other slots are untouched.  max_len (host): the history length becomes
+ *   max(history length, max_len), the caller's bound on every row's pos + 1; 0 <= max_len
+ *   <= capacity (LR_ERR_INVALID_ARG below, LR_ERR_CAPACITY above).  Caches with a window
+ *   return LR_ERR_UNSUPPORTED.  Graph-capturable: pos is read on the device. */
+lr_status lr_kv_append_rows(lr_cache* cache, const void* k, const void* v, const int32_t* pos,
+                            int32_t max_len, void* stream);
+
 /* lr_kv_prefill — append n tokens per sequence from their exact keys and values (a prompt).
  *   k, v: [B][n][D] in dtype, 16-byte aligned (else LR_ERR_INVALID_ARG).  Each token's latents
  *   z = k A_k, z_v = v A_v are computed in fp32 and stored at slots len .. len + n - 1

@@ -12,7 +12,7 @@ lr_cache_truncate, lr_cache_view_get, lr_cache_set_path, lr_cache_plan,
 lr_plan_decode, lr_cache_set_kernel_events, lr_cache_set_trace, lr_device_error, lr_abi_struct_sizes,
 lr_status_string, lr_launch_count, lr_attn_decode_noalloc, lr_cache_set_wait_limit,
 lr_debug_inject_fault, lr_attn_decode_varlen, lr_attn_decode_partial, lr_merge_partials,
-lr_kv_prefill, lr_cache_set_block_table, lr_cache_set_block_table_device.
+lr_kv_prefill, lr_cache_set_block_table, lr_cache_set_block_table_device, lr_kv_append_rows.
 """
 from __future__ import annotations
 
@@ -94,6 +94,7 @@ def _load() -> ctypes.CDLL:
         "lr_attn_decode_varlen": [vp, vp, vp, vp, vp, vp],
         "lr_attn_decode_partial": [vp, vp, vp, vp, vp],
         "lr_kv_prefill": [vp, vp, vp, i32, vp],
+        "lr_kv_append_rows": [vp, vp, vp, vp, i32, vp],
         "lr_merge_partials": [vp, i32, vp, vp, vp, vp, vp],
         "lr_debug_inject_fault": [i32, ctypes.c_int64],
         "lr_attn_decode_noalloc": [ctypes.POINTER(lr_cache_desc), i32, vp, vp, vp, vp, vp, vp, vp, vp],
@@ -225,6 +226,16 @@ def lr_kv_append(cache: Cache, k, v, stream=None) -> None:
     d, dt = cache.desc, _torch_dtype(cache.desc.dtype)
     _check(_lib.lr_kv_append(cache.handle, _ptr(k, dt, (d.batch, cache.D), "k"),
                              _ptr(v, dt, (d.batch, cache.D), "v"), _stream(stream)), "lr_kv_append")
+
+
+def lr_kv_append_rows(cache: Cache, k, v, pos, max_len: int, stream=None) -> None:
+    """pos: int32 CUDA tensor [batch], the history slot of each row's token."""
+    import torch
+    d, dt = cache.desc, _torch_dtype(cache.desc.dtype)
+    _check(_lib.lr_kv_append_rows(cache.handle, _ptr(k, dt, (d.batch, cache.D), "k"),
+                                  _ptr(v, dt, (d.batch, cache.D), "v"),
+                                  _ptr(pos, torch.int32, (d.batch,), "pos"), int(max_len), _stream(stream)),
+           "lr_kv_append_rows")
 
 
 def lr_kv_prefill(cache: Cache, k, v, stream=None) -> None:

@@ -231,6 +231,8 @@ struct AppendArgs {
   void* Zk; void* Zv; uint32_t* codes_k; uint32_t* codes_v; uint32_t* params_k; uint32_t* params_v;
   int rk, rv, Gk, Gv, chunks_k, chunks_v;
   RowMap map; int dst_slot; int project;
+  const int32_t* row_pos;                 // per-row destination slots (device), or null: dst_slot
+  int cap;                                // slots per sequence (a row_pos outside [0, cap) writes nothing)
   const void* new_k; const void* new_v;   // exact token for the ring, or null
   void* win_k; void* win_v; int slots; int new_slot;
   unsigned long long* span;   // timeline span, or null
@@ -300,9 +302,12 @@ __device__ __forceinline__ void append_main(const AppendArgs& a, int x, int b0, 
       float zz = 0.f;
 #pragma unroll
       for (int w = 0; w < 8; ++w) zz += red[w][warp][lane];
-      const long long row = a.map.row(b0 + warp, a.dst_slot);
-      store_latent_chunk(zz, ch, r, a.kind, a.dtype, is_k ? a.Zk : a.Zv, is_k ? a.codes_k : a.codes_v,
-                         is_k ? a.params_k : a.params_v, is_k ? a.Gk : a.Gv, row, !is_k);
+      const int slot = a.row_pos ? __ldg(a.row_pos + b0 + warp) : a.dst_slot;
+      if (slot >= 0 && slot < a.cap) {
+        const long long row = a.map.row(b0 + warp, slot);
+        store_latent_chunk(zz, ch, r, a.kind, a.dtype, is_k ? a.Zk : a.Zv, is_k ? a.codes_k : a.codes_v,
+                           is_k ? a.params_k : a.params_v, is_k ? a.Gk : a.Gv, row, !is_k);
+      }
     }
     return;
   }
@@ -703,6 +708,7 @@ AppendArgs make_append_args(const lr_cache* c, const void* k, const void* v) {
   a.rk = d.rank_k; a.rv = d.rank_v; a.Gk = c->G_k; a.Gv = c->G_v;
   a.chunks_k = (d.rank_k + 31) / 32; a.chunks_v = (d.rank_v + 31) / 32;
   a.map = row_map(c); a.dst_slot = c->hist_len;
+  a.row_pos = nullptr; a.cap = d.capacity;
   a.new_k = win ? k : nullptr; a.new_v = win ? v : nullptr;
   a.win_k = c->win_k; a.win_v = c->win_v; a.slots = c->win_slots;
   a.new_slot = win ? (c->len % c->win_slots) : 0;
@@ -761,9 +767,11 @@ cudaError_t merge_t(const lr_cache* c, int n_splits, void* out, float* lse, cuda
 }
 
 template <typename T>
-cudaError_t append_t(lr_cache* c, const void* k, const void* v, cudaStream_t s, long long bstride) {
+cudaError_t append_t(lr_cache* c, const void* k, const void* v, cudaStream_t s, long long bstride,
+                     const int32_t* row_pos) {
   AppendArgs a = make_append_args(c, k, v);
   if (bstride && !c->win_slots) a.src_bstride = bstride;
+  if (!c->win_slots) a.row_pos = row_pos;
   static std::atomic<uint32_t> optin_done{0};
   cudaError_t e = smem_optin(k_append<T>, optin_done);
   if (e != cudaSuccess) return e;
@@ -804,8 +812,10 @@ cudaError_t launch_merge(const lr_cache* c, int n_splits, void* out, float* lse,
                                   : merge_t<float>(c, n_splits, out, lse, s, src);
 }
 
-cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s, long long bstride) {
-  return c->desc.dtype == LR_BF16 ? append_t<__nv_bfloat16>(c, k, v, s, bstride) : append_t<float>(c, k, v, s, bstride);
+cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s, long long bstride,
+                          const int32_t* row_pos) {
+  return c->desc.dtype == LR_BF16 ? append_t<__nv_bfloat16>(c, k, v, s, bstride, row_pos)
+                                  : append_t<float>(c, k, v, s, bstride, row_pos);
 }
 
 cudaError_t launch_step_pre(lr_cache* c, const void* k, const void* v, const void* q, bool tc, cudaStream_t s) {

@@ -338,6 +338,22 @@ lr_status lr_kv_append(lr_cache* c, const void* k, const void* v, void* stream) 
   return LR_OK;
 }
 
+lr_status lr_kv_append_rows(lr_cache* c, const void* k, const void* v, const int32_t* pos, int32_t max_len,
+                            void* stream) {
+  if (!c || !k || !v || !pos || !c->has_A) return LR_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15) return LR_ERR_INVALID_ARG;
+  if (c->win_slots) return LR_ERR_UNSUPPORTED;
+  if (max_len < 0) return LR_ERR_INVALID_ARG;
+  if (max_len > c->desc.capacity) return LR_ERR_CAPACITY;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  c->undo = 0;
+  cudaError_t e = launch_append(c, k, v, s, 0, pos);
+  if (e != cudaSuccess) return LR_ERR_CUDA;
+  if (max_len > c->hist_len) c->hist_len = c->len = max_len;
+  return LR_OK;
+}
+
 lr_status lr_kv_prefill(lr_cache* c, const void* k, const void* v, int32_t n, void* stream) {
   if (!c || !k || !v || n < 0 || !c->has_A) return LR_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15) return LR_ERR_INVALID_ARG;

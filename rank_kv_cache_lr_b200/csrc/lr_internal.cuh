@@ -182,7 +182,9 @@ cudaError_t launch_basis_update(lr_cache* c, int side, const void* blk, int n, f
                                 void* B_out, void* A_out, cudaStream_t s);
 void isvd_release(lr_cache* c);
 // bstride: elements between the batch rows of k and v (0: D, rows of one token per sequence)
-cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s, long long bstride = 0);
+// row_pos: per-row destination slots (device), or null: the cache's next slot for every row
+cudaError_t launch_append(lr_cache* c, const void* k, const void* v, cudaStream_t s, long long bstride = 0,
+                          const int32_t* row_pos = nullptr);
 // bulk prefill on tensor cores (k_prefill_tc.cu): n tokens per sequence, k / v [B][n][D]
 bool prefill_tc_supported(const lr_cache_desc* d, int D);
 cudaError_t launch_prefill_tc(lr_cache* c, const void* k, const void* v, int n, cudaStream_t s);

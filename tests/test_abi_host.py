@@ -120,6 +120,7 @@ def test_noalloc_refuses_paged_desc_before_any_device_call(lib):
 
 def test_null_arguments(lib):
     assert lib.raw_status("lr_kv_append", None, None, None, None) == lib.LR_ERR_INVALID_ARG
+    assert lib.raw_status("lr_kv_append_rows", None, None, None, None, 0, None) == lib.LR_ERR_INVALID_ARG
     assert lib.raw_status("lr_attn_decode", None, None, None, None, None) == lib.LR_ERR_INVALID_ARG
     assert lib.raw_status("lr_cache_destroy", None) == lib.LR_OK
 
