@@ -300,13 +300,16 @@ def test_sync_identity_is_bit_exact(lib):
     assert np.array_equal(before, after)
 
 
-@pytest.mark.parametrize("which", ["kv", "k", "v"])
-def test_sync_tensor_core_matches_oracle_and_cuda_cores(lib, which):
+@pytest.mark.parametrize("which,hist,batch", [("kv", 700, 2), ("k", 700, 2), ("v", 700, 2),
+                                              ("kv", 5000, 4), ("v", 5000, 4)])
+def test_sync_tensor_core_matches_oracle_and_cuda_cores(lib, which, hist, batch):
     """The tensor-core sync (bf16 latents, r <= 256) against the oracle's rounded fp64
     Z R and against the CUDA-core sync: several 128-token tiles plus a ragged tail,
-    two sequences, one side or both."""
+    several sequences, one side or both; at 5000 tokens x 4 sequences there are more
+    tiles than SMs, so each CTA runs several tiles through its two tile buffers and two
+    accumulators."""
     import torch
-    p = synth.small_variant("hybrid", hist_len=700, batch=2)
+    p = synth.small_variant("hybrid", hist_len=hist, batch=batch)
     c_tc, c_simt = H.fill_cache(lib, p), H.fill_cache(lib, p)
     lib.lr_cache_set_path(c_simt, lib.LR_PATH_SIMT)
     Rk = synth.sync_rotation(0, 3, p.rank_k, "k").astype(np.float32)
