@@ -179,15 +179,36 @@ template <> __device__ __forceinline__ float win_elem<__nv_bfloat16>(const uint8
   return __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(p)) << 16);
 }
 
+// Window attention arguments.  Two modes:
+//  - after the latent decode (lr_attn_decode): q_in is null; the query comes scaled from qd
+//    (written by the query projection) and the newest token from its ring slot, both after
+//    the dependency wait;
+//  - right after the step's append and query projection (lr_decode_step): q_in, k_new, v_new
+//    are the step's inputs; the newest window token is read from k_new / v_new (the append
+//    copies those rows into its ring slot unchanged) and the query is scaled here as the
+//    projection scales it, so the result is the same; hist_len / win_len are the counters
+//    after the append.  Nothing here reads what that kernel writes, so the whole window runs
+//    before the dependency wait, alongside it; the wait comes last, because the decode after
+//    this kernel waits only for this grid, and through it for the append and projection.
+// In both, the window tokens before the newest were written by earlier steps' kernels, which
+// completed before the kernel just before this one passed its own wait (and this grid starts
+// only after that kernel's CTAs have), so their rows are copied before this kernel's wait.
+struct WinArgs {
+  const void* win_k; const void* win_v; const float* qd;
+  const void* q_in; const void* k_new; const void* v_new; float scale_log2;
+  float* win_o; float* win_ml;
+  int Hq, Hkv, d, D, slots, hist_len, win_len;
+  unsigned long long* span;
+};
+
 template <typename T>
-__global__ void __launch_bounds__(kWinThreads) k_window(const void* win_k, const void* win_v, const float* qd,
-                                                        float* win_o, float* win_ml, int Hq, int Hkv, int d,
-                                                        int D, int slots, int hist_len, int win_len,
-                                                        unsigned long long* span) {
+__global__ void __launch_bounds__(kWinThreads) k_window(const WinArgs a) {
   extern __shared__ __align__(16) uint8_t wsm_raw[];
   constexpr int es = sizeof(T);
   constexpr int dtype = es == 2 ? LR_BF16 : LR_F32;
-  const int G = Hq / Hkv;
+  const int Hq = a.Hq, d = a.d, D = a.D, slots = a.slots, hist_len = a.hist_len, win_len = a.win_len;
+  const int G = Hq / a.Hkv;
+  const bool step = a.q_in != nullptr;
   const int pitch = window_pitch(d, es);
   float* q_s = reinterpret_cast<float*>(wsm_raw);          // [d]
   float* o_s = q_s + d;                                    // [d] (unused slot kept for alignment)
@@ -195,9 +216,8 @@ __global__ void __launch_bounds__(kWinThreads) k_window(const void* win_k, const
   uint8_t* v_s = k_s + kWinTok * pitch;
   float* p_s = reinterpret_cast<float*>(v_s + kWinTok * pitch);   // [kWinTok]
   float* red = p_s + kWinTok;                              // [8]: warp maxima, then warp sums
-  span_begin(span);
-  pdl_wait();
-  pdl_trigger();
+  span_begin(a.span);
+  pdl_trigger();   // the next kernel may start its own prologue
   const int h = blockIdx.x, b = blockIdx.y, u = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   constexpr int nw = kWinThreads / 32;
@@ -207,34 +227,71 @@ __global__ void __launch_bounds__(kWinThreads) k_window(const void* win_k, const
   // over rows (no division per copy); otherwise (odd head dims) the general walk
   const bool fixed = (kWinThreads % vpr) == 0;
   const int rstep = fixed ? kWinThreads / vpr : 0;
-  for (int v = tid; v < d / 4; v += kWinThreads) cp_async16(q_s + 4 * v, qd + ((long long)b * Hq + j) * d + 4 * v);
-  float m = -INFINITY, l = 0.f;
-  float o = 0.f;                                           // output column tid (d <= 128 here: tid < d)
-  float o2 = 0.f;                                          // column tid + 128 (d > 128)
-  const uint8_t* gk = reinterpret_cast<const uint8_t*>(win_k) + ((long long)b * slots * D + (long long)h * d) * es;
-  const uint8_t* gv = reinterpret_cast<const uint8_t*>(win_v) + ((long long)b * slots * D + (long long)h * d) * es;
-  for (int t0 = 0; t0 < win_len; t0 += kWinTok) {
-    const int n = min(kWinTok, win_len - t0);
-    __syncthreads();   // the previous round's rows and weights are no longer read
+  const uint8_t* gk = reinterpret_cast<const uint8_t*>(a.win_k) + ((long long)b * slots * D + (long long)h * d) * es;
+  const uint8_t* gv = reinterpret_cast<const uint8_t*>(a.win_v) + ((long long)b * slots * D + (long long)h * d) * es;
+  // rows [t0, t0 + n) of the window into staging rows 0.. (ring slot of window position t:
+  // (hist_len + t) % slots), except position `skip`
+  auto issue = [&](int t0, int n, int skip) {
     if (fixed) {
       const int v = tid % vpr;
       int t = tid / vpr;
-      int slot = (hist_len + t0 + t) % slots;               // ring slot of token t0 + t
+      int slot = (hist_len + t0 + t) % slots;
       const int sstep = rstep % slots;
       for (; t < n; t += rstep) {
-        const long long off = (long long)slot * D * es + v * 16;
-        cp_async16(k_s + t * pitch + v * 16, gk + off);
-        cp_async16(v_s + t * pitch + v * 16, gv + off);
+        if (t0 + t != skip) {
+          const long long off = (long long)slot * D * es + v * 16;
+          cp_async16(k_s + t * pitch + v * 16, gk + off);
+          cp_async16(v_s + t * pitch + v * 16, gv + off);
+        }
         slot += sstep;
         if (slot >= slots) slot -= slots;
       }
     } else {
       for (int idx = tid; idx < n * vpr; idx += kWinThreads) {
         const int t = idx / vpr, v = idx - (idx / vpr) * vpr;
+        if (t0 + t == skip) continue;
         const long long off = (long long)((hist_len + t0 + t) % slots) * D * es + v * 16;
         cp_async16(k_s + t * pitch + v * 16, gk + off);
         cp_async16(v_s + t * pitch + v * 16, gv + off);
       }
+    }
+  };
+  // the newest window token (position win_len - 1) into its staging row when it falls in the
+  // round [t0, t0 + n): from the step's input rows, or from its ring slot
+  const int newest = win_len - 1;
+  auto issue_newest = [&](int t0, int n) {
+    if (newest < t0 || newest >= t0 + n) return;
+    const uint8_t* sk = step ? reinterpret_cast<const uint8_t*>(a.k_new) + ((long long)b * D + (long long)h * d) * es
+                             : gk + (long long)((hist_len + newest) % slots) * D * es;
+    const uint8_t* sv = step ? reinterpret_cast<const uint8_t*>(a.v_new) + ((long long)b * D + (long long)h * d) * es
+                             : gv + (long long)((hist_len + newest) % slots) * D * es;
+    const int t = newest - t0;
+    for (int v = tid; v < vpr; v += kWinThreads) {
+      cp_async16(k_s + t * pitch + v * 16, sk + v * 16);
+      cp_async16(v_s + t * pitch + v * 16, sv + v * 16);
+    }
+  };
+  const int n_first = min(kWinTok, win_len);
+  issue(0, n_first, newest);
+  if (!step) pdl_wait();
+  if (step) {
+    // the query, scaled as the query projection scales it (fp32 product of the stored value)
+    const T* qb = static_cast<const T*>(a.q_in) + ((long long)b * Hq + j) * d;
+    for (int e = tid; e < d; e += kWinThreads) q_s[e] = win_elem<T>(reinterpret_cast<const uint8_t*>(qb + e)) * a.scale_log2;
+  } else {
+    for (int v = tid; v < d / 4; v += kWinThreads)
+      cp_async16(q_s + 4 * v, a.qd + ((long long)b * Hq + j) * d + 4 * v);
+  }
+  issue_newest(0, n_first);
+  float m = -INFINITY, l = 0.f;
+  float o = 0.f;                                           // output column tid (d <= 128 here: tid < d)
+  float o2 = 0.f;                                          // column tid + 128 (d > 128)
+  for (int t0 = 0; t0 < win_len; t0 += kWinTok) {
+    const int n = min(kWinTok, win_len - t0);
+    if (t0 > 0) {
+      __syncthreads();   // the previous round's rows and weights are no longer read
+      issue(t0, n, newest);
+      issue_newest(t0, n);
     }
     cp_async_wait_all();
     __syncthreads();
@@ -299,14 +356,15 @@ __global__ void __launch_bounds__(kWinThreads) k_window(const void* win_k, const
       for (int t = 0; t < n; ++t) o2 = fmaf(p_s[t], win_elem<T>(vc2 + t * pitch), o2);
   }
   cp_async_wait_all();   // (no window tokens: the query copies still complete)
+  if (step) pdl_wait();  // (the previous step's merge completed before the projection's wait)
   const long long ob = ((long long)b * Hq + j) * d;
-  if (tid < d) win_o[ob + tid] = o;
-  if (tid + kWinThreads < d) win_o[ob + tid + kWinThreads] = o2;
+  if (tid < d) a.win_o[ob + tid] = o;
+  if (tid + kWinThreads < d) a.win_o[ob + tid + kWinThreads] = o2;
   if (tid == 0) {
-    win_ml[((long long)b * Hq + j) * 2] = m;
-    win_ml[((long long)b * Hq + j) * 2 + 1] = l;
+    a.win_ml[((long long)b * Hq + j) * 2] = m;
+    a.win_ml[((long long)b * Hq + j) * 2 + 1] = l;
   }
-  span_end(span);
+  span_end(a.span);
 }
 
 // bulk latent fill: one warp per (token, 32-coordinate chunk)
@@ -455,22 +513,32 @@ cudaError_t launch_decode_simt(const lr_cache* c, int n_splits, int split_tokens
   return launch_pdl(k_decode_simt, grid, dim3(256), smem, s, a, c->latent_kind);
 }
 
-cudaError_t launch_window(const lr_cache* c, cudaStream_t s) {
+cudaError_t launch_window(const lr_cache* c, cudaStream_t s, const WindowStep* st) {
   const lr_cache_desc& d = c->desc;
-  const float* qd = d.rope_in_kernel ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k;
   const size_t smem = window_smem(d.n_q_heads / d.n_kv_heads, d.head_dim, (int)c->esize);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   dim3 grid(d.n_kv_heads, d.batch, d.n_q_heads / d.n_kv_heads);
-  using Kern = void (*)(const void*, const void*, const float*, float*, float*, int, int, int, int, int, int, int,
-                       unsigned long long*);
+  WinArgs a;
+  a.win_k = c->win_k;
+  a.win_v = c->win_v;
+  a.qd = d.rope_in_kernel ? c->qt : c->qt + (size_t)d.batch * d.n_q_heads * d.rank_k;
+  a.q_in = st ? st->q : nullptr;
+  a.k_new = st ? st->k : nullptr;
+  a.v_new = st ? st->v : nullptr;
+  a.scale_log2 = c->scale_log2;
+  a.win_o = c->win_o;
+  a.win_ml = c->win_ml;
+  a.Hq = d.n_q_heads; a.Hkv = d.n_kv_heads; a.d = d.head_dim; a.D = c->D; a.slots = c->win_slots;
+  a.hist_len = st ? st->hist_len : c->hist_len;
+  a.win_len = st ? st->win_len : c->win_len;
+  a.span = span_of(c->spans, SPAN_WINDOW);
   const bool bf = d.dtype == LR_BF16;
+  using Kern = void (*)(const WinArgs);
   const Kern kern = bf ? k_window<__nv_bfloat16> : k_window<float>;
   static std::atomic<uint32_t> optin_done[2] = {0, 0};
   cudaError_t e = smem_optin(kern, optin_done[bf ? 1 : 0]);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, grid, dim3(kWinThreads), smem, s, c->win_k, c->win_v, qd, c->win_o, c->win_ml, d.n_q_heads,
-                    d.n_kv_heads, d.head_dim, c->D, c->win_slots, c->hist_len, c->win_len,
-                    span_of(c->spans, SPAN_WINDOW));
+  return launch_pdl(kern, grid, dim3(kWinThreads), smem, s, a);
 }
 
 cudaError_t launch_append_latent(lr_cache* c, const float* zk, const float* zv, int n, cudaStream_t s) {

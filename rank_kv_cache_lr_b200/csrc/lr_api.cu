@@ -409,7 +409,8 @@ namespace {
 
 // The decode after its query projection: split-sequence attention (timed by the
 // caller's events when set), exact window, split merge and output projection.
-cudaError_t decode_rest(lr_cache* c, const lr_plan& p, void* out, float* lse, cudaStream_t s) {
+cudaError_t decode_rest(lr_cache* c, const lr_plan& p, void* out, float* lse, cudaStream_t s,
+                        bool window_done = false) {
   cudaError_t e = cudaSuccess;
   if (c->hist_len > 0) {
     if (c->ev_start) e = record_event(c->ev_start, s);
@@ -419,7 +420,7 @@ cudaError_t decode_rest(lr_cache* c, const lr_plan& p, void* out, float* lse, cu
     if (e == cudaSuccess && c->ev_stop) e = record_event(c->ev_stop, s);
   }
   const int S = c->hist_len > 0 ? p.n_splits : 0;
-  if (e == cudaSuccess && c->win_slots) e = launch_window(c, s);
+  if (e == cudaSuccess && c->win_slots && !window_done) e = launch_window(c, s);
   if (e == cudaSuccess) e = launch_merge(c, S, out, lse, s);
   return e;
 }
@@ -521,13 +522,19 @@ lr_status lr_decode_step(lr_cache* c, const void* k, const void* v, const void* 
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
   cudaError_t e = launch_step_pre(c, k, v, q, p.path == LR_PATH_TC, s);   // uses the pre-append counters
+  if (e == cudaSuccess && c->win_slots) {
+    // the exact window next, alongside the append and projection: its tokens are earlier
+    // steps' ring rows and this step's k, v
+    const WindowStep ws{k, v, q, hist1, win1};
+    e = launch_window(c, s, &ws);
+  }
   if (e != cudaSuccess) return LR_ERR_CUDA;
   c->stable_len = c->hist_len;   // the row the append writes (new token or fold) is not stable
   if (c->win_slots) c->undo = hist1 > c->hist_len ? 2 : 1;
   c->hist_len = hist1;
   c->win_len = win1;
   ++c->len;
-  e = decode_rest(c, p, out, lse, s);
+  e = decode_rest(c, p, out, lse, s, c->win_slots != 0);
   return e == cudaSuccess ? LR_OK : LR_ERR_CUDA;
 }
 

@@ -166,7 +166,15 @@ __device__ __forceinline__ int row_hist(const int32_t* row_len, int b, int hist_
 // which the kernel just before may have written)
 cudaError_t launch_qproj(const lr_cache* c, const void* q, cudaStream_t s, bool pdl = true);
 cudaError_t launch_decode_simt(const lr_cache* c, int n_splits, int split_tokens, cudaStream_t s);
-cudaError_t launch_window(const lr_cache* c, cudaStream_t s);
+// The window of a fused step, launched right after the step's append and query projection
+// and computed from the step's inputs (k, v: the new token's rows; q: the query) and the ring
+// rows of earlier steps, with the counters after the append.
+struct WindowStep {
+  const void* k; const void* v; const void* q;
+  int hist_len, win_len;
+};
+// st: null for the window after the latent decode
+cudaError_t launch_window(const lr_cache* c, cudaStream_t s, const WindowStep* st = nullptr);
 // Where the merge reads its partials and what it writes: by default the cache's own split
 // partials ([B][S][Hq]) merged and projected to `out`; with a MergeSource, partials at other
 // addresses / strides, and (rs_o set) a rank-space result instead of the projection.

@@ -544,6 +544,40 @@ def test_decode_step_equals_append_then_decode(lib, kind):
         assert lib.lr_cache_get_len(c1) == lib.lr_cache_get_len(c2)
 
 
+def test_decode_step_window_paths_equal_append_then_decode(lib):
+    """The fused step computes the exact window ahead of its own kernels, from the ring rows of
+    earlier steps and the step's own k, v and q; right after a standalone append of the same
+    cache it waits before reading the ring.  Both, with a window of two 128-token rounds that
+    fills up and then folds, equal lr_kv_append + lr_attn_decode bit for bit, step by step."""
+    import torch
+    p = synth.small_variant("hybrid", hist_len=300, window=200, win_len=190, batch=2)
+    c1, c2 = H.fill_cache(lib, p, capacity=600), H.fill_cache(lib, p, capacity=600)
+    D = p.kv_dim
+    q = _sharp(p)
+    qd = H.to_dev(p, q)
+    # per step: True = lr_decode_step on c2, False = lr_kv_append + lr_attn_decode on c2 too
+    plan = [True, True, False, True, False, False, True] + [True] * 7
+    for step, fused in enumerate(plan):
+        k, v = synth.hybrid_token("wstep", 0, step, p.batch, D, H.stored_value(p, p.B_k), H.stored_value(p, p.B_v))
+        kd, vd = H.to_dev(p, p.store(k)), H.to_dev(p, p.store(v))
+        o1, o2 = torch.empty_like(qd), torch.empty_like(qd)
+        l1 = torch.empty((p.batch, p.n_q_heads), dtype=torch.float32, device="cuda")
+        l2 = torch.empty_like(l1)
+        lib.lr_kv_append(c1, kd, vd)
+        lib.lr_attn_decode(c1, qd, o1, l1)
+        if fused:
+            lib.lr_decode_step(c2, kd, vd, qd, o2, l2)
+        else:
+            lib.lr_kv_append(c2, kd, vd)
+            lib.lr_attn_decode(c2, qd, o2, l2)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), f"step {step}"
+        assert lib.lr_cache_get_len(c1) == lib.lr_cache_get_len(c2)
+    assert lib.lr_cache_get_len(c1)[2] == 200          # the window filled and folded
+    lib.lr_cache_destroy(c1)
+    lib.lr_cache_destroy(c2)
+
+
 @pytest.mark.parametrize("hq,hkv", [(8, 2), (12, 3), (16, 1), (28, 4)])
 def test_decode_parity_prerope_head_shapes(lib, hq, hkv):
     """Keys before RoPE on tensor cores for other group sizes and KV-head counts: pairs of KV
