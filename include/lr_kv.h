@@ -217,7 +217,7 @@ lr_status lr_attn_decode(lr_cache* cache, const void* q, void* out, float* lse, 
 lr_status lr_attn_decode_varlen(lr_cache* cache, const void* q, void* out, float* lse,
                                 const int32_t* row_len, void* stream);
 
-/* ---- context sharding (SURVEY-style split of the context over GPUs; the pages'
+/* ---- context sharding (a split of each sequence's context over GPUs; the pages'
  *      workload, TraceKV digest Perspective: batch 16 at up to 32K tokens) -----------
  * Several caches (typically one per GPU) hold consecutive slices of the same sequences'
  * context, with the same bases and query.  Each computes a partial result over its slice;
