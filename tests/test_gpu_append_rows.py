@@ -166,3 +166,48 @@ def test_rows_refusals(lib):
         lib.lr_kv_append_rows(cw, kw, kw, torch.zeros((w.batch,), dtype=torch.int32, device="cuda"), 1)
     assert e.value.status == lib.LR_ERR_UNSUPPORTED
     lib.lr_cache_destroy(cw)
+
+
+def test_rows_append_and_varlen_decode_in_a_cuda_graph(lib):
+    """lr_kv_append_rows and lr_attn_decode_varlen read the positions and the row lengths on
+    the device, so one captured graph serves new positions: each replay writes the rows'
+    tokens at the positions then in the device tensor and decodes each row over its length,
+    checked against the oracle of the cache as the replays have left it."""
+    import torch
+    p = _problem("qwen4k")
+    p = dataclasses.replace(p, q=p.store(H.stored_value(p, p.q) * H.sharp_factor(p)))
+    c = _cache(lib, p, False)
+    (kx, zk_new), (vx, zv_new) = _one_hot_tokens(p, seed=5)
+    kd, vd, qd = H.to_dev(p, kx), H.to_dev(p, vx), H.to_dev(p, p.q)
+    pos = torch.zeros((p.batch,), dtype=torch.int32, device="cuda")
+    row_len = torch.ones((p.batch,), dtype=torch.int32, device="cuda")
+    out = torch.empty_like(qd)
+    lse = torch.empty((p.batch, p.n_q_heads), dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        lib.lr_kv_append_rows(c, kd, vd, pos, L + 2, stream=s)
+        lib.lr_attn_decode_varlen(c, qd, out, row_len, lse, stream=s)
+    assert lib.lr_cache_get_len(c) == (L + 2, L + 2, 0)
+    zk = _with_token(p.z_k, [CAP] * p.batch, zk_new, L + 2)
+    zv = _with_token(p.z_v, [CAP] * p.batch, zv_new, L + 2)
+    for rep, positions in enumerate(([5, 128, 299, 300, 301, 0], [127, 3, 300, 301, 64, 200])):
+        pos.copy_(torch.tensor(positions, dtype=torch.int32))
+        row_len.copy_(torch.tensor([q + 1 for q in positions], dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        for b, q in enumerate(positions):
+            zk[b, q] = zk_new[b]
+            zv[b, q] = zv_new[b]
+        got = out.float().cpu().numpy().astype(np.float64)
+        got_lse = lse.cpu().numpy().astype(np.float64)
+        full = dataclasses.replace(p, hist_len=L + 2, z_k=zk, z_v=zv)
+        for b, q in enumerate(positions):
+            n = q + 1
+            pb = dataclasses.replace(full, batch=1, hist_len=n, z_k=zk[b:b + 1, :n], z_v=zv[b:b + 1, :n],
+                                     q=p.q[b:b + 1])
+            ref, ref_lse = H.oracle_decode(pb)
+            H.compare(pb, got[b:b + 1], ref, got_lse[b:b + 1], ref_lse, tag=f"graph replay {rep} row {b} len {n}")
+    del g
+    lib.lr_cache_destroy(c)
